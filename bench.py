@@ -1,0 +1,386 @@
+"""Benchmark of the hybrid-precision attention hot path on B200.
+
+One step is one pass of the whole path on a Llama-3.1-8B-shaped attention
+layer with a 32768-token prompt (B=1, 32 query / 8 KV heads, head_dim 128,
+5% vertical columns + 128-token window, INT4 group-32 KV):
+  1. hq_probe_vertical  on the last 64 prompt queries -> vertical columns
+  2. hq_prefill_attn    hybrid INT8 / bf16 causal attention over the prompt
+  3. hq_pack_kv         the prompt's K / V -> hybrid INT4 + bf16 cache
+  4. hq_decode_attn     the last prompt row re-attends the packed cache
+The L2 cache (126 MB) is flushed before every step and again before the
+decode call (the pack has just written the 47 MB cache into L2), so the
+decode streams its cache from HBM.
+
+Reported: `value` = decode-attention HBM throughput (algorithmic bytes / the
+decode call's device time, CUDA events on the launching stream), plus the
+prefill operator's tensor throughput, both against the measured peaks.  With
+--gpus N (torchrun, one rank per GPU) every rank runs its own layer (weak
+scaling, no data-path collective); timing is the max over ranks.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl hq|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from kv_cache_vertical_b200.synth import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "hybrid decode attn HBM TB/s (% of peak); hybrid prefill TFLOPS (% of peak)"
+WL = WORKLOADS["llama8b_prefill_32k"]          # prompt; decode uses the same layer
+NOMINAL_INT8_OVER_BF16 = 2.0                     # dense INT8 / dense bf16 (vendor ratio)
+
+
+def peaks():
+    p = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "src": "fallback"}
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            m = json.load(f)
+        p.update({k: m[k] for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained") if k in m})
+        p["src"] = "measured"
+    return p
+
+
+# ---------------------------------------------------------------------------
+# Algorithmic work
+# ---------------------------------------------------------------------------
+def decode_bytes(B, Hq, Hkv, D, n_lo, n_hi, bits):
+    """Bytes the decode must move: low codes + fp16 (s, z) + bf16 hi rows + q + fp32 out."""
+    per_lo = 2 * (D * bits // 8 + (D // 32) * 4)
+    per_hi = 2 * D * 2
+    return B * Hkv * (n_lo * per_lo + n_hi * per_hi) + B * Hq * D * 2 + B * Hq * D * 4
+
+
+def prefill_work(idx: np.ndarray, N, W, D, Hq, Hkv):
+    """(INT8 ops, bf16 flops) over causal pairs only, from the actual vertical set."""
+    G = Hq // Hkv
+    win = sum(min(i + 1, W) for i in range(N)) if N < 4096 else (
+        W * (W + 1) // 2 + (N - W) * W if N >= W else N * (N + 1) // 2)
+    total = N * (N + 1) // 2
+    i8 = bf = 0
+    for b in range(idx.shape[0]):
+        for h in range(idx.shape[1]):
+            vert = int(np.maximum(0, N - W - idx[b, h].astype(np.int64)).sum())
+            low = total - win - vert
+            i8 += 2 * D * G * low
+            bf += 2 * D * G * (total + win + vert)   # P.V over all pairs + hi QK
+    return i8, bf
+
+
+# ---------------------------------------------------------------------------
+# Clocks during the timed region
+# ---------------------------------------------------------------------------
+class Clocks:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, dev_index: int):
+        self.dev = dev_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            self.proc.wait()
+
+    def summary(self):
+        rows = []
+        try:
+            for line in open(self.path):
+                f = [x.strip() for x in line.split(",")]
+                if len(f) >= 9:
+                    rows.append(f)
+        except OSError:
+            pass
+        finally:
+            if self.path:
+                os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# The hq arm
+# ---------------------------------------------------------------------------
+def run_hq(args, rank, world, dev):
+    from kv_cache_vertical_b200 import hq as H
+
+    w = WL.replace(seed=WL.seed + rank)
+    B, Hq, Hkv, D, N, W, kv = w.B, w.Hq, w.Hkv, w.D, w.L, w.window, w.k_vert
+    x = make_inputs(w, pin=True)
+    q_h, k_h, v_h = x["q"], x["k"], x["v"]
+    q, k, v = (t.to(dev, non_blocking=True) for t in (q_h, k_h, v_h))
+    stream = torch.cuda.current_stream(dev)
+    idx = torch.empty(B, Hkv, kv, dtype=torch.int32, device=dev)
+    out_p = torch.empty(B, Hq, N, D, dtype=torch.float32, device=dev)
+    out_d = torch.empty(B, Hq, D, dtype=torch.float32, device=dev)
+    cache = H.KVCache.empty(B, Hkv, N, D, W, kv, w.bits, dev, with_pos=False)
+    ws_probe = H.workspace(H.hq_probe_workspace_size(B, Hq, Hkv, 64, N, D), dev)
+    ws_pre = H.workspace(H.hq_prefill_workspace_size(B, Hq, Hkv, N, D, kv), dev)
+    ws_pack = H.workspace(256, dev)
+    ws_dec = H.workspace(H.hq_decode_workspace_size(B, Hq, Hkv, D, cache.n_lo, cache.n_hi, w.bits), dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    q_last = q[:, :, N - 1]                      # [B, Hq, D] view, stride N*D between heads
+    q_dec = torch.empty(B, Hq, D, dtype=torch.bfloat16, device=dev)
+    ev = {n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for n in ("probe", "prefill", "pack", "decode", "step")}
+
+    def step(qq, kk, vv, timed):
+        e = ev if timed else None
+        flush.zero_()
+        if e: e["step"][0].record(stream)
+        if e: e["probe"][0].record(stream)
+        H.hq_probe_vertical(qq[:, :, N - 64:], N * D, kk, B, Hq, Hkv, 64, N, D, W, kv, 0.0, idx,
+                            None, ws_probe)
+        if e: e["probe"][1].record(stream)
+        if e: e["prefill"][0].record(stream)
+        H.hq_prefill_attn(qq, kk, vv, idx, B, Hq, Hkv, N, D, W, kv, 0.0, out_p, ws_pre)
+        if e: e["prefill"][1].record(stream)
+        if e: e["pack"][0].record(stream)
+        H.hq_pack_kv(kk, vv, idx, B, Hkv, N, D, W, kv, w.bits, 32, cache, ws_pack)
+        if e: e["pack"][1].record(stream)
+        q_dec.copy_(qq[:, :, N - 1])
+        flush.zero_()
+        if e: e["decode"][0].record(stream)
+        H.hq_decode_attn(q_dec, cache, B, Hq, Hkv, D, 0.0, out_d, None, ws_dec)
+        if e: e["decode"][1].record(stream)
+        if e: e["step"][1].record(stream)
+
+    for _ in range(args.warmup):
+        step(q, k, v, False)
+    torch.cuda.synchronize(dev)
+    acc = {n: 0.0 for n in ev}
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with Clocks(dev.index if dev.index is not None else 0) as clk:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(args.steps):
+            step(q, k, v, True)
+            torch.cuda.synchronize(dev)   # per-kernel events are read back each step
+            for n, (a, b) in ev.items():
+                acc[n] += a.elapsed_time(b)
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    total_ms = t0.elapsed_time(t1)
+    per = {n: acc[n] / args.steps for n in acc}           # ms per launch
+    per = {n: max_over_ranks(vv_, world, dev) for n, vv_ in per.items()}
+
+    # e2e through the public API: host (pinned) inputs in, results back to host
+    out_p_h = torch.empty(out_p.shape, dtype=out_p.dtype, pin_memory=True)
+    out_d_h = torch.empty(out_d.shape, dtype=out_d.dtype, pin_memory=True)
+    qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    e2e_steps = max(1, min(args.steps, 5))
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for _ in range(e2e_steps):
+        qd.copy_(q_h, non_blocking=True)
+        kd.copy_(k_h, non_blocking=True)
+        vd.copy_(v_h, non_blocking=True)
+        step(qd, kd, vd, False)
+        out_p_h.copy_(out_p, non_blocking=True)
+        out_d_h.copy_(out_d, non_blocking=True)
+    a1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(a0.elapsed_time(a1) / e2e_steps, world, dev)
+    h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h))
+    d2h = out_p.numel() * 4 + out_d.numel() * 4
+
+    idx_np = idx.cpu().numpy()
+    dbytes = decode_bytes(B, Hq, Hkv, D, cache.n_lo, cache.n_hi, w.bits)
+    i8_ops, bf_flops = prefill_work(idx_np, N, W, D, Hq, Hkv)
+    clocks = clk.summary()
+    return dict(per=per, total_ms=max_over_ranks(total_ms / args.steps, world, dev), dbytes=dbytes,
+                i8=i8_ops, bf=bf_flops, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, clocks=clocks,
+                kpad=(kv + 63) // 64 * 64, w=w)
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int, dev) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the fp64 oracle on a bounded sample
+# ---------------------------------------------------------------------------
+def oracle_decode_sample(w, heads_kv: int):
+    """Time the oracle's decode over `heads_kv` KV heads of the workload."""
+    import oracle
+    x = make_inputs(w.replace(Hkv=heads_kv, Hq=heads_kv * w.G))
+    sc = oracle.probe_scores(x["q"][:, :, w.L - 64:].contiguous(), x["k"], heads_kv)
+    idx = oracle.topk(sc, w.window, w.k_vert)
+    c = oracle.pack_kv(x["k"], x["v"], idx, w.window, w.bits)
+    q_dec = x["q"][:, :, w.L - 1].contiguous()
+    t = time.perf_counter()
+    oracle.decode_attn(q_dec, c, heads_kv)
+    dt = time.perf_counter() - t
+    nbytes = decode_bytes(w.B, heads_kv * w.G, heads_kv, w.D, c["n_lo"], c["n_hi"], w.bits)
+    return nbytes, dt, oracle.max_threads()
+
+
+def cpu_baseline(w):
+    nbytes, dt, cores = oracle_decode_sample(w, w.Hkv)
+    return {"value": nbytes / dt / 1e12, "unit": "TB/s", "cores": cores, "kind": "oracle",
+            "sample": f"oracle fp64 decode attention over the full {w.L}-token INT4 cache, "
+                      f"{w.Hq} query heads (one call, {dt:.2f} s)"}
+
+
+def run_reference(args, rank, world):
+    """--impl reference: the oracle as it stands, timed on the host cores."""
+    if rank != 0:
+        return None
+    w = WL
+    vals = []
+    cores = 1
+    hk = 2          # bounded sample per step: 2 of the 8 KV heads
+    for i in range(args.warmup + args.steps):
+        nbytes, dt, cores = oracle_decode_sample(w, hk)
+        if i >= args.warmup:
+            vals.append((nbytes, dt))
+    tb = sum(b for b, _ in vals) / sum(t for _, t in vals) / 1e12
+    ms = 1e3 * sum(t for _, t in vals) / len(vals)
+    cpu = {"value": tb, "unit": "TB/s", "cores": cores, "kind": "oracle",
+           "sample": f"oracle fp64 decode of {hk} of {w.Hkv} KV heads ({hk * w.G} query heads) "
+                     f"over the {w.L}-token INT4 cache per step"}
+    return {"impl": "reference", "metric": METRIC, "value": tb, "unit": "TB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_dict(w, world), "cpu_baseline": cpu,
+            "e2e": {"value": tb, "unit": "TB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def config_dict(w, world):
+    return {"workload": "llama3.1-8b-shaped attention layer, 32768-token prompt: probe + hybrid "
+                        "prefill + INT4 pack + decode",
+            "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "head_dim": w.D, "tokens": w.L,
+            "window": w.window, "vertical_frac": float(w.frac), "kv_bits": w.bits,
+            "group": 32, "parallelism": f"replicas x{world}",
+            "l2": "flushed (256 MB write) before every step and before the decode call"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="hq", choices=["hq", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if world > 1:
+            torch.distributed.init_process_group("gloo", timeout=__import__("datetime").timedelta(seconds=600))
+        r = run_reference(args, rank, world)
+        if r is not None:
+            print(json.dumps(r), flush=True)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        torch.distributed.init_process_group("nccl", device_id=dev,
+                                             timeout=__import__("datetime").timedelta(seconds=300))
+    r = run_hq(args, rank, world, dev)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return
+    pk = peaks()
+    per = r["per"]
+    w = r["w"]
+    dec_tbs = r["dbytes"] / (per["decode"] * 1e-3) / 1e12
+    pre_s = per["prefill"] * 1e-3
+    i8_peak = pk["bf16_tflops"] * NOMINAL_INT8_OVER_BF16
+    t_star = r["bf"] / (pk["bf16_tflops"] * 1e12) + r["i8"] / (i8_peak * 1e12)
+    pre_tflops = (r["bf"] + r["i8"]) / pre_s / 1e12
+    launches_per_step = 4 + (5 + (1 if r["kpad"] > 0 else 0)) + 1 + 2
+    out = {
+        "metric": METRIC,
+        "value": dec_tbs * world,
+        "unit": "TB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": r["total_ms"],
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int4 KV codes -> bf16/fp16 MMA, fp32 accumulate (decode); int8 + bf16/fp16 (prefill)",
+        "data": "synthetic (seeded generator: outlier channels, planted vertical lines)",
+        "config": config_dict(w, world),
+        "roofline": {"kernel": "hq_decode_attn", "bound": "hbm", "achieved": dec_tbs * 1e3,
+                     "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": dec_tbs * 1e3 / pk["hbm_gbs"],
+                     "traffic": None, "algorithmic_bytes": r["dbytes"],
+                     "peak_src": pk["src"] + " (copy bandwidth)",
+                     "frac_of_8TBs": dec_tbs / 8.0},
+        "prefill": {"kernel": "hq_prefill_attn", "bound": "tensor", "ms": per["prefill"],
+                    "achieved": pre_tflops, "unit": "TFLOP/s (INT8 ops + bf16/fp16 flops)",
+                    "int8_tops": r["i8"] / 1e12, "bf16_tflop": r["bf"] / 1e12,
+                    "roofline_ms": t_star * 1e3, "frac": t_star / pre_s,
+                    "peak": {"bf16_tflops": pk["bf16_tflops"], "int8_tops": i8_peak,
+                             "src": pk["src"] + " bf16; int8 = bf16 x nominal ratio 2"},
+                    "traffic": None},
+        "per_call_ms": {n: per[n] for n in ("probe", "prefill", "pack", "decode")},
+        "e2e": {"value": r["dbytes"] / (r["e2e_ms"] * 1e-3) / 1e12 * world, "unit": "TB/s",
+                "ms_per_step": r["e2e_ms"], "h2d_bytes_per_step": r["h2d"],
+                "d2h_bytes_per_step": r["d2h"],
+                "note": "decode bytes / whole-step time with pinned-host inputs copied in and "
+                        "the prefill + decode outputs copied back"},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": r["clocks"],
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(w)
+    print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

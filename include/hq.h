@@ -1,0 +1,211 @@
+/*
+ * hq.h -- C ABI of libhq.so: HyQuant hybrid-precision attention on NVIDIA
+ * B200 (sm_100a).
+ *
+ * Method (web pages on HyQuant):
+ *   - "HyQuant: Hybrid-Precision Quantization for LLM Attention" (wiki
+ *     summary), TL;DR: a small set of vertical-line key columns, found by a
+ *     cheap pattern probe, plus a local sliding window stay in high precision;
+ *     every other key/value position is quantized to low bit.  In prefill this
+ *     is a hybrid-precision attention operator; in decode a hybrid KV cache
+ *     whose dequantization is fused into attention.
+ *   - "How HyQuant uses hybrid-precision attention to cut decode compute"
+ *     (blog), "Why preserve selected positions?": top 5% of key positions plus
+ *     a 128-token window; "What the authors tested": Key-4bit / Value-4bit.
+ *   - ACL Anthology page, HyQuant abstract: the prefill operator and the
+ *     decode KV-cache compression with fused dequantization.
+ *
+ * Conventions for every call
+ *   Layout: row-major, head-major [B, H, T, D], contiguous over D.  bf16 is
+ *     IEEE bfloat16, f16 IEEE binary16, both passed as `const void *`.
+ *     Query head h reads KV head h / (Hq / Hkv).
+ *   Memory: every pointer is a DEVICE pointer owned by the caller, except the
+ *     hq_kv_cache struct itself (host memory, read during the call).  The
+ *     library never allocates or frees memory, never synchronizes the stream
+ *     and keeps no state between calls.  `stream` is a cudaStream_t (NULL is
+ *     the legacy default stream); all work is stream-ordered.
+ *   Workspace: calls that need scratch take (ws, ws_bytes).  Size it with the
+ *     matching hq_*_workspace_size query, allocate it on the device,
+ *     zero it ONCE before its first use (cudaMemset), and keep using it; the
+ *     library leaves it in a reusable state.  The first 16 bytes hold a
+ *     device status word (see hq_read_device_status).  Calls that share one
+ *     workspace must not run concurrently.
+ *   Errors: arguments are checked on the host before any launch; a failed
+ *     check returns an error and launches nothing.  HQ_ERR_CUDA reports a
+ *     launch error (cudaGetLastError).  Checks made on the device (index
+ *     lists out of order or out of range; waits that ran out) never trap:
+ *     they skip the offending access and set a bit in the device status word.
+ *   Supported shapes: D in {64, 128}; Hq % Hkv == 0 with Hq / Hkv <= 8;
+ *     KV bits in {4, 8}; quantization group 32.  Others return
+ *     HQ_ERR_UNSUPPORTED.  There is no CPU path.
+ */
+#ifndef HQ_H
+#define HQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    HQ_OK = 0,
+    HQ_ERR_INVALID_ARG = 1,   /* null pointer, bad size, inconsistent dims */
+    HQ_ERR_UNSUPPORTED = 2,   /* valid but not implemented (D, G, bits, group) */
+    HQ_ERR_WORKSPACE = 3,     /* workspace missing or smaller than required */
+    HQ_ERR_CUDA = 4,          /* a CUDA launch or runtime call failed */
+    HQ_ERR_TIMEOUT = 5,       /* a bounded device wait ran out (status word) */
+    HQ_ERR_DEVICE_CHECK = 6   /* a device-side argument check failed (status word) */
+} hq_status;
+
+/* Device status word bits (hq_read_device_status). */
+#define HQ_DEV_BAD_INDEX 0x1u   /* an index list was unsorted, repeated or out of range */
+#define HQ_DEV_TIMEOUT 0x2u     /* a bounded inter-CTA wait gave up */
+
+/* Human-readable name of a status code (static storage). */
+const char *hq_status_string(int status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int hq_version(void);
+
+/*
+ * Hybrid KV cache (decode).  Plain struct of caller-owned device buffers.
+ * With L cached tokens, window W and k vertical columns per (b, kv head):
+ *   n_lo = L - W - k low-bit rows, n_hi = k + W bf16 rows.
+ *   k_codes, v_codes : u8  [B, Hkv, n_lo, D * bits / 8].  4-bit codes are
+ *                      packed two per byte, even channel in the low nibble.
+ *   k_sz, v_sz       : f16 [B, Hkv, n_lo, D / group, 2], (scale, zero) of each
+ *                      group; dequantized value = scale * code + zero.
+ *   k_hi, v_hi       : bf16 [B, Hkv, n_hi, D]; rows 0..k-1 are the vertical
+ *                      columns in ascending position order, rows k..k+W-1 the
+ *                      window (positions L-W .. L-1).
+ *   lo_pos           : i32 [B, Hkv, n_lo] position of each low row (ascending),
+ *                      or NULL when not wanted.
+ * All pointers must be 16-byte aligned.  The low rows are stored in ascending
+ * position order, with no copy of the vertical rows: attention does not depend
+ * on key order, and storing a vertical row only once is what gives the
+ * pages' "+15% over strict 4-bit at 5% retention" ("Memory and runtime costs").
+ */
+typedef struct {
+    void *k_codes;
+    void *v_codes;
+    void *k_sz;
+    void *v_sz;
+    void *k_hi;
+    void *v_hi;
+    int32_t *lo_pos;
+    int n_lo;
+    int n_hi;
+    int bits;
+    int group;
+} hq_kv_cache;
+
+/*
+ * Copy the device status word out of a workspace (synchronizes `stream`).
+ * *status_out receives the OR of the HQ_DEV_* bits raised since the word was
+ * last cleared; `clear` != 0 resets it to zero afterwards.
+ */
+hq_status hq_read_device_status(const void *ws, int clear, uint32_t *status_out, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* Vertical-line probe (wiki summary, TL;DR: "vertical-line-aware pattern    */
+/* probe"; blog, "Why preserve selected positions?": top 5% + window).       */
+/* ------------------------------------------------------------------------ */
+/*
+ * For every (b, kv head), score[j] = sum over the G query heads of the group
+ * and the P probe rows of the causal softmax weight of key j; probe row p sits
+ * at position L - P + p and sees keys 0 .. L - P + p.  The k_vert columns of
+ * [0, L - window) with the largest score are written to idx_out in ascending
+ * order; equal scores go to the lower index.
+ *   q_probe   : bf16, row p of head h of batch b at
+ *               q_probe + (b * Hq + h) * q_head_stride + p * D  (elements);
+ *               q_head_stride >= P * D lets the caller pass the last P rows
+ *               of a [B, Hq, N, D] prefill Q without a copy (stride N * D).
+ *   k         : bf16 [B, Hkv, L, D].
+ *   idx_out   : i32 [B, Hkv, k_vert], ascending.
+ *   score_out : f32 [B, Hkv, L] or NULL (the column sums; keys never seen 0).
+ *   softmax_scale: 0 selects 1 / sqrt(D).
+ * Requires 1 <= P <= L, 0 <= window, 0 <= k_vert <= L - window.
+ */
+size_t hq_probe_workspace_size(int B, int Hq, int Hkv, int P, int L, int D);
+hq_status hq_probe_vertical(const void *q_probe, int64_t q_head_stride, const void *k, int B,
+                            int Hq, int Hkv, int P, int L, int D, int window, int k_vert,
+                            float softmax_scale, int32_t *idx_out, float *score_out, void *ws,
+                            size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* KV pack: build the hybrid cache (wiki summary, TL;DR: quantize the rest   */
+/* hard, no smoothing; blog, "What the authors tested": Key-4bit/Value-4bit). */
+/* ------------------------------------------------------------------------ */
+/*
+ * Splits [0, L) of every (b, kv head) into the window [L - window, L), the
+ * vertical columns idx (ascending, distinct, in [0, L - window)) and the low
+ * rows (everything else), and writes `out` as described at hq_kv_cache.
+ * Quantizer, per token and group of `group` channels, `bits`-bit asymmetric:
+ *   s = f16_rne((max - min) / (2^bits - 1)),  z = f16_rne(min),
+ *   code = clamp(rne((x - z) / s), 0, 2^bits - 1), all 0 when s == 0,
+ * with every intermediate taken in IEEE double so that each rounding decision
+ * is exact and reproducible.  out->n_lo / n_hi / bits / group must equal
+ * L - window - k_vert, k_vert + window, bits and group.  An idx list that is
+ * unsorted, repeated or out of range sets HQ_DEV_BAD_INDEX in the status word
+ * of `ws` (if given) and leaves the affected rows unwritten.
+ *   k, v: bf16 [B, Hkv, L, D].  ws may be NULL (no status reporting).
+ */
+hq_status hq_pack_kv(const void *k, const void *v, const int32_t *idx, int B, int Hkv, int L,
+                     int D, int window, int k_vert, int bits, int group, const hq_kv_cache *out,
+                     void *ws, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* Decode attention with fused dequantization (wiki summary, "Key results":  */
+/* KV dequantization fused with attention in the decode kernel; abstract).   */
+/* ------------------------------------------------------------------------ */
+/*
+ * out[b, h, :] = softmax_j(q[b, h] . key_j * scale) . value_j over all
+ * n_lo + n_hi cached rows of KV head h / G, the low rows dequantized in
+ * registers (scale * code + zero) and never written back.  Split-KV over the
+ * cache with one combine; no mask (the cache includes the current token).
+ *   q       : bf16 [B, Hq, D].
+ *   out     : f32 [B, Hq, D].
+ *   lse_out : f32 [B, Hq] natural-log sum of exp of the scaled logits, or NULL.
+ */
+size_t hq_decode_workspace_size(int B, int Hq, int Hkv, int D, int n_lo, int n_hi, int bits);
+hq_status hq_decode_attn(const void *q, const hq_kv_cache *cache, int B, int Hq, int Hkv, int D,
+                         float softmax_scale, float *out, float *lse_out, void *ws,
+                         size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* Hybrid-precision prefill (abstract: Prefill stage keeps vertical-line     */
+/* tokens and a local window in full precision, quantizes the rest).         */
+/* ------------------------------------------------------------------------ */
+/*
+ * Pre-pass: symmetric INT8 codes for Q, one scale per (b, head, row), and for
+ * K, one scale per (b, kv head, block of 64 keys):
+ *   s = fl32(amax / 127) (1 when amax == 0),  code = clamp(rne(fl32(x / s)), -127, 127).
+ *   q: bf16 [B, Hq, N, D] -> qi8 i8 [B, Hq, N, D], sq f32 [B, Hq, N]
+ *   k: bf16 [B, Hkv, N, D] -> ki8 i8 [B, Hkv, N, D], sk f32 [B, Hkv, ceil(N / 64)]
+ */
+hq_status hq_prefill_quant(const void *q, const void *k, int B, int Hq, int Hkv, int N, int D,
+                           int8_t *qi8, float *sq, int8_t *ki8, float *sk, void *stream);
+
+/*
+ * Causal attention in which, for query i, key j <= i is "high" when it is in
+ * the window (j > i - window) or is a vertical column of idx, else "low".
+ * High logits are bf16 q . k (fp32 accumulate); low logits are the exact INT8
+ * dot product of the pre-pass codes times sq[i] * sk[j / 64]; one online
+ * softmax covers both; P . V uses fp16 P and V with fp32 accumulation.
+ *   q: bf16 [B, Hq, N, D];  k, v: bf16 [B, Hkv, N, D];
+ *   idx: i32 [B, Hkv, k_vert] ascending (from hq_probe_vertical);
+ *   out: f32 [B, Hq, N, D].  The workspace holds the pre-pass output.
+ */
+size_t hq_prefill_workspace_size(int B, int Hq, int Hkv, int N, int D, int k_vert);
+hq_status hq_prefill_attn(const void *q, const void *k, const void *v, const int32_t *idx, int B,
+                          int Hq, int Hkv, int N, int D, int window, int k_vert,
+                          float softmax_scale, float *out, void *ws, size_t ws_bytes,
+                          void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HQ_H */

@@ -1,0 +1,168 @@
+// api.cu -- the C ABI of libhq.so (declared in include/hq.h): host-side
+// argument checks, workspace carving and kernel dispatch.  Nothing here
+// allocates, frees or synchronizes (except hq_read_device_status, a debug
+// helper that says so).
+#include <math.h>
+
+#include "hq_internal.cuh"
+
+using namespace hq;
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool supported_G(int Hq, int Hkv) {
+  if (Hq <= 0 || Hkv <= 0 || Hq % Hkv) return false;
+  const int G = Hq / Hkv;
+  return G == 1 || G == 2 || G == 4 || G == 8;
+}
+
+float resolve_scale(float s, int D) { return s == 0.0f ? 1.0f / sqrtf((float)D) : s; }
+
+hq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? HQ_OK : HQ_ERR_CUDA; }
+
+uint32_t *status_word(void *ws) { return ws ? reinterpret_cast<uint32_t *>(ws) : nullptr; }
+
+}  // namespace
+
+extern "C" {
+
+const char *hq_status_string(int status) {
+  switch (status) {
+    case HQ_OK: return "HQ_OK";
+    case HQ_ERR_INVALID_ARG: return "HQ_ERR_INVALID_ARG";
+    case HQ_ERR_UNSUPPORTED: return "HQ_ERR_UNSUPPORTED";
+    case HQ_ERR_WORKSPACE: return "HQ_ERR_WORKSPACE";
+    case HQ_ERR_CUDA: return "HQ_ERR_CUDA";
+    case HQ_ERR_TIMEOUT: return "HQ_ERR_TIMEOUT";
+    case HQ_ERR_DEVICE_CHECK: return "HQ_ERR_DEVICE_CHECK";
+    default: return "HQ_ERR_UNKNOWN";
+  }
+}
+
+int hq_version(void) { return 100; }
+
+hq_status hq_read_device_status(const void *ws, int clear, uint32_t *status_out, void *stream) {
+  if (!ws || !status_out) return HQ_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  uint32_t v = 0;
+  if (cudaMemcpyAsync(&v, ws, sizeof v, cudaMemcpyDeviceToHost, s) != cudaSuccess) return HQ_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return HQ_ERR_CUDA;
+  if (clear && cudaMemsetAsync(const_cast<void *>(ws), 0, sizeof v, s) != cudaSuccess) return HQ_ERR_CUDA;
+  *status_out = v;
+  return HQ_OK;
+}
+
+size_t hq_probe_workspace_size(int B, int Hq, int Hkv, int P, int L, int D) {
+  if (B <= 0 || !supported_G(Hq, Hkv) || P <= 0 || L <= 0 || (D != 64 && D != 128)) return 0;
+  return probe_ws_bytes(B, Hq, Hkv, P, L, D);
+}
+
+hq_status hq_probe_vertical(const void *q_probe, int64_t q_head_stride, const void *k, int B,
+                            int Hq, int Hkv, int P, int L, int D, int window, int k_vert,
+                            float softmax_scale, int32_t *idx_out, float *score_out, void *ws,
+                            size_t ws_bytes, void *stream) {
+  if (!q_probe || !k || !idx_out) return HQ_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || P <= 0 || P > L || window < 0 ||
+      k_vert < 0 || k_vert > L - window || q_head_stride < (int64_t)P * D)
+    return HQ_ERR_INVALID_ARG;
+  if ((D != 64 && D != 128) || !supported_G(Hq, Hkv)) return HQ_ERR_UNSUPPORTED;
+  if (!aligned16(q_probe) || !aligned16(k) || (q_head_stride * 2) % 16) return HQ_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < probe_ws_bytes(B, Hq, Hkv, P, L, D)) return HQ_ERR_WORKSPACE;
+  return cuda_status(launch_probe((const __nv_bfloat16 *)q_probe, q_head_stride,
+                                  (const __nv_bfloat16 *)k, B, Hq, Hkv, P, L, D, window, k_vert,
+                                  resolve_scale(softmax_scale, D), idx_out, score_out,
+                                  (uint8_t *)ws, (cudaStream_t)stream));
+}
+
+hq_status hq_pack_kv(const void *k, const void *v, const int32_t *idx, int B, int Hkv, int L,
+                     int D, int window, int k_vert, int bits, int group, const hq_kv_cache *out,
+                     void *ws, size_t ws_bytes, void *stream) {
+  if (!k || !v || !out || (k_vert > 0 && !idx)) return HQ_ERR_INVALID_ARG;
+  if (B <= 0 || Hkv <= 0 || L <= 0 || window < 0 || k_vert < 0 || k_vert > L - window)
+    return HQ_ERR_INVALID_ARG;
+  if ((D != 64 && D != 128) || (bits != 4 && bits != 8) || group != 32) return HQ_ERR_UNSUPPORTED;
+  const int n_lo = L - window - k_vert, n_hi = k_vert + window;
+  if (out->n_lo != n_lo || out->n_hi != n_hi || out->bits != bits || out->group != group)
+    return HQ_ERR_INVALID_ARG;
+  if ((n_lo > 0 && (!out->k_codes || !out->v_codes || !out->k_sz || !out->v_sz)) ||
+      (n_hi > 0 && (!out->k_hi || !out->v_hi)))
+    return HQ_ERR_INVALID_ARG;
+  const void *ptrs[] = {k, v, out->k_codes, out->v_codes, out->k_sz, out->v_sz, out->k_hi, out->v_hi};
+  for (const void *p : ptrs)
+    if (p && !aligned16(p)) return HQ_ERR_INVALID_ARG;
+  if (ws && ws_bytes < kWsHeader) return HQ_ERR_WORKSPACE;
+  return cuda_status(launch_pack((const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, idx, B, Hkv,
+                                 L, D, window, k_vert, bits, *out, status_word(ws),
+                                 (cudaStream_t)stream));
+}
+
+size_t hq_decode_workspace_size(int B, int Hq, int Hkv, int D, int n_lo, int n_hi, int bits) {
+  if (B <= 0 || !supported_G(Hq, Hkv) || (D != 64 && D != 128) || n_lo < 0 || n_hi < 0 ||
+      n_lo + n_hi <= 0 || (bits != 4 && bits != 8))
+    return 0;
+  return decode_ws_bytes(B, Hq, Hkv, D, n_lo, n_hi, bits);
+}
+
+hq_status hq_decode_attn(const void *q, const hq_kv_cache *cache, int B, int Hq, int Hkv, int D,
+                         float softmax_scale, float *out, float *lse_out, void *ws,
+                         size_t ws_bytes, void *stream) {
+  if (!q || !cache || !out) return HQ_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || cache->n_lo < 0 || cache->n_hi < 0 ||
+      cache->n_lo + cache->n_hi <= 0)
+    return HQ_ERR_INVALID_ARG;
+  if ((D != 64 && D != 128) || !supported_G(Hq, Hkv) || (cache->bits != 4 && cache->bits != 8) ||
+      cache->group != 32)
+    return HQ_ERR_UNSUPPORTED;
+  if ((cache->n_lo > 0 && (!cache->k_codes || !cache->v_codes || !cache->k_sz || !cache->v_sz)) ||
+      (cache->n_hi > 0 && (!cache->k_hi || !cache->v_hi)))
+    return HQ_ERR_INVALID_ARG;
+  const void *ptrs[] = {q, cache->k_codes, cache->v_codes, cache->k_sz, cache->v_sz,
+                        cache->k_hi, cache->v_hi, out};
+  for (const void *p : ptrs)
+    if (p && !aligned16(p)) return HQ_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < decode_ws_bytes(B, Hq, Hkv, D, cache->n_lo, cache->n_hi, cache->bits))
+    return HQ_ERR_WORKSPACE;
+  return cuda_status(launch_decode((const __nv_bfloat16 *)q, *cache, B, Hq, Hkv, D,
+                                   resolve_scale(softmax_scale, D), out, lse_out, (uint8_t *)ws,
+                                   status_word(ws), (cudaStream_t)stream));
+}
+
+hq_status hq_prefill_quant(const void *q, const void *k, int B, int Hq, int Hkv, int N, int D,
+                           int8_t *qi8, float *sq, int8_t *ki8, float *sk, void *stream) {
+  if (!q || !k || !qi8 || !sq || !ki8 || !sk) return HQ_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || N <= 0) return HQ_ERR_INVALID_ARG;
+  if ((D != 64 && D != 128) || !supported_G(Hq, Hkv)) return HQ_ERR_UNSUPPORTED;
+  const void *ptrs[] = {q, k, qi8, ki8};
+  for (const void *p : ptrs)
+    if (!aligned16(p)) return HQ_ERR_INVALID_ARG;
+  return cuda_status(launch_prefill_quant((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, B,
+                                          Hq, Hkv, N, D, qi8, sq, ki8, sk, (cudaStream_t)stream));
+}
+
+size_t hq_prefill_workspace_size(int B, int Hq, int Hkv, int N, int D, int k_vert) {
+  if (B <= 0 || !supported_G(Hq, Hkv) || N <= 0 || (D != 64 && D != 128) || k_vert < 0) return 0;
+  return prefill_ws_bytes(B, Hq, Hkv, N, D, k_vert);
+}
+
+hq_status hq_prefill_attn(const void *q, const void *k, const void *v, const int32_t *idx, int B,
+                          int Hq, int Hkv, int N, int D, int window, int k_vert,
+                          float softmax_scale, float *out, void *ws, size_t ws_bytes,
+                          void *stream) {
+  if (!q || !k || !v || !out || (k_vert > 0 && !idx)) return HQ_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || N <= 0 || window < 0 || k_vert < 0 ||
+      k_vert > N - (window < N ? window : N))
+    return HQ_ERR_INVALID_ARG;
+  if ((D != 64 && D != 128) || !supported_G(Hq, Hkv)) return HQ_ERR_UNSUPPORTED;
+  const void *ptrs[] = {q, k, v, out};
+  for (const void *p : ptrs)
+    if (!aligned16(p)) return HQ_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < prefill_ws_bytes(B, Hq, Hkv, N, D, k_vert)) return HQ_ERR_WORKSPACE;
+  return cuda_status(launch_prefill((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k,
+                                    (const __nv_bfloat16 *)v, idx, B, Hq, Hkv, N, D, window,
+                                    k_vert, resolve_scale(softmax_scale, D), out, (uint8_t *)ws,
+                                    status_word(ws), (cudaStream_t)stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,77 @@
+// hq_internal.cuh -- shared declarations of the CUDA side of libhq.so.
+// (Internal to the library; the public ABI is include/hq.h.)
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/hq.h"
+
+namespace hq {
+
+// ---------------------------------------------------------------------------
+// Workspace: the first 16 bytes hold the device status word (+ padding);
+// call-specific scratch starts at kWsHeader.
+// ---------------------------------------------------------------------------
+constexpr size_t kWsHeader = 256;
+
+__device__ __forceinline__ void raise_status(uint32_t *status, uint32_t bit) {
+  if (status) atomicOr(status, bit);
+}
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ---------------------------------------------------------------------------
+// Launchers (one per .cu file).  Arguments are already validated.
+// ---------------------------------------------------------------------------
+cudaError_t launch_pack(const __nv_bfloat16 *k, const __nv_bfloat16 *v, const int32_t *idx,
+                        int B, int Hkv, int L, int D, int window, int k_vert, int bits,
+                        const hq_kv_cache &out, uint32_t *status, cudaStream_t s);
+
+size_t probe_ws_bytes(int B, int Hq, int Hkv, int P, int L, int D);
+cudaError_t launch_probe(const __nv_bfloat16 *q_probe, int64_t q_head_stride,
+                         const __nv_bfloat16 *k, int B, int Hq, int Hkv, int P, int L, int D,
+                         int window, int k_vert, float scale, int32_t *idx_out, float *score_out,
+                         uint8_t *ws, cudaStream_t s);
+
+size_t decode_ws_bytes(int B, int Hq, int Hkv, int D, int n_lo, int n_hi, int bits);
+cudaError_t launch_decode(const __nv_bfloat16 *q, const hq_kv_cache &c, int B, int Hq, int Hkv,
+                          int D, float scale, float *out, float *lse, uint8_t *ws,
+                          uint32_t *status, cudaStream_t s);
+
+cudaError_t launch_prefill_quant(const __nv_bfloat16 *q, const __nv_bfloat16 *k, int B, int Hq,
+                                 int Hkv, int N, int D, int8_t *qi8, float *sq, int8_t *ki8,
+                                 float *sk, cudaStream_t s);
+size_t prefill_ws_bytes(int B, int Hq, int Hkv, int N, int D, int k_vert);
+cudaError_t launch_prefill(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
+                           const __nv_bfloat16 *v, const int32_t *idx, int B, int Hq, int Hkv,
+                           int N, int D, int window, int k_vert, float scale, float *out,
+                           uint8_t *ws, uint32_t *status, cudaStream_t s);
+
+// ---------------------------------------------------------------------------
+// Small device helpers.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+template <typename T>
+__device__ __forceinline__ T warp_sum(T x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+// Index of the first element of sorted a[0..n) that is > x.
+__device__ __forceinline__ int upper_bound_i32(const int32_t *a, int n, int x) {
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    int mid = (lo + hi) >> 1;
+    if (__ldg(a + mid) <= x) lo = mid + 1;
+    else hi = mid;
+  }
+  return lo;
+}
+
+}  // namespace hq

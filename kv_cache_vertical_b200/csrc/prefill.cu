@@ -1,0 +1,526 @@
+// prefill.cu -- hybrid-precision prefill attention.
+//
+// Method: ACL abstract of HyQuant, Prefill stage: a hybrid-precision attention
+// operator keeps the vertical-line tokens and a local sliding window at full
+// precision and quantizes the remaining context; "HyQuant: Hybrid-Precision
+// Quantization for LLM Attention" (wiki summary), TL;DR: the same rule governs
+// prefill and decode.  Per causal pair (i, j <= i): "high" when j is in the
+// window (j > i - W) or is a vertical column, else "low".  High logits are bf16
+// q.k (fp32 accumulate); low logits are INT8 q.k (exact s32) times the per-row
+// Q scale and per-64-key-block K scale; one online softmax covers both; P.V
+// takes fp16 P and V (V converted exactly from bf16) with fp32 accumulation.
+//
+// Pre-pass (P4): INT8 codes for Q and K, fp16 V, a compact bf16 K / fp16 V copy
+// of the vertical rows (so vertical tiles are dense loads, not gathers), their
+// positions, and a per-64-key bitmap of vertical positions.
+//
+// Main kernel: FA2-style, one CTA per (64-query tile, head, batch), 4 warps of
+// 16 rows, warp-level tensor-core MMAs (s8 m16n8k32 for the low QK tiles, bf16
+// m16n8k16 for the window / vertical QK tiles, f16 m16n8k16 for P.V).  For
+// query tile qt the key tiles are: 64-key tiles kt < qt entirely below the
+// window band (INT8 only, vertical columns masked out), the band tiles that
+// meet the window (INT8 and bf16 both computed, each element takes the one its
+// class asks for), and the compact vertical tiles (bf16, key v counted only for
+// rows with v <= i - W, so every pair is counted exactly once).
+#include <float.h>
+#include <limits.h>
+
+#include "hq_internal.cuh"
+#include "warp_mma.cuh"
+
+namespace hq {
+namespace {
+
+constexpr int TILE = 64;        // queries per CTA, keys per tile, K-scale block
+constexpr int FWARPS = 4;
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ---------------------------------------------------------------------------
+// Pre-pass kernels
+// ---------------------------------------------------------------------------
+
+// One warp per Q row: s = amax / 127, code = clamp(rne(x / s), -127, 127),
+// both divisions single IEEE binary32 roundings.
+template <int D>
+__global__ void quant_q_rows(const __nv_bfloat16 *__restrict__ q, long long nrows,
+                             int8_t *__restrict__ qi8, float *__restrict__ sq) {
+  constexpr int CPL = D / 32;
+  const long long row = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= nrows) return;
+  const uint32_t *src = reinterpret_cast<const uint32_t *>(q + row * D) + lane * (CPL / 2);
+  float x[CPL];
+#pragma unroll
+  for (int i = 0; i < CPL / 2; ++i) {
+    const uint32_t w = src[i];
+    x[2 * i] = bf16_lo(w);
+    x[2 * i + 1] = bf16_hi(w);
+  }
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < CPL; ++i) amax = fmaxf(amax, fabsf(x[i]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const float s = amax == 0.f ? 1.f : __fdiv_rn(amax, 127.f);
+  uint32_t packed = 0;
+#pragma unroll
+  for (int i = 0; i < CPL; ++i) {
+    float c = rintf(__fdiv_rn(x[i], s));
+    c = fminf(fmaxf(c, -127.f), 127.f);
+    packed |= ((uint32_t)(int)c & 0xffu) << (8 * i);
+  }
+  if (CPL == 4) reinterpret_cast<uint32_t *>(qi8 + row * D)[lane] = packed;
+  else reinterpret_cast<uint16_t *>(qi8 + row * D)[lane] = (uint16_t)packed;
+  if (lane == 0) sq[row] = s;
+}
+
+// One CTA (256 threads) per block of 64 keys of one (b, kv head).
+template <int D>
+__global__ void __launch_bounds__(256)
+quant_k_blocks(const __nv_bfloat16 *__restrict__ k, int N, int nblk, int8_t *__restrict__ ki8,
+               float *__restrict__ sk) {
+  const int blk = blockIdx.x, bh = blockIdx.y;
+  const int j0 = blk * TILE, n = min(TILE, N - j0);
+  const int nval = n * D;                                       // values in this block
+  const __nv_bfloat16 *src = k + ((size_t)bh * N + j0) * D;
+  int8_t *dst = ki8 + ((size_t)bh * N + j0) * D;
+  __shared__ float red[8];
+  float amax = 0.f;
+  for (int e = threadIdx.x * 2; e < nval; e += blockDim.x * 2) {
+    const uint32_t w = reinterpret_cast<const uint32_t *>(src)[e / 2];
+    amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(w)), fabsf(bf16_hi(w))));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  amax = red[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) amax = fmaxf(amax, red[w]);
+  const float s = amax == 0.f ? 1.f : __fdiv_rn(amax, 127.f);
+  for (int e = threadIdx.x * 2; e < nval; e += blockDim.x * 2) {
+    const uint32_t w = reinterpret_cast<const uint32_t *>(src)[e / 2];
+    float c0 = fminf(fmaxf(rintf(__fdiv_rn(bf16_lo(w), s)), -127.f), 127.f);
+    float c1 = fminf(fmaxf(rintf(__fdiv_rn(bf16_hi(w), s)), -127.f), 127.f);
+    reinterpret_cast<uint16_t *>(dst)[e / 2] =
+        (uint16_t)(((uint32_t)(int)c0 & 0xffu) | (((uint32_t)(int)c1 & 0xffu) << 8));
+  }
+  if (threadIdx.x == 0) sk[(size_t)bh * nblk + blk] = s;
+}
+
+// bf16 V -> fp16 V (exact for |v| in the fp16 normal range).
+__global__ void v_to_f16(const __nv_bfloat16 *__restrict__ v, __half *__restrict__ vh, long long n2) {
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n2;
+       i += (long long)gridDim.x * blockDim.x) {
+    const uint32_t w = reinterpret_cast<const uint32_t *>(v)[i];
+    reinterpret_cast<__half2 *>(vh)[i] = __floats2half2_rn(bf16_lo(w), bf16_hi(w));
+  }
+}
+
+// Compact copies of the vertical rows (padded to a multiple of 64 with zero
+// rows at position INT_MAX) and the per-64-key vertical bitmap.
+template <int D>
+__global__ void gather_vertical(const __nv_bfloat16 *__restrict__ k, const __half *__restrict__ vh,
+                                const int32_t *__restrict__ idx, int N, int k_vert, int kpad,
+                                __nv_bfloat16 *__restrict__ kv_k, __half *__restrict__ kv_v,
+                                int32_t *__restrict__ kv_pos) {
+  const int r = blockIdx.x, bh = blockIdx.y;  // one CTA (D/8 threads) per padded row
+  const int t = threadIdx.x;                  // 16-byte chunk of the row
+  const int pos = r < k_vert ? idx[(size_t)bh * k_vert + r] : INT_MAX;
+  const size_t dst = ((size_t)bh * kpad + r) * D;
+  uint4 kk = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
+  if (r < k_vert && pos >= 0 && pos < N) {
+    kk = reinterpret_cast<const uint4 *>(k + ((size_t)bh * N + pos) * D)[t];
+    vv = reinterpret_cast<const uint4 *>(vh + ((size_t)bh * N + pos) * D)[t];
+  }
+  reinterpret_cast<uint4 *>(kv_k + dst)[t] = kk;
+  reinterpret_cast<uint4 *>(kv_v + dst)[t] = vv;
+  if (t == 0) kv_pos[(size_t)bh * kpad + r] = pos;
+}
+
+__global__ void vertical_bitmap(const int32_t *__restrict__ idx, int k_vert, int nwords,
+                                unsigned long long *__restrict__ bits) {
+  const int w = blockIdx.x * blockDim.x + threadIdx.x, bh = blockIdx.y;
+  if (w >= nwords) return;
+  const int32_t *id = idx + (size_t)bh * k_vert;
+  int lo = 0, hi = k_vert;  // first entry >= 64 w
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (id[mid] < 64 * w) lo = mid + 1;
+    else hi = mid;
+  }
+  unsigned long long m = 0;
+  for (int e = lo; e < k_vert && id[e] < 64 * (w + 1); ++e) m |= 1ull << (id[e] - 64 * w);
+  bits[(size_t)bh * nwords + w] = m;
+}
+
+// ---------------------------------------------------------------------------
+// Main kernel (warp-level MMA version)
+// ---------------------------------------------------------------------------
+struct PrefillArgs {
+  const __nv_bfloat16 *q, *k;
+  const int8_t *qi8, *ki8;
+  const float *sq, *sk;
+  const __half *vh;
+  const __nv_bfloat16 *vk;       // compact vertical K [nbh, kpad, D]
+  const __half *vv;              // compact vertical V
+  const int32_t *vpos;           // [nbh, kpad]
+  const unsigned long long *vbits;  // [nbh, nblk]
+  float *out;
+  int Hq, Hkv, G, N, window, kpad, nblk;
+  float scale_log2;
+};
+
+template <int D>
+struct Smem {
+  uint4 ki8[TILE * D / 16];      // 64 keys x D bytes
+  uint4 kbf[TILE * D / 8];       // 64 keys x D bf16
+  uint4 vh[TILE * D / 8];        // 64 keys x D fp16
+};
+
+// Smem index of 16-byte chunk `ch` of row `row` in a tile with CH chunks per
+// row: the chunk index is XOR-swizzled by the low row bits so that the eight
+// row addresses of one ldmatrix hit distinct bank groups.
+template <int CH>
+__device__ __forceinline__ int swz(int row, int ch) {
+  return row * CH + (ch ^ (row & (CH >= 8 ? 7 : CH - 1)));
+}
+
+// Copy a [rows x RB bytes] tile (rows at stride RB in global) into smem with
+// the 16-byte chunk index XOR-swizzled by (row & 7); rows >= nvalid are zero.
+template <int RB>
+__device__ __forceinline__ void load_tile(uint4 *dst, const uint8_t *src, int nvalid) {
+  constexpr int CH = RB / 16;
+  for (int t = threadIdx.x; t < TILE * CH; t += FWARPS * 32) {
+    const int row = t / CH, ch = t % CH;
+    uint4 val = make_uint4(0, 0, 0, 0);
+    if (row < nvalid) val = *reinterpret_cast<const uint4 *>(src + (size_t)row * RB + ch * 16);
+    dst[swz<CH>(row, ch)] = val;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(FWARPS * 32)
+prefill_mma(PrefillArgs a) {
+  constexpr int CH16 = D / 8;     // 16-byte chunks in a 16-bit row
+  constexpr int CH8 = D / 16;     // 16-byte chunks in an 8-bit row
+  constexpr int NT = TILE / 8;    // 8-key n-tiles per key tile
+  __shared__ Smem<D> sm;
+  const int ntiles = (a.N + TILE - 1) / TILE;
+  const int qt = ntiles - 1 - blockIdx.x;  // heaviest tiles first
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int kh = h / a.G;
+  const size_t bh = (size_t)b * a.Hkv + kh;
+  const size_t bhq = (size_t)b * a.Hq + h;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = lane >> 2, c = lane & 3;
+  const int row0 = qt * TILE + warp * 16;
+  const int rows[2] = {row0 + r, row0 + r + 8};
+  const int W = a.window;
+
+  // Q fragments: bf16 (m16n8k16 A) and INT8 (m16n8k32 A), rows r and r+8.
+  uint32_t qb[D / 16][4], qi[D / 32][4];
+  float sqr[2];
+#pragma unroll
+  for (int hf = 0; hf < 2; ++hf) {
+    const bool ok = rows[hf] < a.N;
+    const uint32_t *pb = reinterpret_cast<const uint32_t *>(a.q + (bhq * a.N + rows[hf]) * D);
+    const uint32_t *pi = reinterpret_cast<const uint32_t *>(a.qi8 + (bhq * a.N + rows[hf]) * D);
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      qb[ks][hf] = ok ? pb[ks * 8 + c] : 0u;
+      qb[ks][hf + 2] = ok ? pb[ks * 8 + 4 + c] : 0u;
+    }
+#pragma unroll
+    for (int ks = 0; ks < D / 32; ++ks) {
+      qi[ks][hf] = ok ? pi[ks * 8 + c] : 0u;
+      qi[ks][hf + 2] = ok ? pi[ks * 8 + 4 + c] : 0u;
+    }
+    sqr[hf] = ok ? a.sq[bhq * a.N + rows[hf]] * a.scale_log2 : 0.f;
+  }
+
+  float o[D / 8][4];
+#pragma unroll
+  for (int nt = 0; nt < D / 8; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+  float m[2] = {-1e30f, -1e30f}, l[2] = {0.f, 0.f};
+
+  // S (16 x 64) -> online softmax -> O += P V for the tile in smem.
+  auto softmax_pv = [&](float (&s)[NT][4]) {
+    float mx[2] = {m[0], m[1]};
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      mx[0] = fmaxf(mx[0], fmaxf(s[nt][0], s[nt][1]));
+      mx[1] = fmaxf(mx[1], fmaxf(s[nt][2], s[nt][3]));
+    }
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      mx[hf] = fmaxf(mx[hf], __shfl_xor_sync(0xffffffffu, mx[hf], 1));
+      mx[hf] = fmaxf(mx[hf], __shfl_xor_sync(0xffffffffu, mx[hf], 2));
+    }
+    const float al[2] = {exp2f(m[0] - mx[0]), exp2f(m[1] - mx[1])};
+    m[0] = mx[0];
+    m[1] = mx[1];
+    uint32_t pa[NT / 2][4];
+    float rs[2] = {0.f, 0.f};
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const float p0 = exp2f(s[nt][0] - mx[0]), p1 = exp2f(s[nt][1] - mx[0]);
+      const float p2 = exp2f(s[nt][2] - mx[1]), p3 = exp2f(s[nt][3] - mx[1]);
+      rs[0] += p0 + p1;
+      rs[1] += p2 + p3;
+      pa[nt / 2][(nt & 1) * 2 + 0] = pack_f16x2(p0, p1);
+      pa[nt / 2][(nt & 1) * 2 + 1] = pack_f16x2(p2, p3);
+    }
+    l[0] = l[0] * al[0] + rs[0];
+    l[1] = l[1] * al[1] + rs[1];
+#pragma unroll
+    for (int nt = 0; nt < D / 8; ++nt) {
+      o[nt][0] *= al[0];
+      o[nt][1] *= al[0];
+      o[nt][2] *= al[1];
+      o[nt][3] *= al[1];
+    }
+#pragma unroll
+    for (int kk = 0; kk < NT / 2; ++kk) {
+#pragma unroll
+      for (int dp = 0; dp < D / 16; ++dp) {
+        // V rows kk*16 .. +15, d chunks 2dp, 2dp+1 -> B frags of n-tiles 2dp, 2dp+1
+        const int key = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+        const int ch = dp * 2 + (lane >> 4);
+        uint32_t vb[4];
+        ldsm_x4_t(vb, smem_u32(&sm.vh[swz<CH16>(key, ch)]));
+        mma_f16_16816(o[2 * dp], pa[kk], vb[0], vb[1]);
+        mma_f16_16816(o[2 * dp + 1], pa[kk], vb[2], vb[3]);
+      }
+    }
+  };
+
+  auto qk_int8 = [&](float (&s)[NT][4], float ks_scale) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      int acc[4] = {0, 0, 0, 0};
+#pragma unroll
+      for (int kp = 0; kp < D / 64; ++kp) {
+        const int key = nt * 8 + (lane & 7);
+        const int ch = kp * 4 + (lane >> 3);
+        uint32_t kb[4];
+        ldsm_x4(kb, smem_u32(&sm.ki8[swz<CH8>(key, ch)]));
+        mma_s8_16832(acc, qi[2 * kp], kb[0], kb[1]);
+        mma_s8_16832(acc, qi[2 * kp + 1], kb[2], kb[3]);
+      }
+      s[nt][0] = (float)acc[0] * (sqr[0] * ks_scale);
+      s[nt][1] = (float)acc[1] * (sqr[0] * ks_scale);
+      s[nt][2] = (float)acc[2] * (sqr[1] * ks_scale);
+      s[nt][3] = (float)acc[3] * (sqr[1] * ks_scale);
+    }
+  };
+
+  auto qk_bf16 = [&](float (&s)[NT][4]) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int kp = 0; kp < D / 32; ++kp) {
+        const int key = nt * 8 + (lane & 7);
+        const int ch = kp * 4 + (lane >> 3);
+        uint32_t kb[4];
+        ldsm_x4(kb, smem_u32(&sm.kbf[swz<CH16>(key, ch)]));
+        mma_bf16_16816(acc, qb[2 * kp], kb[0], kb[1]);
+        mma_bf16_16816(acc, qb[2 * kp + 1], kb[2], kb[3]);
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) s[nt][e] = acc[e] * a.scale_log2;
+    }
+  };
+
+  const int i_min = qt * TILE;
+  // 1) key tiles 0 .. qt (INT8, plus bf16 where the window reaches)
+  for (int kt = 0; kt <= qt; ++kt) {
+    const int j0 = kt * TILE;
+    const int nvalid = min(TILE, a.N - j0);
+    const bool band = (j0 + TILE - 1 >= i_min - W + 1) || kt == qt;
+    __syncthreads();
+    load_tile<D>(sm.ki8, reinterpret_cast<const uint8_t *>(a.ki8 + (bh * a.N + j0) * D), nvalid);
+    load_tile<D * 2>(sm.vh, reinterpret_cast<const uint8_t *>(a.vh + (bh * a.N + j0) * D), nvalid);
+    if (band && W > 0)
+      load_tile<D * 2>(sm.kbf, reinterpret_cast<const uint8_t *>(a.k + (bh * a.N + j0) * D), nvalid);
+    __syncthreads();
+    const unsigned long long vbits = a.vbits[bh * a.nblk + kt];
+    float s[NT][4];
+    qk_int8(s, a.sk[bh * a.nblk + kt]);
+    if (band) {
+      float sb[NT][4];
+      if (W > 0) qk_bf16(sb);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i = rows[e >> 1];
+          const int jj = nt * 8 + 2 * c + (e & 1);
+          const int j = j0 + jj;
+          float v = s[nt][e];
+          if (j > i) v = -INFINITY;
+          else if (j > i - W) v = W > 0 ? sb[nt][e] : v;
+          else if ((vbits >> jj) & 1ull) v = -INFINITY;
+          s[nt][e] = v;
+        }
+    } else if (vbits) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int jj = nt * 8 + 2 * c + (e & 1);
+          if ((vbits >> jj) & 1ull) s[nt][e] = -INFINITY;
+        }
+    }
+    softmax_pv(s);
+  }
+  // 2) compact vertical tiles: key v counts for row i only when v <= i - W
+  const int i_max = min(qt * TILE + TILE - 1, a.N - 1);
+  const int32_t *vp = a.vpos + bh * a.kpad;
+  for (int vt = 0; vt * TILE < a.kpad; ++vt) {
+    if (vp[vt * TILE] > i_max - W) break;
+    __syncthreads();
+    load_tile<D * 2>(sm.kbf, reinterpret_cast<const uint8_t *>(a.vk + (bh * a.kpad + vt * TILE) * D), TILE);
+    load_tile<D * 2>(sm.vh, reinterpret_cast<const uint8_t *>(a.vv + (bh * a.kpad + vt * TILE) * D), TILE);
+    __syncthreads();
+    float s[NT][4];
+    qk_bf16(s);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = rows[e >> 1];
+        const int pos = vp[vt * TILE + nt * 8 + 2 * c + (e & 1)];
+        if (pos > i - W) s[nt][e] = -INFINITY;  // INT_MAX padding is masked too
+      }
+    softmax_pv(s);
+  }
+  // 3) normalize and store fp32 rows
+#pragma unroll
+  for (int hf = 0; hf < 2; ++hf) {
+    l[hf] += __shfl_xor_sync(0xffffffffu, l[hf], 1);
+    l[hf] += __shfl_xor_sync(0xffffffffu, l[hf], 2);
+  }
+#pragma unroll
+  for (int hf = 0; hf < 2; ++hf) {
+    if (rows[hf] >= a.N) continue;
+    const float inv = 1.f / l[hf];
+    float *dst = a.out + (bhq * a.N + rows[hf]) * D;
+#pragma unroll
+    for (int nt = 0; nt < D / 8; ++nt)
+      *reinterpret_cast<float2 *>(dst + nt * 8 + 2 * c) =
+          make_float2(o[nt][2 * hf] * inv, o[nt][2 * hf + 1] * inv);
+  }
+}
+
+struct PrefillWs {
+  int8_t *qi8, *ki8;
+  float *sq, *sk;
+  __half *vh, *vv;
+  __nv_bfloat16 *vk;
+  int32_t *vpos;
+  unsigned long long *vbits;
+  size_t total;
+};
+
+PrefillWs carve(uint8_t *base, int B, int Hq, int Hkv, int N, int D, int k_vert) {
+  PrefillWs w;
+  const size_t nbh = (size_t)B * Hkv, nbq = (size_t)B * Hq;
+  const int nblk = (N + TILE - 1) / TILE;
+  const size_t kpad = (size_t)((k_vert + TILE - 1) / TILE) * TILE;
+  size_t off = kWsHeader;
+  auto take = [&](size_t bytes) {
+    uint8_t *p = base ? base + off : nullptr;
+    off = align_up(off + bytes, 256);
+    return p;
+  };
+  w.qi8 = (int8_t *)take(nbq * N * D);
+  w.sq = (float *)take(nbq * N * sizeof(float));
+  w.ki8 = (int8_t *)take(nbh * N * D);
+  w.sk = (float *)take(nbh * nblk * sizeof(float));
+  w.vh = (__half *)take(nbh * N * D * 2);
+  w.vk = (__nv_bfloat16 *)take(nbh * kpad * D * 2);
+  w.vv = (__half *)take(nbh * kpad * D * 2);
+  w.vpos = (int32_t *)take(nbh * kpad * sizeof(int32_t));
+  w.vbits = (unsigned long long *)take(nbh * nblk * sizeof(unsigned long long));
+  w.total = off;
+  return w;
+}
+
+template <int D>
+cudaError_t quant_t(const __nv_bfloat16 *q, const __nv_bfloat16 *k, int B, int Hq, int Hkv, int N,
+                    int8_t *qi8, float *sq, int8_t *ki8, float *sk, cudaStream_t s) {
+  const long long nrows = (long long)B * Hq * N;
+  quant_q_rows<D><<<(unsigned)((nrows + 7) / 8), 256, 0, s>>>(q, nrows, qi8, sq);
+  const int nblk = (N + TILE - 1) / TILE;
+  quant_k_blocks<D><<<dim3(nblk, B * Hkv), 256, 0, s>>>(k, N, nblk, ki8, sk);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t prefill_t(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
+                      const int32_t *idx, int B, int Hq, int Hkv, int N, int window, int k_vert,
+                      float scale, float *out, uint8_t *ws, cudaStream_t s) {
+  PrefillWs w = carve(ws, B, Hq, Hkv, N, D, k_vert);
+  const int nbh = B * Hkv;
+  const int nblk = (N + TILE - 1) / TILE;
+  const int kpad = (k_vert + TILE - 1) / TILE * TILE;
+  cudaError_t e = quant_t<D>(q, k, B, Hq, Hkv, N, w.qi8, w.sq, w.ki8, w.sk, s);
+  if (e != cudaSuccess) return e;
+  const long long n2 = (long long)nbh * N * D / 2;
+  v_to_f16<<<1184, 256, 0, s>>>(v, w.vh, n2);
+  if (kpad > 0)
+    gather_vertical<D><<<dim3(kpad, nbh), D / 8, 0, s>>>(k, w.vh, idx, N, k_vert, kpad, w.vk,
+                                                         w.vv, w.vpos);
+  vertical_bitmap<<<dim3((nblk + 127) / 128, nbh), 128, 0, s>>>(idx, k_vert, nblk, w.vbits);
+  PrefillArgs a;
+  a.q = q;
+  a.k = k;
+  a.qi8 = w.qi8;
+  a.ki8 = w.ki8;
+  a.sq = w.sq;
+  a.sk = w.sk;
+  a.vh = w.vh;
+  a.vk = w.vk;
+  a.vv = w.vv;
+  a.vpos = w.vpos;
+  a.vbits = w.vbits;
+  a.out = out;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.G = Hq / Hkv;
+  a.N = N;
+  a.window = window;
+  a.kpad = kpad;
+  a.nblk = nblk;
+  a.scale_log2 = scale * kLog2e;
+  prefill_mma<D><<<dim3(nblk, Hq, B), FWARPS * 32, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_quant(const __nv_bfloat16 *q, const __nv_bfloat16 *k, int B, int Hq,
+                                 int Hkv, int N, int D, int8_t *qi8, float *sq, int8_t *ki8,
+                                 float *sk, cudaStream_t s) {
+  if (D == 128) return quant_t<128>(q, k, B, Hq, Hkv, N, qi8, sq, ki8, sk, s);
+  if (D == 64) return quant_t<64>(q, k, B, Hq, Hkv, N, qi8, sq, ki8, sk, s);
+  return cudaErrorInvalidValue;
+}
+
+size_t prefill_ws_bytes(int B, int Hq, int Hkv, int N, int D, int k_vert) {
+  return carve(nullptr, B, Hq, Hkv, N, D, k_vert).total;
+}
+
+cudaError_t launch_prefill(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
+                           const __nv_bfloat16 *v, const int32_t *idx, int B, int Hq, int Hkv,
+                           int N, int D, int window, int k_vert, float scale, float *out,
+                           uint8_t *ws, uint32_t *status, cudaStream_t s) {
+  (void)status;
+  if (D == 128) return prefill_t<128>(q, k, v, idx, B, Hq, Hkv, N, window, k_vert, scale, out, ws, s);
+  if (D == 64) return prefill_t<64>(q, k, v, idx, B, Hq, Hkv, N, window, k_vert, scale, out, ws, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace hq

@@ -1,0 +1,254 @@
+"""ctypes binding of libhq.so (include/hq.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of libhq.so.  PyTorch supplies device memory and the current CUDA
+stream.  The ``hq_*`` functions mirror the C entry points one to one (device
+tensors in, status checked); the lower-case helpers allocate outputs and
+workspaces with torch and then call them.
+
+There is no CPU fallback: importing this module raises if libhq.so is
+missing, and every call needs CUDA tensors.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import math
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libhq.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is not built; run `python -m kv_cache_vertical_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+_SZ = ctypes.c_size_t
+
+HQ_OK = 0
+HQ_DEV_BAD_INDEX = 0x1
+HQ_DEV_TIMEOUT = 0x2
+
+
+class hq_kv_cache(ctypes.Structure):
+    _fields_ = [("k_codes", _P), ("v_codes", _P), ("k_sz", _P), ("v_sz", _P), ("k_hi", _P),
+                ("v_hi", _P), ("lo_pos", _P), ("n_lo", _I), ("n_hi", _I), ("bits", _I),
+                ("group", _I)]
+
+
+def _sig(name, restype, *argtypes):
+    f = getattr(_lib, name)
+    f.restype = restype
+    f.argtypes = list(argtypes)
+    return f
+
+
+_status_string = _sig("hq_status_string", ctypes.c_char_p, _I)
+hq_version = _sig("hq_version", _I)
+_read_status = _sig("hq_read_device_status", _I, _P, _I, ctypes.POINTER(ctypes.c_uint32), _P)
+hq_probe_workspace_size = _sig("hq_probe_workspace_size", _SZ, _I, _I, _I, _I, _I, _I)
+_probe = _sig("hq_probe_vertical", _I, _P, ctypes.c_int64, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F,
+              _P, _P, _P, _SZ, _P)
+_pack = _sig("hq_pack_kv", _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I,
+             ctypes.POINTER(hq_kv_cache), _P, _SZ, _P)
+hq_decode_workspace_size = _sig("hq_decode_workspace_size", _SZ, _I, _I, _I, _I, _I, _I, _I)
+_decode = _sig("hq_decode_attn", _I, _P, ctypes.POINTER(hq_kv_cache), _I, _I, _I, _I, _F, _P, _P,
+               _P, _SZ, _P)
+_pquant = _sig("hq_prefill_quant", _I, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P)
+hq_prefill_workspace_size = _sig("hq_prefill_workspace_size", _SZ, _I, _I, _I, _I, _I, _I)
+_prefill = _sig("hq_prefill_attn", _I, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P,
+                _SZ, _P)
+
+EXPORTED = ["hq_status_string", "hq_version", "hq_read_device_status", "hq_probe_workspace_size",
+            "hq_probe_vertical", "hq_pack_kv", "hq_decode_workspace_size", "hq_decode_attn",
+            "hq_prefill_quant", "hq_prefill_workspace_size", "hq_prefill_attn"]
+
+
+class HQError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {hq_status_string(status)}")
+
+
+def hq_status_string(status: int) -> str:
+    return _status_string(status).decode()
+
+
+def _check(rc: int, what: str):
+    if rc != HQ_OK:
+        raise HQError(rc, what)
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libhq takes CUDA tensors only")
+    return t.data_ptr()
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def workspace(nbytes: int, device=None) -> torch.Tensor:
+    """A zeroed device workspace (the library keeps it reusable afterwards)."""
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device or "cuda")
+
+
+def hq_read_device_status(ws: torch.Tensor, clear: bool = False, stream=None) -> int:
+    v = ctypes.c_uint32(0)
+    _check(_read_status(_ptr(ws), int(clear), ctypes.byref(v), _stream(stream)),
+           "hq_read_device_status")
+    return v.value
+
+
+# ---------------------------------------------------------------------------
+# Hybrid KV cache
+# ---------------------------------------------------------------------------
+@dataclasses.dataclass
+class KVCache:
+    k_codes: torch.Tensor
+    v_codes: torch.Tensor
+    k_sz: torch.Tensor
+    v_sz: torch.Tensor
+    k_hi: torch.Tensor
+    v_hi: torch.Tensor
+    lo_pos: torch.Tensor | None
+    n_lo: int
+    n_hi: int
+    bits: int
+    group: int = 32
+
+    @classmethod
+    def empty(cls, B, Hkv, L, D, window, k_vert, bits, device="cuda", with_pos=True):
+        n_lo, n_hi = L - window - k_vert, k_vert + window
+        u8 = dict(dtype=torch.uint8, device=device)
+        return cls(
+            k_codes=torch.empty(B, Hkv, n_lo, D * bits // 8, **u8),
+            v_codes=torch.empty(B, Hkv, n_lo, D * bits // 8, **u8),
+            k_sz=torch.empty(B, Hkv, n_lo, D // 32, 2, dtype=torch.float16, device=device),
+            v_sz=torch.empty(B, Hkv, n_lo, D // 32, 2, dtype=torch.float16, device=device),
+            k_hi=torch.empty(B, Hkv, n_hi, D, dtype=torch.bfloat16, device=device),
+            v_hi=torch.empty(B, Hkv, n_hi, D, dtype=torch.bfloat16, device=device),
+            lo_pos=torch.empty(B, Hkv, n_lo, dtype=torch.int32, device=device) if with_pos else None,
+            n_lo=n_lo, n_hi=n_hi, bits=bits)
+
+    def struct(self) -> hq_kv_cache:
+        return hq_kv_cache(_ptr(self.k_codes), _ptr(self.v_codes), _ptr(self.k_sz),
+                           _ptr(self.v_sz), _ptr(self.k_hi), _ptr(self.v_hi), _ptr(self.lo_pos),
+                           self.n_lo, self.n_hi, self.bits, self.group)
+
+    def nbytes(self, with_pos: bool = False) -> int:
+        ts = [self.k_codes, self.v_codes, self.k_sz, self.v_sz, self.k_hi, self.v_hi]
+        if with_pos and self.lo_pos is not None:
+            ts.append(self.lo_pos)
+        return sum(t.numel() * t.element_size() for t in ts)
+
+
+# ---------------------------------------------------------------------------
+# Entry points (same names as the C ABI)
+# ---------------------------------------------------------------------------
+def hq_probe_vertical(q_probe, q_head_stride, k, B, Hq, Hkv, P, L, D, window, k_vert,
+                      softmax_scale, idx_out, score_out, ws, stream=None):
+    _check(_probe(_ptr(q_probe), int(q_head_stride), _ptr(k), B, Hq, Hkv, P, L, D, window, k_vert,
+                  float(softmax_scale), _ptr(idx_out), _ptr(score_out), _ptr(ws),
+                  ws.numel() if ws is not None else 0, _stream(stream)), "hq_probe_vertical")
+
+
+def hq_pack_kv(k, v, idx, B, Hkv, L, D, window, k_vert, bits, group, cache: KVCache, ws=None,
+               stream=None):
+    st = cache.struct()
+    _check(_pack(_ptr(k), _ptr(v), _ptr(idx), B, Hkv, L, D, window, k_vert, bits, group,
+                 ctypes.byref(st), _ptr(ws), ws.numel() if ws is not None else 0,
+                 _stream(stream)), "hq_pack_kv")
+
+
+def hq_decode_attn(q, cache: KVCache, B, Hq, Hkv, D, softmax_scale, out, lse_out, ws, stream=None):
+    st = cache.struct()
+    _check(_decode(_ptr(q), ctypes.byref(st), B, Hq, Hkv, D, float(softmax_scale), _ptr(out),
+                   _ptr(lse_out), _ptr(ws), ws.numel() if ws is not None else 0, _stream(stream)),
+           "hq_decode_attn")
+
+
+def hq_prefill_quant(q, k, B, Hq, Hkv, N, D, qi8, sq, ki8, sk, stream=None):
+    _check(_pquant(_ptr(q), _ptr(k), B, Hq, Hkv, N, D, _ptr(qi8), _ptr(sq), _ptr(ki8), _ptr(sk),
+                   _stream(stream)), "hq_prefill_quant")
+
+
+def hq_prefill_attn(q, k, v, idx, B, Hq, Hkv, N, D, window, k_vert, softmax_scale, out, ws,
+                    stream=None):
+    _check(_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(idx), B, Hq, Hkv, N, D, window, k_vert,
+                    float(softmax_scale), _ptr(out), _ptr(ws), ws.numel() if ws is not None else 0,
+                    _stream(stream)), "hq_prefill_attn")
+
+
+# ---------------------------------------------------------------------------
+# Convenience helpers (allocate with torch, then call the entry points)
+# ---------------------------------------------------------------------------
+def probe_vertical(q_probe, k, window, k_vert, scale=0.0, want_scores=False, ws=None):
+    """q_probe: bf16 [B,Hq,P,D] (any head stride, rows contiguous); k: bf16 [B,Hkv,L,D]."""
+    B, Hq, P, D = q_probe.shape
+    Hkv, L = k.shape[1], k.shape[2]
+    assert q_probe.stride(3) == 1 and q_probe.stride(2) == D and q_probe.stride(0) == Hq * q_probe.stride(1)
+    idx = torch.empty(B, Hkv, k_vert, dtype=torch.int32, device=k.device)
+    score = torch.empty(B, Hkv, L, dtype=torch.float32, device=k.device) if want_scores else None
+    if ws is None:
+        ws = workspace(hq_probe_workspace_size(B, Hq, Hkv, P, L, D), k.device)
+    hq_probe_vertical(q_probe, q_probe.stride(1), k, B, Hq, Hkv, P, L, D, window, k_vert, scale,
+                      idx, score, ws)
+    return (idx, score) if want_scores else idx
+
+
+def pack_kv(k, v, idx, window, bits=4, ws=None, with_pos=True) -> KVCache:
+    B, Hkv, L, D = k.shape
+    k_vert = idx.shape[2]
+    cache = KVCache.empty(B, Hkv, L, D, window, k_vert, bits, k.device, with_pos)
+    hq_pack_kv(k, v, idx, B, Hkv, L, D, window, k_vert, bits, 32, cache, ws)
+    return cache
+
+
+def decode_attn(q, cache: KVCache, Hkv, scale=0.0, ws=None, want_lse=False):
+    B, Hq, D = q.shape
+    out = torch.empty(B, Hq, D, dtype=torch.float32, device=q.device)
+    lse = torch.empty(B, Hq, dtype=torch.float32, device=q.device) if want_lse else None
+    if ws is None:
+        ws = workspace(hq_decode_workspace_size(B, Hq, Hkv, D, cache.n_lo, cache.n_hi, cache.bits),
+                       q.device)
+    hq_decode_attn(q, cache, B, Hq, Hkv, D, scale, out, lse, ws)
+    return (out, lse) if want_lse else out
+
+
+def prefill_quant(q, k):
+    B, Hq, N, D = q.shape
+    Hkv = k.shape[1]
+    nblk = (N + 63) // 64
+    qi8 = torch.empty(B, Hq, N, D, dtype=torch.int8, device=q.device)
+    sq = torch.empty(B, Hq, N, dtype=torch.float32, device=q.device)
+    ki8 = torch.empty(B, Hkv, N, D, dtype=torch.int8, device=q.device)
+    sk = torch.empty(B, Hkv, nblk, dtype=torch.float32, device=q.device)
+    hq_prefill_quant(q, k, B, Hq, Hkv, N, D, qi8, sq, ki8, sk)
+    return qi8, sq, ki8, sk
+
+
+def prefill_attn(q, k, v, idx, window, scale=0.0, ws=None, out=None):
+    B, Hq, N, D = q.shape
+    Hkv = k.shape[1]
+    k_vert = idx.shape[2]
+    if out is None:
+        out = torch.empty(B, Hq, N, D, dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = workspace(hq_prefill_workspace_size(B, Hq, Hkv, N, D, k_vert), q.device)
+    hq_prefill_attn(q, k, v, idx, B, Hq, Hkv, N, D, window, k_vert, scale, out, ws)
+    return out
+
+
+def default_scale(D: int) -> float:
+    return 1.0 / math.sqrt(D)

@@ -1,0 +1,96 @@
+"""GPU parity of the hybrid prefill path: INT8 pre-pass and hybrid attention.
+
+The index list comes from the oracle's probe (checked against the GPU probe
+modulo ties); every expected value is the fp64 oracle's on the same inputs.
+"""
+import fractions
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from hq_testutil import assert_close, assert_index_sets, to_dev
+from kv_cache_vertical_b200.synth import F5, WORKLOADS, Workload, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def hq():
+    from kv_cache_vertical_b200 import hq as m
+    return m
+
+
+def oracle_idx(x, w: Workload):
+    if w.k_vert == 0:
+        return np.zeros((w.B, w.Hkv, 0), np.int32), None
+    qp = x["q"][:, :, w.L - 64:].contiguous()
+    sc = oracle.probe_scores(qp, x["k"], w.Hkv)
+    return oracle.topk(sc, w.window, w.k_vert), sc
+
+
+def run_prefill_case(w: Workload, rows=None, check_probe=True):
+    H = hq()
+    x = make_inputs(w)
+    d = to_dev(x)
+    ridx, rsc = oracle_idx(x, w)
+    if check_probe and w.k_vert > 0:
+        gidx = H.probe_vertical(d["q"][:, :, w.L - 64:], d["k"], w.window, w.k_vert)
+        torch.cuda.synchronize()
+        assert_index_sets(gidx.cpu().numpy(), ridx, rsc, w.window)
+    # INT8 pre-pass: bit-exact
+    gq = [t.cpu().numpy() for t in H.prefill_quant(d["q"], d["k"])]
+    rq = oracle.prefill_quant(x["q"], x["k"], w.Hkv)
+    for g, r, name in zip(gq, rq, ("qi8", "sq", "ki8", "sk")):
+        assert np.array_equal(g, r), f"{name} differs"
+    out = H.prefill_attn(d["q"], d["k"], d["v"], torch.from_numpy(ridx).cuda(), w.window)
+    torch.cuda.synchronize()
+    ref = oracle.prefill_attn(x["q"], x["k"], x["v"], ridx, w.window, quant=rq, rows=rows)
+    g = out.cpu().numpy()
+    if rows is not None:
+        g = g[:, :, rows]
+    return assert_close(g, ref, f"prefill {w.name}")
+
+
+@pytest.mark.parametrize("G", [1, 4])
+def test_prefill_small_ragged(G):
+    w = Workload("p", "prefill", 1, 2 * G, 2, 128, 1000, 128, F5, 4, 11 + G)
+    run_prefill_case(w)
+
+
+def test_prefill_head_dim_64_batch_2():
+    w = Workload("p64", "prefill", 2, 4, 1, 64, 700, 64, F5, 4, 21)
+    run_prefill_case(w)
+
+
+def test_prefill_window_larger_than_sequence():
+    # everything is high precision: plain causal bf16 attention
+    w = Workload("allhi", "prefill", 1, 2, 1, 128, 300, 400, fractions.Fraction(0), 4, 22)
+    run_prefill_case(w, check_probe=False)
+
+
+def test_prefill_no_window_no_vertical():
+    # everything INT8
+    w = Workload("alllo", "prefill", 1, 2, 1, 128, 513, 0, fractions.Fraction(0), 4, 23)
+    run_prefill_case(w, check_probe=False)
+
+
+def test_prefill_many_verticals_small_window():
+    w = Workload("vert", "prefill", 1, 8, 1, 128, 1100, 16, fractions.Fraction(1, 4), 4, 24)
+    run_prefill_case(w)
+
+
+def test_prefill_medium_all_rows():
+    w = Workload("med", "prefill", 1, 8, 2, 128, 4096, 128, F5, 4, 25)
+    run_prefill_case(w)
+
+
+@pytest.mark.slow
+def test_prefill_full_size_sampled_rows():
+    w = WORKLOADS["llama8b_prefill_32k"]
+    rng = np.random.default_rng(5)
+    N, W = w.L, w.window
+    rows = np.unique(np.concatenate([
+        np.arange(0, 8), np.arange(W - 4, W + 4), rng.integers(0, N, 48),
+        np.arange(N - 64, N, 8), [N - 1]])).astype(np.int32)
+    run_prefill_case(w, rows=rows)
