@@ -10,7 +10,9 @@
 // Work split: one CTA per (split of the cached rows, b, kv head); a CTA scores
 // its rows for the G query heads of the KV head, keeps an online softmax
 // (running max, sum, output) per head, and writes one partial; a combine
-// kernel merges the partials with the usual max-rescaled sums.
+// kernel merges the partials with the usual max-rescaled sums.  This simple
+// CUDA-core version serves head_dim 64; head_dim 128 goes to the TMA +
+// tensor-core kernel of decode_tma.cu.
 #include <float.h>
 
 #include "hq_internal.cuh"
@@ -197,7 +199,7 @@ cudaError_t launch_g(const DecodeArgs &a, int nbh, float *out, float *lse, cudaS
 }  // namespace
 
 size_t decode_ws_bytes(int B, int Hq, int Hkv, int D, int n_lo, int n_hi, int bits) {
-  (void)bits;
+  if (decode_tma_supported(D, bits, Hq / Hkv)) return decode_tma_ws_bytes(B, Hq, Hkv, n_lo, n_hi, bits);
   const int nbh = B * Hkv;
   const int ns = choose_nsplit(nbh, n_lo + n_hi);
   size_t off = kWsHeader;
@@ -209,7 +211,8 @@ size_t decode_ws_bytes(int B, int Hq, int Hkv, int D, int n_lo, int n_hi, int bi
 cudaError_t launch_decode(const __nv_bfloat16 *q, const hq_kv_cache &c, int B, int Hq, int Hkv,
                           int D, float scale, float *out, float *lse, uint8_t *ws,
                           uint32_t *status, cudaStream_t s) {
-  (void)status;
+  if (decode_tma_supported(D, c.bits, Hq / Hkv))
+    return launch_decode_tma(q, c, B, Hq, Hkv, scale, out, lse, ws, status, s);
   DecodeArgs a;
   a.q = q;
   a.k_codes = (const uint8_t *)c.k_codes;

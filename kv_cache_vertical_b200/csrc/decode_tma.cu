@@ -1,0 +1,815 @@
+// decode_tma.cu -- bandwidth-oriented split-KV decode over the hybrid KV cache
+// (head_dim 128), dequantization fused into tensor-core MMAs.
+//
+// Method: "HyQuant: Hybrid-Precision Quantization for LLM Attention" (wiki
+// summary), TL;DR and "Key results": the decode kernel reads the low-bit cache
+// and dequantizes inside attention, so no dequantized value returns to memory;
+// the vertical-line rows and the window are read in bf16.
+//
+// Layout of the work: each CTA owns a contiguous range of 64-token tiles of
+// the low segment or of the bf16 segment of one (b, kv head)
+// ("split"), streamed global -> shared memory by TMA (one producer warp,
+// mbarrier ring of NSTAGE stages, 64B/128B swizzle so that ldmatrix reads are
+// bank-conflict free).  Each of the four consumer warps takes one 16-token
+// sub-tile of every stage:
+//
+//   S^T = Kcode * q'  -- tokens are the MMA rows, the G <= 8 query heads of the
+//       KV head the 8 MMA columns.  Codes enter the MMA exactly (fp16 1024+c
+//       bit tricks), one accumulator per 32-channel group, so the per-token
+//       fp16 scale is applied afterwards in fp32:  q.k^ = sum_g s_g (q_g . c_g)
+//       + sum_g z_g Q_g, the second term by one more MMA (z exact in fp16, Q_g
+//       split into two fp16 halves).
+//   O^T += Vcode^T * (P o s_v)  -- channels are the MMA rows, P (fp16, moved
+//       into the B layout with movmatrix) is scaled per group by the token's V
+//       scale; the zero-point term sum_t p_t z_t,g is one more MMA.
+//
+// Online softmax per head with lazy rescaling (the running max only moves when
+// a tile exceeds it by more than 2^8), a CTA-level merge of the warps, then the
+// last CTA of each (b, kv head) merges all splits (an atomic ticket, no spin
+// waits) and writes the fp32 output and log-sum-exp.
+#include <cuda.h>
+#include <float.h>
+
+#include "hq_internal.cuh"
+#include "tma.cuh"
+#include "warp_mma.cuh"
+
+namespace hq {
+namespace {
+
+constexpr int D = 128;
+constexpr int NCW = 4;                      // consumer warps
+constexpr int NTHREADS = (NCW + 1) * 32;    // + one producer warp
+constexpr int T_LO = 64, T_HI = 64;         // tokens per stage; 16 per consumer warp
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLazy = 8.0f;               // rescale only when the max grows by > 2^8
+
+// Every consumer warp takes one 16-token sub-tile of EVERY stage, so each warp
+// waits on every phase of every barrier in order (a warp that skipped stages
+// could wait on a phase two ahead, which the parity scheme cannot tell apart).
+// A low-bit CTA runs NSTAGE stages of STAGE bytes; a bf16 CTA runs NSTAGE/2
+// stages of 2*STAGE bytes (its 64-token tiles are larger).
+template <int BITS>
+struct Cfg {
+  static constexpr int ROWB = D * BITS / 8;               // packed bytes per low row
+  static constexpr int KC = T_LO * ROWB;                  // codes per stage (K or V)
+  static constexpr int SZ = T_LO * 16;                    // (scale, zero) x 4 groups per token
+  static constexpr int LO_BYTES = 2 * KC + 2 * SZ;
+  static constexpr int HI_BOX = T_HI * 128;               // 64 channels x 64 tokens, bf16
+  static constexpr int HI_BYTES = 4 * HI_BOX;
+  static constexpr int STAGE = LO_BYTES > HI_BYTES / 2 ? LO_BYTES : HI_BYTES / 2;
+  static constexpr int NSTAGE = 4;
+  static constexpr int SMEM = NSTAGE * STAGE + 1024 + 512;  // + alignment slack + barriers
+};
+
+struct DecArgs {
+  const __nv_bfloat16 *q;
+  float *part_o;          // [B*Hq, nsplit, D]  unnormalized partial outputs
+  float2 *part_ml;        // [B*Hq, nsplit]     (max in log2 units, sum)
+  unsigned *counters;     // [B*Hkv] arrival tickets, left at zero
+  float *out, *lse;
+  uint32_t *status;
+  int Hq, Hkv, n_lo, n_hi, nsplit_lo, nsplit_hi;
+  float sl;               // softmax scale * log2(e)
+};
+
+__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;\n" : "=r"(d) : "r"(a), "r"(b), "r"(c));  // (a & b) | c
+  return d;
+}
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;\n" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+__device__ __forceinline__ uint32_t hsub2_u(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("sub.rn.f16x2 %0, %1, %2;\n" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t hfma2_u(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;\n" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ uint32_t hmul2_u(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.f16x2 %0, %1, %2;\n" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
+  return pack_f16x2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+__device__ __forceinline__ float half_lo_f(uint32_t w) {
+  return __half2float(__ushort_as_half((unsigned short)(w & 0xffffu)));
+}
+
+constexpr uint32_t F16_1024x2 = 0x64006400u;   // (1024, 1024)
+constexpr uint32_t F16_1_16x2 = 0x2C002C00u;   // (1/16, 1/16)
+constexpr uint32_t F16_M64x2 = 0xD400D400u;    // (-64, -64)
+
+// Swizzled byte offset of 16-byte chunk `ch` of row `row` in a TMA box whose
+// rows are RB bytes (64B or 128B swizzle mode).
+template <int RB>
+__device__ __forceinline__ uint32_t swz_off(int row, int ch) {
+  if (RB == 64) return row * 64 + ((ch ^ ((row >> 1) & 3)) << 4);
+  return row * 128 + ((ch ^ (row & 7)) << 4);
+}
+
+template <int BITS, int G>
+__global__ void __launch_bounds__(NTHREADS, 3)
+decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_vc,
+           const __grid_constant__ CUtensorMap tm_ksz, const __grid_constant__ CUtensorMap tm_vsz,
+           const __grid_constant__ CUtensorMap tm_khi, const __grid_constant__ CUtensorMap tm_vhi,
+           DecArgs a) {
+  using C = Cfg<BITS>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::NSTAGE * C::STAGE);
+  uint64_t *empty = full + C::NSTAGE;
+  float *qsum = reinterpret_cast<float *>(empty + C::NSTAGE);   // [8 heads][4 groups]
+  float *qbias = qsum + 32;                                      // [8 heads][4 groups]
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(qbias + 32);
+  int *last_flag = reinterpret_cast<int *>(qbias + 33);
+
+  const int split = blockIdx.x, bh = blockIdx.y;
+  const int b = bh / a.Hkv, kh = bh % a.Hkv;
+  const int nsplit = a.nsplit_lo + a.nsplit_hi;
+  const bool hi = split >= a.nsplit_lo;
+  const int sidx = hi ? split - a.nsplit_lo : split;
+  const int ns = hi ? a.nsplit_hi : a.nsplit_lo;
+  const int T = hi ? T_HI : T_LO;
+  const int nst = hi ? C::NSTAGE / 2 : C::NSTAGE;              // stages of this CTA
+  const int stage_bytes = hi ? 2 * C::STAGE : C::STAGE;
+  const int n_tok = hi ? a.n_hi : a.n_lo;
+  const int ntile = (n_tok + T - 1) / T;
+  const int tile0 = (int)((long long)ntile * sidx / ns);
+  const int tile1 = (int)((long long)ntile * (sidx + 1) / ns);
+  const int my_tiles = tile1 - tile0;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = lane >> 2, c = lane & 3;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::NSTAGE; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], NCW);
+    }
+    fence_mbar_init();
+    *abort_flag = 0;
+    *last_flag = 0;
+  }
+  // Per-head q statistics: group sums (for the zero-point term) and the
+  // constant the 1024-offset code encoding adds to each group accumulator.
+  // Thread t < 128: head t/16, group (t/4)%4, eight channels 8*(t%4)...
+  if (threadIdx.x < 128) {
+    const int h = threadIdx.x >> 4, g = (threadIdx.x >> 2) & 3, part = threadIdx.x & 3;
+    float s = 0.f, bias = 0.f;
+    if (h < G) {
+      const uint4 w = *reinterpret_cast<const uint4 *>(a.q + ((size_t)b * a.Hq + kh * G + h) * D +
+                                                      32 * g + 8 * part);
+      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float x = (i & 1) ? bf16_hi(ww[i >> 1]) : bf16_lo(ww[i >> 1]);
+        s += x;
+        const float x16 = __half2float(__float2half_rn(x));
+        if (BITS == 8 || (i & 1) == 0) bias += 1024.f * x16;
+        else bias += 1024.f * __half2float(__float2half_rn(x16 * 0.0625f));
+      }
+    }
+    s += __shfl_xor_sync(0xffffffffu, s, 1);
+    s += __shfl_xor_sync(0xffffffffu, s, 2);
+    bias += __shfl_xor_sync(0xffffffffu, bias, 1);
+    bias += __shfl_xor_sync(0xffffffffu, bias, 2);
+    if (part == 0) {
+      qsum[h * 4 + g] = s;
+      qbias[h * 4 + g] = bias;
+    }
+  }
+  __syncthreads();
+
+  if (warp == NCW) {
+    // ------------------------------ producer ------------------------------
+    if (lane == 0 && my_tiles > 0) {
+      if (hi) {
+        tma_prefetch_desc(&tm_khi);
+        tma_prefetch_desc(&tm_vhi);
+      } else {
+        tma_prefetch_desc(&tm_kc);
+        tma_prefetch_desc(&tm_vc);
+        tma_prefetch_desc(&tm_ksz);
+        tma_prefetch_desc(&tm_vsz);
+      }
+      int issued = 0;
+      for (int it = 0; it < my_tiles; ++it) {
+        const int s = it % nst;
+        if (it >= nst && !mbar_wait(&empty[s], ((it / nst) & 1) ^ 1)) {
+          *abort_flag = 1;
+          raise_status(a.status, HQ_DEV_TIMEOUT);
+          break;
+        }
+        if (*abort_flag) break;
+        uint8_t *st = smem + s * stage_bytes;
+        const int tok = (tile0 + it) * T;
+        if (!hi) {
+          mbar_arrive_expect_tx(&full[s], C::LO_BYTES);
+          tma_load_3d(st, &tm_kc, &full[s], 0, tok, bh);
+          tma_load_3d(st + C::KC, &tm_vc, &full[s], 0, tok, bh);
+          tma_load_3d(st + 2 * C::KC, &tm_ksz, &full[s], 0, tok, bh);
+          tma_load_3d(st + 2 * C::KC + C::SZ, &tm_vsz, &full[s], 0, tok, bh);
+        } else {
+          mbar_arrive_expect_tx(&full[s], C::HI_BYTES);
+          tma_load_3d(st, &tm_khi, &full[s], 0, tok, bh);
+          tma_load_3d(st + C::HI_BOX, &tm_khi, &full[s], 64, tok, bh);
+          tma_load_3d(st + 2 * C::HI_BOX, &tm_vhi, &full[s], 0, tok, bh);
+          tma_load_3d(st + 3 * C::HI_BOX, &tm_vhi, &full[s], 64, tok, bh);
+        }
+        issued = it + 1;
+      }
+      // Never leave the CTA with copies in flight.
+      for (int it = issued > nst ? issued - nst : 0; it < issued; ++it)
+        if (!mbar_wait(&full[it % nst], (it / nst) & 1)) raise_status(a.status, HQ_DEV_TIMEOUT);
+    }
+  }
+
+  // ------------------------------ consumers -------------------------------
+  // Softmax state for heads 2c, 2c+1 (log2 units), partial sums, outputs.
+  float m0 = -1e30f, m1 = -1e30f, l0 = 0.f, l1 = 0.f;
+  float o[8][4];
+  float oz[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+
+  if (warp < NCW) {
+    // B fragments of q: 8 k16-chunks x 2 registers.
+    uint32_t qb[8][2];
+    const __nv_bfloat16 *qh = a.q + ((size_t)b * a.Hq + kh * G + (r < G ? r : 0)) * D;
+    const bool hv = r < G;
+    if (hi) {
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        qb[kk][0] = hv ? *reinterpret_cast<const uint32_t *>(qh + 16 * kk + 2 * c) : 0u;
+        qb[kk][1] = hv ? *reinterpret_cast<const uint32_t *>(qh + 16 * kk + 8 + 2 * c) : 0u;
+      }
+    } else if (BITS == 4) {
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        float x[8];
+        const uint4 w = hv ? *reinterpret_cast<const uint4 *>(qh + 32 * g + 8 * c) : make_uint4(0, 0, 0, 0);
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          x[2 * i] = bf16_lo(ww[i]);
+          x[2 * i + 1] = bf16_hi(ww[i]);
+        }
+        // chunk 2g+0: slots (2c,2c+1) <- ch 0,4; (2c+8,2c+9) <- ch 1/16, 5/16
+        // chunk 2g+1: slots (2c,2c+1) <- ch 2,6; (2c+8,2c+9) <- ch 3/16, 7/16
+        auto f16 = [](float v) { return __half2float(__float2half_rn(v)); };
+        qb[2 * g][0] = pack_f16x2(x[0], x[4]);
+        qb[2 * g][1] = pack_f16x2(f16(x[1]) * 0.0625f, f16(x[5]) * 0.0625f);
+        qb[2 * g + 1][0] = pack_f16x2(x[2], x[6]);
+        qb[2 * g + 1][1] = pack_f16x2(f16(x[3]) * 0.0625f, f16(x[7]) * 0.0625f);
+      }
+    } else {
+#pragma unroll
+      for (int kc = 0; kc < 8; ++kc) {
+        const uint2 w = hv ? *reinterpret_cast<const uint2 *>(qh + 16 * kc + 4 * c) : make_uint2(0, 0);
+        qb[kc][0] = pack_f16x2(bf16_lo(w.x), bf16_hi(w.x));
+        qb[kc][1] = pack_f16x2(bf16_lo(w.y), bf16_hi(w.y));
+      }
+    }
+    // Z-term B operand (k = 2*group + {hi, lo} half of Q_group, n = head r).
+    uint32_t zb0 = 0u;
+    if (!hi && hv) {
+      const float Q = qsum[r * 4 + c];
+      const __half qh16 = __float2half_rn(Q);
+      const __half ql16 = __float2half_rn(Q - __half2float(qh16));
+      zb0 = (uint32_t)__half_as_ushort(qh16) | ((uint32_t)__half_as_ushort(ql16) << 16);
+    }
+    float nb[4][2];  // -bias of each group for heads 2c, 2c+1 (accumulator start)
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      nb[g][0] = (2 * c < G) ? -qbias[(2 * c) * 4 + g] : 0.f;
+      nb[g][1] = (2 * c + 1 < G) ? -qbias[(2 * c + 1) * 4 + g] : 0.f;
+    }
+
+    const int j = warp;  // this warp's 16-token sub-tile of every stage
+    for (int it = 0; it < my_tiles; ++it) {
+      const int s = it % nst;
+      if (!mbar_wait(&full[s], (it / nst) & 1)) {
+        *abort_flag = 1;
+        raise_status(a.status, HQ_DEV_TIMEOUT);
+        break;
+      }
+      uint8_t *const stp = smem + s * stage_bytes;
+      const uint32_t st = smem_u32(stp);
+      const int tok0 = (tile0 + it) * T + j * 16;
+      const int row0 = j * 16;
+      const bool ok_r = tok0 + r < n_tok, ok_r8 = tok0 + r + 8 < n_tok;
+      float x[4];
+      // ---------------- scores S^T (16 tokens x 8 heads) ----------------
+      if (!hi) {
+        float acc[4][4];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          acc[g][0] = nb[g][0];
+          acc[g][1] = nb[g][1];
+          acc[g][2] = nb[g][0];
+          acc[g][3] = nb[g][1];
+        }
+        const int mi = lane >> 3;
+        const int lrow = row0 + (mi & 1) * 8 + (lane & 7);
+        if (BITS == 4) {
+#pragma unroll
+          for (int gp = 0; gp < 2; ++gp) {
+            uint32_t kx[4];
+            ldsm_x4(kx, st + swz_off<C::ROWB>(lrow, 2 * gp + (mi >> 1)));
+#pragma unroll
+            for (int gg = 0; gg < 2; ++gg) {
+              const int g = 2 * gp + gg;
+              const uint32_t A0 = kx[2 * gg], A1 = kx[2 * gg + 1];
+              const uint32_t A08 = A0 >> 8, A18 = A1 >> 8;
+              uint32_t fa[4], fb[4];
+              fa[0] = lop3_and_or(A0, 0x000F000Fu, F16_1024x2);
+              fa[1] = lop3_and_or(A1, 0x000F000Fu, F16_1024x2);
+              fa[2] = lop3_and_or(A0, 0x00F000F0u, F16_1024x2);
+              fa[3] = lop3_and_or(A1, 0x00F000F0u, F16_1024x2);
+              fb[0] = lop3_and_or(A08, 0x000F000Fu, F16_1024x2);
+              fb[1] = lop3_and_or(A18, 0x000F000Fu, F16_1024x2);
+              fb[2] = lop3_and_or(A08, 0x00F000F0u, F16_1024x2);
+              fb[3] = lop3_and_or(A18, 0x00F000F0u, F16_1024x2);
+              mma_f16_16816(acc[g], fa, qb[2 * g][0], qb[2 * g][1]);
+              mma_f16_16816(acc[g], fb, qb[2 * g + 1][0], qb[2 * g + 1][1]);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int cp = 0; cp < 4; ++cp) {
+            uint32_t kx[4];
+            ldsm_x4(kx, st + swz_off<C::ROWB>(lrow, 2 * cp + (mi >> 1)));
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+              const int kc = 2 * cp + cc;
+              const uint32_t A0 = kx[2 * cc], A1 = kx[2 * cc + 1];
+              uint32_t fa[4];
+              // bytes of F16_1024x2 as prmt source 4..7: 0x00, 0x64, 0x00, 0x64
+              fa[0] = prmt(A0, F16_1024x2, 0x5150);
+              fa[1] = prmt(A1, F16_1024x2, 0x5150);
+              fa[2] = prmt(A0, F16_1024x2, 0x5352);
+              fa[3] = prmt(A1, F16_1024x2, 0x5352);
+              mma_f16_16816(acc[kc >> 1], fa, qb[kc][0], qb[kc][1]);
+            }
+          }
+        }
+        // zero-point term and per-group scales of the two tokens
+        const uint4 s_r = *reinterpret_cast<const uint4 *>(stp + 2 * C::KC + (row0 + r) * 16);
+        const uint4 s_r8 = *reinterpret_cast<const uint4 *>(stp + 2 * C::KC + (row0 + r + 8) * 16);
+        const uint32_t wr[4] = {s_r.x, s_r.y, s_r.z, s_r.w};
+        const uint32_t wr8[4] = {s_r8.x, s_r8.y, s_r8.z, s_r8.w};
+        uint32_t za[4];
+        za[0] = prmt(wr[c], wr[c], 0x3232);
+        za[1] = prmt(wr8[c], wr8[c], 0x3232);
+        za[2] = 0u;
+        za[3] = 0u;
+        float zacc[4] = {0.f, 0.f, 0.f, 0.f};
+        mma_f16_16816(zacc, za, zb0, 0u);
+        x[0] = zacc[0];
+        x[1] = zacc[1];
+        x[2] = zacc[2];
+        x[3] = zacc[3];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const float sa = half_lo_f(wr[g]), sb = half_lo_f(wr8[g]);
+          x[0] = fmaf(sa, acc[g][0], x[0]);
+          x[1] = fmaf(sa, acc[g][1], x[1]);
+          x[2] = fmaf(sb, acc[g][2], x[2]);
+          x[3] = fmaf(sb, acc[g][3], x[3]);
+        }
+      } else {
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        const int mi = lane >> 3;
+        const int lrow = row0 + (mi & 1) * 8 + (lane & 7);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          uint32_t ka[4];
+          const uint32_t box = st + (kk >> 2) * C::HI_BOX;
+          ldsm_x4(ka, box + swz_off<128>(lrow, 2 * (kk & 3) + (mi >> 1)));
+          mma_bf16_16816(acc, ka, qb[kk][0], qb[kk][1]);
+        }
+        x[0] = acc[0];
+        x[1] = acc[1];
+        x[2] = acc[2];
+        x[3] = acc[3];
+      }
+      if (!ok_r) x[0] = x[1] = -INFINITY;
+      if (!ok_r8) x[2] = x[3] = -INFINITY;
+
+      // ---------------- online softmax (lazy rescale) ----------------
+      float t0 = fmaxf(x[0], x[2]) * a.sl, t1 = fmaxf(x[1], x[3]) * a.sl;
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        t0 = fmaxf(t0, __shfl_xor_sync(0xffffffffu, t0, off));
+        t1 = fmaxf(t1, __shfl_xor_sync(0xffffffffu, t1, off));
+      }
+      const bool need = (t0 > m0 + kLazy) || (t1 > m1 + kLazy);
+      if (__any_sync(0xffffffffu, need)) {
+        const float n0 = fmaxf(m0, t0), n1 = fmaxf(m1, t1);
+        const float al0 = exp2f(m0 - n0), al1 = exp2f(m1 - n1);
+        m0 = n0;
+        m1 = n1;
+        l0 *= al0;
+        l1 *= al1;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          o[i][0] *= al0;
+          o[i][1] *= al1;
+          o[i][2] *= al0;
+          o[i][3] *= al1;
+        }
+        oz[0] *= al0;
+        oz[1] *= al1;
+        oz[2] *= al0;
+        oz[3] *= al1;
+      }
+      const float p0 = fast_exp2(fmaf(x[0], a.sl, -m0)), p1 = fast_exp2(fmaf(x[1], a.sl, -m1));
+      const float p2 = fast_exp2(fmaf(x[2], a.sl, -m0)), p3 = fast_exp2(fmaf(x[3], a.sl, -m1));
+      l0 += p0 + p2;
+      l1 += p1 + p3;
+      const uint32_t pb0 = movmatrix_t(pack_f16x2(p0, p1));   // (head r; tokens 2c, 2c+1)
+      const uint32_t pb1 = movmatrix_t(pack_f16x2(p2, p3));   // (head r; tokens 2c+8, 2c+9)
+
+      // ---------------- O^T += V^T P ----------------
+      if (!hi) {
+        const uint8_t *vszp = stp + 2 * C::KC + C::SZ;
+        const int ta = row0 + 2 * c;
+        const uint4 wa = *reinterpret_cast<const uint4 *>(vszp + ta * 16);
+        const uint4 wb = *reinterpret_cast<const uint4 *>(vszp + (ta + 1) * 16);
+        const uint4 wc = *reinterpret_cast<const uint4 *>(vszp + (ta + 8) * 16);
+        const uint4 wd = *reinterpret_cast<const uint4 *>(vszp + (ta + 9) * 16);
+        const uint32_t A_[4] = {wa.x, wa.y, wa.z, wa.w}, B_[4] = {wb.x, wb.y, wb.z, wb.w};
+        const uint32_t C_[4] = {wc.x, wc.y, wc.z, wc.w}, D_[4] = {wd.x, wd.y, wd.z, wd.w};
+        // zero-point term: rows = group (r & 3), k = tokens
+        {
+          const int gz = r & 3;
+          const uint32_t za0 = *reinterpret_cast<const uint32_t *>(vszp + ta * 16 + gz * 4);
+          const uint32_t zb_ = *reinterpret_cast<const uint32_t *>(vszp + (ta + 1) * 16 + gz * 4);
+          const uint32_t zc = *reinterpret_cast<const uint32_t *>(vszp + (ta + 8) * 16 + gz * 4);
+          const uint32_t zd = *reinterpret_cast<const uint32_t *>(vszp + (ta + 9) * 16 + gz * 4);
+          uint32_t zaf[4];
+          zaf[0] = prmt(za0, zb_, 0x7632);
+          zaf[1] = 0u;
+          zaf[2] = prmt(zc, zd, 0x7632);
+          zaf[3] = 0u;
+          mma_f16_16816(oz, zaf, pb0, pb1);
+        }
+        const int mi = lane >> 3;
+        const int lrow = row0 + (mi & 1) * 8 + (lane & 7);
+        const uint32_t vbase = st + C::KC;
+        if (BITS == 4) {
+#pragma unroll
+          for (int gp = 0; gp < 2; ++gp) {
+            uint32_t vx[4];
+            ldsm_x4_t(vx, vbase + swz_off<C::ROWB>(lrow, 2 * gp + (mi >> 1)));
+#pragma unroll
+            for (int gg = 0; gg < 2; ++gg) {
+              const int g = 2 * gp + gg;
+              const uint32_t bs0 = hmul2_u(pb0, prmt(A_[g], B_[g], 0x5410));
+              const uint32_t bs1 = hmul2_u(pb1, prmt(C_[g], D_[g], 0x5410));
+              const uint32_t X = vx[2 * gg], Xp = vx[2 * gg + 1];
+              const uint32_t X8 = X >> 8, Xp8 = Xp >> 8;
+              uint32_t fa[4], fb[4];
+              fa[0] = hsub2_u(lop3_and_or(X, 0x000F000Fu, F16_1024x2), F16_1024x2);
+              fa[1] = hfma2_u(lop3_and_or(X, 0x00F000F0u, F16_1024x2), F16_1_16x2, F16_M64x2);
+              fa[2] = hsub2_u(lop3_and_or(Xp, 0x000F000Fu, F16_1024x2), F16_1024x2);
+              fa[3] = hfma2_u(lop3_and_or(Xp, 0x00F000F0u, F16_1024x2), F16_1_16x2, F16_M64x2);
+              fb[0] = hsub2_u(lop3_and_or(X8, 0x000F000Fu, F16_1024x2), F16_1024x2);
+              fb[1] = hfma2_u(lop3_and_or(X8, 0x00F000F0u, F16_1024x2), F16_1_16x2, F16_M64x2);
+              fb[2] = hsub2_u(lop3_and_or(Xp8, 0x000F000Fu, F16_1024x2), F16_1024x2);
+              fb[3] = hfma2_u(lop3_and_or(Xp8, 0x00F000F0u, F16_1024x2), F16_1_16x2, F16_M64x2);
+              mma_f16_16816(o[2 * g], fa, bs0, bs1);
+              mma_f16_16816(o[2 * g + 1], fb, bs0, bs1);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int cp = 0; cp < 4; ++cp) {
+            uint32_t vx[4];
+            ldsm_x4_t(vx, vbase + swz_off<C::ROWB>(lrow, 2 * cp + (mi >> 1)));
+            const int g = cp;  // chunks 2cp, 2cp+1 form group cp
+            const uint32_t bs0 = hmul2_u(pb0, prmt(A_[g], B_[g], 0x5410));
+            const uint32_t bs1 = hmul2_u(pb1, prmt(C_[g], D_[g], 0x5410));
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+              const uint32_t X = vx[2 * cc], Xp = vx[2 * cc + 1];
+              uint32_t fa[4];
+              fa[0] = hsub2_u(prmt(X, F16_1024x2, 0x5250), F16_1024x2);
+              fa[1] = hsub2_u(prmt(X, F16_1024x2, 0x5351), F16_1024x2);
+              fa[2] = hsub2_u(prmt(Xp, F16_1024x2, 0x5250), F16_1024x2);
+              fa[3] = hsub2_u(prmt(Xp, F16_1024x2, 0x5351), F16_1024x2);
+              mma_f16_16816(o[2 * cp + cc], fa, bs0, bs1);
+            }
+          }
+        }
+      } else {
+        const int mi = lane >> 3;
+        const int lrow = row0 + (mi >> 1) * 8 + (lane & 7);
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          uint32_t va[4];
+          const uint32_t box = st + 2 * C::HI_BOX + (mt >> 2) * C::HI_BOX;
+          ldsm_x4_t(va, box + swz_off<128>(lrow, 2 * (mt & 3) + (mi & 1)));
+          uint32_t fa[4];
+          fa[0] = bf16x2_to_f16x2(va[0]);
+          fa[1] = bf16x2_to_f16x2(va[1]);
+          fa[2] = bf16x2_to_f16x2(va[2]);
+          fa[3] = bf16x2_to_f16x2(va[3]);
+          mma_f16_16816(o[mt], fa, pb0, pb1);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+    }
+  }
+
+  // ---------------- merge the consumer warps ----------------
+  __syncthreads();  // all copies have landed and every stage is consumed
+  float *wml = reinterpret_cast<float *>(smem);             // [NCW][8][2]
+  float *wz = wml + NCW * 16;                               // [NCW][8 heads][4 groups]
+  float *wo = wz + NCW * 32;                                // [NCW][8 heads][D]
+  if (warp < NCW) {
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+    }
+    if (r == 0) {
+      wml[(warp * 8 + 2 * c) * 2 + 0] = m0;
+      wml[(warp * 8 + 2 * c) * 2 + 1] = l0;
+      wml[(warp * 8 + 2 * c + 1) * 2 + 0] = m1;
+      wml[(warp * 8 + 2 * c + 1) * 2 + 1] = l1;
+    }
+    if (!hi && r < 4) {
+      wz[(warp * 8 + 2 * c) * 4 + r] = oz[0];
+      wz[(warp * 8 + 2 * c + 1) * 4 + r] = oz[1];
+    }
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const int row = r + 8 * hf;
+        int ch;
+        if (hi) ch = 16 * mt + row;
+        else if (BITS == 4) ch = 32 * (mt >> 1) + 4 * r + 2 * (mt & 1) + hf;
+        else ch = 16 * mt + 2 * r + hf;
+        wo[(warp * 8 + 2 * c) * D + ch] = o[mt][2 * hf];
+        wo[(warp * 8 + 2 * c + 1) * D + ch] = o[mt][2 * hf + 1];
+      }
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < G * D; e += NTHREADS) {
+    const int h = e / D, d = e % D;
+    float mm = -1e30f;
+#pragma unroll
+    for (int w = 0; w < NCW; ++w) mm = fmaxf(mm, wml[(w * 8 + h) * 2]);
+    float ll = 0.f, oo = 0.f;
+#pragma unroll
+    for (int w = 0; w < NCW; ++w) {
+      const float f = exp2f(wml[(w * 8 + h) * 2] - mm);
+      ll += f * wml[(w * 8 + h) * 2 + 1];
+      float ov = wo[(w * 8 + h) * D + d];
+      if (!hi) ov += wz[(w * 8 + h) * 4 + d / 32];
+      oo += f * ov;
+    }
+    const size_t hq = (size_t)b * a.Hq + kh * G + h;
+    a.part_o[(hq * nsplit + split) * D + d] = oo;
+    if (d == 0) a.part_ml[hq * nsplit + split] = make_float2(mm, ll);
+  }
+
+  // ---------------- last CTA of this (b, kv head) merges the splits ----------------
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const unsigned ticket = atomicAdd(&a.counters[bh], 1u);
+    *last_flag = (ticket == (unsigned)(nsplit - 1));
+  }
+  __syncthreads();
+  if (!*last_flag) return;
+  __threadfence();
+  // Merge all splits of the G heads: (max, sum) of every split into shared
+  // memory; one warp per head reduces them (lanes over splits); then every
+  // thread accumulates float4 output columns over a quarter of the splits with
+  // eight independent loads in flight, and the quarters are summed in smem.
+  float *cm = reinterpret_cast<float *>(smem);          // [G][nsplit] split maxima -> weights
+  float *cl = cm + G * nsplit;                           // [G][nsplit] split sums
+  float *cstar = cl + G * nsplit;                        // [G] 1 / total sum
+  float4 *cacc = reinterpret_cast<float4 *>((reinterpret_cast<uintptr_t>(cstar + 8) + 15) & ~uintptr_t(15));  // [4][G * D/4]
+  const size_t hq0 = (size_t)b * a.Hq + kh * G;
+  for (int e = threadIdx.x; e < G * nsplit; e += NTHREADS) {
+    const float2 ml = __ldcg(&a.part_ml[hq0 * nsplit + e]);
+    cm[e] = ml.x;
+    cl[e] = ml.y;
+  }
+  __syncthreads();
+  for (int h = warp; h < G; h += NTHREADS / 32) {
+    float mm = -1e30f;
+    for (int sp = lane; sp < nsplit; sp += 32) mm = fmaxf(mm, cm[h * nsplit + sp]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mm = fmaxf(mm, __shfl_xor_sync(0xffffffffu, mm, off));
+    float ll = 0.f;
+    for (int sp = lane; sp < nsplit; sp += 32) {
+      const float f = exp2f(cm[h * nsplit + sp] - mm);
+      cm[h * nsplit + sp] = f;
+      ll += f * cl[h * nsplit + sp];
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ll += __shfl_xor_sync(0xffffffffu, ll, off);
+    if (lane == 0) {
+      cstar[h] = 1.f / ll;
+      if (a.lse) a.lse[hq0 + h] = (mm + log2f(ll)) * 0.6931471805599453f;
+    }
+  }
+  __syncthreads();
+  constexpr int NCOL = D / 4;
+  for (int e = threadIdx.x; e < 4 * G * NCOL; e += NTHREADS) {
+    const int quarter = e / (G * NCOL), item = e % (G * NCOL);
+    const int h = item / NCOL, d4 = item % NCOL;
+    const float4 *po = reinterpret_cast<const float4 *>(a.part_o + (hq0 + h) * nsplit * D) + d4;
+    const float *f = cm + h * nsplit;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int sp0 = quarter; sp0 < nsplit; sp0 += 32) {
+      float4 x[8];
+      float fw[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int sp = sp0 + 4 * u;
+        x[u] = sp < nsplit ? __ldcg(po + (size_t)sp * NCOL) : make_float4(0.f, 0.f, 0.f, 0.f);
+        fw[u] = sp < nsplit ? f[sp] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        acc.x = fmaf(fw[u], x[u].x, acc.x);
+        acc.y = fmaf(fw[u], x[u].y, acc.y);
+        acc.z = fmaf(fw[u], x[u].z, acc.z);
+        acc.w = fmaf(fw[u], x[u].w, acc.w);
+      }
+    }
+    cacc[quarter * G * NCOL + item] = acc;
+  }
+  __syncthreads();
+  for (int item = threadIdx.x; item < G * NCOL; item += NTHREADS) {
+    const int h = item / NCOL, d4 = item % NCOL;
+    float4 s4 = cacc[item];
+#pragma unroll
+    for (int q4 = 1; q4 < 4; ++q4) {
+      const float4 t4 = cacc[q4 * G * NCOL + item];
+      s4.x += t4.x;
+      s4.y += t4.y;
+      s4.z += t4.z;
+      s4.w += t4.w;
+    }
+    const float inv = cstar[h];
+    reinterpret_cast<float4 *>(a.out + (hq0 + h) * D)[d4] =
+        make_float4(s4.x * inv, s4.y * inv, s4.z * inv, s4.w * inv);
+  }
+  if (threadIdx.x == 0) a.counters[bh] = 0u;
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+struct Plan {
+  int nsplit_lo, nsplit_hi;
+};
+
+template <int BITS, int G>
+int occupancy() {
+  static int occ = -1;
+  if (occ < 0) {
+    cudaFuncSetAttribute(decode_tma<BITS, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         Cfg<BITS>::SMEM);
+    int o = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, decode_tma<BITS, G>, NTHREADS,
+                                                      Cfg<BITS>::SMEM) != cudaSuccess || o < 1)
+      o = 1;
+    occ = o;
+  }
+  return occ;
+}
+
+Plan make_plan(int nbh, int n_lo, int n_hi, int bits, int occ) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int slots = sms * occ;
+  int per_bh = slots / nbh;
+  if (per_bh < 1) per_bh = 1;
+  const double lo_b = (double)n_lo * (2 * (D * bits / 8) + 32);
+  const double hi_b = (double)n_hi * 512.0;
+  const int tl = (n_lo + T_LO - 1) / T_LO, th = (n_hi + T_HI - 1) / T_HI;
+  Plan p;
+  if (n_hi == 0) {
+    p.nsplit_lo = per_bh;
+    p.nsplit_hi = 0;
+  } else if (n_lo == 0) {
+    p.nsplit_lo = 0;
+    p.nsplit_hi = per_bh;
+  } else {
+    int nh = (int)(per_bh * hi_b / (lo_b + hi_b) + 0.5);
+    if (nh < 1) nh = 1;
+    if (nh > per_bh - 1) nh = per_bh - 1 > 0 ? per_bh - 1 : 1;
+    p.nsplit_hi = nh;
+    p.nsplit_lo = per_bh - nh > 0 ? per_bh - nh : 1;
+  }
+  if (p.nsplit_lo > tl) p.nsplit_lo = tl;
+  if (p.nsplit_hi > th) p.nsplit_hi = th;
+  return p;
+}
+
+int occupancy_for(int bits, int G) {
+#define HQ_OCC(BITS, GG) if (bits == BITS && G == GG) return occupancy<BITS, GG>();
+  HQ_OCC(4, 1) HQ_OCC(4, 2) HQ_OCC(4, 4) HQ_OCC(4, 8)
+  HQ_OCC(8, 1) HQ_OCC(8, 2) HQ_OCC(8, 4) HQ_OCC(8, 8)
+#undef HQ_OCC
+  return 1;
+}
+
+struct WsLayout {
+  size_t counters, part_ml, part_o, total;
+};
+
+WsLayout ws_layout(int B, int Hq, int Hkv, int nsplit) {
+  WsLayout w;
+  size_t off = kWsHeader;
+  w.counters = off;
+  off = align_up(off + (size_t)B * Hkv * sizeof(unsigned), 256);
+  w.part_ml = off;
+  off = align_up(off + (size_t)B * Hq * nsplit * sizeof(float2), 256);
+  w.part_o = off;
+  off = align_up(off + (size_t)B * Hq * nsplit * D * sizeof(float), 256);
+  w.total = off;
+  return w;
+}
+
+template <int BITS, int G>
+cudaError_t launch_tg(const DecArgs &a0, const hq_kv_cache &c, int nbh, cudaStream_t s) {
+  DecArgs a = a0;
+  CUtensorMap m[6];
+  const int rowb = D * BITS / 8;
+  const CUtensorMapSwizzle sw = rowb == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+  bool ok = true;
+  ok &= make_map_3d(&m[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, c.k_codes, rowb, c.n_lo, nbh, rowb, T_LO, sw);
+  ok &= make_map_3d(&m[1], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, c.v_codes, rowb, c.n_lo, nbh, rowb, T_LO, sw);
+  ok &= make_map_3d(&m[2], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, c.k_sz, 16, c.n_lo, nbh, 16, T_LO, CU_TENSOR_MAP_SWIZZLE_NONE);
+  ok &= make_map_3d(&m[3], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, c.v_sz, 16, c.n_lo, nbh, 16, T_LO, CU_TENSOR_MAP_SWIZZLE_NONE);
+  ok &= make_map_3d(&m[4], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, c.k_hi, D, c.n_hi, nbh, 64, T_HI, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_map_3d(&m[5], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, c.v_hi, D, c.n_hi, nbh, 64, T_HI, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) return cudaErrorInvalidValue;
+  occupancy<BITS, G>();  // sets the dynamic shared memory attribute once
+  dim3 grid(a.nsplit_lo + a.nsplit_hi, nbh);
+  decode_tma<BITS, G><<<grid, NTHREADS, Cfg<BITS>::SMEM, s>>>(m[0], m[1], m[2], m[3], m[4], m[5], a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool decode_tma_supported(int D_, int bits, int G) {
+  return D_ == 128 && (bits == 4 || bits == 8) && (G == 1 || G == 2 || G == 4 || G == 8);
+}
+
+size_t decode_tma_ws_bytes(int B, int Hq, int Hkv, int n_lo, int n_hi, int bits) {
+  const int G = Hq / Hkv;
+  const Plan p = make_plan(B * Hkv, n_lo, n_hi, bits, occupancy_for(bits, G));
+  return ws_layout(B, Hq, Hkv, p.nsplit_lo + p.nsplit_hi).total;
+}
+
+cudaError_t launch_decode_tma(const __nv_bfloat16 *q, const hq_kv_cache &c, int B, int Hq,
+                              int Hkv, float scale, float *out, float *lse, uint8_t *ws,
+                              uint32_t *status, cudaStream_t s) {
+  const int G = Hq / Hkv, nbh = B * Hkv;
+  const Plan p = make_plan(nbh, c.n_lo, c.n_hi, c.bits, occupancy_for(c.bits, G));
+  const WsLayout w = ws_layout(B, Hq, Hkv, p.nsplit_lo + p.nsplit_hi);
+  DecArgs a;
+  a.q = q;
+  a.part_o = reinterpret_cast<float *>(ws + w.part_o);
+  a.part_ml = reinterpret_cast<float2 *>(ws + w.part_ml);
+  a.counters = reinterpret_cast<unsigned *>(ws + w.counters);
+  a.out = out;
+  a.lse = lse;
+  a.status = status;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.n_lo = c.n_lo;
+  a.n_hi = c.n_hi;
+  a.nsplit_lo = p.nsplit_lo;
+  a.nsplit_hi = p.nsplit_hi;
+  a.sl = scale * kLog2e;
+#define HQ_L(BITS, GG) if (c.bits == BITS && G == GG) return launch_tg<BITS, GG>(a, c, nbh, s);
+  HQ_L(4, 1) HQ_L(4, 2) HQ_L(4, 4) HQ_L(4, 8)
+  HQ_L(8, 1) HQ_L(8, 2) HQ_L(8, 4) HQ_L(8, 8)
+#undef HQ_L
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace hq

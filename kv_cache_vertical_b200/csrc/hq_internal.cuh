@@ -36,6 +36,11 @@ cudaError_t launch_probe(const __nv_bfloat16 *q_probe, int64_t q_head_stride,
                          int window, int k_vert, float scale, int32_t *idx_out, float *score_out,
                          uint8_t *ws, cudaStream_t s);
 
+bool decode_tma_supported(int D, int bits, int G);
+size_t decode_tma_ws_bytes(int B, int Hq, int Hkv, int n_lo, int n_hi, int bits);
+cudaError_t launch_decode_tma(const __nv_bfloat16 *q, const hq_kv_cache &c, int B, int Hq,
+                              int Hkv, float scale, float *out, float *lse, uint8_t *ws,
+                              uint32_t *status, cudaStream_t s);
 size_t decode_ws_bytes(int B, int Hq, int Hkv, int D, int n_lo, int n_hi, int bits);
 cudaError_t launch_decode(const __nv_bfloat16 *q, const hq_kv_cache &c, int B, int Hq, int Hkv,
                           int D, float scale, float *out, float *lse, uint8_t *ws,
@@ -44,6 +49,24 @@ cudaError_t launch_decode(const __nv_bfloat16 *q, const hq_kv_cache &c, int B, i
 cudaError_t launch_prefill_quant(const __nv_bfloat16 *q, const __nv_bfloat16 *k, int B, int Hq,
                                  int Hkv, int N, int D, int8_t *qi8, float *sq, int8_t *ki8,
                                  float *sk, cudaStream_t s);
+// tcgen05 prefill (head_dim 128, an even number of query heads per KV head).
+struct TcLaunch {
+  const __nv_bfloat16 *q, *k;        // bf16 [B,Hq,N,D], [B,Hkv,N,D]
+  const int8_t *qi8, *ki8;           // pre-pass codes
+  const float *sq, *sk;              // pre-pass scales (sk per 64 keys)
+  const __half *vh;                  // fp16 V [B,Hkv,N,D]
+  const __nv_bfloat16 *vk;           // compact vertical K [B,Hkv,kpad,D]
+  const __half *vv;                  // compact vertical V
+  const int32_t *vpos, *idx;
+  const unsigned long long *vbits;
+  float *out;
+  uint32_t *status;
+  int B, Hq, Hkv, N, window, k_vert, kpad, nblk64;
+  float scale;
+};
+bool prefill_tc_supported(int D, int Hq, int Hkv);
+cudaError_t launch_prefill_tc(const TcLaunch &p, cudaStream_t s);
+
 size_t prefill_ws_bytes(int B, int Hq, int Hkv, int N, int D, int k_vert);
 cudaError_t launch_prefill(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
                            const __nv_bfloat16 *v, const int32_t *idx, int B, int Hq, int Hkv,

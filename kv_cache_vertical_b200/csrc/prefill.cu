@@ -428,7 +428,7 @@ PrefillWs carve(uint8_t *base, int B, int Hq, int Hkv, int N, int D, int k_vert)
   PrefillWs w;
   const size_t nbh = (size_t)B * Hkv, nbq = (size_t)B * Hq;
   const int nblk = (N + TILE - 1) / TILE;
-  const size_t kpad = (size_t)((k_vert + TILE - 1) / TILE) * TILE;
+  const size_t kpad = (size_t)((k_vert + 127) / 128) * 128;  // whole 128-row tiles
   size_t off = kWsHeader;
   auto take = [&](size_t bytes) {
     uint8_t *p = base ? base + off : nullptr;
@@ -461,11 +461,11 @@ cudaError_t quant_t(const __nv_bfloat16 *q, const __nv_bfloat16 *k, int B, int H
 template <int D>
 cudaError_t prefill_t(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
                       const int32_t *idx, int B, int Hq, int Hkv, int N, int window, int k_vert,
-                      float scale, float *out, uint8_t *ws, cudaStream_t s) {
+                      float scale, float *out, uint8_t *ws, uint32_t *status, cudaStream_t s) {
   PrefillWs w = carve(ws, B, Hq, Hkv, N, D, k_vert);
   const int nbh = B * Hkv;
   const int nblk = (N + TILE - 1) / TILE;
-  const int kpad = (k_vert + TILE - 1) / TILE * TILE;
+  const int kpad = (k_vert + 127) / 128 * 128;
   cudaError_t e = quant_t<D>(q, k, B, Hq, Hkv, N, w.qi8, w.sq, w.ki8, w.sk, s);
   if (e != cudaSuccess) return e;
   const long long n2 = (long long)nbh * N * D / 2;
@@ -474,6 +474,33 @@ cudaError_t prefill_t(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
     gather_vertical<D><<<dim3(kpad, nbh), D / 8, 0, s>>>(k, w.vh, idx, N, k_vert, kpad, w.vk,
                                                          w.vv, w.vpos);
   vertical_bitmap<<<dim3((nblk + 127) / 128, nbh), 128, 0, s>>>(idx, k_vert, nblk, w.vbits);
+  if (prefill_tc_supported(D, Hq, Hkv)) {
+    TcLaunch p;
+    p.q = q;
+    p.k = k;
+    p.qi8 = w.qi8;
+    p.ki8 = w.ki8;
+    p.sq = w.sq;
+    p.sk = w.sk;
+    p.vh = w.vh;
+    p.vk = w.vk;
+    p.vv = w.vv;
+    p.vpos = w.vpos;
+    p.idx = idx;
+    p.vbits = w.vbits;
+    p.out = out;
+    p.status = status;
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.N = N;
+    p.window = window;
+    p.k_vert = k_vert;
+    p.kpad = kpad;
+    p.nblk64 = nblk;
+    p.scale = scale;
+    return launch_prefill_tc(p, s);
+  }
   PrefillArgs a;
   a.q = q;
   a.k = k;
@@ -517,9 +544,8 @@ cudaError_t launch_prefill(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
                            const __nv_bfloat16 *v, const int32_t *idx, int B, int Hq, int Hkv,
                            int N, int D, int window, int k_vert, float scale, float *out,
                            uint8_t *ws, uint32_t *status, cudaStream_t s) {
-  (void)status;
-  if (D == 128) return prefill_t<128>(q, k, v, idx, B, Hq, Hkv, N, window, k_vert, scale, out, ws, s);
-  if (D == 64) return prefill_t<64>(q, k, v, idx, B, Hq, Hkv, N, window, k_vert, scale, out, ws, s);
+  if (D == 128) return prefill_t<128>(q, k, v, idx, B, Hq, Hkv, N, window, k_vert, scale, out, ws, status, s);
+  if (D == 64) return prefill_t<64>(q, k, v, idx, B, Hq, Hkv, N, window, k_vert, scale, out, ws, status, s);
   return cudaErrorInvalidValue;
 }
 

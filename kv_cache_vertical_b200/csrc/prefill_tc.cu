@@ -1,0 +1,434 @@
+// prefill_tc.cu -- hybrid-precision prefill attention on the 5th-generation
+// tensor cores (tcgen05, accumulators in tensor memory), head_dim 128.
+//
+// Method: ACL abstract of HyQuant, Prefill stage -- a hybrid-precision attention
+// operator keeps the vertical-line tokens and a local sliding window at full
+// precision and quantizes the remaining context; "HyQuant: Hybrid-Precision
+// Quantization for LLM Attention" (wiki summary), TL;DR.  Per causal pair
+// (i, j <= i): window (j > i - W) or vertical column -> bf16 logit; otherwise
+// INT8 logit (exact s32 dot product x per-row Q scale x per-64-key K scale);
+// one online softmax; P.V with fp16 P and fp16 V, fp32 accumulation.
+//
+// One CTA per (128-query tile, pair of query heads that share a KV head): the
+// two heads ("A" and "B") see exactly the same key tiles, so every K / V tile
+// loaded once feeds both.  Warp roles:
+//   warp 0      TMA producer: the four Q tiles once, then a 2-stage ring of
+//               (K tile, V tile) pairs;
+//   warp 1      allocates 512 TMEM columns; lane 0 issues every MMA:
+//               S_X = Q_X K^T (kind::i8 into s32, or kind::f16 bf16 into f32)
+//               and O_X += P_X V (kind::f16, P read from tensor memory);
+//   warps 2-5   softmax of head A, warps 6-9 softmax of head B: one thread per
+//               query row (TMEM lane), so row max / sum need no shuffles.
+// TMEM: S_A [0,128) (P_A aliases its first 64 columns as packed fp16 pairs),
+// O_A [128,256), S_B [256,384), O_B [384,512).
+// The MMA thread alternates the heads (PV_A(t), QK_A(t+1), PV_B(t), QK_B(t+1)),
+// so one head's softmax overlaps the other head's tensor-core work.
+// Key tiles per query tile, each its own iteration of the online softmax:
+//   INT8 tiles  kt with kt*128 <= i_max - W: keep j <= i - W, not vertical;
+//   window      bf16 tiles meeting (i - W, i]: keep i - W < j <= i;
+//   vertical    compact bf16 rows (sorted): keep v <= i - W;
+// so every causal pair is counted exactly once.
+#include <cuda.h>
+#include <float.h>
+#include <limits.h>
+
+#include "hq_internal.cuh"
+#include "tcgen05.cuh"
+#include "tma.cuh"
+#include "warp_mma.cuh"
+
+namespace hq {
+namespace {
+
+constexpr int BM = 128, BN = 128, D = 128;
+constexpr int NWARP = 10, NT = NWARP * 32;
+constexpr uint32_t SM_QI8 = 0;                 // [2 heads][128 rows x 128 B]
+constexpr uint32_t SM_QBF = 32768;             // [2 heads][2 boxes][128 rows x 128 B]
+constexpr uint32_t SM_KV = 98304;              // [2 stages][K 32 KB | V 32 KB]
+constexpr uint32_t KV_STAGE = 65536;
+constexpr uint32_t SM_BAR = SM_KV + 2 * KV_STAGE;
+constexpr uint32_t SMEM_BYTES = SM_BAR + 256 + 1024;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLazy = 8.0f;                   // rescale O only when the max grows by > 2^8
+constexpr float kMagic = 12582912.0f;           // 2^23 + 2^22
+constexpr uint32_t kMagicBits = 0x4B400000u;    // bits of kMagic
+
+constexpr uint32_t IDESC_I8 = make_idesc(2, 1, 1, 0, 0, 128, 128);   // s32 <- s8 x s8
+constexpr uint32_t IDESC_BF = make_idesc(1, 1, 1, 0, 0, 128, 128);   // f32 <- bf16 x bf16
+constexpr uint32_t IDESC_PV = make_idesc(1, 0, 0, 0, 1, 128, 128);   // f32 <- f16 x f16 (V MN-major)
+
+enum { IT_I8 = 0, IT_WIN = 1, IT_VERT = 2 };
+
+struct TcArgs {
+  const float *sq;                    // [B*Hq, N]
+  const float *sk;                    // [B*Hkv, nblk64]
+  const unsigned long long *vbits;    // [B*Hkv, nblk64] vertical bitmap per 64 keys
+  const int32_t *vpos;                // [B*Hkv, kpad] compact vertical positions (INT_MAX pad)
+  const int32_t *idx;                 // [B*Hkv, k_vert]
+  float *out;                         // [B*Hq, N, D]
+  uint32_t *status;
+  int Hq, Hkv, N, window, k_vert, kpad, nblk64;
+  float sl;                           // softmax scale * log2(e)
+};
+
+struct Sched {
+  int n_i8, n_w, kw0, n;
+  __device__ __forceinline__ int type(int it) const {
+    return it < n_i8 ? IT_I8 : (it < n_i8 + n_w ? IT_WIN : IT_VERT);
+  }
+  __device__ __forceinline__ int tile(int it) const {
+    return it < n_i8 ? it : (it < n_i8 + n_w ? kw0 + it - n_i8 : it - n_i8 - n_w);
+  }
+};
+
+__device__ __forceinline__ Sched make_sched(const TcArgs &a, int i0, size_t bh) {
+  Sched s;
+  const int i_max = min(i0 + BM - 1, a.N - 1);
+  const int W = a.window;
+  s.n_i8 = (i_max - W >= 0) ? (i_max - W) / BN + 1 : 0;
+  if (W > 0) {
+    s.kw0 = max(0, i0 - W + 1) / BN;
+    s.n_w = i_max / BN - s.kw0 + 1;
+  } else {
+    s.kw0 = 0;
+    s.n_w = 0;
+  }
+  int cnt = 0;
+  if (a.k_vert > 0 && i_max - W >= 0) cnt = upper_bound_i32(a.idx + bh * a.k_vert, a.k_vert, i_max - W);
+  s.n = s.n_i8 + s.n_w + (cnt + BN - 1) / BN;
+  return s;
+}
+
+__global__ void __launch_bounds__(NT, 1)
+prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ CUtensorMap tm_qbf,
+           const __grid_constant__ CUtensorMap tm_ki8, const __grid_constant__ CUtensorMap tm_kbf,
+           const __grid_constant__ CUtensorMap tm_v16, const __grid_constant__ CUtensorMap tm_vk,
+           const __grid_constant__ CUtensorMap tm_vv, TcArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *bar = reinterpret_cast<uint64_t *>(smem + SM_BAR);
+  uint64_t *q_full = bar;
+  uint64_t *kv_full = bar + 1;   // [2]
+  uint64_t *kv_free = bar + 3;   // [2]
+  uint64_t *s_full = bar + 5;    // [2 heads]
+  uint64_t *p_full = bar + 7;    // [2 heads]
+  uint64_t *o_final = bar + 9;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 10);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(bar + 11);
+
+  const int ntq = (a.N + BM - 1) / BM;
+  const int qt = ntq - 1 - (int)blockIdx.x;      // longest rows first
+  const int hp = blockIdx.y, b = blockIdx.z;
+  const int G = a.Hq / a.Hkv;
+  const int hA = 2 * hp;
+  const int kh = hA / G;
+  const size_t bh = (size_t)b * a.Hkv + kh;
+  const int i0 = qt * BM;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const Sched sc = make_sched(a, i0, bh);
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_free[s], 1);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&p_full[s], 128);
+    }
+    mbar_init(o_final, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------ producer ------------------------------
+    if (lane == 0) {
+      const int bqA = b * a.Hq + hA, bqB = bqA + 1;
+      mbar_arrive_expect_tx(q_full, 2 * 16384 + 2 * 32768);
+      tma_load_3d(smem + SM_QI8, &tm_qi8, q_full, 0, i0, bqA);
+      tma_load_3d(smem + SM_QI8 + 16384, &tm_qi8, q_full, 0, i0, bqB);
+      tma_load_3d(smem + SM_QBF, &tm_qbf, q_full, 0, i0, bqA);
+      tma_load_3d(smem + SM_QBF + 16384, &tm_qbf, q_full, 64, i0, bqA);
+      tma_load_3d(smem + SM_QBF + 32768, &tm_qbf, q_full, 0, i0, bqB);
+      tma_load_3d(smem + SM_QBF + 49152, &tm_qbf, q_full, 64, i0, bqB);
+      int issued = 0;
+      for (int it = 0; it < sc.n; ++it) {
+        const int s = it & 1;
+        if (it >= 2 && !mbar_wait(&kv_free[s], ((it >> 1) & 1) ^ 1)) {
+          *abort_flag = 1;
+          raise_status(a.status, HQ_DEV_TIMEOUT);
+          break;
+        }
+        if (*abort_flag) break;
+        uint8_t *ks = smem + SM_KV + s * KV_STAGE;
+        uint8_t *vs = ks + 32768;
+        const int ty = sc.type(it), t = sc.tile(it);
+        const int row = t * BN;
+        if (ty == IT_I8) {
+          mbar_arrive_expect_tx(&kv_full[s], 16384 + 32768);
+          tma_load_3d(ks, &tm_ki8, &kv_full[s], 0, row, (int)bh);
+        } else {
+          mbar_arrive_expect_tx(&kv_full[s], 65536);
+          const CUtensorMap *km = ty == IT_WIN ? &tm_kbf : &tm_vk;
+          tma_load_3d(ks, km, &kv_full[s], 0, row, (int)bh);
+          tma_load_3d(ks + 16384, km, &kv_full[s], 64, row, (int)bh);
+        }
+        const CUtensorMap *vm = ty == IT_VERT ? &tm_vv : &tm_v16;
+        tma_load_3d(vs, vm, &kv_full[s], 0, row, (int)bh);
+        tma_load_3d(vs + 16384, vm, &kv_full[s], 64, row, (int)bh);
+        issued = it + 1;
+      }
+      if (!mbar_wait(q_full, 0)) raise_status(a.status, HQ_DEV_TIMEOUT);
+      for (int it = issued > 2 ? issued - 2 : 0; it < issued; ++it)
+        if (!mbar_wait(&kv_full[it & 1], (it >> 1) & 1)) raise_status(a.status, HQ_DEV_TIMEOUT);
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer ------------------------------
+    if (lane == 0) {
+      const uint32_t sQi8 = smem_u32(smem + SM_QI8), sQbf = smem_u32(smem + SM_QBF);
+      const uint32_t sKV = smem_u32(smem + SM_KV);
+      bool ok = mbar_wait(q_full, 0);
+      auto issue_qk = [&](int x, int it) {
+        const uint32_t kslot = sKV + (it & 1) * KV_STAGE;
+        const uint32_t dt = tmem + x * 256;
+        if (sc.type(it) == IT_I8) {
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t ad = make_sdesc_sw128(sQi8 + x * 16384 + ks * 32, 16, 1024);
+            const uint64_t bd = make_sdesc_sw128(kslot + ks * 32, 16, 1024);
+            mma_i8_ss(dt, ad, bd, IDESC_I8, ks > 0);
+          }
+        } else {
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+            const uint64_t ad = make_sdesc_sw128(sQbf + x * 32768 + off, 16, 1024);
+            const uint64_t bd = make_sdesc_sw128(kslot + off, 16, 1024);
+            mma_f16_ss(dt, ad, bd, IDESC_BF, ks > 0);
+          }
+        }
+        tc_commit(&s_full[x]);
+      };
+      auto issue_pv = [&](int x, int it) {
+        const uint32_t vslot = sKV + (it & 1) * KV_STAGE + 32768;
+        const uint32_t dt = tmem + x * 256 + 128, at = tmem + x * 256;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint64_t bd = make_sdesc_sw128(vslot + ks * 2048, 16384, 1024);
+          mma_f16_ts(dt, at + ks * 8, bd, IDESC_PV, (it > 0 || ks > 0) ? 1u : 0u);
+        }
+      };
+      if (ok && sc.n > 0) {
+        ok = mbar_wait(&kv_full[0], 0);
+        if (ok) {
+          tc_fence_after();
+          issue_qk(0, 0);
+          issue_qk(1, 0);
+        }
+      }
+      for (int it = 0; ok && it < sc.n; ++it) {
+        if (!(ok = mbar_wait(&p_full[0], it & 1))) break;
+        tc_fence_after();
+        issue_pv(0, it);
+        if (it + 1 < sc.n) {
+          if (!(ok = mbar_wait(&kv_full[(it + 1) & 1], ((it + 1) >> 1) & 1))) break;
+          tc_fence_after();
+          issue_qk(0, it + 1);
+        }
+        if (!(ok = mbar_wait(&p_full[1], it & 1))) break;
+        tc_fence_after();
+        issue_pv(1, it);
+        tc_commit(&kv_free[it & 1]);
+        if (it + 1 < sc.n) issue_qk(1, it + 1);
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        raise_status(a.status, HQ_DEV_TIMEOUT);
+      }
+      tc_commit(o_final);
+    }
+  } else {
+    // ------------------------------ softmax ------------------------------
+    const int X = (warp - 2) >> 2;                 // 0: head A, 1: head B
+    const int hq = hA + X;
+    const int quarter = warp & 3;                  // TMEM lanes 32*quarter ..
+    const int r = quarter * 32 + lane;
+    const int i = i0 + r;
+    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t tS = tl + X * 256, tO = tS + 128;
+    const size_t bhq = (size_t)b * a.Hq + hq;
+    const float sqi = (i < a.N) ? a.sq[bhq * a.N + i] * a.sl : 0.f;
+    const int W = a.window;
+    float m = -1e30f, l = 0.f;
+    bool ok = true;
+    for (int it = 0; it < sc.n; ++it) {
+      if (!mbar_wait(&s_full[X], it & 1)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int ty = sc.type(it), t = sc.tile(it);
+      float x[128];
+      float mt = -INFINITY;
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t raw[32];
+        tmem_ld32(tS + ch * 32, raw);
+        const int j0 = t * BN + ch * 32;
+        if (ty == IT_I8) {
+          const int blk = t * 2 + (ch >> 1);
+          const float scl = sqi * a.sk[bh * a.nblk64 + blk];
+          const float off = -kMagic * scl;
+          const uint32_t mw = (uint32_t)(a.vbits[bh * a.nblk64 + blk] >> ((ch & 1) * 32));
+          const int lim = i - W;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            float v = fmaf(__uint_as_float(raw[e] + kMagicBits), scl, off);
+            if (j0 + e > lim || ((mw >> e) & 1u)) v = -INFINITY;
+            x[ch * 32 + e] = v;
+            mt = fmaxf(mt, v);
+          }
+        } else if (ty == IT_WIN) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            float v = __uint_as_float(raw[e]) * a.sl;
+            const int j = j0 + e;
+            if (j > i || j <= i - W) v = -INFINITY;
+            x[ch * 32 + e] = v;
+            mt = fmaxf(mt, v);
+          }
+        } else {
+          const int32_t *vp = a.vpos + bh * a.kpad + j0;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            float v = __uint_as_float(raw[e]) * a.sl;
+            if (__ldg(vp + e) > i - W) v = -INFINITY;
+            x[ch * 32 + e] = v;
+            mt = fmaxf(mt, v);
+          }
+        }
+      }
+      // lazy rescale of the running max (and of O, which the MMA of the
+      // previous iteration has finished: the commit this thread waited on
+      // covers every MMA issued before it)
+      const bool need = mt > m + kLazy;
+      if (__any_sync(0xffffffffu, need)) {
+        const float mn = fmaxf(m, mt);
+        const float al = exp2f(m - mn);
+        m = mn;
+        l *= al;
+        if (it > 0) {
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            uint32_t o[32];
+            tmem_ld32(tO + ch * 32, o);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * al);
+            tmem_st32(tO + ch * 32, o);
+          }
+          tmem_wait_st();
+        }
+      }
+      float rs = 0.f;
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float p0 = fast_exp2(x[h2 * 64 + 2 * e] - m);
+          const float p1 = fast_exp2(x[h2 * 64 + 2 * e + 1] - m);
+          rs += p0 + p1;
+          pk[e] = pack_f16x2(p0, p1);
+        }
+        tmem_st32(tS + h2 * 32, pk);
+      }
+      l += rs;
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&p_full[X]);
+    }
+    if (ok) ok = mbar_wait(o_final, 0);
+    if (!ok) {
+      *abort_flag = 1;
+      raise_status(a.status, HQ_DEV_TIMEOUT);
+    }
+    tc_fence_after();
+    const float inv = (ok && l > 0.f) ? 1.f / l : 0.f;
+#pragma unroll
+    for (int ch = 0; ch < 4; ++ch) {
+      uint32_t o[32];
+      tmem_ld32(tO + ch * 32, o);
+      if (ok && i < a.N) {
+        float4 *dst = reinterpret_cast<float4 *>(a.out + (bhq * a.N + i) * D + ch * 32);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          dst[e] = make_float4(__uint_as_float(o[4 * e]) * inv, __uint_as_float(o[4 * e + 1]) * inv,
+                               __uint_as_float(o[4 * e + 2]) * inv, __uint_as_float(o[4 * e + 3]) * inv);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    // every MMA has completed once o_final fired; wait for it (bounded) in case
+    // a softmax warp gave up before it did
+    if (!mbar_wait(o_final, 0)) raise_status(a.status, HQ_DEV_TIMEOUT);
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+bool prefill_tc_supported(int D_, int Hq, int Hkv) {
+  return D_ == 128 && Hq % Hkv == 0 && (Hq / Hkv) % 2 == 0;
+}
+
+cudaError_t launch_prefill_tc(const TcLaunch &p, cudaStream_t s) {
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(prefill_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
+      return cudaErrorInvalidValue;
+    attr = true;
+  }
+  const int nbq = p.B * p.Hq, nbh = p.B * p.Hkv;
+  CUtensorMap m[7];
+  bool ok = true;
+  ok &= make_map_3d(&m[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (void *)p.qi8, D, p.N, nbq, 128, BM, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_map_3d(&m[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (void *)p.q, D, p.N, nbq, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_map_3d(&m[2], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (void *)p.ki8, D, p.N, nbh, 128, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_map_3d(&m[3], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (void *)p.k, D, p.N, nbh, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_map_3d(&m[4], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (void *)p.vh, D, p.N, nbh, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_map_3d(&m[5], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (void *)p.vk, D, p.kpad, nbh, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_map_3d(&m[6], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (void *)p.vv, D, p.kpad, nbh, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) return cudaErrorInvalidValue;
+  TcArgs a;
+  a.sq = p.sq;
+  a.sk = p.sk;
+  a.vbits = p.vbits;
+  a.vpos = p.vpos;
+  a.idx = p.idx;
+  a.out = p.out;
+  a.status = p.status;
+  a.Hq = p.Hq;
+  a.Hkv = p.Hkv;
+  a.N = p.N;
+  a.window = p.window;
+  a.k_vert = p.k_vert;
+  a.kpad = p.kpad;
+  a.nblk64 = p.nblk64;
+  a.sl = p.scale * kLog2e;
+  dim3 grid((p.N + BM - 1) / BM, p.Hq / 2, p.B);
+  prefill_tc<<<grid, NT, SMEM_BYTES, s>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], a);
+  return cudaGetLastError();
+}
+
+}  // namespace hq

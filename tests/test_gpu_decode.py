@@ -20,13 +20,18 @@ def hq():
     return m
 
 
-def run_decode_case(w: Workload, check_probe=True):
+def run_decode_case(w: Workload, check_probe=True, planted_idx=False):
     H = hq()
     x = make_inputs(w)
     d = to_dev(x)
-    # probe (GPU) vs oracle
-    ref_score = oracle.probe_scores(x["q_probe"], x["k"], w.Hkv)
-    ref_idx = oracle.topk(ref_score, w.window, w.k_vert)
+    # probe (GPU) vs oracle; or, for large pack/decode cases, the seeded
+    # planted positions (sorted, distinct, outside the window) as the list
+    if planted_idx:
+        ref_idx = x["planted"].numpy().astype(np.int32)
+        check_probe = False
+    else:
+        ref_score = oracle.probe_scores(x["q_probe"], x["k"], w.Hkv)
+        ref_idx = oracle.topk(ref_score, w.window, w.k_vert)
     if check_probe:
         gidx, gscore = H.probe_vertical(d["q_probe"], d["k"], w.window, w.k_vert, want_scores=True)
         torch.cuda.synchronize()
@@ -103,6 +108,14 @@ def test_pack_reports_bad_index_lists():
     idx = torch.arange(w.k_vert, dtype=torch.int32, device="cuda").view(1, 1, -1) + 290  # >= L - W
     H.pack_kv(x["k"], x["v"], idx.contiguous(), w.window, 4, ws=ws)
     assert H.hq_read_device_status(ws) & H.HQ_DEV_BAD_INDEX
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_decode_many_tiles_per_cta(bits):
+    # 32 (b, kv head) pairs over the SMs: every CTA streams many tiles through
+    # its shared-memory ring, so every stage and barrier phase is reused
+    w = Workload("multitile", "decode", 4, 32, 8, 128, 20000, 128, F5, bits, 31)
+    run_decode_case(w, planted_idx=True)
 
 
 def test_llama8b_decode_full_size():
