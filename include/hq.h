@@ -56,7 +56,8 @@ typedef enum {
     HQ_ERR_WORKSPACE = 3,     /* workspace missing or smaller than required */
     HQ_ERR_CUDA = 4,          /* a CUDA launch or runtime call failed */
     HQ_ERR_TIMEOUT = 5,       /* a bounded device wait ran out (status word) */
-    HQ_ERR_DEVICE_CHECK = 6   /* a device-side argument check failed (status word) */
+    HQ_ERR_DEVICE_CHECK = 6,  /* a device-side argument check failed (status word) */
+    HQ_ERR_SCRATCH_LIMIT = 7  /* the problem needs more scratch than a fixed-size buffer holds */
 } hq_status;
 
 /* Device status word bits (hq_read_device_status). */
@@ -173,6 +174,31 @@ size_t hq_decode_workspace_size(int B, int Hq, int Hkv, int D, int n_lo, int n_h
 hq_status hq_decode_attn(const void *q, const hq_kv_cache *cache, int B, int Hq, int Hkv, int D,
                          float softmax_scale, float *out, float *lse_out, void *ws,
                          size_t ws_bytes, void *stream);
+
+/*
+ * hq_decode_attn without a caller-supplied workspace, for callers that cannot
+ * allocate device memory at call time: code running under someone else's
+ * stream capture (where a cudaMalloc would break the capture), serving runtimes
+ * whose device memory is fixed at start-up, and hosts that forbid allocation
+ * after initialization.  It computes exactly what hq_decode_attn computes
+ * (same kernels, same results); the pages have no counterpart of this call.
+ * Its scratch is one file-scope device array of HQ_STATIC_SCRATCH_BYTES that
+ * every GPU loading the library holds until the process exits.
+ *   - The first call on a device looks up that array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture begins.
+ *   - Every call shares the one array and leaves its contents behind; each call
+ *     first clears (cudaMemsetAsync on `stream`) the part that must start at
+ *     zero.  Calls whose work overlaps on the GPU (different streams, or graph
+ *     replays that run concurrently) race on the array: serialize them.
+ *   - Problems whose scratch would exceed HQ_STATIC_SCRATCH_BYTES (see
+ *     hq_decode_workspace_size) return HQ_ERR_SCRATCH_LIMIT and launch nothing.
+ *   - No cudaMalloc / cudaFree or allocating library routine is called.
+ */
+#define HQ_STATIC_SCRATCH_BYTES (8u << 20)
+hq_status hq_decode_attn_static(const void *q, const hq_kv_cache *cache, int B, int Hq, int Hkv,
+                                int D, float softmax_scale, float *out, float *lse_out,
+                                void *stream);
 
 /* ------------------------------------------------------------------------ */
 /* Hybrid-precision prefill (abstract: Prefill stage keeps vertical-line     */

@@ -26,6 +26,30 @@ uint32_t *status_word(void *ws) { return ws ? reinterpret_cast<uint32_t *>(ws) :
 
 }  // namespace
 
+namespace hq {
+// Host checks of a decode call without the workspace (used by the scratch-free
+// entry point; no launch happens on failure).
+hq_status check_decode_args(const void *q, const hq_kv_cache *cache, int B, int Hq, int Hkv,
+                            int D, const float *out) {
+  if (!q || !cache || !out) return HQ_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || cache->n_lo < 0 || cache->n_hi < 0 ||
+      cache->n_lo + cache->n_hi <= 0)
+    return HQ_ERR_INVALID_ARG;
+  if ((D != 64 && D != 128) || !supported_G(Hq, Hkv) || (cache->bits != 4 && cache->bits != 8) ||
+      cache->group != 32)
+    return HQ_ERR_UNSUPPORTED;
+  if ((cache->n_lo > 0 && (!cache->k_codes || !cache->v_codes || !cache->k_sz || !cache->v_sz)) ||
+      (cache->n_hi > 0 && (!cache->k_hi || !cache->v_hi)))
+    return HQ_ERR_INVALID_ARG;
+  const void *ptrs[] = {q, cache->k_codes, cache->v_codes, cache->k_sz, cache->v_sz,
+                        cache->k_hi, cache->v_hi, out};
+  for (const void *p : ptrs)
+    if (p && !aligned16(p)) return HQ_ERR_INVALID_ARG;
+  return HQ_OK;
+}
+float resolve_softmax_scale(float s, int D) { return resolve_scale(s, D); }
+}  // namespace hq
+
 extern "C" {
 
 const char *hq_status_string(int status) {
@@ -37,6 +61,7 @@ const char *hq_status_string(int status) {
     case HQ_ERR_CUDA: return "HQ_ERR_CUDA";
     case HQ_ERR_TIMEOUT: return "HQ_ERR_TIMEOUT";
     case HQ_ERR_DEVICE_CHECK: return "HQ_ERR_DEVICE_CHECK";
+    case HQ_ERR_SCRATCH_LIMIT: return "HQ_ERR_SCRATCH_LIMIT";
     default: return "HQ_ERR_UNKNOWN";
   }
 }

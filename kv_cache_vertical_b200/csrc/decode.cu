@@ -208,6 +208,11 @@ size_t decode_ws_bytes(int B, int Hq, int Hkv, int D, int n_lo, int n_hi, int bi
   return off;
 }
 
+size_t decode_ws_zero_bytes(int B, int Hq, int Hkv, int D, int n_lo, int n_hi, int bits) {
+  if (decode_tma_supported(D, bits, Hq / Hkv)) return decode_tma_ws_zero_bytes(B, Hq, Hkv, n_lo, n_hi, bits);
+  return kWsHeader;
+}
+
 cudaError_t launch_decode(const __nv_bfloat16 *q, const hq_kv_cache &c, int B, int Hq, int Hkv,
                           int D, float scale, float *out, float *lse, uint8_t *ws,
                           uint32_t *status, cudaStream_t s) {

@@ -784,6 +784,12 @@ size_t decode_tma_ws_bytes(int B, int Hq, int Hkv, int n_lo, int n_hi, int bits)
   return ws_layout(B, Hq, Hkv, p.nsplit_lo + p.nsplit_hi).total;
 }
 
+size_t decode_tma_ws_zero_bytes(int B, int Hq, int Hkv, int n_lo, int n_hi, int bits) {
+  const int G = Hq / Hkv;
+  const Plan p = make_plan(B * Hkv, n_lo, n_hi, bits, occupancy_for(bits, G));
+  return ws_layout(B, Hq, Hkv, p.nsplit_lo + p.nsplit_hi).part_ml;
+}
+
 cudaError_t launch_decode_tma(const __nv_bfloat16 *q, const hq_kv_cache &c, int B, int Hq,
                               int Hkv, float scale, float *out, float *lse, uint8_t *ws,
                               uint32_t *status, cudaStream_t s) {

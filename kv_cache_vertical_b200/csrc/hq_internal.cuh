@@ -42,6 +42,13 @@ cudaError_t launch_decode_tma(const __nv_bfloat16 *q, const hq_kv_cache &c, int 
                               int Hkv, float scale, float *out, float *lse, uint8_t *ws,
                               uint32_t *status, cudaStream_t s);
 size_t decode_ws_bytes(int B, int Hq, int Hkv, int D, int n_lo, int n_hi, int bits);
+// Leading bytes of the decode workspace that must be zero before a call
+// (status word and split tickets).
+size_t decode_ws_zero_bytes(int B, int Hq, int Hkv, int D, int n_lo, int n_hi, int bits);
+size_t decode_tma_ws_zero_bytes(int B, int Hq, int Hkv, int n_lo, int n_hi, int bits);
+hq_status check_decode_args(const void *q, const hq_kv_cache *cache, int B, int Hq, int Hkv,
+                            int D, const float *out);
+float resolve_softmax_scale(float s, int D);
 cudaError_t launch_decode(const __nv_bfloat16 *q, const hq_kv_cache &c, int B, int Hq, int Hkv,
                           int D, float scale, float *out, float *lse, uint8_t *ws,
                           uint32_t *status, cudaStream_t s);

@@ -1,0 +1,57 @@
+// static_scratch.cu -- hq_decode_attn_static: decode attention whose scratch is
+// a fixed, file-scope device array instead of a caller-allocated workspace.
+//
+// For callers that cannot allocate device memory when they call: code that
+// runs while someone else is capturing the stream into a CUDA graph (a
+// cudaMalloc there would break the capture), serving runtimes that fix their
+// device memory at start-up, and hosts that forbid allocation after
+// initialization.  The kernels and results are those of hq_decode_attn.
+//
+// The array lives in every GPU that loads the library, until the process
+// exits.  In host code its name only stands for it (a host-side shadow): the
+// device address is looked up once per device with cudaGetSymbolAddress, with
+// that device current, on the first call made on it, and cached.  Every call
+// shares the array: it first clears the part that must start at zero (status
+// word and split tickets); calls that overlap on the GPU race on it.
+#include <atomic>
+
+#include "hq_internal.cuh"
+
+namespace {
+
+__device__ __align__(256) uint8_t g_static_scratch[HQ_STATIC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::atomic<void *> g_scratch_addr[kMaxDevices];
+
+// Device address of g_static_scratch on the current device (nullptr on error).
+void *scratch_address() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  void *p = g_scratch_addr[dev].load(std::memory_order_acquire);
+  if (p) return p;
+  if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return nullptr;
+  g_scratch_addr[dev].store(p, std::memory_order_release);
+  return p;
+}
+
+}  // namespace
+
+extern "C" hq_status hq_decode_attn_static(const void *q, const hq_kv_cache *cache, int B,
+                                           int Hq, int Hkv, int D, float softmax_scale,
+                                           float *out, float *lse_out, void *stream) {
+  const hq_status st = hq::check_decode_args(q, cache, B, Hq, Hkv, D, out);
+  if (st != HQ_OK) return st;
+  const size_t need = hq::decode_ws_bytes(B, Hq, Hkv, D, cache->n_lo, cache->n_hi, cache->bits);
+  if (need > HQ_STATIC_SCRATCH_BYTES) return HQ_ERR_SCRATCH_LIMIT;
+  uint8_t *ws = static_cast<uint8_t *>(scratch_address());
+  if (!ws) return HQ_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t zero = hq::decode_ws_zero_bytes(B, Hq, Hkv, D, cache->n_lo, cache->n_hi, cache->bits);
+  if (cudaMemsetAsync(ws, 0, zero, s) != cudaSuccess) return HQ_ERR_CUDA;
+  const cudaError_t e =
+      hq::launch_decode(static_cast<const __nv_bfloat16 *>(q), *cache, B, Hq, Hkv, D,
+                        hq::resolve_softmax_scale(softmax_scale, D), out, lse_out, ws,
+                        reinterpret_cast<uint32_t *>(ws), s);
+  return e == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+}

@@ -60,6 +60,8 @@ _pack = _sig("hq_pack_kv", _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I,
 hq_decode_workspace_size = _sig("hq_decode_workspace_size", _SZ, _I, _I, _I, _I, _I, _I, _I)
 _decode = _sig("hq_decode_attn", _I, _P, ctypes.POINTER(hq_kv_cache), _I, _I, _I, _I, _F, _P, _P,
                _P, _SZ, _P)
+_decode_static = _sig("hq_decode_attn_static", _I, _P, ctypes.POINTER(hq_kv_cache), _I, _I, _I,
+                      _I, _F, _P, _P, _P)
 _pquant = _sig("hq_prefill_quant", _I, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P)
 hq_prefill_workspace_size = _sig("hq_prefill_workspace_size", _SZ, _I, _I, _I, _I, _I, _I)
 _prefill = _sig("hq_prefill_attn", _I, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P,
@@ -67,7 +69,11 @@ _prefill = _sig("hq_prefill_attn", _I, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _
 
 EXPORTED = ["hq_status_string", "hq_version", "hq_read_device_status", "hq_probe_workspace_size",
             "hq_probe_vertical", "hq_pack_kv", "hq_decode_workspace_size", "hq_decode_attn",
-            "hq_prefill_quant", "hq_prefill_workspace_size", "hq_prefill_attn"]
+            "hq_prefill_quant", "hq_prefill_workspace_size", "hq_prefill_attn",
+            "hq_decode_attn_static"]
+
+HQ_ERR_SCRATCH_LIMIT = 7
+STATIC_SCRATCH_BYTES = 8 << 20
 
 
 class HQError(RuntimeError):
@@ -176,6 +182,18 @@ def hq_decode_attn(q, cache: KVCache, B, Hq, Hkv, D, softmax_scale, out, lse_out
     _check(_decode(_ptr(q), ctypes.byref(st), B, Hq, Hkv, D, float(softmax_scale), _ptr(out),
                    _ptr(lse_out), _ptr(ws), ws.numel() if ws is not None else 0, _stream(stream)),
            "hq_decode_attn")
+
+
+def hq_decode_attn_static(q, cache: KVCache, B, Hq, Hkv, D, softmax_scale, out, lse_out,
+                          stream=None):
+    """Decode without a workspace argument: for callers that cannot allocate
+    device memory when they call (stream capture in progress, memory fixed at
+    start-up).  Its scratch is the library's fixed device array; make the first
+    call on each device before any stream capture begins, and do not overlap
+    calls on the GPU."""
+    st = cache.struct()
+    _check(_decode_static(_ptr(q), ctypes.byref(st), B, Hq, Hkv, D, float(softmax_scale),
+                          _ptr(out), _ptr(lse_out), _stream(stream)), "hq_decode_attn_static")
 
 
 def hq_prefill_quant(q, k, B, Hq, Hkv, N, D, qi8, sq, ki8, sk, stream=None):
