@@ -206,20 +206,25 @@ hq_status hq_decode_attn_static(const void *q, const hq_kv_cache *cache, int B, 
 /* ------------------------------------------------------------------------ */
 /*
  * Pre-pass: symmetric INT8 codes for Q, one scale per (b, head, row), and for
- * K, one scale per (b, kv head, block of 64 keys):
+ * the remaining keys -- those that are not vertical columns (idx), taken in
+ * position order -- one scale per (b, kv head, block of 64 consecutive
+ * remaining keys).  Vertical-column keys are never quantized.
  *   s = fl32(amax / 127) (1 when amax == 0),  code = clamp(rne(fl32(x / s)), -127, 127).
  *   q: bf16 [B, Hq, N, D] -> qi8 i8 [B, Hq, N, D], sq f32 [B, Hq, N]
- *   k: bf16 [B, Hkv, N, D] -> ki8 i8 [B, Hkv, N, D], sk f32 [B, Hkv, ceil(N / 64)]
+ *   k: bf16 [B, Hkv, N, D], idx i32 [B, Hkv, k_vert] (ascending) ->
+ *      ki8 i8 [B, Hkv, N - k_vert, D], sk f32 [B, Hkv, ceil((N - k_vert) / 64)]
  */
-hq_status hq_prefill_quant(const void *q, const void *k, int B, int Hq, int Hkv, int N, int D,
-                           int8_t *qi8, float *sq, int8_t *ki8, float *sk, void *stream);
+hq_status hq_prefill_quant(const void *q, const void *k, const int32_t *idx, int B, int Hq,
+                           int Hkv, int N, int D, int k_vert, int8_t *qi8, float *sq,
+                           int8_t *ki8, float *sk, void *stream);
 
 /*
  * Causal attention in which, for query i, key j <= i is "high" when it is in
  * the window (j > i - window) or is a vertical column of idx, else "low".
  * High logits are bf16 q . k (fp32 accumulate); low logits are the exact INT8
- * dot product of the pre-pass codes times sq[i] * sk[j / 64]; one online
- * softmax covers both; P . V uses fp16 P and V with fp32 accumulation.
+ * dot product of the pre-pass codes times sq[i] and the scale of the key's
+ * block of remaining keys; one online softmax covers both; P . V uses fp16 P
+ * and V with fp32 accumulation.
  *   q: bf16 [B, Hq, N, D];  k, v: bf16 [B, Hkv, N, D];
  *   idx: i32 [B, Hkv, k_vert] ascending (from hq_probe_vertical);
  *   out: f32 [B, Hq, N, D].  The workspace holds the pre-pass output.

@@ -154,16 +154,20 @@ hq_status hq_decode_attn(const void *q, const hq_kv_cache *cache, int B, int Hq,
                                    status_word(ws), (cudaStream_t)stream));
 }
 
-hq_status hq_prefill_quant(const void *q, const void *k, int B, int Hq, int Hkv, int N, int D,
-                           int8_t *qi8, float *sq, int8_t *ki8, float *sk, void *stream) {
-  if (!q || !k || !qi8 || !sq || !ki8 || !sk) return HQ_ERR_INVALID_ARG;
-  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || N <= 0) return HQ_ERR_INVALID_ARG;
+hq_status hq_prefill_quant(const void *q, const void *k, const int32_t *idx, int B, int Hq,
+                           int Hkv, int N, int D, int k_vert, int8_t *qi8, float *sq,
+                           int8_t *ki8, float *sk, void *stream) {
+  if (!q || !k || !qi8 || !sq || (k_vert < N && (!ki8 || !sk)) || (k_vert > 0 && !idx))
+    return HQ_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || N <= 0 || k_vert < 0 || k_vert > N)
+    return HQ_ERR_INVALID_ARG;
   if ((D != 64 && D != 128) || !supported_G(Hq, Hkv)) return HQ_ERR_UNSUPPORTED;
   const void *ptrs[] = {q, k, qi8, ki8};
   for (const void *p : ptrs)
-    if (!aligned16(p)) return HQ_ERR_INVALID_ARG;
-  return cuda_status(launch_prefill_quant((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, B,
-                                          Hq, Hkv, N, D, qi8, sq, ki8, sk, (cudaStream_t)stream));
+    if (p && !aligned16(p)) return HQ_ERR_INVALID_ARG;
+  return cuda_status(launch_prefill_quant((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, idx,
+                                          B, Hq, Hkv, N, D, k_vert, qi8, sq, ki8, sk,
+                                          (cudaStream_t)stream));
 }
 
 size_t hq_prefill_workspace_size(int B, int Hq, int Hkv, int N, int D, int k_vert) {

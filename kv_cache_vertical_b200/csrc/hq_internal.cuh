@@ -53,22 +53,23 @@ cudaError_t launch_decode(const __nv_bfloat16 *q, const hq_kv_cache &c, int B, i
                           int D, float scale, float *out, float *lse, uint8_t *ws,
                           uint32_t *status, cudaStream_t s);
 
-cudaError_t launch_prefill_quant(const __nv_bfloat16 *q, const __nv_bfloat16 *k, int B, int Hq,
-                                 int Hkv, int N, int D, int8_t *qi8, float *sq, int8_t *ki8,
-                                 float *sk, cudaStream_t s);
+cudaError_t launch_prefill_quant(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
+                                 const int32_t *idx, int B, int Hq, int Hkv, int N, int D,
+                                 int k_vert, int8_t *qi8, float *sq, int8_t *ki8, float *sk,
+                                 cudaStream_t s);
 // tcgen05 prefill (head_dim 128, an even number of query heads per KV head).
 struct TcLaunch {
   const __nv_bfloat16 *q, *k;        // bf16 [B,Hq,N,D], [B,Hkv,N,D]
-  const int8_t *qi8, *ki8;           // pre-pass codes
-  const float *sq, *sk;              // pre-pass scales (sk per 64 keys)
-  const __half *vh;                  // fp16 V [B,Hkv,N,D]
+  const int8_t *qi8, *ki8;           // pre-pass codes (ki8 over the remaining keys)
+  const float *sq, *sk;              // pre-pass scales (sk per 64 remaining keys)
+  const __half *vh;                  // fp16 V in position order [B,Hkv,N,D]
+  const __half *vc;                  // fp16 V of the remaining keys [B,Hkv,N-k_vert,D]
   const __nv_bfloat16 *vk;           // compact vertical K [B,Hkv,kpad,D]
   const __half *vv;                  // compact vertical V
-  const int32_t *vpos, *idx;
-  const unsigned long long *vbits;
+  const int32_t *idx;
   float *out;
   uint32_t *status;
-  int B, Hq, Hkv, N, window, k_vert, kpad, nblk64;
+  int B, Hq, Hkv, N, window, k_vert, kpad, nblk_r;
   float scale;
 };
 bool prefill_tc_supported(int D, int Hq, int Hkv);

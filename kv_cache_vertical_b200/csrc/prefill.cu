@@ -74,20 +74,37 @@ __global__ void quant_q_rows(const __nv_bfloat16 *__restrict__ q, long long nrow
   if (lane == 0) sq[row] = s;
 }
 
-// One CTA (256 threads) per block of 64 keys of one (b, kv head).
+// Position of the c-th remaining (non-vertical) key: c plus the number of
+// vertical columns before it, i.e. the count of r with idx[r] - r <= c.
+__device__ __forceinline__ int remaining_pos(const int32_t *id, int k_vert, int c) {
+  int lo = 0, hi = k_vert;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(id + mid) - mid <= c) lo = mid + 1;
+    else hi = mid;
+  }
+  return c + lo;
+}
+
+// One CTA (256 threads) per block of 64 consecutive remaining keys of one
+// (b, kv head): INT8 codes with one symmetric scale per block.
 template <int D>
 __global__ void __launch_bounds__(256)
-quant_k_blocks(const __nv_bfloat16 *__restrict__ k, int N, int nblk, int8_t *__restrict__ ki8,
-               float *__restrict__ sk) {
+quant_k_remaining(const __nv_bfloat16 *__restrict__ k, const int32_t *__restrict__ idx, int N,
+                  int k_vert, int nblk, int8_t *__restrict__ ki8, float *__restrict__ sk) {
+  constexpr int WPR = D / 2;                                    // 32-bit words per row
   const int blk = blockIdx.x, bh = blockIdx.y;
-  const int j0 = blk * TILE, n = min(TILE, N - j0);
-  const int nval = n * D;                                       // values in this block
-  const __nv_bfloat16 *src = k + ((size_t)bh * N + j0) * D;
-  int8_t *dst = ki8 + ((size_t)bh * N + j0) * D;
+  const int nr = N - k_vert;
+  const int c0 = blk * TILE, n = min(TILE, nr - c0);
+  const int32_t *id = idx + (size_t)bh * k_vert;
+  __shared__ int pos[TILE];
   __shared__ float red[8];
+  if (threadIdx.x < n) pos[threadIdx.x] = remaining_pos(id, k_vert, c0 + threadIdx.x);
+  __syncthreads();
+  const uint32_t *src = reinterpret_cast<const uint32_t *>(k + (size_t)bh * N * D);
   float amax = 0.f;
-  for (int e = threadIdx.x * 2; e < nval; e += blockDim.x * 2) {
-    const uint32_t w = reinterpret_cast<const uint32_t *>(src)[e / 2];
+  for (int e = threadIdx.x; e < n * WPR; e += blockDim.x) {
+    const uint32_t w = src[(size_t)pos[e / WPR] * WPR + e % WPR];
     amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(w)), fabsf(bf16_hi(w))));
   }
 #pragma unroll
@@ -98,27 +115,48 @@ quant_k_blocks(const __nv_bfloat16 *__restrict__ k, int N, int nblk, int8_t *__r
 #pragma unroll
   for (int w = 1; w < 8; ++w) amax = fmaxf(amax, red[w]);
   const float s = amax == 0.f ? 1.f : __fdiv_rn(amax, 127.f);
-  for (int e = threadIdx.x * 2; e < nval; e += blockDim.x * 2) {
-    const uint32_t w = reinterpret_cast<const uint32_t *>(src)[e / 2];
-    float c0 = fminf(fmaxf(rintf(__fdiv_rn(bf16_lo(w), s)), -127.f), 127.f);
-    float c1 = fminf(fmaxf(rintf(__fdiv_rn(bf16_hi(w), s)), -127.f), 127.f);
-    reinterpret_cast<uint16_t *>(dst)[e / 2] =
-        (uint16_t)(((uint32_t)(int)c0 & 0xffu) | (((uint32_t)(int)c1 & 0xffu) << 8));
+  uint16_t *dst = reinterpret_cast<uint16_t *>(ki8 + ((size_t)bh * nr + c0) * D);
+  for (int e = threadIdx.x; e < n * WPR; e += blockDim.x) {
+    const uint32_t w = src[(size_t)pos[e / WPR] * WPR + e % WPR];
+    float c0f = fminf(fmaxf(rintf(__fdiv_rn(bf16_lo(w), s)), -127.f), 127.f);
+    float c1f = fminf(fmaxf(rintf(__fdiv_rn(bf16_hi(w), s)), -127.f), 127.f);
+    dst[e] = (uint16_t)(((uint32_t)(int)c0f & 0xffu) | (((uint32_t)(int)c1f & 0xffu) << 8));
   }
   if (threadIdx.x == 0) sk[(size_t)bh * nblk + blk] = s;
 }
 
-// bf16 V -> fp16 V (exact for |v| in the fp16 normal range).
-__global__ void v_to_f16(const __nv_bfloat16 *__restrict__ v, __half *__restrict__ vh, long long n2) {
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n2;
-       i += (long long)gridDim.x * blockDim.x) {
-    const uint32_t w = reinterpret_cast<const uint32_t *>(v)[i];
-    reinterpret_cast<__half2 *>(vh)[i] = __floats2half2_rn(bf16_lo(w), bf16_hi(w));
+// bf16 V -> fp16 V (exact for |v| in the fp16 normal range), both in position
+// order (window tiles) and compacted to the remaining keys (low-bit tiles).
+// One warp per (b, kv head, position).
+template <int D>
+__global__ void v_prep(const __nv_bfloat16 *__restrict__ v, const int32_t *__restrict__ idx,
+                       int nbh, int N, int k_vert, __half *__restrict__ vh,
+                       __half *__restrict__ vc) {
+  constexpr int W32 = D / 64;                                    // 32-bit words per lane
+  const int lane = threadIdx.x & 31;
+  const long long total = (long long)nbh * N;
+  const int nr = N - k_vert;
+  for (long long wi = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); wi < total;
+       wi += (long long)gridDim.x * (blockDim.x / 32)) {
+    const int bh = (int)(wi / N), j = (int)(wi % N);
+    const int32_t *id = idx + (size_t)bh * k_vert;
+    const int cnt = upper_bound_i32(id, k_vert, j);              // verticals <= j
+    const bool vert = cnt > 0 && __ldg(id + cnt - 1) == j;
+    const uint32_t *src = reinterpret_cast<const uint32_t *>(v + wi * D) + lane * W32;
+    __half2 *dh = reinterpret_cast<__half2 *>(vh + wi * D) + lane * W32;
+    __half2 *dc = reinterpret_cast<__half2 *>(vc + ((size_t)bh * nr + (j - cnt)) * D) + lane * W32;
+#pragma unroll
+    for (int i = 0; i < W32; ++i) {
+      const uint32_t w = src[i];
+      const __half2 x = __floats2half2_rn(bf16_lo(w), bf16_hi(w));
+      dh[i] = x;
+      if (!vert) dc[i] = x;
+    }
   }
 }
 
-// Compact copies of the vertical rows (padded to a multiple of 64 with zero
-// rows at position INT_MAX) and the per-64-key vertical bitmap.
+// Compact copies of the vertical rows (padded to whole 128-row tiles with zero
+// rows at position INT_MAX).
 template <int D>
 __global__ void gather_vertical(const __nv_bfloat16 *__restrict__ k, const __half *__restrict__ vh,
                                 const int32_t *__restrict__ idx, int N, int k_vert, int kpad,
@@ -138,38 +176,27 @@ __global__ void gather_vertical(const __nv_bfloat16 *__restrict__ k, const __hal
   if (t == 0) kv_pos[(size_t)bh * kpad + r] = pos;
 }
 
-__global__ void vertical_bitmap(const int32_t *__restrict__ idx, int k_vert, int nwords,
-                                unsigned long long *__restrict__ bits) {
-  const int w = blockIdx.x * blockDim.x + threadIdx.x, bh = blockIdx.y;
-  if (w >= nwords) return;
-  const int32_t *id = idx + (size_t)bh * k_vert;
-  int lo = 0, hi = k_vert;  // first entry >= 64 w
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (id[mid] < 64 * w) lo = mid + 1;
-    else hi = mid;
-  }
-  unsigned long long m = 0;
-  for (int e = lo; e < k_vert && id[e] < 64 * (w + 1); ++e) m |= 1ull << (id[e] - 64 * w);
-  bits[(size_t)bh * nwords + w] = m;
-}
-
 // ---------------------------------------------------------------------------
 // Main kernel (warp-level MMA version)
 // ---------------------------------------------------------------------------
 struct PrefillArgs {
   const __nv_bfloat16 *q, *k;
-  const int8_t *qi8, *ki8;
-  const float *sq, *sk;
-  const __half *vh;
+  const int8_t *qi8, *ki8;       // ki8: remaining keys [nbh, nr, D]
+  const float *sq, *sk;          // sk: per 64 remaining keys [nbh, nblk_r]
+  const __half *vh;              // fp16 V in position order [nbh, N, D]
+  const __half *vc;              // fp16 V of the remaining keys [nbh, nr, D]
   const __nv_bfloat16 *vk;       // compact vertical K [nbh, kpad, D]
   const __half *vv;              // compact vertical V
-  const int32_t *vpos;           // [nbh, kpad]
-  const unsigned long long *vbits;  // [nbh, nblk]
+  const int32_t *idx;            // [nbh, k_vert]
   float *out;
-  int Hq, Hkv, G, N, window, kpad, nblk;
+  int Hq, Hkv, G, N, window, k_vert, kpad, nr, nblk_r;
   float scale_log2;
 };
+
+// Remaining (non-vertical) keys at positions <= x.
+__device__ __forceinline__ int remaining_upto(const int32_t *id, int k_vert, int x) {
+  return x < 0 ? 0 : x + 1 - upper_bound_i32(id, k_vert, x);
+}
 
 template <int D>
 struct Smem {
@@ -334,52 +361,62 @@ prefill_mma(PrefillArgs a) {
   };
 
   const int i_min = qt * TILE;
-  // 1) key tiles 0 .. qt (INT8, plus bf16 where the window reaches)
-  for (int kt = 0; kt <= qt; ++kt) {
-    const int j0 = kt * TILE;
-    const int nvalid = min(TILE, a.N - j0);
-    const bool band = (j0 + TILE - 1 >= i_min - W + 1) || kt == qt;
+  const int i_max = min(qt * TILE + TILE - 1, a.N - 1);
+  const int32_t *id = a.idx + bh * a.k_vert;
+  // Per row: remaining keys with position <= i - W (low-bit pairs) and
+  // vertical columns <= i - W (high pairs); both grow with i.
+  int cnt[2], nvt[2];
+#pragma unroll
+  for (int hf = 0; hf < 2; ++hf) {
+    cnt[hf] = remaining_upto(id, a.k_vert, rows[hf] - W);
+    nvt[hf] = rows[hf] - W >= 0 ? upper_bound_i32(id, a.k_vert, rows[hf] - W) : 0;
+  }
+  const int cnt_lo = remaining_upto(id, a.k_vert, i_min - W);
+  const int cnt_hi = remaining_upto(id, a.k_vert, i_max - W);
+  // 1) low-bit tiles over the remaining keys (INT8 QK, compact fp16 V)
+  for (int t = 0; t * TILE < cnt_hi; ++t) {
+    const int c0 = t * TILE;
+    const int nvalid = min(TILE, a.nr - c0);
     __syncthreads();
-    load_tile<D>(sm.ki8, reinterpret_cast<const uint8_t *>(a.ki8 + (bh * a.N + j0) * D), nvalid);
-    load_tile<D * 2>(sm.vh, reinterpret_cast<const uint8_t *>(a.vh + (bh * a.N + j0) * D), nvalid);
-    if (band && W > 0)
-      load_tile<D * 2>(sm.kbf, reinterpret_cast<const uint8_t *>(a.k + (bh * a.N + j0) * D), nvalid);
+    load_tile<D>(sm.ki8, reinterpret_cast<const uint8_t *>(a.ki8 + (bh * a.nr + c0) * D), nvalid);
+    load_tile<D * 2>(sm.vh, reinterpret_cast<const uint8_t *>(a.vc + (bh * a.nr + c0) * D), nvalid);
     __syncthreads();
-    const unsigned long long vbits = a.vbits[bh * a.nblk + kt];
     float s[NT][4];
-    qk_int8(s, a.sk[bh * a.nblk + kt]);
-    if (band) {
-      float sb[NT][4];
-      if (W > 0) qk_bf16(sb);
+    qk_int8(s, a.sk[bh * a.nblk_r + t]);
+    if (c0 + TILE > cnt_lo) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (c0 + nt * 8 + 2 * c + (e & 1) >= cnt[e >> 1]) s[nt][e] = -INFINITY;
+    }
+    softmax_pv(s);
+  }
+  // 2) window tiles in position order (bf16 QK): keep i - W < j <= i
+  if (W > 0) {
+    for (int kt = max(0, i_min - W + 1) / TILE; kt * TILE <= i_max; ++kt) {
+      const int j0 = kt * TILE;
+      const int nvalid = min(TILE, a.N - j0);
+      __syncthreads();
+      load_tile<D * 2>(sm.kbf, reinterpret_cast<const uint8_t *>(a.k + (bh * a.N + j0) * D), nvalid);
+      load_tile<D * 2>(sm.vh, reinterpret_cast<const uint8_t *>(a.vh + (bh * a.N + j0) * D), nvalid);
+      __syncthreads();
+      float s[NT][4];
+      qk_bf16(s);
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int i = rows[e >> 1];
-          const int jj = nt * 8 + 2 * c + (e & 1);
-          const int j = j0 + jj;
-          float v = s[nt][e];
-          if (j > i) v = -INFINITY;
-          else if (j > i - W) v = W > 0 ? sb[nt][e] : v;
-          else if ((vbits >> jj) & 1ull) v = -INFINITY;
-          s[nt][e] = v;
+          const int j = j0 + nt * 8 + 2 * c + (e & 1);
+          if (j > i || j <= i - W) s[nt][e] = -INFINITY;
         }
-    } else if (vbits) {
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int jj = nt * 8 + 2 * c + (e & 1);
-          if ((vbits >> jj) & 1ull) s[nt][e] = -INFINITY;
-        }
+      softmax_pv(s);
     }
-    softmax_pv(s);
   }
-  // 2) compact vertical tiles: key v counts for row i only when v <= i - W
-  const int i_max = min(qt * TILE + TILE - 1, a.N - 1);
-  const int32_t *vp = a.vpos + bh * a.kpad;
-  for (int vt = 0; vt * TILE < a.kpad; ++vt) {
-    if (vp[vt * TILE] > i_max - W) break;
+  // 3) compact vertical tiles (bf16 QK): column v counts for row i when v <= i - W
+  const int nv_max = i_max - W >= 0 ? upper_bound_i32(id, a.k_vert, i_max - W) : 0;
+  for (int vt = 0; vt * TILE < nv_max; ++vt) {
     __syncthreads();
     load_tile<D * 2>(sm.kbf, reinterpret_cast<const uint8_t *>(a.vk + (bh * a.kpad + vt * TILE) * D), TILE);
     load_tile<D * 2>(sm.vh, reinterpret_cast<const uint8_t *>(a.vv + (bh * a.kpad + vt * TILE) * D), TILE);
@@ -389,11 +426,8 @@ prefill_mma(PrefillArgs a) {
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int i = rows[e >> 1];
-        const int pos = vp[vt * TILE + nt * 8 + 2 * c + (e & 1)];
-        if (pos > i - W) s[nt][e] = -INFINITY;  // INT_MAX padding is masked too
-      }
+      for (int e = 0; e < 4; ++e)
+        if (vt * TILE + nt * 8 + 2 * c + (e & 1) >= nvt[e >> 1]) s[nt][e] = -INFINITY;
     softmax_pv(s);
   }
   // 3) normalize and store fp32 rows
@@ -417,17 +451,17 @@ prefill_mma(PrefillArgs a) {
 struct PrefillWs {
   int8_t *qi8, *ki8;
   float *sq, *sk;
-  __half *vh, *vv;
+  __half *vh, *vc, *vv;
   __nv_bfloat16 *vk;
   int32_t *vpos;
-  unsigned long long *vbits;
   size_t total;
 };
 
 PrefillWs carve(uint8_t *base, int B, int Hq, int Hkv, int N, int D, int k_vert) {
   PrefillWs w;
   const size_t nbh = (size_t)B * Hkv, nbq = (size_t)B * Hq;
-  const int nblk = (N + TILE - 1) / TILE;
+  const size_t nr = (size_t)(N - k_vert);
+  const size_t nblk_r = (nr + TILE - 1) / TILE;
   const size_t kpad = (size_t)((k_vert + 127) / 128) * 128;  // whole 128-row tiles
   size_t off = kWsHeader;
   auto take = [&](size_t bytes) {
@@ -437,24 +471,26 @@ PrefillWs carve(uint8_t *base, int B, int Hq, int Hkv, int N, int D, int k_vert)
   };
   w.qi8 = (int8_t *)take(nbq * N * D);
   w.sq = (float *)take(nbq * N * sizeof(float));
-  w.ki8 = (int8_t *)take(nbh * N * D);
-  w.sk = (float *)take(nbh * nblk * sizeof(float));
+  w.ki8 = (int8_t *)take(nbh * nr * D);
+  w.sk = (float *)take(nbh * nblk_r * sizeof(float));
   w.vh = (__half *)take(nbh * N * D * 2);
+  w.vc = (__half *)take(nbh * nr * D * 2);
   w.vk = (__nv_bfloat16 *)take(nbh * kpad * D * 2);
   w.vv = (__half *)take(nbh * kpad * D * 2);
   w.vpos = (int32_t *)take(nbh * kpad * sizeof(int32_t));
-  w.vbits = (unsigned long long *)take(nbh * nblk * sizeof(unsigned long long));
   w.total = off;
   return w;
 }
 
 template <int D>
-cudaError_t quant_t(const __nv_bfloat16 *q, const __nv_bfloat16 *k, int B, int Hq, int Hkv, int N,
-                    int8_t *qi8, float *sq, int8_t *ki8, float *sk, cudaStream_t s) {
+cudaError_t quant_t(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const int32_t *idx, int B,
+                    int Hq, int Hkv, int N, int k_vert, int8_t *qi8, float *sq, int8_t *ki8,
+                    float *sk, cudaStream_t s) {
   const long long nrows = (long long)B * Hq * N;
   quant_q_rows<D><<<(unsigned)((nrows + 7) / 8), 256, 0, s>>>(q, nrows, qi8, sq);
-  const int nblk = (N + TILE - 1) / TILE;
-  quant_k_blocks<D><<<dim3(nblk, B * Hkv), 256, 0, s>>>(k, N, nblk, ki8, sk);
+  const int nblk_r = (N - k_vert + TILE - 1) / TILE;
+  if (nblk_r > 0)
+    quant_k_remaining<D><<<dim3(nblk_r, B * Hkv), 256, 0, s>>>(k, idx, N, k_vert, nblk_r, ki8, sk);
   return cudaGetLastError();
 }
 
@@ -464,16 +500,22 @@ cudaError_t prefill_t(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
                       float scale, float *out, uint8_t *ws, uint32_t *status, cudaStream_t s) {
   PrefillWs w = carve(ws, B, Hq, Hkv, N, D, k_vert);
   const int nbh = B * Hkv;
-  const int nblk = (N + TILE - 1) / TILE;
+  const int nr = N - k_vert;
+  const int nblk_r = (nr + TILE - 1) / TILE;
   const int kpad = (k_vert + 127) / 128 * 128;
-  cudaError_t e = quant_t<D>(q, k, B, Hq, Hkv, N, w.qi8, w.sq, w.ki8, w.sk, s);
+  cudaError_t e = quant_t<D>(q, k, idx, B, Hq, Hkv, N, k_vert, w.qi8, w.sq, w.ki8, w.sk, s);
   if (e != cudaSuccess) return e;
-  const long long n2 = (long long)nbh * N * D / 2;
-  v_to_f16<<<1184, 256, 0, s>>>(v, w.vh, n2);
+  {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    long long blocks = ((long long)nbh * N + 7) / 8;
+    if (blocks > 8LL * sms) blocks = 8LL * sms;
+    v_prep<D><<<(unsigned)blocks, 256, 0, s>>>(v, idx, nbh, N, k_vert, w.vh, w.vc);
+  }
   if (kpad > 0)
     gather_vertical<D><<<dim3(kpad, nbh), D / 8, 0, s>>>(k, w.vh, idx, N, k_vert, kpad, w.vk,
                                                          w.vv, w.vpos);
-  vertical_bitmap<<<dim3((nblk + 127) / 128, nbh), 128, 0, s>>>(idx, k_vert, nblk, w.vbits);
   if (prefill_tc_supported(D, Hq, Hkv)) {
     TcLaunch p;
     p.q = q;
@@ -483,11 +525,10 @@ cudaError_t prefill_t(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
     p.sq = w.sq;
     p.sk = w.sk;
     p.vh = w.vh;
+    p.vc = w.vc;
     p.vk = w.vk;
     p.vv = w.vv;
-    p.vpos = w.vpos;
     p.idx = idx;
-    p.vbits = w.vbits;
     p.out = out;
     p.status = status;
     p.B = B;
@@ -497,7 +538,7 @@ cudaError_t prefill_t(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
     p.window = window;
     p.k_vert = k_vert;
     p.kpad = kpad;
-    p.nblk64 = nblk;
+    p.nblk_r = nblk_r;
     p.scale = scale;
     return launch_prefill_tc(p, s);
   }
@@ -509,30 +550,33 @@ cudaError_t prefill_t(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
   a.sq = w.sq;
   a.sk = w.sk;
   a.vh = w.vh;
+  a.vc = w.vc;
   a.vk = w.vk;
   a.vv = w.vv;
-  a.vpos = w.vpos;
-  a.vbits = w.vbits;
+  a.idx = idx;
   a.out = out;
   a.Hq = Hq;
   a.Hkv = Hkv;
   a.G = Hq / Hkv;
   a.N = N;
   a.window = window;
+  a.k_vert = k_vert;
   a.kpad = kpad;
-  a.nblk = nblk;
+  a.nr = nr;
+  a.nblk_r = nblk_r;
   a.scale_log2 = scale * kLog2e;
-  prefill_mma<D><<<dim3(nblk, Hq, B), FWARPS * 32, 0, s>>>(a);
+  prefill_mma<D><<<dim3((N + TILE - 1) / TILE, Hq, B), FWARPS * 32, 0, s>>>(a);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_prefill_quant(const __nv_bfloat16 *q, const __nv_bfloat16 *k, int B, int Hq,
-                                 int Hkv, int N, int D, int8_t *qi8, float *sq, int8_t *ki8,
-                                 float *sk, cudaStream_t s) {
-  if (D == 128) return quant_t<128>(q, k, B, Hq, Hkv, N, qi8, sq, ki8, sk, s);
-  if (D == 64) return quant_t<64>(q, k, B, Hq, Hkv, N, qi8, sq, ki8, sk, s);
+cudaError_t launch_prefill_quant(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
+                                 const int32_t *idx, int B, int Hq, int Hkv, int N, int D,
+                                 int k_vert, int8_t *qi8, float *sq, int8_t *ki8, float *sk,
+                                 cudaStream_t s) {
+  if (D == 128) return quant_t<128>(q, k, idx, B, Hq, Hkv, N, k_vert, qi8, sq, ki8, sk, s);
+  if (D == 64) return quant_t<64>(q, k, idx, B, Hq, Hkv, N, k_vert, qi8, sq, ki8, sk, s);
   return cudaErrorInvalidValue;
 }
 

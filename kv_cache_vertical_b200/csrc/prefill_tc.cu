@@ -24,8 +24,11 @@
 // The MMA thread alternates the heads (PV_A(t), QK_A(t+1), PV_B(t), QK_B(t+1)),
 // so one head's softmax overlaps the other head's tensor-core work.
 // Key tiles per query tile, each its own iteration of the online softmax:
-//   INT8 tiles  kt with kt*128 <= i_max - W: keep j <= i - W, not vertical;
-//   window      bf16 tiles meeting (i - W, i]: keep i - W < j <= i;
+//   INT8 tiles  128 consecutive REMAINING (non-vertical) keys, compacted in
+//               position order by the pre-pass: keep the keys at positions
+//               <= i - W (a prefix of the compact order, so only the last
+//               tiles need a per-row bound and no tile needs a vertical mask);
+//   window      bf16 tiles of positions meeting (i - W, i]: keep i - W < j <= i;
 //   vertical    compact bf16 rows (sorted): keep v <= i - W;
 // so every causal pair is counted exactly once.
 #include <cuda.h>
@@ -59,17 +62,26 @@ constexpr uint32_t IDESC_PV = make_idesc(1, 0, 0, 0, 1, 128, 128);   // f32 <- f
 
 enum { IT_I8 = 0, IT_WIN = 1, IT_VERT = 2 };
 
+// Raw INT8-tile score that marks a masked entry: as an int it is below any
+// reachable dot product (|s| <= 128 * 127 * 127 < 2^22), and after adding the
+// bits of 2^23 + 2^22 it is the bit pattern of -inf.
+constexpr uint32_t kMaskRaw = 0xFF800000u - kMagicBits;
+constexpr uint32_t kNegInfBits = 0xFF800000u;
+
 struct TcArgs {
   const float *sq;                    // [B*Hq, N]
-  const float *sk;                    // [B*Hkv, nblk64]
-  const unsigned long long *vbits;    // [B*Hkv, nblk64] vertical bitmap per 64 keys
-  const int32_t *vpos;                // [B*Hkv, kpad] compact vertical positions (INT_MAX pad)
-  const int32_t *idx;                 // [B*Hkv, k_vert]
+  const float *sk;                    // [B*Hkv, nblk_r] one scale per 64 remaining keys
+  const int32_t *idx;                 // [B*Hkv, k_vert] vertical columns, ascending
   float *out;                         // [B*Hq, N, D]
   uint32_t *status;
-  int Hq, Hkv, N, window, k_vert, kpad, nblk64;
+  int Hq, Hkv, N, window, k_vert, nblk_r;
   float sl;                           // softmax scale * log2(e)
 };
+
+// Remaining (non-vertical) keys at positions <= x.
+__device__ __forceinline__ int remaining_upto(const int32_t *id, int k_vert, int x) {
+  return x < 0 ? 0 : x + 1 - upper_bound_i32(id, k_vert, x);
+}
 
 struct Sched {
   int n_i8, n_w, kw0, n;
@@ -85,7 +97,8 @@ __device__ __forceinline__ Sched make_sched(const TcArgs &a, int i0, size_t bh) 
   Sched s;
   const int i_max = min(i0 + BM - 1, a.N - 1);
   const int W = a.window;
-  s.n_i8 = (i_max - W >= 0) ? (i_max - W) / BN + 1 : 0;
+  const int32_t *id = a.idx + bh * a.k_vert;
+  s.n_i8 = (remaining_upto(id, a.k_vert, i_max - W) + BN - 1) / BN;
   if (W > 0) {
     s.kw0 = max(0, i0 - W + 1) / BN;
     s.n_w = i_max / BN - s.kw0 + 1;
@@ -93,8 +106,7 @@ __device__ __forceinline__ Sched make_sched(const TcArgs &a, int i0, size_t bh) 
     s.kw0 = 0;
     s.n_w = 0;
   }
-  int cnt = 0;
-  if (a.k_vert > 0 && i_max - W >= 0) cnt = upper_bound_i32(a.idx + bh * a.k_vert, a.k_vert, i_max - W);
+  const int cnt = i_max - W >= 0 ? upper_bound_i32(id, a.k_vert, i_max - W) : 0;
   s.n = s.n_i8 + s.n_w + (cnt + BN - 1) / BN;
   return s;
 }
@@ -103,7 +115,8 @@ __global__ void __launch_bounds__(NT, 1)
 prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ CUtensorMap tm_qbf,
            const __grid_constant__ CUtensorMap tm_ki8, const __grid_constant__ CUtensorMap tm_kbf,
            const __grid_constant__ CUtensorMap tm_v16, const __grid_constant__ CUtensorMap tm_vk,
-           const __grid_constant__ CUtensorMap tm_vv, TcArgs a) {
+           const __grid_constant__ CUtensorMap tm_vv, const __grid_constant__ CUtensorMap tm_vc,
+           TcArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bar = reinterpret_cast<uint64_t *>(smem + SM_BAR);
@@ -181,7 +194,7 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
           tma_load_3d(ks, km, &kv_full[s], 0, row, (int)bh);
           tma_load_3d(ks + 16384, km, &kv_full[s], 64, row, (int)bh);
         }
-        const CUtensorMap *vm = ty == IT_VERT ? &tm_vv : &tm_v16;
+        const CUtensorMap *vm = ty == IT_VERT ? &tm_vv : (ty == IT_I8 ? &tm_vc : &tm_v16);
         tma_load_3d(vs, vm, &kv_full[s], 0, row, (int)bh);
         tma_load_3d(vs + 16384, vm, &kv_full[s], 64, row, (int)bh);
         issued = it + 1;
@@ -257,6 +270,11 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
     }
   } else {
     // ------------------------------ softmax ------------------------------
+    // Two passes over the S row in tensor memory (64 columns at a time): the
+    // row max first, then exp2 / row sum / fp16 packing of P, so that only a
+    // half row is ever held in registers.  INT8 scores stay integers until
+    // the exp: their max is an integer max, and s -> float is one add of the
+    // bits of 2^23 + 2^22 (exact for |s| < 2^22) folded into the scaling FMA.
     const int X = (warp - 2) >> 2;                 // 0: head A, 1: head B
     const int hq = hA + X;
     const int quarter = warp & 3;                  // TMEM lanes 32*quarter ..
@@ -265,8 +283,13 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
     const uint32_t tS = tl + X * 256, tO = tS + 128;
     const size_t bhq = (size_t)b * a.Hq + hq;
-    const float sqi = (i < a.N) ? a.sq[bhq * a.N + i] * a.sl : 0.f;
+    const float sqi = (i < a.N) ? a.sq[bhq * a.N + i] * a.sl : 1.f;
     const int W = a.window;
+    const int lim = i - W;                         // low-bit and vertical keys need j <= lim
+    const int32_t *id = a.idx + bh * a.k_vert;
+    const int cnt_i = remaining_upto(id, a.k_vert, lim);        // low-bit keys of this row
+    const int cnt_lo = remaining_upto(id, a.k_vert, i0 - W);     // ... of the tile's first row
+    const int nvert = lim >= 0 ? upper_bound_i32(id, a.k_vert, lim) : 0;
     float m = -1e30f, l = 0.f;
     bool ok = true;
     for (int it = 0; it < sc.n; ++it) {
@@ -276,49 +299,62 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
       }
       tc_fence_after();
       const int ty = sc.type(it), t = sc.tile(it);
-      float x[128];
-      float mt = -INFINITY;
+      const int j0 = t * BN;
+      float scl[2] = {0.f, 0.f};
+      bool need_lim = false;
+      int nvalid = BN;
+      if (ty == IT_I8) {
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t raw[32];
-        tmem_ld32(tS + ch * 32, raw);
-        const int j0 = t * BN + ch * 32;
+        for (int h = 0; h < 2; ++h) {
+          const int blk = 2 * t + h;
+          scl[h] = sqi * (blk < a.nblk_r ? __ldg(a.sk + bh * a.nblk_r + blk) : 1.f);
+        }
+        need_lim = j0 + BN > cnt_lo;               // same for every row of the tile
+        nvalid = cnt_i - j0;
+      } else if (ty == IT_VERT) {
+        nvalid = nvert - j0;
+      }
+      auto apply_masks = [&](uint32_t (&x)[64], int h) {
         if (ty == IT_I8) {
-          const int blk = t * 2 + (ch >> 1);
-          const float scl = sqi * a.sk[bh * a.nblk64 + blk];
-          const float off = -kMagic * scl;
-          const uint32_t mw = (uint32_t)(a.vbits[bh * a.nblk64 + blk] >> ((ch & 1) * 32));
-          const int lim = i - W;
+          if (need_lim) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            float v = fmaf(__uint_as_float(raw[e] + kMagicBits), scl, off);
-            if (j0 + e > lim || ((mw >> e) & 1u)) v = -INFINITY;
-            x[ch * 32 + e] = v;
-            mt = fmaxf(mt, v);
+            for (int e = 0; e < 64; ++e)
+              if (h * 64 + e >= nvalid) x[e] = kMaskRaw;
           }
         } else if (ty == IT_WIN) {
+          const int jh = j0 + h * 64;
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            float v = __uint_as_float(raw[e]) * a.sl;
-            const int j = j0 + e;
-            if (j > i || j <= i - W) v = -INFINITY;
-            x[ch * 32 + e] = v;
-            mt = fmaxf(mt, v);
+          for (int e = 0; e < 64; ++e) {
+            const int j = jh + e;
+            if (j > i || j <= lim) x[e] = kNegInfBits;
           }
         } else {
-          const int32_t *vp = a.vpos + bh * a.kpad + j0;
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            float v = __uint_as_float(raw[e]) * a.sl;
-            if (__ldg(vp + e) > i - W) v = -INFINITY;
-            x[ch * 32 + e] = v;
-            mt = fmaxf(mt, v);
-          }
+          for (int e = 0; e < 64; ++e)
+            if (h * 64 + e >= nvalid) x[e] = kNegInfBits;
+        }
+      };
+      // ---- pass 1: row max (log2 units) ----
+      float mt = -INFINITY;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t x[64];
+        tmem_ld64(tS + h * 64, x);
+        apply_masks(x, h);
+        if (ty == IT_I8) {
+          int mx = (int)kMaskRaw;
+#pragma unroll
+          for (int e = 0; e < 64; ++e) mx = max(mx, (int)x[e]);
+          mt = fmaxf(mt, fmaf(__uint_as_float((uint32_t)mx + kMagicBits), scl[h], -kMagic * scl[h]));
+        } else {
+          float mx = -INFINITY;
+#pragma unroll
+          for (int e = 0; e < 64; ++e) mx = fmaxf(mx, __uint_as_float(x[e]));
+          mt = fmaxf(mt, mx * a.sl);
         }
       }
-      // lazy rescale of the running max (and of O, which the MMA of the
-      // previous iteration has finished: the commit this thread waited on
-      // covers every MMA issued before it)
+      // ---- lazy rescale of the running max (and of O: the commit this
+      // thread waited on covers every MMA issued before it) ----
       const bool need = mt > m + kLazy;
       if (__any_sync(0xffffffffu, need)) {
         const float mn = fmaxf(m, mt);
@@ -337,18 +373,34 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
           tmem_wait_st();
         }
       }
+      // ---- pass 2: P = exp2(x - m) as packed fp16 into the first 64 columns ----
       float rs = 0.f;
 #pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
+      for (int h = 0; h < 2; ++h) {
+        uint32_t x[64];
+        tmem_ld64(tS + h * 64, x);
+        apply_masks(x, h);
         uint32_t pk[32];
+        if (ty == IT_I8) {
+          const float sc_ = scl[h], c_ = -kMagic * scl[h] - m;
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const float p0 = fast_exp2(x[h2 * 64 + 2 * e] - m);
-          const float p1 = fast_exp2(x[h2 * 64 + 2 * e + 1] - m);
-          rs += p0 + p1;
-          pk[e] = pack_f16x2(p0, p1);
+          for (int e = 0; e < 32; ++e) {
+            const float p0 = fast_exp2(fmaf(__uint_as_float(x[2 * e] + kMagicBits), sc_, c_));
+            const float p1 = fast_exp2(fmaf(__uint_as_float(x[2 * e + 1] + kMagicBits), sc_, c_));
+            rs += p0 + p1;
+            pk[e] = pack_f16x2(p0, p1);
+          }
+        } else {
+          const float c_ = -m;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float p0 = fast_exp2(fmaf(__uint_as_float(x[2 * e]), a.sl, c_));
+            const float p1 = fast_exp2(fmaf(__uint_as_float(x[2 * e + 1]), a.sl, c_));
+            rs += p0 + p1;
+            pk[e] = pack_f16x2(p0, p1);
+          }
         }
-        tmem_st32(tS + h2 * 32, pk);
+        tmem_st32(tS + h * 32, pk);                 // keys 64h .. 64h+63
       }
       l += rs;
       tmem_wait_st();
@@ -400,21 +452,21 @@ cudaError_t launch_prefill_tc(const TcLaunch &p, cudaStream_t s) {
     attr = true;
   }
   const int nbq = p.B * p.Hq, nbh = p.B * p.Hkv;
-  CUtensorMap m[7];
+  const int nr = p.N - p.k_vert;                      // remaining keys per (b, kv head)
+  CUtensorMap m[8];
   bool ok = true;
   ok &= make_map_3d(&m[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (void *)p.qi8, D, p.N, nbq, 128, BM, CU_TENSOR_MAP_SWIZZLE_128B);
   ok &= make_map_3d(&m[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (void *)p.q, D, p.N, nbq, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B);
-  ok &= make_map_3d(&m[2], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (void *)p.ki8, D, p.N, nbh, 128, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_map_3d(&m[2], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (void *)p.ki8, D, nr, nbh, 128, BN, CU_TENSOR_MAP_SWIZZLE_128B);
   ok &= make_map_3d(&m[3], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (void *)p.k, D, p.N, nbh, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B);
   ok &= make_map_3d(&m[4], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (void *)p.vh, D, p.N, nbh, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B);
   ok &= make_map_3d(&m[5], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (void *)p.vk, D, p.kpad, nbh, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B);
   ok &= make_map_3d(&m[6], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (void *)p.vv, D, p.kpad, nbh, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_map_3d(&m[7], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (void *)p.vc, D, nr, nbh, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return cudaErrorInvalidValue;
   TcArgs a;
   a.sq = p.sq;
   a.sk = p.sk;
-  a.vbits = p.vbits;
-  a.vpos = p.vpos;
   a.idx = p.idx;
   a.out = p.out;
   a.status = p.status;
@@ -423,11 +475,10 @@ cudaError_t launch_prefill_tc(const TcLaunch &p, cudaStream_t s) {
   a.N = p.N;
   a.window = p.window;
   a.k_vert = p.k_vert;
-  a.kpad = p.kpad;
-  a.nblk64 = p.nblk64;
+  a.nblk_r = p.nblk_r;
   a.sl = p.scale * kLog2e;
   dim3 grid((p.N + BM - 1) / BM, p.Hq / 2, p.B);
-  prefill_tc<<<grid, NT, SMEM_BYTES, s>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], a);
+  prefill_tc<<<grid, NT, SMEM_BYTES, s>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7], a);
   return cudaGetLastError();
 }
 

@@ -62,7 +62,7 @@ _decode = _sig("hq_decode_attn", _I, _P, ctypes.POINTER(hq_kv_cache), _I, _I, _I
                _P, _SZ, _P)
 _decode_static = _sig("hq_decode_attn_static", _I, _P, ctypes.POINTER(hq_kv_cache), _I, _I, _I,
                       _I, _F, _P, _P, _P)
-_pquant = _sig("hq_prefill_quant", _I, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P)
+_pquant = _sig("hq_prefill_quant", _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P)
 hq_prefill_workspace_size = _sig("hq_prefill_workspace_size", _SZ, _I, _I, _I, _I, _I, _I)
 _prefill = _sig("hq_prefill_attn", _I, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P,
                 _SZ, _P)
@@ -196,9 +196,9 @@ def hq_decode_attn_static(q, cache: KVCache, B, Hq, Hkv, D, softmax_scale, out, 
                           _ptr(out), _ptr(lse_out), _stream(stream)), "hq_decode_attn_static")
 
 
-def hq_prefill_quant(q, k, B, Hq, Hkv, N, D, qi8, sq, ki8, sk, stream=None):
-    _check(_pquant(_ptr(q), _ptr(k), B, Hq, Hkv, N, D, _ptr(qi8), _ptr(sq), _ptr(ki8), _ptr(sk),
-                   _stream(stream)), "hq_prefill_quant")
+def hq_prefill_quant(q, k, idx, B, Hq, Hkv, N, D, k_vert, qi8, sq, ki8, sk, stream=None):
+    _check(_pquant(_ptr(q), _ptr(k), _ptr(idx), B, Hq, Hkv, N, D, k_vert, _ptr(qi8), _ptr(sq),
+                   _ptr(ki8), _ptr(sk), _stream(stream)), "hq_prefill_quant")
 
 
 def hq_prefill_attn(q, k, v, idx, B, Hq, Hkv, N, D, window, k_vert, softmax_scale, out, ws,
@@ -244,15 +244,18 @@ def decode_attn(q, cache: KVCache, Hkv, scale=0.0, ws=None, want_lse=False):
     return (out, lse) if want_lse else out
 
 
-def prefill_quant(q, k):
+def prefill_quant(q, k, idx):
+    """INT8 pre-pass: Q per row; K over the remaining (non-vertical) keys."""
     B, Hq, N, D = q.shape
     Hkv = k.shape[1]
-    nblk = (N + 63) // 64
+    k_vert = idx.shape[2]
+    nr = N - k_vert
+    nblk = (nr + 63) // 64
     qi8 = torch.empty(B, Hq, N, D, dtype=torch.int8, device=q.device)
     sq = torch.empty(B, Hq, N, dtype=torch.float32, device=q.device)
-    ki8 = torch.empty(B, Hkv, N, D, dtype=torch.int8, device=q.device)
+    ki8 = torch.empty(B, Hkv, nr, D, dtype=torch.int8, device=q.device)
     sk = torch.empty(B, Hkv, nblk, dtype=torch.float32, device=q.device)
-    hq_prefill_quant(q, k, B, Hq, Hkv, N, D, qi8, sq, ki8, sk)
+    hq_prefill_quant(q, k, idx, B, Hq, Hkv, N, D, k_vert, qi8, sq, ki8, sk)
     return qi8, sq, ki8, sk
 
 

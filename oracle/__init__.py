@@ -51,7 +51,7 @@ def _load():
         lib.hqo_quant_row.argtypes = [P, I, I, I, P, P]
         lib.hqo_pack_kv.argtypes = [P, P, P] + [I] * 8 + [P] * 7
         lib.hqo_decode_attn.argtypes = [P] * 7 + [I] * 8 + [D, P, P]
-        lib.hqo_prefill_quant.argtypes = [P, P] + [I] * 6 + [P] * 4
+        lib.hqo_prefill_quant.argtypes = [P, P, P] + [I] * 7 + [P] * 4
         lib.hqo_prefill_attn.argtypes = [P] * 8 + [I] * 8 + [D, P, I, P]
         lib.hqo_max_threads.argtypes = []
         for f in ("hqo_probe_scores", "hqo_topk", "hqo_quant_row", "hqo_pack_kv",
@@ -177,16 +177,22 @@ def decode_attn(q, cache: dict, Hkv: int, scale: float | None = None):
     return out, lse
 
 
-def prefill_quant(q, k, Hkv: int, kblock: int = 64):
-    """INT8 codes + fp32 scales: Q per token [B,Hq,N], K per kblock keys [B,Hkv,ceil(N/kblock)]."""
+def prefill_quant(q, k, idx, kblock: int = 64):
+    """INT8 codes + fp32 scales.  Q per token: qi8 [B,Hq,N,D], sq [B,Hq,N].
+    K over the remaining (non-vertical) keys in position order, one scale per
+    kblock of them: ki8 [B,Hkv,N-kv,D], sk [B,Hkv,ceil((N-kv)/kblock)]."""
     qq, kk = _u16(q), _u16(k)
     B, Hq, N, D = qq.shape
-    nblk = (N + kblock - 1) // kblock
+    Hkv = kk.shape[1]
+    idx = np.ascontiguousarray(idx, np.int32)
+    kv = idx.shape[2]
+    nr = N - kv
+    nblk = (nr + kblock - 1) // kblock
     qi8 = np.zeros((B, Hq, N, D), np.int8)
     sq = np.zeros((B, Hq, N), np.float32)
-    ki8 = np.zeros((B, Hkv, N, D), np.int8)
+    ki8 = np.zeros((B, Hkv, nr, D), np.int8)
     sk = np.zeros((B, Hkv, nblk), np.float32)
-    rc = _load().hqo_prefill_quant(_p(qq), _p(kk), B, Hq, Hkv, N, D, kblock,
+    rc = _load().hqo_prefill_quant(_p(qq), _p(kk), _p(idx), B, Hq, Hkv, N, D, kv, kblock,
                                    _p(qi8), _p(sq), _p(ki8), _p(sk))
     assert rc == 0, rc
     return qi8, sq, ki8, sk
@@ -201,7 +207,7 @@ def prefill_attn(q, k, v, idx, window: int, quant=None, rows=None, kblock: int =
     idx = np.ascontiguousarray(idx, np.int32)
     kv = idx.shape[2]
     if quant is None:
-        quant = prefill_quant(qq, kk, Hkv, kblock)
+        quant = prefill_quant(qq, kk, idx, kblock)
     qi8, sq, ki8, sk = (np.ascontiguousarray(a) for a in quant)
     r = None if rows is None else np.ascontiguousarray(rows, np.int32)
     nrows = N if r is None else int(r.shape[0])

@@ -434,15 +434,20 @@ int hqo_decode_attn(const uint16_t *q, const uint8_t *k_codes, const uint8_t *v_
 }
 
 /* ------------------------------------------------------------------------ */
-/* P4  Prefill pre-pass: symmetric INT8 codes for Q (per token) and K (per   */
-/*     block of 64 keys).                                                    */
+/* P4  Prefill pre-pass: symmetric INT8 codes for Q (per token) and for the  */
+/*     remaining (non-vertical) keys (per block of 64 of them).              */
 /* ------------------------------------------------------------------------ */
 /*
- * [W] TL;DR / [A]: during prefill the low part of attention runs at low
- * precision.  Readings taken: Q gets one scale per (batch, head, query row),
- * K one scale per (batch, KV head, block of `kblock` consecutive keys, all
- * keys of the block included).  These are integer decisions, so they are
- * taken in binary32, the precision of the kernel that also takes them:
+ * [W] TL;DR / [A]: during prefill the vertical-line tokens and the window stay
+ * in full precision and the remaining context is quantized ([B] "What
+ * hybrid-precision attention changes": the rest of the context in low
+ * precision).  Readings taken: Q gets one scale per (batch, head, query row).
+ * K: the keys that are not vertical-line columns, taken in position order
+ * (the "remaining" keys; window keys are among them, since every key is
+ * outside the window of later queries), get one scale per block of `kblock`
+ * consecutive such keys.  A vertical-line key is never quantized.
+ * These are integer decisions, so they are taken in binary32, the precision of
+ * the kernel that also takes them:
  *   amax = max |x| (exact);  s = fl32(amax / 127), s = 1 when amax == 0;
  *   c = clamp(rne(fl32(x / s)), -127, 127).
  * (A single rounded binary32 division, written with volatile to keep the
@@ -470,10 +475,17 @@ static int8_t q8_code(uint16_t xb, float s)
     return (int8_t)r;
 }
 
-int hqo_prefill_quant(const uint16_t *q, const uint16_t *k, int B, int Hq, int Hkv, int N,
-                      int D, int kblock, int8_t *qi8, float *sq, int8_t *ki8, float *sk)
+/*
+ * q: bf16 [B, Hq, N, D] -> qi8 [B, Hq, N, D], sq [B, Hq, N].
+ * k: bf16 [B, Hkv, N, D], idx [B, Hkv, kv] (ascending) ->
+ *    ki8 [B, Hkv, N - kv, D] (the remaining keys, compacted in position order),
+ *    sk  [B, Hkv, ceil((N - kv) / kblock)].
+ */
+int hqo_prefill_quant(const uint16_t *q, const uint16_t *k, const int32_t *idx, int B, int Hq,
+                      int Hkv, int N, int D, int kv, int kblock, int8_t *qi8, float *sq,
+                      int8_t *ki8, float *sk)
 {
-    if (B <= 0 || Hq <= 0 || Hkv <= 0 || N <= 0 || D <= 0 || kblock <= 0)
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || N <= 0 || D <= 0 || kblock <= 0 || kv < 0 || kv > N)
         return 1;
     const long long nq = (long long)B * Hq * N;
 #pragma omp parallel for schedule(static)
@@ -484,18 +496,32 @@ int hqo_prefill_quant(const uint16_t *q, const uint16_t *k, int B, int Hq, int H
         for (int d = 0; d < D; ++d)
             qi8[(size_t)r * D + d] = q8_code(x[d], s);
     }
-    const int nblk = (N + kblock - 1) / kblock;
-    const long long nk = (long long)B * Hkv * nblk;
-#pragma omp parallel for schedule(static)
-    for (long long r = 0; r < nk; ++r) {
-        const long long bh = r / nblk;
-        const int blk = (int)(r % nblk);
-        const int j0 = blk * kblock, n = (N - j0 < kblock ? N - j0 : kblock);
-        const uint16_t *x = k + ((size_t)bh * N + j0) * D;
-        float s = q8_scale(x, n * D);
-        sk[r] = s;
-        for (int e = 0; e < n * D; ++e)
-            ki8[((size_t)bh * N + j0) * D + e] = q8_code(x[e], s);
+    const int nr = N - kv;                        /* remaining keys per (b, kv head) */
+    const int nblk = (nr + kblock - 1) / kblock;
+    const long long nbh = (long long)B * Hkv;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long long bh = 0; bh < nbh; ++bh) {
+        const int32_t *id = idx + (size_t)bh * kv;
+        /* gather the remaining keys, in position order */
+        uint16_t *rem = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)nr * D);
+        int c = 0, vi = 0;
+        for (int j = 0; j < N; ++j) {
+            if (vi < kv && id[vi] == j) {
+                ++vi;
+                continue;
+            }
+            memcpy(rem + (size_t)c * D, k + ((size_t)bh * N + j) * D, sizeof(uint16_t) * D);
+            ++c;
+        }
+        for (int blk = 0; blk < nblk; ++blk) {
+            const int c0 = blk * kblock, n = (nr - c0 < kblock ? nr - c0 : kblock);
+            const uint16_t *x = rem + (size_t)c0 * D;
+            float s = q8_scale(x, n * D);
+            sk[(size_t)bh * nblk + blk] = s;
+            for (int e = 0; e < n * D; ++e)
+                ki8[((size_t)bh * nr + c0) * D + e] = q8_code(x[e], s);
+        }
+        free(rem);
     }
     return 0;
 }
@@ -510,8 +536,9 @@ int hqo_prefill_quant(const uint16_t *q, const uint16_t *k, int B, int Hq, int H
  * causal attention; for query i and key j <= i the pair is "high" when j is
  * in the window (j > i - W) or j is a vertical column, else "low".  A high
  * logit is q_i . k_j * scale from the bf16 values; a low logit is
- *   (sum_d qi8[i,d] * ki8[j,d]) * sq[i] * sk[j / kblock] * scale
- * with the integer dot product exact.  One exact softmax over all j <= i;
+ *   (sum_d qi8[i,d] * ki8[c,d]) * sq[i] * sk[c / kblock] * scale
+ * with the integer dot product exact, where c = j - #(vertical columns < j) is
+ * the key's rank among the remaining keys (see the pre-pass).  One exact softmax over all j <= i;
  * the output is sum_j p_ij v_j with v in bf16 and p unrounded.
  *
  * rows: the query rows to compute (nrows of them), or NULL for all N rows;
@@ -527,7 +554,7 @@ int hqo_prefill_attn(const uint16_t *q, const uint16_t *k, const uint16_t *v,
         return 1;
     if (!rows)
         nrows = N;
-    const int G = Hq / Hkv, nblk = (N + kblock - 1) / kblock;
+    const int G = Hq / Hkv, nr = N - kv, nblk = (nr + kblock - 1) / kblock;
     const long long nunits = (long long)B * Hq * nrows;
 #pragma omp parallel for schedule(dynamic, 4)
     for (long long u = 0; u < nunits; ++u) {
@@ -554,12 +581,13 @@ int hqo_prefill_attn(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                     acc += bf16_to_f64(qr[d]) * bf16_to_f64(kr[d]);
                 logit = acc * scale;
             } else {
-                const int8_t *kc = ki8 + (bh * N + j) * D;
+                const int c = j - vi;                  /* vi = #(vertical columns < j) */
+                const int8_t *kc = ki8 + (bh * nr + c) * D;
                 long long acc = 0;
                 for (int d = 0; d < D; ++d)
                     acc += (long long)qc[d] * (long long)kc[d];
                 logit = (double)acc * (double)sq[(size_t)bhq * N + i] *
-                        (double)sk[bh * nblk + j / kblock] * scale;
+                        (double)sk[bh * nblk + c / kblock] * scale;
             }
             s[j] = logit;
             if (logit > m) m = logit;

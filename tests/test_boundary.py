@@ -141,4 +141,6 @@ def test_probe_and_prefill_argument_checks(lib):
     assert pre(wsb=need - 1) == 3
     qq = lib.hq_prefill_quant
     qq.restype = ctypes.c_int
-    assert qq(FAKE, FAKE, 1, 4, 2, 256, 64, None, FAKE, FAKE, FAKE, None) == 1
+    assert qq(FAKE, FAKE, FAKE, 1, 4, 2, 256, 64, 12, None, FAKE, FAKE, FAKE, None) == 1
+    assert qq(FAKE, FAKE, None, 1, 4, 2, 256, 64, 12, FAKE, FAKE, FAKE, FAKE, None) == 1
+    assert qq(FAKE, FAKE, FAKE, 1, 4, 2, 256, 64, 300, FAKE, FAKE, FAKE, FAKE, None) == 1

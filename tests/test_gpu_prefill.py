@@ -39,11 +39,12 @@ def run_prefill_case(w: Workload, rows=None, check_probe=True):
         torch.cuda.synchronize()
         assert_index_sets(gidx.cpu().numpy(), ridx, rsc, w.window)
     # INT8 pre-pass: bit-exact
-    gq = [t.cpu().numpy() for t in H.prefill_quant(d["q"], d["k"])]
-    rq = oracle.prefill_quant(x["q"], x["k"], w.Hkv)
+    idx_d = torch.from_numpy(ridx).cuda()
+    gq = [t.cpu().numpy() for t in H.prefill_quant(d["q"], d["k"], idx_d)]
+    rq = oracle.prefill_quant(x["q"], x["k"], ridx)
     for g, r, name in zip(gq, rq, ("qi8", "sq", "ki8", "sk")):
         assert np.array_equal(g, r), f"{name} differs"
-    out = H.prefill_attn(d["q"], d["k"], d["v"], torch.from_numpy(ridx).cuda(), w.window)
+    out = H.prefill_attn(d["q"], d["k"], d["v"], idx_d, w.window)
     torch.cuda.synchronize()
     ref = oracle.prefill_attn(x["q"], x["k"], x["v"], ridx, w.window, quant=rq, rows=rows)
     g = out.cpu().numpy()

@@ -330,17 +330,21 @@ def test_decode_matches_dequantize_then_attend(bits):
 # --------------------------------------------------------------------------
 
 def test_prefill_quant_matches_numpy_float32():
-    B, Hq, Hkv, N, D = 1, 2, 1, 150, 64
+    B, Hq, Hkv, N, D = 1, 2, 1, 160, 64
     q = bf16(RNG.standard_normal((B, Hq, N, D)) * 3)
     k = bf16(RNG.standard_normal((B, Hkv, N, D)))
-    k[0, 0, 64:128] = 0                           # an all-zero block -> scale 1, codes 0
-    qi8, sq, ki8, sk = oracle.prefill_quant(q, k, Hkv, 64)
+    idx = np.array([[[2, 5, 70, 71, 100]]], np.int32)      # vertical columns (never quantized)
+    rem = np.setdiff1d(np.arange(N), idx[0, 0])             # remaining keys, position order
+    k[0, 0, rem[64:128]] = 0                                 # an all-zero block -> scale 1, codes 0
+    k[0, 0, 70] = 1000.0                                     # a huge vertical key must not widen any scale
+    qi8, sq, ki8, sk = oracle.prefill_quant(q, k, idx, 64)
+    assert ki8.shape == (B, Hkv, N - 5, D) and sk.shape == (B, Hkv, 3)
     qf = q.float().numpy()
     amax = np.abs(qf).max(-1)
     assert np.array_equal(sq, (amax / np.float32(127)).astype(np.float32))
     want = np.clip(np.rint(qf / sq[..., None]), -127, 127)
     assert np.array_equal(qi8, want.astype(np.int8))
-    kf = k.float().numpy()[0, 0]
+    kf = k.float().numpy()[0, 0][rem]
     for blk in range(3):
         seg = kf[64 * blk:64 * blk + 64]
         a = np.abs(seg).max()
@@ -349,6 +353,7 @@ def test_prefill_quant_matches_numpy_float32():
         assert np.array_equal(ki8[0, 0, 64 * blk:64 * blk + 64],
                               np.clip(np.rint(seg / s), -127, 127).astype(np.int8))
     assert np.abs(qi8).max() == 127 and sk[0, 0, 1] == 1 and not ki8[0, 0, 64:128].any()
+    assert sk.max() < 1000.0 / 127
 
 
 def test_prefill_all_high_precision_equals_causal_attention():
@@ -388,7 +393,7 @@ def test_prefill_mixed_pairs_follow_window_and_vertical_sets():
     k = bf16(RNG.standard_normal((B, Hkv, N, D)) * 2)
     v = bf16(RNG.standard_normal((B, Hkv, N, D)))
     idx = np.array([[[3, 50, 51, 120, 170]]], np.int32)
-    quant = oracle.prefill_quant(q, k, Hkv)
+    quant = oracle.prefill_quant(q, k, idx)
     qi8, sq, ki8, sk = quant
     rows = np.array([0, 1, 23, 24, 25, 50, 74, 75, 120, 143, 144, 145, 199], np.int32)
     out = oracle.prefill_attn(q, k, v, idx, W, quant=quant, rows=rows)
@@ -401,8 +406,9 @@ def test_prefill_mixed_pairs_follow_window_and_vertical_sets():
                 if i - j < W or j in vert:
                     logits[j] = float(f64(q[0, h, i]) @ f64(k[0, 0, j])) * sc
                 else:
-                    dot = int(np.dot(qi8[0, h, i].astype(np.int64), ki8[0, 0, j].astype(np.int64)))
-                    logits[j] = dot * float(sq[0, h, i]) * float(sk[0, 0, j // 64]) * sc
+                    c = j - int((idx[0, 0] < j).sum())   # rank among the remaining keys
+                    dot = int(np.dot(qi8[0, h, i].astype(np.int64), ki8[0, 0, c].astype(np.int64)))
+                    logits[j] = dot * float(sq[0, h, i]) * float(sk[0, 0, c // 64]) * sc
             p = torch.softmax(torch.from_numpy(logits), 0).numpy()
             ref = p @ f64(v[0, 0, :i + 1]).numpy()
             assert np.allclose(out[0, h, ri], ref, atol=1e-12), (h, i)
