@@ -44,7 +44,12 @@ namespace hq {
 namespace {
 
 constexpr int BM = 128, BN = 128, D = 128;
-constexpr int NWARP = 10, NT = NWARP * 32;
+// Two builds of the kernel: ONE_PASS (12 warps; the softmax warpgroups raise
+// their register budget with setmaxnreg and read each S row with a single
+// 128-column TMEM load) and the 10-warp fallback (two 64-column passes).
+constexpr int nwarps(bool one_pass) { return one_pass ? 12 : 10; }
+constexpr int kRegsLaunch = 168;        // 65536 / 384, what a 384-thread CTA starts with
+constexpr int kRegsLow = 56, kRegsHigh = 224;   // 128 * 56 + 256 * 224 == 384 * 168
 constexpr uint32_t SM_QI8 = 0;                 // [2 heads][128 rows x 128 B]
 constexpr uint32_t SM_QBF = 32768;             // [2 heads][2 boxes][128 rows x 128 B]
 constexpr uint32_t SM_KV = 98304;              // [2 stages][K 32 KB | V 32 KB]
@@ -111,7 +116,8 @@ __device__ __forceinline__ Sched make_sched(const TcArgs &a, int i0, size_t bh) 
   return s;
 }
 
-__global__ void __launch_bounds__(NT, 1)
+template <bool ONE_PASS>
+__global__ void __launch_bounds__(nwarps(ONE_PASS) * 32, 1)
 prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ CUtensorMap tm_qbf,
            const __grid_constant__ CUtensorMap tm_ki8, const __grid_constant__ CUtensorMap tm_kbf,
            const __grid_constant__ CUtensorMap tm_v16, const __grid_constant__ CUtensorMap tm_vk,
@@ -160,7 +166,12 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
+  constexpr int SM_WARP0 = ONE_PASS ? 4 : 2;       // first softmax warp
+  constexpr int NTHR = nwarps(ONE_PASS) * 32;
+  // Each role runs to its own end (named barrier 1, then return), so the code
+  // of the register-poor warps and of the softmax warps never merges again.
+  if (warp < SM_WARP0) {
+    if (ONE_PASS) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kRegsLow));
   if (warp == 0) {
     // ------------------------------ producer ------------------------------
     if (lane == 0) {
@@ -268,14 +279,27 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
       }
       tc_commit(o_final);
     }
-  } else {
+    }
+    tc_fence_before();
+    asm volatile("bar.sync 1, %0;\n" ::"r"(NTHR) : "memory");
+    if (warp == 1) {
+      tc_fence_after();
+      // every MMA has completed once o_final fired; wait for it (bounded) in
+      // case a softmax warp gave up before it did
+      if (!mbar_wait(o_final, 0)) raise_status(a.status, HQ_DEV_TIMEOUT);
+      tmem_dealloc(tmem, 512);
+    }
+    return;
+  }
+  if (ONE_PASS) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kRegsHigh));
+  {
     // ------------------------------ softmax ------------------------------
     // Two passes over the S row in tensor memory (64 columns at a time): the
     // row max first, then exp2 / row sum / fp16 packing of P, so that only a
     // half row is ever held in registers.  INT8 scores stay integers until
     // the exp: their max is an integer max, and s -> float is one add of the
     // bits of 2^23 + 2^22 (exact for |s| < 2^22) folded into the scaling FMA.
-    const int X = (warp - 2) >> 2;                 // 0: head A, 1: head B
+    const int X = (warp - SM_WARP0) >> 2;          // 0: head A, 1: head B
     const int hq = hA + X;
     const int quarter = warp & 3;                  // TMEM lanes 32*quarter ..
     const int r = quarter * 32 + lane;
@@ -334,23 +358,64 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
             if (h * 64 + e >= nvalid) x[e] = kNegInfBits;
         }
       };
-      // ---- pass 1: row max (log2 units) ----
-      float mt = -INFINITY;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t x[64];
-        tmem_ld64(tS + h * 64, x);
-        apply_masks(x, h);
+      // row max of one 64-column half (log2 units)
+      auto half_max = [&](uint32_t (&x)[64], int h) -> float {
         if (ty == IT_I8) {
-          int mx = (int)kMaskRaw;
+          int t8[8];                               // 8 independent chains, then a tree
 #pragma unroll
-          for (int e = 0; e < 64; ++e) mx = max(mx, (int)x[e]);
-          mt = fmaxf(mt, fmaf(__uint_as_float((uint32_t)mx + kMagicBits), scl[h], -kMagic * scl[h]));
+          for (int u = 0; u < 8; ++u) t8[u] = (int)x[u];
+#pragma unroll
+          for (int e = 8; e < 64; ++e) t8[e & 7] = max(t8[e & 7], (int)x[e]);
+          const int mx = max(max(max(t8[0], t8[1]), max(t8[2], t8[3])),
+                             max(max(t8[4], t8[5]), max(t8[6], t8[7])));
+          return fmaf(__uint_as_float((uint32_t)mx + kMagicBits), scl[h], -kMagic * scl[h]);
+        }
+        float t8[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) t8[u] = __uint_as_float(x[u]);
+#pragma unroll
+        for (int e = 8; e < 64; ++e) t8[e & 7] = fmaxf(t8[e & 7], __uint_as_float(x[e]));
+        const float mx = fmaxf(fmaxf(fmaxf(t8[0], t8[1]), fmaxf(t8[2], t8[3])),
+                               fmaxf(fmaxf(t8[4], t8[5]), fmaxf(t8[6], t8[7])));
+        return mx * a.sl;
+      };
+      // P = exp2(x - m) of one half, packed fp16 pairs, with partial row sums
+      auto half_exp = [&](uint32_t (&x)[64], int h, uint32_t (&pk)[32], float (&rs4)[4]) {
+        if (ty == IT_I8) {
+          const float sc_ = scl[h], c_ = -kMagic * scl[h] - m;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float p0 = fast_exp2(fmaf(__uint_as_float(x[2 * e] + kMagicBits), sc_, c_));
+            const float p1 = fast_exp2(fmaf(__uint_as_float(x[2 * e + 1] + kMagicBits), sc_, c_));
+            rs4[e & 3] += p0 + p1;
+            pk[e] = pack_f16x2(p0, p1);
+          }
         } else {
-          float mx = -INFINITY;
+          const float c_ = -m;
 #pragma unroll
-          for (int e = 0; e < 64; ++e) mx = fmaxf(mx, __uint_as_float(x[e]));
-          mt = fmaxf(mt, mx * a.sl);
+          for (int e = 0; e < 32; ++e) {
+            const float p0 = fast_exp2(fmaf(__uint_as_float(x[2 * e]), a.sl, c_));
+            const float p1 = fast_exp2(fmaf(__uint_as_float(x[2 * e + 1]), a.sl, c_));
+            rs4[e & 3] += p0 + p1;
+            pk[e] = pack_f16x2(p0, p1);
+          }
+        }
+      };
+      // ---- row max ----
+      float mt = -INFINITY;
+      uint32_t xa0[ONE_PASS ? 64 : 1], xa1[ONE_PASS ? 64 : 1];
+      if constexpr (ONE_PASS) {
+        tmem_ld64x2(tS, xa0, xa1);                  // the whole S row, one wait
+        apply_masks(xa0, 0);
+        apply_masks(xa1, 1);
+        mt = fmaxf(half_max(xa0, 0), half_max(xa1, 1));
+      } else {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t x[64];
+          tmem_ld64(tS + h * 64, x);
+          apply_masks(x, h);
+          mt = fmaxf(mt, half_max(x, h));
         }
       }
       // ---- lazy rescale of the running max (and of O: the commit this
@@ -373,36 +438,39 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
           tmem_wait_st();
         }
       }
-      // ---- pass 2: P = exp2(x - m) as packed fp16 into the first 64 columns ----
-      float rs = 0.f;
+      // ---- P = exp2(x - m) as packed fp16 into the first 64 columns ----
+      float rs4[4] = {0.f, 0.f, 0.f, 0.f};           // independent partial row sums
+      if constexpr (ONE_PASS) {
+        // 16 packed pairs (32 keys) at a time, stored as soon as they are made
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t x[64];
-        tmem_ld64(tS + h * 64, x);
-        apply_masks(x, h);
-        uint32_t pk[32];
-        if (ty == IT_I8) {
-          const float sc_ = scl[h], c_ = -kMagic * scl[h] - m;
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint32_t(&xh)[64] = (q4 < 2) ? xa0 : xa1;
+          const int h = q4 >> 1, base = (q4 & 1) * 32;
+          uint32_t pk[16];
+          const float sc_ = ty == IT_I8 ? scl[h] : a.sl;
+          const float c_ = ty == IT_I8 ? -kMagic * scl[h] - m : -m;
+          const uint32_t add = ty == IT_I8 ? kMagicBits : 0u;
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float p0 = fast_exp2(fmaf(__uint_as_float(x[2 * e] + kMagicBits), sc_, c_));
-            const float p1 = fast_exp2(fmaf(__uint_as_float(x[2 * e + 1] + kMagicBits), sc_, c_));
-            rs += p0 + p1;
+          for (int e = 0; e < 16; ++e) {
+            const float p0 = fast_exp2(fmaf(__uint_as_float(xh[base + 2 * e] + add), sc_, c_));
+            const float p1 = fast_exp2(fmaf(__uint_as_float(xh[base + 2 * e + 1] + add), sc_, c_));
+            rs4[e & 3] += p0 + p1;
             pk[e] = pack_f16x2(p0, p1);
           }
-        } else {
-          const float c_ = -m;
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float p0 = fast_exp2(fmaf(__uint_as_float(x[2 * e]), a.sl, c_));
-            const float p1 = fast_exp2(fmaf(__uint_as_float(x[2 * e + 1]), a.sl, c_));
-            rs += p0 + p1;
-            pk[e] = pack_f16x2(p0, p1);
-          }
+          tmem_st16(tS + q4 * 16, pk);              // keys 32*q4 .. 32*q4+31
         }
-        tmem_st32(tS + h * 32, pk);                 // keys 64h .. 64h+63
+      } else {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pk[32];
+          uint32_t x[64];
+          tmem_ld64(tS + h * 64, x);
+          apply_masks(x, h);
+          half_exp(x, h, pk, rs4);
+          tmem_st32(tS + h * 32, pk);               // keys 64h .. 64h+63
+        }
       }
-      l += rs;
+      l += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[X]);
@@ -428,14 +496,7 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
     }
   }
   tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    // every MMA has completed once o_final fired; wait for it (bounded) in case
-    // a softmax warp gave up before it did
-    if (!mbar_wait(o_final, 0)) raise_status(a.status, HQ_DEV_TIMEOUT);
-    tmem_dealloc(tmem, 512);
-  }
+  asm volatile("bar.sync 1, %0;\n" ::"r"(NTHR) : "memory");
 }
 
 }  // namespace
@@ -445,11 +506,18 @@ bool prefill_tc_supported(int D_, int Hq, int Hkv) {
 }
 
 cudaError_t launch_prefill_tc(const TcLaunch &p, cudaStream_t s) {
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(prefill_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
+  // The one-pass build redistributes registers with setmaxnreg; that is only
+  // valid when the CTA starts with exactly kRegsLaunch registers per thread
+  // (checked once from the compiled kernel), else the 10-warp build is used.
+  static int mode = -1;                     // 1: one pass, 0: two passes
+  if (mode < 0) {
+    cudaFuncAttributes fa;
+    const bool one = cudaFuncGetAttributes(&fa, prefill_tc<true>) == cudaSuccess &&
+                     fa.numRegs == kRegsLaunch;
+    const auto kern = one ? prefill_tc<true> : prefill_tc<false>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
       return cudaErrorInvalidValue;
-    attr = true;
+    mode = one ? 1 : 0;
   }
   const int nbq = p.B * p.Hq, nbh = p.B * p.Hkv;
   const int nr = p.N - p.k_vert;                      // remaining keys per (b, kv head)
@@ -478,7 +546,10 @@ cudaError_t launch_prefill_tc(const TcLaunch &p, cudaStream_t s) {
   a.nblk_r = p.nblk_r;
   a.sl = p.scale * kLog2e;
   dim3 grid((p.N + BM - 1) / BM, p.Hq / 2, p.B);
-  prefill_tc<<<grid, NT, SMEM_BYTES, s>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7], a);
+  if (mode == 1)
+    prefill_tc<true><<<grid, nwarps(true) * 32, SMEM_BYTES, s>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7], a);
+  else
+    prefill_tc<false><<<grid, nwarps(false) * 32, SMEM_BYTES, s>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7], a);
   return cudaGetLastError();
 }
 
