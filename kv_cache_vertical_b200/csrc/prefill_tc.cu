@@ -44,12 +44,11 @@ namespace hq {
 namespace {
 
 constexpr int BM = 128, BN = 128, D = 128;
-// Two builds of the kernel: ONE_PASS (12 warps; the softmax warpgroups raise
-// their register budget with setmaxnreg and read each S row with a single
-// 128-column TMEM load) and the 10-warp fallback (two 64-column passes).
-constexpr int nwarps(bool one_pass) { return one_pass ? 12 : 10; }
-constexpr int kRegsLaunch = 168;        // 65536 / 384, what a 384-thread CTA starts with
+constexpr int NWARPS = 12, NTHR = NWARPS * 32;
+constexpr int SM_WARP0 = 4;                     // warps 4-7: head A, 8-11: head B
+constexpr int kRegsLaunch = 168;                // 65536 / 384, what a 384-thread CTA starts with
 constexpr int kRegsLow = 56, kRegsHigh = 224;   // 128 * 56 + 256 * 224 == 384 * 168
+constexpr int NCHUNK = 4;                       // P handed to the MMA in 32-key chunks
 constexpr uint32_t SM_QI8 = 0;                 // [2 heads][128 rows x 128 B]
 constexpr uint32_t SM_QBF = 32768;             // [2 heads][2 boxes][128 rows x 128 B]
 constexpr uint32_t SM_KV = 98304;              // [2 stages][K 32 KB | V 32 KB]
@@ -72,6 +71,55 @@ enum { IT_I8 = 0, IT_WIN = 1, IT_VERT = 2 };
 // bits of 2^23 + 2^22 it is the bit pattern of -inf.
 constexpr uint32_t kMaskRaw = 0xFF800000u - kMagicBits;
 constexpr uint32_t kNegInfBits = 0xFF800000u;
+
+// Paired fp32 arithmetic (one instruction for two lanes of work).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n .reg .b64 ra, rb, rc, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n"
+      " mov.b64 rc, {%6, %7};\n fma.rn.f32x2 rd, ra, rb, rc;\n mov.b64 {%0, %1}, rd;\n}\n"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n .reg .b64 ra, rb, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n"
+      " add.rn.f32x2 rd, ra, rb;\n mov.b64 {%0, %1}, rd;\n}\n"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;\n" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// Max of 64 floats given as bits: 21 three-input maxes in 4 independent chains.
+__device__ __forceinline__ float max64(const uint32_t (&x)[64]) {
+  float c[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) c[u] = fmax3(__uint_as_float(x[u]), __uint_as_float(x[4 + u]), __uint_as_float(x[8 + u]));
+#pragma unroll
+  for (int e = 12; e + 8 <= 64; e += 8) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (e + u + 4 < 64) c[u] = fmax3(c[u], __uint_as_float(x[e + u]), __uint_as_float(x[e + u + 4]));
+  }
+  // e = 12, 20, ..., 52 covers 12..59; the last four are 60..63
+#pragma unroll
+  for (int u = 0; u < 4; ++u) c[u] = fmaxf(c[u], __uint_as_float(x[60 + u]));
+  return fmax3(fmaxf(c[0], c[1]), c[2], c[3]);
+}
+
+// Max of 64 signed ints: 8 independent chains, then a tree.
+__device__ __forceinline__ int imax64(const uint32_t (&x)[64]) {
+  int c[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) c[u] = (int)x[u];
+#pragma unroll
+  for (int e = 8; e < 64; ++e) c[e & 7] = max(c[e & 7], (int)x[e]);
+  return max(max(max(c[0], c[1]), max(c[2], c[3])), max(max(c[4], c[5]), max(c[6], c[7])));
+}
 
 struct TcArgs {
   const float *sq;                    // [B*Hq, N]
@@ -116,8 +164,7 @@ __device__ __forceinline__ Sched make_sched(const TcArgs &a, int i0, size_t bh) 
   return s;
 }
 
-template <bool ONE_PASS>
-__global__ void __launch_bounds__(nwarps(ONE_PASS) * 32, 1)
+__global__ void __launch_bounds__(NTHR, 1)
 prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ CUtensorMap tm_qbf,
            const __grid_constant__ CUtensorMap tm_ki8, const __grid_constant__ CUtensorMap tm_kbf,
            const __grid_constant__ CUtensorMap tm_v16, const __grid_constant__ CUtensorMap tm_vk,
@@ -130,10 +177,10 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
   uint64_t *kv_full = bar + 1;   // [2]
   uint64_t *kv_free = bar + 3;   // [2]
   uint64_t *s_full = bar + 5;    // [2 heads]
-  uint64_t *p_full = bar + 7;    // [2 heads]
-  uint64_t *o_final = bar + 9;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 10);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(bar + 11);
+  uint64_t *p_full = bar + 7;    // [2 heads][NCHUNK], one arrival per softmax warp
+  uint64_t *o_final = bar + 15;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 16);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(bar + 17);
 
   const int ntq = (a.N + BM - 1) / BM;
   const int qt = ntq - 1 - (int)blockIdx.x;      // longest rows first
@@ -152,8 +199,8 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_free[s], 1);
       mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], 128);
     }
+    for (int s = 0; s < 2 * NCHUNK; ++s) mbar_init(&p_full[s], 4);
     mbar_init(o_final, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -166,12 +213,10 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  constexpr int SM_WARP0 = ONE_PASS ? 4 : 2;       // first softmax warp
-  constexpr int NTHR = nwarps(ONE_PASS) * 32;
   // Each role runs to its own end (named barrier 1, then return), so the code
   // of the register-poor warps and of the softmax warps never merges again.
   if (warp < SM_WARP0) {
-    if (ONE_PASS) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kRegsLow));
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kRegsLow));
   if (warp == 0) {
     // ------------------------------ producer ------------------------------
     if (lane == 0) {
@@ -210,12 +255,17 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
         tma_load_3d(vs + 16384, vm, &kv_full[s], 64, row, (int)bh);
         issued = it + 1;
       }
+      // do not leave with copies in flight
       if (!mbar_wait(q_full, 0)) raise_status(a.status, HQ_DEV_TIMEOUT);
       for (int it = issued > 2 ? issued - 2 : 0; it < issued; ++it)
         if (!mbar_wait(&kv_full[it & 1], (it >> 1) & 1)) raise_status(a.status, HQ_DEV_TIMEOUT);
     }
   } else if (warp == 1) {
     // ------------------------------ MMA issuer ------------------------------
+    // Order per tile t: P.V of head A chunk by chunk as its softmax hands the
+    // chunks over, QK of head A for tile t + 1, the same for head B, so one
+    // head's softmax overlaps the other head's tensor-core work and most of a
+    // head's own P.V overlaps the end of its exp phase.
     if (lane == 0) {
       const uint32_t sQi8 = smem_u32(smem + SM_QI8), sQbf = smem_u32(smem + SM_QBF);
       const uint32_t sKV = smem_u32(smem + SM_KV);
@@ -241,14 +291,22 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
         }
         tc_commit(&s_full[x]);
       };
-      auto issue_pv = [&](int x, int it) {
+      // P.V of head x, tile it, as each 32-key chunk of P arrives
+      auto issue_pv = [&](int x, int it) -> bool {
         const uint32_t vslot = sKV + (it & 1) * KV_STAGE + 32768;
         const uint32_t dt = tmem + x * 256 + 128, at = tmem + x * 256;
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint64_t bd = make_sdesc_sw128(vslot + ks * 2048, 16384, 1024);
-          mma_f16_ts(dt, at + ks * 8, bd, IDESC_PV, (it > 0 || ks > 0) ? 1u : 0u);
+        for (int c = 0; c < NCHUNK; ++c) {
+          if (!mbar_wait(&p_full[x * NCHUNK + c], it & 1)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int ks = 2 * c + j;
+            const uint64_t bd = make_sdesc_sw128(vslot + ks * 2048, 16384, 1024);
+            mma_f16_ts(dt, at + ks * 8, bd, IDESC_PV, (it > 0 || ks > 0) ? 1u : 0u);
+          }
         }
+        return true;
       };
       if (ok && sc.n > 0) {
         ok = mbar_wait(&kv_full[0], 0);
@@ -259,17 +317,13 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
         }
       }
       for (int it = 0; ok && it < sc.n; ++it) {
-        if (!(ok = mbar_wait(&p_full[0], it & 1))) break;
-        tc_fence_after();
-        issue_pv(0, it);
+        if (!(ok = issue_pv(0, it))) break;
         if (it + 1 < sc.n) {
           if (!(ok = mbar_wait(&kv_full[(it + 1) & 1], ((it + 1) >> 1) & 1))) break;
           tc_fence_after();
           issue_qk(0, it + 1);
         }
-        if (!(ok = mbar_wait(&p_full[1], it & 1))) break;
-        tc_fence_after();
-        issue_pv(1, it);
+        if (!(ok = issue_pv(1, it))) break;
         tc_commit(&kv_free[it & 1]);
         if (it + 1 < sc.n) issue_qk(1, it + 1);
       }
@@ -279,7 +333,7 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
       }
       tc_commit(o_final);
     }
-    }
+  }
     tc_fence_before();
     asm volatile("bar.sync 1, %0;\n" ::"r"(NTHR) : "memory");
     if (warp == 1) {
@@ -291,14 +345,14 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
     }
     return;
   }
-  if (ONE_PASS) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kRegsHigh));
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kRegsHigh));
   {
     // ------------------------------ softmax ------------------------------
-    // Two passes over the S row in tensor memory (64 columns at a time): the
-    // row max first, then exp2 / row sum / fp16 packing of P, so that only a
-    // half row is ever held in registers.  INT8 scores stay integers until
-    // the exp: their max is an integer max, and s -> float is one add of the
-    // bits of 2^23 + 2^22 (exact for |s| < 2^22) folded into the scaling FMA.
+    // One thread per query row (TMEM lane), the whole 128-key S row in
+    // registers.  INT8 scores stay integers until the exp: their row max is an
+    // integer max, and adding the bits of 2^23 + 2^22 turns s into the float
+    // 2^23 + 2^22 + s (exact for |s| < 2^22), whose offset is folded into the
+    // scaling FMA.
     const int X = (warp - SM_WARP0) >> 2;          // 0: head A, 1: head B
     const int hq = hA + X;
     const int quarter = warp & 3;                  // TMEM lanes 32*quarter ..
@@ -314,9 +368,25 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
     const int cnt_i = remaining_upto(id, a.k_vert, lim);        // low-bit keys of this row
     const int cnt_lo = remaining_upto(id, a.k_vert, i0 - W);     // ... of the tile's first row
     const int nvert = lim >= 0 ? upper_bound_i32(id, a.k_vert, lim) : 0;
-    float m = -1e30f, l = 0.f;
+    const float *skp = a.sk + bh * a.nblk_r;
+    // K scales of an INT8 tile (two 64-key blocks), fetched one tile ahead
+    auto fetch_scales = [&](int it, float (&k2)[2]) {
+      k2[0] = k2[1] = 1.f;
+      if (it < sc.n && sc.type(it) == IT_I8) {
+        const int t = sc.tile(it);
+        if (2 * t < a.nblk_r) k2[0] = __ldg(skp + 2 * t);
+        if (2 * t + 1 < a.nblk_r) k2[1] = __ldg(skp + 2 * t + 1);
+      }
+    };
+    float kn[2];
+    fetch_scales(0, kn);
+    float m = -1e30f;
+    float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                     make_float2(0.f, 0.f)};       // independent partial row sums
     bool ok = true;
     for (int it = 0; it < sc.n; ++it) {
+      const float k0 = kn[0], k1 = kn[1];
+      fetch_scales(it + 1, kn);
       if (!mbar_wait(&s_full[X], it & 1)) {
         ok = false;
         break;
@@ -324,99 +394,45 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
       tc_fence_after();
       const int ty = sc.type(it), t = sc.tile(it);
       const int j0 = t * BN;
-      float scl[2] = {0.f, 0.f};
-      bool need_lim = false;
-      int nvalid = BN;
+      uint32_t xa0[64], xa1[64];
+      tmem_ld64x2(tS, xa0, xa1);                    // the whole S row, one wait
+      float sc0, sc1, c0, c1, mt;                   // per-half scale and offset (log2 units)
+      uint32_t add = 0u;                            // bits added to a raw score before the FMA
       if (ty == IT_I8) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int blk = 2 * t + h;
-          scl[h] = sqi * (blk < a.nblk_r ? __ldg(a.sk + bh * a.nblk_r + blk) : 1.f);
-        }
-        need_lim = j0 + BN > cnt_lo;               // same for every row of the tile
-        nvalid = cnt_i - j0;
-      } else if (ty == IT_VERT) {
-        nvalid = nvert - j0;
-      }
-      auto apply_masks = [&](uint32_t (&x)[64], int h) {
-        if (ty == IT_I8) {
-          if (need_lim) {
-#pragma unroll
-            for (int e = 0; e < 64; ++e)
-              if (h * 64 + e >= nvalid) x[e] = kMaskRaw;
-          }
-        } else if (ty == IT_WIN) {
-          const int jh = j0 + h * 64;
+        sc0 = sqi * k0;
+        sc1 = sqi * k1;
+        if (j0 + BN > cnt_lo) {                     // same for every row of the tile
+          const int nvalid = cnt_i - j0;
 #pragma unroll
           for (int e = 0; e < 64; ++e) {
-            const int j = jh + e;
-            if (j > i || j <= lim) x[e] = kNegInfBits;
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 64; ++e)
-            if (h * 64 + e >= nvalid) x[e] = kNegInfBits;
-        }
-      };
-      // row max of one 64-column half (log2 units)
-      auto half_max = [&](uint32_t (&x)[64], int h) -> float {
-        if (ty == IT_I8) {
-          int t8[8];                               // 8 independent chains, then a tree
-#pragma unroll
-          for (int u = 0; u < 8; ++u) t8[u] = (int)x[u];
-#pragma unroll
-          for (int e = 8; e < 64; ++e) t8[e & 7] = max(t8[e & 7], (int)x[e]);
-          const int mx = max(max(max(t8[0], t8[1]), max(t8[2], t8[3])),
-                             max(max(t8[4], t8[5]), max(t8[6], t8[7])));
-          return fmaf(__uint_as_float((uint32_t)mx + kMagicBits), scl[h], -kMagic * scl[h]);
-        }
-        float t8[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) t8[u] = __uint_as_float(x[u]);
-#pragma unroll
-        for (int e = 8; e < 64; ++e) t8[e & 7] = fmaxf(t8[e & 7], __uint_as_float(x[e]));
-        const float mx = fmaxf(fmaxf(fmaxf(t8[0], t8[1]), fmaxf(t8[2], t8[3])),
-                               fmaxf(fmaxf(t8[4], t8[5]), fmaxf(t8[6], t8[7])));
-        return mx * a.sl;
-      };
-      // P = exp2(x - m) of one half, packed fp16 pairs, with partial row sums
-      auto half_exp = [&](uint32_t (&x)[64], int h, uint32_t (&pk)[32], float (&rs4)[4]) {
-        if (ty == IT_I8) {
-          const float sc_ = scl[h], c_ = -kMagic * scl[h] - m;
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float p0 = fast_exp2(fmaf(__uint_as_float(x[2 * e] + kMagicBits), sc_, c_));
-            const float p1 = fast_exp2(fmaf(__uint_as_float(x[2 * e + 1] + kMagicBits), sc_, c_));
-            rs4[e & 3] += p0 + p1;
-            pk[e] = pack_f16x2(p0, p1);
-          }
-        } else {
-          const float c_ = -m;
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float p0 = fast_exp2(fmaf(__uint_as_float(x[2 * e]), a.sl, c_));
-            const float p1 = fast_exp2(fmaf(__uint_as_float(x[2 * e + 1]), a.sl, c_));
-            rs4[e & 3] += p0 + p1;
-            pk[e] = pack_f16x2(p0, p1);
+            if (e >= nvalid) xa0[e] = kMaskRaw;
+            if (64 + e >= nvalid) xa1[e] = kMaskRaw;
           }
         }
-      };
-      // ---- row max ----
-      float mt = -INFINITY;
-      uint32_t xa0[ONE_PASS ? 64 : 1], xa1[ONE_PASS ? 64 : 1];
-      if constexpr (ONE_PASS) {
-        tmem_ld64x2(tS, xa0, xa1);                  // the whole S row, one wait
-        apply_masks(xa0, 0);
-        apply_masks(xa1, 1);
-        mt = fmaxf(half_max(xa0, 0), half_max(xa1, 1));
+        c0 = -kMagic * sc0;
+        c1 = -kMagic * sc1;
+        add = kMagicBits;
+        mt = fmaxf(fmaf(__uint_as_float((uint32_t)imax64(xa0) + kMagicBits), sc0, c0),
+                   fmaf(__uint_as_float((uint32_t)imax64(xa1) + kMagicBits), sc1, c1));
       } else {
+        sc0 = sc1 = a.sl;
+        c0 = c1 = 0.f;
+        if (ty == IT_WIN) {
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t x[64];
-          tmem_ld64(tS + h * 64, x);
-          apply_masks(x, h);
-          mt = fmaxf(mt, half_max(x, h));
+          for (int e = 0; e < 64; ++e) {
+            const int j = j0 + e;
+            if (j > i || j <= lim) xa0[e] = kNegInfBits;
+            if (j + 64 > i || j + 64 <= lim) xa1[e] = kNegInfBits;
+          }
+        } else {
+          const int nvalid = nvert - j0;
+#pragma unroll
+          for (int e = 0; e < 64; ++e) {
+            if (e >= nvalid) xa0[e] = kNegInfBits;
+            if (64 + e >= nvalid) xa1[e] = kNegInfBits;
+          }
         }
+        mt = fmaxf(max64(xa0), max64(xa1)) * a.sl;
       }
       // ---- lazy rescale of the running max (and of O: the commit this
       // thread waited on covers every MMA issued before it) ----
@@ -425,7 +441,8 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
         const float mn = fmaxf(m, mt);
         const float al = exp2f(m - mn);
         m = mn;
-        l *= al;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) acc[u] = make_float2(acc[u].x * al, acc[u].y * al);
         if (it > 0) {
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch) {
@@ -435,46 +452,43 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
             for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * al);
             tmem_st32(tO + ch * 32, o);
           }
+        }
+      }
+      // ---- P = exp2(x * scale + offset - m) as packed fp16, 32 keys per
+      // chunk, each chunk handed to the MMA as soon as it is in TMEM ----
+      c0 -= m;
+      c1 -= m;
+#pragma unroll
+      for (int q4 = 0; q4 < NCHUNK; ++q4) {
+        uint32_t(&xh)[64] = (q4 < 2) ? xa0 : xa1;
+        const int base = (q4 & 1) * 32;
+        const float2 s2 = q4 < 2 ? make_float2(sc0, sc0) : make_float2(sc1, sc1);
+        const float2 o2 = q4 < 2 ? make_float2(c0, c0) : make_float2(c1, c1);
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float2 y = ffma2(make_float2(__uint_as_float(xh[base + 2 * e] + add),
+                                             __uint_as_float(xh[base + 2 * e + 1] + add)), s2, o2);
+          const float2 p = make_float2(fast_exp2(y.x), fast_exp2(y.y));
+          acc[e & 3] = fadd2(acc[e & 3], p);
+          pk[e] = pack_f16x2(p.x, p.y);
+        }
+        // hand over the previous chunk (its store has had this chunk's exps
+        // to complete), then store this one
+        if (q4 > 0) {
           tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&p_full[X * NCHUNK + q4 - 1]);
         }
+        tmem_st16(tS + q4 * 16, pk);              // keys 32*q4 .. 32*q4+31
       }
-      // ---- P = exp2(x - m) as packed fp16 into the first 64 columns ----
-      float rs4[4] = {0.f, 0.f, 0.f, 0.f};           // independent partial row sums
-      if constexpr (ONE_PASS) {
-        // 16 packed pairs (32 keys) at a time, stored as soon as they are made
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          uint32_t(&xh)[64] = (q4 < 2) ? xa0 : xa1;
-          const int h = q4 >> 1, base = (q4 & 1) * 32;
-          uint32_t pk[16];
-          const float sc_ = ty == IT_I8 ? scl[h] : a.sl;
-          const float c_ = ty == IT_I8 ? -kMagic * scl[h] - m : -m;
-          const uint32_t add = ty == IT_I8 ? kMagicBits : 0u;
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float p0 = fast_exp2(fmaf(__uint_as_float(xh[base + 2 * e] + add), sc_, c_));
-            const float p1 = fast_exp2(fmaf(__uint_as_float(xh[base + 2 * e + 1] + add), sc_, c_));
-            rs4[e & 3] += p0 + p1;
-            pk[e] = pack_f16x2(p0, p1);
-          }
-          tmem_st16(tS + q4 * 16, pk);              // keys 32*q4 .. 32*q4+31
-        }
-      } else {
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t pk[32];
-          uint32_t x[64];
-          tmem_ld64(tS + h * 64, x);
-          apply_masks(x, h);
-          half_exp(x, h, pk, rs4);
-          tmem_st32(tS + h * 32, pk);               // keys 64h .. 64h+63
-        }
-      }
-      l += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&p_full[X]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[X * NCHUNK + NCHUNK - 1]);
     }
+    const float l = (acc[0].x + acc[0].y + acc[1].x + acc[1].y) + (acc[2].x + acc[2].y + acc[3].x + acc[3].y);
     if (ok) ok = mbar_wait(o_final, 0);
     if (!ok) {
       *abort_flag = 1;
@@ -501,24 +515,26 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
 
 }  // namespace
 
+// The kernel redistributes registers with setmaxnreg, which is only valid
+// when the CTA starts with exactly kRegsLaunch registers per thread; that is
+// checked once from the compiled kernel (else the CUDA-core kernel is used).
+static bool prefill_tc_ready() {
+  static int ready = -1;
+  if (ready < 0) {
+    cudaFuncAttributes fa;
+    ready = cudaFuncGetAttributes(&fa, prefill_tc) == cudaSuccess && fa.numRegs == kRegsLaunch &&
+            cudaFuncSetAttribute(prefill_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 SMEM_BYTES) == cudaSuccess;
+  }
+  return ready == 1;
+}
+
 bool prefill_tc_supported(int D_, int Hq, int Hkv) {
-  return D_ == 128 && Hq % Hkv == 0 && (Hq / Hkv) % 2 == 0;
+  return D_ == 128 && Hq % Hkv == 0 && (Hq / Hkv) % 2 == 0 && prefill_tc_ready();
 }
 
 cudaError_t launch_prefill_tc(const TcLaunch &p, cudaStream_t s) {
-  // The one-pass build redistributes registers with setmaxnreg; that is only
-  // valid when the CTA starts with exactly kRegsLaunch registers per thread
-  // (checked once from the compiled kernel), else the 10-warp build is used.
-  static int mode = -1;                     // 1: one pass, 0: two passes
-  if (mode < 0) {
-    cudaFuncAttributes fa;
-    const bool one = cudaFuncGetAttributes(&fa, prefill_tc<true>) == cudaSuccess &&
-                     fa.numRegs == kRegsLaunch;
-    const auto kern = one ? prefill_tc<true> : prefill_tc<false>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
-      return cudaErrorInvalidValue;
-    mode = one ? 1 : 0;
-  }
+  if (!prefill_tc_ready()) return cudaErrorInvalidValue;
   const int nbq = p.B * p.Hq, nbh = p.B * p.Hkv;
   const int nr = p.N - p.k_vert;                      // remaining keys per (b, kv head)
   CUtensorMap m[8];
@@ -546,10 +562,7 @@ cudaError_t launch_prefill_tc(const TcLaunch &p, cudaStream_t s) {
   a.nblk_r = p.nblk_r;
   a.sl = p.scale * kLog2e;
   dim3 grid((p.N + BM - 1) / BM, p.Hq / 2, p.B);
-  if (mode == 1)
-    prefill_tc<true><<<grid, nwarps(true) * 32, SMEM_BYTES, s>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7], a);
-  else
-    prefill_tc<false><<<grid, nwarps(false) * 32, SMEM_BYTES, s>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7], a);
+  prefill_tc<<<grid, NTHR, SMEM_BYTES, s>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7], a);
   return cudaGetLastError();
 }
 
