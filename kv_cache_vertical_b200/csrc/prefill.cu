@@ -156,15 +156,20 @@ __global__ void v_prep(const __nv_bfloat16 *__restrict__ v, const int32_t *__res
 }
 
 // Compact copies of the vertical rows (padded to whole 128-row tiles with zero
-// rows at position INT_MAX).
+// rows at position INT_MAX).  Also checks the index list: strictly ascending,
+// every column in [0, N - window); a violation sets HQ_DEV_BAD_INDEX (the
+// attention that follows stays in bounds but its result is meaningless).
 template <int D>
 __global__ void gather_vertical(const __nv_bfloat16 *__restrict__ k, const __half *__restrict__ vh,
-                                const int32_t *__restrict__ idx, int N, int k_vert, int kpad,
-                                __nv_bfloat16 *__restrict__ kv_k, __half *__restrict__ kv_v,
-                                int32_t *__restrict__ kv_pos) {
+                                const int32_t *__restrict__ idx, int N, int window, int k_vert,
+                                int kpad, __nv_bfloat16 *__restrict__ kv_k, __half *__restrict__ kv_v,
+                                int32_t *__restrict__ kv_pos, uint32_t *status) {
   const int r = blockIdx.x, bh = blockIdx.y;  // one CTA (D/8 threads) per padded row
   const int t = threadIdx.x;                  // 16-byte chunk of the row
   const int pos = r < k_vert ? idx[(size_t)bh * k_vert + r] : INT_MAX;
+  if (t == 0 && r < k_vert &&
+      (pos < 0 || pos >= N - window || (r > 0 && idx[(size_t)bh * k_vert + r - 1] >= pos)))
+    raise_status(status, HQ_DEV_BAD_INDEX);
   const size_t dst = ((size_t)bh * kpad + r) * D;
   uint4 kk = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
   if (r < k_vert && pos >= 0 && pos < N) {
@@ -514,8 +519,8 @@ cudaError_t prefill_t(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
     v_prep<D><<<(unsigned)blocks, 256, 0, s>>>(v, idx, nbh, N, k_vert, w.vh, w.vc);
   }
   if (kpad > 0)
-    gather_vertical<D><<<dim3(kpad, nbh), D / 8, 0, s>>>(k, w.vh, idx, N, k_vert, kpad, w.vk,
-                                                         w.vv, w.vpos);
+    gather_vertical<D><<<dim3(kpad, nbh), D / 8, 0, s>>>(k, w.vh, idx, N, window, k_vert, kpad,
+                                                         w.vk, w.vv, w.vpos, status);
   if (prefill_tc_supported(D, Hq, Hkv)) {
     TcLaunch p;
     p.q = q;

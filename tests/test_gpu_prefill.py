@@ -95,3 +95,25 @@ def test_prefill_full_size_sampled_rows():
         np.arange(0, 8), np.arange(W - 4, W + 4), rng.integers(0, N, 48),
         np.arange(N - 64, N, 8), [N - 1]])).astype(np.int32)
     run_prefill_case(w, rows=rows)
+
+
+def test_prefill_reports_bad_index_lists():
+    """An index list that is not strictly ascending inside [0, N - window)
+    sets HQ_DEV_BAD_INDEX in the workspace status word; a valid one does not.
+    Every access stays in bounds either way (remaining-key positions are
+    clamped by construction, vertical rows are gathered only when in range)."""
+    H = hq()
+    w = Workload("p", "prefill", 1, 4, 2, 128, 640, 128, F5, 4, 31)
+    x = make_inputs(w)
+    d = to_dev(x)
+    ridx, _ = oracle_idx(x, w)
+    ws = H.workspace(H.hq_prefill_workspace_size(w.B, w.Hq, w.Hkv, w.L, w.D, w.k_vert))
+    good = torch.from_numpy(ridx).cuda()
+    H.prefill_attn(d["q"], d["k"], d["v"], good, w.window, ws=ws)
+    assert H.hq_read_device_status(ws) == 0
+    for bad in (ridx[:, :, ::-1].copy(),                        # descending
+                np.where(np.arange(w.k_vert) == 3, w.L - 1, ridx).astype(np.int32),  # in the window
+                np.where(np.arange(w.k_vert) == 0, -5, ridx).astype(np.int32)):      # negative
+        H.prefill_attn(d["q"], d["k"], d["v"], torch.from_numpy(bad).cuda(), w.window, ws=ws)
+        assert H.hq_read_device_status(ws, clear=True) & H.HQ_DEV_BAD_INDEX
+        assert H.hq_read_device_status(ws) == 0
