@@ -64,33 +64,47 @@ struct Cfg {
 
 struct DecArgs {
   const __nv_bfloat16 *q;
-  float *part_o;          // [B*Hq, nsplit, D]  unnormalized partial outputs
-  float2 *part_ml;        // [B*Hq, nsplit]     (max in log2 units, sum)
+  float *part_o;          // [nslot][G][D]  unnormalized partial outputs
+  float2 *part_ml;        // [nslot][G]     (max in log2 units, sum)
   unsigned *counters;     // [B*Hkv] arrival tickets, left at zero
   float *out, *lse;
   uint32_t *status;
-  int Hq, Hkv, n_lo, n_hi, nsplit_lo, nsplit_hi;
+  int Hq, Hkv, n_lo, n_hi;
+  int nbh;                // B * Hkv
+  int tl, th;             // 64-token tiles of the low / bf16 segment per (b, kv head)
+  int nc_lo, nc_hi;       // CTAs streaming low tiles (blockIdx.x < nc_lo) and bf16 tiles
   float sl;               // softmax scale * log2(e)
 };
 
-__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t d;
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;\n" : "=r"(d) : "r"(a), "r"(b), "r"(c));  // (a & b) | c
-  return d;
+// Each kind of tile (low-bit, bf16) of all (b, kv head) pairs is laid end to
+// end, pair-major, and cut into equal contiguous ranges, one per CTA of that
+// kind.  A CTA's tiles of one pair form a "piece" with its own partial result.
+// Partial slots: low CTA i on pair bh -> i + bh; bf16 CTA j on pair bh ->
+// (nc_lo + nbh) + j + bh (consecutive pieces of one pair get consecutive
+// slots, and no two pieces share one).
+struct Line {
+  int n;          // CTAs on this line
+  int t;          // tiles per pair
+  long long T;    // tiles in all
+  int slot0;      // first partial slot of the line
+};
+__device__ __forceinline__ Line line_of(const DecArgs &a, bool hi) {
+  Line L;
+  L.n = hi ? a.nc_hi : a.nc_lo;
+  L.t = hi ? a.th : a.tl;
+  L.T = (long long)L.t * a.nbh;
+  L.slot0 = hi ? a.nc_lo + a.nbh : 0;
+  return L;
 }
+__device__ __forceinline__ long long range_start(const Line &L, int i) { return L.T * i / L.n; }
+// The CTA of the line whose range holds global tile g.
+__device__ __forceinline__ int cta_of(const Line &L, long long g) {
+  return (int)(((g + 1) * (long long)L.n - 1) / L.T);
+}
+
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t d;
   asm("prmt.b32 %0, %1, %2, %3;\n" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
-  return d;
-}
-__device__ __forceinline__ uint32_t hsub2_u(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("sub.rn.f16x2 %0, %1, %2;\n" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-__device__ __forceinline__ uint32_t hfma2_u(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t d;
-  asm("fma.rn.f16x2 %0, %1, %2, %3;\n" : "=r"(d) : "r"(a), "r"(b), "r"(c));
   return d;
 }
 __device__ __forceinline__ uint32_t hmul2_u(uint32_t a, uint32_t b) {
@@ -105,9 +119,13 @@ __device__ __forceinline__ float half_lo_f(uint32_t w) {
   return __half2float(__ushort_as_half((unsigned short)(w & 0xffffu)));
 }
 
-constexpr uint32_t F16_1024x2 = 0x64006400u;   // (1024, 1024)
-constexpr uint32_t F16_1_16x2 = 0x2C002C00u;   // (1/16, 1/16)
-constexpr uint32_t F16_M64x2 = 0xD400D400u;    // (-64, -64)
+// Codes enter the MMAs as fp16 subnormals: the bit pattern c (0 <= c < 2^10)
+// is the number c * 2^-24, exactly, so a mask (or a byte permute with zero
+// high bytes) turns packed codes into MMA operands with no arithmetic.  A
+// high nibble kept in place (bits 4..7) is 16 c * 2^-24.  The 2^24 (2^20 for
+// high nibbles) comes back in fp32 after the MMA.
+constexpr float kCodeUnit = 16777216.0f;     // 2^24
+constexpr float kHiNibbleUnit = 1048576.0f;  // 2^20
 
 // Swizzled byte offset of 16-byte chunk `ch` of row `row` in a TMA box whose
 // rows are RB bytes (64B or 128B swizzle mode).
@@ -128,70 +146,53 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::NSTAGE * C::STAGE);
   uint64_t *empty = full + C::NSTAGE;
-  float *qsum = reinterpret_cast<float *>(empty + C::NSTAGE);   // [8 heads][4 groups]
-  float *qbias = qsum + 32;                                      // [8 heads][4 groups]
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(qbias + 32);
-  int *last_flag = reinterpret_cast<int *>(qbias + 33);
+  uint64_t *merged = empty + C::NSTAGE;                         // one phase per finished piece
+  float *qsum = reinterpret_cast<float *>(merged + 1);          // [8 heads][4 groups]
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(qsum + 32);
+  int *last_flag = reinterpret_cast<int *>(qsum + 33);
 
-  const int split = blockIdx.x, bh = blockIdx.y;
-  const int b = bh / a.Hkv, kh = bh % a.Hkv;
-  const int nsplit = a.nsplit_lo + a.nsplit_hi;
-  const bool hi = split >= a.nsplit_lo;
-  const int sidx = hi ? split - a.nsplit_lo : split;
-  const int ns = hi ? a.nsplit_hi : a.nsplit_lo;
+  const bool hi = (int)blockIdx.x >= a.nc_lo;
+  const int cta = hi ? (int)blockIdx.x - a.nc_lo : (int)blockIdx.x;
+  const Line L = line_of(a, hi);
+  const long long g0 = range_start(L, cta), g1 = range_start(L, cta + 1);
+  const int bh_a = (int)(g0 / L.t), bh_b = (int)((g1 - 1) / L.t);   // pairs of this CTA's pieces
   const int T = hi ? T_HI : T_LO;
-  const int nst = hi ? C::NSTAGE / 2 : C::NSTAGE;              // stages of this CTA
+  const int nst = hi ? C::NSTAGE / 2 : C::NSTAGE;              // stages of this CTA (power of 2)
+  const int lnst = hi ? 1 : 2;                                  // log2(nst)
+  static_assert(C::NSTAGE == 4, "stage arithmetic assumes 4 / 2 stages");
   const int stage_bytes = hi ? 2 * C::STAGE : C::STAGE;
   const int n_tok = hi ? a.n_hi : a.n_lo;
-  const int ntile = (n_tok + T - 1) / T;
-  const int tile0 = (int)((long long)ntile * sidx / ns);
-  const int tile1 = (int)((long long)ntile * (sidx + 1) / ns);
-  const int my_tiles = tile1 - tile0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = lane >> 2, c = lane & 3;
+  // tiles [t0, t1) of pair bh held by this CTA
+  auto piece = [&](int bh, int &t0, int &t1) {
+    const long long base = (long long)bh * L.t;
+    t0 = (int)((g0 > base ? g0 : base) - base);
+    t1 = (int)((g1 < base + L.t ? g1 : base + L.t) - base);
+  };
+
+  // named barrier of the four consumer warps (the producer never joins it)
+  auto consumer_sync = [] { asm volatile("bar.sync 1, %0;\n" ::"n"(NCW * 32) : "memory"); };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NSTAGE; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], NCW);
     }
+    mbar_init(merged, NCW);
     fence_mbar_init();
     *abort_flag = 0;
     *last_flag = 0;
-  }
-  // Per-head q statistics: group sums (for the zero-point term) and the
-  // constant the 1024-offset code encoding adds to each group accumulator.
-  // Thread t < 128: head t/16, group (t/4)%4, eight channels 8*(t%4)...
-  if (threadIdx.x < 128) {
-    const int h = threadIdx.x >> 4, g = (threadIdx.x >> 2) & 3, part = threadIdx.x & 3;
-    float s = 0.f, bias = 0.f;
-    if (h < G) {
-      const uint4 w = *reinterpret_cast<const uint4 *>(a.q + ((size_t)b * a.Hq + kh * G + h) * D +
-                                                      32 * g + 8 * part);
-      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float x = (i & 1) ? bf16_hi(ww[i >> 1]) : bf16_lo(ww[i >> 1]);
-        s += x;
-        const float x16 = __half2float(__float2half_rn(x));
-        if (BITS == 8 || (i & 1) == 0) bias += 1024.f * x16;
-        else bias += 1024.f * __half2float(__float2half_rn(x16 * 0.0625f));
-      }
-    }
-    s += __shfl_xor_sync(0xffffffffu, s, 1);
-    s += __shfl_xor_sync(0xffffffffu, s, 2);
-    bias += __shfl_xor_sync(0xffffffffu, bias, 1);
-    bias += __shfl_xor_sync(0xffffffffu, bias, 2);
-    if (part == 0) {
-      qsum[h * 4 + g] = s;
-      qbias[h * 4 + g] = bias;
-    }
   }
   __syncthreads();
 
   if (warp == NCW) {
     // ------------------------------ producer ------------------------------
-    if (lane == 0 && my_tiles > 0) {
+    // Streams the tiles of every piece back to back; before the first tile of
+    // a new piece it waits until the consumers have merged the previous one
+    // (the merge borrows the stage memory).  Starts at once: the consumers'
+    // per-pair prologue overlaps the first copies.
+    if (lane == 0) {
       if (hi) {
         tma_prefetch_desc(&tm_khi);
         tma_prefetch_desc(&tm_vhi);
@@ -201,486 +202,545 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
         tma_prefetch_desc(&tm_ksz);
         tma_prefetch_desc(&tm_vsz);
       }
-      int issued = 0;
-      for (int it = 0; it < my_tiles; ++it) {
-        const int s = it % nst;
-        if (it >= nst && !mbar_wait(&empty[s], ((it / nst) & 1) ^ 1)) {
+      int n = 0;                                   // tiles issued
+      bool stop = false;
+      for (int bh = bh_a; bh <= bh_b && !stop; ++bh) {
+        int t0, t1;
+        piece(bh, t0, t1);
+        if (bh > bh_a && !mbar_wait(merged, (bh - bh_a - 1) & 1)) {
           *abort_flag = 1;
           raise_status(a.status, HQ_DEV_TIMEOUT);
           break;
         }
-        if (*abort_flag) break;
-        uint8_t *st = smem + s * stage_bytes;
-        const int tok = (tile0 + it) * T;
-        if (!hi) {
-          mbar_arrive_expect_tx(&full[s], C::LO_BYTES);
-          tma_load_3d(st, &tm_kc, &full[s], 0, tok, bh);
-          tma_load_3d(st + C::KC, &tm_vc, &full[s], 0, tok, bh);
-          tma_load_3d(st + 2 * C::KC, &tm_ksz, &full[s], 0, tok, bh);
-          tma_load_3d(st + 2 * C::KC + C::SZ, &tm_vsz, &full[s], 0, tok, bh);
-        } else {
-          mbar_arrive_expect_tx(&full[s], C::HI_BYTES);
-          tma_load_3d(st, &tm_khi, &full[s], 0, tok, bh);
-          tma_load_3d(st + C::HI_BOX, &tm_khi, &full[s], 64, tok, bh);
-          tma_load_3d(st + 2 * C::HI_BOX, &tm_vhi, &full[s], 0, tok, bh);
-          tma_load_3d(st + 3 * C::HI_BOX, &tm_vhi, &full[s], 64, tok, bh);
+        for (int t = t0; t < t1; ++t) {
+          const int s = n & (nst - 1);
+          if (n >= nst && !mbar_wait(&empty[s], ((n >> lnst) & 1) ^ 1)) {
+            *abort_flag = 1;
+            raise_status(a.status, HQ_DEV_TIMEOUT);
+            stop = true;
+            break;
+          }
+          if (*abort_flag) {
+            stop = true;
+            break;
+          }
+          uint8_t *st = smem + s * stage_bytes;
+          const int tok = t * T;
+          if (!hi) {
+            mbar_arrive_expect_tx(&full[s], C::LO_BYTES);
+            tma_load_3d(st, &tm_kc, &full[s], 0, tok, bh);
+            tma_load_3d(st + C::KC, &tm_vc, &full[s], 0, tok, bh);
+            tma_load_3d(st + 2 * C::KC, &tm_ksz, &full[s], 0, tok, bh);
+            tma_load_3d(st + 2 * C::KC + C::SZ, &tm_vsz, &full[s], 0, tok, bh);
+          } else {
+            mbar_arrive_expect_tx(&full[s], C::HI_BYTES);
+            tma_load_3d(st, &tm_khi, &full[s], 0, tok, bh);
+            tma_load_3d(st + C::HI_BOX, &tm_khi, &full[s], 64, tok, bh);
+            tma_load_3d(st + 2 * C::HI_BOX, &tm_vhi, &full[s], 0, tok, bh);
+            tma_load_3d(st + 3 * C::HI_BOX, &tm_vhi, &full[s], 64, tok, bh);
+          }
+          ++n;
         }
-        issued = it + 1;
       }
       // Never leave the CTA with copies in flight.
-      for (int it = issued > nst ? issued - nst : 0; it < issued; ++it)
-        if (!mbar_wait(&full[it % nst], (it / nst) & 1)) raise_status(a.status, HQ_DEV_TIMEOUT);
+      for (int i = n > nst ? n - nst : 0; i < n; ++i)
+        if (!mbar_wait(&full[i & (nst - 1)], (i >> lnst) & 1)) raise_status(a.status, HQ_DEV_TIMEOUT);
     }
+    __syncwarp();
   }
 
   // ------------------------------ consumers -------------------------------
-  // Softmax state for heads 2c, 2c+1 (log2 units), partial sums, outputs.
-  float m0 = -1e30f, m1 = -1e30f, l0 = 0.f, l1 = 0.f;
-  float o[8][4];
-  float oz[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-  for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-
+  // One pass per piece: per-pair q set-up, the piece's tiles, then the warps'
+  // merge into the piece's partial result, the arrival ticket of the pair and,
+  // for the last arrival, the merge of all the pair's pieces.
   if (warp < NCW) {
-    // B fragments of q: 8 k16-chunks x 2 registers.
-    uint32_t qb[8][2];
-    const __nv_bfloat16 *qh = a.q + ((size_t)b * a.Hq + kh * G + (r < G ? r : 0)) * D;
-    const bool hv = r < G;
-    if (hi) {
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        qb[kk][0] = hv ? *reinterpret_cast<const uint32_t *>(qh + 16 * kk + 2 * c) : 0u;
-        qb[kk][1] = hv ? *reinterpret_cast<const uint32_t *>(qh + 16 * kk + 8 + 2 * c) : 0u;
-      }
-    } else if (BITS == 4) {
-#pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        float x[8];
-        const uint4 w = hv ? *reinterpret_cast<const uint4 *>(qh + 32 * g + 8 * c) : make_uint4(0, 0, 0, 0);
-        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          x[2 * i] = bf16_lo(ww[i]);
-          x[2 * i + 1] = bf16_hi(ww[i]);
-        }
-        // chunk 2g+0: slots (2c,2c+1) <- ch 0,4; (2c+8,2c+9) <- ch 1/16, 5/16
-        // chunk 2g+1: slots (2c,2c+1) <- ch 2,6; (2c+8,2c+9) <- ch 3/16, 7/16
-        auto f16 = [](float v) { return __half2float(__float2half_rn(v)); };
-        qb[2 * g][0] = pack_f16x2(x[0], x[4]);
-        qb[2 * g][1] = pack_f16x2(f16(x[1]) * 0.0625f, f16(x[5]) * 0.0625f);
-        qb[2 * g + 1][0] = pack_f16x2(x[2], x[6]);
-        qb[2 * g + 1][1] = pack_f16x2(f16(x[3]) * 0.0625f, f16(x[7]) * 0.0625f);
-      }
-    } else {
-#pragma unroll
-      for (int kc = 0; kc < 8; ++kc) {
-        const uint2 w = hv ? *reinterpret_cast<const uint2 *>(qh + 16 * kc + 4 * c) : make_uint2(0, 0);
-        qb[kc][0] = pack_f16x2(bf16_lo(w.x), bf16_hi(w.x));
-        qb[kc][1] = pack_f16x2(bf16_lo(w.y), bf16_hi(w.y));
-      }
-    }
-    // Z-term B operand (k = 2*group + {hi, lo} half of Q_group, n = head r).
-    uint32_t zb0 = 0u;
-    if (!hi && hv) {
-      const float Q = qsum[r * 4 + c];
-      const __half qh16 = __float2half_rn(Q);
-      const __half ql16 = __float2half_rn(Q - __half2float(qh16));
-      zb0 = (uint32_t)__half_as_ushort(qh16) | ((uint32_t)__half_as_ushort(ql16) << 16);
-    }
-    float nb[4][2];  // -bias of each group for heads 2c, 2c+1 (accumulator start)
-#pragma unroll
-    for (int g = 0; g < 4; ++g) {
-      nb[g][0] = (2 * c < G) ? -qbias[(2 * c) * 4 + g] : 0.f;
-      nb[g][1] = (2 * c + 1 < G) ? -qbias[(2 * c + 1) * 4 + g] : 0.f;
-    }
-
     const int j = warp;  // this warp's 16-token sub-tile of every stage
-    for (int it = 0; it < my_tiles; ++it) {
-      const int s = it % nst;
-      if (!mbar_wait(&full[s], (it / nst) & 1)) {
-        *abort_flag = 1;
-        raise_status(a.status, HQ_DEV_TIMEOUT);
-        break;
+    int n = 0;           // tiles consumed
+    for (int bh = bh_a; bh <= bh_b; ++bh) {
+      const int b = bh / a.Hkv, kh = bh % a.Hkv;
+      int t0, t1;
+      piece(bh, t0, t1);
+      // ---- q statistics of this pair: group sums (for the zero-point term);
+      // thread t: head t/16, group (t/4)%4, channels 8*(t%4).. ----
+      {
+        const int h = threadIdx.x >> 4, g = (threadIdx.x >> 2) & 3, part = threadIdx.x & 3;
+        float sm = 0.f;
+        if (h < G) {
+          const uint4 w = *reinterpret_cast<const uint4 *>(a.q + ((size_t)b * a.Hq + kh * G + h) * D +
+                                                          32 * g + 8 * part);
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) sm += bf16_lo(ww[i]) + bf16_hi(ww[i]);
+        }
+        sm += __shfl_xor_sync(0xffffffffu, sm, 1);
+        sm += __shfl_xor_sync(0xffffffffu, sm, 2);
+        if (part == 0) qsum[h * 4 + g] = sm;
       }
-      uint8_t *const stp = smem + s * stage_bytes;
-      const uint32_t st = smem_u32(stp);
-      const int tok0 = (tile0 + it) * T + j * 16;
-      const int row0 = j * 16;
-      const bool ok_r = tok0 + r < n_tok, ok_r8 = tok0 + r + 8 < n_tok;
-      float x[4];
-      // ---------------- scores S^T (16 tokens x 8 heads) ----------------
-      if (!hi) {
-        float acc[4][4];
+      consumer_sync();
+      // Softmax state for heads 2c, 2c+1 (log2 units), partial sums, outputs.
+      float m0 = -1e30f, m1 = -1e30f, l0 = 0.f, l1 = 0.f;
+      float o[8][4];
+      float oz[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          acc[g][0] = nb[g][0];
-          acc[g][1] = nb[g][1];
-          acc[g][2] = nb[g][0];
-          acc[g][3] = nb[g][1];
+      for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+      // B fragments of q: 8 k16-chunks x 2 registers.
+      uint32_t qb[8][2];
+      const __nv_bfloat16 *qh = a.q + ((size_t)b * a.Hq + kh * G + (r < G ? r : 0)) * D;
+      const bool hv = r < G;
+      if (hi) {
+  #pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          qb[kk][0] = hv ? *reinterpret_cast<const uint32_t *>(qh + 16 * kk + 2 * c) : 0u;
+          qb[kk][1] = hv ? *reinterpret_cast<const uint32_t *>(qh + 16 * kk + 8 + 2 * c) : 0u;
         }
-        const int mi = lane >> 3;
-        const int lrow = row0 + (mi & 1) * 8 + (lane & 7);
-        if (BITS == 4) {
-#pragma unroll
-          for (int gp = 0; gp < 2; ++gp) {
-            uint32_t kx[4];
-            ldsm_x4(kx, st + swz_off<C::ROWB>(lrow, 2 * gp + (mi >> 1)));
-#pragma unroll
-            for (int gg = 0; gg < 2; ++gg) {
-              const int g = 2 * gp + gg;
-              const uint32_t A0 = kx[2 * gg], A1 = kx[2 * gg + 1];
-              const uint32_t A08 = A0 >> 8, A18 = A1 >> 8;
-              uint32_t fa[4], fb[4];
-              fa[0] = lop3_and_or(A0, 0x000F000Fu, F16_1024x2);
-              fa[1] = lop3_and_or(A1, 0x000F000Fu, F16_1024x2);
-              fa[2] = lop3_and_or(A0, 0x00F000F0u, F16_1024x2);
-              fa[3] = lop3_and_or(A1, 0x00F000F0u, F16_1024x2);
-              fb[0] = lop3_and_or(A08, 0x000F000Fu, F16_1024x2);
-              fb[1] = lop3_and_or(A18, 0x000F000Fu, F16_1024x2);
-              fb[2] = lop3_and_or(A08, 0x00F000F0u, F16_1024x2);
-              fb[3] = lop3_and_or(A18, 0x00F000F0u, F16_1024x2);
-              mma_f16_16816(acc[g], fa, qb[2 * g][0], qb[2 * g][1]);
-              mma_f16_16816(acc[g], fb, qb[2 * g + 1][0], qb[2 * g + 1][1]);
-            }
-          }
-        } else {
-#pragma unroll
-          for (int cp = 0; cp < 4; ++cp) {
-            uint32_t kx[4];
-            ldsm_x4(kx, st + swz_off<C::ROWB>(lrow, 2 * cp + (mi >> 1)));
-#pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-              const int kc = 2 * cp + cc;
-              const uint32_t A0 = kx[2 * cc], A1 = kx[2 * cc + 1];
-              uint32_t fa[4];
-              // bytes of F16_1024x2 as prmt source 4..7: 0x00, 0x64, 0x00, 0x64
-              fa[0] = prmt(A0, F16_1024x2, 0x5150);
-              fa[1] = prmt(A1, F16_1024x2, 0x5150);
-              fa[2] = prmt(A0, F16_1024x2, 0x5352);
-              fa[3] = prmt(A1, F16_1024x2, 0x5352);
-              mma_f16_16816(acc[kc >> 1], fa, qb[kc][0], qb[kc][1]);
-            }
-          }
-        }
-        // zero-point term and per-group scales of the two tokens
-        const uint4 s_r = *reinterpret_cast<const uint4 *>(stp + 2 * C::KC + (row0 + r) * 16);
-        const uint4 s_r8 = *reinterpret_cast<const uint4 *>(stp + 2 * C::KC + (row0 + r + 8) * 16);
-        const uint32_t wr[4] = {s_r.x, s_r.y, s_r.z, s_r.w};
-        const uint32_t wr8[4] = {s_r8.x, s_r8.y, s_r8.z, s_r8.w};
-        uint32_t za[4];
-        za[0] = prmt(wr[c], wr[c], 0x3232);
-        za[1] = prmt(wr8[c], wr8[c], 0x3232);
-        za[2] = 0u;
-        za[3] = 0u;
-        float zacc[4] = {0.f, 0.f, 0.f, 0.f};
-        mma_f16_16816(zacc, za, zb0, 0u);
-        x[0] = zacc[0];
-        x[1] = zacc[1];
-        x[2] = zacc[2];
-        x[3] = zacc[3];
-#pragma unroll
+      } else if (BITS == 4) {
+  #pragma unroll
         for (int g = 0; g < 4; ++g) {
-          const float sa = half_lo_f(wr[g]), sb = half_lo_f(wr8[g]);
-          x[0] = fmaf(sa, acc[g][0], x[0]);
-          x[1] = fmaf(sa, acc[g][1], x[1]);
-          x[2] = fmaf(sb, acc[g][2], x[2]);
-          x[3] = fmaf(sb, acc[g][3], x[3]);
+          float x[8];
+          const uint4 w = hv ? *reinterpret_cast<const uint4 *>(qh + 32 * g + 8 * c) : make_uint4(0, 0, 0, 0);
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+  #pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            x[2 * i] = bf16_lo(ww[i]);
+            x[2 * i + 1] = bf16_hi(ww[i]);
+          }
+          // chunk 2g+0: slots (2c,2c+1) <- ch 0,4; (2c+8,2c+9) <- ch 1/16, 5/16
+          // chunk 2g+1: slots (2c,2c+1) <- ch 2,6; (2c+8,2c+9) <- ch 3/16, 7/16
+          auto f16 = [](float v) { return __half2float(__float2half_rn(v)); };
+          qb[2 * g][0] = pack_f16x2(x[0], x[4]);
+          qb[2 * g][1] = pack_f16x2(f16(x[1]) * 0.0625f, f16(x[5]) * 0.0625f);
+          qb[2 * g + 1][0] = pack_f16x2(x[2], x[6]);
+          qb[2 * g + 1][1] = pack_f16x2(f16(x[3]) * 0.0625f, f16(x[7]) * 0.0625f);
         }
       } else {
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        const int mi = lane >> 3;
-        const int lrow = row0 + (mi & 1) * 8 + (lane & 7);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          uint32_t ka[4];
-          const uint32_t box = st + (kk >> 2) * C::HI_BOX;
-          ldsm_x4(ka, box + swz_off<128>(lrow, 2 * (kk & 3) + (mi >> 1)));
-          mma_bf16_16816(acc, ka, qb[kk][0], qb[kk][1]);
+  #pragma unroll
+        for (int kc = 0; kc < 8; ++kc) {
+          const uint2 w = hv ? *reinterpret_cast<const uint2 *>(qh + 16 * kc + 4 * c) : make_uint2(0, 0);
+          qb[kc][0] = pack_f16x2(bf16_lo(w.x), bf16_hi(w.x));
+          qb[kc][1] = pack_f16x2(bf16_lo(w.y), bf16_hi(w.y));
         }
-        x[0] = acc[0];
-        x[1] = acc[1];
-        x[2] = acc[2];
-        x[3] = acc[3];
       }
-      if (!ok_r) x[0] = x[1] = -INFINITY;
-      if (!ok_r8) x[2] = x[3] = -INFINITY;
+      // Z-term B operand (k = 2*group + {hi, lo} half of Q_group, n = head r).
+      uint32_t zb0 = 0u;
+      if (!hi && hv) {
+        const float Q = qsum[r * 4 + c];
+        const __half qh16 = __float2half_rn(Q);
+        const __half ql16 = __float2half_rn(Q - __half2float(qh16));
+        zb0 = (uint32_t)__half_as_ushort(qh16) | ((uint32_t)__half_as_ushort(ql16) << 16);
+      }
+      for (int t = t0; t < t1; ++t, ++n) {
+        const int s = n & (nst - 1);
+        if (!*abort_flag && !mbar_wait(&full[s], (n >> lnst) & 1)) {
+          *abort_flag = 1;
+          raise_status(a.status, HQ_DEV_TIMEOUT);
+        }
+        if (!*abort_flag) {
+        uint8_t *const stp = smem + s * stage_bytes;
+        const uint32_t st = smem_u32(stp);
+        const int tok0 = t * T + j * 16;
+        const int row0 = j * 16;
+        const bool ok_r = tok0 + r < n_tok, ok_r8 = tok0 + r + 8 < n_tok;
+        float x[4];
+        // ---------------- scores S^T (16 tokens x 8 heads) ----------------
+        if (!hi) {
+          float acc[4][4];
+  #pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            acc[g][0] = acc[g][1] = acc[g][2] = acc[g][3] = 0.f;
+          }
+          const int mi = lane >> 3;
+          const int lrow = row0 + (mi & 1) * 8 + (lane & 7);
+          if (BITS == 4) {
+  #pragma unroll
+            for (int gp = 0; gp < 2; ++gp) {
+              uint32_t kx[4];
+              ldsm_x4(kx, st + swz_off<C::ROWB>(lrow, 2 * gp + (mi >> 1)));
+  #pragma unroll
+              for (int gg = 0; gg < 2; ++gg) {
+                const int g = 2 * gp + gg;
+                const uint32_t A0 = kx[2 * gg], A1 = kx[2 * gg + 1];
+                const uint32_t A08 = A0 >> 8, A18 = A1 >> 8;
+                uint32_t fa[4], fb[4];
+                fa[0] = A0 & 0x000F000Fu;
+                fa[1] = A1 & 0x000F000Fu;
+                fa[2] = A0 & 0x00F000F0u;
+                fa[3] = A1 & 0x00F000F0u;
+                fb[0] = A08 & 0x000F000Fu;
+                fb[1] = A18 & 0x000F000Fu;
+                fb[2] = A08 & 0x00F000F0u;
+                fb[3] = A18 & 0x00F000F0u;
+                mma_f16_16816(acc[g], fa, qb[2 * g][0], qb[2 * g][1]);
+                mma_f16_16816(acc[g], fb, qb[2 * g + 1][0], qb[2 * g + 1][1]);
+              }
+            }
+          } else {
+  #pragma unroll
+            for (int cp = 0; cp < 4; ++cp) {
+              uint32_t kx[4];
+              ldsm_x4(kx, st + swz_off<C::ROWB>(lrow, 2 * cp + (mi >> 1)));
+  #pragma unroll
+              for (int cc = 0; cc < 2; ++cc) {
+                const int kc = 2 * cp + cc;
+                const uint32_t A0 = kx[2 * cc], A1 = kx[2 * cc + 1];
+                uint32_t fa[4];
+                // byte pairs (c, 0): selector 4 takes byte 0 of the zero operand
+                fa[0] = prmt(A0, 0u, 0x4140);
+                fa[1] = prmt(A1, 0u, 0x4140);
+                fa[2] = prmt(A0, 0u, 0x4342);
+                fa[3] = prmt(A1, 0u, 0x4342);
+                mma_f16_16816(acc[kc >> 1], fa, qb[kc][0], qb[kc][1]);
+              }
+            }
+          }
+          // zero-point term and per-group scales of the two tokens
+          const uint4 s_r = *reinterpret_cast<const uint4 *>(stp + 2 * C::KC + (row0 + r) * 16);
+          const uint4 s_r8 = *reinterpret_cast<const uint4 *>(stp + 2 * C::KC + (row0 + r + 8) * 16);
+          const uint32_t wr[4] = {s_r.x, s_r.y, s_r.z, s_r.w};
+          const uint32_t wr8[4] = {s_r8.x, s_r8.y, s_r8.z, s_r8.w};
+          uint32_t za[4];
+          // (z of group c) in both halves; c is lane-dependent, so select
+          // instead of indexing (an indexed array would live in local memory)
+          const uint32_t wc_ = c == 0 ? wr[0] : c == 1 ? wr[1] : c == 2 ? wr[2] : wr[3];
+          const uint32_t wc8 = c == 0 ? wr8[0] : c == 1 ? wr8[1] : c == 2 ? wr8[2] : wr8[3];
+          za[0] = prmt(wc_, wc_, 0x3232);
+          za[1] = prmt(wc8, wc8, 0x3232);
+          za[2] = 0u;
+          za[3] = 0u;
+          float zacc[4] = {0.f, 0.f, 0.f, 0.f};
+          mma_f16_16816(zacc, za, zb0, 0u);
+          float y[4] = {0.f, 0.f, 0.f, 0.f};
+  #pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const float sa = half_lo_f(wr[g]), sb = half_lo_f(wr8[g]);
+            y[0] = fmaf(sa, acc[g][0], y[0]);
+            y[1] = fmaf(sa, acc[g][1], y[1]);
+            y[2] = fmaf(sb, acc[g][2], y[2]);
+            y[3] = fmaf(sb, acc[g][3], y[3]);
+          }
+  #pragma unroll
+          for (int e = 0; e < 4; ++e) x[e] = fmaf(y[e], kCodeUnit, zacc[e]);
+        } else {
+          float acc[4] = {0.f, 0.f, 0.f, 0.f};
+          const int mi = lane >> 3;
+          const int lrow = row0 + (mi & 1) * 8 + (lane & 7);
+  #pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            uint32_t ka[4];
+            const uint32_t box = st + (kk >> 2) * C::HI_BOX;
+            ldsm_x4(ka, box + swz_off<128>(lrow, 2 * (kk & 3) + (mi >> 1)));
+            mma_bf16_16816(acc, ka, qb[kk][0], qb[kk][1]);
+          }
+          x[0] = acc[0];
+          x[1] = acc[1];
+          x[2] = acc[2];
+          x[3] = acc[3];
+        }
+        if (!ok_r) x[0] = x[1] = -INFINITY;
+        if (!ok_r8) x[2] = x[3] = -INFINITY;
 
-      // ---------------- online softmax (lazy rescale) ----------------
-      float t0 = fmaxf(x[0], x[2]) * a.sl, t1 = fmaxf(x[1], x[3]) * a.sl;
-#pragma unroll
-      for (int off = 4; off < 32; off <<= 1) {
-        t0 = fmaxf(t0, __shfl_xor_sync(0xffffffffu, t0, off));
-        t1 = fmaxf(t1, __shfl_xor_sync(0xffffffffu, t1, off));
-      }
-      const bool need = (t0 > m0 + kLazy) || (t1 > m1 + kLazy);
-      if (__any_sync(0xffffffffu, need)) {
-        const float n0 = fmaxf(m0, t0), n1 = fmaxf(m1, t1);
-        const float al0 = exp2f(m0 - n0), al1 = exp2f(m1 - n1);
-        m0 = n0;
-        m1 = n1;
-        l0 *= al0;
-        l1 *= al1;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          o[i][0] *= al0;
-          o[i][1] *= al1;
-          o[i][2] *= al0;
-          o[i][3] *= al1;
+        // ---------------- online softmax (lazy rescale) ----------------
+        // This lane's maxima first: the tile maximum (three shuffle rounds)
+        // is only needed when some lane's score exceeds the running max by
+        // more than 2^8, which is rare after the first tiles.
+        float t0 = fmaxf(x[0], x[2]) * a.sl, t1 = fmaxf(x[1], x[3]) * a.sl;
+        if (__any_sync(0xffffffffu, (t0 > m0 + kLazy) || (t1 > m1 + kLazy))) {
+  #pragma unroll
+          for (int off = 4; off < 32; off <<= 1) {
+            t0 = fmaxf(t0, __shfl_xor_sync(0xffffffffu, t0, off));
+            t1 = fmaxf(t1, __shfl_xor_sync(0xffffffffu, t1, off));
+          }
+          const float n0 = fmaxf(m0, t0), n1 = fmaxf(m1, t1);
+          const float al0 = exp2f(m0 - n0), al1 = exp2f(m1 - n1);
+          m0 = n0;
+          m1 = n1;
+          l0 *= al0;
+          l1 *= al1;
+  #pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            o[i][0] *= al0;
+            o[i][1] *= al1;
+            o[i][2] *= al0;
+            o[i][3] *= al1;
+          }
+          oz[0] *= al0;
+          oz[1] *= al1;
+          oz[2] *= al0;
+          oz[3] *= al1;
         }
-        oz[0] *= al0;
-        oz[1] *= al1;
-        oz[2] *= al0;
-        oz[3] *= al1;
-      }
-      const float p0 = fast_exp2(fmaf(x[0], a.sl, -m0)), p1 = fast_exp2(fmaf(x[1], a.sl, -m1));
-      const float p2 = fast_exp2(fmaf(x[2], a.sl, -m0)), p3 = fast_exp2(fmaf(x[3], a.sl, -m1));
-      l0 += p0 + p2;
-      l1 += p1 + p3;
-      const uint32_t pb0 = movmatrix_t(pack_f16x2(p0, p1));   // (head r; tokens 2c, 2c+1)
-      const uint32_t pb1 = movmatrix_t(pack_f16x2(p2, p3));   // (head r; tokens 2c+8, 2c+9)
+        const float p0 = fast_exp2(fmaf(x[0], a.sl, -m0)), p1 = fast_exp2(fmaf(x[1], a.sl, -m1));
+        const float p2 = fast_exp2(fmaf(x[2], a.sl, -m0)), p3 = fast_exp2(fmaf(x[3], a.sl, -m1));
+        l0 += p0 + p2;
+        l1 += p1 + p3;
+        const uint32_t pb0 = movmatrix_t(pack_f16x2(p0, p1));   // (head r; tokens 2c, 2c+1)
+        const uint32_t pb1 = movmatrix_t(pack_f16x2(p2, p3));   // (head r; tokens 2c+8, 2c+9)
 
-      // ---------------- O^T += V^T P ----------------
-      if (!hi) {
-        const uint8_t *vszp = stp + 2 * C::KC + C::SZ;
-        const int ta = row0 + 2 * c;
-        const uint4 wa = *reinterpret_cast<const uint4 *>(vszp + ta * 16);
-        const uint4 wb = *reinterpret_cast<const uint4 *>(vszp + (ta + 1) * 16);
-        const uint4 wc = *reinterpret_cast<const uint4 *>(vszp + (ta + 8) * 16);
-        const uint4 wd = *reinterpret_cast<const uint4 *>(vszp + (ta + 9) * 16);
-        const uint32_t A_[4] = {wa.x, wa.y, wa.z, wa.w}, B_[4] = {wb.x, wb.y, wb.z, wb.w};
-        const uint32_t C_[4] = {wc.x, wc.y, wc.z, wc.w}, D_[4] = {wd.x, wd.y, wd.z, wd.w};
-        // zero-point term: rows = group (r & 3), k = tokens
-        {
-          const int gz = r & 3;
-          const uint32_t za0 = *reinterpret_cast<const uint32_t *>(vszp + ta * 16 + gz * 4);
-          const uint32_t zb_ = *reinterpret_cast<const uint32_t *>(vszp + (ta + 1) * 16 + gz * 4);
-          const uint32_t zc = *reinterpret_cast<const uint32_t *>(vszp + (ta + 8) * 16 + gz * 4);
-          const uint32_t zd = *reinterpret_cast<const uint32_t *>(vszp + (ta + 9) * 16 + gz * 4);
-          uint32_t zaf[4];
-          zaf[0] = prmt(za0, zb_, 0x7632);
-          zaf[1] = 0u;
-          zaf[2] = prmt(zc, zd, 0x7632);
-          zaf[3] = 0u;
-          mma_f16_16816(oz, zaf, pb0, pb1);
-        }
-        const int mi = lane >> 3;
-        const int lrow = row0 + (mi & 1) * 8 + (lane & 7);
-        const uint32_t vbase = st + C::KC;
-        if (BITS == 4) {
-#pragma unroll
-          for (int gp = 0; gp < 2; ++gp) {
-            uint32_t vx[4];
-            ldsm_x4_t(vx, vbase + swz_off<C::ROWB>(lrow, 2 * gp + (mi >> 1)));
-#pragma unroll
-            for (int gg = 0; gg < 2; ++gg) {
-              const int g = 2 * gp + gg;
+        // ---------------- O^T += V^T P ----------------
+        if (!hi) {
+          const uint8_t *vszp = stp + 2 * C::KC + C::SZ;
+          const int ta = row0 + 2 * c;
+          const uint4 wa = *reinterpret_cast<const uint4 *>(vszp + ta * 16);
+          const uint4 wb = *reinterpret_cast<const uint4 *>(vszp + (ta + 1) * 16);
+          const uint4 wc = *reinterpret_cast<const uint4 *>(vszp + (ta + 8) * 16);
+          const uint4 wd = *reinterpret_cast<const uint4 *>(vszp + (ta + 9) * 16);
+          const uint32_t A_[4] = {wa.x, wa.y, wa.z, wa.w}, B_[4] = {wb.x, wb.y, wb.z, wb.w};
+          const uint32_t C_[4] = {wc.x, wc.y, wc.z, wc.w}, D_[4] = {wd.x, wd.y, wd.z, wd.w};
+          // zero-point term: rows = group (r & 3), k = tokens
+          {
+            const int gz = r & 3;
+            const uint32_t za0 = *reinterpret_cast<const uint32_t *>(vszp + ta * 16 + gz * 4);
+            const uint32_t zb_ = *reinterpret_cast<const uint32_t *>(vszp + (ta + 1) * 16 + gz * 4);
+            const uint32_t zc = *reinterpret_cast<const uint32_t *>(vszp + (ta + 8) * 16 + gz * 4);
+            const uint32_t zd = *reinterpret_cast<const uint32_t *>(vszp + (ta + 9) * 16 + gz * 4);
+            uint32_t zaf[4];
+            zaf[0] = prmt(za0, zb_, 0x7632);
+            zaf[1] = 0u;
+            zaf[2] = prmt(zc, zd, 0x7632);
+            zaf[3] = 0u;
+            mma_f16_16816(oz, zaf, pb0, pb1);
+          }
+          const int mi = lane >> 3;
+          const int lrow = row0 + (mi & 1) * 8 + (lane & 7);
+          const uint32_t vbase = st + C::KC;
+          if (BITS == 4) {
+  #pragma unroll
+            for (int gp = 0; gp < 2; ++gp) {
+              uint32_t vx[4];
+              ldsm_x4_t(vx, vbase + swz_off<C::ROWB>(lrow, 2 * gp + (mi >> 1)));
+  #pragma unroll
+              for (int gg = 0; gg < 2; ++gg) {
+                const int g = 2 * gp + gg;
+                const uint32_t bs0 = hmul2_u(pb0, prmt(A_[g], B_[g], 0x5410));
+                const uint32_t bs1 = hmul2_u(pb1, prmt(C_[g], D_[g], 0x5410));
+                const uint32_t X = vx[2 * gg], Xp = vx[2 * gg + 1];
+                const uint32_t X8 = X >> 8, Xp8 = Xp >> 8;
+                uint32_t fa[4], fb[4];
+                fa[0] = X & 0x000F000Fu;
+                fa[1] = X & 0x00F000F0u;
+                fa[2] = Xp & 0x000F000Fu;
+                fa[3] = Xp & 0x00F000F0u;
+                fb[0] = X8 & 0x000F000Fu;
+                fb[1] = X8 & 0x00F000F0u;
+                fb[2] = Xp8 & 0x000F000Fu;
+                fb[3] = Xp8 & 0x00F000F0u;
+                mma_f16_16816(o[2 * g], fa, bs0, bs1);
+                mma_f16_16816(o[2 * g + 1], fb, bs0, bs1);
+              }
+            }
+          } else {
+  #pragma unroll
+            for (int cp = 0; cp < 4; ++cp) {
+              uint32_t vx[4];
+              ldsm_x4_t(vx, vbase + swz_off<C::ROWB>(lrow, 2 * cp + (mi >> 1)));
+              const int g = cp;  // chunks 2cp, 2cp+1 form group cp
               const uint32_t bs0 = hmul2_u(pb0, prmt(A_[g], B_[g], 0x5410));
               const uint32_t bs1 = hmul2_u(pb1, prmt(C_[g], D_[g], 0x5410));
-              const uint32_t X = vx[2 * gg], Xp = vx[2 * gg + 1];
-              const uint32_t X8 = X >> 8, Xp8 = Xp >> 8;
-              uint32_t fa[4], fb[4];
-              fa[0] = hsub2_u(lop3_and_or(X, 0x000F000Fu, F16_1024x2), F16_1024x2);
-              fa[1] = hfma2_u(lop3_and_or(X, 0x00F000F0u, F16_1024x2), F16_1_16x2, F16_M64x2);
-              fa[2] = hsub2_u(lop3_and_or(Xp, 0x000F000Fu, F16_1024x2), F16_1024x2);
-              fa[3] = hfma2_u(lop3_and_or(Xp, 0x00F000F0u, F16_1024x2), F16_1_16x2, F16_M64x2);
-              fb[0] = hsub2_u(lop3_and_or(X8, 0x000F000Fu, F16_1024x2), F16_1024x2);
-              fb[1] = hfma2_u(lop3_and_or(X8, 0x00F000F0u, F16_1024x2), F16_1_16x2, F16_M64x2);
-              fb[2] = hsub2_u(lop3_and_or(Xp8, 0x000F000Fu, F16_1024x2), F16_1024x2);
-              fb[3] = hfma2_u(lop3_and_or(Xp8, 0x00F000F0u, F16_1024x2), F16_1_16x2, F16_M64x2);
-              mma_f16_16816(o[2 * g], fa, bs0, bs1);
-              mma_f16_16816(o[2 * g + 1], fb, bs0, bs1);
+  #pragma unroll
+              for (int cc = 0; cc < 2; ++cc) {
+                const uint32_t X = vx[2 * cc], Xp = vx[2 * cc + 1];
+                uint32_t fa[4];
+                fa[0] = prmt(X, 0u, 0x4240);
+                fa[1] = prmt(X, 0u, 0x4341);
+                fa[2] = prmt(Xp, 0u, 0x4240);
+                fa[3] = prmt(Xp, 0u, 0x4341);
+                mma_f16_16816(o[2 * cp + cc], fa, bs0, bs1);
+              }
             }
           }
         } else {
-#pragma unroll
-          for (int cp = 0; cp < 4; ++cp) {
-            uint32_t vx[4];
-            ldsm_x4_t(vx, vbase + swz_off<C::ROWB>(lrow, 2 * cp + (mi >> 1)));
-            const int g = cp;  // chunks 2cp, 2cp+1 form group cp
-            const uint32_t bs0 = hmul2_u(pb0, prmt(A_[g], B_[g], 0x5410));
-            const uint32_t bs1 = hmul2_u(pb1, prmt(C_[g], D_[g], 0x5410));
-#pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-              const uint32_t X = vx[2 * cc], Xp = vx[2 * cc + 1];
-              uint32_t fa[4];
-              fa[0] = hsub2_u(prmt(X, F16_1024x2, 0x5250), F16_1024x2);
-              fa[1] = hsub2_u(prmt(X, F16_1024x2, 0x5351), F16_1024x2);
-              fa[2] = hsub2_u(prmt(Xp, F16_1024x2, 0x5250), F16_1024x2);
-              fa[3] = hsub2_u(prmt(Xp, F16_1024x2, 0x5351), F16_1024x2);
-              mma_f16_16816(o[2 * cp + cc], fa, bs0, bs1);
-            }
+          const int mi = lane >> 3;
+          const int lrow = row0 + (mi >> 1) * 8 + (lane & 7);
+  #pragma unroll
+          for (int mt = 0; mt < 8; ++mt) {
+            uint32_t va[4];
+            const uint32_t box = st + 2 * C::HI_BOX + (mt >> 2) * C::HI_BOX;
+            ldsm_x4_t(va, box + swz_off<128>(lrow, 2 * (mt & 3) + (mi & 1)));
+            uint32_t fa[4];
+            fa[0] = bf16x2_to_f16x2(va[0]);
+            fa[1] = bf16x2_to_f16x2(va[1]);
+            fa[2] = bf16x2_to_f16x2(va[2]);
+            fa[3] = bf16x2_to_f16x2(va[3]);
+            mma_f16_16816(o[mt], fa, pb0, pb1);
           }
         }
-      } else {
-        const int mi = lane >> 3;
-        const int lrow = row0 + (mi >> 1) * 8 + (lane & 7);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+      }
+      // ---------------- merge this piece's warps (the stage memory is free:
+      // every copy of the piece has landed, and the producer waits for
+      // `merged` before it issues the next piece) ----------------
+      consumer_sync();
+      float *wml = reinterpret_cast<float *>(smem);             // [NCW][8][2]
+      float *wz = wml + NCW * 16;                               // [NCW][8 heads][4 groups]
+      float *wo = wz + NCW * 32;                                // [NCW][8 heads][D]
 #pragma unroll
-        for (int mt = 0; mt < 8; ++mt) {
-          uint32_t va[4];
-          const uint32_t box = st + 2 * C::HI_BOX + (mt >> 2) * C::HI_BOX;
-          ldsm_x4_t(va, box + swz_off<128>(lrow, 2 * (mt & 3) + (mi & 1)));
-          uint32_t fa[4];
-          fa[0] = bf16x2_to_f16x2(va[0]);
-          fa[1] = bf16x2_to_f16x2(va[1]);
-          fa[2] = bf16x2_to_f16x2(va[2]);
-          fa[3] = bf16x2_to_f16x2(va[3]);
-          mma_f16_16816(o[mt], fa, pb0, pb1);
+      for (int off = 4; off < 32; off <<= 1) {
+        l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+      }
+      if (r == 0) {
+        wml[(warp * 8 + 2 * c) * 2 + 0] = m0;
+        wml[(warp * 8 + 2 * c) * 2 + 1] = l0;
+        wml[(warp * 8 + 2 * c + 1) * 2 + 0] = m1;
+        wml[(warp * 8 + 2 * c + 1) * 2 + 1] = l1;
+      }
+      if (r < 4) {
+        wz[(warp * 8 + 2 * c) * 4 + r] = oz[0];
+        wz[(warp * 8 + 2 * c + 1) * 4 + r] = oz[1];
+      }
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const int row = r + 8 * hf;
+          int ch;
+          if (hi) ch = 16 * mt + row;
+          else if (BITS == 4) ch = 32 * (mt >> 1) + 4 * r + 2 * (mt & 1) + hf;
+          else ch = 16 * mt + 2 * r + hf;
+          // undo the code unit of the low-bit V operand
+          const float u = hi ? 1.f : (BITS == 4 && hf == 1 ? kHiNibbleUnit : kCodeUnit);
+          wo[(warp * 8 + 2 * c) * D + ch] = o[mt][2 * hf] * u;
+          wo[(warp * 8 + 2 * c + 1) * D + ch] = o[mt][2 * hf + 1] * u;
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
-    }
-  }
-
-  // ---------------- merge the consumer warps ----------------
-  __syncthreads();  // all copies have landed and every stage is consumed
-  float *wml = reinterpret_cast<float *>(smem);             // [NCW][8][2]
-  float *wz = wml + NCW * 16;                               // [NCW][8 heads][4 groups]
-  float *wo = wz + NCW * 32;                                // [NCW][8 heads][D]
-  if (warp < NCW) {
+      consumer_sync();
+      const size_t slot = (size_t)L.slot0 + cta + bh;
+      for (int e = threadIdx.x; e < G * D; e += NCW * 32) {
+        const int h = e / D, d = e % D;
+        float mm = -1e30f;
 #pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-      l0 += __shfl_xor_sync(0xffffffffu, l0, off);
-      l1 += __shfl_xor_sync(0xffffffffu, l1, off);
-    }
-    if (r == 0) {
-      wml[(warp * 8 + 2 * c) * 2 + 0] = m0;
-      wml[(warp * 8 + 2 * c) * 2 + 1] = l0;
-      wml[(warp * 8 + 2 * c + 1) * 2 + 0] = m1;
-      wml[(warp * 8 + 2 * c + 1) * 2 + 1] = l1;
-    }
-    if (!hi && r < 4) {
-      wz[(warp * 8 + 2 * c) * 4 + r] = oz[0];
-      wz[(warp * 8 + 2 * c + 1) * 4 + r] = oz[1];
-    }
+        for (int w = 0; w < NCW; ++w) mm = fmaxf(mm, wml[(w * 8 + h) * 2]);
+        float ll = 0.f, oo = 0.f;
 #pragma unroll
-    for (int mt = 0; mt < 8; ++mt) {
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        const int row = r + 8 * hf;
-        int ch;
-        if (hi) ch = 16 * mt + row;
-        else if (BITS == 4) ch = 32 * (mt >> 1) + 4 * r + 2 * (mt & 1) + hf;
-        else ch = 16 * mt + 2 * r + hf;
-        wo[(warp * 8 + 2 * c) * D + ch] = o[mt][2 * hf];
-        wo[(warp * 8 + 2 * c + 1) * D + ch] = o[mt][2 * hf + 1];
+        for (int w = 0; w < NCW; ++w) {
+          const float f = exp2f(wml[(w * 8 + h) * 2] - mm);
+          ll += f * wml[(w * 8 + h) * 2 + 1];
+          oo += f * (wo[(w * 8 + h) * D + d] + wz[(w * 8 + h) * 4 + d / 32]);
+        }
+        a.part_o[(slot * G + h) * D + d] = oo;
+        if (d == 0) a.part_ml[slot * G + h] = make_float2(mm, ll);
       }
-    }
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < G * D; e += NTHREADS) {
-    const int h = e / D, d = e % D;
-    float mm = -1e30f;
-#pragma unroll
-    for (int w = 0; w < NCW; ++w) mm = fmaxf(mm, wml[(w * 8 + h) * 2]);
-    float ll = 0.f, oo = 0.f;
-#pragma unroll
-    for (int w = 0; w < NCW; ++w) {
-      const float f = exp2f(wml[(w * 8 + h) * 2] - mm);
-      ll += f * wml[(w * 8 + h) * 2 + 1];
-      float ov = wo[(w * 8 + h) * D + d];
-      if (!hi) ov += wz[(w * 8 + h) * 4 + d / 32];
-      oo += f * ov;
-    }
-    const size_t hq = (size_t)b * a.Hq + kh * G + h;
-    a.part_o[(hq * nsplit + split) * D + d] = oo;
-    if (d == 0) a.part_ml[hq * nsplit + split] = make_float2(mm, ll);
-  }
-
-  // ---------------- last CTA of this (b, kv head) merges the splits ----------------
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const unsigned ticket = atomicAdd(&a.counters[bh], 1u);
-    *last_flag = (ticket == (unsigned)(nsplit - 1));
-  }
-  __syncthreads();
-  if (!*last_flag) return;
-  __threadfence();
-  // Merge all splits of the G heads: (max, sum) of every split into shared
-  // memory; one warp per head reduces them (lanes over splits); then every
-  // thread accumulates float4 output columns over a quarter of the splits with
-  // eight independent loads in flight, and the quarters are summed in smem.
-  float *cm = reinterpret_cast<float *>(smem);          // [G][nsplit] split maxima -> weights
-  float *cl = cm + G * nsplit;                           // [G][nsplit] split sums
-  float *cstar = cl + G * nsplit;                        // [G] 1 / total sum
-  float4 *cacc = reinterpret_cast<float4 *>((reinterpret_cast<uintptr_t>(cstar + 8) + 15) & ~uintptr_t(15));  // [4][G * D/4]
-  const size_t hq0 = (size_t)b * a.Hq + kh * G;
-  for (int e = threadIdx.x; e < G * nsplit; e += NTHREADS) {
-    const float2 ml = __ldcg(&a.part_ml[hq0 * nsplit + e]);
-    cm[e] = ml.x;
-    cl[e] = ml.y;
-  }
-  __syncthreads();
-  for (int h = warp; h < G; h += NTHREADS / 32) {
-    float mm = -1e30f;
-    for (int sp = lane; sp < nsplit; sp += 32) mm = fmaxf(mm, cm[h * nsplit + sp]);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) mm = fmaxf(mm, __shfl_xor_sync(0xffffffffu, mm, off));
-    float ll = 0.f;
-    for (int sp = lane; sp < nsplit; sp += 32) {
-      const float f = exp2f(cm[h * nsplit + sp] - mm);
-      cm[h * nsplit + sp] = f;
-      ll += f * cl[h * nsplit + sp];
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) ll += __shfl_xor_sync(0xffffffffu, ll, off);
-    if (lane == 0) {
-      cstar[h] = 1.f / ll;
-      if (a.lse) a.lse[hq0 + h] = (mm + log2f(ll)) * 0.6931471805599453f;
-    }
-  }
-  __syncthreads();
-  constexpr int NCOL = D / 4;
-  for (int e = threadIdx.x; e < 4 * G * NCOL; e += NTHREADS) {
-    const int quarter = e / (G * NCOL), item = e % (G * NCOL);
-    const int h = item / NCOL, d4 = item % NCOL;
-    const float4 *po = reinterpret_cast<const float4 *>(a.part_o + (hq0 + h) * nsplit * D) + d4;
-    const float *f = cm + h * nsplit;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int sp0 = quarter; sp0 < nsplit; sp0 += 32) {
-      float4 x[8];
-      float fw[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int sp = sp0 + 4 * u;
-        x[u] = sp < nsplit ? __ldcg(po + (size_t)sp * NCOL) : make_float4(0.f, 0.f, 0.f, 0.f);
-        fw[u] = sp < nsplit ? f[sp] : 0.f;
+      __threadfence();
+      consumer_sync();
+      // ---------------- arrival ticket of the pair ----------------
+      // Pieces of pair bh: CTAs i0l..i1l of the low line, i0h..i1h of the
+      // bf16 line; their partial slots are consecutive on each line.
+      int i0l = 0, i1l = -1, i0h = 0, i1h = -1;
+      if (a.tl > 0) {
+        const Line Ll = line_of(a, false);
+        i0l = cta_of(Ll, (long long)bh * a.tl);
+        i1l = cta_of(Ll, (long long)bh * a.tl + a.tl - 1);
       }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        acc.x = fmaf(fw[u], x[u].x, acc.x);
-        acc.y = fmaf(fw[u], x[u].y, acc.y);
-        acc.z = fmaf(fw[u], x[u].z, acc.z);
-        acc.w = fmaf(fw[u], x[u].w, acc.w);
+      if (a.th > 0) {
+        const Line Lh = line_of(a, true);
+        i0h = cta_of(Lh, (long long)bh * a.th);
+        i1h = cta_of(Lh, (long long)bh * a.th + a.th - 1);
       }
-    }
-    cacc[quarter * G * NCOL + item] = acc;
-  }
-  __syncthreads();
-  for (int item = threadIdx.x; item < G * NCOL; item += NTHREADS) {
-    const int h = item / NCOL, d4 = item % NCOL;
-    float4 s4 = cacc[item];
+      const int np_lo = i1l - i0l + 1, np = np_lo + (i1h - i0h + 1);
+      if (threadIdx.x == 0) {
+        const unsigned ticket = atomicAdd(&a.counters[bh], 1u);
+        *last_flag = (ticket == (unsigned)(np - 1));
+      }
+      consumer_sync();
+      if (*last_flag) {
+        // ------------- last arrival: merge all pieces of the pair -------------
+        // (max, sum) of every piece into shared memory; one warp per head
+        // reduces them; then every thread accumulates float4 output columns
+        // over a quarter of the pieces with eight loads in flight, and the
+        // quarters are summed in shared memory.
+        __threadfence();
+        auto slot_of = [&](int sp) -> size_t {
+          return sp < np_lo ? (size_t)(i0l + bh + sp) : (size_t)(a.nc_lo + a.nbh + i0h + bh + (sp - np_lo));
+        };
+        float *cm = reinterpret_cast<float *>(smem);          // [G][np] piece maxima -> weights
+        float *cl = cm + G * np;                              // [G][np] piece sums
+        float *cstar = cl + G * np;                           // [G] 1 / total sum
+        float4 *cacc = reinterpret_cast<float4 *>((reinterpret_cast<uintptr_t>(cstar + 8) + 15) & ~uintptr_t(15));  // [4][G * D/4]
+        const size_t hq0 = (size_t)b * a.Hq + kh * G;
+        for (int e = threadIdx.x; e < G * np; e += NCW * 32) {
+          const int h = e / np, sp = e % np;
+          const float2 ml = __ldcg(&a.part_ml[slot_of(sp) * G + h]);
+          cm[e] = ml.x;
+          cl[e] = ml.y;
+        }
+        consumer_sync();
+        for (int h = warp; h < G; h += NCW) {
+          float mm = -1e30f;
+          for (int sp = lane; sp < np; sp += 32) mm = fmaxf(mm, cm[h * np + sp]);
 #pragma unroll
-    for (int q4 = 1; q4 < 4; ++q4) {
-      const float4 t4 = cacc[q4 * G * NCOL + item];
-      s4.x += t4.x;
-      s4.y += t4.y;
-      s4.z += t4.z;
-      s4.w += t4.w;
+          for (int off = 16; off > 0; off >>= 1) mm = fmaxf(mm, __shfl_xor_sync(0xffffffffu, mm, off));
+          float ll = 0.f;
+          for (int sp = lane; sp < np; sp += 32) {
+            const float f = exp2f(cm[h * np + sp] - mm);
+            cm[h * np + sp] = f;
+            ll += f * cl[h * np + sp];
+          }
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) ll += __shfl_xor_sync(0xffffffffu, ll, off);
+          if (lane == 0) {
+            cstar[h] = 1.f / ll;
+            if (a.lse) a.lse[hq0 + h] = (mm + log2f(ll)) * 0.6931471805599453f;
+          }
+        }
+        consumer_sync();
+        constexpr int NCOL = D / 4;
+        for (int e = threadIdx.x; e < 4 * G * NCOL; e += NCW * 32) {
+          const int quarter = e / (G * NCOL), item = e % (G * NCOL);
+          const int h = item / NCOL, d4 = item % NCOL;
+          const float *f = cm + h * np;
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int sp0 = quarter; sp0 < np; sp0 += 32) {
+            float4 x[8];
+            float fw[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int sp = sp0 + 4 * u;
+              x[u] = sp < np ? __ldcg(reinterpret_cast<const float4 *>(a.part_o + (slot_of(sp) * G + h) * D) + d4)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+              fw[u] = sp < np ? f[sp] : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              acc.x = fmaf(fw[u], x[u].x, acc.x);
+              acc.y = fmaf(fw[u], x[u].y, acc.y);
+              acc.z = fmaf(fw[u], x[u].z, acc.z);
+              acc.w = fmaf(fw[u], x[u].w, acc.w);
+            }
+          }
+          cacc[quarter * G * NCOL + item] = acc;
+        }
+        consumer_sync();
+        for (int item = threadIdx.x; item < G * NCOL; item += NCW * 32) {
+          const int h = item / NCOL, d4 = item % NCOL;
+          float4 s4 = cacc[item];
+#pragma unroll
+          for (int q4 = 1; q4 < 4; ++q4) {
+            const float4 t4 = cacc[q4 * G * NCOL + item];
+            s4.x += t4.x;
+            s4.y += t4.y;
+            s4.z += t4.z;
+            s4.w += t4.w;
+          }
+          const float inv = cstar[h];
+          reinterpret_cast<float4 *>(a.out + (hq0 + h) * D)[d4] =
+              make_float4(s4.x * inv, s4.y * inv, s4.z * inv, s4.w * inv);
+        }
+        if (threadIdx.x == 0) a.counters[bh] = 0u;
+      }
+      // the stage memory goes back to the producer
+      asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+      consumer_sync();
+      if (lane == 0) mbar_arrive(merged);
     }
-    const float inv = cstar[h];
-    reinterpret_cast<float4 *>(a.out + (hq0 + h) * D)[d4] =
-        make_float4(s4.x * inv, s4.y * inv, s4.z * inv, s4.w * inv);
   }
-  if (threadIdx.x == 0) a.counters[bh] = 0u;
 }
 
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
 struct Plan {
-  int nsplit_lo, nsplit_hi;
+  int nbh, tl, th, nc_lo, nc_hi;
+  int nslot() const { return nc_lo + nc_hi + 2 * nbh; }
 };
 
 template <int BITS, int G>
@@ -698,32 +758,56 @@ int occupancy() {
   return occ;
 }
 
+// Relative cost of one 64-token tile (measured stream rates of the kernel):
+// a low INT4 tile is compute-bound (~0.83 us per CTA on B200), a bf16 tile
+// ~1.15 us; INT8 is close to bandwidth-bound, so its costs follow the bytes.
+inline void tile_costs(int bits, int &cl, int &ch) {
+  if (bits == 4) {
+    cl = 10;
+    ch = 14;
+  } else {
+    cl = 18;
+    ch = 32;
+  }
+}
+
+// One wave of CTAs (SM count x resident CTAs per SM), shared between the low
+// and the bf16 line in proportion to their cost.  A line is aligned to whole
+// pairs (no CTA spans two pairs) when that idles at most 2% of its CTAs;
+// every CTA gets at least two tiles.
 Plan make_plan(int nbh, int n_lo, int n_hi, int bits, int occ) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int slots = sms * occ;
-  int per_bh = slots / nbh;
-  if (per_bh < 1) per_bh = 1;
-  const double lo_b = (double)n_lo * (2 * (D * bits / 8) + 32);
-  const double hi_b = (double)n_hi * 512.0;
-  const int tl = (n_lo + T_LO - 1) / T_LO, th = (n_hi + T_HI - 1) / T_HI;
   Plan p;
-  if (n_hi == 0) {
-    p.nsplit_lo = per_bh;
-    p.nsplit_hi = 0;
-  } else if (n_lo == 0) {
-    p.nsplit_lo = 0;
-    p.nsplit_hi = per_bh;
+  p.nbh = nbh;
+  p.tl = (n_lo + T_LO - 1) / T_LO;
+  p.th = (n_hi + T_HI - 1) / T_HI;
+  int cl, ch;
+  tile_costs(bits, cl, ch);
+  const double c_lo = (double)p.tl * cl, c_hi = (double)p.th * ch;
+  if (p.th == 0) {
+    p.nc_lo = slots;
+    p.nc_hi = 0;
+  } else if (p.tl == 0) {
+    p.nc_lo = 0;
+    p.nc_hi = slots;
   } else {
-    int nh = (int)(per_bh * hi_b / (lo_b + hi_b) + 0.5);
-    if (nh < 1) nh = 1;
-    if (nh > per_bh - 1) nh = per_bh - 1 > 0 ? per_bh - 1 : 1;
-    p.nsplit_hi = nh;
-    p.nsplit_lo = per_bh - nh > 0 ? per_bh - nh : 1;
+    p.nc_hi = (int)(slots * c_hi / (c_lo + c_hi) + 0.5);
+    if (p.nc_hi < 1) p.nc_hi = 1;
+    if (p.nc_hi > slots - 1) p.nc_hi = slots - 1;
+    p.nc_lo = slots - p.nc_hi;
   }
-  if (p.nsplit_lo > tl) p.nsplit_lo = tl;
-  if (p.nsplit_hi > th) p.nsplit_hi = th;
+  auto fit = [nbh](int n, int t) {
+    if (t == 0) return 0;
+    const long long tiles = (long long)t * nbh;
+    if (n >= nbh && (n % nbh) * 50 <= n) n = n / nbh * nbh;
+    if ((long long)n * 2 > tiles) n = (int)(tiles / 2 > 0 ? tiles / 2 : 1);
+    return n < 1 ? 1 : n;
+  };
+  p.nc_lo = fit(p.nc_lo, p.tl);
+  p.nc_hi = fit(p.nc_hi, p.th);
   return p;
 }
 
@@ -739,15 +823,15 @@ struct WsLayout {
   size_t counters, part_ml, part_o, total;
 };
 
-WsLayout ws_layout(int B, int Hq, int Hkv, int nsplit) {
+WsLayout ws_layout(int B, int Hkv, int G, int nslot) {
   WsLayout w;
   size_t off = kWsHeader;
   w.counters = off;
   off = align_up(off + (size_t)B * Hkv * sizeof(unsigned), 256);
   w.part_ml = off;
-  off = align_up(off + (size_t)B * Hq * nsplit * sizeof(float2), 256);
+  off = align_up(off + (size_t)nslot * G * sizeof(float2), 256);
   w.part_o = off;
-  off = align_up(off + (size_t)B * Hq * nsplit * D * sizeof(float), 256);
+  off = align_up(off + (size_t)nslot * G * D * sizeof(float), 256);
   w.total = off;
   return w;
 }
@@ -767,7 +851,7 @@ cudaError_t launch_tg(const DecArgs &a0, const hq_kv_cache &c, int nbh, cudaStre
   ok &= make_map_3d(&m[5], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, c.v_hi, D, c.n_hi, nbh, 64, T_HI, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return cudaErrorInvalidValue;
   occupancy<BITS, G>();  // sets the dynamic shared memory attribute once
-  dim3 grid(a.nsplit_lo + a.nsplit_hi, nbh);
+  dim3 grid(a.nc_lo + a.nc_hi);
   decode_tma<BITS, G><<<grid, NTHREADS, Cfg<BITS>::SMEM, s>>>(m[0], m[1], m[2], m[3], m[4], m[5], a);
   return cudaGetLastError();
 }
@@ -781,13 +865,13 @@ bool decode_tma_supported(int D_, int bits, int G) {
 size_t decode_tma_ws_bytes(int B, int Hq, int Hkv, int n_lo, int n_hi, int bits) {
   const int G = Hq / Hkv;
   const Plan p = make_plan(B * Hkv, n_lo, n_hi, bits, occupancy_for(bits, G));
-  return ws_layout(B, Hq, Hkv, p.nsplit_lo + p.nsplit_hi).total;
+  return ws_layout(B, Hkv, G, p.nslot()).total;
 }
 
 size_t decode_tma_ws_zero_bytes(int B, int Hq, int Hkv, int n_lo, int n_hi, int bits) {
   const int G = Hq / Hkv;
   const Plan p = make_plan(B * Hkv, n_lo, n_hi, bits, occupancy_for(bits, G));
-  return ws_layout(B, Hq, Hkv, p.nsplit_lo + p.nsplit_hi).part_ml;
+  return ws_layout(B, Hkv, G, p.nslot()).part_ml;
 }
 
 cudaError_t launch_decode_tma(const __nv_bfloat16 *q, const hq_kv_cache &c, int B, int Hq,
@@ -795,7 +879,7 @@ cudaError_t launch_decode_tma(const __nv_bfloat16 *q, const hq_kv_cache &c, int 
                               uint32_t *status, cudaStream_t s) {
   const int G = Hq / Hkv, nbh = B * Hkv;
   const Plan p = make_plan(nbh, c.n_lo, c.n_hi, c.bits, occupancy_for(c.bits, G));
-  const WsLayout w = ws_layout(B, Hq, Hkv, p.nsplit_lo + p.nsplit_hi);
+  const WsLayout w = ws_layout(B, Hkv, G, p.nslot());
   DecArgs a;
   a.q = q;
   a.part_o = reinterpret_cast<float *>(ws + w.part_o);
@@ -808,8 +892,11 @@ cudaError_t launch_decode_tma(const __nv_bfloat16 *q, const hq_kv_cache &c, int 
   a.Hkv = Hkv;
   a.n_lo = c.n_lo;
   a.n_hi = c.n_hi;
-  a.nsplit_lo = p.nsplit_lo;
-  a.nsplit_hi = p.nsplit_hi;
+  a.nbh = nbh;
+  a.tl = p.tl;
+  a.th = p.th;
+  a.nc_lo = p.nc_lo;
+  a.nc_hi = p.nc_hi;
   a.sl = scale * kLog2e;
 #define HQ_L(BITS, GG) if (c.bits == BITS && G == GG) return launch_tg<BITS, GG>(a, c, nbh, s);
   HQ_L(4, 1) HQ_L(4, 2) HQ_L(4, 4) HQ_L(4, 8)
