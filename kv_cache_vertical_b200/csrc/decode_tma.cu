@@ -147,7 +147,8 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::NSTAGE * C::STAGE);
   uint64_t *empty = full + C::NSTAGE;
   uint64_t *merged = empty + C::NSTAGE;                         // one phase per finished piece
-  float *qsum = reinterpret_cast<float *>(merged + 1);          // [8 heads][4 groups]
+  uint64_t *cbar = merged + 1;                                  // [2] partial chunks of a pair merge
+  float *qsum = reinterpret_cast<float *>(cbar + 2);            // [8 heads][4 groups]
   volatile int *abort_flag = reinterpret_cast<volatile int *>(qsum + 32);
   int *last_flag = reinterpret_cast<int *>(qsum + 33);
 
@@ -180,6 +181,8 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
       mbar_init(&empty[s], NCW);
     }
     mbar_init(merged, NCW);
+    mbar_init(&cbar[0], 1);
+    mbar_init(&cbar[1], 1);
     fence_mbar_init();
     *abort_flag = 0;
     *last_flag = 0;
@@ -256,6 +259,7 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
   if (warp < NCW) {
     const int j = warp;  // this warp's 16-token sub-tile of every stage
     int n = 0;           // tiles consumed
+    int cq = 0;          // partial chunks loaded so far (phases of cbar)
     for (int bh = bh_a; bh <= bh_b; ++bh) {
       const int b = bh / a.Hkv, kh = bh % a.Hkv;
       int t0, t1;
@@ -604,21 +608,34 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
         }
       }
       consumer_sync();
-      const size_t slot = (size_t)L.slot0 + cta + bh;
-      for (int e = threadIdx.x; e < G * D; e += NCW * 32) {
-        const int h = e / D, d = e % D;
+      // weights of the warps' partials, once per head
+      float *wf = wo + NCW * 8 * D;                             // [8 heads][NCW]
+      float *wm = wf + 8 * NCW;                                 // [8] max, [8] sum
+      if (threadIdx.x < G) {
+        const int h = threadIdx.x;
         float mm = -1e30f;
 #pragma unroll
         for (int w = 0; w < NCW; ++w) mm = fmaxf(mm, wml[(w * 8 + h) * 2]);
-        float ll = 0.f, oo = 0.f;
+        float ll = 0.f;
 #pragma unroll
         for (int w = 0; w < NCW; ++w) {
           const float f = exp2f(wml[(w * 8 + h) * 2] - mm);
+          wf[h * NCW + w] = f;
           ll += f * wml[(w * 8 + h) * 2 + 1];
-          oo += f * (wo[(w * 8 + h) * D + d] + wz[(w * 8 + h) * 4 + d / 32]);
         }
+        wm[h] = mm;
+        wm[8 + h] = ll;
+      }
+      consumer_sync();
+      const size_t slot = (size_t)L.slot0 + cta + bh;
+      for (int e = threadIdx.x; e < G * D; e += NCW * 32) {
+        const int h = e / D, d = e % D;
+        float oo = 0.f;
+#pragma unroll
+        for (int w = 0; w < NCW; ++w)
+          oo = fmaf(wf[h * NCW + w], wo[(w * 8 + h) * D + d] + wz[(w * 8 + h) * 4 + d / 32], oo);
         a.part_o[(slot * G + h) * D + d] = oo;
-        if (d == 0) a.part_ml[slot * G + h] = make_float2(mm, ll);
+        if (d == 0) a.part_ml[slot * G + h] = make_float2(wm[h], wm[8 + h]);
       }
       __threadfence();
       consumer_sync();
@@ -644,10 +661,10 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
       consumer_sync();
       if (*last_flag) {
         // ------------- last arrival: merge all pieces of the pair -------------
-        // (max, sum) of every piece into shared memory; one warp per head
-        // reduces them; then every thread accumulates float4 output columns
-        // over a quarter of the pieces with eight loads in flight, and the
-        // quarters are summed in shared memory.
+        // (max, sum) of every piece into shared memory and one warp per head
+        // turns them into weights; the pieces' partial outputs (consecutive
+        // slots on each line) stream into two shared buffers by bulk copies,
+        // chunk k+1 in flight while chunk k is accumulated.
         __threadfence();
         auto slot_of = [&](int sp) -> size_t {
           return sp < np_lo ? (size_t)(i0l + bh + sp) : (size_t)(a.nc_lo + a.nbh + i0h + bh + (sp - np_lo));
@@ -655,7 +672,12 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
         float *cm = reinterpret_cast<float *>(smem);          // [G][np] piece maxima -> weights
         float *cl = cm + G * np;                              // [G][np] piece sums
         float *cstar = cl + G * np;                           // [G] 1 / total sum
-        float4 *cacc = reinterpret_cast<float4 *>((reinterpret_cast<uintptr_t>(cstar + 8) + 15) & ~uintptr_t(15));  // [4][G * D/4]
+        uint8_t *cbuf0 = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(cstar + 8) + 127) & ~uintptr_t(127));
+        constexpr uint32_t PB = G * D * 4;                    // bytes of one piece's partial output
+        const uint32_t avail = (uint32_t)(smem + C::NSTAGE * C::STAGE - cbuf0);
+        int chk = (int)(avail / 2 / PB);
+        chk = chk < 1 ? 1 : (chk > 32 ? 32 : chk);
+        uint8_t *const cbuf1 = cbuf0 + chk * PB;
         const size_t hq0 = (size_t)b * a.Hq + kh * G;
         for (int e = threadIdx.x; e < G * np; e += NCW * 32) {
           const int h = e / np, sp = e % np;
@@ -682,48 +704,68 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
             if (a.lse) a.lse[hq0 + h] = (mm + log2f(ll)) * 0.6931471805599453f;
           }
         }
-        consumer_sync();
+        // chunks of at most chk consecutive pieces, never across the two lines
+        const int ncl = (np_lo + chk - 1) / chk, nchunks = ncl + (np - np_lo + chk - 1) / chk;
+        auto chunk = [&](int k, int &sp0, int &cnt) {
+          if (k < ncl) {
+            sp0 = k * chk;
+            cnt = min(chk, np_lo - sp0);
+          } else {
+            sp0 = np_lo + (k - ncl) * chk;
+            cnt = min(chk, np - sp0);
+          }
+        };
+        auto issue = [&](int k) {
+          int sp0, cnt;
+          chunk(k, sp0, cnt);
+          const int gk = cq + k;
+          mbar_arrive_expect_tx(&cbar[gk & 1], cnt * PB);
+          bulk_load((gk & 1) ? cbuf1 : cbuf0, a.part_o + slot_of(sp0) * G * D, cnt * PB, &cbar[gk & 1]);
+        };
+        consumer_sync();                                      // weights ready; buffers free
+        if (threadIdx.x == 0) issue(0);
         constexpr int NCOL = D / 4;
-        for (int e = threadIdx.x; e < 4 * G * NCOL; e += NCW * 32) {
-          const int quarter = e / (G * NCOL), item = e % (G * NCOL);
-          const int h = item / NCOL, d4 = item % NCOL;
-          const float *f = cm + h * np;
-          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-          for (int sp0 = quarter; sp0 < np; sp0 += 32) {
-            float4 x[8];
-            float fw[8];
+        float4 acc[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
+        for (int k = 0; k < nchunks; ++k) {
+          if (threadIdx.x == 0 && k + 1 < nchunks) issue(k + 1);   // its buffer was released below
+          const int gk = cq + k;
+          const bool ready = !*abort_flag && mbar_wait(&cbar[gk & 1], (gk >> 1) & 1);
+          if (!ready && !*abort_flag) {
+            *abort_flag = 1;
+            raise_status(a.status, HQ_DEV_TIMEOUT);
+          }
+          if (ready) {
+            int sp0, cnt;
+            chunk(k, sp0, cnt);
+            const float4 *buf = reinterpret_cast<const float4 *>((gk & 1) ? cbuf1 : cbuf0);
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const int sp = sp0 + 4 * u;
-              x[u] = sp < np ? __ldcg(reinterpret_cast<const float4 *>(a.part_o + (slot_of(sp) * G + h) * D) + d4)
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
-              fw[u] = sp < np ? f[sp] : 0.f;
-            }
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              acc.x = fmaf(fw[u], x[u].x, acc.x);
-              acc.y = fmaf(fw[u], x[u].y, acc.y);
-              acc.z = fmaf(fw[u], x[u].z, acc.z);
-              acc.w = fmaf(fw[u], x[u].w, acc.w);
+            for (int jj = 0; jj < 2; ++jj) {
+              const int item = threadIdx.x + jj * NCW * 32;
+              if (item < G * NCOL) {
+                const int h = item / NCOL, d4 = item % NCOL;
+                const float *f = cm + h * np + sp0;
+                for (int u = 0; u < cnt; ++u) {
+                  const float4 x = buf[(u * G + h) * NCOL + d4];
+                  acc[jj].x = fmaf(f[u], x.x, acc[jj].x);
+                  acc[jj].y = fmaf(f[u], x.y, acc[jj].y);
+                  acc[jj].z = fmaf(f[u], x.z, acc[jj].z);
+                  acc[jj].w = fmaf(f[u], x.w, acc[jj].w);
+                }
+              }
             }
           }
-          cacc[quarter * G * NCOL + item] = acc;
+          consumer_sync();                                    // buffer gk & 1 may be refilled
         }
-        consumer_sync();
-        for (int item = threadIdx.x; item < G * NCOL; item += NCW * 32) {
-          const int h = item / NCOL, d4 = item % NCOL;
-          float4 s4 = cacc[item];
+        cq += nchunks;
 #pragma unroll
-          for (int q4 = 1; q4 < 4; ++q4) {
-            const float4 t4 = cacc[q4 * G * NCOL + item];
-            s4.x += t4.x;
-            s4.y += t4.y;
-            s4.z += t4.z;
-            s4.w += t4.w;
+        for (int jj = 0; jj < 2; ++jj) {
+          const int item = threadIdx.x + jj * NCW * 32;
+          if (item < G * NCOL) {
+            const int h = item / NCOL, d4 = item % NCOL;
+            const float inv = cstar[h];
+            reinterpret_cast<float4 *>(a.out + (hq0 + h) * D)[d4] =
+                make_float4(acc[jj].x * inv, acc[jj].y * inv, acc[jj].z * inv, acc[jj].w * inv);
           }
-          const float inv = cstar[h];
-          reinterpret_cast<float4 *>(a.out + (hq0 + h) * D)[d4] =
-              make_float4(s4.x * inv, s4.y * inv, s4.z * inv, s4.w * inv);
         }
         if (threadIdx.x == 0) a.counters[bh] = 0u;
       }
@@ -738,6 +780,19 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
+// SM count of the current device (cached per device).
+int sm_count() {
+  static thread_local int dev_cached = -1, sms_cached = 148;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev != dev_cached) {
+    int sms = 148;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess) sms_cached = sms;
+    dev_cached = dev;
+  }
+  return sms_cached;
+}
+
 struct Plan {
   int nbh, tl, th, nc_lo, nc_hi;
   int nslot() const { return nc_lo + nc_hi + 2 * nbh; }
@@ -758,13 +813,13 @@ int occupancy() {
   return occ;
 }
 
-// Relative cost of one 64-token tile (measured stream rates of the kernel):
-// a low INT4 tile is compute-bound (~0.83 us per CTA on B200), a bf16 tile
-// ~1.15 us; INT8 is close to bandwidth-bound, so its costs follow the bytes.
+// Relative cost of one 64-token tile, from the measured per-CTA stream rates
+// on B200: a low INT4 tile is compute-bound and takes ~0.63 of a bf16 tile;
+// INT8 is close to bandwidth-bound, so its costs follow the bytes.
 inline void tile_costs(int bits, int &cl, int &ch) {
   if (bits == 4) {
     cl = 10;
-    ch = 14;
+    ch = 16;
   } else {
     cl = 18;
     ch = 32;
@@ -774,12 +829,10 @@ inline void tile_costs(int bits, int &cl, int &ch) {
 // One wave of CTAs (SM count x resident CTAs per SM), shared between the low
 // and the bf16 line in proportion to their cost.  A line is aligned to whole
 // pairs (no CTA spans two pairs) when that idles at most 2% of its CTAs;
-// every CTA gets at least two tiles.
+// every CTA gets at least eight tiles (fewer, longer pieces keep the final
+// merge short).
 Plan make_plan(int nbh, int n_lo, int n_hi, int bits, int occ) {
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int slots = sms * occ;
+  const int slots = sm_count() * occ;
   Plan p;
   p.nbh = nbh;
   p.tl = (n_lo + T_LO - 1) / T_LO;
@@ -803,7 +856,7 @@ Plan make_plan(int nbh, int n_lo, int n_hi, int bits, int occ) {
     if (t == 0) return 0;
     const long long tiles = (long long)t * nbh;
     if (n >= nbh && (n % nbh) * 50 <= n) n = n / nbh * nbh;
-    if ((long long)n * 2 > tiles) n = (int)(tiles / 2 > 0 ? tiles / 2 : 1);
+    if ((long long)n * 8 > tiles) n = (int)(tiles / 8 > 0 ? tiles / 8 : 1);
     return n < 1 ? 1 : n;
   };
   p.nc_lo = fit(p.nc_lo, p.tl);
@@ -839,17 +892,38 @@ WsLayout ws_layout(int B, int Hkv, int G, int nslot) {
 template <int BITS, int G>
 cudaError_t launch_tg(const DecArgs &a0, const hq_kv_cache &c, int nbh, cudaStream_t s) {
   DecArgs a = a0;
-  CUtensorMap m[6];
-  const int rowb = D * BITS / 8;
-  const CUtensorMapSwizzle sw = rowb == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
-  bool ok = true;
-  ok &= make_map_3d(&m[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, c.k_codes, rowb, c.n_lo, nbh, rowb, T_LO, sw);
-  ok &= make_map_3d(&m[1], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, c.v_codes, rowb, c.n_lo, nbh, rowb, T_LO, sw);
-  ok &= make_map_3d(&m[2], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, c.k_sz, 16, c.n_lo, nbh, 16, T_LO, CU_TENSOR_MAP_SWIZZLE_NONE);
-  ok &= make_map_3d(&m[3], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, c.v_sz, 16, c.n_lo, nbh, 16, T_LO, CU_TENSOR_MAP_SWIZZLE_NONE);
-  ok &= make_map_3d(&m[4], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, c.k_hi, D, c.n_hi, nbh, 64, T_HI, CU_TENSOR_MAP_SWIZZLE_128B);
-  ok &= make_map_3d(&m[5], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, c.v_hi, D, c.n_hi, nbh, 64, T_HI, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (!ok) return cudaErrorInvalidValue;
+  // The six tensor maps depend only on the cache buffers and sizes; the last
+  // set is kept per host thread so that repeated calls on one cache skip the
+  // encoding.
+  struct MapCache {
+    const void *p[6];
+    int n_lo, n_hi, nbh;
+    bool valid;
+    CUtensorMap m[6];
+  };
+  static thread_local MapCache mc = {};
+  const void *ptrs[6] = {c.k_codes, c.v_codes, c.k_sz, c.v_sz, c.k_hi, c.v_hi};
+  bool hit = mc.valid && mc.n_lo == c.n_lo && mc.n_hi == c.n_hi && mc.nbh == nbh;
+  for (int i = 0; i < 6 && hit; ++i) hit = mc.p[i] == ptrs[i];
+  if (!hit) {
+    const int rowb = D * BITS / 8;
+    const CUtensorMapSwizzle sw = rowb == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+    CUtensorMap *m = mc.m;
+    bool ok = true;
+    ok &= make_map_3d(&m[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, c.k_codes, rowb, c.n_lo, nbh, rowb, T_LO, sw);
+    ok &= make_map_3d(&m[1], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, c.v_codes, rowb, c.n_lo, nbh, rowb, T_LO, sw);
+    ok &= make_map_3d(&m[2], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, c.k_sz, 16, c.n_lo, nbh, 16, T_LO, CU_TENSOR_MAP_SWIZZLE_NONE);
+    ok &= make_map_3d(&m[3], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, c.v_sz, 16, c.n_lo, nbh, 16, T_LO, CU_TENSOR_MAP_SWIZZLE_NONE);
+    ok &= make_map_3d(&m[4], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, c.k_hi, D, c.n_hi, nbh, 64, T_HI, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= make_map_3d(&m[5], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, c.v_hi, D, c.n_hi, nbh, 64, T_HI, CU_TENSOR_MAP_SWIZZLE_128B);
+    mc.valid = ok;
+    if (!ok) return cudaErrorInvalidValue;
+    for (int i = 0; i < 6; ++i) mc.p[i] = ptrs[i];
+    mc.n_lo = c.n_lo;
+    mc.n_hi = c.n_hi;
+    mc.nbh = nbh;
+  }
+  const CUtensorMap *m = mc.m;
   occupancy<BITS, G>();  // sets the dynamic shared memory attribute once
   dim3 grid(a.nc_lo + a.nc_hi);
   decode_tma<BITS, G><<<grid, NTHREADS, Cfg<BITS>::SMEM, s>>>(m[0], m[1], m[2], m[3], m[4], m[5], a);
