@@ -6,27 +6,29 @@
 // and dequantizes inside attention, so no dequantized value returns to memory;
 // the vertical-line rows and the window are read in bf16.
 //
-// Layout of the work: each CTA owns a contiguous range of 64-token tiles of
-// the low segment or of the bf16 segment of one (b, kv head)
-// ("split"), streamed global -> shared memory by TMA (one producer warp,
-// mbarrier ring of NSTAGE stages, 64B/128B swizzle so that ldmatrix reads are
-// bank-conflict free).  Each of the four consumer warps takes one 16-token
-// sub-tile of every stage:
+// Layout of the work: the low-bit tiles (64 tokens) and the bf16 tiles of all
+// (b, kv head) pairs form two lines, shared out over one wave of CTAs in
+// proportion to their cost; a CTA serves one or a few consecutive pairs and
+// claims their tiles dynamically (see Line below).  Tiles stream global ->
+// shared memory by TMA (one producer warp, mbarrier ring of NSTAGE stages,
+// 64B/128B swizzle so that ldmatrix reads are bank-conflict free).  Each of
+// the four consumer warps takes one 16-token sub-tile of every stage:
 //
 //   S^T = Kcode * q'  -- tokens are the MMA rows, the G <= 8 query heads of the
-//       KV head the 8 MMA columns.  Codes enter the MMA exactly (fp16 1024+c
-//       bit tricks), one accumulator per 32-channel group, so the per-token
-//       fp16 scale is applied afterwards in fp32:  q.k^ = sum_g s_g (q_g . c_g)
-//       + sum_g z_g Q_g, the second term by one more MMA (z exact in fp16, Q_g
-//       split into two fp16 halves).
+//       KV head the 8 MMA columns.  A code c enters the MMA exactly, as the
+//       fp16 subnormal c * 2^-24 (a mask, no arithmetic), one accumulator per
+//       32-channel group, so the per-token fp16 scale is applied afterwards in
+//       fp32:  q.k^ = 2^24 sum_g s_g (q_g . c_g) + sum_g z_g Q_g, the second
+//       term by one more MMA (z exact in fp16, Q_g split into two fp16 halves).
 //   O^T += Vcode^T * (P o s_v)  -- channels are the MMA rows, P (fp16, moved
 //       into the B layout with movmatrix) is scaled per group by the token's V
-//       scale; the zero-point term sum_t p_t z_t,g is one more MMA.
+//       scale; the zero-point term sum_t p_t z_t,g is one more MMA; the code
+//       unit 2^24 is undone when the warps are merged.
 //
 // Online softmax per head with lazy rescaling (the running max only moves when
-// a tile exceeds it by more than 2^8), a CTA-level merge of the warps, then the
-// last CTA of each (b, kv head) merges all splits (an atomic ticket, no spin
-// waits) and writes the fp32 output and log-sum-exp.
+// a tile exceeds it by more than 2^8), a merge of the warps per piece, then the
+// last piece of each (b, kv head) to finish merges all pieces (an atomic
+// ticket, no spin waits) and writes the fp32 output and log-sum-exp.
 #include <cuda.h>
 #include <float.h>
 
@@ -67,6 +69,7 @@ struct DecArgs {
   float *part_o;          // [nslot][G][D]  unnormalized partial outputs
   float2 *part_ml;        // [nslot][G]     (max in log2 units, sum)
   unsigned *counters;     // [B*Hkv] arrival tickets, left at zero
+  unsigned *tilectr;      // [2][B*Hkv] next unclaimed tile of each pair (low, bf16 line), left at zero
   float *out, *lse;
   uint32_t *status;
   int Hq, Hkv, n_lo, n_hi;
@@ -78,7 +81,10 @@ struct DecArgs {
 
 // Each kind of tile (low-bit, bf16) of all (b, kv head) pairs is laid end to
 // end, pair-major, and cut into equal contiguous ranges, one per CTA of that
-// kind.  A CTA's tiles of one pair form a "piece" with its own partial result.
+// kind.  A CTA's tiles of one pair form a "piece" with its own partial
+// result.  The CTAs whose ranges lie inside one pair pool their tiles and
+// claim them one at a time from a shared counter, so uneven CTA speeds even
+// out; a CTA spanning pairs keeps exactly its own tiles.
 // Partial slots: low CTA i on pair bh -> i + bh; bf16 CTA j on pair bh ->
 // (nc_lo + nbh) + j + bh (consecutive pieces of one pair get consecutive
 // slots, and no two pieces share one).
@@ -151,6 +157,7 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
   float *qsum = reinterpret_cast<float *>(cbar + 2);            // [8 heads][4 groups]
   volatile int *abort_flag = reinterpret_cast<volatile int *>(qsum + 32);
   int *last_flag = reinterpret_cast<int *>(qsum + 33);
+  int *meta = last_flag + 1;                                     // [NSTAGE] tile of each stage, -1: end of piece
 
   const bool hi = (int)blockIdx.x >= a.nc_lo;
   const int cta = hi ? (int)blockIdx.x - a.nc_lo : (int)blockIdx.x;
@@ -165,12 +172,6 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
   const int n_tok = hi ? a.n_hi : a.n_lo;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = lane >> 2, c = lane & 3;
-  // tiles [t0, t1) of pair bh held by this CTA
-  auto piece = [&](int bh, int &t0, int &t1) {
-    const long long base = (long long)bh * L.t;
-    t0 = (int)((g0 > base ? g0 : base) - base);
-    t1 = (int)((g1 < base + L.t ? g1 : base + L.t) - base);
-  };
 
   // named barrier of the four consumer warps (the producer never joins it)
   auto consumer_sync = [] { asm volatile("bar.sync 1, %0;\n" ::"n"(NCW * 32) : "memory"); };
@@ -205,17 +206,36 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
         tma_prefetch_desc(&tm_ksz);
         tma_prefetch_desc(&tm_vsz);
       }
-      int n = 0;                                   // tiles issued
+      // A CTA whose range spans pairs streams exactly its own tiles of each.
+      // The CTAs whose ranges lie inside one pair share the middle of that
+      // pair (everything but its boundary CTAs' tiles): each claims the next
+      // tile from the pair's counter, one claim ahead of use so that the
+      // atomic's latency hides behind the stage wait.  A stage with tile -1
+      // and no copy ends the piece.
+      int n = 0;                                   // stages issued
       bool stop = false;
       for (int bh = bh_a; bh <= bh_b && !stop; ++bh) {
-        int t0, t1;
-        piece(bh, t0, t1);
         if (bh > bh_a && !mbar_wait(merged, (bh - bh_a - 1) & 1)) {
           *abort_flag = 1;
           raise_status(a.status, HQ_DEV_TIMEOUT);
           break;
         }
-        for (int t = t0; t < t1; ++t) {
+        const long long base = (long long)bh * L.t;
+        const bool dyn = bh_a == bh_b;
+        int t0, t1;
+        if (dyn) {
+          const int i0 = cta_of(L, base), i1 = cta_of(L, base + L.t - 1);
+          const long long s0 = range_start(L, i0) < base ? range_start(L, i0 + 1) : base;
+          const long long s1 = range_start(L, i1 + 1) > base + L.t ? range_start(L, i1) : base + L.t;
+          t0 = (int)(s0 - base);
+          t1 = (int)(s1 - base);
+        } else {
+          t0 = (int)((g0 > base ? g0 : base) - base);
+          t1 = (int)((g1 < base + L.t ? g1 : base + L.t) - base);
+        }
+        unsigned *ctr = a.tilectr + (hi ? a.nbh : 0) + bh;
+        int t = dyn ? t0 + (int)atomicAdd(ctr, 1u) : t0;
+        for (;;) {
           const int s = n & (nst - 1);
           if (n >= nst && !mbar_wait(&empty[s], ((n >> lnst) & 1) ^ 1)) {
             *abort_flag = 1;
@@ -227,6 +247,14 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
             stop = true;
             break;
           }
+          ++n;
+          if (t >= t1) {                           // the piece is done: end marker
+            meta[s] = -1;
+            mbar_arrive(&full[s]);
+            break;
+          }
+          const int t_next = dyn ? t0 + (int)atomicAdd(ctr, 1u) : t + 1;
+          meta[s] = t;
           uint8_t *st = smem + s * stage_bytes;
           const int tok = t * T;
           if (!hi) {
@@ -242,7 +270,7 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
             tma_load_3d(st + 2 * C::HI_BOX, &tm_vhi, &full[s], 0, tok, bh);
             tma_load_3d(st + 3 * C::HI_BOX, &tm_vhi, &full[s], 64, tok, bh);
           }
-          ++n;
+          t = t_next;
         }
       }
       // Never leave the CTA with copies in flight.
@@ -262,8 +290,6 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
     int cq = 0;          // partial chunks loaded so far (phases of cbar)
     for (int bh = bh_a; bh <= bh_b; ++bh) {
       const int b = bh / a.Hkv, kh = bh % a.Hkv;
-      int t0, t1;
-      piece(bh, t0, t1);
       // ---- q statistics of this pair: group sums (for the zero-point term);
       // thread t: head t/16, group (t/4)%4, channels 8*(t%4).. ----
       {
@@ -332,11 +358,20 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
         const __half ql16 = __float2half_rn(Q - __half2float(qh16));
         zb0 = (uint32_t)__half_as_ushort(qh16) | ((uint32_t)__half_as_ushort(ql16) << 16);
       }
-      for (int t = t0; t < t1; ++t, ++n) {
+      for (;;) {
+        if (*abort_flag) break;
         const int s = n & (nst - 1);
-        if (!*abort_flag && !mbar_wait(&full[s], (n >> lnst) & 1)) {
+        if (!mbar_wait(&full[s], (n >> lnst) & 1)) {
           *abort_flag = 1;
           raise_status(a.status, HQ_DEV_TIMEOUT);
+          break;
+        }
+        ++n;
+        const int t = meta[s];
+        if (t < 0) {                               // end of this piece
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty[s]);
+          break;
         }
         if (!*abort_flag) {
         uint8_t *const stp = smem + s * stage_bytes;
@@ -767,7 +802,12 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
                 make_float4(acc[jj].x * inv, acc[jj].y * inv, acc[jj].z * inv, acc[jj].w * inv);
           }
         }
-        if (threadIdx.x == 0) a.counters[bh] = 0u;
+        if (threadIdx.x == 0) {
+          // every piece of the pair has stopped claiming tiles: rearm
+          a.tilectr[bh] = 0u;
+          a.tilectr[a.nbh + bh] = 0u;
+          a.counters[bh] = 0u;
+        }
       }
       // the stage memory goes back to the producer
       asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
@@ -814,12 +854,12 @@ int occupancy() {
 }
 
 // Relative cost of one 64-token tile, from the measured per-CTA stream rates
-// on B200: a low INT4 tile is compute-bound and takes ~0.63 of a bf16 tile;
+// on B200: a low INT4 tile is compute-bound and takes ~0.77 of a bf16 tile;
 // INT8 is close to bandwidth-bound, so its costs follow the bytes.
 inline void tile_costs(int bits, int &cl, int &ch) {
   if (bits == 4) {
     cl = 10;
-    ch = 16;
+    ch = 13;
   } else {
     cl = 18;
     ch = 32;
@@ -880,7 +920,7 @@ WsLayout ws_layout(int B, int Hkv, int G, int nslot) {
   WsLayout w;
   size_t off = kWsHeader;
   w.counters = off;
-  off = align_up(off + (size_t)B * Hkv * sizeof(unsigned), 256);
+  off = align_up(off + (size_t)3 * B * Hkv * sizeof(unsigned), 256);   // tickets + two tile counters
   w.part_ml = off;
   off = align_up(off + (size_t)nslot * G * sizeof(float2), 256);
   w.part_o = off;
@@ -959,6 +999,7 @@ cudaError_t launch_decode_tma(const __nv_bfloat16 *q, const hq_kv_cache &c, int 
   a.part_o = reinterpret_cast<float *>(ws + w.part_o);
   a.part_ml = reinterpret_cast<float2 *>(ws + w.part_ml);
   a.counters = reinterpret_cast<unsigned *>(ws + w.counters);
+  a.tilectr = a.counters + nbh;
   a.out = out;
   a.lse = lse;
   a.status = status;
