@@ -27,7 +27,9 @@
  *   Workspace: calls that need scratch take (ws, ws_bytes).  Size it with the
  *     matching hq_*_workspace_size query, allocate it on the device,
  *     zero it ONCE before its first use (cudaMemset), and keep using it; the
- *     library leaves it in a reusable state.  The first 16 bytes hold a
+ *     library leaves it in a reusable state (the decode's arrival tickets and
+ *     tile counters return to zero at the end of every call).  After a call
+ *     that reported HQ_DEV_TIMEOUT, zero it again.  The first 16 bytes hold a
  *     device status word (see hq_read_device_status).  Calls that share one
  *     workspace must not run concurrently.
  *   Errors: arguments are checked on the host before any launch; a failed
