@@ -290,29 +290,6 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
     int cq = 0;          // partial chunks loaded so far (phases of cbar)
     for (int bh = bh_a; bh <= bh_b; ++bh) {
       const int b = bh / a.Hkv, kh = bh % a.Hkv;
-      // ---- q statistics of this pair: group sums (for the zero-point term);
-      // thread t: head t/16, group (t/4)%4, channels 8*(t%4).. ----
-      {
-        const int h = threadIdx.x >> 4, g = (threadIdx.x >> 2) & 3, part = threadIdx.x & 3;
-        float sm = 0.f;
-        if (h < G) {
-          const uint4 w = *reinterpret_cast<const uint4 *>(a.q + ((size_t)b * a.Hq + kh * G + h) * D +
-                                                          32 * g + 8 * part);
-          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-          for (int i = 0; i < 4; ++i) sm += bf16_lo(ww[i]) + bf16_hi(ww[i]);
-        }
-        sm += __shfl_xor_sync(0xffffffffu, sm, 1);
-        sm += __shfl_xor_sync(0xffffffffu, sm, 2);
-        if (part == 0) qsum[h * 4 + g] = sm;
-      }
-      consumer_sync();
-      // Softmax state for heads 2c, 2c+1 (log2 units), partial sums, outputs.
-      float m0 = -1e30f, m1 = -1e30f, l0 = 0.f, l1 = 0.f;
-      float o[8][4];
-      float oz[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
       // B fragments of q: 8 k16-chunks x 2 registers.
       uint32_t qb[8][2];
       const __nv_bfloat16 *qh = a.q + ((size_t)b * a.Hq + kh * G + (r < G ? r : 0)) * D;
@@ -350,6 +327,29 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
           qb[kc][1] = pack_f16x2(bf16_lo(w.y), bf16_hi(w.y));
         }
       }
+      // ---- q statistics of this pair: group sums (for the zero-point term);
+      // thread t: head t/16, group (t/4)%4, channels 8*(t%4).. ----
+      {
+        const int h = threadIdx.x >> 4, g = (threadIdx.x >> 2) & 3, part = threadIdx.x & 3;
+        float sm = 0.f;
+        if (h < G) {
+          const uint4 w = *reinterpret_cast<const uint4 *>(a.q + ((size_t)b * a.Hq + kh * G + h) * D +
+                                                          32 * g + 8 * part);
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) sm += bf16_lo(ww[i]) + bf16_hi(ww[i]);
+        }
+        sm += __shfl_xor_sync(0xffffffffu, sm, 1);
+        sm += __shfl_xor_sync(0xffffffffu, sm, 2);
+        if (part == 0) qsum[h * 4 + g] = sm;
+      }
+      // Softmax state for heads 2c, 2c+1 (log2 units), partial sums, outputs.
+      float m0 = -1e30f, m1 = -1e30f, l0 = 0.f, l1 = 0.f;
+      float o[8][4];
+      float oz[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+      consumer_sync();
       // Z-term B operand (k = 2*group + {hi, lo} half of Q_group, n = head r).
       uint32_t zb0 = 0u;
       if (!hi && hv) {
@@ -869,8 +869,8 @@ inline void tile_costs(int bits, int &cl, int &ch) {
 // One wave of CTAs (SM count x resident CTAs per SM), shared between the low
 // and the bf16 line in proportion to their cost.  A line is aligned to whole
 // pairs (no CTA spans two pairs) when that idles at most 2% of its CTAs;
-// every CTA gets at least eight tiles (fewer, longer pieces keep the final
-// merge short).
+// every low-bit CTA gets at least eight tiles and every bf16 CTA four (fewer,
+// longer pieces keep the final merge short).
 Plan make_plan(int nbh, int n_lo, int n_hi, int bits, int occ) {
   const int slots = sm_count() * occ;
   Plan p;
@@ -892,15 +892,15 @@ Plan make_plan(int nbh, int n_lo, int n_hi, int bits, int occ) {
     if (p.nc_hi > slots - 1) p.nc_hi = slots - 1;
     p.nc_lo = slots - p.nc_hi;
   }
-  auto fit = [nbh](int n, int t) {
+  auto fit = [nbh](int n, int t, int min_tiles) {
     if (t == 0) return 0;
     const long long tiles = (long long)t * nbh;
     if (n >= nbh && (n % nbh) * 50 <= n) n = n / nbh * nbh;
-    if ((long long)n * 8 > tiles) n = (int)(tiles / 8 > 0 ? tiles / 8 : 1);
+    if ((long long)n * min_tiles > tiles) n = (int)(tiles / min_tiles > 0 ? tiles / min_tiles : 1);
     return n < 1 ? 1 : n;
   };
-  p.nc_lo = fit(p.nc_lo, p.tl);
-  p.nc_hi = fit(p.nc_hi, p.th);
+  p.nc_lo = fit(p.nc_lo, p.tl, 8);
+  p.nc_hi = fit(p.nc_hi, p.th, 4);   // bf16 tiles: a 2-deep ring, so keep their CTAs short
   return p;
 }
 
