@@ -16,8 +16,10 @@
 //               (K tile, V tile) pairs;
 //   warp 1      allocates 512 TMEM columns; lane 0 issues every MMA:
 //               S_X = Q_X K^T (kind::i8 into s32, or kind::f16 bf16 into f32)
-//               and O_X += P_X V (kind::f16, P read from tensor memory);
-//   warps 2-5   softmax of head A, warps 6-9 softmax of head B: one thread per
+//               and O_X += P_X V (kind::f16, P read from tensor memory, in
+//               32-key chunks as the softmax hands them over);
+//   warps 2-3   idle (they keep the softmax warpgroups aligned to TMEM lanes);
+//   warps 4-7   softmax of head A, warps 8-11 softmax of head B: one thread per
 //               query row (TMEM lane), so row max / sum need no shuffles.
 // TMEM: S_A [0,128) (P_A aliases its first 64 columns as packed fp16 pairs),
 // O_A [128,256), S_B [256,384), O_B [384,512).
