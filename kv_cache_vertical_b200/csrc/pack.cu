@@ -10,16 +10,35 @@
 //
 // One warp per (b, kv head, position): it classifies the position with a
 // binary search in the sorted index list, then either copies the bf16 rows or
-// quantizes them.  Every rounding decision of the quantizer is taken in IEEE
-// double, so the codes, scales and zeros are exactly the ones the library's
-// specification defines.  HBM-bound: read 2 * D * 2 bytes per position, write
+// quantizes them.  Every rounding decision of the quantizer is the one IEEE
+// double arithmetic takes (an fp32 estimate settles the codes that are not
+// near a tie), so the codes, scales and zeros are exactly the ones the
+// library's specification defines.  HBM-bound: read 2 * D * 2 bytes per position, write
 // the packed rows.
+#include <limits.h>
+
 #include "hq_internal.cuh"
 
 namespace hq {
 namespace {
 
 constexpr int kWarps = 8;
+
+// fp16((mx - mn) / qmax) with the quotient first rounded to IEEE double, as
+// the specification states.  The fp32 quotient (mx - mn is exact in fp32 for
+// bf16 inputs within 2^15 of each other; otherwise one more rounding) lies
+// within 2^-22 relative of the exact one, so unless it is that close to a
+// point halfway between two fp16 numbers, or below the fp16 normal range,
+// rounding it to fp16 gives the same result; those few cases divide in
+// double.
+__device__ __forceinline__ __half scale_f16(float mx, float mn, int qmax) {
+  const float q = __fdiv_rn(mx - mn, (float)qmax);
+  const uint32_t low = __float_as_uint(q) & 0x1fffu;       // the 13 bits below fp16 precision
+  const bool near_tie = low >= 0x1000u - 8u && low <= 0x1000u + 8u;
+  if (near_tie || q < 6.103515625e-05f)                   // 2^-14
+    return __double2half(((double)mx - (double)mn) / (double)qmax);
+  return __float2half_rn(q);
+}
 
 // D / 32 channels per lane; a group of 32 channels spans 32 / (D/32) lanes.
 template <int D, int BITS>
@@ -45,16 +64,27 @@ __device__ __forceinline__ void quant_store(const uint32_t (&w)[D / 64], uint8_t
     mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   }
-  double dmn = (double)mn;
-  if (dmn == 0.0) dmn = 0.0;  // a -0 minimum is stored as +0
-  const __half hs = __double2half(((double)mx - (double)mn) / (double)QMAX);
-  const __half hz = __double2half(dmn);
-  const double s = (double)__half2float(hs), z = (double)__half2float(hz);
+  const float fmn = mn == 0.f ? 0.f : mn;  // a -0 minimum is stored as +0
+  const __half hs = scale_f16(mx, mn, QMAX);
+  const __half hz = __float2half_rn(fmn);   // mn is bf16: exact in fp32, one rounding
+  // code = clamp(rint((x - z) / s), 0, QMAX) with the quotient in IEEE
+  // double.  An fp32 estimate (error below 2^-14 for |q| < 2^9) decides every
+  // code whose quotient is not within 2^-12 of a half-integer: there the
+  // double quotient rounds to the same integer.  The rest take the double
+  // path itself.
+  const float sf = __half2float(hs), zf = __half2float(hz);
+  const float rs = sf != 0.f ? __frcp_rn(sf) : 0.f;
   uint32_t c[CPL];
 #pragma unroll
   for (int i = 0; i < CPL; ++i) {
-    double t = s != 0.0 ? rint(((double)x[i] - z) / s) : 0.0;
-    t = fmin(fmax(t, 0.0), (double)QMAX);
+    const float q = (x[i] - zf) * rs;
+    float t = rintf(q);
+    if (sf == 0.f) {
+      t = 0.f;
+    } else if (fabsf(q - t) > 0.5f - 1.f / 4096.f) {
+      t = (float)rint(((double)x[i] - (double)zf) / (double)sf);
+    }
+    t = fminf(fmaxf(t, 0.f), (float)QMAX);
     c[i] = (uint32_t)t;
   }
   if (BITS == 4) {
@@ -87,7 +117,6 @@ pack_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict
   constexpr int NG = D / 32;
   const int lane = threadIdx.x & 31;
   const int n_lo = L - window - k_vert, n_hi = k_vert + window;
-  const long long total = (long long)nbh * L;
   const long long warp0 = (long long)blockIdx.x * kWarps + (threadIdx.x >> 5);
   const long long nwarps = (long long)gridDim.x * kWarps;
 
@@ -99,39 +128,63 @@ pack_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict
     if (x < 0 || x >= L - window || (r > 0 && idx[t - 1] >= x)) raise_status(status, HQ_DEV_BAD_INDEX);
   }
 
-  for (long long wi = warp0; wi < total; wi += nwarps) {
-    const int bh = (int)(wi / L);
-    const int j = (int)(wi % L);
-    const size_t src = ((size_t)bh * L + j) * D;
-    uint32_t kw[W32], vw[W32];
+  // Eight consecutive positions of one pair per warp task: one binary search
+  // finds the verticals before the chunk, the next (at most eight) index
+  // entries say which chunk positions are vertical, and all sixteen row loads
+  // are issued before any quantization.
+  constexpr int PCH = 8;
+  const long long ntask = (long long)nbh * ((L + PCH - 1) / PCH);
+  const int cpb = (L + PCH - 1) / PCH;                // chunks per pair
+  for (long long task = warp0; task < ntask; task += nwarps) {
+    const int bh = (int)(task / cpb);
+    const int j0 = (int)(task % cpb) * PCH;
+    const int32_t *id = idx + (size_t)bh * k_vert;
+    const int cnt0 = j0 > 0 ? upper_bound_i32(id, k_vert, j0 - 1) : 0;   // verticals before j0
+    const int e = cnt0 + (lane & (PCH - 1));
+    const int ve = (lane < PCH && e < k_vert) ? __ldg(id + e) : INT_MAX;
+    const uint32_t vbit = (ve >= j0 && ve < j0 + PCH) ? 1u << (ve - j0) : 0u;
+    const uint32_t vbits = __reduce_or_sync(0xffffffffu, vbit);            // vertical positions of the chunk
+    uint32_t kw[PCH][W32], vw[PCH][W32];
 #pragma unroll
-    for (int i = 0; i < W32; ++i) {
-      kw[i] = __ldg(reinterpret_cast<const uint32_t *>(k + src) + lane * W32 + i);
-      vw[i] = __ldg(reinterpret_cast<const uint32_t *>(v + src) + lane * W32 + i);
-    }
-    int hi_row = -1, lo_row = -1;
-    if (j >= L - window) {
-      hi_row = k_vert + (j - (L - window));
-    } else {
-      const int32_t *id = idx + (size_t)bh * k_vert;
-      const int cnt = upper_bound_i32(id, k_vert, j);  // entries <= j
-      if (cnt > 0 && __ldg(id + cnt - 1) == j) hi_row = cnt - 1;
-      else lo_row = j - cnt;
-    }
-    if (hi_row >= 0) {
-      if (hi_row >= n_hi) { if (lane == 0) raise_status(status, HQ_DEV_BAD_INDEX); continue; }
-      const size_t dst = ((size_t)bh * n_hi + hi_row) * D;
+    for (int p = 0; p < PCH; ++p) {
+      const int j = j0 + p;
+      const size_t src = ((size_t)bh * L + (j < L ? j : L - 1)) * D;
 #pragma unroll
       for (int i = 0; i < W32; ++i) {
-        reinterpret_cast<uint32_t *>(k_hi + dst)[lane * W32 + i] = kw[i];
-        reinterpret_cast<uint32_t *>(v_hi + dst)[lane * W32 + i] = vw[i];
+        kw[p][i] = __ldg(reinterpret_cast<const uint32_t *>(k + src) + lane * W32 + i);
+        vw[p][i] = __ldg(reinterpret_cast<const uint32_t *>(v + src) + lane * W32 + i);
       }
-    } else {
-      if (lo_row < 0 || lo_row >= n_lo) { if (lane == 0) raise_status(status, HQ_DEV_BAD_INDEX); continue; }
-      const size_t r = (size_t)bh * n_lo + lo_row;
-      quant_store<D, BITS>(kw, k_codes + r * ROWB, k_sz + r * NG, lane);
-      quant_store<D, BITS>(vw, v_codes + r * ROWB, v_sz + r * NG, lane);
-      if (lo_pos && lane == 0) lo_pos[r] = j;
+    }
+#pragma unroll
+    for (int p = 0; p < PCH; ++p) {
+      const int j = j0 + p;
+      if (j >= L) break;
+      const int cnt = cnt0 + __popc(vbits & ((1u << p) - 1u));            // verticals before j
+      int hi_row = -1, lo_row = -1;
+      if (j >= L - window) hi_row = k_vert + (j - (L - window));
+      else if (vbits & (1u << p)) hi_row = cnt;
+      else lo_row = j - cnt;
+      if (hi_row >= 0) {
+        if (hi_row >= n_hi) {
+          if (lane == 0) raise_status(status, HQ_DEV_BAD_INDEX);
+          continue;
+        }
+        const size_t dst = ((size_t)bh * n_hi + hi_row) * D;
+#pragma unroll
+        for (int i = 0; i < W32; ++i) {
+          reinterpret_cast<uint32_t *>(k_hi + dst)[lane * W32 + i] = kw[p][i];
+          reinterpret_cast<uint32_t *>(v_hi + dst)[lane * W32 + i] = vw[p][i];
+        }
+      } else {
+        if (lo_row < 0 || lo_row >= n_lo) {
+          if (lane == 0) raise_status(status, HQ_DEV_BAD_INDEX);
+          continue;
+        }
+        const size_t r = (size_t)bh * n_lo + lo_row;
+        quant_store<D, BITS>(kw[p], k_codes + r * ROWB, k_sz + r * NG, lane);
+        quant_store<D, BITS>(vw[p], v_codes + r * ROWB, v_sz + r * NG, lane);
+        if (lo_pos && lane == 0) lo_pos[r] = j;
+      }
     }
   }
 }
@@ -143,7 +196,7 @@ cudaError_t launch_pack_t(const __nv_bfloat16 *k, const __nv_bfloat16 *v, const 
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const long long warps = (long long)nbh * L;
+  const long long warps = (long long)nbh * ((L + 7) / 8);     // one warp task per 8 positions
   long long blocks = (warps + kWarps - 1) / kWarps;
   const long long cap = (long long)sms * 8;
   if (blocks > cap) blocks = cap;

@@ -39,39 +39,79 @@ constexpr float kLog2e = 1.4426950408889634f;
 // Pre-pass kernels
 // ---------------------------------------------------------------------------
 
-// One warp per Q row: s = amax / 127, code = clamp(rne(x / s), -127, 127),
-// both divisions single IEEE binary32 roundings.
+// x / s rounded to the nearest integer (ties to even), with the quotient a
+// single IEEE binary32 rounding.  The product with the rounded reciprocal is
+// within 2^-16 of the quotient for |x / s| <= 2^7, so it decides every code
+// that is not within 2^-12 of a half-integer; the rest divide exactly.
+__device__ __forceinline__ float rint_div(float x, float s, float rcp_s) {
+  const float q = x * rcp_s;
+  const float t = rintf(q);
+  return fabsf(q - t) > 0.5f - 1.f / 4096.f ? rintf(__fdiv_rn(x, s)) : t;
+}
+
+// Q rows, four per warp (loads first, then four independent reductions):
+// s = amax / 127, code = clamp(rne(x / s), -127, 127), both divisions single
+// IEEE binary32 roundings.
 template <int D>
-__global__ void quant_q_rows(const __nv_bfloat16 *__restrict__ q, long long nrows,
-                             int8_t *__restrict__ qi8, float *__restrict__ sq) {
-  constexpr int CPL = D / 32;
-  const long long row = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+__global__ void __launch_bounds__(256)
+quant_q_rows(const __nv_bfloat16 *__restrict__ q, long long nrows, int8_t *__restrict__ qi8,
+             float *__restrict__ sq) {
+  constexpr int CPL = D / 32;                   // channels per lane: 4 or 2
+  constexpr int RPW = 4;                        // rows per warp
   const int lane = threadIdx.x & 31;
-  if (row >= nrows) return;
-  const uint32_t *src = reinterpret_cast<const uint32_t *>(q + row * D) + lane * (CPL / 2);
-  float x[CPL];
+  const long long row0 = ((long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5)) * RPW;
+  float x[RPW][CPL];
 #pragma unroll
-  for (int i = 0; i < CPL / 2; ++i) {
-    const uint32_t w = src[i];
-    x[2 * i] = bf16_lo(w);
-    x[2 * i + 1] = bf16_hi(w);
+  for (int rr = 0; rr < RPW; ++rr) {
+    const long long row = row0 + rr;
+    uint32_t w[CPL / 2];
+    if (row < nrows) {
+      const uint32_t *src = reinterpret_cast<const uint32_t *>(q + row * D) + lane * (CPL / 2);
+      if (CPL == 4) {
+        const uint2 v2 = __ldg(reinterpret_cast<const uint2 *>(src));
+        w[0] = v2.x;
+        w[CPL / 2 - 1] = v2.y;
+      } else {
+        w[0] = __ldg(src);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < CPL / 2; ++i) w[i] = 0u;
+    }
+#pragma unroll
+    for (int i = 0; i < CPL / 2; ++i) {
+      x[rr][2 * i] = bf16_lo(w[i]);
+      x[rr][2 * i + 1] = bf16_hi(w[i]);
+    }
   }
-  float amax = 0.f;
+  float amax[RPW];
 #pragma unroll
-  for (int i = 0; i < CPL; ++i) amax = fmaxf(amax, fabsf(x[i]));
+  for (int rr = 0; rr < RPW; ++rr) {
+    amax[rr] = 0.f;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  const float s = amax == 0.f ? 1.f : __fdiv_rn(amax, 127.f);
-  uint32_t packed = 0;
-#pragma unroll
-  for (int i = 0; i < CPL; ++i) {
-    float c = rintf(__fdiv_rn(x[i], s));
-    c = fminf(fmaxf(c, -127.f), 127.f);
-    packed |= ((uint32_t)(int)c & 0xffu) << (8 * i);
+    for (int i = 0; i < CPL; ++i) amax[rr] = fmaxf(amax[rr], fabsf(x[rr][i]));
   }
-  if (CPL == 4) reinterpret_cast<uint32_t *>(qi8 + row * D)[lane] = packed;
-  else reinterpret_cast<uint16_t *>(qi8 + row * D)[lane] = (uint16_t)packed;
-  if (lane == 0) sq[row] = s;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+    for (int rr = 0; rr < RPW; ++rr) amax[rr] = fmaxf(amax[rr], __shfl_xor_sync(0xffffffffu, amax[rr], o));
+  }
+#pragma unroll
+  for (int rr = 0; rr < RPW; ++rr) {
+    const long long row = row0 + rr;
+    if (row >= nrows) break;
+    const float s = amax[rr] == 0.f ? 1.f : __fdiv_rn(amax[rr], 127.f);
+    const float rcp = __frcp_rn(s);
+    uint32_t packed = 0;
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) {
+      const float c = fminf(fmaxf(rint_div(x[rr][i], s, rcp), -127.f), 127.f);
+      packed |= ((uint32_t)(int)c & 0xffu) << (8 * i);
+    }
+    if (CPL == 4) reinterpret_cast<uint32_t *>(qi8 + row * D)[lane] = packed;
+    else reinterpret_cast<uint16_t *>(qi8 + row * D)[lane] = (uint16_t)packed;
+    if (lane == 0) sq[row] = s;
+  }
 }
 
 // Position of the c-th remaining (non-vertical) key: c plus the number of
@@ -115,11 +155,12 @@ quant_k_remaining(const __nv_bfloat16 *__restrict__ k, const int32_t *__restrict
 #pragma unroll
   for (int w = 1; w < 8; ++w) amax = fmaxf(amax, red[w]);
   const float s = amax == 0.f ? 1.f : __fdiv_rn(amax, 127.f);
+  const float rcp = __frcp_rn(s);
   uint16_t *dst = reinterpret_cast<uint16_t *>(ki8 + ((size_t)bh * nr + c0) * D);
   for (int e = threadIdx.x; e < n * WPR; e += blockDim.x) {
     const uint32_t w = src[(size_t)pos[e / WPR] * WPR + e % WPR];
-    float c0f = fminf(fmaxf(rintf(__fdiv_rn(bf16_lo(w), s)), -127.f), 127.f);
-    float c1f = fminf(fmaxf(rintf(__fdiv_rn(bf16_hi(w), s)), -127.f), 127.f);
+    float c0f = fminf(fmaxf(rint_div(bf16_lo(w), s, rcp), -127.f), 127.f);
+    float c1f = fminf(fmaxf(rint_div(bf16_hi(w), s, rcp), -127.f), 127.f);
     dst[e] = (uint16_t)(((uint32_t)(int)c0f & 0xffu) | (((uint32_t)(int)c1f & 0xffu) << 8));
   }
   if (threadIdx.x == 0) sk[(size_t)bh * nblk + blk] = s;
@@ -492,7 +533,7 @@ cudaError_t quant_t(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const int32_
                     int Hq, int Hkv, int N, int k_vert, int8_t *qi8, float *sq, int8_t *ki8,
                     float *sk, cudaStream_t s) {
   const long long nrows = (long long)B * Hq * N;
-  quant_q_rows<D><<<(unsigned)((nrows + 7) / 8), 256, 0, s>>>(q, nrows, qi8, sq);
+  quant_q_rows<D><<<(unsigned)((nrows + 31) / 32), 256, 0, s>>>(q, nrows, qi8, sq);   // 8 warps x 4 rows
   const int nblk_r = (N - k_vert + TILE - 1) / TILE;
   if (nblk_r > 0)
     quant_k_remaining<D><<<dim3(nblk_r, B * Hkv), 256, 0, s>>>(k, idx, N, k_vert, nblk_r, ki8, sk);
