@@ -10,14 +10,17 @@
 // The signal of key j (per batch element and KV head) is the sum of the exact
 // causal softmax weights that the P most recent queries of the G query heads of
 // that KV head put on j.  Three kernels:
-//   1. probe_qk<STATS>: per (key chunk of 128, KV head) CTA, S = Q K^T on
-//      tensor cores (bf16 mma.sync, fp32 accumulate) for all G*P rows; writes
-//      per-(row, chunk) partial max / sum-of-exp.
+//   1. probe_qk<STATS>: per (key chunk of 256, KV head) CTA, S = Q K^T on
+//      tensor cores (bf16 mma.sync, fp32 accumulate) for all G*P rows; each
+//      warp keeps one 16-row tile's Q fragments while the chunk's two
+//      128-key halves stream through a double-buffered shared-memory ring
+//      (cp.async); writes per-(row, chunk) partial max / sum-of-exp.
 //   2. probe_row_stats: merges the partials into the row max m and sum Z.
 //   3. probe_qk<COLSUM>: recomputes S, p = exp(s - m) / Z, and sums each
 //      column over the G*P rows in a fixed order.
 //   4. probe_topk: radix select of the k-th largest score in [0, L - W) with
-//      (score desc, index asc) order, then an ordered compaction, so the list
+//      (score desc, index asc) order (keys staged in shared memory), then an
+//      ordered compaction over contiguous per-thread segments, so the list
 //      comes out ascending and ties go to the lower index.
 #include <float.h>
 
@@ -27,8 +30,10 @@
 namespace hq {
 namespace {
 
-constexpr int KC = 128;          // keys per CTA
-constexpr int PWARPS = 8;
+constexpr int KSUB = 128;        // keys per shared-memory stage
+constexpr int NSUB = 2;          // stages per CTA
+constexpr int KC = KSUB * NSUB;  // keys per CTA
+constexpr int PWARPS = 16;       // one 16-row tile of the probe rows per warp (more rows: loop)
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct ProbeArgs {
@@ -66,130 +71,185 @@ __device__ __forceinline__ void load_q_frag(const ProbeArgs &a, int b, int kh, i
   }
 }
 
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid) {
+  // 16-byte global -> shared copy; an invalid source reads as zeros
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
+
+template <int D>
+constexpr int probe_smem_bytes() {
+  return 2 * KSUB * D * 2 + PWARPS * KSUB * 4;   // K ring + per-warp column sums
+}
+
 template <int D, bool COLSUM>
-__global__ void __launch_bounds__(PWARPS * 32) probe_qk(ProbeArgs a) {
+__global__ void __launch_bounds__(PWARPS * 32, 1) probe_qk(ProbeArgs a) {
   constexpr int CH = D / 8;                    // 16-byte chunks per key row
-  __shared__ __align__(128) uint4 ks[KC * CH];  // K chunk, XOR-swizzled by key
-  __shared__ float colacc[PWARPS][KC];
+  extern __shared__ __align__(128) uint8_t psm[];
+  uint4 *ring = reinterpret_cast<uint4 *>(psm);                         // [2][KSUB * CH], XOR-swizzled by key
+  float *colacc = reinterpret_cast<float *>(psm + 2 * KSUB * D * 2);    // [PWARPS][KSUB]
   const int chunk = blockIdx.x, bh = blockIdx.y;
   const int b = bh / a.Hkv, kh = bh % a.Hkv;
-  const int j0 = chunk * KC;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  const uint4 *kg = reinterpret_cast<const uint4 *>(a.k + ((size_t)bh * a.L) * D);
-  for (int t = threadIdx.x; t < KC * CH; t += blockDim.x) {
-    const int key = t / CH, ch = t % CH;
-    uint4 val = make_uint4(0, 0, 0, 0);
-    if (j0 + key < a.L) val = __ldg(kg + (size_t)(j0 + key) * CH + ch);
-    ks[key * CH + (ch ^ (key & 7))] = val;
-  }
-  if (COLSUM)
-    for (int t = threadIdx.x; t < PWARPS * KC; t += blockDim.x) (&colacc[0][0])[t] = 0.f;
-  __syncthreads();
-
   const int r = lane >> 2, c = lane & 3;
+  const uint4 *kg = reinterpret_cast<const uint4 *>(a.k + ((size_t)bh * a.L) * D);
+  auto load_sub = [&](int sub) {
+    uint4 *dst = ring + (sub & 1) * KSUB * CH;
+    const int jb = chunk * KC + sub * KSUB;
+    for (int t = threadIdx.x; t < KSUB * CH; t += blockDim.x) {
+      const int key = t / CH, ch = t % CH;
+      const bool valid = jb + key < a.L;
+      cp_async16(smem_u32(&dst[key * CH + (ch ^ (key & 7))]), kg + (size_t)(valid ? jb + key : 0) * CH + ch, valid);
+    }
+    cp_async_commit();
+  };
+  load_sub(0);
+  if (NSUB > 1) load_sub(1);
+
   const int ntile_rows = (a.R + 15) / 16;
-  for (int rt = warp; rt < ntile_rows; rt += PWARPS) {
-    uint32_t qa[D / 16][4];
-    load_q_frag<D>(a, b, kh, rt * 16, qa);
-    float acc[KC / 8][4];
-#pragma unroll
-    for (int nt = 0; nt < KC / 8; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-#pragma unroll
-    for (int nt = 0; nt < KC / 8; ++nt) {
-#pragma unroll
-      for (int kp = 0; kp < D / 32; ++kp) {
-        const int key = nt * 8 + (lane & 7);
-        const int ch = kp * 4 + (lane >> 3);
-        uint32_t bf[4];
-        ldsm_x4(bf, smem_u32(&ks[key * CH + (ch ^ (key & 7))]));
-        mma_bf16_16816(acc[nt], qa[2 * kp], bf[0], bf[1]);
-        mma_bf16_16816(acc[nt], qa[2 * kp + 1], bf[2], bf[3]);
-      }
-    }
-    // Rows of this thread: rt*16 + r (+8).  Visible keys: j <= L - P + p.
-    int lastj[2];
-    bool valid[2];
-#pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
-      const int row = rt * 16 + r + hf * 8;
-      valid[hf] = row < a.R;
-      lastj[hf] = valid[hf] ? a.L - a.P + (row % a.P) : -1;
-    }
-    if (!COLSUM) {
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        float m = -FLT_MAX;
-#pragma unroll
-        for (int nt = 0; nt < KC / 8; ++nt)
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int j = j0 + nt * 8 + 2 * c + e;
-            if (j <= lastj[hf]) m = fmaxf(m, acc[nt][2 * hf + e] * a.scale_log2);
-          }
-        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-        float sum = 0.f;
-#pragma unroll
-        for (int nt = 0; nt < KC / 8; ++nt)
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int j = j0 + nt * 8 + 2 * c + e;
-            if (j <= lastj[hf]) sum += exp2f(acc[nt][2 * hf + e] * a.scale_log2 - m);
-          }
-        sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-        sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-        if (c == 0 && valid[hf]) {
-          const int row = rt * 16 + r + hf * 8;
-          a.partial[((size_t)bh * a.R + row) * a.nchunk + chunk] = make_float2(m, sum);
-        }
-      }
-    } else {
-      float2 st[2];
+  // With at most PWARPS row tiles, each warp's tile fragments load once and
+  // stay in registers; with more, every tile reloads them per stage.
+  const bool resident = ntile_rows <= PWARPS;
+  uint32_t qa[D / 16][4];
+  if (resident && warp < ntile_rows) load_q_frag<D>(a, b, kh, warp * 16, qa);
+
+  for (int sub = 0; sub < NSUB; ++sub) {
+    if (sub + 1 < NSUB) cp_async_wait<1>();
+    else cp_async_wait<0>();
+    __syncthreads();
+    const uint4 *ks = ring + (sub & 1) * KSUB * CH;
+    const int j0 = chunk * KC + sub * KSUB;
+    if (COLSUM)
+      for (int t = lane; t < KSUB; t += 32) colacc[warp * KSUB + t] = 0.f;
+    for (int rt = warp; rt < ntile_rows; rt += PWARPS) {
+      if (!resident) load_q_frag<D>(a, b, kh, rt * 16, qa);
+      const uint32_t(&q)[D / 16][4] = qa;
+      // Rows of this thread: rt*16 + r (+8).  Visible keys: j <= L - P + p.
+      int lastj[2];
+      bool valid[2];
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         const int row = rt * 16 + r + hf * 8;
-        st[hf] = valid[hf] ? a.stats[(size_t)bh * a.R + row] : make_float2(0.f, 0.f);
+        valid[hf] = row < a.R;
+        lastj[hf] = valid[hf] ? a.L - a.P + (row % a.P) : -1;
       }
+      float2 sx[2];                              // COLSUM: (max, 1/Z) of the two rows
+      if (COLSUM)
 #pragma unroll
-      for (int nt = 0; nt < KC / 8; ++nt) {
+        for (int hf = 0; hf < 2; ++hf) {
+          const int row = rt * 16 + r + hf * 8;
+          sx[hf] = valid[hf] ? a.stats[(size_t)bh * a.R + row] : make_float2(0.f, 0.f);
+        }
+      float pm[2] = {-FLT_MAX, -FLT_MAX}, ps[2] = {0.f, 0.f};   // STATS over the stage
+      // the stage's keys in two halves of 64 (32 accumulators at a time)
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int j = j0 + nt * 8 + 2 * c + e;
-          float col = 0.f;
+      for (int kh2 = 0; kh2 < 2; ++kh2) {
+        constexpr int NT = KSUB / 16;            // 8-key MMA tiles per half
+        float acc[NT][4];
 #pragma unroll
-          for (int hf = 0; hf < 2; ++hf)
-            if (j <= lastj[hf]) col += exp2f(acc[nt][2 * hf + e] * a.scale_log2 - st[hf].x) * st[hf].y;
-          col += __shfl_xor_sync(0xffffffffu, col, 4);
-          col += __shfl_xor_sync(0xffffffffu, col, 8);
-          col += __shfl_xor_sync(0xffffffffu, col, 16);
-          if (r == 0) colacc[warp][nt * 8 + 2 * c + e] += col;
+        for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+          for (int kp = 0; kp < D / 32; ++kp) {
+            const int key = kh2 * 64 + nt * 8 + (lane & 7);
+            const int ch = kp * 4 + (lane >> 3);
+            uint32_t bf[4];
+            ldsm_x4(bf, smem_u32(&ks[key * CH + (ch ^ (key & 7))]));
+            mma_bf16_16816(acc[nt], q[2 * kp], bf[0], bf[1]);
+            mma_bf16_16816(acc[nt], q[2 * kp + 1], bf[2], bf[3]);
+          }
+        }
+        const int jh = j0 + kh2 * 64;
+        if (!COLSUM) {
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            float m = -FLT_MAX;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const int j = jh + nt * 8 + 2 * c + e;
+                if (j <= lastj[hf]) m = fmaxf(m, acc[nt][2 * hf + e] * a.scale_log2);
+              }
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+            float sum = 0.f;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const int j = jh + nt * 8 + 2 * c + e;
+                if (j <= lastj[hf]) sum += exp2f(acc[nt][2 * hf + e] * a.scale_log2 - m);
+              }
+            sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+            sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+            // merge with the stage's first half
+            const float mn = fmaxf(pm[hf], m);
+            ps[hf] = (pm[hf] == -FLT_MAX ? 0.f : ps[hf] * exp2f(pm[hf] - mn)) +
+                     (m == -FLT_MAX ? 0.f : sum * exp2f(m - mn));
+            pm[hf] = mn;
+          }
+        } else {
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int j = jh + nt * 8 + 2 * c + e;
+              float col = 0.f;
+#pragma unroll
+              for (int hf = 0; hf < 2; ++hf)
+                if (j <= lastj[hf]) col += exp2f(acc[nt][2 * hf + e] * a.scale_log2 - sx[hf].x) * sx[hf].y;
+              col += __shfl_xor_sync(0xffffffffu, col, 4);
+              col += __shfl_xor_sync(0xffffffffu, col, 8);
+              col += __shfl_xor_sync(0xffffffffu, col, 16);
+              if (r == 0) colacc[warp * KSUB + kh2 * 64 + nt * 8 + 2 * c + e] += col;
+            }
+          }
         }
       }
-    }
-  }
-  if (COLSUM) {
-    __syncthreads();
-    for (int t = threadIdx.x; t < KC; t += blockDim.x) {
-      float s = 0.f;
+      if (!COLSUM)
 #pragma unroll
-      for (int w = 0; w < PWARPS; ++w) s += colacc[w][t];
-      if (j0 + t < a.L) a.score[(size_t)bh * a.L + j0 + t] = s;
+        for (int hf = 0; hf < 2; ++hf)
+          if (c == 0 && valid[hf] && j0 < a.L) {   // one partial per (row, 128-key stage)
+            const int row = rt * 16 + r + hf * 8;
+            a.partial[((size_t)bh * a.R + row) * a.nchunk + chunk * NSUB + sub] = make_float2(pm[hf], ps[hf]);
+          }
     }
+    __syncthreads();   // every warp is done with this stage's keys (and column sums)
+    if (COLSUM)
+      for (int t = threadIdx.x; t < KSUB; t += blockDim.x) {
+        float sm = 0.f;
+#pragma unroll
+        for (int w = 0; w < PWARPS; ++w) sm += colacc[w * KSUB + t];
+        if (j0 + t < a.L) a.score[(size_t)bh * a.L + j0 + t] = sm;
+      }
+    if (sub + 2 < NSUB) load_sub(sub + 2);
+    if (COLSUM) __syncthreads();    // column sums read before the next stage clears them
   }
 }
 
-// Row max / 1/Z from the per-chunk partials (log2 domain).
+// Row max / 1/Z from the per-stage partials (log2 domain): one warp per row,
+// lanes over the partials, merged in a fixed order.
 __global__ void probe_row_stats(const float2 *__restrict__ partial, float2 *__restrict__ stats,
                                 int nrows, int nchunk) {
-  const int row = blockIdx.x * blockDim.x + threadIdx.x;
+  const int row = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
   if (row >= nrows) return;
   const float2 *pr = partial + (size_t)row * nchunk;
   float m = -FLT_MAX;
-  for (int c = 0; c < nchunk; ++c) m = fmaxf(m, pr[c].x);
+  for (int c = lane; c < nchunk; c += 32) m = fmaxf(m, pr[c].x);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   float z = 0.f;
-  for (int c = 0; c < nchunk; ++c) z += pr[c].y * exp2f(pr[c].x - m);
-  stats[row] = make_float2(m, 1.0f / z);
+  for (int c = lane; c < nchunk; c += 32) z += pr[c].y * exp2f(pr[c].x - m);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+  if (lane == 0) stats[row] = make_float2(m, 1.0f / z);
 }
 
 // ---------------------------------------------------------------------------
@@ -231,8 +291,15 @@ __device__ int block_exclusive_scan(int v, int *tmp, int &excl) {
   return total;
 }
 
+constexpr int TK_STAGE = 32768;   // candidates staged in shared memory (more: read from L2)
+
+// Staged key of candidate j: one pad word per 32, so that the per-thread
+// segment walks below hit 32 different banks.
+__device__ __forceinline__ int tk_slot(int j) { return j + (j >> 5); }
+
 __global__ void __launch_bounds__(TK_THREADS)
 probe_topk(const float *__restrict__ score, int L, int ncand, int k, int32_t *__restrict__ idx) {
+  extern __shared__ uint32_t skey[];                 // staged keys (tk_slot layout)
   __shared__ int hist[256];
   __shared__ int tmp[32];
   __shared__ uint32_t sel_prefix, sel_mask;
@@ -241,19 +308,28 @@ probe_topk(const float *__restrict__ score, int L, int ncand, int k, int32_t *__
   const float *s = score + (size_t)bh * L;
   int32_t *out = idx + (size_t)bh * k;
   if (k == 0) return;
+  const bool staged = ncand <= TK_STAGE;
+  auto key_of = [&](int j) -> uint32_t { return staged ? skey[tk_slot(j)] : score_key(__ldg(s + j)); };
+  if (staged)
+    for (int j = threadIdx.x; j < ncand; j += blockDim.x) skey[tk_slot(j)] = score_key(s[j]);
   if (threadIdx.x == 0) {
     sel_prefix = 0;
     sel_mask = 0;
     remain = k;
   }
-  // Radix select of the k-th largest key, 8 bits at a time from the top.
+  // Radix select of the k-th largest key, 8 bits at a time from the top; the
+  // histogram atomics are aggregated per warp over lanes with the same bin.
   for (int shift = 24; shift >= 0; shift -= 8) {
     for (int t = threadIdx.x; t < 256; t += blockDim.x) hist[t] = 0;
     __syncthreads();
     const uint32_t pre = sel_prefix, msk = sel_mask;
-    for (int j = threadIdx.x; j < ncand; j += blockDim.x) {
-      const uint32_t key = score_key(s[j]);
-      if ((key & msk) == pre) atomicAdd(&hist[(key >> shift) & 0xff], 1);
+    const int jend = (ncand + blockDim.x - 1) / blockDim.x * blockDim.x;   // whole warps iterate
+    for (int j = threadIdx.x; j < jend; j += blockDim.x) {
+      const uint32_t key = j < ncand ? key_of(j) : 0u;
+      const bool in = j < ncand && (key & msk) == pre;
+      const int bin = in ? (int)((key >> shift) & 0xff) : -1;
+      const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+      if (in && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
     }
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -270,34 +346,62 @@ probe_topk(const float *__restrict__ score, int L, int ncand, int k, int32_t *__
   }
   const uint32_t thr = sel_prefix;  // key of the k-th largest score
   const int take_eq = remain;       // equal keys to take, lowest indices first
-  int out_base = 0, eq_base = 0;
-  for (int base = 0; base < ncand; base += blockDim.x) {
-    const int j = base + threadIdx.x;
-    uint32_t key = 0;
-    if (j < ncand) key = score_key(s[j]);
-    const int gt = (j < ncand) && key > thr;
-    const int eq = (j < ncand) && key == thr;
-    int eq_excl;
-    const int eq_tot = block_exclusive_scan(eq, tmp, eq_excl);
-    const int take = gt || (eq && (eq_base + eq_excl) < take_eq);
-    int pos;
-    const int tot = block_exclusive_scan(take, tmp, pos);
-    if (take) out[out_base + pos] = j;
-    out_base += tot;
-    eq_base += eq_tot;
+  // Ordered compaction over contiguous per-thread segments: the keys equal to
+  // the threshold that come before a segment decide how many of its equal
+  // keys are taken; a second scan places every taken index.
+  const int seg = (ncand + blockDim.x - 1) / blockDim.x;
+  const int jb = min((int)threadIdx.x * seg, ncand), je = min(jb + seg, ncand);
+  int n_eq = 0;
+  for (int j = jb; j < je; ++j) n_eq += key_of(j) == thr;
+  int eq_before;
+  block_exclusive_scan(n_eq, tmp, eq_before);
+  int n_take = 0;
+  {
+    int e = eq_before;
+    for (int j = jb; j < je; ++j) {
+      const uint32_t key = key_of(j);
+      if (key > thr) ++n_take;
+      else if (key == thr) n_take += (e++ < take_eq);
+    }
+  }
+  int pos;
+  block_exclusive_scan(n_take, tmp, pos);
+  {
+    int e = eq_before;
+    for (int j = jb; j < je; ++j) {
+      const uint32_t key = key_of(j);
+      const bool take = key > thr || (key == thr && e++ < take_eq);
+      if (take) out[pos++] = j;
+    }
   }
 }
 
 template <int D>
 cudaError_t launch_probe_t(ProbeArgs a, int nbh, int k_vert, int window, int32_t *idx,
                            cudaStream_t s) {
-  dim3 grid(a.nchunk, nbh);
-  probe_qk<D, false><<<grid, PWARPS * 32, 0, s>>>(a);
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(probe_qk<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, probe_smem_bytes<D>()) != cudaSuccess ||
+        cudaFuncSetAttribute(probe_qk<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, probe_smem_bytes<D>()) != cudaSuccess)
+      return cudaErrorInvalidValue;
+    attr = true;
+  }
+  dim3 grid((a.L + KC - 1) / KC, nbh);
+  probe_qk<D, false><<<grid, PWARPS * 32, probe_smem_bytes<D>(), s>>>(a);
   const int nrows = nbh * a.R;
-  probe_row_stats<<<(nrows + 255) / 256, 256, 0, s>>>(a.partial, const_cast<float2 *>(a.stats),
+  probe_row_stats<<<(nrows + 7) / 8, 256, 0, s>>>(a.partial, const_cast<float2 *>(a.stats),   // a warp per row
                                                       nrows, a.nchunk);
-  probe_qk<D, true><<<grid, PWARPS * 32, 0, s>>>(a);
-  probe_topk<<<nbh, TK_THREADS, 0, s>>>(a.score, a.L, a.L - window, k_vert, idx);
+  probe_qk<D, true><<<grid, PWARPS * 32, probe_smem_bytes<D>(), s>>>(a);
+  const int ncand = a.L - window;
+  const size_t tk_smem = ncand <= TK_STAGE ? (size_t)(ncand + (ncand >> 5) + 1) * 4 : 0;
+  static bool tk_attr = false;
+  if (!tk_attr) {
+    if (cudaFuncSetAttribute(probe_topk, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (TK_STAGE + TK_STAGE / 32 + 1) * 4) != cudaSuccess)
+      return cudaErrorInvalidValue;
+    tk_attr = true;
+  }
+  probe_topk<<<nbh, TK_THREADS, tk_smem, s>>>(a.score, a.L, ncand, k_vert, idx);
   return cudaGetLastError();
 }
 
@@ -306,7 +410,7 @@ cudaError_t launch_probe_t(ProbeArgs a, int nbh, int k_vert, int window, int32_t
 size_t probe_ws_bytes(int B, int Hq, int Hkv, int P, int L, int D) {
   (void)D;
   const size_t nbh = (size_t)B * Hkv, R = (size_t)(Hq / Hkv) * P;
-  const size_t nchunk = (L + KC - 1) / KC;
+  const size_t nchunk = (L + KSUB - 1) / KSUB;    // partials per row: one per 128-key stage
   size_t off = kWsHeader;
   off = align_up(off + nbh * R * nchunk * sizeof(float2), 256);  // partials
   off = align_up(off + nbh * R * sizeof(float2), 256);           // stats
@@ -328,7 +432,7 @@ cudaError_t launch_probe(const __nv_bfloat16 *q_probe, int64_t q_head_stride,
   a.L = L;
   a.G = Hq / Hkv;
   a.R = a.G * P;
-  a.nchunk = (L + KC - 1) / KC;
+  a.nchunk = (L + KSUB - 1) / KSUB;
   a.scale_log2 = scale * kLog2e;
   const size_t nbh = (size_t)B * Hkv;
   size_t off = kWsHeader;
