@@ -168,30 +168,50 @@ quant_k_remaining(const __nv_bfloat16 *__restrict__ k, const int32_t *__restrict
 
 // bf16 V -> fp16 V (exact for |v| in the fp16 normal range), both in position
 // order (window tiles) and compacted to the remaining keys (low-bit tiles).
-// One warp per (b, kv head, position).
+// Eight consecutive positions of one (b, kv head) per warp task: one binary
+// search finds the verticals before the chunk, a ballot over the next index
+// entries marks the chunk's own, and all eight rows load before any store.
 template <int D>
-__global__ void v_prep(const __nv_bfloat16 *__restrict__ v, const int32_t *__restrict__ idx,
-                       int nbh, int N, int k_vert, __half *__restrict__ vh,
-                       __half *__restrict__ vc) {
+__global__ void __launch_bounds__(256)
+v_prep(const __nv_bfloat16 *__restrict__ v, const int32_t *__restrict__ idx, int nbh, int N,
+       int k_vert, __half *__restrict__ vh, __half *__restrict__ vc) {
   constexpr int W32 = D / 64;                                    // 32-bit words per lane
+  constexpr int PCH = 8;
   const int lane = threadIdx.x & 31;
-  const long long total = (long long)nbh * N;
+  const int cpb = (N + PCH - 1) / PCH;
+  const long long ntask = (long long)nbh * cpb;
   const int nr = N - k_vert;
-  for (long long wi = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); wi < total;
-       wi += (long long)gridDim.x * (blockDim.x / 32)) {
-    const int bh = (int)(wi / N), j = (int)(wi % N);
+  for (long long task = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); task < ntask;
+       task += (long long)gridDim.x * (blockDim.x / 32)) {
+    const int bh = (int)(task / cpb), j0 = (int)(task % cpb) * PCH;
     const int32_t *id = idx + (size_t)bh * k_vert;
-    const int cnt = upper_bound_i32(id, k_vert, j);              // verticals <= j
-    const bool vert = cnt > 0 && __ldg(id + cnt - 1) == j;
-    const uint32_t *src = reinterpret_cast<const uint32_t *>(v + wi * D) + lane * W32;
-    __half2 *dh = reinterpret_cast<__half2 *>(vh + wi * D) + lane * W32;
-    __half2 *dc = reinterpret_cast<__half2 *>(vc + ((size_t)bh * nr + (j - cnt)) * D) + lane * W32;
+    const int cnt0 = j0 > 0 ? upper_bound_i32(id, k_vert, j0 - 1) : 0;   // verticals before j0
+    const int e = cnt0 + (lane & (PCH - 1));
+    const int ve = (lane < PCH && e < k_vert) ? __ldg(id + e) : INT_MAX;
+    const uint32_t vbit = (ve >= j0 && ve < j0 + PCH) ? 1u << (ve - j0) : 0u;
+    const uint32_t vbits = __reduce_or_sync(0xffffffffu, vbit);
+    uint32_t w[PCH][W32];
 #pragma unroll
-    for (int i = 0; i < W32; ++i) {
-      const uint32_t w = src[i];
-      const __half2 x = __floats2half2_rn(bf16_lo(w), bf16_hi(w));
-      dh[i] = x;
-      if (!vert) dc[i] = x;
+    for (int p = 0; p < PCH; ++p) {
+      const int j = j0 + p < N ? j0 + p : N - 1;
+      const uint32_t *src = reinterpret_cast<const uint32_t *>(v + ((size_t)bh * N + j) * D) + lane * W32;
+#pragma unroll
+      for (int i = 0; i < W32; ++i) w[p][i] = __ldg(src + i);
+    }
+#pragma unroll
+    for (int p = 0; p < PCH; ++p) {
+      const int j = j0 + p;
+      if (j >= N) break;
+      const bool vert = (vbits >> p) & 1u;
+      const int rank = j - cnt0 - __popc(vbits & ((1u << p) - 1u));       // among the remaining keys
+      __half2 *dh = reinterpret_cast<__half2 *>(vh + ((size_t)bh * N + j) * D) + lane * W32;
+      __half2 *dc = reinterpret_cast<__half2 *>(vc + ((size_t)bh * nr + rank) * D) + lane * W32;
+#pragma unroll
+      for (int i = 0; i < W32; ++i) {
+        const __half2 x = __floats2half2_rn(bf16_lo(w[p][i]), bf16_hi(w[p][i]));
+        dh[i] = x;
+        if (!vert && rank >= 0 && rank < nr) dc[i] = x;
+      }
     }
   }
 }
@@ -555,7 +575,7 @@ cudaError_t prefill_t(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    long long blocks = ((long long)nbh * N + 7) / 8;
+    long long blocks = ((long long)nbh * ((N + 7) / 8) + 7) / 8;   // 8 warps x 8 positions per block
     if (blocks > 8LL * sms) blocks = 8LL * sms;
     v_prep<D><<<(unsigned)blocks, 256, 0, s>>>(v, idx, nbh, N, k_vert, w.vh, w.vc);
   }

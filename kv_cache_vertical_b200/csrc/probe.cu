@@ -310,8 +310,22 @@ probe_topk(const float *__restrict__ score, int L, int ncand, int k, int32_t *__
   if (k == 0) return;
   const bool staged = ncand <= TK_STAGE;
   auto key_of = [&](int j) -> uint32_t { return staged ? skey[tk_slot(j)] : score_key(__ldg(s + j)); };
-  if (staged)
-    for (int j = threadIdx.x; j < ncand; j += blockDim.x) skey[tk_slot(j)] = score_key(s[j]);
+  if (staged) {
+    // eight loads in flight per thread (a lone CTA per pair: latency-bound)
+    for (int j0 = threadIdx.x; j0 < ncand; j0 += 8 * blockDim.x) {
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int j = j0 + u * blockDim.x;
+        v[u] = j < ncand ? __ldg(s + j) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int j = j0 + u * blockDim.x;
+        if (j < ncand) skey[tk_slot(j)] = score_key(v[u]);
+      }
+    }
+  }
   if (threadIdx.x == 0) {
     sel_prefix = 0;
     sel_mask = 0;
