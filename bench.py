@@ -242,13 +242,63 @@ def run_hq(args, rank, world, dev):
     h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h))
     d2h = out_p.numel() * 4 + out_d.numel() * 4
 
+    loop = decode_loop(H, w, q, k, v, q_dec, dev, stream, world)
+
     idx_np = idx.cpu().numpy()
     dbytes = decode_bytes(B, Hq, Hkv, D, cache.n_lo, cache.n_hi, w.bits)
     i8_ops, bf_flops = prefill_work(idx_np, N, W, D, Hq, Hkv)
     clocks = clk.summary()
     return dict(per=per, total_ms=max_over_ranks(total_ms / args.steps, world, dev), dbytes=dbytes,
                 i8=i8_ops, bf=bf_flops, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, clocks=clocks,
-                kpad=(kv + 63) // 64 * 64, w=w)
+                kpad=(kv + 63) // 64 * 64, w=w, loop=loop)
+
+
+def decode_loop(H, w, q, k, v, q_dec, dev, stream, world, T=64):
+    """Token-by-token decode after a prompt of N - T tokens: per token, the
+    cache maintenance call (token enters the window ring, the oldest window
+    token is quantized into the low segment) and then the decode attention.
+    Measured after the timed steps, L2 not flushed (consecutive tokens)."""
+    B, Hq, Hkv, D, N, W = w.B, w.Hq, w.Hkv, w.D, w.L, w.window
+    N0 = N - T
+    kv0 = int(w.frac * N0)
+    k0, v0 = k[:, :, :N0].contiguous(), v[:, :, :N0].contiguous()
+    idx0 = torch.empty(B, Hkv, kv0, dtype=torch.int32, device=dev)
+    ws_probe = H.workspace(H.hq_probe_workspace_size(B, Hq, Hkv, 64, N0, D), dev)
+    H.hq_probe_vertical(q[:, :, N0 - 64:N0], N * D, k0, B, Hq, Hkv, 64, N0, D, W, kv0, 0.0, idx0,
+                        None, ws_probe)
+    n_lo0 = N0 - W - kv0
+    cache = H.KVCache.empty(B, Hkv, N0, D, W, kv0, w.bits, dev, with_pos=False, lo_cap=n_lo0 + T)
+    H.hq_pack_kv(k0, v0, idx0, B, Hkv, N0, D, W, kv0, w.bits, 32, cache, None)
+    k_new = k[:, :, N0:].permute(2, 0, 1, 3).contiguous()      # [T, B, Hkv, D]
+    v_new = v[:, :, N0:].permute(2, 0, 1, 3).contiguous()
+    ws_bytes = max(H.hq_decode_workspace_size(B, Hq, Hkv, D, n_lo0 + i, cache.n_hi, w.bits)
+                   for i in range(1, T + 1))
+    ws = H.workspace(ws_bytes, dev)
+    out = torch.empty(B, Hq, D, dtype=torch.float32, device=dev)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(T)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    # hold the stream for ~20 ms so that all T tokens are queued before the
+    # first one runs: the times below are then the device's, not the host's
+    # (queued_ahead reports whether that held)
+    torch.cuda._sleep(40_000_000)
+    for i in range(T):
+        e = evs[i]
+        e[0].record(stream)
+        H.hq_kv_append(k_new[i], v_new[i], B, Hkv, D, N0 + i, W, kv0, cache)
+        cache.n_lo += 1
+        e[1].record(stream)
+        H.hq_decode_attn(q_dec, cache, B, Hq, Hkv, D, 0.0, out, None, ws)
+        e[2].record(stream)
+    ahead = not evs[0][0].query()          # the first token had not run when the last was queued
+    torch.cuda.synchronize(dev)
+    app = [e[0].elapsed_time(e[1]) * 1e3 for e in evs]
+    dec = [e[1].elapsed_time(e[2]) * 1e3 for e in evs]
+    tot = evs[0][0].elapsed_time(evs[-1][2]) * 1e3 / T
+    return {"tokens": T, "context": [N0 + 1, N], "append_us": max_over_ranks(float(np.median(app)), world, dev),
+            "decode_us": max_over_ranks(float(np.median(dec)), world, dev),
+            "us_per_token": max_over_ranks(tot, world, dev), "launches_per_token": 2,
+            "l2": "not flushed", "queued_ahead": bool(ahead)}
 
 
 def barrier(world):
@@ -392,6 +442,8 @@ def main():
                    "us": per["decode"] * 1e3, "peak_src": pk["src"] + " (copy bandwidth)",
                    "frac_of_8TBs": dec_tbs / 8.0},
         "per_call_ms": {n: per[n] for n in ("probe", "prefill", "pack", "decode")},
+        # token-by-token decode after the timed steps: cache maintenance + attention
+        "decode_loop": r["loop"],
         "e2e": {"value": r["dbytes"] / (r["e2e_ms"] * 1e-3) / 1e12 * world, "unit": "TB/s",
                 "ms_per_step": r["e2e_ms"], "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"],

@@ -76,15 +76,21 @@ int hq_version(void);
  * Hybrid KV cache (decode).  Plain struct of caller-owned device buffers.
  * With L cached tokens, window W and k vertical columns per (b, kv head):
  *   n_lo = L - W - k low-bit rows, n_hi = k + W bf16 rows.
- *   k_codes, v_codes : u8  [B, Hkv, n_lo, D * bits / 8].  4-bit codes are
- *                      packed two per byte, even channel in the low nibble.
- *   k_sz, v_sz       : f16 [B, Hkv, n_lo, D / group, 2], (scale, zero) of each
+ *   k_codes, v_codes : u8  [B, Hkv, C, D * bits / 8], C = the low-row
+ *                      capacity (lo_cap, or n_lo when lo_cap is 0); rows
+ *                      0..n_lo-1 of each (b, kv head) are in use.  4-bit codes
+ *                      are packed two per byte, even channel in the low nibble.
+ *   k_sz, v_sz       : f16 [B, Hkv, C, D / group, 2], (scale, zero) of each
  *                      group; dequantized value = scale * code + zero.
  *   k_hi, v_hi       : bf16 [B, Hkv, n_hi, D]; rows 0..k-1 are the vertical
  *                      columns in ascending position order, rows k..k+W-1 the
- *                      window (positions L-W .. L-1).
- *   lo_pos           : i32 [B, Hkv, n_lo] position of each low row (ascending),
+ *                      window as a ring keyed by position: window position p
+ *                      (L-W <= p < L) sits in row k + p mod W.
+ *   lo_pos           : i32 [B, Hkv, C] position of each low row (ascending),
  *                      or NULL when not wanted.
+ *   lo_cap           : low rows allocated per (b, kv head); 0 means n_lo.
+ *                      Spare rows let hq_kv_append grow the low segment in
+ *                      place during decode.  Rows n_lo..C-1 are never read.
  * All pointers must be 16-byte aligned.  The low rows are stored in ascending
  * position order, with no copy of the vertical rows: attention does not depend
  * on key order, and storing a vertical row only once is what gives the
@@ -102,6 +108,7 @@ typedef struct {
     int n_hi;
     int bits;
     int group;
+    int lo_cap;
 } hq_kv_cache;
 
 /*
@@ -201,6 +208,35 @@ hq_status hq_decode_attn(const void *q, const hq_kv_cache *cache, int B, int Hq,
 hq_status hq_decode_attn_static(const void *q, const hq_kv_cache *cache, int B, int Hq, int Hkv,
                                 int D, float softmax_scale, float *out, float *lse_out,
                                 void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* Decode cache maintenance (wiki summary, TL;DR: in decode the same rule    */
+/* is a KV cache compression policy; blog, "What hybrid-precision attention  */
+/* changes": the decode cache is mostly low-bit, selected positions high).   */
+/* ------------------------------------------------------------------------ */
+/*
+ * Append token L (the newly decoded position; the cache holds positions
+ * 0..L-1) to every (b, kv head) of the cache, before the decode attention of
+ * that token.  The pages do not spell the step out; the library's reading:
+ * the vertical set chosen at prefill stays fixed, and the window stays the W
+ * most recent positions.  So position L - W leaves the window: its bf16 rows
+ * (window row k_vert + L mod W) are quantized exactly as hq_pack_kv
+ * quantizes a low row and written as low row n_lo with lo_pos = L - W; then
+ * token L's bf16 K/V take that window row.  With window == 0 token L itself
+ * becomes low row n_lo (lo_pos = L).  A cache packed from L tokens and given
+ * tokens L..L+t-1 this way is bit-identical to the cache packed from L + t
+ * tokens with the same vertical set.
+ *   k_new, v_new : bf16 [B, Hkv, D], token L's key and value.
+ *   cache        : must satisfy n_lo == L - window - k_vert, n_hi == k_vert +
+ *                  window and n_lo < lo_cap (room for one more low row).
+ *                  The struct is only read: after the call the caller sets
+ *                  cache->n_lo to n_lo + 1.
+ * One launch, no workspace, no device-side checks (everything is checked on
+ * the host).  Stream-ordered: a decode attention issued after it on the same
+ * stream sees the new token.
+ */
+hq_status hq_kv_append(const void *k_new, const void *v_new, int B, int Hkv, int D, int L,
+                       int window, int k_vert, const hq_kv_cache *cache, void *stream);
 
 /* ------------------------------------------------------------------------ */
 /* Hybrid-precision prefill (abstract: Prefill stage keeps vertical-line     */

@@ -24,6 +24,8 @@ hq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? HQ_OK : HQ_ERR_
 
 uint32_t *status_word(void *ws) { return ws ? reinterpret_cast<uint32_t *>(ws) : nullptr; }
 
+bool lo_cap_ok(const hq_kv_cache &c) { return c.lo_cap == 0 || c.lo_cap >= c.n_lo; }
+
 }  // namespace
 
 namespace hq {
@@ -33,7 +35,7 @@ hq_status check_decode_args(const void *q, const hq_kv_cache *cache, int B, int 
                             int D, const float *out) {
   if (!q || !cache || !out) return HQ_ERR_INVALID_ARG;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || cache->n_lo < 0 || cache->n_hi < 0 ||
-      cache->n_lo + cache->n_hi <= 0)
+      cache->n_lo + cache->n_hi <= 0 || !lo_cap_ok(*cache))
     return HQ_ERR_INVALID_ARG;
   if ((D != 64 && D != 128) || !supported_G(Hq, Hkv) || (cache->bits != 4 && cache->bits != 8) ||
       cache->group != 32)
@@ -109,7 +111,8 @@ hq_status hq_pack_kv(const void *k, const void *v, const int32_t *idx, int B, in
     return HQ_ERR_INVALID_ARG;
   if ((D != 64 && D != 128) || (bits != 4 && bits != 8) || group != 32) return HQ_ERR_UNSUPPORTED;
   const int n_lo = L - window - k_vert, n_hi = k_vert + window;
-  if (out->n_lo != n_lo || out->n_hi != n_hi || out->bits != bits || out->group != group)
+  if (out->n_lo != n_lo || out->n_hi != n_hi || out->bits != bits || out->group != group ||
+      !lo_cap_ok(*out))
     return HQ_ERR_INVALID_ARG;
   if ((n_lo > 0 && (!out->k_codes || !out->v_codes || !out->k_sz || !out->v_sz)) ||
       (n_hi > 0 && (!out->k_hi || !out->v_hi)))
@@ -121,6 +124,26 @@ hq_status hq_pack_kv(const void *k, const void *v, const int32_t *idx, int B, in
   return cuda_status(launch_pack((const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, idx, B, Hkv,
                                  L, D, window, k_vert, bits, *out, status_word(ws),
                                  (cudaStream_t)stream));
+}
+
+hq_status hq_kv_append(const void *k_new, const void *v_new, int B, int Hkv, int D, int L,
+                       int window, int k_vert, const hq_kv_cache *cache, void *stream) {
+  if (!k_new || !v_new || !cache) return HQ_ERR_INVALID_ARG;
+  if (B <= 0 || Hkv <= 0 || window < 0 || k_vert < 0 || L < window + k_vert) return HQ_ERR_INVALID_ARG;
+  if ((D != 64 && D != 128) || (cache->bits != 4 && cache->bits != 8) || cache->group != 32)
+    return HQ_ERR_UNSUPPORTED;
+  if (cache->n_lo != L - window - k_vert || cache->n_hi != k_vert + window ||
+      cache->lo_cap <= cache->n_lo)
+    return HQ_ERR_INVALID_ARG;
+  if (!cache->k_codes || !cache->v_codes || !cache->k_sz || !cache->v_sz ||
+      (window > 0 && (!cache->k_hi || !cache->v_hi)))
+    return HQ_ERR_INVALID_ARG;
+  const void *ptrs[] = {k_new, v_new, cache->k_codes, cache->v_codes, cache->k_sz, cache->v_sz,
+                        cache->k_hi, cache->v_hi};
+  for (const void *p : ptrs)
+    if (p && !aligned16(p)) return HQ_ERR_INVALID_ARG;
+  return cuda_status(launch_kv_append((const __nv_bfloat16 *)k_new, (const __nv_bfloat16 *)v_new,
+                                      B, Hkv, D, L, window, k_vert, *cache, (cudaStream_t)stream));
 }
 
 size_t hq_decode_workspace_size(int B, int Hq, int Hkv, int D, int n_lo, int n_hi, int bits) {
@@ -135,7 +158,7 @@ hq_status hq_decode_attn(const void *q, const hq_kv_cache *cache, int B, int Hq,
                          size_t ws_bytes, void *stream) {
   if (!q || !cache || !out) return HQ_ERR_INVALID_ARG;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || cache->n_lo < 0 || cache->n_hi < 0 ||
-      cache->n_lo + cache->n_hi <= 0)
+      cache->n_lo + cache->n_hi <= 0 || !lo_cap_ok(*cache))
     return HQ_ERR_INVALID_ARG;
   if ((D != 64 && D != 128) || !supported_G(Hq, Hkv) || (cache->bits != 4 && cache->bits != 8) ||
       cache->group != 32)

@@ -28,7 +28,7 @@ struct DecodeArgs {
   const uint8_t *k_codes, *v_codes;
   const __half2 *k_sz, *v_sz;
   const __nv_bfloat16 *k_hi, *v_hi;
-  int Hq, Hkv, G, n_lo, n_hi, nsplit;
+  int Hq, Hkv, G, n_lo, n_hi, lo_cap, nsplit;
   float scale_log2;
   float *part_o;     // [B*Hq, nsplit, D]
   float2 *part_ml;   // [B*Hq, nsplit]
@@ -37,11 +37,11 @@ struct DecodeArgs {
 // Channels lane*CPL .. lane*CPL+CPL-1 of one cached row, as fp32.
 template <int D, int BITS>
 __device__ __forceinline__ void load_row(const uint8_t *codes, const __half2 *sz,
-                                         const __nv_bfloat16 *hi, int n_lo, int n_hi, size_t bh,
-                                         int t, int lane, float (&x)[D / 32]) {
+                                         const __nv_bfloat16 *hi, int n_lo, int n_hi, int lo_cap,
+                                         size_t bh, int t, int lane, float (&x)[D / 32]) {
   constexpr int CPL = D / 32;
   if (t < n_lo) {
-    const size_t row = bh * n_lo + t;
+    const size_t row = bh * lo_cap + t;
     const float2 s_z = __half22float2(sz[row * (D / 32) + (lane * CPL) / 32]);
     uint32_t c[CPL];
     const uint8_t *cr = codes + row * (D * BITS / 8);
@@ -99,8 +99,8 @@ __global__ void __launch_bounds__(DWARPS * 32) decode_split(DecodeArgs a) {
   }
   for (int t = t0 + warp; t < t1; t += DWARPS) {
     float kx[CPL], vx[CPL];
-    load_row<D, BITS>(a.k_codes, a.k_sz, a.k_hi, a.n_lo, a.n_hi, (size_t)bh, t, lane, kx);
-    load_row<D, BITS>(a.v_codes, a.v_sz, a.v_hi, a.n_lo, a.n_hi, (size_t)bh, t, lane, vx);
+    load_row<D, BITS>(a.k_codes, a.k_sz, a.k_hi, a.n_lo, a.n_hi, a.lo_cap, (size_t)bh, t, lane, kx);
+    load_row<D, BITS>(a.v_codes, a.v_sz, a.v_hi, a.n_lo, a.n_hi, a.lo_cap, (size_t)bh, t, lane, vx);
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       float s = 0.f;
@@ -231,6 +231,7 @@ cudaError_t launch_decode(const __nv_bfloat16 *q, const hq_kv_cache &c, int B, i
   a.G = Hq / Hkv;
   a.n_lo = c.n_lo;
   a.n_hi = c.n_hi;
+  a.lo_cap = lo_rows(c);
   const int nbh = B * Hkv;
   a.nsplit = choose_nsplit(nbh, c.n_lo + c.n_hi);
   a.scale_log2 = scale * kLog2e;

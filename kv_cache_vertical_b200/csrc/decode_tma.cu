@@ -937,23 +937,27 @@ cudaError_t launch_tg(const DecArgs &a0, const hq_kv_cache &c, int nbh, cudaStre
   // encoding.
   struct MapCache {
     const void *p[6];
-    int n_lo, n_hi, nbh;
+    int n_lo, n_hi, nbh, lo_cap;
     bool valid;
     CUtensorMap m[6];
   };
   static thread_local MapCache mc = {};
   const void *ptrs[6] = {c.k_codes, c.v_codes, c.k_sz, c.v_sz, c.k_hi, c.v_hi};
-  bool hit = mc.valid && mc.n_lo == c.n_lo && mc.n_hi == c.n_hi && mc.nbh == nbh;
+  const int cap = lo_rows(c);
+  bool hit = mc.valid && mc.n_lo == c.n_lo && mc.n_hi == c.n_hi && mc.nbh == nbh && mc.lo_cap == cap;
   for (int i = 0; i < 6 && hit; ++i) hit = mc.p[i] == ptrs[i];
   if (!hit) {
     const int rowb = D * BITS / 8;
     const CUtensorMapSwizzle sw = rowb == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
     CUtensorMap *m = mc.m;
     bool ok = true;
-    ok &= make_map_3d(&m[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, c.k_codes, rowb, c.n_lo, nbh, rowb, T_LO, sw);
-    ok &= make_map_3d(&m[1], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, c.v_codes, rowb, c.n_lo, nbh, rowb, T_LO, sw);
-    ok &= make_map_3d(&m[2], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, c.k_sz, 16, c.n_lo, nbh, 16, T_LO, CU_TENSOR_MAP_SWIZZLE_NONE);
-    ok &= make_map_3d(&m[3], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, c.v_sz, 16, c.n_lo, nbh, 16, T_LO, CU_TENSOR_MAP_SWIZZLE_NONE);
+    // The low maps end at row n_lo (a tail tile reads zeros beyond it, never
+    // the spare rows of a cache that grows during decode); slices are lo_cap
+    // rows apart.
+    ok &= make_map_3d(&m[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, c.k_codes, rowb, c.n_lo, nbh, rowb, T_LO, sw, cap);
+    ok &= make_map_3d(&m[1], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, c.v_codes, rowb, c.n_lo, nbh, rowb, T_LO, sw, cap);
+    ok &= make_map_3d(&m[2], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, c.k_sz, 16, c.n_lo, nbh, 16, T_LO, CU_TENSOR_MAP_SWIZZLE_NONE, cap);
+    ok &= make_map_3d(&m[3], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, c.v_sz, 16, c.n_lo, nbh, 16, T_LO, CU_TENSOR_MAP_SWIZZLE_NONE, cap);
     ok &= make_map_3d(&m[4], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, c.k_hi, D, c.n_hi, nbh, 64, T_HI, CU_TENSOR_MAP_SWIZZLE_128B);
     ok &= make_map_3d(&m[5], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, c.v_hi, D, c.n_hi, nbh, 64, T_HI, CU_TENSOR_MAP_SWIZZLE_128B);
     mc.valid = ok;
@@ -961,6 +965,7 @@ cudaError_t launch_tg(const DecArgs &a0, const hq_kv_cache &c, int nbh, cudaStre
     for (int i = 0; i < 6; ++i) mc.p[i] = ptrs[i];
     mc.n_lo = c.n_lo;
     mc.n_hi = c.n_hi;
+    mc.lo_cap = cap;
     mc.nbh = nbh;
   }
   const CUtensorMap *m = mc.m;

@@ -26,9 +26,15 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // ---------------------------------------------------------------------------
 // Launchers (one per .cu file).  Arguments are already validated.
 // ---------------------------------------------------------------------------
+// Low rows allocated per (b, kv head) of a cache (lo_cap, 0 meaning n_lo).
+inline int lo_rows(const hq_kv_cache &c) { return c.lo_cap > 0 ? c.lo_cap : c.n_lo; }
+
 cudaError_t launch_pack(const __nv_bfloat16 *k, const __nv_bfloat16 *v, const int32_t *idx,
                         int B, int Hkv, int L, int D, int window, int k_vert, int bits,
                         const hq_kv_cache &out, uint32_t *status, cudaStream_t s);
+cudaError_t launch_kv_append(const __nv_bfloat16 *k_new, const __nv_bfloat16 *v_new, int B,
+                             int Hkv, int D, int L, int window, int k_vert,
+                             const hq_kv_cache &c, cudaStream_t s);
 
 size_t probe_ws_bytes(int B, int Hq, int Hkv, int P, int L, int D);
 cudaError_t launch_probe(const __nv_bfloat16 *q_probe, int64_t q_head_stride,

@@ -107,7 +107,7 @@ __device__ __forceinline__ void quant_store(const uint32_t (&w)[D / 64], uint8_t
 template <int D, int BITS>
 __global__ void __launch_bounds__(kWarps * 32)
 pack_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ v,
-            const int32_t *__restrict__ idx, int nbh, int L, int window, int k_vert,
+            const int32_t *__restrict__ idx, int nbh, int L, int window, int k_vert, int lo_cap,
             uint8_t *__restrict__ k_codes, uint8_t *__restrict__ v_codes,
             __half2 *__restrict__ k_sz, __half2 *__restrict__ v_sz,
             __nv_bfloat16 *__restrict__ k_hi, __nv_bfloat16 *__restrict__ v_hi,
@@ -161,7 +161,7 @@ pack_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict
       if (j >= L) break;
       const int cnt = cnt0 + __popc(vbits & ((1u << p) - 1u));            // verticals before j
       int hi_row = -1, lo_row = -1;
-      if (j >= L - window) hi_row = k_vert + (j - (L - window));
+      if (j >= L - window) hi_row = k_vert + j % window;          // the window ring
       else if (vbits & (1u << p)) hi_row = cnt;
       else lo_row = j - cnt;
       if (hi_row >= 0) {
@@ -180,7 +180,7 @@ pack_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict
           if (lane == 0) raise_status(status, HQ_DEV_BAD_INDEX);
           continue;
         }
-        const size_t r = (size_t)bh * n_lo + lo_row;
+        const size_t r = (size_t)bh * lo_cap + lo_row;
         quant_store<D, BITS>(kw[p], k_codes + r * ROWB, k_sz + r * NG, lane);
         quant_store<D, BITS>(vw[p], v_codes + r * ROWB, v_sz + r * NG, lane);
         if (lo_pos && lane == 0) lo_pos[r] = j;
@@ -202,9 +202,75 @@ cudaError_t launch_pack_t(const __nv_bfloat16 *k, const __nv_bfloat16 *v, const 
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
   pack_kernel<D, BITS><<<(unsigned)blocks, kWarps * 32, 0, s>>>(
-      k, v, idx, nbh, L, window, k_vert, (uint8_t *)o.k_codes, (uint8_t *)o.v_codes,
+      k, v, idx, nbh, L, window, k_vert, lo_rows(o), (uint8_t *)o.k_codes, (uint8_t *)o.v_codes,
       (__half2 *)o.k_sz, (__half2 *)o.v_sz, (__nv_bfloat16 *)o.k_hi, (__nv_bfloat16 *)o.v_hi,
       o.lo_pos, status);
+  return cudaGetLastError();
+}
+
+// Decode cache maintenance: one warp per (b, kv head).  The warp reads the
+// window row that position L - W occupies (row k_vert + L mod W of the ring)
+// and the new token's rows, quantizes the old occupant into low row n_lo with
+// the pack's quantizer, then overwrites the window row with the new token.
+// Each lane reads and writes only its own words of the row, so the in-place
+// overwrite after the reads needs no barrier.  With no window the new token
+// goes straight to the low segment.
+template <int D, int BITS>
+__global__ void __launch_bounds__(kWarps * 32)
+kv_append_kernel(const __nv_bfloat16 *__restrict__ k_new, const __nv_bfloat16 *__restrict__ v_new,
+                 int nbh, int L, int window, int k_vert, int n_lo, int lo_cap,
+                 uint8_t *__restrict__ k_codes, uint8_t *__restrict__ v_codes,
+                 __half2 *__restrict__ k_sz, __half2 *__restrict__ v_sz,
+                 __nv_bfloat16 *__restrict__ k_hi, __nv_bfloat16 *__restrict__ v_hi,
+                 int32_t *__restrict__ lo_pos) {
+  constexpr int W32 = D / 64;
+  constexpr int ROWB = D * BITS / 8;
+  constexpr int NG = D / 32;
+  const int lane = threadIdx.x & 31;
+  const int bh = blockIdx.x * kWarps + (threadIdx.x >> 5);
+  if (bh >= nbh) return;
+  const uint32_t *kn = reinterpret_cast<const uint32_t *>(k_new + (size_t)bh * D) + lane * W32;
+  const uint32_t *vn = reinterpret_cast<const uint32_t *>(v_new + (size_t)bh * D) + lane * W32;
+  uint32_t kw[W32], vw[W32], ko[W32], vo[W32];
+#pragma unroll
+  for (int i = 0; i < W32; ++i) {
+    kw[i] = __ldg(kn + i);
+    vw[i] = __ldg(vn + i);
+  }
+  const size_t r = (size_t)bh * lo_cap + n_lo;
+  if (window == 0) {
+    quant_store<D, BITS>(kw, k_codes + r * ROWB, k_sz + r * NG, lane);
+    quant_store<D, BITS>(vw, v_codes + r * ROWB, v_sz + r * NG, lane);
+    if (lo_pos && lane == 0) lo_pos[r] = L;
+    return;
+  }
+  const size_t hrow = ((size_t)bh * (k_vert + window) + k_vert + L % window) * D;
+  uint32_t *kh = reinterpret_cast<uint32_t *>(k_hi + hrow) + lane * W32;
+  uint32_t *vh = reinterpret_cast<uint32_t *>(v_hi + hrow) + lane * W32;
+#pragma unroll
+  for (int i = 0; i < W32; ++i) {
+    ko[i] = kh[i];
+    vo[i] = vh[i];
+  }
+  quant_store<D, BITS>(ko, k_codes + r * ROWB, k_sz + r * NG, lane);
+  quant_store<D, BITS>(vo, v_codes + r * ROWB, v_sz + r * NG, lane);
+  if (lo_pos && lane == 0) lo_pos[r] = L - window;
+#pragma unroll
+  for (int i = 0; i < W32; ++i) {
+    kh[i] = kw[i];
+    vh[i] = vw[i];
+  }
+}
+
+template <int D, int BITS>
+cudaError_t launch_kv_append_t(const __nv_bfloat16 *k_new, const __nv_bfloat16 *v_new, int nbh,
+                               int L, int window, int k_vert, const hq_kv_cache &c,
+                               cudaStream_t s) {
+  const int blocks = (nbh + kWarps - 1) / kWarps;
+  kv_append_kernel<D, BITS><<<blocks, kWarps * 32, 0, s>>>(
+      k_new, v_new, nbh, L, window, k_vert, c.n_lo, lo_rows(c), (uint8_t *)c.k_codes,
+      (uint8_t *)c.v_codes, (__half2 *)c.k_sz, (__half2 *)c.v_sz, (__nv_bfloat16 *)c.k_hi,
+      (__nv_bfloat16 *)c.v_hi, c.lo_pos);
   return cudaGetLastError();
 }
 
@@ -218,6 +284,17 @@ cudaError_t launch_pack(const __nv_bfloat16 *k, const __nv_bfloat16 *v, const in
   if (D == 128 && bits == 8) return launch_pack_t<128, 8>(k, v, idx, nbh, L, window, k_vert, out, status, s);
   if (D == 64 && bits == 4) return launch_pack_t<64, 4>(k, v, idx, nbh, L, window, k_vert, out, status, s);
   if (D == 64 && bits == 8) return launch_pack_t<64, 8>(k, v, idx, nbh, L, window, k_vert, out, status, s);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_kv_append(const __nv_bfloat16 *k_new, const __nv_bfloat16 *v_new, int B,
+                             int Hkv, int D, int L, int window, int k_vert,
+                             const hq_kv_cache &c, cudaStream_t s) {
+  const int nbh = B * Hkv;
+  if (D == 128 && c.bits == 4) return launch_kv_append_t<128, 4>(k_new, v_new, nbh, L, window, k_vert, c, s);
+  if (D == 128 && c.bits == 8) return launch_kv_append_t<128, 8>(k_new, v_new, nbh, L, window, k_vert, c, s);
+  if (D == 64 && c.bits == 4) return launch_kv_append_t<64, 4>(k_new, v_new, nbh, L, window, k_vert, c, s);
+  if (D == 64 && c.bits == 8) return launch_kv_append_t<64, 8>(k_new, v_new, nbh, L, window, k_vert, c, s);
   return cudaErrorInvalidValue;
 }
 

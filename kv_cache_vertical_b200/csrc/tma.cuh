@@ -105,15 +105,17 @@ inline EncodeTiledFn tma_encode_fn() {
 // Map over a row-major [outer][rows][inner] array of `esize`-byte elements;
 // a map with no rows is left zeroed (such maps are never used).  Rows and
 // outer slices outside the array read as zeros.  Returns false on failure.
+// rows_alloc: rows between consecutive outer slices in memory (>= rows; 0
+// means rows).  Rows rows..rows_alloc-1 of a slice are outside the map.
 inline bool make_map_3d(CUtensorMap *m, CUtensorMapDataType dt, int esize, void *base,
                         uint64_t inner, uint64_t rows, uint64_t outer, uint32_t box_inner,
-                        uint32_t box_rows, CUtensorMapSwizzle sw) {
+                        uint32_t box_rows, CUtensorMapSwizzle sw, uint64_t rows_alloc = 0) {
   memset(m, 0, sizeof *m);
   if (rows == 0 || outer == 0 || base == nullptr) return true;
   EncodeTiledFn fn = tma_encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {inner, rows, outer};
-  cuuint64_t strides[2] = {inner * esize, inner * esize * rows};
+  cuuint64_t strides[2] = {inner * esize, inner * esize * (rows_alloc > rows ? rows_alloc : rows)};
   cuuint32_t box[3] = {box_inner, box_rows, 1};
   cuuint32_t es[3] = {1, 1, 1};
   return fn(m, dt, 3, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,

@@ -39,7 +39,7 @@ HQ_DEV_TIMEOUT = 0x2
 class hq_kv_cache(ctypes.Structure):
     _fields_ = [("k_codes", _P), ("v_codes", _P), ("k_sz", _P), ("v_sz", _P), ("k_hi", _P),
                 ("v_hi", _P), ("lo_pos", _P), ("n_lo", _I), ("n_hi", _I), ("bits", _I),
-                ("group", _I)]
+                ("group", _I), ("lo_cap", _I)]
 
 
 def _sig(name, restype, *argtypes):
@@ -60,6 +60,7 @@ _pack = _sig("hq_pack_kv", _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I,
 hq_decode_workspace_size = _sig("hq_decode_workspace_size", _SZ, _I, _I, _I, _I, _I, _I, _I)
 _decode = _sig("hq_decode_attn", _I, _P, ctypes.POINTER(hq_kv_cache), _I, _I, _I, _I, _F, _P, _P,
                _P, _SZ, _P)
+_append = _sig("hq_kv_append", _I, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.POINTER(hq_kv_cache), _P)
 _decode_static = _sig("hq_decode_attn_static", _I, _P, ctypes.POINTER(hq_kv_cache), _I, _I, _I,
                       _I, _F, _P, _P, _P)
 _pquant = _sig("hq_prefill_quant", _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P)
@@ -70,7 +71,7 @@ _prefill = _sig("hq_prefill_attn", _I, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _
 EXPORTED = ["hq_status_string", "hq_version", "hq_read_device_status", "hq_probe_workspace_size",
             "hq_probe_vertical", "hq_pack_kv", "hq_decode_workspace_size", "hq_decode_attn",
             "hq_prefill_quant", "hq_prefill_workspace_size", "hq_prefill_attn",
-            "hq_decode_attn_static"]
+            "hq_decode_attn_static", "hq_kv_append"]
 
 HQ_ERR_SCRATCH_LIMIT = 7
 STATIC_SCRATCH_BYTES = 8 << 20
@@ -134,29 +135,40 @@ class KVCache:
     group: int = 32
 
     @classmethod
-    def empty(cls, B, Hkv, L, D, window, k_vert, bits, device="cuda", with_pos=True):
+    def empty(cls, B, Hkv, L, D, window, k_vert, bits, device="cuda", with_pos=True,
+              lo_cap=None):
+        """Buffers for a cache of L tokens.  lo_cap (default: exactly the
+        n_lo low rows) reserves low rows per (b, kv head) for decode appends."""
         n_lo, n_hi = L - window - k_vert, k_vert + window
+        C = n_lo if lo_cap is None else int(lo_cap)
+        assert C >= n_lo, "lo_cap below the number of low rows"
         u8 = dict(dtype=torch.uint8, device=device)
         return cls(
-            k_codes=torch.empty(B, Hkv, n_lo, D * bits // 8, **u8),
-            v_codes=torch.empty(B, Hkv, n_lo, D * bits // 8, **u8),
-            k_sz=torch.empty(B, Hkv, n_lo, D // 32, 2, dtype=torch.float16, device=device),
-            v_sz=torch.empty(B, Hkv, n_lo, D // 32, 2, dtype=torch.float16, device=device),
+            k_codes=torch.empty(B, Hkv, C, D * bits // 8, **u8),
+            v_codes=torch.empty(B, Hkv, C, D * bits // 8, **u8),
+            k_sz=torch.empty(B, Hkv, C, D // 32, 2, dtype=torch.float16, device=device),
+            v_sz=torch.empty(B, Hkv, C, D // 32, 2, dtype=torch.float16, device=device),
             k_hi=torch.empty(B, Hkv, n_hi, D, dtype=torch.bfloat16, device=device),
             v_hi=torch.empty(B, Hkv, n_hi, D, dtype=torch.bfloat16, device=device),
-            lo_pos=torch.empty(B, Hkv, n_lo, dtype=torch.int32, device=device) if with_pos else None,
+            lo_pos=torch.empty(B, Hkv, C, dtype=torch.int32, device=device) if with_pos else None,
             n_lo=n_lo, n_hi=n_hi, bits=bits)
+
+    @property
+    def lo_cap(self) -> int:
+        return self.k_codes.shape[2] if self.k_codes.dim() == 4 else self.n_lo
 
     def struct(self) -> hq_kv_cache:
         return hq_kv_cache(_ptr(self.k_codes), _ptr(self.v_codes), _ptr(self.k_sz),
                            _ptr(self.v_sz), _ptr(self.k_hi), _ptr(self.v_hi), _ptr(self.lo_pos),
-                           self.n_lo, self.n_hi, self.bits, self.group)
+                           self.n_lo, self.n_hi, self.bits, self.group, self.lo_cap)
 
     def nbytes(self, with_pos: bool = False) -> int:
-        ts = [self.k_codes, self.v_codes, self.k_sz, self.v_sz, self.k_hi, self.v_hi]
+        """Bytes of the rows in use (spare low rows not counted)."""
+        lo = [self.k_codes, self.v_codes, self.k_sz, self.v_sz]
         if with_pos and self.lo_pos is not None:
-            ts.append(self.lo_pos)
-        return sum(t.numel() * t.element_size() for t in ts)
+            lo.append(self.lo_pos)
+        n = sum(t[:, :, :self.n_lo].numel() * t.element_size() for t in lo)
+        return n + sum(t.numel() * t.element_size() for t in (self.k_hi, self.v_hi))
 
 
 # ---------------------------------------------------------------------------
@@ -175,6 +187,12 @@ def hq_pack_kv(k, v, idx, B, Hkv, L, D, window, k_vert, bits, group, cache: KVCa
     _check(_pack(_ptr(k), _ptr(v), _ptr(idx), B, Hkv, L, D, window, k_vert, bits, group,
                  ctypes.byref(st), _ptr(ws), ws.numel() if ws is not None else 0,
                  _stream(stream)), "hq_pack_kv")
+
+
+def hq_kv_append(k_new, v_new, B, Hkv, D, L, window, k_vert, cache: KVCache, stream=None):
+    st = cache.struct()
+    _check(_append(_ptr(k_new), _ptr(v_new), B, Hkv, D, L, window, k_vert, ctypes.byref(st),
+                   _stream(stream)), "hq_kv_append")
 
 
 def hq_decode_attn(q, cache: KVCache, B, Hq, Hkv, D, softmax_scale, out, lse_out, ws, stream=None):
@@ -225,11 +243,20 @@ def probe_vertical(q_probe, k, window, k_vert, scale=0.0, want_scores=False, ws=
     return (idx, score) if want_scores else idx
 
 
-def pack_kv(k, v, idx, window, bits=4, ws=None, with_pos=True) -> KVCache:
+def pack_kv(k, v, idx, window, bits=4, ws=None, with_pos=True, lo_cap=None) -> KVCache:
     B, Hkv, L, D = k.shape
     k_vert = idx.shape[2]
-    cache = KVCache.empty(B, Hkv, L, D, window, k_vert, bits, k.device, with_pos)
+    cache = KVCache.empty(B, Hkv, L, D, window, k_vert, bits, k.device, with_pos, lo_cap)
     hq_pack_kv(k, v, idx, B, Hkv, L, D, window, k_vert, bits, 32, cache, ws)
+    return cache
+
+
+def kv_append(cache: KVCache, k_new, v_new, L, window, stream=None):
+    """Token L (bf16 [B, Hkv, D] key and value) enters the cache; the cache's
+    n_lo grows by one (the position that left the window)."""
+    B, Hkv, D = k_new.shape
+    hq_kv_append(k_new, v_new, B, Hkv, D, L, window, cache.n_hi - window, cache, stream)
+    cache.n_lo += 1
     return cache
 
 

@@ -50,11 +50,12 @@ def _load():
         lib.hqo_topk.argtypes = [P, I, I, I, I, I, P]
         lib.hqo_quant_row.argtypes = [P, I, I, I, P, P]
         lib.hqo_pack_kv.argtypes = [P, P, P] + [I] * 8 + [P] * 7
+        lib.hqo_kv_append.argtypes = [P, P] + [I] * 10 + [P] * 7
         lib.hqo_decode_attn.argtypes = [P] * 7 + [I] * 8 + [D, P, P]
         lib.hqo_prefill_quant.argtypes = [P, P, P] + [I] * 7 + [P] * 4
         lib.hqo_prefill_attn.argtypes = [P] * 8 + [I] * 8 + [D, P, I, P]
         lib.hqo_max_threads.argtypes = []
-        for f in ("hqo_probe_scores", "hqo_topk", "hqo_quant_row", "hqo_pack_kv",
+        for f in ("hqo_probe_scores", "hqo_topk", "hqo_quant_row", "hqo_pack_kv", "hqo_kv_append",
                   "hqo_decode_attn", "hqo_prefill_quant", "hqo_prefill_attn", "hqo_max_threads"):
             getattr(lib, f).restype = I
         _lib = lib
@@ -157,6 +158,31 @@ def pack_kv(k, v, idx, window: int, bits_: int = 4, group: int = 32) -> dict:
                              _p(out["v_sz"]), _p(out["k_hi"]), _p(out["v_hi"]), _p(out["lo_pos"]))
     assert rc == 0, rc
     out.update(n_lo=n_lo, n_hi=n_hi, bits=bits_, group=group)
+    return out
+
+
+def kv_append(cache: dict, k_new, v_new, L: int, window: int) -> dict:
+    """One decode step of cache maintenance: token L (bf16 K/V [B, Hkv, D])
+    enters the window ring, position L - W leaves it for the low segment.
+    Returns a new cache dict with n_lo + 1 low rows; ``cache`` is not changed."""
+    kn, vn = _u16(k_new), _u16(v_new)
+    B, Hkv, D = kn.shape
+    n_lo, n_hi = int(cache["n_lo"]), int(cache["n_hi"])
+    kv = n_hi - window
+    out = {}
+    for name in ("k_codes", "v_codes", "k_sz", "v_sz", "lo_pos"):
+        a = np.asarray(cache[name])
+        grown = np.zeros((B, Hkv, n_lo + 1) + a.shape[3:], a.dtype)
+        grown[:, :, :n_lo] = a[:, :, :n_lo]
+        out[name] = grown
+    out["k_hi"] = np.array(cache["k_hi"], np.uint16, copy=True)
+    out["v_hi"] = np.array(cache["v_hi"], np.uint16, copy=True)
+    rc = _load().hqo_kv_append(
+        _p(kn), _p(vn), B, Hkv, D, L, window, kv, int(cache["bits"]), int(cache["group"]),
+        n_lo, n_lo + 1, _p(out["k_codes"]), _p(out["v_codes"]), _p(bits(out["k_sz"])),
+        _p(bits(out["v_sz"])), _p(out["k_hi"]), _p(out["v_hi"]), _p(out["lo_pos"]))
+    assert rc == 0, rc
+    out.update(n_lo=n_lo + 1, n_hi=n_hi, bits=cache["bits"], group=cache["group"])
     return out
 
 

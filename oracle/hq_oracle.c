@@ -299,10 +299,15 @@ int hqo_quant_row(const uint16_t *x, int D, int bits, int group, uint8_t *packed
  *   k_codes, v_codes: u8  [B, Hkv, n_lo, D*bits/8]
  *   k_sz, v_sz:       f16 [B, Hkv, n_lo, D/group, 2]
  *   k_hi, v_hi:       bf16 [B, Hkv, n_hi, D]  (vertical rows in ascending
- *                     index order, then the window rows L-W .. L-1)
+ *                     index order, then the window: window position p in row
+ *                     kv + p mod W)
  *   lo_pos:           i32 [B, Hkv, n_lo]  (nullable)
  * with n_lo = L - W - kv and n_hi = kv + W.
  * idx: [B, Hkv, kv] ascending, distinct, each in [0, L - W).
+ * Window placement (reading; the pages do not fix a layout): the window is a
+ * ring keyed by position, so that sliding it by one token during decode
+ * rewrites one row and moves none (hqo_kv_append).  Attention does not
+ * depend on the order of the rows.
  */
 int hqo_pack_kv(const uint16_t *k, const uint16_t *v, const int32_t *idx, int B, int Hkv,
                 int L, int D, int window, int kv, int bits, int group, uint8_t *k_codes,
@@ -329,7 +334,7 @@ int hqo_pack_kv(const uint16_t *k, const uint16_t *v, const int32_t *idx, int B,
         for (int j = 0; j < L; ++j) {
             const uint16_t *kr = kb + (size_t)j * D, *vr = vb + (size_t)j * D;
             if (j >= L - window) {                       /* window row */
-                size_t o = ((size_t)bh * n_hi + kv + (j - (L - window))) * D;
+                size_t o = ((size_t)bh * n_hi + kv + j % window) * D;
                 memcpy(k_hi + o, kr, sizeof(uint16_t) * D);
                 memcpy(v_hi + o, vr, sizeof(uint16_t) * D);
             } else if (vi < kv && id[vi] == j) {         /* vertical row */
@@ -346,6 +351,63 @@ int hqo_pack_kv(const uint16_t *k, const uint16_t *v, const int32_t *idx, int B,
                 ++lo;
             }
         }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Decode cache maintenance: one new token.                                 */
+/* ------------------------------------------------------------------------ */
+/*
+ * [W] TL;DR: in decode the prefill rule becomes a KV cache compression policy;
+ * [B] "What hybrid-precision attention changes": most of the decode cache is
+ * low-bit, the selected positions stay in higher precision.  The pages do not
+ * say how the cache changes from one token to the next.  Readings taken:
+ *   - the vertical set chosen at prefill stays fixed during decode;
+ *   - the window is always the W most recent positions, so when token L (the
+ *     new one) arrives, position L - W leaves the window and is quantized
+ *     with the same row quantizer as the pack (quant_row); it becomes the last
+ *     low row, which keeps the low rows in ascending position order because
+ *     every earlier low position is below L - W;
+ *   - the new token's bf16 K/V take the window row that position L - W held,
+ *     row kv + L mod W (the ring placement of hqo_pack_kv);
+ *   - W = 0: the new token itself is quantized into the low segment.
+ * With these readings, the cache packed from L tokens and then given tokens
+ * L .. L+t-1 one by one equals, field for field, the cache packed from L + t
+ * tokens with the same vertical set.
+ *
+ * Cache arrays as in hqo_pack_kv, except that the low arrays hold lo_cap rows
+ * per (b, kv head), of which the first n_lo are in use; n_lo = L - W - kv
+ * must hold and n_lo < lo_cap.  k_new, v_new: bf16 [B, Hkv, D].  After the
+ * call the low segment holds n_lo + 1 rows.
+ */
+int hqo_kv_append(const uint16_t *k_new, const uint16_t *v_new, int B, int Hkv, int D, int L,
+                  int window, int kv, int bits, int group, int n_lo, int lo_cap,
+                  uint8_t *k_codes, uint8_t *v_codes, uint16_t *k_sz, uint16_t *v_sz,
+                  uint16_t *k_hi, uint16_t *v_hi, int32_t *lo_pos)
+{
+    if ((bits != 4 && bits != 8) || group <= 0 || D % group || D > 512 || window < 0 ||
+        kv < 0 || n_lo != L - window - kv || n_lo < 0 || n_lo >= lo_cap)
+        return 1;
+    const int row_bytes = D * bits / 8, ng = D / group, n_hi = kv + window;
+    for (long long bh = 0; bh < (long long)B * Hkv; ++bh) {
+        const uint16_t *kn = k_new + (size_t)bh * D, *vn = v_new + (size_t)bh * D;
+        const size_t r = (size_t)bh * lo_cap + n_lo;          /* the new low row */
+        if (window == 0) {
+            quant_row(kn, D, bits, group, k_codes + r * row_bytes, k_sz + r * 2 * ng);
+            quant_row(vn, D, bits, group, v_codes + r * row_bytes, v_sz + r * 2 * ng);
+            if (lo_pos)
+                lo_pos[r] = L;
+            continue;
+        }
+        uint16_t *kh = k_hi + ((size_t)bh * n_hi + kv + L % window) * D;
+        uint16_t *vh = v_hi + ((size_t)bh * n_hi + kv + L % window) * D;
+        quant_row(kh, D, bits, group, k_codes + r * row_bytes, k_sz + r * 2 * ng);
+        quant_row(vh, D, bits, group, v_codes + r * row_bytes, v_sz + r * 2 * ng);
+        if (lo_pos)
+            lo_pos[r] = L - window;
+        memcpy(kh, kn, sizeof(uint16_t) * D);
+        memcpy(vh, vn, sizeof(uint16_t) * D);
     }
     return 0;
 }

@@ -44,11 +44,14 @@ def assert_index_sets(gpu_idx: np.ndarray, ref_idx: np.ndarray, ref_score: np.nd
 
 
 def cache_to_np(cache) -> dict:
+    """The rows in use of a device cache (spare low rows left out)."""
+    n = cache.n_lo
     return dict(
-        k_codes=cache.k_codes.cpu().numpy(), v_codes=cache.v_codes.cpu().numpy(),
-        k_sz=oracle.bits(cache.k_sz.cpu()), v_sz=oracle.bits(cache.v_sz.cpu()),
+        k_codes=cache.k_codes[:, :, :n].cpu().numpy(), v_codes=cache.v_codes[:, :, :n].cpu().numpy(),
+        k_sz=oracle.bits(cache.k_sz[:, :, :n].cpu()), v_sz=oracle.bits(cache.v_sz[:, :, :n].cpu()),
         k_hi=oracle.bits(cache.k_hi.cpu()), v_hi=oracle.bits(cache.v_hi.cpu()),
-        lo_pos=cache.lo_pos.cpu().numpy() if cache.lo_pos is not None else None,
+        lo_pos=cache.lo_pos[:, :, :n].cpu().numpy() if cache.lo_pos is not None else None,
+        n_lo=n, n_hi=cache.n_hi, bits=cache.bits, group=cache.group,
     )
 
 

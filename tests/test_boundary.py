@@ -56,7 +56,7 @@ def test_status_strings(lib):
 class _Cache(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("k_codes", "v_codes", "k_sz", "v_sz", "k_hi", "v_hi", "lo_pos")] + \
-               [(n, ctypes.c_int) for n in ("n_lo", "n_hi", "bits", "group")]
+               [(n, ctypes.c_int) for n in ("n_lo", "n_hi", "bits", "group", "lo_cap")]
 
 
 FAKE = ctypes.c_void_p(0x10000)      # 16-byte aligned, never dereferenced on the host
@@ -84,6 +84,39 @@ def test_pack_argument_checks(lib):
     assert call(k=ODD) == 1                   # misaligned
     bad = _Cache(FAKE, FAKE, FAKE, FAKE, None, FAKE, None, 845, 179, 4, 32)
     assert call(cache=bad) == 1               # missing hi buffer
+
+
+def test_cache_struct_matches_header():
+    """The binding's struct has the header's fields, in the header's order."""
+    from kv_cache_vertical_b200 import hq
+    text = open(os.path.join(ROOT, "include", "hq.h")).read()
+    body = re.search(r"typedef struct \{([^}]*)\} hq_kv_cache;", text).group(1)
+    names = re.findall(r"(\w+);", body)
+    assert names == [n for n, _ in hq.hq_kv_cache._fields_]
+    assert [n for n, _ in _Cache._fields_] == names
+
+
+def test_append_argument_checks(lib):
+    f = lib.hq_kv_append
+    f.restype = ctypes.c_int
+    L, W, kv = 1024, 128, 51
+    c = _Cache(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, L - W - kv, kv + W, 4, 32, L - W - kv + 8)
+
+    def call(k=FAKE, v=FAKE, B=1, Hkv=1, D=64, L=L, W=W, kv=kv, cache=c):
+        return f(k, v, B, Hkv, D, L, W, kv, ctypes.byref(cache), None)
+    assert call(k=None) == 1
+    assert call(D=96) == 2
+    assert call(L=L + 1) == 1                 # n_lo != L - window - k_vert
+    assert call(W=W - 1, L=L - 1) == 1        # n_hi != k_vert + window
+    assert call(v=ODD) == 1                   # misaligned
+    full = _Cache(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, L - W - kv, kv + W, 4, 32, L - W - kv)
+    assert call(cache=full) == 1              # no spare low row
+    exact = _Cache(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, L - W - kv, kv + W, 4, 32, 0)
+    assert call(cache=exact) == 1             # lo_cap 0 means exactly n_lo rows: no room
+    small = _Cache(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 845, 179, 4, 32, 800)
+    lib.hq_decode_attn.restype = ctypes.c_int
+    assert lib.hq_decode_attn(FAKE, ctypes.byref(small), 1, 2, 1, 64, ctypes.c_float(0.0), FAKE,
+                              None, FAKE, ctypes.c_size_t(1 << 30), None) == 1   # lo_cap < n_lo
 
 
 def test_decode_argument_checks(lib):

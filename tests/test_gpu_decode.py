@@ -146,7 +146,7 @@ def _full_size_sampled(w: Workload, samples):
         if not np.array_equal(gidx[b:b + 1, h:h + 1], ridx):
             continue  # a tie swapped members: the rest of this slice is not comparable
         rc = oracle.pack_kv(ks, vs, ridx, w.window, w.bits)
-        assert_pack_equal({k: (v[b:b + 1, h:h + 1] if v is not None else None)
+        assert_pack_equal({k: (v[b:b + 1, h:h + 1] if isinstance(v, np.ndarray) else None)
                            for k, v in gc.items()}, rc)
         ro, _ = oracle.decode_attn(qs, rc, 1)
         assert_close(gout[b:b + 1, h * G:(h + 1) * G], ro, f"{w.name} b={b} h={h}")

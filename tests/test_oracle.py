@@ -233,13 +233,67 @@ def test_pack_partition_and_rows(bits):
             allpos = np.concatenate([lo, idx[b, h], np.arange(L - W, L)])
             assert np.array_equal(np.sort(allpos), np.arange(L))       # exact partition
             assert np.all(np.diff(lo) > 0)                              # ascending, compacted
-            hi_src = np.concatenate([idx[b, h], np.arange(L - W, L)])
+            win = np.arange(L - W, L)
+            hi_src = np.concatenate([idx[b, h], win[np.argsort(win % W)]])   # ring: row kv + p mod W
             assert np.array_equal(c["k_hi"][b, h], kb[b, h, hi_src])
             assert np.array_equal(c["v_hi"][b, h], vb[b, h, hi_src])
             for r in (0, len(lo) // 2, len(lo) - 1):
                 pk, szk = oracle.quant_row(k[b, h, lo[r]], bits, 32)
                 assert np.array_equal(c["k_codes"][b, h, r], pk)
                 assert np.array_equal(c["k_sz"][b, h, r].reshape(-1), szk)
+
+
+# --------------------------------------------------------------------------
+# Decode cache maintenance: append = pack of the longer prefix
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits,D,W", [(4, 64, 32), (8, 64, 32), (4, 128, 7), (8, 128, 0)])
+def test_append_equals_pack_of_longer_prefix(bits, D, W):
+    """Packing L0 tokens and appending tokens L0 .. L0+t-1 one by one gives the
+    cache packed from L0 + t tokens with the same vertical set, field for
+    field: the evicted position, its low row, lo_pos, the ring slot and the
+    quantizer all have to be right for that.  t > W so the ring wraps."""
+    B, Hkv, L0, t, kv = 2, 2, 150, 45, 9
+    k = bf16(RNG.standard_normal((B, Hkv, L0 + t, D)) * 2.0)
+    v = bf16(RNG.standard_normal((B, Hkv, L0 + t, D)))
+    idx = np.sort(np.stack([np.stack([RNG.choice(L0 - W, kv, replace=False) for _ in range(Hkv)])
+                            for _ in range(B)]), -1).astype(np.int32)
+    c = oracle.pack_kv(k[:, :, :L0], v[:, :, :L0], idx, W, bits, 32)
+    for L in range(L0, L0 + t):
+        c = oracle.kv_append(c, k[:, :, L], v[:, :, L], L, W)
+    ref = oracle.pack_kv(k, v, idx, W, bits, 32)
+    assert c["n_lo"] == ref["n_lo"] and c["n_hi"] == ref["n_hi"]
+    for name in ("k_codes", "v_codes", "k_sz", "v_sz", "k_hi", "v_hi", "lo_pos"):
+        assert np.array_equal(c[name], ref[name]), name
+
+
+def test_append_moves_exactly_one_token():
+    """One append: the window row kv + L mod W now holds token L, the old
+    occupant (position L - W) is the new last low row, quantized by the row
+    quantizer, and nothing else changed."""
+    B, Hkv, L, D, W, kv = 1, 3, 200, 64, 16, 11
+    k = bf16(RNG.standard_normal((B, Hkv, L + 1, D)))
+    v = bf16(RNG.standard_normal((B, Hkv, L + 1, D)))
+    idx = np.sort(np.stack([np.stack([RNG.choice(L - W, kv, replace=False) for _ in range(Hkv)])
+                            for _ in range(B)]), -1).astype(np.int32)
+    c0 = oracle.pack_kv(k[:, :, :L], v[:, :, :L], idx, W, 4, 32)
+    c1 = oracle.kv_append(c0, k[:, :, L], v[:, :, L], L, W)
+    kb, vb = oracle.bits(k), oracle.bits(v)
+    slot = kv + L % W
+    for h in range(Hkv):
+        assert np.array_equal(c1["k_hi"][0, h, slot], kb[0, h, L])
+        assert np.array_equal(c1["v_hi"][0, h, slot], vb[0, h, L])
+        assert np.array_equal(c0["k_hi"][0, h, slot], kb[0, h, L - W])      # the evicted token
+        others = np.arange(kv + W) != slot
+        assert np.array_equal(c1["k_hi"][0, h, others], c0["k_hi"][0, h, others])
+        assert c1["lo_pos"][0, h, -1] == L - W
+        assert np.array_equal(c1["lo_pos"][0, h, :-1], c0["lo_pos"][0, h])
+        pk, szk = oracle.quant_row(k[0, h, L - W], 4, 32)
+        assert np.array_equal(c1["k_codes"][0, h, -1], pk)
+        assert np.array_equal(c1["k_sz"][0, h, -1].reshape(-1), szk)
+        pv, szv = oracle.quant_row(v[0, h, L - W], 4, 32)
+        assert np.array_equal(c1["v_codes"][0, h, -1], pv)
+        assert np.array_equal(c1["v_sz"][0, h, -1].reshape(-1), szv)
 
 
 def test_memory_overhead_matches_the_pages():
