@@ -189,6 +189,10 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
     *last_flag = 0;
   }
   __syncthreads();
+  // Everything above touched only shared memory and kernel parameters; the
+  // cache, q and the workspace may be written by the kernel before this one.
+  pdl_wait();
+  pdl_trigger();
 
   if (warp == NCW) {
     // ------------------------------ producer ------------------------------
@@ -970,9 +974,8 @@ cudaError_t launch_tg(const DecArgs &a0, const hq_kv_cache &c, int nbh, cudaStre
   }
   const CUtensorMap *m = mc.m;
   occupancy<BITS, G>();  // sets the dynamic shared memory attribute once
-  dim3 grid(a.nc_lo + a.nc_hi);
-  decode_tma<BITS, G><<<grid, NTHREADS, Cfg<BITS>::SMEM, s>>>(m[0], m[1], m[2], m[3], m[4], m[5], a);
-  return cudaGetLastError();
+  return pdl_launch(decode_tma<BITS, G>, dim3(a.nc_lo + a.nc_hi), dim3(NTHREADS), Cfg<BITS>::SMEM, s,
+                    m[0], m[1], m[2], m[3], m[4], m[5], a);
 }
 
 }  // namespace

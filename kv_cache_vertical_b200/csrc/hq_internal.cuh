@@ -24,6 +24,34 @@ __device__ __forceinline__ void raise_status(uint32_t *status, uint32_t bit) {
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch.  A kernel launched with pdl_launch() may be
+// scheduled while the kernel before it in the stream is still finishing; it
+// must call pdl_wait() before it touches any memory an earlier kernel writes
+// (the wait returns once that kernel has completed and its writes are
+// visible; without the launch attribute it returns at once).
+// pdl_trigger() lets the next such kernel be scheduled early.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
+template <typename... Params, typename... Args>
+cudaError_t pdl_launch(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
 // Launchers (one per .cu file).  Arguments are already validated.
 // ---------------------------------------------------------------------------
 // Low rows allocated per (b, kv head) of a cache (lo_cap, 0 meaning n_lo).

@@ -228,6 +228,8 @@ kv_append_kernel(const __nv_bfloat16 *__restrict__ k_new, const __nv_bfloat16 *_
   constexpr int NG = D / 32;
   const int lane = threadIdx.x & 31;
   const int bh = blockIdx.x * kWarps + (threadIdx.x >> 5);
+  pdl_wait();      // the token's K/V and the cache rows come from earlier kernels
+  pdl_trigger();
   if (bh >= nbh) return;
   const uint32_t *kn = reinterpret_cast<const uint32_t *>(k_new + (size_t)bh * D) + lane * W32;
   const uint32_t *vn = reinterpret_cast<const uint32_t *>(v_new + (size_t)bh * D) + lane * W32;
@@ -267,11 +269,10 @@ cudaError_t launch_kv_append_t(const __nv_bfloat16 *k_new, const __nv_bfloat16 *
                                int L, int window, int k_vert, const hq_kv_cache &c,
                                cudaStream_t s) {
   const int blocks = (nbh + kWarps - 1) / kWarps;
-  kv_append_kernel<D, BITS><<<blocks, kWarps * 32, 0, s>>>(
-      k_new, v_new, nbh, L, window, k_vert, c.n_lo, lo_rows(c), (uint8_t *)c.k_codes,
-      (uint8_t *)c.v_codes, (__half2 *)c.k_sz, (__half2 *)c.v_sz, (__nv_bfloat16 *)c.k_hi,
-      (__nv_bfloat16 *)c.v_hi, c.lo_pos);
-  return cudaGetLastError();
+  return pdl_launch(kv_append_kernel<D, BITS>, dim3(blocks), dim3(kWarps * 32), 0, s, k_new, v_new,
+                    nbh, L, window, k_vert, c.n_lo, lo_rows(c), (uint8_t *)c.k_codes,
+                    (uint8_t *)c.v_codes, (__half2 *)c.k_sz, (__half2 *)c.v_sz,
+                    (__nv_bfloat16 *)c.k_hi, (__nv_bfloat16 *)c.v_hi, c.lo_pos);
 }
 
 }  // namespace
