@@ -48,10 +48,14 @@ def _load():
         lib.hqo_f64_to_f16.restype = ctypes.c_uint16
         lib.hqo_probe_scores.argtypes = [P, P, I, I, I, I, I, I, D, P]
         lib.hqo_topk.argtypes = [P, I, I, I, I, I, P]
-        lib.hqo_quant_row.argtypes = [P, I, I, I, P, P]
-        lib.hqo_pack_kv.argtypes = [P, P, P] + [I] * 8 + [P] * 7
-        lib.hqo_kv_append.argtypes = [P, P] + [I] * 10 + [P] * 7
-        lib.hqo_decode_attn.argtypes = [P] * 7 + [I] * 8 + [D, P, P]
+        lib.hqo_e4m3_to_f64.argtypes = [ctypes.c_uint8]
+        lib.hqo_e4m3_to_f64.restype = D
+        lib.hqo_f64_to_e4m3.argtypes = [D]
+        lib.hqo_f64_to_e4m3.restype = ctypes.c_uint8
+        lib.hqo_quant_row.argtypes = [P, I, I, I, I, P, P]
+        lib.hqo_pack_kv.argtypes = [P, P, P] + [I] * 9 + [P] * 7
+        lib.hqo_kv_append.argtypes = [P, P] + [I] * 11 + [P] * 7
+        lib.hqo_decode_attn.argtypes = [P] * 7 + [I] * 9 + [D, P, P]
         lib.hqo_prefill_quant.argtypes = [P, P, P] + [I] * 7 + [P] * 4
         lib.hqo_prefill_attn.argtypes = [P] * 8 + [I] * 8 + [D, P, I, P]
         lib.hqo_max_threads.argtypes = []
@@ -125,18 +129,29 @@ def topk(score: np.ndarray, window: int, kv: int) -> np.ndarray:
     return idx
 
 
-def quant_row(x, bits_: int = 4, group: int = 32):
+FMT_INT, FMT_FP8 = 0, 1      # low-bit code formats: asymmetric integer, FP8 E4M3
+
+
+def e4m3_to_f64(c: int) -> float:
+    return _load().hqo_e4m3_to_f64(int(c))
+
+
+def f64_to_e4m3(v: float) -> int:
+    return _load().hqo_f64_to_e4m3(float(v))
+
+
+def quant_row(x, bits_: int = 4, group: int = 32, fmt: int = FMT_INT):
     """Quantize one row of bf16 values -> (packed codes u8, interleaved (s, z) f16 bits)."""
     xb = _u16(x).reshape(-1)
     D = xb.shape[0]
     packed = np.zeros(D * bits_ // 8, np.uint8)
     sz = np.zeros(2 * (D // group), np.uint16)
-    rc = _load().hqo_quant_row(_p(xb), D, bits_, group, _p(packed), _p(sz))
+    rc = _load().hqo_quant_row(_p(xb), D, bits_, group, fmt, _p(packed), _p(sz))
     assert rc == 0, rc
     return packed, sz
 
 
-def pack_kv(k, v, idx, window: int, bits_: int = 4, group: int = 32) -> dict:
+def pack_kv(k, v, idx, window: int, bits_: int = 4, group: int = 32, fmt: int = FMT_INT) -> dict:
     """Build the hybrid cache (canonical layout) from bf16 K, V [B, Hkv, L, D]."""
     kk, vv = _u16(k), _u16(v)
     B, Hkv, L, D = kk.shape
@@ -153,11 +168,11 @@ def pack_kv(k, v, idx, window: int, bits_: int = 4, group: int = 32) -> dict:
         v_hi=np.zeros((B, Hkv, n_hi, D), np.uint16),
         lo_pos=np.zeros((B, Hkv, n_lo), np.int32),
     )
-    rc = _load().hqo_pack_kv(_p(kk), _p(vv), _p(idx), B, Hkv, L, D, window, kv, bits_, group,
+    rc = _load().hqo_pack_kv(_p(kk), _p(vv), _p(idx), B, Hkv, L, D, window, kv, bits_, group, fmt,
                              _p(out["k_codes"]), _p(out["v_codes"]), _p(out["k_sz"]),
                              _p(out["v_sz"]), _p(out["k_hi"]), _p(out["v_hi"]), _p(out["lo_pos"]))
     assert rc == 0, rc
-    out.update(n_lo=n_lo, n_hi=n_hi, bits=bits_, group=group)
+    out.update(n_lo=n_lo, n_hi=n_hi, bits=bits_, group=group, fmt=fmt)
     return out
 
 
@@ -179,10 +194,11 @@ def kv_append(cache: dict, k_new, v_new, L: int, window: int) -> dict:
     out["v_hi"] = np.array(cache["v_hi"], np.uint16, copy=True)
     rc = _load().hqo_kv_append(
         _p(kn), _p(vn), B, Hkv, D, L, window, kv, int(cache["bits"]), int(cache["group"]),
-        n_lo, n_lo + 1, _p(out["k_codes"]), _p(out["v_codes"]), _p(bits(out["k_sz"])),
+        int(cache.get("fmt", FMT_INT)), n_lo, n_lo + 1, _p(out["k_codes"]), _p(out["v_codes"]), _p(bits(out["k_sz"])),
         _p(bits(out["v_sz"])), _p(out["k_hi"]), _p(out["v_hi"]), _p(out["lo_pos"]))
     assert rc == 0, rc
-    out.update(n_lo=n_lo + 1, n_hi=n_hi, bits=cache["bits"], group=cache["group"])
+    out.update(n_lo=n_lo + 1, n_hi=n_hi, bits=cache["bits"], group=cache["group"],
+               fmt=cache.get("fmt", FMT_INT))
     return out
 
 
@@ -197,7 +213,7 @@ def decode_attn(q, cache: dict, Hkv: int, scale: float | None = None):
     rc = _load().hqo_decode_attn(
         _p(qq), _p(c["k_codes"]), _p(c["v_codes"]), _p(bits(c["k_sz"])), _p(bits(c["v_sz"])),
         _p(bits(c["k_hi"])), _p(bits(c["v_hi"])), B, Hq, Hkv, D, int(cache["n_lo"]),
-        int(cache["n_hi"]), int(cache["bits"]), int(cache["group"]),
+        int(cache["n_hi"]), int(cache["bits"]), int(cache["group"]), int(cache.get("fmt", FMT_INT)),
         default_scale(D) if scale is None else scale, _p(out), _p(lse))
     assert rc == 0, rc
     return out, lse

@@ -269,13 +269,89 @@ static void quant_group(const uint16_t *x, int n, int bits, uint8_t *codes,
     *z_out = zb;
 }
 
+/*
+ * FP8 E4M3 codes (the "FN" variant of the OCP 8-bit floating-point formats):
+ * 1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits; exponent field 0
+ * holds subnormals m/8 * 2^-6; there is no infinity and only S.1111.111 is
+ * NaN, so the largest finite magnitude is 1.75 * 2^8 = 448.  Written from
+ * that definition.
+ */
+static double e4m3_to_f64(uint8_t c)
+{
+    const int e = (c >> 3) & 15, m = c & 7;
+    double v;
+    if (e == 15 && m == 7)
+        return NAN;
+    v = e == 0 ? ldexp((double)m, -9) : ldexp((double)(8 + m), e - 10);
+    return (c & 0x80) ? -v : v;
+}
+
+/* Round a double to E4M3, ties to the even code, magnitudes past the largest
+ * finite one saturating to +-448 (never NaN).  The sign survives rounding to
+ * zero (-0 is 0x80). */
+static uint8_t f64_to_e4m3_rne_sat(double v)
+{
+    const uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    const double a = fabs(v);
+    if (a >= 448.0)
+        return sign | 0x7E;
+    if (a < ldexp(1.0, -6))                        /* subnormal spacing 2^-9 */
+        return sign | (uint8_t)nearbyint(a * 512.0);   /* 8 = the smallest normal */
+    int e2;
+    frexp(a, &e2);                                 /* a in [2^(e2-1), 2^e2) */
+    int E = e2 - 1;
+    double m = nearbyint(ldexp(a, 3 - E));         /* 8 .. 16 */
+    if (m == 16.0) {
+        m = 8.0;
+        E += 1;
+    }
+    int code = ((E + 7) << 3) | ((int)m - 8);
+    if (code > 0x7E)
+        code = 0x7E;
+    return sign | (uint8_t)code;
+}
+
+/* Exposed for the format pins. */
+double hqo_e4m3_to_f64(uint8_t c) { return e4m3_to_f64(c); }
+uint8_t hqo_f64_to_e4m3(double v) { return f64_to_e4m3_rne_sat(v); }
+
+/*
+ * FP8 low-bit format (fmt 1; a reading for the third precision point the
+ * wiki summary's "Gaps" names for Blackwell -- the pages fix no FP8 recipe):
+ * per token, per group of `group` channels, symmetric:
+ *   amax = max |x| of the group (exact);
+ *   s = f16_rne(amax / 448) (the quotient in double, rounded once);
+ *   c = e4m3_rne_sat(x / s) (double quotient); all codes 0 if s == 0;
+ *   z = +0 (stored, so the layout is that of the 8-bit integer format);
+ *   dequantized x^ = s * e4m3(c).
+ */
+static void quant_group_fp8(const uint16_t *x, int n, uint8_t *codes, uint16_t *s_out,
+                            uint16_t *z_out)
+{
+    double amax = 0.0;
+    for (int i = 0; i < n; ++i) {
+        const double a = fabs(bf16_to_f64(x[i]));
+        if (a > amax)
+            amax = a;
+    }
+    const uint16_t sb = f64_to_f16_rne(amax / 448.0);
+    const double s = f16_to_f64(sb);
+    for (int i = 0; i < n; ++i)
+        codes[i] = s != 0.0 ? f64_to_e4m3_rne_sat(bf16_to_f64(x[i]) / s) : 0;
+    *s_out = sb;
+    *z_out = 0;
+}
+
 /* Quantize one row of D channels into packed codes + interleaved (s, z). */
-static void quant_row(const uint16_t *x, int D, int bits, int group, uint8_t *packed,
+static void quant_row(const uint16_t *x, int D, int bits, int group, int fmt, uint8_t *packed,
                       uint16_t *sz)
 {
     uint8_t c[512];
     for (int g = 0; g < D / group; ++g) {
-        quant_group(x + g * group, group, bits, c + g * group, &sz[2 * g], &sz[2 * g + 1]);
+        if (fmt == 1)
+            quant_group_fp8(x + g * group, group, c + g * group, &sz[2 * g], &sz[2 * g + 1]);
+        else
+            quant_group(x + g * group, group, bits, c + g * group, &sz[2 * g], &sz[2 * g + 1]);
     }
     if (bits == 8) {
         memcpy(packed, c, (size_t)D);
@@ -286,11 +362,13 @@ static void quant_row(const uint16_t *x, int D, int bits, int group, uint8_t *pa
 }
 
 /* Exposed for the quantizer pins: one row of D bf16 values. */
-int hqo_quant_row(const uint16_t *x, int D, int bits, int group, uint8_t *packed, uint16_t *sz)
+int hqo_quant_row(const uint16_t *x, int D, int bits, int group, int fmt, uint8_t *packed,
+                  uint16_t *sz)
 {
-    if ((bits != 4 && bits != 8) || group <= 0 || D % group || D > 512)
+    if ((bits != 4 && bits != 8) || group <= 0 || D % group || D > 512 || fmt < 0 || fmt > 1 ||
+        (fmt == 1 && bits != 8))
         return 1;
-    quant_row(x, D, bits, group, packed, sz);
+    quant_row(x, D, bits, group, fmt, packed, sz);
     return 0;
 }
 
@@ -310,12 +388,12 @@ int hqo_quant_row(const uint16_t *x, int D, int bits, int group, uint8_t *packed
  * depend on the order of the rows.
  */
 int hqo_pack_kv(const uint16_t *k, const uint16_t *v, const int32_t *idx, int B, int Hkv,
-                int L, int D, int window, int kv, int bits, int group, uint8_t *k_codes,
+                int L, int D, int window, int kv, int bits, int group, int fmt, uint8_t *k_codes,
                 uint8_t *v_codes, uint16_t *k_sz, uint16_t *v_sz, uint16_t *k_hi,
                 uint16_t *v_hi, int32_t *lo_pos)
 {
     if ((bits != 4 && bits != 8) || group <= 0 || D % group || D > 512 || window < 0 ||
-        kv < 0 || kv > L - window)
+        kv < 0 || kv > L - window || fmt < 0 || fmt > 1 || (fmt == 1 && bits != 8))
         return 1;
     const int n_lo = L - window - kv, n_hi = kv + window;
     const int row_bytes = D * bits / 8, ng = D / group;
@@ -344,8 +422,8 @@ int hqo_pack_kv(const uint16_t *k, const uint16_t *v, const int32_t *idx, int B,
                 ++vi;
             } else {                                     /* low row */
                 size_t r = (size_t)bh * n_lo + lo;
-                quant_row(kr, D, bits, group, k_codes + r * row_bytes, k_sz + r * 2 * ng);
-                quant_row(vr, D, bits, group, v_codes + r * row_bytes, v_sz + r * 2 * ng);
+                quant_row(kr, D, bits, group, fmt, k_codes + r * row_bytes, k_sz + r * 2 * ng);
+                quant_row(vr, D, bits, group, fmt, v_codes + r * row_bytes, v_sz + r * 2 * ng);
                 if (lo_pos)
                     lo_pos[r] = j;
                 ++lo;
@@ -382,28 +460,29 @@ int hqo_pack_kv(const uint16_t *k, const uint16_t *v, const int32_t *idx, int B,
  * call the low segment holds n_lo + 1 rows.
  */
 int hqo_kv_append(const uint16_t *k_new, const uint16_t *v_new, int B, int Hkv, int D, int L,
-                  int window, int kv, int bits, int group, int n_lo, int lo_cap,
+                  int window, int kv, int bits, int group, int fmt, int n_lo, int lo_cap,
                   uint8_t *k_codes, uint8_t *v_codes, uint16_t *k_sz, uint16_t *v_sz,
                   uint16_t *k_hi, uint16_t *v_hi, int32_t *lo_pos)
 {
     if ((bits != 4 && bits != 8) || group <= 0 || D % group || D > 512 || window < 0 ||
-        kv < 0 || n_lo != L - window - kv || n_lo < 0 || n_lo >= lo_cap)
+        kv < 0 || n_lo != L - window - kv || n_lo < 0 || n_lo >= lo_cap || fmt < 0 || fmt > 1 ||
+        (fmt == 1 && bits != 8))
         return 1;
     const int row_bytes = D * bits / 8, ng = D / group, n_hi = kv + window;
     for (long long bh = 0; bh < (long long)B * Hkv; ++bh) {
         const uint16_t *kn = k_new + (size_t)bh * D, *vn = v_new + (size_t)bh * D;
         const size_t r = (size_t)bh * lo_cap + n_lo;          /* the new low row */
         if (window == 0) {
-            quant_row(kn, D, bits, group, k_codes + r * row_bytes, k_sz + r * 2 * ng);
-            quant_row(vn, D, bits, group, v_codes + r * row_bytes, v_sz + r * 2 * ng);
+            quant_row(kn, D, bits, group, fmt, k_codes + r * row_bytes, k_sz + r * 2 * ng);
+            quant_row(vn, D, bits, group, fmt, v_codes + r * row_bytes, v_sz + r * 2 * ng);
             if (lo_pos)
                 lo_pos[r] = L;
             continue;
         }
         uint16_t *kh = k_hi + ((size_t)bh * n_hi + kv + L % window) * D;
         uint16_t *vh = v_hi + ((size_t)bh * n_hi + kv + L % window) * D;
-        quant_row(kh, D, bits, group, k_codes + r * row_bytes, k_sz + r * 2 * ng);
-        quant_row(vh, D, bits, group, v_codes + r * row_bytes, v_sz + r * 2 * ng);
+        quant_row(kh, D, bits, group, fmt, k_codes + r * row_bytes, k_sz + r * 2 * ng);
+        quant_row(vh, D, bits, group, fmt, v_codes + r * row_bytes, v_sz + r * 2 * ng);
         if (lo_pos)
             lo_pos[r] = L - window;
         memcpy(kh, kn, sizeof(uint16_t) * D);
@@ -427,20 +506,23 @@ int hqo_kv_append(const uint16_t *k_new, const uint16_t *v_new, int B, int Hkv, 
  * q: bf16 [B, Hq, D];  out: double [B, Hq, D];  lse: double [B, Hq] (nullable,
  * natural-log sum of exp of the scaled logits).
  */
-static double dequant(const uint8_t *row, const uint16_t *sz, int bits, int group, int d)
+static double dequant(const uint8_t *row, const uint16_t *sz, int bits, int group, int fmt, int d)
 {
+    const int g = d / group;
+    if (fmt == 1)                                    /* FP8: s * e4m3(c) */
+        return f16_to_f64(sz[2 * g]) * e4m3_to_f64(row[d]);
     int c = bits == 8 ? row[d] : ((row[d >> 1] >> ((d & 1) * 4)) & 0xf);
-    int g = d / group;
     return f16_to_f64(sz[2 * g]) * (double)c + f16_to_f64(sz[2 * g + 1]);
 }
 
 int hqo_decode_attn(const uint16_t *q, const uint8_t *k_codes, const uint8_t *v_codes,
                     const uint16_t *k_sz, const uint16_t *v_sz, const uint16_t *k_hi,
                     const uint16_t *v_hi, int B, int Hq, int Hkv, int D, int n_lo, int n_hi,
-                    int bits, int group, double scale, double *out, double *lse)
+                    int bits, int group, int fmt, double scale, double *out, double *lse)
 {
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || n_lo < 0 || n_hi < 0 ||
-        n_lo + n_hi <= 0 || (bits != 4 && bits != 8) || group <= 0 || D % group)
+        n_lo + n_hi <= 0 || (bits != 4 && bits != 8) || group <= 0 || D % group || fmt < 0 ||
+        fmt > 1 || (fmt == 1 && bits != 8))
         return 1;
     const int G = Hq / Hkv, row_bytes = D * bits / 8, ng = D / group;
     const long long nbh = (long long)B * Hq;
@@ -458,7 +540,7 @@ int hqo_decode_attn(const uint16_t *q, const uint8_t *k_codes, const uint8_t *v_
                 const uint8_t *cr = k_codes + (bh * n_lo + t) * row_bytes;
                 const uint16_t *sz = k_sz + (bh * n_lo + t) * 2 * ng;
                 for (int d = 0; d < D; ++d)
-                    acc += bf16_to_f64(qr[d]) * dequant(cr, sz, bits, group, d);
+                    acc += bf16_to_f64(qr[d]) * dequant(cr, sz, bits, group, fmt, d);
             } else {
                 const uint16_t *kr = k_hi + (bh * n_hi + (t - n_lo)) * D;
                 for (int d = 0; d < D; ++d)
@@ -481,7 +563,7 @@ int hqo_decode_attn(const uint16_t *q, const uint8_t *k_codes, const uint8_t *v_
                 const uint8_t *cr = v_codes + (bh * n_lo + t) * row_bytes;
                 const uint16_t *sz = v_sz + (bh * n_lo + t) * 2 * ng;
                 for (int d = 0; d < D; ++d)
-                    o[d] += p * dequant(cr, sz, bits, group, d);
+                    o[d] += p * dequant(cr, sz, bits, group, fmt, d);
             } else {
                 const uint16_t *vr = v_hi + (bh * n_hi + (t - n_lo)) * D;
                 for (int d = 0; d < D; ++d)

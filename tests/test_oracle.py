@@ -150,6 +150,94 @@ def test_quant_round_trip_bound(bits):
 
 
 # --------------------------------------------------------------------------
+# FP8 (E4M3) low-bit format
+# --------------------------------------------------------------------------
+
+def _e4m3_torch(codes) -> np.ndarray:
+    """Decode E4M3 bytes with torch's float8_e4m3fn (library routine)."""
+    t = torch.as_tensor(np.asarray(codes, np.uint8)).view(torch.float8_e4m3fn)
+    return t.to(torch.float64).numpy()
+
+
+def test_e4m3_decode_all_codes_matches_torch():
+    ref = _e4m3_torch(np.arange(256))
+    got = np.array([oracle.e4m3_to_f64(c) for c in range(256)])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan) and nan.sum() == 2        # S.1111.111 only
+    assert np.array_equal(got[~nan], ref[~nan])
+    assert got[0x7E] == 448.0 and got[0x01] == 2.0 ** -9 and got[0x08] == 2.0 ** -6
+
+
+def test_e4m3_encode_round_trip_ties_and_saturation():
+    vals = np.array([oracle.e4m3_to_f64(c) for c in range(256)])
+    for c in range(256):
+        if c & 0x7F == 0x7F:
+            continue
+        assert oracle.f64_to_e4m3(vals[c]) == c, c                        # exact values
+    pos = [c for c in range(0x7F)]                                        # 0 .. 448 ascending
+    for lo_c, hi_c in zip(pos[:-1], pos[1:]):
+        mid = (vals[lo_c] + vals[hi_c]) / 2                               # ties: even code
+        assert oracle.f64_to_e4m3(mid) == (lo_c if lo_c % 2 == 0 else hi_c)
+        assert oracle.f64_to_e4m3(-mid) == 0x80 | (lo_c if lo_c % 2 == 0 else hi_c)
+        assert oracle.f64_to_e4m3(np.nextafter(mid, 0)) == lo_c
+        assert oracle.f64_to_e4m3(np.nextafter(mid, 1e9)) == hi_c
+    for v in (448.0, 460.0, 464.0, 480.0, 1e6, np.inf):                   # satfinite
+        assert oracle.f64_to_e4m3(v) == 0x7E and oracle.f64_to_e4m3(-v) == 0xFE
+    assert oracle.f64_to_e4m3(-0.0) == 0x80 and oracle.f64_to_e4m3(-1e-9) == 0x80
+    # in range, RNE agrees with torch's float32 -> float8_e4m3fn cast
+    x = (RNG.standard_normal(20000) * RNG.choice([1e-3, 0.1, 1.0, 50.0], 20000)).astype(np.float32)
+    x = x[np.abs(x) < 440]
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle.f64_to_e4m3(float(v)) for v in x], np.uint8)
+    assert np.array_equal(got, ref)
+
+
+def _fp8_row(xb):
+    packed, sz = oracle.quant_row(xb, 8, 32, oracle.FMT_FP8)
+    s = np.array([float(np.frombuffer(np.uint16(b).tobytes(), np.float16)[0]) for b in sz[0::2]])
+    z = sz[1::2]
+    return packed, s, z
+
+
+def test_fp8_quant_closed_forms():
+    # power-of-two scale: values that are E4M3 numbers times 2^-3, with the
+    # group maximum 448 * 2^-3, quantize exactly
+    codes = RNG.integers(0, 0x7E, 32).astype(np.uint8) | (RNG.integers(0, 2, 32).astype(np.uint8) << 7)
+    codes[5] = 0x7E
+    x = _e4m3_torch(codes) * 2.0 ** -3
+    packed, s, z = _fp8_row(bf16(np.concatenate([x, x, x, x])))
+    assert np.all(s == 2.0 ** -3) and np.all(z == 0)
+    got = _e4m3_torch(packed[:32])
+    assert np.array_equal(got * s[0], x)
+    # constant group: every code is 448 (or -448), the scale is fp16(|c| / 448)
+    for val in (1.0, -3.25, 1e-3):
+        packed, s, z = _fp8_row(bf16(np.full(128, val)))
+        assert np.all(packed == (0x7E if val > 0 else 0xFE))
+        assert np.all(s == float(np.float16(abs(float(bf16([val])[0])) / 448)))
+    # zero group: scale 0, codes 0
+    packed, s, z = _fp8_row(bf16(np.zeros(128)))
+    assert np.all(packed == 0) and np.all(s == 0)
+
+
+def test_fp8_quant_round_trip_bound():
+    x = RNG.standard_normal((200, 128)) * RNG.choice([0.01, 1.0, 10.0], (200, 1))
+    xb = bf16(x)
+    for r in range(200):
+        packed, s, z = _fp8_row(xb[r])
+        xv = f64(xb[r]).numpy()
+        xh = _e4m3_torch(packed) * np.repeat(s, 32)
+        for g in range(4):
+            seg, hg = xv[32 * g:32 * g + 32], xh[32 * g:32 * g + 32]
+            amax = np.abs(seg).max()
+            assert s[g] == float(np.float16(amax / 448))
+            # half a unit of the 3-bit mantissa, or of the subnormal spacing,
+            # plus the saturation slack of a rounded-down scale
+            bound = np.maximum(np.abs(hg) * 2.0 ** -4, s[g] * 2.0 ** -10) + amax * 2.0 ** -10
+            assert np.all(np.abs(hg - seg) <= bound * (1 + 1e-12))
+            assert np.all(np.sign(hg) * np.sign(seg) >= 0)
+
+
+# --------------------------------------------------------------------------
 # Probe (column sums) and top-k
 # --------------------------------------------------------------------------
 
@@ -247,8 +335,9 @@ def test_pack_partition_and_rows(bits):
 # Decode cache maintenance: append = pack of the longer prefix
 # --------------------------------------------------------------------------
 
-@pytest.mark.parametrize("bits,D,W", [(4, 64, 32), (8, 64, 32), (4, 128, 7), (8, 128, 0)])
-def test_append_equals_pack_of_longer_prefix(bits, D, W):
+@pytest.mark.parametrize("bits,D,W,fmt", [(4, 64, 32, 0), (8, 64, 32, 0), (4, 128, 7, 0),
+                                         (8, 128, 0, 0), (8, 128, 16, 1)])
+def test_append_equals_pack_of_longer_prefix(bits, D, W, fmt):
     """Packing L0 tokens and appending tokens L0 .. L0+t-1 one by one gives the
     cache packed from L0 + t tokens with the same vertical set, field for
     field: the evicted position, its low row, lo_pos, the ring slot and the
@@ -258,10 +347,10 @@ def test_append_equals_pack_of_longer_prefix(bits, D, W):
     v = bf16(RNG.standard_normal((B, Hkv, L0 + t, D)))
     idx = np.sort(np.stack([np.stack([RNG.choice(L0 - W, kv, replace=False) for _ in range(Hkv)])
                             for _ in range(B)]), -1).astype(np.int32)
-    c = oracle.pack_kv(k[:, :, :L0], v[:, :, :L0], idx, W, bits, 32)
+    c = oracle.pack_kv(k[:, :, :L0], v[:, :, :L0], idx, W, bits, 32, fmt)
     for L in range(L0, L0 + t):
         c = oracle.kv_append(c, k[:, :, L], v[:, :, L], L, W)
-    ref = oracle.pack_kv(k, v, idx, W, bits, 32)
+    ref = oracle.pack_kv(k, v, idx, W, bits, 32, fmt)
     assert c["n_lo"] == ref["n_lo"] and c["n_hi"] == ref["n_hi"]
     for name in ("k_codes", "v_codes", "k_sz", "v_sz", "k_hi", "v_hi", "lo_pos"):
         assert np.array_equal(c[name], ref[name]), name
@@ -349,21 +438,22 @@ def _dequant_np(codes, sz, bits, D):
     return c * np.repeat(s, 32, axis=1) + np.repeat(z, 32, axis=1)
 
 
-@pytest.mark.parametrize("bits", [4, 8])
-def test_decode_matches_dequantize_then_attend(bits):
+@pytest.mark.parametrize("bits,fmt", [(4, 0), (8, 0), (8, 1)])
+def test_decode_matches_dequantize_then_attend(bits, fmt):
     w = Workload("t", "decode", 2, 4, 2, 64, 256, 32, F5, bits, 7)
     x = make_inputs(w)
     sc = oracle.probe_scores(x["q_probe"], x["k"], w.Hkv)
     idx = oracle.topk(sc, w.window, w.k_vert)
-    c = oracle.pack_kv(x["k"], x["v"], idx, w.window, bits)
+    c = oracle.pack_kv(x["k"], x["v"], idx, w.window, bits, 32, fmt)
+    dq = _dequant_np if fmt == 0 else (lambda codes, sz, bits_, D: _dequant_fp8_np(codes, sz, D))
     out, lse = oracle.decode_attn(x["q"], c, w.Hkv)
     for b in range(w.B):
         for h in range(w.Hq):
             kh = h // w.G
-            kd = np.concatenate([_dequant_np(c["k_codes"][b, kh], c["k_sz"][b, kh], bits, w.D),
+            kd = np.concatenate([dq(c["k_codes"][b, kh], c["k_sz"][b, kh], bits, w.D),
                                  f64(x["k"][b, kh][np.concatenate(
                                      [idx[b, kh], np.arange(w.L - w.window, w.L)])]).numpy()])
-            vd = np.concatenate([_dequant_np(c["v_codes"][b, kh], c["v_sz"][b, kh], bits, w.D),
+            vd = np.concatenate([dq(c["v_codes"][b, kh], c["v_sz"][b, kh], bits, w.D),
                                  f64(x["v"][b, kh][np.concatenate(
                                      [idx[b, kh], np.arange(w.L - w.window, w.L)])]).numpy()])
             qd = f64(x["q"][b, h]).numpy()
@@ -377,6 +467,12 @@ def test_decode_matches_dequantize_then_attend(bits):
     exact = _sdpa(x["q"][:, :, None], kk, vv, 1 / math.sqrt(w.D))[:, :, 0].numpy()
     err = np.abs(out - exact).mean()
     assert 0 < err < (0.5 if bits == 4 else 0.05)
+
+
+def _dequant_fp8_np(codes, sz, D):
+    """s * e4m3(c) with torch's float8 decoding and numpy float16 scales."""
+    s = np.asarray(sz).reshape(codes.shape[0], D // 32, 2)[..., 0].view(np.float16).astype(np.float64)
+    return _e4m3_torch(codes) * np.repeat(s, 32, axis=1)
 
 
 # --------------------------------------------------------------------------
