@@ -62,6 +62,10 @@ typedef enum {
     HQ_ERR_SCRATCH_LIMIT = 7  /* the problem needs more scratch than a fixed-size buffer holds */
 } hq_status;
 
+/* Low-bit code formats of a hybrid KV cache (hq_kv_cache.fmt). */
+#define HQ_KV_INT 0   /* asymmetric integer codes, 4 or 8 bits: x^ = s * c + z */
+#define HQ_KV_FP8 1   /* FP8 E4M3 codes, 8 bits, symmetric: x^ = s * e4m3(c), z stored as 0 */
+
 /* Device status word bits (hq_read_device_status). */
 #define HQ_DEV_BAD_INDEX 0x1u   /* an index list was unsorted, repeated or out of range */
 #define HQ_DEV_TIMEOUT 0x2u     /* a bounded inter-CTA wait gave up */
@@ -91,6 +95,13 @@ int hq_version(void);
  *   lo_cap           : low rows allocated per (b, kv head); 0 means n_lo.
  *                      Spare rows let hq_kv_append grow the low segment in
  *                      place during decode.  Rows n_lo..C-1 are never read.
+ *   fmt              : HQ_KV_INT (0) or HQ_KV_FP8 (1, with bits == 8).  The
+ *                      FP8 format answers the wiki summary's "Gaps" remark
+ *                      that Blackwell offers FP8 as a third precision point;
+ *                      the recipe is the library's reading: per token and
+ *                      group, s = fp16(amax / 448) (amax = largest |x|, the
+ *                      quotient rounded once), c = E4M3 of x / s rounded to
+ *                      nearest even and saturated to +-448, z = 0.
  * All pointers must be 16-byte aligned.  The low rows are stored in ascending
  * position order, with no copy of the vertical rows: attention does not depend
  * on key order, and storing a vertical row only once is what gives the
@@ -109,6 +120,7 @@ typedef struct {
     int bits;
     int group;
     int lo_cap;
+    int fmt;
 } hq_kv_cache;
 
 /*
@@ -152,11 +164,13 @@ hq_status hq_probe_vertical(const void *q_probe, int64_t q_head_stride, const vo
  * Splits [0, L) of every (b, kv head) into the window [L - window, L), the
  * vertical columns idx (ascending, distinct, in [0, L - window)) and the low
  * rows (everything else), and writes `out` as described at hq_kv_cache.
- * Quantizer, per token and group of `group` channels, `bits`-bit asymmetric:
+ * Quantizer (out->fmt == HQ_KV_INT), per token and group of `group`
+ * channels, `bits`-bit asymmetric:
  *   s = f16_rne((max - min) / (2^bits - 1)),  z = f16_rne(min),
- *   code = clamp(rne((x - z) / s), 0, 2^bits - 1), all 0 when s == 0,
- * with every intermediate taken in IEEE double so that each rounding decision
- * is exact and reproducible.  out->n_lo / n_hi / bits / group must equal
+ *   code = clamp(rne((x - z) / s), 0, 2^bits - 1), all 0 when s == 0;
+ * with out->fmt == HQ_KV_FP8 (bits 8) the FP8 recipe at hq_kv_cache.  Every
+ * intermediate is taken in IEEE double so that each rounding decision is
+ * exact and reproducible.  out->n_lo / n_hi / bits / group must equal
  * L - window - k_vert, k_vert + window, bits and group.  An idx list that is
  * unsorted, repeated or out of range sets HQ_DEV_BAD_INDEX in the status word
  * of `ws` (if given) and leaves the affected rows unwritten.

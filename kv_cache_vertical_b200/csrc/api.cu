@@ -26,6 +26,11 @@ uint32_t *status_word(void *ws) { return ws ? reinterpret_cast<uint32_t *>(ws) :
 
 bool lo_cap_ok(const hq_kv_cache &c) { return c.lo_cap == 0 || c.lo_cap >= c.n_lo; }
 
+// HQ_KV_FP8 is an 8-bit format; any other fmt value is not supported.
+bool fmt_ok(const hq_kv_cache &c) {
+  return c.fmt == HQ_KV_INT || (c.fmt == HQ_KV_FP8 && c.bits == 8);
+}
+
 }  // namespace
 
 namespace hq {
@@ -38,7 +43,7 @@ hq_status check_decode_args(const void *q, const hq_kv_cache *cache, int B, int 
       cache->n_lo + cache->n_hi <= 0 || !lo_cap_ok(*cache))
     return HQ_ERR_INVALID_ARG;
   if ((D != 64 && D != 128) || !supported_G(Hq, Hkv) || (cache->bits != 4 && cache->bits != 8) ||
-      cache->group != 32)
+      cache->group != 32 || !fmt_ok(*cache))
     return HQ_ERR_UNSUPPORTED;
   if ((cache->n_lo > 0 && (!cache->k_codes || !cache->v_codes || !cache->k_sz || !cache->v_sz)) ||
       (cache->n_hi > 0 && (!cache->k_hi || !cache->v_hi)))
@@ -110,6 +115,7 @@ hq_status hq_pack_kv(const void *k, const void *v, const int32_t *idx, int B, in
   if (B <= 0 || Hkv <= 0 || L <= 0 || window < 0 || k_vert < 0 || k_vert > L - window)
     return HQ_ERR_INVALID_ARG;
   if ((D != 64 && D != 128) || (bits != 4 && bits != 8) || group != 32) return HQ_ERR_UNSUPPORTED;
+  if (out->bits == bits && !fmt_ok(*out)) return HQ_ERR_UNSUPPORTED;
   const int n_lo = L - window - k_vert, n_hi = k_vert + window;
   if (out->n_lo != n_lo || out->n_hi != n_hi || out->bits != bits || out->group != group ||
       !lo_cap_ok(*out))
@@ -130,7 +136,8 @@ hq_status hq_kv_append(const void *k_new, const void *v_new, int B, int Hkv, int
                        int window, int k_vert, const hq_kv_cache *cache, void *stream) {
   if (!k_new || !v_new || !cache) return HQ_ERR_INVALID_ARG;
   if (B <= 0 || Hkv <= 0 || window < 0 || k_vert < 0 || L < window + k_vert) return HQ_ERR_INVALID_ARG;
-  if ((D != 64 && D != 128) || (cache->bits != 4 && cache->bits != 8) || cache->group != 32)
+  if ((D != 64 && D != 128) || (cache->bits != 4 && cache->bits != 8) || cache->group != 32 ||
+      !fmt_ok(*cache))
     return HQ_ERR_UNSUPPORTED;
   if (cache->n_lo != L - window - k_vert || cache->n_hi != k_vert + window ||
       cache->lo_cap <= cache->n_lo)
@@ -161,7 +168,7 @@ hq_status hq_decode_attn(const void *q, const hq_kv_cache *cache, int B, int Hq,
       cache->n_lo + cache->n_hi <= 0 || !lo_cap_ok(*cache))
     return HQ_ERR_INVALID_ARG;
   if ((D != 64 && D != 128) || !supported_G(Hq, Hkv) || (cache->bits != 4 && cache->bits != 8) ||
-      cache->group != 32)
+      cache->group != 32 || !fmt_ok(*cache))
     return HQ_ERR_UNSUPPORTED;
   if ((cache->n_lo > 0 && (!cache->k_codes || !cache->v_codes || !cache->k_sz || !cache->v_sz)) ||
       (cache->n_hi > 0 && (!cache->k_hi || !cache->v_hi)))

@@ -15,6 +15,8 @@
 // tensor-core kernel of decode_tma.cu.
 #include <float.h>
 
+#include <cuda_fp8.h>
+
 #include "hq_internal.cuh"
 
 namespace hq {
@@ -29,6 +31,7 @@ struct DecodeArgs {
   const __half2 *k_sz, *v_sz;
   const __nv_bfloat16 *k_hi, *v_hi;
   int Hq, Hkv, G, n_lo, n_hi, lo_cap, nsplit;
+  int fp8;           // low rows hold FP8 E4M3 codes (x^ = s * e4m3(c)) instead of integers
   float scale_log2;
   float *part_o;     // [B*Hq, nsplit, D]
   float2 *part_ml;   // [B*Hq, nsplit]
@@ -38,7 +41,7 @@ struct DecodeArgs {
 template <int D, int BITS>
 __device__ __forceinline__ void load_row(const uint8_t *codes, const __half2 *sz,
                                          const __nv_bfloat16 *hi, int n_lo, int n_hi, int lo_cap,
-                                         size_t bh, int t, int lane, float (&x)[D / 32]) {
+                                         bool fp8, size_t bh, int t, int lane, float (&x)[D / 32]) {
   constexpr int CPL = D / 32;
   if (t < n_lo) {
     const size_t row = bh * lo_cap + t;
@@ -55,8 +58,14 @@ __device__ __forceinline__ void load_row(const uint8_t *codes, const __half2 *sz
 #pragma unroll
       for (int i = 0; i < CPL; ++i) c[i] = (w >> (8 * i)) & 0xff;
     }
+    if (BITS == 8 && fp8) {
 #pragma unroll
-    for (int i = 0; i < CPL; ++i) x[i] = fmaf(s_z.x, (float)c[i], s_z.y);
+      for (int i = 0; i < CPL; ++i)
+        x[i] = s_z.x * __half2float(__half(__nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)c[i], __NV_E4M3)));
+    } else {
+#pragma unroll
+      for (int i = 0; i < CPL; ++i) x[i] = fmaf(s_z.x, (float)c[i], s_z.y);
+    }
   } else {
     const uint32_t *hr = reinterpret_cast<const uint32_t *>(hi + (bh * n_hi + (t - n_lo)) * D);
 #pragma unroll
@@ -99,8 +108,8 @@ __global__ void __launch_bounds__(DWARPS * 32) decode_split(DecodeArgs a) {
   }
   for (int t = t0 + warp; t < t1; t += DWARPS) {
     float kx[CPL], vx[CPL];
-    load_row<D, BITS>(a.k_codes, a.k_sz, a.k_hi, a.n_lo, a.n_hi, a.lo_cap, (size_t)bh, t, lane, kx);
-    load_row<D, BITS>(a.v_codes, a.v_sz, a.v_hi, a.n_lo, a.n_hi, a.lo_cap, (size_t)bh, t, lane, vx);
+    load_row<D, BITS>(a.k_codes, a.k_sz, a.k_hi, a.n_lo, a.n_hi, a.lo_cap, a.fp8 != 0, (size_t)bh, t, lane, kx);
+    load_row<D, BITS>(a.v_codes, a.v_sz, a.v_hi, a.n_lo, a.n_hi, a.lo_cap, a.fp8 != 0, (size_t)bh, t, lane, vx);
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       float s = 0.f;
@@ -232,6 +241,7 @@ cudaError_t launch_decode(const __nv_bfloat16 *q, const hq_kv_cache &c, int B, i
   a.n_lo = c.n_lo;
   a.n_hi = c.n_hi;
   a.lo_cap = lo_rows(c);
+  a.fp8 = c.fmt == HQ_KV_FP8;
   const int nbh = B * Hkv;
   a.nsplit = choose_nsplit(nbh, c.n_lo + c.n_hi);
   a.scale_log2 = scale * kLog2e;

@@ -121,6 +121,20 @@ __device__ __forceinline__ uint32_t hmul2_u(uint32_t a, uint32_t b) {
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
   return pack_f16x2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
 }
+// Two FP8 E4M3 bytes, placed by `sel` in the high byte of each 16-bit half,
+// as the fp16 patterns of e4m3(b) * 2^-8 (exact for every code, subnormals
+// included): shifting each half right by one puts the 4-bit exponent and the
+// 3-bit mantissa where fp16 keeps them (the bias difference 15 - 7 becomes
+// the factor 2^-8) and the sign one place low; adding the sign bit to itself
+// moves it up.  Four integer operations per pair, cheaper here than the
+// hardware conversion.
+constexpr float kF8Unit = 256.0f;            // the 2^-8 comes back in fp32
+__device__ __forceinline__ uint32_t f8pair(uint32_t w, uint32_t sel) {
+  uint32_t x;
+  asm("prmt.b32 %0, %1, %2, %3;\n" : "=r"(x) : "r"(w), "r"(0u), "r"(sel));
+  const uint32_t t = x >> 1;
+  return t + (t & 0x40004000u);
+}
 __device__ __forceinline__ float half_lo_f(uint32_t w) {
   return __half2float(__ushort_as_half((unsigned short)(w & 0xffffu)));
 }
@@ -141,7 +155,7 @@ __device__ __forceinline__ uint32_t swz_off(int row, int ch) {
   return row * 128 + ((ch ^ (row & 7)) << 4);
 }
 
-template <int BITS, int G>
+template <int BITS, int G, bool F8>
 __global__ void __launch_bounds__(NTHREADS, 3)
 decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_vc,
            const __grid_constant__ CUtensorMap tm_ksz, const __grid_constant__ CUtensorMap tm_vsz,
@@ -416,6 +430,25 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
                 mma_f16_16816(acc[g], fb, qb[2 * g + 1][0], qb[2 * g + 1][1]);
               }
             }
+          } else if (F8) {
+            // FP8 codes become fp16 values (times 2^-8) from the same byte
+            // pairs as the integer path, so the q fragments are shared
+  #pragma unroll
+            for (int cp = 0; cp < 4; ++cp) {
+              uint32_t kx[4];
+              ldsm_x4(kx, st + swz_off<C::ROWB>(lrow, 2 * cp + (mi >> 1)));
+  #pragma unroll
+              for (int cc = 0; cc < 2; ++cc) {
+                const int kc = 2 * cp + cc;
+                const uint32_t A0 = kx[2 * cc], A1 = kx[2 * cc + 1];
+                uint32_t fa[4];
+                fa[0] = f8pair(A0, 0x1404);       // bytes 0, 1
+                fa[1] = f8pair(A1, 0x1404);
+                fa[2] = f8pair(A0, 0x3424);       // bytes 2, 3
+                fa[3] = f8pair(A1, 0x3424);
+                mma_f16_16816(acc[kc >> 1], fa, qb[kc][0], qb[kc][1]);
+              }
+            }
           } else {
   #pragma unroll
             for (int cp = 0; cp < 4; ++cp) {
@@ -450,7 +483,7 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
           za[2] = 0u;
           za[3] = 0u;
           float zacc[4] = {0.f, 0.f, 0.f, 0.f};
-          mma_f16_16816(zacc, za, zb0, 0u);
+          if (!F8) mma_f16_16816(zacc, za, zb0, 0u);   // FP8 has no zero point
           float y[4] = {0.f, 0.f, 0.f, 0.f};
   #pragma unroll
           for (int g = 0; g < 4; ++g) {
@@ -461,7 +494,7 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
             y[3] = fmaf(sb, acc[g][3], y[3]);
           }
   #pragma unroll
-          for (int e = 0; e < 4; ++e) x[e] = fmaf(y[e], kCodeUnit, zacc[e]);
+          for (int e = 0; e < 4; ++e) x[e] = F8 ? y[e] * kF8Unit : fmaf(y[e], kCodeUnit, zacc[e]);
         } else {
           float acc[4] = {0.f, 0.f, 0.f, 0.f};
           const int mi = lane >> 3;
@@ -539,7 +572,7 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
             zaf[1] = 0u;
             zaf[2] = prmt(zc, zd, 0x7632);
             zaf[3] = 0u;
-            mma_f16_16816(oz, zaf, pb0, pb1);
+            if (!F8) mma_f16_16816(oz, zaf, pb0, pb1);
           }
           const int mi = lane >> 3;
           const int lrow = row0 + (mi & 1) * 8 + (lane & 7);
@@ -567,6 +600,26 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
                 fb[3] = Xp8 & 0x00F000F0u;
                 mma_f16_16816(o[2 * g], fa, bs0, bs1);
                 mma_f16_16816(o[2 * g + 1], fb, bs0, bs1);
+              }
+            }
+          } else if (F8) {
+  #pragma unroll
+            for (int cp = 0; cp < 4; ++cp) {
+              uint32_t vx[4];
+              ldsm_x4_t(vx, vbase + swz_off<C::ROWB>(lrow, 2 * cp + (mi >> 1)));
+              const int g = cp;  // chunks 2cp, 2cp+1 form group cp
+              const uint32_t bs0 = hmul2_u(pb0, prmt(A_[g], B_[g], 0x5410));
+              const uint32_t bs1 = hmul2_u(pb1, prmt(C_[g], D_[g], 0x5410));
+  #pragma unroll
+              for (int cc = 0; cc < 2; ++cc) {
+                const uint32_t X = vx[2 * cc], Xp = vx[2 * cc + 1];
+                uint32_t fa[4];
+                // the byte pairs (0, 2) and (1, 3) of the integer path
+                fa[0] = f8pair(X, 0x2404);        // bytes 0, 2
+                fa[1] = f8pair(X, 0x3414);        // bytes 1, 3
+                fa[2] = f8pair(Xp, 0x2404);
+                fa[3] = f8pair(Xp, 0x3414);
+                mma_f16_16816(o[2 * cp + cc], fa, bs0, bs1);
               }
             }
           } else {
@@ -641,7 +694,7 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
           else if (BITS == 4) ch = 32 * (mt >> 1) + 4 * r + 2 * (mt & 1) + hf;
           else ch = 16 * mt + 2 * r + hf;
           // undo the code unit of the low-bit V operand
-          const float u = hi ? 1.f : (BITS == 4 && hf == 1 ? kHiNibbleUnit : kCodeUnit);
+          const float u = hi ? 1.f : F8 ? kF8Unit : (BITS == 4 && hf == 1 ? kHiNibbleUnit : kCodeUnit);
           wo[(warp * 8 + 2 * c) * D + ch] = o[mt][2 * hf] * u;
           wo[(warp * 8 + 2 * c + 1) * D + ch] = o[mt][2 * hf + 1] * u;
         }
@@ -842,14 +895,18 @@ struct Plan {
   int nslot() const { return nc_lo + nc_hi + 2 * nbh; }
 };
 
-template <int BITS, int G>
+// Resident CTAs per SM of one kernel variant (sets its shared memory limit
+// once).  Plans (and so workspace sizes) use the integer variant's figure for
+// both code formats; a grid is correct whatever its residency, since no CTA
+// waits for another.
+template <int BITS, int G, bool F8 = false>
 int occupancy() {
   static int occ = -1;
   if (occ < 0) {
-    cudaFuncSetAttribute(decode_tma<BITS, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(decode_tma<BITS, G, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          Cfg<BITS>::SMEM);
     int o = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, decode_tma<BITS, G>, NTHREADS,
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, decode_tma<BITS, G, F8>, NTHREADS,
                                                       Cfg<BITS>::SMEM) != cudaSuccess || o < 1)
       o = 1;
     occ = o;
@@ -933,7 +990,7 @@ WsLayout ws_layout(int B, int Hkv, int G, int nslot) {
   return w;
 }
 
-template <int BITS, int G>
+template <int BITS, int G, bool F8>
 cudaError_t launch_tg(const DecArgs &a0, const hq_kv_cache &c, int nbh, cudaStream_t s) {
   DecArgs a = a0;
   // The six tensor maps depend only on the cache buffers and sizes; the last
@@ -973,8 +1030,8 @@ cudaError_t launch_tg(const DecArgs &a0, const hq_kv_cache &c, int nbh, cudaStre
     mc.nbh = nbh;
   }
   const CUtensorMap *m = mc.m;
-  occupancy<BITS, G>();  // sets the dynamic shared memory attribute once
-  return pdl_launch(decode_tma<BITS, G>, dim3(a.nc_lo + a.nc_hi), dim3(NTHREADS), Cfg<BITS>::SMEM, s,
+  occupancy<BITS, G, F8>();  // sets the dynamic shared memory attribute once
+  return pdl_launch(decode_tma<BITS, G, F8>, dim3(a.nc_lo + a.nc_hi), dim3(NTHREADS), Cfg<BITS>::SMEM, s,
                     m[0], m[1], m[2], m[3], m[4], m[5], a);
 }
 
@@ -1021,9 +1078,12 @@ cudaError_t launch_decode_tma(const __nv_bfloat16 *q, const hq_kv_cache &c, int 
   a.nc_lo = p.nc_lo;
   a.nc_hi = p.nc_hi;
   a.sl = scale * kLog2e;
-#define HQ_L(BITS, GG) if (c.bits == BITS && G == GG) return launch_tg<BITS, GG>(a, c, nbh, s);
-  HQ_L(4, 1) HQ_L(4, 2) HQ_L(4, 4) HQ_L(4, 8)
-  HQ_L(8, 1) HQ_L(8, 2) HQ_L(8, 4) HQ_L(8, 8)
+  const bool f8 = c.fmt == HQ_KV_FP8;
+#define HQ_L(BITS, GG, FF) \
+  if (c.bits == BITS && G == GG && f8 == FF) return launch_tg<BITS, GG, FF>(a, c, nbh, s);
+  HQ_L(4, 1, false) HQ_L(4, 2, false) HQ_L(4, 4, false) HQ_L(4, 8, false)
+  HQ_L(8, 1, false) HQ_L(8, 2, false) HQ_L(8, 4, false) HQ_L(8, 8, false)
+  HQ_L(8, 1, true) HQ_L(8, 2, true) HQ_L(8, 4, true) HQ_L(8, 8, true)
 #undef HQ_L
   return cudaErrorInvalidValue;
 }

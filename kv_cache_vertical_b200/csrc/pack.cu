@@ -15,6 +15,7 @@
 // near a tie), so the codes, scales and zeros are exactly the ones the
 // library's specification defines.  HBM-bound: read 2 * D * 2 bytes per position, write
 // the packed rows.
+#include <cuda_fp8.h>
 #include <limits.h>
 
 #include "hq_internal.cuh"
@@ -104,7 +105,114 @@ __device__ __forceinline__ void quant_store(const uint32_t (&w)[D / 64], uint8_t
   if (lane % LPG == 0) sz_row[lane / LPG] = __halves2half2(hs, hz);
 }
 
-template <int D, int BITS>
+// The double d rounded to fp32 toward zero, with the last bit set when that
+// dropped anything (round to odd).  Rounding this to a format with far fewer
+// bits (E4M3 keeps 4) gives the same result as rounding d itself.
+__device__ __forceinline__ float f32_round_odd(double d) {
+  const float r = __double2float_rz(d);
+  return (double)r == d ? r : __uint_as_float(__float_as_uint(r) | 1u);
+}
+
+// True when an fp32 estimate q (relative error a few units of 2^-24) of a
+// quotient lies so close to a point halfway between two E4M3 neighbours that
+// the exact quotient might round the other way.  Normal range: the 20 bits
+// below the 3-bit mantissa within 16 units of the halfway pattern; subnormal
+// range (|q| < 2^-6, spacing 2^-9): the fraction of q * 2^9 within 2^-12 of 1/2.
+__device__ __forceinline__ bool e4m3_near_tie(float q) {
+  const float a = fabsf(q);
+  if (a >= 0.015625f) {
+    const uint32_t low = __float_as_uint(a) & 0xFFFFFu;
+    return low >= 0x80000u - 16u && low <= 0x80000u + 16u;
+  }
+  const float t = a * 512.f;
+  return fabsf(t - floorf(t) - 0.5f) < 1.f / 4096.f;
+}
+
+// FP8 format: per group of 32 channels s = fp16(amax / 448) (the quotient
+// rounded once: scale_f16 with range amax - 0), c = E4M3(x / s) rounded to
+// nearest even and saturated, z = 0.  The hardware conversion (nearest even,
+// saturating) rounds an fp32 estimate of x / s, except where the estimate is
+// near an E4M3 tie; there it rounds the double quotient taken to fp32 with
+// round to odd.  Bit-exact to the definition.
+template <int D>
+__device__ __forceinline__ void quant_store_fp8(const uint32_t (&w)[D / 64], uint8_t *codes_row,
+                                                __half2 *sz_row, int lane) {
+  constexpr int CPL = D / 32;          // channels per lane: 4 (D=128) or 2 (D=64)
+  constexpr int LPG = 32 / CPL;        // lanes per group
+  float x[CPL];
+#pragma unroll
+  for (int i = 0; i < CPL / 2; ++i) {
+    x[2 * i] = bf16_lo(w[i]);
+    x[2 * i + 1] = bf16_hi(w[i]);
+  }
+  float amax = fabsf(x[0]);
+#pragma unroll
+  for (int i = 1; i < CPL; ++i) amax = fmaxf(amax, fabsf(x[i]));
+#pragma unroll
+  for (int o = LPG / 2; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const __half hs = scale_f16(amax, 0.f, 448);
+  const float sf = __half2float(hs);
+  const float rs = sf != 0.f ? __frcp_rn(sf) : 0.f;
+  uint32_t c[CPL];
+#pragma unroll
+  for (int i = 0; i < CPL; i += 2) {
+    float q0 = x[i] * rs, q1 = x[i + 1] * rs;
+    if (e4m3_near_tie(q0)) q0 = f32_round_odd((double)x[i] / (double)sf);
+    if (e4m3_near_tie(q1)) q1 = f32_round_odd((double)x[i + 1] / (double)sf);
+    // one paired hardware conversion, nearest even, saturating (low byte = q0)
+    const uint32_t two = (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(q0, q1), __NV_SATFINITE, __NV_E4M3);
+    c[i] = sf != 0.f ? two & 0xffu : 0u;
+    c[i + 1] = sf != 0.f ? two >> 8 : 0u;
+  }
+  if (CPL == 4)
+    reinterpret_cast<uint32_t *>(codes_row)[lane] = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
+  else
+    reinterpret_cast<uint16_t *>(codes_row)[lane] = (uint16_t)(c[0] | (c[1] << 8));
+  if (lane % LPG == 0) sz_row[lane / LPG] = __halves2half2(hs, __ushort_as_half((unsigned short)0));
+}
+
+// One row of the low segment in the cache's code format.
+template <int D, int BITS, bool F8>
+__device__ __forceinline__ void quant_row_store(const uint32_t (&w)[D / 64], uint8_t *codes_row,
+                                                __half2 *sz_row, int lane) {
+  if (F8)
+    quant_store_fp8<D>(w, codes_row, sz_row, lane);
+  else
+    quant_store<D, BITS>(w, codes_row, sz_row, lane);
+}
+
+// Positions per CTA: kWarps warps x kChunks chunks x 8 positions.
+constexpr int kChunks = 4;
+constexpr int kSpan = kWarps * kChunks * 8;   // 256
+
+// Number of entries of the ascending list a[0, n) below x, found by one warp
+// with 32-way splits (about three rounds of loads for thousands of entries
+// instead of a dozen dependent ones).  Every lane returns the result.
+__device__ __forceinline__ int warp_count_below(const int32_t *__restrict__ a, int n, int x,
+                                                int lane) {
+  int lo = 0, hi = n;                       // the count lies in [lo, hi]
+  while (hi - lo > 32) {
+    const int len = hi - lo;
+    const int si = lo + (int)(((long long)lane * len) >> 5);        // lane 0 samples lo
+    const unsigned below = __ballot_sync(0xffffffffu, __ldg(a + si) < x);
+    const int m = __popc(below);            // samples 0 .. m-1 are below x
+    if (m == 0) return lo;
+    const int s_last = lo + (int)(((long long)(m - 1) * len) >> 5);
+    const int s_next = m < 32 ? lo + (int)(((long long)m * len) >> 5) : hi;
+    lo = s_last + 1;
+    hi = s_next;
+  }
+  const bool in = lane < hi - lo;
+  const unsigned below = __ballot_sync(0xffffffffu, in && __ldg(a + lo + (in ? lane : 0)) < x);
+  return lo + __popc(below);
+}
+
+// One CTA per span of kSpan consecutive positions of one (b, kv head): warp 0
+// counts the vertical columns before the span (one search per CTA) and marks
+// those inside it in a shared bit mask, while every warp issues the row loads
+// of its first chunk; then each warp classifies and writes its four chunks of
+// eight positions (copy the bf16 rows, or quantize them into the next low rows).
+template <int D, int BITS, bool F8>
 __global__ void __launch_bounds__(kWarps * 32)
 pack_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ v,
             const int32_t *__restrict__ idx, int nbh, int L, int window, int k_vert, int lo_cap,
@@ -115,10 +223,16 @@ pack_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict
   constexpr int W32 = D / 64;                 // 32-bit words of bf16 per lane
   constexpr int ROWB = D * BITS / 8;          // packed bytes per low row
   constexpr int NG = D / 32;
-  const int lane = threadIdx.x & 31;
+  constexpr int PCH = 8;
+  __shared__ uint32_t vmask[kSpan / 32];
+  __shared__ int s_lo;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int n_lo = L - window - k_vert, n_hi = k_vert + window;
-  const long long warp0 = (long long)blockIdx.x * kWarps + (threadIdx.x >> 5);
-  const long long nwarps = (long long)gridDim.x * kWarps;
+  const int nspan = (L + kSpan - 1) / kSpan;
+  const int bh = (int)(blockIdx.x / nspan);
+  const int p0 = (int)(blockIdx.x % nspan) * kSpan;
+  const int p1 = min(p0 + kSpan, L);
+  const int32_t *id = idx + (size_t)bh * k_vert;
 
   // Device-side check of the index list (ascending, distinct, in range).
   for (long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x; t < (long long)nbh * k_vert;
@@ -128,23 +242,9 @@ pack_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict
     if (x < 0 || x >= L - window || (r > 0 && idx[t - 1] >= x)) raise_status(status, HQ_DEV_BAD_INDEX);
   }
 
-  // Eight consecutive positions of one pair per warp task: one binary search
-  // finds the verticals before the chunk, the next (at most eight) index
-  // entries say which chunk positions are vertical, and all sixteen row loads
-  // are issued before any quantization.
-  constexpr int PCH = 8;
-  const long long ntask = (long long)nbh * ((L + PCH - 1) / PCH);
-  const int cpb = (L + PCH - 1) / PCH;                // chunks per pair
-  for (long long task = warp0; task < ntask; task += nwarps) {
-    const int bh = (int)(task / cpb);
-    const int j0 = (int)(task % cpb) * PCH;
-    const int32_t *id = idx + (size_t)bh * k_vert;
-    const int cnt0 = j0 > 0 ? upper_bound_i32(id, k_vert, j0 - 1) : 0;   // verticals before j0
-    const int e = cnt0 + (lane & (PCH - 1));
-    const int ve = (lane < PCH && e < k_vert) ? __ldg(id + e) : INT_MAX;
-    const uint32_t vbit = (ve >= j0 && ve < j0 + PCH) ? 1u << (ve - j0) : 0u;
-    const uint32_t vbits = __reduce_or_sync(0xffffffffu, vbit);            // vertical positions of the chunk
-    uint32_t kw[PCH][W32], vw[PCH][W32];
+  if (threadIdx.x < kSpan / 32) vmask[threadIdx.x] = 0u;
+  uint32_t kw[PCH][W32], vw[PCH][W32];
+  auto load_chunk = [&](int j0) {
 #pragma unroll
     for (int p = 0; p < PCH; ++p) {
       const int j = j0 + p;
@@ -155,6 +255,34 @@ pack_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict
         vw[p][i] = __ldg(reinterpret_cast<const uint32_t *>(v + src) + lane * W32 + i);
       }
     }
+  };
+  const int jw = p0 + warp * kChunks * PCH;    // this warp's first position
+  if (jw < p1) load_chunk(jw);
+  __syncthreads();                             // mask cleared
+  if (warp == 0) {
+    const int lo = warp_count_below(id, k_vert, p0, lane);
+    if (lane == 0) s_lo = lo;
+    // mark the span's verticals (at most kSpan entries follow lo)
+    for (int t = lo + lane;; t += 32) {
+      const int x = t < k_vert ? __ldg(id + t) : INT_MAX;
+      if (x >= p0 && x < p1) atomicOr(&vmask[(x - p0) >> 5], 1u << ((x - p0) & 31));
+      if (__any_sync(0xffffffffu, x >= p1)) break;
+    }
+  }
+  __syncthreads();                             // mask and count ready
+  const int lo = s_lo;
+
+  for (int ci = 0; ci < kChunks; ++ci) {
+    const int j0 = jw + ci * PCH;
+    if (j0 >= p1) break;
+    if (ci > 0) load_chunk(j0);
+    const int o = j0 - p0;                     // offset in the span, a multiple of 8
+    uint32_t before = 0;                       // verticals in the span before j0
+    for (int wdx = 0; wdx < (o >> 5); ++wdx) before += __popc(vmask[wdx]);
+    const uint32_t word = vmask[o >> 5];
+    before += __popc(word & ((1u << (o & 31)) - 1u));
+    const uint32_t vbits = (word >> (o & 31)) & 0xffu;   // vertical positions of the chunk
+    const int cnt0 = lo + (int)before;
 #pragma unroll
     for (int p = 0; p < PCH; ++p) {
       const int j = j0 + p;
@@ -181,27 +309,21 @@ pack_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict
           continue;
         }
         const size_t r = (size_t)bh * lo_cap + lo_row;
-        quant_store<D, BITS>(kw[p], k_codes + r * ROWB, k_sz + r * NG, lane);
-        quant_store<D, BITS>(vw[p], v_codes + r * ROWB, v_sz + r * NG, lane);
+        quant_row_store<D, BITS, F8>(kw[p], k_codes + r * ROWB, k_sz + r * NG, lane);
+        quant_row_store<D, BITS, F8>(vw[p], v_codes + r * ROWB, v_sz + r * NG, lane);
         if (lo_pos && lane == 0) lo_pos[r] = j;
       }
     }
   }
 }
 
-template <int D, int BITS>
+template <int D, int BITS, bool F8>
 cudaError_t launch_pack_t(const __nv_bfloat16 *k, const __nv_bfloat16 *v, const int32_t *idx,
                           int nbh, int L, int window, int k_vert, const hq_kv_cache &o,
                           uint32_t *status, cudaStream_t s) {
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const long long warps = (long long)nbh * ((L + 7) / 8);     // one warp task per 8 positions
-  long long blocks = (warps + kWarps - 1) / kWarps;
-  const long long cap = (long long)sms * 8;
-  if (blocks > cap) blocks = cap;
-  if (blocks < 1) blocks = 1;
-  pack_kernel<D, BITS><<<(unsigned)blocks, kWarps * 32, 0, s>>>(
+  const long long blocks = (long long)nbh * ((L + kSpan - 1) / kSpan);
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  pack_kernel<D, BITS, F8><<<(unsigned)blocks, kWarps * 32, 0, s>>>(
       k, v, idx, nbh, L, window, k_vert, lo_rows(o), (uint8_t *)o.k_codes, (uint8_t *)o.v_codes,
       (__half2 *)o.k_sz, (__half2 *)o.v_sz, (__nv_bfloat16 *)o.k_hi, (__nv_bfloat16 *)o.v_hi,
       o.lo_pos, status);
@@ -215,7 +337,7 @@ cudaError_t launch_pack_t(const __nv_bfloat16 *k, const __nv_bfloat16 *v, const 
 // Each lane reads and writes only its own words of the row, so the in-place
 // overwrite after the reads needs no barrier.  With no window the new token
 // goes straight to the low segment.
-template <int D, int BITS>
+template <int D, int BITS, bool F8>
 __global__ void __launch_bounds__(kWarps * 32)
 kv_append_kernel(const __nv_bfloat16 *__restrict__ k_new, const __nv_bfloat16 *__restrict__ v_new,
                  int nbh, int L, int window, int k_vert, int n_lo, int lo_cap,
@@ -241,8 +363,8 @@ kv_append_kernel(const __nv_bfloat16 *__restrict__ k_new, const __nv_bfloat16 *_
   }
   const size_t r = (size_t)bh * lo_cap + n_lo;
   if (window == 0) {
-    quant_store<D, BITS>(kw, k_codes + r * ROWB, k_sz + r * NG, lane);
-    quant_store<D, BITS>(vw, v_codes + r * ROWB, v_sz + r * NG, lane);
+    quant_row_store<D, BITS, F8>(kw, k_codes + r * ROWB, k_sz + r * NG, lane);
+    quant_row_store<D, BITS, F8>(vw, v_codes + r * ROWB, v_sz + r * NG, lane);
     if (lo_pos && lane == 0) lo_pos[r] = L;
     return;
   }
@@ -254,8 +376,8 @@ kv_append_kernel(const __nv_bfloat16 *__restrict__ k_new, const __nv_bfloat16 *_
     ko[i] = kh[i];
     vo[i] = vh[i];
   }
-  quant_store<D, BITS>(ko, k_codes + r * ROWB, k_sz + r * NG, lane);
-  quant_store<D, BITS>(vo, v_codes + r * ROWB, v_sz + r * NG, lane);
+  quant_row_store<D, BITS, F8>(ko, k_codes + r * ROWB, k_sz + r * NG, lane);
+  quant_row_store<D, BITS, F8>(vo, v_codes + r * ROWB, v_sz + r * NG, lane);
   if (lo_pos && lane == 0) lo_pos[r] = L - window;
 #pragma unroll
   for (int i = 0; i < W32; ++i) {
@@ -264,12 +386,12 @@ kv_append_kernel(const __nv_bfloat16 *__restrict__ k_new, const __nv_bfloat16 *_
   }
 }
 
-template <int D, int BITS>
+template <int D, int BITS, bool F8>
 cudaError_t launch_kv_append_t(const __nv_bfloat16 *k_new, const __nv_bfloat16 *v_new, int nbh,
                                int L, int window, int k_vert, const hq_kv_cache &c,
                                cudaStream_t s) {
   const int blocks = (nbh + kWarps - 1) / kWarps;
-  return pdl_launch(kv_append_kernel<D, BITS>, dim3(blocks), dim3(kWarps * 32), 0, s, k_new, v_new,
+  return pdl_launch(kv_append_kernel<D, BITS, F8>, dim3(blocks), dim3(kWarps * 32), 0, s, k_new, v_new,
                     nbh, L, window, k_vert, c.n_lo, lo_rows(c), (uint8_t *)c.k_codes,
                     (uint8_t *)c.v_codes, (__half2 *)c.k_sz, (__half2 *)c.v_sz,
                     (__nv_bfloat16 *)c.k_hi, (__nv_bfloat16 *)c.v_hi, c.lo_pos);
@@ -281,10 +403,12 @@ cudaError_t launch_pack(const __nv_bfloat16 *k, const __nv_bfloat16 *v, const in
                         int B, int Hkv, int L, int D, int window, int k_vert, int bits,
                         const hq_kv_cache &out, uint32_t *status, cudaStream_t s) {
   const int nbh = B * Hkv;
-  if (D == 128 && bits == 4) return launch_pack_t<128, 4>(k, v, idx, nbh, L, window, k_vert, out, status, s);
-  if (D == 128 && bits == 8) return launch_pack_t<128, 8>(k, v, idx, nbh, L, window, k_vert, out, status, s);
-  if (D == 64 && bits == 4) return launch_pack_t<64, 4>(k, v, idx, nbh, L, window, k_vert, out, status, s);
-  if (D == 64 && bits == 8) return launch_pack_t<64, 8>(k, v, idx, nbh, L, window, k_vert, out, status, s);
+  const bool f8 = out.fmt == HQ_KV_FP8;
+#define HQ_P(DD, BB, FF) \
+  if (D == DD && bits == BB && f8 == FF) return launch_pack_t<DD, BB, FF>(k, v, idx, nbh, L, window, k_vert, out, status, s);
+  HQ_P(128, 4, false) HQ_P(128, 8, false) HQ_P(64, 4, false) HQ_P(64, 8, false)
+  HQ_P(128, 8, true) HQ_P(64, 8, true)
+#undef HQ_P
   return cudaErrorInvalidValue;
 }
 
@@ -292,10 +416,12 @@ cudaError_t launch_kv_append(const __nv_bfloat16 *k_new, const __nv_bfloat16 *v_
                              int Hkv, int D, int L, int window, int k_vert,
                              const hq_kv_cache &c, cudaStream_t s) {
   const int nbh = B * Hkv;
-  if (D == 128 && c.bits == 4) return launch_kv_append_t<128, 4>(k_new, v_new, nbh, L, window, k_vert, c, s);
-  if (D == 128 && c.bits == 8) return launch_kv_append_t<128, 8>(k_new, v_new, nbh, L, window, k_vert, c, s);
-  if (D == 64 && c.bits == 4) return launch_kv_append_t<64, 4>(k_new, v_new, nbh, L, window, k_vert, c, s);
-  if (D == 64 && c.bits == 8) return launch_kv_append_t<64, 8>(k_new, v_new, nbh, L, window, k_vert, c, s);
+  const bool f8 = c.fmt == HQ_KV_FP8;
+#define HQ_A(DD, BB, FF) \
+  if (D == DD && c.bits == BB && f8 == FF) return launch_kv_append_t<DD, BB, FF>(k_new, v_new, nbh, L, window, k_vert, c, s);
+  HQ_A(128, 4, false) HQ_A(128, 8, false) HQ_A(64, 4, false) HQ_A(64, 8, false)
+  HQ_A(128, 8, true) HQ_A(64, 8, true)
+#undef HQ_A
   return cudaErrorInvalidValue;
 }
 

@@ -34,12 +34,13 @@ _SZ = ctypes.c_size_t
 HQ_OK = 0
 HQ_DEV_BAD_INDEX = 0x1
 HQ_DEV_TIMEOUT = 0x2
+HQ_KV_INT, HQ_KV_FP8 = 0, 1      # low-bit code formats (hq_kv_cache.fmt)
 
 
 class hq_kv_cache(ctypes.Structure):
     _fields_ = [("k_codes", _P), ("v_codes", _P), ("k_sz", _P), ("v_sz", _P), ("k_hi", _P),
                 ("v_hi", _P), ("lo_pos", _P), ("n_lo", _I), ("n_hi", _I), ("bits", _I),
-                ("group", _I), ("lo_cap", _I)]
+                ("group", _I), ("lo_cap", _I), ("fmt", _I)]
 
 
 def _sig(name, restype, *argtypes):
@@ -133,10 +134,11 @@ class KVCache:
     n_hi: int
     bits: int
     group: int = 32
+    fmt: int = HQ_KV_INT
 
     @classmethod
     def empty(cls, B, Hkv, L, D, window, k_vert, bits, device="cuda", with_pos=True,
-              lo_cap=None):
+              lo_cap=None, fmt=HQ_KV_INT):
         """Buffers for a cache of L tokens.  lo_cap (default: exactly the
         n_lo low rows) reserves low rows per (b, kv head) for decode appends."""
         n_lo, n_hi = L - window - k_vert, k_vert + window
@@ -151,7 +153,7 @@ class KVCache:
             k_hi=torch.empty(B, Hkv, n_hi, D, dtype=torch.bfloat16, device=device),
             v_hi=torch.empty(B, Hkv, n_hi, D, dtype=torch.bfloat16, device=device),
             lo_pos=torch.empty(B, Hkv, C, dtype=torch.int32, device=device) if with_pos else None,
-            n_lo=n_lo, n_hi=n_hi, bits=bits)
+            n_lo=n_lo, n_hi=n_hi, bits=bits, fmt=fmt)
 
     @property
     def lo_cap(self) -> int:
@@ -160,7 +162,7 @@ class KVCache:
     def struct(self) -> hq_kv_cache:
         return hq_kv_cache(_ptr(self.k_codes), _ptr(self.v_codes), _ptr(self.k_sz),
                            _ptr(self.v_sz), _ptr(self.k_hi), _ptr(self.v_hi), _ptr(self.lo_pos),
-                           self.n_lo, self.n_hi, self.bits, self.group, self.lo_cap)
+                           self.n_lo, self.n_hi, self.bits, self.group, self.lo_cap, self.fmt)
 
     def nbytes(self, with_pos: bool = False) -> int:
         """Bytes of the rows in use (spare low rows not counted)."""
@@ -243,10 +245,11 @@ def probe_vertical(q_probe, k, window, k_vert, scale=0.0, want_scores=False, ws=
     return (idx, score) if want_scores else idx
 
 
-def pack_kv(k, v, idx, window, bits=4, ws=None, with_pos=True, lo_cap=None) -> KVCache:
+def pack_kv(k, v, idx, window, bits=4, ws=None, with_pos=True, lo_cap=None,
+            fmt=HQ_KV_INT) -> KVCache:
     B, Hkv, L, D = k.shape
     k_vert = idx.shape[2]
-    cache = KVCache.empty(B, Hkv, L, D, window, k_vert, bits, k.device, with_pos, lo_cap)
+    cache = KVCache.empty(B, Hkv, L, D, window, k_vert, bits, k.device, with_pos, lo_cap, fmt)
     hq_pack_kv(k, v, idx, B, Hkv, L, D, window, k_vert, bits, 32, cache, ws)
     return cache
 

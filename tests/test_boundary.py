@@ -56,7 +56,7 @@ def test_status_strings(lib):
 class _Cache(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("k_codes", "v_codes", "k_sz", "v_sz", "k_hi", "v_hi", "lo_pos")] + \
-               [(n, ctypes.c_int) for n in ("n_lo", "n_hi", "bits", "group", "lo_cap")]
+               [(n, ctypes.c_int) for n in ("n_lo", "n_hi", "bits", "group", "lo_cap", "fmt")]
 
 
 FAKE = ctypes.c_void_p(0x10000)      # 16-byte aligned, never dereferenced on the host

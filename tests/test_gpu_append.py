@@ -32,7 +32,7 @@ def prefix_vertical_set(planted: np.ndarray, limit: int) -> np.ndarray:
     return np.ascontiguousarray(np.array([[x[:k] for x in row] for row in below], np.int32))
 
 
-def run_append_case(w: Workload, t: int, check_steps=(), decode_steps=()):
+def run_append_case(w: Workload, t: int, check_steps=(), decode_steps=(), fmt=0):
     """Pack the first L0 = w.L - t tokens, append the other t one by one on the
     GPU, then compare the cache and a decode against the oracle."""
     H = hq()
@@ -43,8 +43,8 @@ def run_append_case(w: Workload, t: int, check_steps=(), decode_steps=()):
     kv = idx.shape[2]
     n_lo0 = L0 - W - kv
     cache = H.pack_kv(d["k"][:, :, :L0].contiguous(), d["v"][:, :, :L0].contiguous(),
-                      torch.from_numpy(idx).cuda(), W, w.bits, lo_cap=n_lo0 + t)
-    ref = oracle.pack_kv(x["k"][:, :, :L0], x["v"][:, :, :L0], idx, W, w.bits)
+                      torch.from_numpy(idx).cuda(), W, w.bits, lo_cap=n_lo0 + t, fmt=fmt)
+    ref = oracle.pack_kv(x["k"][:, :, :L0], x["v"][:, :, :L0], idx, W, w.bits, 32, fmt)
     for s in range(t):
         L = L0 + s
         H.kv_append(cache, d["k"][:, :, L].contiguous(), d["v"][:, :, L].contiguous(), L, W)
@@ -62,7 +62,7 @@ def run_append_case(w: Workload, t: int, check_steps=(), decode_steps=()):
     got = cache_to_np(cache)
     assert_pack_equal(got, ref)
     # the appended cache is the pack of the whole sequence
-    full = oracle.pack_kv(x["k"], x["v"], idx, W, w.bits)
+    full = oracle.pack_kv(x["k"], x["v"], idx, W, w.bits, 32, fmt)
     assert_pack_equal(got, full)
     out, lse = H.decode_attn(d["q"], cache, w.Hkv, want_lse=True)
     ref_out, ref_lse = oracle.decode_attn(x["q"], full, w.Hkv)
@@ -98,3 +98,9 @@ def test_llama8b_append_full_size():
     # heads, D = 128, W = 128, INT4; the last 16 tokens arrive by append
     w = Workload("llama8b_append_32k", "decode", 1, 32, 8, 128, 32768, 128, F5, 4, 2024)
     run_append_case(w, t=16, check_steps=(0,))
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_append_fp8(D):
+    w = Workload("append_fp8", "decode", 2, 8, 2, D, 1300 + 70, 64, F5, 8, 91 + D)
+    run_append_case(w, t=70, check_steps=(0, 64), decode_steps=(3,), fmt=1)

@@ -20,7 +20,7 @@ def hq():
     return m
 
 
-def run_decode_case(w: Workload, check_probe=True, planted_idx=False):
+def run_decode_case(w: Workload, check_probe=True, planted_idx=False, fmt=0):
     H = hq()
     x = make_inputs(w)
     d = to_dev(x)
@@ -43,8 +43,8 @@ def run_decode_case(w: Workload, check_probe=True, planted_idx=False):
     # pack with the oracle's index list on both sides: bit-exact
     idx_d = torch.from_numpy(ref_idx).cuda()
     ws = H.workspace(256)
-    cache = H.pack_kv(d["k"], d["v"], idx_d, w.window, w.bits, ws=ws)
-    ref_cache = oracle.pack_kv(x["k"], x["v"], ref_idx, w.window, w.bits)
+    cache = H.pack_kv(d["k"], d["v"], idx_d, w.window, w.bits, ws=ws, fmt=fmt)
+    ref_cache = oracle.pack_kv(x["k"], x["v"], ref_idx, w.window, w.bits, 32, fmt)
     torch.cuda.synchronize()
     assert H.hq_read_device_status(ws) == 0
     assert_pack_equal(cache_to_np(cache), ref_cache)
@@ -122,14 +122,14 @@ def test_llama8b_decode_full_size():
     run_decode_case(WORKLOADS["llama8b_decode_32k"])
 
 
-def _full_size_sampled(w: Workload, samples):
+def _full_size_sampled(w: Workload, samples, fmt=0):
     """Run probe / pack / decode at full size in the benchmark's launch
     configuration; compare the sampled (b, kv head) slices with the oracle."""
     H = hq()
     x = make_inputs(w)
     d = to_dev(x)
     idx = H.probe_vertical(d["q_probe"], d["k"], w.window, w.k_vert)
-    cache = H.pack_kv(d["k"], d["v"], idx, w.window, w.bits)
+    cache = H.pack_kv(d["k"], d["v"], idx, w.window, w.bits, fmt=fmt)
     out = H.decode_attn(d["q"], cache, w.Hkv)
     torch.cuda.synchronize()
     gidx = idx.cpu().numpy()
@@ -145,7 +145,7 @@ def _full_size_sampled(w: Workload, samples):
         assert_index_sets(gidx[b:b + 1, h:h + 1], ridx, sc, w.window)
         if not np.array_equal(gidx[b:b + 1, h:h + 1], ridx):
             continue  # a tie swapped members: the rest of this slice is not comparable
-        rc = oracle.pack_kv(ks, vs, ridx, w.window, w.bits)
+        rc = oracle.pack_kv(ks, vs, ridx, w.window, w.bits, 32, fmt)
         assert_pack_equal({k: (v[b:b + 1, h:h + 1] if isinstance(v, np.ndarray) else None)
                            for k, v in gc.items()}, rc)
         ro, _ = oracle.decode_attn(qs, rc, 1)
@@ -165,3 +165,32 @@ def test_batched_decode_int8_full_size():
 @pytest.mark.slow
 def test_70b_decode_full_size():
     _full_size_sampled(WORKLOADS["70b_decode_64k"], [(0, 0), (31, 7), (17, 3)])
+
+
+# --------------------------------------------------------------------------
+# FP8 (E4M3) low-bit format
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("G", [1, 4, 8])
+@pytest.mark.parametrize("D", [64, 128])
+def test_decode_fp8_ragged(G, D):
+    # codes and scales bit-exact, decode within tolerance; ragged L, several
+    # tiles per CTA on both lines
+    w = Workload("fp8", "decode", 2, 2 * G, 2, D, 5003, 128, F5, 8, 177 + G + D)
+    run_decode_case(w, fmt=1)
+
+
+def test_decode_fp8_many_tiles_per_cta():
+    w = Workload("fp8_multitile", "decode", 4, 32, 8, 128, 20000, 128, F5, 8, 41)
+    run_decode_case(w, planted_idx=True, fmt=1)
+
+
+def test_llama8b_decode_fp8_full_size():
+    w = WORKLOADS["llama8b_decode_32k"].replace(bits=8)
+    run_decode_case(w, fmt=1)
+
+
+@pytest.mark.slow
+def test_batched_decode_fp8_full_size():
+    w = WORKLOADS["batched_decode_128k_int8"]
+    _full_size_sampled(w, [(1, 4), (5, 0)], fmt=1)
