@@ -199,6 +199,22 @@ hq_status hq_decode_attn(const void *q, const hq_kv_cache *cache, int B, int Hq,
                          size_t ws_bytes, void *stream);
 
 /*
+ * Merge of decode results computed over disjoint parts of one cache's rows,
+ * for a context split across GPUs (each rank decodes its part with lse_out,
+ * the parts are gathered, one rank or all merge).  Attention does not depend
+ * on the order of the cached rows (wiki summary, "Key results": one softmax
+ * over all cached positions), so with m = max_r lse_r and w_r = exp(lse_r - m)
+ *   out = sum_r w_r part_out[r] / sum_r w_r,   lse_out = m + log(sum_r w_r)
+ * is the decode over the union of the parts.  A part with lse = -inf has
+ * weight 0; if every part has, out is 0 and lse_out -inf.
+ *   part_out : f32 [R, B, Hq, D];  part_lse : f32 [R, B, Hq] (natural log).
+ *   out      : f32 [B, Hq, D];     lse_out  : f32 [B, Hq] or NULL.
+ * part_out and out must be 16-byte aligned; D in {64, 128}.
+ */
+hq_status hq_decode_merge(const float *part_out, const float *part_lse, int R, int B, int Hq,
+                          int D, float *out, float *lse_out, void *stream);
+
+/*
  * hq_decode_attn without a caller-supplied workspace, for callers that cannot
  * allocate device memory at call time: code running under someone else's
  * stream capture (where a cudaMalloc would break the capture), serving runtimes

@@ -153,6 +153,18 @@ hq_status hq_kv_append(const void *k_new, const void *v_new, int B, int Hkv, int
                                       B, Hkv, D, L, window, k_vert, *cache, (cudaStream_t)stream));
 }
 
+hq_status hq_decode_merge(const float *part_out, const float *part_lse, int R, int B, int Hq,
+                          int D, float *out, float *lse_out, void *stream) {
+  if (!part_out || !part_lse || !out) return HQ_ERR_INVALID_ARG;
+  if (R <= 0 || B <= 0 || Hq <= 0) return HQ_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return HQ_ERR_UNSUPPORTED;
+  const void *ptrs[] = {part_out, out};
+  for (const void *p : ptrs)
+    if (!aligned16(p)) return HQ_ERR_INVALID_ARG;
+  return cuda_status(launch_decode_merge(part_out, part_lse, R, B, Hq, D, out, lse_out,
+                                         (cudaStream_t)stream));
+}
+
 size_t hq_decode_workspace_size(int B, int Hq, int Hkv, int D, int n_lo, int n_hi, int bits) {
   if (B <= 0 || !supported_G(Hq, Hkv) || (D != 64 && D != 128) || n_lo < 0 || n_hi < 0 ||
       n_lo + n_hi <= 0 || (bits != 4 && bits != 8))

@@ -256,4 +256,53 @@ cudaError_t launch_decode(const __nv_bfloat16 *q, const hq_kv_cache &c, int B, i
   return cudaErrorInvalidValue;
 }
 
+// ---------------------------------------------------------------------------
+// Merge of decode results over disjoint parts of one cache (a context split
+// across ranks): with m = max_r lse_r and w_r = exp(lse_r - m),
+//   out = sum_r w_r out_r / sum_r w_r,   lse = m + log(sum_r w_r),
+// the exact softmax over the union of the parts' rows.  One warp per
+// (b, query head); a part with lse = -inf (no rows) has weight 0.
+// ---------------------------------------------------------------------------
+namespace {
+template <int D>
+__global__ void __launch_bounds__(128)
+decode_merge_kernel(const float *__restrict__ part_out, const float *__restrict__ part_lse, int R,
+                    int nq, float *__restrict__ out, float *__restrict__ lse) {
+  constexpr int CPL = D / 32;
+  const int lane = threadIdx.x & 31;
+  const int bq = blockIdx.x * 4 + (threadIdx.x >> 5);
+  if (bq >= nq) return;
+  float m = -INFINITY;
+  for (int r = 0; r < R; ++r) m = fmaxf(m, __ldg(part_lse + (size_t)r * nq + bq));
+  float acc[CPL] = {};
+  float sum = 0.f;
+  if (m > -INFINITY) {
+    for (int r = 0; r < R; ++r) {
+      const float w = expf(__ldg(part_lse + (size_t)r * nq + bq) - m);
+      const float *o = part_out + ((size_t)r * nq + bq) * D + lane * CPL;
+      sum += w;
+#pragma unroll
+      for (int i = 0; i < CPL; ++i) acc[i] = fmaf(w, __ldg(o + i), acc[i]);
+    }
+  }
+  const float inv = sum > 0.f ? 1.f / sum : 0.f;
+#pragma unroll
+  for (int i = 0; i < CPL; ++i) out[(size_t)bq * D + lane * CPL + i] = acc[i] * inv;
+  if (lse && lane == 0) lse[bq] = sum > 0.f ? m + logf(sum) : -INFINITY;
+}
+}  // namespace
+
+cudaError_t launch_decode_merge(const float *part_out, const float *part_lse, int R, int B,
+                                int Hq, int D, float *out, float *lse, cudaStream_t s) {
+  const int nq = B * Hq;
+  const int blocks = (nq + 3) / 4;
+  if (D == 128)
+    decode_merge_kernel<128><<<blocks, 128, 0, s>>>(part_out, part_lse, R, nq, out, lse);
+  else if (D == 64)
+    decode_merge_kernel<64><<<blocks, 128, 0, s>>>(part_out, part_lse, R, nq, out, lse);
+  else
+    return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
 }  // namespace hq

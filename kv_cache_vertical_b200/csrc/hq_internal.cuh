@@ -86,6 +86,8 @@ float resolve_softmax_scale(float s, int D);
 cudaError_t launch_decode(const __nv_bfloat16 *q, const hq_kv_cache &c, int B, int Hq, int Hkv,
                           int D, float scale, float *out, float *lse, uint8_t *ws,
                           uint32_t *status, cudaStream_t s);
+cudaError_t launch_decode_merge(const float *part_out, const float *part_lse, int R, int B,
+                                int Hq, int D, float *out, float *lse, cudaStream_t s);
 
 cudaError_t launch_prefill_quant(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
                                  const int32_t *idx, int B, int Hq, int Hkv, int N, int D,

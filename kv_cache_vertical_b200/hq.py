@@ -62,6 +62,7 @@ hq_decode_workspace_size = _sig("hq_decode_workspace_size", _SZ, _I, _I, _I, _I,
 _decode = _sig("hq_decode_attn", _I, _P, ctypes.POINTER(hq_kv_cache), _I, _I, _I, _I, _F, _P, _P,
                _P, _SZ, _P)
 _append = _sig("hq_kv_append", _I, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.POINTER(hq_kv_cache), _P)
+_merge = _sig("hq_decode_merge", _I, _P, _P, _I, _I, _I, _I, _P, _P, _P)
 _decode_static = _sig("hq_decode_attn_static", _I, _P, ctypes.POINTER(hq_kv_cache), _I, _I, _I,
                       _I, _F, _P, _P, _P)
 _pquant = _sig("hq_prefill_quant", _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P)
@@ -72,7 +73,7 @@ _prefill = _sig("hq_prefill_attn", _I, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _
 EXPORTED = ["hq_status_string", "hq_version", "hq_read_device_status", "hq_probe_workspace_size",
             "hq_probe_vertical", "hq_pack_kv", "hq_decode_workspace_size", "hq_decode_attn",
             "hq_prefill_quant", "hq_prefill_workspace_size", "hq_prefill_attn",
-            "hq_decode_attn_static", "hq_kv_append"]
+            "hq_decode_attn_static", "hq_kv_append", "hq_decode_merge"]
 
 HQ_ERR_SCRATCH_LIMIT = 7
 STATIC_SCRATCH_BYTES = 8 << 20
@@ -157,12 +158,33 @@ class KVCache:
 
     @property
     def lo_cap(self) -> int:
-        return self.k_codes.shape[2] if self.k_codes.dim() == 4 else self.n_lo
+        """Rows between consecutive (b, kv head) slices of the low arrays (the
+        allocation, or the parent's for a row view)."""
+        t = self.k_codes
+        if t.dim() != 4:
+            return self.n_lo
+        return t.stride(1) // t.stride(2) if t.shape[2] > 0 else t.shape[2]
+
+    def rows_view(self, lo_start: int, lo_end: int, with_hi: bool) -> "KVCache":
+        """The cache restricted to low rows [lo_start, lo_end) and, if
+        with_hi, all bf16 rows: views, no copy (the low arrays keep their row
+        stride through lo_cap).  Attention over the union of disjoint views
+        equals attention over the cache."""
+        sl = slice(lo_start, lo_end)
+        return KVCache(
+            k_codes=self.k_codes[:, :, sl], v_codes=self.v_codes[:, :, sl],
+            k_sz=self.k_sz[:, :, sl], v_sz=self.v_sz[:, :, sl],
+            k_hi=self.k_hi if with_hi else self.k_hi[:, :, :0],
+            v_hi=self.v_hi if with_hi else self.v_hi[:, :, :0],
+            lo_pos=self.lo_pos[:, :, sl] if self.lo_pos is not None else None,
+            n_lo=lo_end - lo_start, n_hi=self.n_hi if with_hi else 0, bits=self.bits,
+            group=self.group, fmt=self.fmt)
 
     def struct(self) -> hq_kv_cache:
         return hq_kv_cache(_ptr(self.k_codes), _ptr(self.v_codes), _ptr(self.k_sz),
                            _ptr(self.v_sz), _ptr(self.k_hi), _ptr(self.v_hi), _ptr(self.lo_pos),
-                           self.n_lo, self.n_hi, self.bits, self.group, self.lo_cap, self.fmt)
+                           self.n_lo, self.n_hi, self.bits, self.group,
+                           self.lo_cap if self.n_lo > 0 else 0, self.fmt)
 
     def nbytes(self, with_pos: bool = False) -> int:
         """Bytes of the rows in use (spare low rows not counted)."""
@@ -195,6 +217,11 @@ def hq_kv_append(k_new, v_new, B, Hkv, D, L, window, k_vert, cache: KVCache, str
     st = cache.struct()
     _check(_append(_ptr(k_new), _ptr(v_new), B, Hkv, D, L, window, k_vert, ctypes.byref(st),
                    _stream(stream)), "hq_kv_append")
+
+
+def hq_decode_merge(part_out, part_lse, R, B, Hq, D, out, lse_out, stream=None):
+    _check(_merge(_ptr(part_out), _ptr(part_lse), R, B, Hq, D, _ptr(out), _ptr(lse_out),
+                  _stream(stream)), "hq_decode_merge")
 
 
 def hq_decode_attn(q, cache: KVCache, B, Hq, Hkv, D, softmax_scale, out, lse_out, ws, stream=None):
@@ -303,3 +330,63 @@ def prefill_attn(q, k, v, idx, window, scale=0.0, ws=None, out=None):
 
 def default_scale(D: int) -> float:
     return 1.0 / math.sqrt(D)
+
+
+# ---------------------------------------------------------------------------
+# Context split of the decode across ranks
+# ---------------------------------------------------------------------------
+def context_split_plan(n_lo: int, n_hi: int, R: int, D: int, bits: int, align: int = 64):
+    """Share the rows of one cache among R ranks for a context-split decode:
+    rank r gets low rows [lo0, lo1) and the last rank also every bf16 row.
+    Attention does not depend on the order of the rows, so any disjoint cover
+    works; this one gives each rank about the same number of bytes to read
+    (a low row is 2*(D*bits/8 + D/8) bytes, a bf16 row 4*D) and puts the low
+    boundaries on multiples of `align` rows (whole decode tiles, 16-byte
+    aligned views).  Returns [(lo0, lo1, with_hi)] * R."""
+    if R < 1:
+        raise ValueError("R must be at least 1")
+    b_lo = 2 * (D * bits // 8 + D // 8)
+    b_hi = 4 * D
+    total = n_lo * b_lo + n_hi * b_hi
+    lo_last = max(0, min(n_lo, round((total / R - n_hi * b_hi) / b_lo))) if R > 1 else n_lo
+    rest = (n_lo - lo_last) // align * align          # rows of ranks 0 .. R-2
+    cuts = [min(rest, (rest * r // max(R - 1, 1)) // align * align) for r in range(R)]
+    cuts[R - 1] = rest
+    plan = []
+    for r in range(R - 1):
+        plan.append((cuts[r], cuts[r + 1], False))
+    plan.append((rest, n_lo, True))
+    return plan
+
+
+def decode_merge(part_out, part_lse):
+    """Merge R partial decodes: part_out f32 [R, B, Hq, D], part_lse f32 [R, B, Hq]."""
+    R, B, Hq, D = part_out.shape
+    out = torch.empty(B, Hq, D, dtype=torch.float32, device=part_out.device)
+    lse = torch.empty(B, Hq, dtype=torch.float32, device=part_out.device)
+    hq_decode_merge(part_out.contiguous(), part_lse.contiguous(), R, B, Hq, D, out, lse)
+    return out, lse
+
+
+def decode_context_parallel(q, cache: KVCache, Hkv, group=None, scale=0.0):
+    """Decode one step with the cache's rows split over the ranks of `group`
+    (torch.distributed, NCCL): each rank decodes its rows of context_split_plan
+    (views of its full copy of the packed cache, or its own part), the
+    (out, lse) pairs are all-gathered, and every rank merges them.  Returns
+    (out, lse) of the whole cache."""
+    import torch.distributed as dist
+    R = dist.get_world_size(group)
+    r = dist.get_rank(group)
+    B, Hq, D = q.shape
+    lo0, lo1, with_hi = context_split_plan(cache.n_lo, cache.n_hi, R, D, cache.bits)[r]
+    part = cache.rows_view(lo0, lo1, with_hi)
+    if part.n_lo + part.n_hi > 0:
+        out_r, lse_r = decode_attn(q, part, Hkv, scale=scale, want_lse=True)
+    else:
+        out_r = torch.zeros(B, Hq, D, dtype=torch.float32, device=q.device)
+        lse_r = torch.full((B, Hq), float("-inf"), dtype=torch.float32, device=q.device)
+    outs = [torch.empty_like(out_r) for _ in range(R)]
+    lses = [torch.empty_like(lse_r) for _ in range(R)]
+    dist.all_gather(outs, out_r, group=group)
+    dist.all_gather(lses, lse_r, group=group)
+    return decode_merge(torch.stack(outs), torch.stack(lses))

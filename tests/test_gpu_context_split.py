@@ -1,0 +1,86 @@
+"""GPU parity of the context-split decode, its ranks run one after another on
+one GPU: each part of the plan is decoded through a row view of one packed
+cache, the parts are merged by hq_decode_merge, and the result is compared
+with the oracle's decode of the whole cache (the CUDA path's cache is the
+oracle's, bit for bit, as the pack tests show)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from hq_testutil import assert_close, to_dev
+from kv_cache_vertical_b200.synth import F5, WORKLOADS, Workload, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def hq():
+    from kv_cache_vertical_b200 import hq as m
+    return m
+
+
+def run_split(w: Workload, R: int, fmt=0):
+    H = hq()
+    x = make_inputs(w)
+    d = to_dev(x)
+    idx = x["planted"].numpy()
+    cache = H.pack_kv(d["k"], d["v"], torch.from_numpy(idx).cuda(), w.window, w.bits, fmt=fmt)
+    ref = oracle.pack_kv(x["k"], x["v"], idx, w.window, w.bits, 32, fmt)
+    full, full_lse = oracle.decode_attn(x["q"], ref, w.Hkv)
+    outs, lses = [], []
+    for lo0, lo1, with_hi in H.context_split_plan(cache.n_lo, cache.n_hi, R, w.D, w.bits):
+        part = cache.rows_view(lo0, lo1, with_hi)
+        if part.n_lo + part.n_hi == 0:
+            outs.append(torch.zeros(w.B, w.Hq, w.D, device="cuda"))
+            lses.append(torch.full((w.B, w.Hq), float("-inf"), device="cuda"))
+            continue
+        o, l = H.decode_attn(d["q"], part, w.Hkv, want_lse=True)
+        outs.append(o)
+        lses.append(l)
+    out, lse = H.decode_merge(torch.stack(outs), torch.stack(lses))
+    torch.cuda.synchronize()
+    assert_close(out.cpu().numpy(), full, f"context split R={R}")
+    assert np.allclose(lse.cpu().numpy(), full_lse, atol=1e-4, rtol=1e-5)
+
+
+@pytest.mark.parametrize("R", [2, 3, 4])
+@pytest.mark.parametrize("bits,D", [(4, 128), (8, 128), (4, 64)])
+def test_context_split_matches_whole_cache(R, bits, D):
+    w = Workload("cs", "decode", 2, 8, 2, D, 6001, 128, F5, bits, 11 * R + bits + D)
+    run_split(w, R)
+
+
+def test_context_split_fp8_and_empty_rank():
+    # 3 ranks over a cache with few low rows: one rank has nothing to read
+    w = Workload("cs_fp8", "decode", 1, 4, 1, 128, 400, 256, F5, 8, 3)
+    H = hq()
+    assert any(lo1 == lo0 and not wh for lo0, lo1, wh in
+               H.context_split_plan(400 - 256 - w.k_vert, 256 + w.k_vert, 3, 128, 8))
+    run_split(w, 3, fmt=1)
+
+
+def test_context_split_llama8b_full_size():
+    run_split(WORKLOADS["llama8b_decode_32k"], 2)
+
+
+def test_merge_kernel_against_numpy():
+    H = hq()
+    g = torch.Generator().manual_seed(5)
+    R, B, Hq, D = 5, 3, 8, 128
+    po = torch.randn(R, B, Hq, D, generator=g)
+    pl = torch.randn(R, B, Hq, generator=g) * 4
+    pl[1, 0, :] = float("-inf")                       # an empty part
+    pl[:, 2, 3] = float("-inf")                       # every part empty for one head
+    out, lse = H.decode_merge(po.cuda(), pl.cuda())
+    torch.cuda.synchronize()
+    m = pl.double().amax(0)
+    wgt = torch.exp(pl.double() - torch.where(torch.isinf(m), torch.zeros_like(m), m))
+    ref = (wgt[..., None] * po.double()).sum(0) / wgt.sum(0)[..., None]
+    ref[2, 3] = 0.0
+    got = out.cpu().double()
+    assert torch.allclose(got, ref, atol=1e-5, rtol=1e-5)
+    assert torch.isinf(lse[2, 3].cpu()) and lse[2, 3].item() < 0
+    ok = torch.ones(B, Hq, dtype=torch.bool)
+    ok[2, 3] = False
+    ref_lse = m + torch.log(wgt.sum(0))
+    assert torch.allclose(lse.cpu().double()[ok], ref_lse[ok], atol=1e-5)

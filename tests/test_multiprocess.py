@@ -1,9 +1,12 @@
-"""The multi-rank plumbing of bench.py, on CPU with the gloo backend.
+"""The multi-rank paths, on CPU with the gloo backend.
 
 `bench.py --gpus N` runs one independent replica per rank (weak scaling: the
 hot path has no cross-rank exchange) and reports the slowest rank's time and
-the sum of all ranks' work.  These tests run two gloo ranks on the host and
-check the barrier and the max-over-ranks reduction that the GPU run uses.
+the sum of all ranks' work; the first test checks its barrier and
+max-over-ranks reduction.  The context-split decode (one cache's rows shared
+among ranks) does exchange: every rank gathers all (out, lse) pairs and
+merges them; the second test runs that exchange on two gloo ranks, with the
+oracle computing each rank's part on the host.
 """
 import os
 import socket
@@ -59,3 +62,53 @@ def test_two_gloo_ranks_max_time_and_distinct_replicas():
     for rank, t, digests in results:
         assert t == 10.0 + (world - 1)          # max over ranks, seen by every rank
         assert digests[0] != digests[1]         # replicas draw different inputs
+
+
+def _cp_worker(rank, world, port, q):
+    """One rank of a context-split decode: decode this rank's rows of the
+    shared cache (the oracle stands in for the GPU decode on the host), gather
+    every rank's (out, lse) and merge."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world))
+    import datetime
+    import numpy as np
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        import oracle
+        from kv_cache_vertical_b200 import hq
+        from kv_cache_vertical_b200.synth import F5, Workload, make_inputs
+        from test_context_split import _sub, merge_np
+        w = Workload("cp", "decode", 1, 8, 2, 128, 2500, 128, F5, 4, 123)
+        x = make_inputs(w)                       # the same seed on every rank: one cache
+        c = oracle.pack_kv(x["k"], x["v"], x["planted"].numpy(), w.window, 4)
+        lo0, lo1, with_hi = hq.context_split_plan(c["n_lo"], c["n_hi"], world, w.D, 4)[rank]
+        out, lse = oracle.decode_attn(x["q"], _sub(c, lo0, lo1, with_hi), w.Hkv)
+        outs = [torch.empty(out.shape, dtype=torch.float64) for _ in range(world)]
+        lses = [torch.empty(lse.shape, dtype=torch.float64) for _ in range(world)]
+        dist.all_gather(outs, torch.from_numpy(out))
+        dist.all_gather(lses, torch.from_numpy(lse))
+        merged, mlse = merge_np([t.numpy() for t in outs], [t.numpy() for t in lses])
+        full, full_lse = oracle.decode_attn(x["q"], c, w.Hkv)
+        q.put((rank, float(np.abs(merged - full).max()), float(np.abs(mlse - full_lse).max()),
+               lo1 - lo0))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.timeout(180)
+def test_two_gloo_ranks_context_split_decode():
+    world = 2
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_cp_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    results = [q.get(timeout=150) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert all(r[3] > 0 for r in results)              # both ranks hold low rows
+    for rank, err, lse_err, _ in results:
+        assert err < 1e-12 and lse_err < 1e-12, (rank, err, lse_err)
