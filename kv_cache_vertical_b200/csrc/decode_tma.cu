@@ -931,7 +931,8 @@ inline void tile_costs(int bits, int &cl, int &ch) {
 // and the bf16 line in proportion to their cost.  A line is aligned to whole
 // pairs (no CTA spans two pairs) when that idles at most 2% of its CTAs;
 // every low-bit CTA gets at least eight tiles and every bf16 CTA four (fewer,
-// longer pieces keep the final merge short).
+// longer pieces keep the final merge short), unless that would leave fewer
+// CTAs than pairs on a line.
 Plan make_plan(int nbh, int n_lo, int n_hi, int bits, int occ) {
   const int slots = sm_count() * occ;
   Plan p;
@@ -957,7 +958,13 @@ Plan make_plan(int nbh, int n_lo, int n_hi, int bits, int occ) {
     if (t == 0) return 0;
     const long long tiles = (long long)t * nbh;
     if (n >= nbh && (n % nbh) * 50 <= n) n = n / nbh * nbh;
-    if ((long long)n * min_tiles > tiles) n = (int)(tiles / min_tiles > 0 ? tiles / min_tiles : 1);
+    if ((long long)n * min_tiles > tiles) {
+      // a short line: fewer, longer pieces, but never fewer CTAs than pairs
+      // (one CTA walking many pairs would serialize their pieces)
+      long long m = tiles / min_tiles;
+      if (m < nbh) m = nbh < n ? nbh : n;
+      n = (int)(m > 0 ? m : 1);
+    }
     return n < 1 ? 1 : n;
   };
   p.nc_lo = fit(p.nc_lo, p.tl, 8);

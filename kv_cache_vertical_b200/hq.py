@@ -165,19 +165,23 @@ class KVCache:
             return self.n_lo
         return t.stride(1) // t.stride(2) if t.shape[2] > 0 else t.shape[2]
 
-    def rows_view(self, lo_start: int, lo_end: int, with_hi: bool) -> "KVCache":
-        """The cache restricted to low rows [lo_start, lo_end) and, if
-        with_hi, all bf16 rows: views, no copy (the low arrays keep their row
-        stride through lo_cap).  Attention over the union of disjoint views
-        equals attention over the cache."""
+    def rows_part(self, lo_start: int, lo_end: int, hi_start: int = 0, hi_end: int = 0) -> "KVCache":
+        """The cache restricted to low rows [lo_start, lo_end) (views, no copy:
+        the low arrays keep their row stride through lo_cap) and bf16 rows
+        [hi_start, hi_end) (copied unless that is every bf16 row, since the
+        bf16 arrays carry no row stride).  Attention over the union of
+        disjoint parts equals attention over the cache."""
         sl = slice(lo_start, lo_end)
+        if (hi_start, hi_end) == (0, self.n_hi):
+            k_hi, v_hi = self.k_hi, self.v_hi
+        else:
+            k_hi = self.k_hi[:, :, hi_start:hi_end].contiguous()
+            v_hi = self.v_hi[:, :, hi_start:hi_end].contiguous()
         return KVCache(
             k_codes=self.k_codes[:, :, sl], v_codes=self.v_codes[:, :, sl],
-            k_sz=self.k_sz[:, :, sl], v_sz=self.v_sz[:, :, sl],
-            k_hi=self.k_hi if with_hi else self.k_hi[:, :, :0],
-            v_hi=self.v_hi if with_hi else self.v_hi[:, :, :0],
+            k_sz=self.k_sz[:, :, sl], v_sz=self.v_sz[:, :, sl], k_hi=k_hi, v_hi=v_hi,
             lo_pos=self.lo_pos[:, :, sl] if self.lo_pos is not None else None,
-            n_lo=lo_end - lo_start, n_hi=self.n_hi if with_hi else 0, bits=self.bits,
+            n_lo=lo_end - lo_start, n_hi=hi_end - hi_start, bits=self.bits,
             group=self.group, fmt=self.fmt)
 
     def struct(self) -> hq_kv_cache:
@@ -335,28 +339,18 @@ def default_scale(D: int) -> float:
 # ---------------------------------------------------------------------------
 # Context split of the decode across ranks
 # ---------------------------------------------------------------------------
-def context_split_plan(n_lo: int, n_hi: int, R: int, D: int, bits: int, align: int = 64):
+def context_split_plan(n_lo: int, n_hi: int, R: int, align: int = 64):
     """Share the rows of one cache among R ranks for a context-split decode:
-    rank r gets low rows [lo0, lo1) and the last rank also every bf16 row.
-    Attention does not depend on the order of the rows, so any disjoint cover
-    works; this one gives each rank about the same number of bytes to read
-    (a low row is 2*(D*bits/8 + D/8) bytes, a bf16 row 4*D) and puts the low
-    boundaries on multiples of `align` rows (whole decode tiles, 16-byte
-    aligned views).  Returns [(lo0, lo1, with_hi)] * R."""
+    rank r gets low rows [lo0, lo1) and bf16 rows [hi0, hi1).  Attention does
+    not depend on the order of the rows, so any disjoint cover works; equal
+    shares of both kinds give every rank the same bytes to read.  Low
+    boundaries fall on multiples of `align` rows (whole decode tiles, 16-byte
+    aligned views).  Returns [(lo0, lo1, hi0, hi1)] * R."""
     if R < 1:
         raise ValueError("R must be at least 1")
-    b_lo = 2 * (D * bits // 8 + D // 8)
-    b_hi = 4 * D
-    total = n_lo * b_lo + n_hi * b_hi
-    lo_last = max(0, min(n_lo, round((total / R - n_hi * b_hi) / b_lo))) if R > 1 else n_lo
-    rest = (n_lo - lo_last) // align * align          # rows of ranks 0 .. R-2
-    cuts = [min(rest, (rest * r // max(R - 1, 1)) // align * align) for r in range(R)]
-    cuts[R - 1] = rest
-    plan = []
-    for r in range(R - 1):
-        plan.append((cuts[r], cuts[r + 1], False))
-    plan.append((rest, n_lo, True))
-    return plan
+    lo = [min(n_lo, (n_lo * r // R) // align * align) for r in range(R)] + [n_lo]
+    hi = [n_hi * r // R for r in range(R + 1)]
+    return [(lo[r], lo[r + 1], hi[r], hi[r + 1]) for r in range(R)]
 
 
 def decode_merge(part_out, part_lse):
@@ -370,16 +364,15 @@ def decode_merge(part_out, part_lse):
 
 def decode_context_parallel(q, cache: KVCache, Hkv, group=None, scale=0.0):
     """Decode one step with the cache's rows split over the ranks of `group`
-    (torch.distributed, NCCL): each rank decodes its rows of context_split_plan
-    (views of its full copy of the packed cache, or its own part), the
+    (torch.distributed, NCCL): each rank decodes its part of context_split_plan
+    (taken from its copy of the packed cache), the
     (out, lse) pairs are all-gathered, and every rank merges them.  Returns
     (out, lse) of the whole cache."""
     import torch.distributed as dist
     R = dist.get_world_size(group)
     r = dist.get_rank(group)
     B, Hq, D = q.shape
-    lo0, lo1, with_hi = context_split_plan(cache.n_lo, cache.n_hi, R, D, cache.bits)[r]
-    part = cache.rows_view(lo0, lo1, with_hi)
+    part = cache.rows_part(*context_split_plan(cache.n_lo, cache.n_hi, R)[r])
     if part.n_lo + part.n_hi > 0:
         out_r, lse_r = decode_attn(q, part, Hkv, scale=scale, want_lse=True)
     else:

@@ -28,8 +28,8 @@ def run_split(w: Workload, R: int, fmt=0):
     ref = oracle.pack_kv(x["k"], x["v"], idx, w.window, w.bits, 32, fmt)
     full, full_lse = oracle.decode_attn(x["q"], ref, w.Hkv)
     outs, lses = [], []
-    for lo0, lo1, with_hi in H.context_split_plan(cache.n_lo, cache.n_hi, R, w.D, w.bits):
-        part = cache.rows_view(lo0, lo1, with_hi)
+    for rows in H.context_split_plan(cache.n_lo, cache.n_hi, R):
+        part = cache.rows_part(*rows)
         if part.n_lo + part.n_hi == 0:
             outs.append(torch.zeros(w.B, w.Hq, w.D, device="cuda"))
             lses.append(torch.full((w.B, w.Hq), float("-inf"), device="cuda"))
@@ -50,13 +50,19 @@ def test_context_split_matches_whole_cache(R, bits, D):
     run_split(w, R)
 
 
-def test_context_split_fp8_and_empty_rank():
-    # 3 ranks over a cache with few low rows: one rank has nothing to read
+def test_context_split_fp8_few_low_rows():
+    # 3 ranks over a cache with few low rows: some ranks read bf16 rows only
     w = Workload("cs_fp8", "decode", 1, 4, 1, 128, 400, 256, F5, 8, 3)
     H = hq()
-    assert any(lo1 == lo0 and not wh for lo0, lo1, wh in
-               H.context_split_plan(400 - 256 - w.k_vert, 256 + w.k_vert, 3, 128, 8))
+    assert any(lo1 == lo0 for lo0, lo1, _, _ in
+               H.context_split_plan(400 - 256 - w.k_vert, 256 + w.k_vert, 3))
     run_split(w, 3, fmt=1)
+
+
+def test_context_split_more_ranks_than_pairs_rows():
+    # 8 ranks over a short cache: several parts are small, one may be empty
+    w = Workload("cs_short", "decode", 1, 8, 2, 128, 700, 128, F5, 4, 8)
+    run_split(w, 8)
 
 
 def test_context_split_llama8b_full_size():

@@ -82,8 +82,8 @@ def _cp_worker(rank, world, port, q):
         w = Workload("cp", "decode", 1, 8, 2, 128, 2500, 128, F5, 4, 123)
         x = make_inputs(w)                       # the same seed on every rank: one cache
         c = oracle.pack_kv(x["k"], x["v"], x["planted"].numpy(), w.window, 4)
-        lo0, lo1, with_hi = hq.context_split_plan(c["n_lo"], c["n_hi"], world, w.D, 4)[rank]
-        out, lse = oracle.decode_attn(x["q"], _sub(c, lo0, lo1, with_hi), w.Hkv)
+        part = hq.context_split_plan(c["n_lo"], c["n_hi"], world)[rank]
+        out, lse = oracle.decode_attn(x["q"], _sub(c, *part), w.Hkv)
         outs = [torch.empty(out.shape, dtype=torch.float64) for _ in range(world)]
         lses = [torch.empty(lse.shape, dtype=torch.float64) for _ in range(world)]
         dist.all_gather(outs, torch.from_numpy(out))
@@ -91,7 +91,7 @@ def _cp_worker(rank, world, port, q):
         merged, mlse = merge_np([t.numpy() for t in outs], [t.numpy() for t in lses])
         full, full_lse = oracle.decode_attn(x["q"], c, w.Hkv)
         q.put((rank, float(np.abs(merged - full).max()), float(np.abs(mlse - full_lse).max()),
-               lo1 - lo0))
+               part[1] - part[0]))
     finally:
         dist.destroy_process_group()
 
