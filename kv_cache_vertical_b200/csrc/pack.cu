@@ -181,6 +181,101 @@ __device__ __forceinline__ void quant_row_store(const uint32_t (&w)[D / 64], uin
     quant_store<D, BITS>(w, codes_row, sz_row, lane);
 }
 
+// ---------------------------------------------------------------------------
+// One lane, one group: the pack kernel gives each lane the 32 channels of one
+// quantization group of one row (16 words of bf16 pairs), so the group's
+// min / max need no shuffles and its scale is computed once.  The arithmetic
+// per value is that of quant_store / quant_store_fp8, so the codes, scales
+// and zeros are the same bit for bit.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t bmin2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("min.bf16x2 %0, %1, %2;\n" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t bmax2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.bf16x2 %0, %1, %2;\n" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// Codes of one group into `codes` (32 * BITS / 8 bytes, 16-byte aligned) and
+// its (scale, zero) into *sz.
+template <int BITS, bool F8>
+__device__ __forceinline__ void quant_group_lane(const uint32_t (&w)[16], uint8_t *codes, __half2 *sz) {
+  if (F8) {
+    uint32_t am = w[0] & 0x7fff7fffu;                  // |x| of both halves (sign cleared)
+#pragma unroll
+    for (int i = 1; i < 16; ++i) am = bmax2(am, w[i] & 0x7fff7fffu);
+    const float amax = fmaxf(bf16_lo(am), bf16_hi(am));
+    const __half hs = scale_f16(amax, 0.f, 448);
+    const float sf = __half2float(hs);
+    const float rs = sf != 0.f ? __frcp_rn(sf) : 0.f;
+    uint32_t out[8];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float x0 = bf16_lo(w[i]), x1 = bf16_hi(w[i]);
+      float q0 = x0 * rs, q1 = x1 * rs;
+      if (e4m3_near_tie(q0)) q0 = f32_round_odd((double)x0 / (double)sf);
+      if (e4m3_near_tie(q1)) q1 = f32_round_odd((double)x1 / (double)sf);
+      const uint32_t two = sf != 0.f
+          ? (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(q0, q1), __NV_SATFINITE, __NV_E4M3) : 0u;
+      if (i & 1) out[i >> 1] |= two << 16;
+      else out[i >> 1] = two;
+    }
+    reinterpret_cast<uint4 *>(codes)[0] = make_uint4(out[0], out[1], out[2], out[3]);
+    reinterpret_cast<uint4 *>(codes)[1] = make_uint4(out[4], out[5], out[6], out[7]);
+    *sz = __halves2half2(hs, __ushort_as_half((unsigned short)0));
+    return;
+  }
+  constexpr int QMAX = (1 << BITS) - 1;
+  uint32_t mnw = w[0], mxw = w[0];
+#pragma unroll
+  for (int i = 1; i < 16; ++i) {
+    mnw = bmin2(mnw, w[i]);
+    mxw = bmax2(mxw, w[i]);
+  }
+  const float mn = fminf(bf16_lo(mnw), bf16_hi(mnw)), mx = fmaxf(bf16_lo(mxw), bf16_hi(mxw));
+  const float fmn = mn == 0.f ? 0.f : mn;              // a -0 minimum is stored as +0
+  const __half hs = scale_f16(mx, mn, QMAX);
+  const __half hz = __float2half_rn(fmn);
+  const float sf = __half2float(hs), zf = __half2float(hz);
+  const float rs = sf != 0.f ? __frcp_rn(sf) : 0.f;
+  uint32_t c[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const float x = (i & 1) ? bf16_hi(w[i >> 1]) : bf16_lo(w[i >> 1]);
+    const float q = (x - zf) * rs;
+    float t = rintf(q);
+    if (sf == 0.f) {
+      t = 0.f;
+    } else if (fabsf(q - t) > 0.5f - 1.f / 4096.f) {
+      t = (float)rint(((double)x - (double)zf) / (double)sf);
+    }
+    t = fminf(fmaxf(t, 0.f), (float)QMAX);
+    c[i] = (uint32_t)t;
+  }
+  if (BITS == 4) {
+    uint32_t out[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      uint32_t v = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v |= c[8 * k + e] << (4 * e);   // even channel in the low nibble
+      out[k] = v;
+    }
+    reinterpret_cast<uint4 *>(codes)[0] = make_uint4(out[0], out[1], out[2], out[3]);
+  } else {
+    uint32_t out[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      out[k] = c[4 * k] | (c[4 * k + 1] << 8) | (c[4 * k + 2] << 16) | (c[4 * k + 3] << 24);
+    reinterpret_cast<uint4 *>(codes)[0] = make_uint4(out[0], out[1], out[2], out[3]);
+    reinterpret_cast<uint4 *>(codes)[1] = make_uint4(out[4], out[5], out[6], out[7]);
+  }
+  *sz = __halves2half2(hs, hz);
+}
+
 // Positions per CTA: kWarps warps x kChunks chunks x 8 positions.
 constexpr int kChunks = 4;
 constexpr int kSpan = kWarps * kChunks * 8;   // 256
@@ -211,7 +306,8 @@ __device__ __forceinline__ int warp_count_below(const int32_t *__restrict__ a, i
 // counts the vertical columns before the span (one search per CTA) and marks
 // those inside it in a shared bit mask, while every warp issues the row loads
 // of its first chunk; then each warp classifies and writes its four chunks of
-// eight positions (copy the bf16 rows, or quantize them into the next low rows).
+// eight positions (copy the bf16 rows, or quantize them into the next low
+// rows), each lane one 32-channel group of one row.
 template <int D, int BITS, bool F8>
 __global__ void __launch_bounds__(kWarps * 32)
 pack_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ v,
@@ -220,9 +316,8 @@ pack_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict
             __half2 *__restrict__ k_sz, __half2 *__restrict__ v_sz,
             __nv_bfloat16 *__restrict__ k_hi, __nv_bfloat16 *__restrict__ v_hi,
             int32_t *__restrict__ lo_pos, uint32_t *status) {
-  constexpr int W32 = D / 64;                 // 32-bit words of bf16 per lane
   constexpr int ROWB = D * BITS / 8;          // packed bytes per low row
-  constexpr int NG = D / 32;
+  constexpr int NG = D / 32;                  // quantization groups per row
   constexpr int PCH = 8;
   __shared__ uint32_t vmask[kSpan / 32];
   __shared__ int s_lo;
@@ -243,16 +338,25 @@ pack_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict
   }
 
   if (threadIdx.x < kSpan / 32) vmask[threadIdx.x] = 0u;
-  uint32_t kw[PCH][W32], vw[PCH][W32];
+  // A chunk is 16 rows (K and V of eight positions); each lane takes one
+  // 32-channel group of one row per pass: lane = row-in-pass * NG + group.
+  constexpr int RP = 32 / NG;                 // rows per pass: 8 (D = 128) or 16 (D = 64)
+  constexpr int NPASS = 16 / RP;
+  const int g = lane % NG, rsub = lane / NG;
+  uint32_t w[NPASS][16];
   auto load_chunk = [&](int j0) {
 #pragma unroll
-    for (int p = 0; p < PCH; ++p) {
-      const int j = j0 + p;
-      const size_t src = ((size_t)bh * L + (j < L ? j : L - 1)) * D;
+    for (int pi = 0; pi < NPASS; ++pi) {
+      const int rho = pi * RP + rsub;          // 0-7: K of position rho, 8-15: V of rho - 8
+      const int j = min(j0 + (rho & 7), L - 1);
+      const __nv_bfloat16 *src = (rho < 8 ? k : v) + ((size_t)bh * L + j) * D + g * 32;
 #pragma unroll
-      for (int i = 0; i < W32; ++i) {
-        kw[p][i] = __ldg(reinterpret_cast<const uint32_t *>(k + src) + lane * W32 + i);
-        vw[p][i] = __ldg(reinterpret_cast<const uint32_t *>(v + src) + lane * W32 + i);
+      for (int u = 0; u < 4; ++u) {
+        const uint4 t = __ldg(reinterpret_cast<const uint4 *>(src) + u);
+        w[pi][4 * u] = t.x;
+        w[pi][4 * u + 1] = t.y;
+        w[pi][4 * u + 2] = t.z;
+        w[pi][4 * u + 3] = t.w;
       }
     }
   };
@@ -284,9 +388,12 @@ pack_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict
     const uint32_t vbits = (word >> (o & 31)) & 0xffu;   // vertical positions of the chunk
     const int cnt0 = lo + (int)before;
 #pragma unroll
-    for (int p = 0; p < PCH; ++p) {
+    for (int pi = 0; pi < NPASS; ++pi) {
+      const int rho = pi * RP + rsub;
+      const bool is_v = rho >= 8;
+      const int p = rho & 7;
       const int j = j0 + p;
-      if (j >= L) break;
+      if (j >= L) continue;
       const int cnt = cnt0 + __popc(vbits & ((1u << p) - 1u));            // verticals before j
       int hi_row = -1, lo_row = -1;
       if (j >= L - window) hi_row = k_vert + j % window;          // the window ring
@@ -294,24 +401,22 @@ pack_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict
       else lo_row = j - cnt;
       if (hi_row >= 0) {
         if (hi_row >= n_hi) {
-          if (lane == 0) raise_status(status, HQ_DEV_BAD_INDEX);
+          raise_status(status, HQ_DEV_BAD_INDEX);
           continue;
         }
-        const size_t dst = ((size_t)bh * n_hi + hi_row) * D;
+        uint4 *dst = reinterpret_cast<uint4 *>((is_v ? v_hi : k_hi) + ((size_t)bh * n_hi + hi_row) * D + g * 32);
 #pragma unroll
-        for (int i = 0; i < W32; ++i) {
-          reinterpret_cast<uint32_t *>(k_hi + dst)[lane * W32 + i] = kw[p][i];
-          reinterpret_cast<uint32_t *>(v_hi + dst)[lane * W32 + i] = vw[p][i];
-        }
+        for (int u = 0; u < 4; ++u)
+          dst[u] = make_uint4(w[pi][4 * u], w[pi][4 * u + 1], w[pi][4 * u + 2], w[pi][4 * u + 3]);
       } else {
         if (lo_row < 0 || lo_row >= n_lo) {
-          if (lane == 0) raise_status(status, HQ_DEV_BAD_INDEX);
+          raise_status(status, HQ_DEV_BAD_INDEX);
           continue;
         }
         const size_t r = (size_t)bh * lo_cap + lo_row;
-        quant_row_store<D, BITS, F8>(kw[p], k_codes + r * ROWB, k_sz + r * NG, lane);
-        quant_row_store<D, BITS, F8>(vw[p], v_codes + r * ROWB, v_sz + r * NG, lane);
-        if (lo_pos && lane == 0) lo_pos[r] = j;
+        quant_group_lane<BITS, F8>(w[pi], (is_v ? v_codes : k_codes) + r * ROWB + g * (32 * BITS / 8),
+                                   (is_v ? v_sz : k_sz) + r * NG + g);
+        if (lo_pos && !is_v && g == 0) lo_pos[r] = j;
       }
     }
   }
