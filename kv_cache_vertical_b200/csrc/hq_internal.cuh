@@ -141,4 +141,26 @@ __device__ __forceinline__ int upper_bound_i32(const int32_t *a, int n, int x) {
   return lo;
 }
 
+// Number of entries of the ascending list a[0, n) below x, found by one warp
+// with 32-way splits (about three rounds of loads for thousands of entries
+// instead of a dozen dependent ones).  Every lane returns the result.
+__device__ __forceinline__ int warp_count_below(const int32_t *__restrict__ a, int n, int x,
+                                                int lane) {
+  int lo = 0, hi = n;                       // the count lies in [lo, hi]
+  while (hi - lo > 32) {
+    const int len = hi - lo;
+    const int si = lo + (int)(((long long)lane * len) >> 5);        // lane 0 samples lo
+    const unsigned below = __ballot_sync(0xffffffffu, __ldg(a + si) < x);
+    const int m = __popc(below);            // samples 0 .. m-1 are below x
+    if (m == 0) return lo;
+    const int s_last = lo + (int)(((long long)(m - 1) * len) >> 5);
+    const int s_next = m < 32 ? lo + (int)(((long long)m * len) >> 5) : hi;
+    lo = s_last + 1;
+    hi = s_next;
+  }
+  const bool in = lane < hi - lo;
+  const unsigned below = __ballot_sync(0xffffffffu, in && __ldg(a + lo + (in ? lane : 0)) < x);
+  return lo + __popc(below);
+}
+
 }  // namespace hq

@@ -49,68 +49,69 @@ __device__ __forceinline__ float rint_div(float x, float s, float rcp_s) {
   return fabsf(q - t) > 0.5f - 1.f / 4096.f ? rintf(__fdiv_rn(x, s)) : t;
 }
 
-// Q rows, four per warp (loads first, then four independent reductions):
-// s = amax / 127, code = clamp(rne(x / s), -127, 127), both divisions single
-// IEEE binary32 roundings.
+// Q rows: s = amax / 127, code = clamp(rne(x / s), -127, 127), both
+// divisions single IEEE binary32 roundings.  Each lane takes one 32-channel
+// group of a row (D / 32 lanes per row, two or one shuffles for the row's
+// maximum), a warp QPASS passes of 32 / (D / 32) rows with every load issued
+// first; codes leave in 16-byte stores.
+constexpr int QPASS = 2;
 template <int D>
 __global__ void __launch_bounds__(256)
 quant_q_rows(const __nv_bfloat16 *__restrict__ q, long long nrows, int8_t *__restrict__ qi8,
              float *__restrict__ sq) {
-  constexpr int CPL = D / 32;                   // channels per lane: 4 or 2
-  constexpr int RPW = 4;                        // rows per warp
+  constexpr int NG = D / 32;                    // lanes per row
+  constexpr int RP = 32 / NG;                   // rows per pass
   const int lane = threadIdx.x & 31;
-  const long long row0 = ((long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5)) * RPW;
-  float x[RPW][CPL];
+  const int g = lane % NG;
+  const long long row0 = ((long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5)) * (RP * QPASS) +
+                         lane / NG;
+  uint32_t w[QPASS][16];
 #pragma unroll
-  for (int rr = 0; rr < RPW; ++rr) {
-    const long long row = row0 + rr;
-    uint32_t w[CPL / 2];
-    if (row < nrows) {
-      const uint32_t *src = reinterpret_cast<const uint32_t *>(q + row * D) + lane * (CPL / 2);
-      if (CPL == 4) {
-        const uint2 v2 = __ldg(reinterpret_cast<const uint2 *>(src));
-        w[0] = v2.x;
-        w[CPL / 2 - 1] = v2.y;
-      } else {
-        w[0] = __ldg(src);
-      }
-    } else {
+  for (int pi = 0; pi < QPASS; ++pi) {
+    const long long row = row0 + pi * RP;
+    const uint4 *src = reinterpret_cast<const uint4 *>(q + (row < nrows ? row : nrows - 1) * D + g * 32);
 #pragma unroll
-      for (int i = 0; i < CPL / 2; ++i) w[i] = 0u;
-    }
-#pragma unroll
-    for (int i = 0; i < CPL / 2; ++i) {
-      x[rr][2 * i] = bf16_lo(w[i]);
-      x[rr][2 * i + 1] = bf16_hi(w[i]);
+    for (int u = 0; u < 4; ++u) {
+      const uint4 t = __ldg(src + u);
+      w[pi][4 * u] = t.x;
+      w[pi][4 * u + 1] = t.y;
+      w[pi][4 * u + 2] = t.z;
+      w[pi][4 * u + 3] = t.w;
     }
   }
-  float amax[RPW];
 #pragma unroll
-  for (int rr = 0; rr < RPW; ++rr) {
-    amax[rr] = 0.f;
+  for (int pi = 0; pi < QPASS; ++pi) {
+    const long long row = row0 + pi * RP;
+    uint32_t am = w[pi][0] & 0x7fff7fffu;       // |x| of both halves
 #pragma unroll
-    for (int i = 0; i < CPL; ++i) amax[rr] = fmaxf(amax[rr], fabsf(x[rr][i]));
-  }
+    for (int i = 1; i < 16; ++i) {
+      uint32_t d;
+      asm("max.bf16x2 %0, %1, %2;\n" : "=r"(d) : "r"(am), "r"(w[pi][i] & 0x7fff7fffu));
+      am = d;
+    }
+    float amax = fmaxf(bf16_lo(am), bf16_hi(am));
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-#pragma unroll
-    for (int rr = 0; rr < RPW; ++rr) amax[rr] = fmaxf(amax[rr], __shfl_xor_sync(0xffffffffu, amax[rr], o));
-  }
-#pragma unroll
-  for (int rr = 0; rr < RPW; ++rr) {
-    const long long row = row0 + rr;
-    if (row >= nrows) break;
-    const float s = amax[rr] == 0.f ? 1.f : __fdiv_rn(amax[rr], 127.f);
+    for (int o = NG / 2; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if (row >= nrows) continue;
+    const float s = amax == 0.f ? 1.f : __fdiv_rn(amax, 127.f);
     const float rcp = __frcp_rn(s);
-    uint32_t packed = 0;
+    uint32_t out[8];
 #pragma unroll
-    for (int i = 0; i < CPL; ++i) {
-      const float c = fminf(fmaxf(rint_div(x[rr][i], s, rcp), -127.f), 127.f);
-      packed |= ((uint32_t)(int)c & 0xffu) << (8 * i);
+    for (int k = 0; k < 8; ++k) {
+      uint32_t packed = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t word = w[pi][2 * k + (e >> 1)];
+        const float x = (e & 1) ? bf16_hi(word) : bf16_lo(word);
+        const float c = fminf(fmaxf(rint_div(x, s, rcp), -127.f), 127.f);
+        packed |= ((uint32_t)(int)c & 0xffu) << (8 * e);
+      }
+      out[k] = packed;
     }
-    if (CPL == 4) reinterpret_cast<uint32_t *>(qi8 + row * D)[lane] = packed;
-    else reinterpret_cast<uint16_t *>(qi8 + row * D)[lane] = (uint16_t)packed;
-    if (lane == 0) sq[row] = s;
+    uint4 *dst = reinterpret_cast<uint4 *>(qi8 + row * D + g * 32);
+    dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+    dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+    if (g == 0) sq[row] = s;
   }
 }
 
@@ -127,12 +128,15 @@ __device__ __forceinline__ int remaining_pos(const int32_t *id, int k_vert, int 
 }
 
 // One CTA (256 threads) per block of 64 consecutive remaining keys of one
-// (b, kv head): INT8 codes with one symmetric scale per block.
+// (b, kv head): INT8 codes with one symmetric scale per block.  The block's
+// rows are read once, 16 bytes per load, and held in registers for both the
+// maximum and the codes.
 template <int D>
 __global__ void __launch_bounds__(256)
 quant_k_remaining(const __nv_bfloat16 *__restrict__ k, const int32_t *__restrict__ idx, int N,
                   int k_vert, int nblk, int8_t *__restrict__ ki8, float *__restrict__ sk) {
-  constexpr int WPR = D / 2;                                    // 32-bit words per row
+  constexpr int U = D / 8;                                      // 16-byte pieces per row
+  constexpr int PER = TILE * U / 256;                           // pieces per thread: 4 or 2
   const int blk = blockIdx.x, bh = blockIdx.y;
   const int nr = N - k_vert;
   const int c0 = blk * TILE, n = min(TILE, nr - c0);
@@ -141,12 +145,22 @@ quant_k_remaining(const __nv_bfloat16 *__restrict__ k, const int32_t *__restrict
   __shared__ float red[8];
   if (threadIdx.x < n) pos[threadIdx.x] = remaining_pos(id, k_vert, c0 + threadIdx.x);
   __syncthreads();
-  const uint32_t *src = reinterpret_cast<const uint32_t *>(k + (size_t)bh * N * D);
-  float amax = 0.f;
-  for (int e = threadIdx.x; e < n * WPR; e += blockDim.x) {
-    const uint32_t w = src[(size_t)pos[e / WPR] * WPR + e % WPR];
-    amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(w)), fabsf(bf16_hi(w))));
+  const uint4 *src = reinterpret_cast<const uint4 *>(k + (size_t)bh * N * D);
+  uint4 v[PER];
+  uint32_t am = 0u;
+#pragma unroll
+  for (int q = 0; q < PER; ++q) {
+    const int e = threadIdx.x + q * 256;                        // piece e % U of row e / U
+    v[q] = e < n * U ? __ldg(src + (size_t)pos[e / U] * U + e % U) : make_uint4(0, 0, 0, 0);
+    const uint32_t ww[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t d;
+      asm("max.bf16x2 %0, %1, %2;\n" : "=r"(d) : "r"(am), "r"(ww[i] & 0x7fff7fffu));
+      am = d;
+    }
   }
+  float amax = fmaxf(bf16_lo(am), bf16_hi(am));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
@@ -156,62 +170,103 @@ quant_k_remaining(const __nv_bfloat16 *__restrict__ k, const int32_t *__restrict
   for (int w = 1; w < 8; ++w) amax = fmaxf(amax, red[w]);
   const float s = amax == 0.f ? 1.f : __fdiv_rn(amax, 127.f);
   const float rcp = __frcp_rn(s);
-  uint16_t *dst = reinterpret_cast<uint16_t *>(ki8 + ((size_t)bh * nr + c0) * D);
-  for (int e = threadIdx.x; e < n * WPR; e += blockDim.x) {
-    const uint32_t w = src[(size_t)pos[e / WPR] * WPR + e % WPR];
-    float c0f = fminf(fmaxf(rint_div(bf16_lo(w), s, rcp), -127.f), 127.f);
-    float c1f = fminf(fmaxf(rint_div(bf16_hi(w), s, rcp), -127.f), 127.f);
-    dst[e] = (uint16_t)(((uint32_t)(int)c0f & 0xffu) | (((uint32_t)(int)c1f & 0xffu) << 8));
+  uint2 *dst = reinterpret_cast<uint2 *>(ki8 + ((size_t)bh * nr + c0) * D);   // 8 codes per piece
+#pragma unroll
+  for (int q = 0; q < PER; ++q) {
+    const int e = threadIdx.x + q * 256;
+    if (e >= n * U) break;
+    const uint32_t ww[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+    uint32_t out[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t packed = 0;
+#pragma unroll
+      for (int e4 = 0; e4 < 4; ++e4) {
+        const uint32_t word = ww[2 * h + (e4 >> 1)];
+        const float x = (e4 & 1) ? bf16_hi(word) : bf16_lo(word);
+        const float c = fminf(fmaxf(rint_div(x, s, rcp), -127.f), 127.f);
+        packed |= ((uint32_t)(int)c & 0xffu) << (8 * e4);
+      }
+      out[h] = packed;
+    }
+    dst[e] = make_uint2(out[0], out[1]);
   }
   if (threadIdx.x == 0) sk[(size_t)bh * nblk + blk] = s;
 }
 
 // bf16 V -> fp16 V (exact for |v| in the fp16 normal range), both in position
 // order (window tiles) and compacted to the remaining keys (low-bit tiles).
-// Eight consecutive positions of one (b, kv head) per warp task: one binary
-// search finds the verticals before the chunk, a ballot over the next index
-// entries marks the chunk's own, and all eight rows load before any store.
+// One CTA per span of VSPAN consecutive positions of one (b, kv head): warp 0
+// counts the verticals before the span (one warp search) and marks those in
+// it in a shared bit mask while every warp loads its first rows; each warp
+// then converts and stores its 32 positions, 16 bytes per lane and access.
+constexpr int VSPAN = 256;
 template <int D>
 __global__ void __launch_bounds__(256)
 v_prep(const __nv_bfloat16 *__restrict__ v, const int32_t *__restrict__ idx, int nbh, int N,
        int k_vert, __half *__restrict__ vh, __half *__restrict__ vc) {
-  constexpr int W32 = D / 64;                                    // 32-bit words per lane
-  constexpr int PCH = 8;
-  const int lane = threadIdx.x & 31;
-  const int cpb = (N + PCH - 1) / PCH;
-  const long long ntask = (long long)nbh * cpb;
+  constexpr int LPR = D / 8;                                     // lanes per row (16 bytes each)
+  constexpr int RPI = 32 / LPR;                                  // rows per warp access: 2 or 4
+  constexpr int PCH = 8;                                         // positions per chunk
+  constexpr int NA = PCH / RPI;                                  // accesses per chunk per lane
+  __shared__ uint32_t vmask[VSPAN / 32];
+  __shared__ int s_lo;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nspan = (N + VSPAN - 1) / VSPAN;
+  const int bh = (int)(blockIdx.x / nspan);
+  const int p0 = (int)(blockIdx.x % nspan) * VSPAN;
+  const int p1 = min(p0 + VSPAN, N);
   const int nr = N - k_vert;
-  for (long long task = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); task < ntask;
-       task += (long long)gridDim.x * (blockDim.x / 32)) {
-    const int bh = (int)(task / cpb), j0 = (int)(task % cpb) * PCH;
-    const int32_t *id = idx + (size_t)bh * k_vert;
-    const int cnt0 = j0 > 0 ? upper_bound_i32(id, k_vert, j0 - 1) : 0;   // verticals before j0
-    const int e = cnt0 + (lane & (PCH - 1));
-    const int ve = (lane < PCH && e < k_vert) ? __ldg(id + e) : INT_MAX;
-    const uint32_t vbit = (ve >= j0 && ve < j0 + PCH) ? 1u << (ve - j0) : 0u;
-    const uint32_t vbits = __reduce_or_sync(0xffffffffu, vbit);
-    uint32_t w[PCH][W32];
+  const int32_t *id = idx + (size_t)bh * k_vert;
+  const int piece = lane % LPR, rsub = lane / LPR;
+  if (threadIdx.x < VSPAN / 32) vmask[threadIdx.x] = 0u;
+  uint4 w[NA];
+  auto load_chunk = [&](int j0) {
 #pragma unroll
-    for (int p = 0; p < PCH; ++p) {
-      const int j = j0 + p < N ? j0 + p : N - 1;
-      const uint32_t *src = reinterpret_cast<const uint32_t *>(v + ((size_t)bh * N + j) * D) + lane * W32;
-#pragma unroll
-      for (int i = 0; i < W32; ++i) w[p][i] = __ldg(src + i);
+    for (int a = 0; a < NA; ++a) {
+      const int j = min(j0 + a * RPI + rsub, N - 1);
+      w[a] = __ldg(reinterpret_cast<const uint4 *>(v + ((size_t)bh * N + j) * D) + piece);
     }
+  };
+  const int jw = p0 + warp * (VSPAN / 8);                       // this warp's 32 positions
+  if (jw < p1) load_chunk(jw);
+  __syncthreads();                                               // mask cleared
+  if (warp == 0) {
+    const int lo = warp_count_below(id, k_vert, p0, lane);
+    if (lane == 0) s_lo = lo;
+    for (int t = lo + lane;; t += 32) {
+      const int x = t < k_vert ? __ldg(id + t) : INT_MAX;
+      if (x >= p0 && x < p1) atomicOr(&vmask[(x - p0) >> 5], 1u << ((x - p0) & 31));
+      if (__any_sync(0xffffffffu, x >= p1)) break;
+    }
+  }
+  __syncthreads();
+  const int lo = s_lo;
+  for (int ci = 0; ci < VSPAN / 8 / PCH; ++ci) {
+    const int j0 = jw + ci * PCH;
+    if (j0 >= p1) break;
+    if (ci > 0) load_chunk(j0);
 #pragma unroll
-    for (int p = 0; p < PCH; ++p) {
-      const int j = j0 + p;
-      if (j >= N) break;
-      const bool vert = (vbits >> p) & 1u;
-      const int rank = j - cnt0 - __popc(vbits & ((1u << p) - 1u));       // among the remaining keys
-      __half2 *dh = reinterpret_cast<__half2 *>(vh + ((size_t)bh * N + j) * D) + lane * W32;
-      __half2 *dc = reinterpret_cast<__half2 *>(vc + ((size_t)bh * nr + rank) * D) + lane * W32;
+    for (int a = 0; a < NA; ++a) {
+      const int j = j0 + a * RPI + rsub;
+      if (j >= p1) continue;
+      const int o = j - p0;
+      uint32_t before = 0;                                       // verticals in the span before j
+      for (int wdx = 0; wdx < (o >> 5); ++wdx) before += __popc(vmask[wdx]);
+      const uint32_t word = vmask[o >> 5];
+      before += __popc(word & ((1u << (o & 31)) - 1u));
+      const bool vert = (word >> (o & 31)) & 1u;
+      const int rank = j - lo - (int)before;                     // among the remaining keys
+      const uint32_t ww[4] = {w[a].x, w[a].y, w[a].z, w[a].w};
+      uint32_t hh[4];
 #pragma unroll
-      for (int i = 0; i < W32; ++i) {
-        const __half2 x = __floats2half2_rn(bf16_lo(w[p][i]), bf16_hi(w[p][i]));
-        dh[i] = x;
-        if (!vert && rank >= 0 && rank < nr) dc[i] = x;
+      for (int i = 0; i < 4; ++i) {
+        const __half2 x = __floats2half2_rn(bf16_lo(ww[i]), bf16_hi(ww[i]));
+        hh[i] = *reinterpret_cast<const uint32_t *>(&x);
       }
+      const uint4 out = make_uint4(hh[0], hh[1], hh[2], hh[3]);
+      reinterpret_cast<uint4 *>(vh + ((size_t)bh * N + j) * D)[piece] = out;
+      if (!vert && rank >= 0 && rank < nr) reinterpret_cast<uint4 *>(vc + ((size_t)bh * nr + rank) * D)[piece] = out;
     }
   }
 }
@@ -553,7 +608,8 @@ cudaError_t quant_t(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const int32_
                     int Hq, int Hkv, int N, int k_vert, int8_t *qi8, float *sq, int8_t *ki8,
                     float *sk, cudaStream_t s) {
   const long long nrows = (long long)B * Hq * N;
-  quant_q_rows<D><<<(unsigned)((nrows + 31) / 32), 256, 0, s>>>(q, nrows, qi8, sq);   // 8 warps x 4 rows
+  const long long rows_per_block = 8LL * (32 / (D / 32)) * QPASS;        // 8 warps
+  quant_q_rows<D><<<(unsigned)((nrows + rows_per_block - 1) / rows_per_block), 256, 0, s>>>(q, nrows, qi8, sq);
   const int nblk_r = (N - k_vert + TILE - 1) / TILE;
   if (nblk_r > 0)
     quant_k_remaining<D><<<dim3(nblk_r, B * Hkv), 256, 0, s>>>(k, idx, N, k_vert, nblk_r, ki8, sk);
@@ -572,11 +628,7 @@ cudaError_t prefill_t(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
   cudaError_t e = quant_t<D>(q, k, idx, B, Hq, Hkv, N, k_vert, w.qi8, w.sq, w.ki8, w.sk, s);
   if (e != cudaSuccess) return e;
   {
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    long long blocks = ((long long)nbh * ((N + 7) / 8) + 7) / 8;   // 8 warps x 8 positions per block
-    if (blocks > 8LL * sms) blocks = 8LL * sms;
+    const long long blocks = (long long)nbh * ((N + VSPAN - 1) / VSPAN);   // one CTA per span
     v_prep<D><<<(unsigned)blocks, 256, 0, s>>>(v, idx, nbh, N, k_vert, w.vh, w.vc);
   }
   if (kpad > 0)
