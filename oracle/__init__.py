@@ -56,8 +56,8 @@ def _load():
         lib.hqo_pack_kv.argtypes = [P, P, P] + [I] * 9 + [P] * 7
         lib.hqo_kv_append.argtypes = [P, P] + [I] * 11 + [P] * 7
         lib.hqo_decode_attn.argtypes = [P] * 7 + [I] * 9 + [D, P, P]
-        lib.hqo_prefill_quant.argtypes = [P, P, P] + [I] * 7 + [P] * 4
-        lib.hqo_prefill_attn.argtypes = [P] * 8 + [I] * 8 + [D, P, I, P]
+        lib.hqo_prefill_quant.argtypes = [P, P, P] + [I] * 8 + [P] * 4
+        lib.hqo_prefill_attn.argtypes = [P] * 8 + [I] * 9 + [D, P, I, P]
         lib.hqo_max_threads.argtypes = []
         for f in ("hqo_probe_scores", "hqo_topk", "hqo_quant_row", "hqo_pack_kv", "hqo_kv_append",
                   "hqo_decode_attn", "hqo_prefill_quant", "hqo_prefill_attn", "hqo_max_threads"):
@@ -219,10 +219,11 @@ def decode_attn(q, cache: dict, Hkv: int, scale: float | None = None):
     return out, lse
 
 
-def prefill_quant(q, k, idx, kblock: int = 64):
-    """INT8 codes + fp32 scales.  Q per token: qi8 [B,Hq,N,D], sq [B,Hq,N].
-    K over the remaining (non-vertical) keys in position order, one scale per
-    kblock of them: ki8 [B,Hkv,N-kv,D], sk [B,Hkv,ceil((N-kv)/kblock)]."""
+def prefill_quant(q, k, idx, kblock: int = 64, fmt: int = FMT_INT):
+    """INT8 (fmt 0) or E4M3 (fmt 1, bits in the int8 arrays) codes + fp32
+    scales.  Q per token: qi8 [B,Hq,N,D], sq [B,Hq,N].  K over the remaining
+    (non-vertical) keys in position order, one scale per kblock of them:
+    ki8 [B,Hkv,N-kv,D], sk [B,Hkv,ceil((N-kv)/kblock)]."""
     qq, kk = _u16(q), _u16(k)
     B, Hq, N, D = qq.shape
     Hkv = kk.shape[1]
@@ -234,14 +235,14 @@ def prefill_quant(q, k, idx, kblock: int = 64):
     sq = np.zeros((B, Hq, N), np.float32)
     ki8 = np.zeros((B, Hkv, nr, D), np.int8)
     sk = np.zeros((B, Hkv, nblk), np.float32)
-    rc = _load().hqo_prefill_quant(_p(qq), _p(kk), _p(idx), B, Hq, Hkv, N, D, kv, kblock,
+    rc = _load().hqo_prefill_quant(_p(qq), _p(kk), _p(idx), B, Hq, Hkv, N, D, kv, kblock, fmt,
                                    _p(qi8), _p(sq), _p(ki8), _p(sk))
     assert rc == 0, rc
     return qi8, sq, ki8, sk
 
 
 def prefill_attn(q, k, v, idx, window: int, quant=None, rows=None, kblock: int = 64,
-                 scale: float | None = None) -> np.ndarray:
+                 scale: float | None = None, fmt: int = FMT_INT) -> np.ndarray:
     """Hybrid prefill attention, fp64 [B, Hq, nrows, D] for the given query rows."""
     qq, kk, vv = _u16(q), _u16(k), _u16(v)
     B, Hq, N, D = qq.shape
@@ -249,13 +250,13 @@ def prefill_attn(q, k, v, idx, window: int, quant=None, rows=None, kblock: int =
     idx = np.ascontiguousarray(idx, np.int32)
     kv = idx.shape[2]
     if quant is None:
-        quant = prefill_quant(qq, kk, idx, kblock)
+        quant = prefill_quant(qq, kk, idx, kblock, fmt)
     qi8, sq, ki8, sk = (np.ascontiguousarray(a) for a in quant)
     r = None if rows is None else np.ascontiguousarray(rows, np.int32)
     nrows = N if r is None else int(r.shape[0])
     out = np.zeros((B, Hq, nrows, D), np.float64)
     rc = _load().hqo_prefill_attn(_p(qq), _p(kk), _p(vv), _p(idx), _p(qi8), _p(sq), _p(ki8),
-                                  _p(sk), B, Hq, Hkv, N, D, window, kv, kblock,
+                                  _p(sk), B, Hq, Hkv, N, D, window, kv, kblock, fmt,
                                   default_scale(D) if scale is None else scale, _p(r), nrows,
                                   _p(out))
     assert rc == 0, rc

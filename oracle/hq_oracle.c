@@ -620,25 +620,58 @@ static int8_t q8_code(uint16_t xb, float s)
 }
 
 /*
+ * FP8 low part (fmt 1; a reading for the pages' FP8 "third precision point",
+ * wiki summary "Gaps"): the same granularity, symmetric E4M3 codes,
+ *   s = fl32(amax / 448), s = 1 when amax == 0;  c = e4m3_rne_sat(fl32(x / s)),
+ * the binary32 quotient rounded once more, to E4M3 (nearest even,
+ * saturating); the code's bits are stored in the 8-bit array.
+ */
+static float f8_scale(const uint16_t *x, int n)
+{
+    float amax = 0.0f;
+    for (int i = 0; i < n; ++i) {
+        float a = fabsf((float)bf16_to_f64(x[i]));
+        if (a > amax) amax = a;
+    }
+    if (amax == 0.0f)
+        return 1.0f;
+    volatile float s = amax / 448.0f;
+    return s;
+}
+
+static int8_t f8_code(uint16_t xb, float s)
+{
+    volatile float t = (float)bf16_to_f64(xb) / s;
+    return (int8_t)f64_to_e4m3_rne_sat((double)t);
+}
+
+/* A low-part code as a number: the integer, or the E4M3 value. */
+static double low_value(int8_t c, int fmt)
+{
+    return fmt == 1 ? e4m3_to_f64((uint8_t)c) : (double)c;
+}
+
+/*
  * q: bf16 [B, Hq, N, D] -> qi8 [B, Hq, N, D], sq [B, Hq, N].
  * k: bf16 [B, Hkv, N, D], idx [B, Hkv, kv] (ascending) ->
  *    ki8 [B, Hkv, N - kv, D] (the remaining keys, compacted in position order),
  *    sk  [B, Hkv, ceil((N - kv) / kblock)].
  */
 int hqo_prefill_quant(const uint16_t *q, const uint16_t *k, const int32_t *idx, int B, int Hq,
-                      int Hkv, int N, int D, int kv, int kblock, int8_t *qi8, float *sq,
+                      int Hkv, int N, int D, int kv, int kblock, int fmt, int8_t *qi8, float *sq,
                       int8_t *ki8, float *sk)
 {
-    if (B <= 0 || Hq <= 0 || Hkv <= 0 || N <= 0 || D <= 0 || kblock <= 0 || kv < 0 || kv > N)
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || N <= 0 || D <= 0 || kblock <= 0 || kv < 0 || kv > N ||
+        fmt < 0 || fmt > 1)
         return 1;
     const long long nq = (long long)B * Hq * N;
 #pragma omp parallel for schedule(static)
     for (long long r = 0; r < nq; ++r) {
         const uint16_t *x = q + (size_t)r * D;
-        float s = q8_scale(x, D);
+        float s = fmt == 1 ? f8_scale(x, D) : q8_scale(x, D);
         sq[r] = s;
         for (int d = 0; d < D; ++d)
-            qi8[(size_t)r * D + d] = q8_code(x[d], s);
+            qi8[(size_t)r * D + d] = fmt == 1 ? f8_code(x[d], s) : q8_code(x[d], s);
     }
     const int nr = N - kv;                        /* remaining keys per (b, kv head) */
     const int nblk = (nr + kblock - 1) / kblock;
@@ -660,10 +693,10 @@ int hqo_prefill_quant(const uint16_t *q, const uint16_t *k, const int32_t *idx, 
         for (int blk = 0; blk < nblk; ++blk) {
             const int c0 = blk * kblock, n = (nr - c0 < kblock ? nr - c0 : kblock);
             const uint16_t *x = rem + (size_t)c0 * D;
-            float s = q8_scale(x, n * D);
+            float s = fmt == 1 ? f8_scale(x, n * D) : q8_scale(x, n * D);
             sk[(size_t)bh * nblk + blk] = s;
             for (int e = 0; e < n * D; ++e)
-                ki8[((size_t)bh * nr + c0) * D + e] = q8_code(x[e], s);
+                ki8[((size_t)bh * nr + c0) * D + e] = fmt == 1 ? f8_code(x[e], s) : q8_code(x[e], s);
         }
         free(rem);
     }
@@ -681,7 +714,9 @@ int hqo_prefill_quant(const uint16_t *q, const uint16_t *k, const int32_t *idx, 
  * in the window (j > i - W) or j is a vertical column, else "low".  A high
  * logit is q_i . k_j * scale from the bf16 values; a low logit is
  *   (sum_d qi8[i,d] * ki8[c,d]) * sq[i] * sk[c / kblock] * scale
- * with the integer dot product exact, where c = j - #(vertical columns < j) is
+ * with the dot product of the codes exact (integers, or E4M3 values for
+ * fmt 1: products of 4-bit significands, summed in double without rounding
+ * for D <= 512), where c = j - #(vertical columns < j) is
  * the key's rank among the remaining keys (see the pre-pass).  One exact softmax over all j <= i;
  * the output is sum_j p_ij v_j with v in bf16 and p unrounded.
  *
@@ -691,10 +726,11 @@ int hqo_prefill_quant(const uint16_t *q, const uint16_t *k, const int32_t *idx, 
 int hqo_prefill_attn(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                      const int32_t *idx, const int8_t *qi8, const float *sq, const int8_t *ki8,
                      const float *sk, int B, int Hq, int Hkv, int N, int D, int window, int kv,
-                     int kblock, double scale, const int32_t *rows, int nrows, double *out)
+                     int kblock, int fmt, double scale, const int32_t *rows, int nrows,
+                     double *out)
 {
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || N <= 0 || D <= 0 || window < 0 ||
-        kv < 0 || kv > N || kblock <= 0)
+        kv < 0 || kv > N || kblock <= 0 || fmt < 0 || fmt > 1)
         return 1;
     if (!rows)
         nrows = N;
@@ -727,10 +763,10 @@ int hqo_prefill_attn(const uint16_t *q, const uint16_t *k, const uint16_t *v,
             } else {
                 const int c = j - vi;                  /* vi = #(vertical columns < j) */
                 const int8_t *kc = ki8 + (bh * nr + c) * D;
-                long long acc = 0;
+                double acc = 0.0;                      /* exact for both formats */
                 for (int d = 0; d < D; ++d)
-                    acc += (long long)qc[d] * (long long)kc[d];
-                logit = (double)acc * (double)sq[(size_t)bhq * N + i] *
+                    acc += low_value(qc[d], fmt) * low_value(kc[d], fmt);
+                logit = acc * (double)sq[(size_t)bhq * N + i] *
                         (double)sk[bh * nblk + c / kblock] * scale;
             }
             s[j] = logit;

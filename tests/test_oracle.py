@@ -506,6 +506,62 @@ def test_prefill_quant_matches_numpy_float32():
     assert sk.max() < 1000.0 / 127
 
 
+def test_prefill_fp8_quant_matches_float32_and_torch_cast():
+    """FP8 low part: s = fl32(amax / 448), c = E4M3(fl32(x / s)) -- numpy
+    float32 for the divisions, torch's float8_e4m3fn cast (nearest even) for
+    the last rounding; vertical keys never quantized, zero blocks scale 1."""
+    B, Hq, Hkv, N, D = 1, 2, 1, 160, 64
+    q = bf16(RNG.standard_normal((B, Hq, N, D)) * 3)
+    k = bf16(RNG.standard_normal((B, Hkv, N, D)))
+    idx = np.array([[[2, 5, 70, 71, 100]]], np.int32)
+    rem = np.setdiff1d(np.arange(N), idx[0, 0])
+    k[0, 0, rem[64:128]] = 0
+    k[0, 0, 70] = 1000.0
+    qc, sq, kc, sk = oracle.prefill_quant(q, k, idx, 64, fmt=oracle.FMT_FP8)
+
+    def e4m3(x32):          # float32 quotients, all within +-448 (1 + 2^-23)
+        x32 = np.clip(x32, -448, 448)
+        return torch.from_numpy(x32).to(torch.float8_e4m3fn).view(torch.int8).numpy()
+    qf = q.float().numpy()
+    assert np.array_equal(sq, (np.abs(qf).max(-1) / np.float32(448)).astype(np.float32))
+    assert np.array_equal(qc, e4m3((qf / sq[..., None]).astype(np.float32)))
+    kf = k.float().numpy()[0, 0][rem]
+    for blk in range(3):
+        seg = kf[64 * blk:64 * blk + 64]
+        a = np.abs(seg).max()
+        sblk = np.float32(1) if a == 0 else np.float32(a) / np.float32(448)
+        assert sk[0, 0, blk] == sblk
+        assert np.array_equal(kc[0, 0, 64 * blk:64 * blk + 64], e4m3((seg / sblk).astype(np.float32)))
+    assert sk[0, 0, 1] == 1 and not kc[0, 0, 64:128].any()
+    assert np.abs(_e4m3_torch(qc.view(np.uint8))).max() == 448      # the row maximum maps to 448
+
+
+def test_prefill_fp8_path_is_exact_on_e4m3_inputs():
+    # rows and blocks whose maximum is 448 get scale 1 and codes equal to the
+    # values when the values are E4M3 numbers: the all-low FP8 path is then
+    # exact attention on those values
+    B, Hq, Hkv, N, D = 1, 2, 1, 128, 16
+    vals = _e4m3_torch(np.arange(0, 0x60, 3).astype(np.uint8))       # 0 .. 96, exact in bf16
+    vals = np.concatenate([vals, -vals])
+    q = RNG.choice(vals, (B, Hq, N, D))
+    k = RNG.choice(vals, (B, Hkv, N, D))
+    q[..., 0] = 448
+    k[..., 0, :] = 0
+    k[..., 0, 1] = 448
+    k[..., 64, 1] = -448
+    v = RNG.standard_normal((B, Hkv, N, D))
+    scale = 1 / 2 ** 18
+    out = oracle.prefill_attn(bf16(q), bf16(k), bf16(v), np.zeros((B, Hkv, 0), np.int32),
+                              window=0, scale=scale, fmt=oracle.FMT_FP8)
+    ref = _sdpa(bf16(q), bf16(k).repeat_interleave(2, 1), bf16(v).repeat_interleave(2, 1),
+                scale, True)
+    assert np.allclose(out, ref.numpy(), atol=1e-12)
+    # and the INT8 reading of the same inputs is not exact (its grid is coarser)
+    out8 = oracle.prefill_attn(bf16(q), bf16(k), bf16(v), np.zeros((B, Hkv, 0), np.int32),
+                               window=0, scale=scale)
+    assert np.abs(out8 - ref.numpy()).max() > 1e-9
+
+
 def test_prefill_all_high_precision_equals_causal_attention():
     B, Hq, Hkv, N, D = 1, 4, 2, 70, 32
     q = bf16(RNG.standard_normal((B, Hq, N, D)))
