@@ -285,6 +285,17 @@ hq_status hq_kv_append(const void *k_new, const void *v_new, int B, int Hkv, int
 hq_status hq_prefill_quant(const void *q, const void *k, const int32_t *idx, int B, int Hq,
                            int Hkv, int N, int D, int k_vert, int8_t *qi8, float *sq,
                            int8_t *ki8, float *sk, void *stream);
+/*
+ * The same with a choice of low-part format: HQ_KV_INT (the INT8 codes
+ * above) or HQ_KV_FP8, the FP8 third precision point the wiki summary's
+ * "Gaps" names for Blackwell, taken at the same granularity (library
+ * reading): s = fl32(amax / 448) (1 if amax = 0), code = E4M3 of fl32(x / s)
+ * rounded to nearest even and saturated to +-448; the code bits go to the
+ * same int8 arrays.
+ */
+hq_status hq_prefill_quant_ex(const void *q, const void *k, const int32_t *idx, int B, int Hq,
+                              int Hkv, int N, int D, int k_vert, int low_fmt, int8_t *qi8,
+                              float *sq, int8_t *ki8, float *sk, void *stream);
 
 /*
  * Causal attention in which, for query i, key j <= i is "high" when it is in
@@ -302,6 +313,17 @@ hq_status hq_prefill_attn(const void *q, const void *k, const void *v, const int
                           int Hq, int Hkv, int N, int D, int window, int k_vert,
                           float softmax_scale, float *out, void *ws, size_t ws_bytes,
                           void *stream);
+/*
+ * The same with a choice of low-part format (HQ_KV_INT: the INT8 low part
+ * above; HQ_KV_FP8: the E4M3 codes of hq_prefill_quant_ex, whose low logit is
+ * the fp32-accumulated dot product of the E4M3 values times sq[i] and the
+ * key block's scale).  HQ_KV_FP8 needs the tcgen05 path (D = 128, an even
+ * number of query heads per KV head), else HQ_ERR_UNSUPPORTED.
+ */
+hq_status hq_prefill_attn_ex(const void *q, const void *k, const void *v, const int32_t *idx,
+                             int B, int Hq, int Hkv, int N, int D, int window, int k_vert,
+                             float softmax_scale, int low_fmt, float *out, void *ws,
+                             size_t ws_bytes, void *stream);
 
 #ifdef __cplusplus
 }

@@ -196,20 +196,29 @@ hq_status hq_decode_attn(const void *q, const hq_kv_cache *cache, int B, int Hq,
                                    status_word(ws), (cudaStream_t)stream));
 }
 
-hq_status hq_prefill_quant(const void *q, const void *k, const int32_t *idx, int B, int Hq,
-                           int Hkv, int N, int D, int k_vert, int8_t *qi8, float *sq,
-                           int8_t *ki8, float *sk, void *stream) {
+hq_status hq_prefill_quant_ex(const void *q, const void *k, const int32_t *idx, int B, int Hq,
+                              int Hkv, int N, int D, int k_vert, int low_fmt, int8_t *qi8,
+                              float *sq, int8_t *ki8, float *sk, void *stream) {
   if (!q || !k || !qi8 || !sq || (k_vert < N && (!ki8 || !sk)) || (k_vert > 0 && !idx))
     return HQ_ERR_INVALID_ARG;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || N <= 0 || k_vert < 0 || k_vert > N)
     return HQ_ERR_INVALID_ARG;
-  if ((D != 64 && D != 128) || !supported_G(Hq, Hkv)) return HQ_ERR_UNSUPPORTED;
+  if ((D != 64 && D != 128) || !supported_G(Hq, Hkv) ||
+      (low_fmt != HQ_KV_INT && low_fmt != HQ_KV_FP8))
+    return HQ_ERR_UNSUPPORTED;
   const void *ptrs[] = {q, k, qi8, ki8};
   for (const void *p : ptrs)
     if (p && !aligned16(p)) return HQ_ERR_INVALID_ARG;
   return cuda_status(launch_prefill_quant((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, idx,
-                                          B, Hq, Hkv, N, D, k_vert, qi8, sq, ki8, sk,
+                                          B, Hq, Hkv, N, D, k_vert, low_fmt, qi8, sq, ki8, sk,
                                           (cudaStream_t)stream));
+}
+
+hq_status hq_prefill_quant(const void *q, const void *k, const int32_t *idx, int B, int Hq,
+                           int Hkv, int N, int D, int k_vert, int8_t *qi8, float *sq,
+                           int8_t *ki8, float *sk, void *stream) {
+  return hq_prefill_quant_ex(q, k, idx, B, Hq, Hkv, N, D, k_vert, HQ_KV_INT, qi8, sq, ki8, sk,
+                             stream);
 }
 
 size_t hq_prefill_workspace_size(int B, int Hq, int Hkv, int N, int D, int k_vert) {
@@ -217,23 +226,33 @@ size_t hq_prefill_workspace_size(int B, int Hq, int Hkv, int N, int D, int k_ver
   return prefill_ws_bytes(B, Hq, Hkv, N, D, k_vert);
 }
 
-hq_status hq_prefill_attn(const void *q, const void *k, const void *v, const int32_t *idx, int B,
-                          int Hq, int Hkv, int N, int D, int window, int k_vert,
-                          float softmax_scale, float *out, void *ws, size_t ws_bytes,
-                          void *stream) {
+hq_status hq_prefill_attn_ex(const void *q, const void *k, const void *v, const int32_t *idx,
+                             int B, int Hq, int Hkv, int N, int D, int window, int k_vert,
+                             float softmax_scale, int low_fmt, float *out, void *ws,
+                             size_t ws_bytes, void *stream) {
   if (!q || !k || !v || !out || (k_vert > 0 && !idx)) return HQ_ERR_INVALID_ARG;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || N <= 0 || window < 0 || k_vert < 0 ||
       k_vert > N - (window < N ? window : N))
     return HQ_ERR_INVALID_ARG;
   if ((D != 64 && D != 128) || !supported_G(Hq, Hkv)) return HQ_ERR_UNSUPPORTED;
+  if (low_fmt != HQ_KV_INT && (low_fmt != HQ_KV_FP8 || !prefill_tc_supported(D, Hq, Hkv)))
+    return HQ_ERR_UNSUPPORTED;
   const void *ptrs[] = {q, k, v, out};
   for (const void *p : ptrs)
     if (!aligned16(p)) return HQ_ERR_INVALID_ARG;
   if (!ws || ws_bytes < prefill_ws_bytes(B, Hq, Hkv, N, D, k_vert)) return HQ_ERR_WORKSPACE;
   return cuda_status(launch_prefill((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k,
                                     (const __nv_bfloat16 *)v, idx, B, Hq, Hkv, N, D, window,
-                                    k_vert, resolve_scale(softmax_scale, D), out, (uint8_t *)ws,
-                                    status_word(ws), (cudaStream_t)stream));
+                                    k_vert, resolve_scale(softmax_scale, D), low_fmt, out,
+                                    (uint8_t *)ws, status_word(ws), (cudaStream_t)stream));
+}
+
+hq_status hq_prefill_attn(const void *q, const void *k, const void *v, const int32_t *idx, int B,
+                          int Hq, int Hkv, int N, int D, int window, int k_vert,
+                          float softmax_scale, float *out, void *ws, size_t ws_bytes,
+                          void *stream) {
+  return hq_prefill_attn_ex(q, k, v, idx, B, Hq, Hkv, N, D, window, k_vert, softmax_scale,
+                            HQ_KV_INT, out, ws, ws_bytes, stream);
 }
 
 }  // extern "C"

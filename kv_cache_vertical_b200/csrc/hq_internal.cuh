@@ -91,8 +91,8 @@ cudaError_t launch_decode_merge(const float *part_out, const float *part_lse, in
 
 cudaError_t launch_prefill_quant(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
                                  const int32_t *idx, int B, int Hq, int Hkv, int N, int D,
-                                 int k_vert, int8_t *qi8, float *sq, int8_t *ki8, float *sk,
-                                 cudaStream_t s);
+                                 int k_vert, int low_fmt, int8_t *qi8, float *sq, int8_t *ki8,
+                                 float *sk, cudaStream_t s);
 // tcgen05 prefill (head_dim 128, an even number of query heads per KV head).
 struct TcLaunch {
   const __nv_bfloat16 *q, *k;        // bf16 [B,Hq,N,D], [B,Hkv,N,D]
@@ -107,6 +107,7 @@ struct TcLaunch {
   uint32_t *status;
   int B, Hq, Hkv, N, window, k_vert, kpad, nblk_r;
   float scale;
+  bool f8;                           // low part in FP8 E4M3 (kind::f8f6f4) instead of INT8
 };
 bool prefill_tc_supported(int D, int Hq, int Hkv);
 cudaError_t launch_prefill_tc(const TcLaunch &p, cudaStream_t s);
@@ -114,8 +115,8 @@ cudaError_t launch_prefill_tc(const TcLaunch &p, cudaStream_t s);
 size_t prefill_ws_bytes(int B, int Hq, int Hkv, int N, int D, int k_vert);
 cudaError_t launch_prefill(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
                            const __nv_bfloat16 *v, const int32_t *idx, int B, int Hq, int Hkv,
-                           int N, int D, int window, int k_vert, float scale, float *out,
-                           uint8_t *ws, uint32_t *status, cudaStream_t s);
+                           int N, int D, int window, int k_vert, float scale, int low_fmt,
+                           float *out, uint8_t *ws, uint32_t *status, cudaStream_t s);
 
 // ---------------------------------------------------------------------------
 // Small device helpers.
@@ -161,6 +162,29 @@ __device__ __forceinline__ int warp_count_below(const int32_t *__restrict__ a, i
   const bool in = lane < hi - lo;
   const unsigned below = __ballot_sync(0xffffffffu, in && __ldg(a + lo + (in ? lane : 0)) < x);
   return lo + __popc(below);
+}
+
+// The double d rounded to fp32 toward zero, with the last bit set when that
+// dropped anything (round to odd).  Rounding this to a format with far fewer
+// bits (E4M3 keeps 4) gives the same result as rounding d itself.
+__device__ __forceinline__ float f32_round_odd(double d) {
+  const float r = __double2float_rz(d);
+  return (double)r == d ? r : __uint_as_float(__float_as_uint(r) | 1u);
+}
+
+// True when an fp32 estimate q (relative error a few units of 2^-24) of a
+// quotient lies so close to a point halfway between two E4M3 neighbours that
+// the exact quotient might round the other way.  Normal range: the 20 bits
+// below the 3-bit mantissa within 16 units of the halfway pattern; subnormal
+// range (|q| < 2^-6, spacing 2^-9): the fraction of q * 2^9 within 2^-12 of 1/2.
+__device__ __forceinline__ bool e4m3_near_tie(float q) {
+  const float a = fabsf(q);
+  if (a >= 0.015625f) {
+    const uint32_t low = __float_as_uint(a) & 0xFFFFFu;
+    return low >= 0x80000u - 16u && low <= 0x80000u + 16u;
+  }
+  const float t = a * 512.f;
+  return fabsf(t - floorf(t) - 0.5f) < 1.f / 4096.f;
 }
 
 }  // namespace hq

@@ -105,29 +105,6 @@ __device__ __forceinline__ void quant_store(const uint32_t (&w)[D / 64], uint8_t
   if (lane % LPG == 0) sz_row[lane / LPG] = __halves2half2(hs, hz);
 }
 
-// The double d rounded to fp32 toward zero, with the last bit set when that
-// dropped anything (round to odd).  Rounding this to a format with far fewer
-// bits (E4M3 keeps 4) gives the same result as rounding d itself.
-__device__ __forceinline__ float f32_round_odd(double d) {
-  const float r = __double2float_rz(d);
-  return (double)r == d ? r : __uint_as_float(__float_as_uint(r) | 1u);
-}
-
-// True when an fp32 estimate q (relative error a few units of 2^-24) of a
-// quotient lies so close to a point halfway between two E4M3 neighbours that
-// the exact quotient might round the other way.  Normal range: the 20 bits
-// below the 3-bit mantissa within 16 units of the halfway pattern; subnormal
-// range (|q| < 2^-6, spacing 2^-9): the fraction of q * 2^9 within 2^-12 of 1/2.
-__device__ __forceinline__ bool e4m3_near_tie(float q) {
-  const float a = fabsf(q);
-  if (a >= 0.015625f) {
-    const uint32_t low = __float_as_uint(a) & 0xFFFFFu;
-    return low >= 0x80000u - 16u && low <= 0x80000u + 16u;
-  }
-  const float t = a * 512.f;
-  return fabsf(t - floorf(t) - 0.5f) < 1.f / 4096.f;
-}
-
 // FP8 format: per group of 32 channels s = fp16(amax / 448) (the quotient
 // rounded once: scale_f16 with range amax - 0), c = E4M3(x / s) rounded to
 // nearest even and saturated, z = 0.  The hardware conversion (nearest even,

@@ -25,6 +25,8 @@
 #include <float.h>
 #include <limits.h>
 
+#include <cuda_fp8.h>
+
 #include "hq_internal.cuh"
 #include "warp_mma.cuh"
 
@@ -49,13 +51,25 @@ __device__ __forceinline__ float rint_div(float x, float s, float rcp_s) {
   return fabsf(q - t) > 0.5f - 1.f / 4096.f ? rintf(__fdiv_rn(x, s)) : t;
 }
 
+// FP8 low part: E4M3 codes of fl32(x0 / s), fl32(x1 / s) (nearest even,
+// saturating), low byte first.  The paired hardware conversion rounds the
+// reciprocal products, which lie within two units of the binary32 quotients;
+// where one is near an E4M3 tie the quotient itself is taken.
+__device__ __forceinline__ uint32_t f8_pair_div(float x0, float x1, float s, float rcp) {
+  float q0 = x0 * rcp, q1 = x1 * rcp;
+  if (e4m3_near_tie(q0)) q0 = __fdiv_rn(x0, s);
+  if (e4m3_near_tie(q1)) q1 = __fdiv_rn(x1, s);
+  return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(q0, q1), __NV_SATFINITE, __NV_E4M3);
+}
+
 // Q rows: s = amax / 127, code = clamp(rne(x / s), -127, 127), both
 // divisions single IEEE binary32 roundings.  Each lane takes one 32-channel
 // group of a row (D / 32 lanes per row, two or one shuffles for the row's
 // maximum), a warp QPASS passes of 32 / (D / 32) rows with every load issued
 // first; codes leave in 16-byte stores.
 constexpr int QPASS = 2;
-template <int D>
+// With F8 the codes are E4M3 of fl32(x / s), s = amax / 448 (f8_pair_div).
+template <int D, bool F8>
 __global__ void __launch_bounds__(256)
 quant_q_rows(const __nv_bfloat16 *__restrict__ q, long long nrows, int8_t *__restrict__ qi8,
              float *__restrict__ sq) {
@@ -93,18 +107,24 @@ quant_q_rows(const __nv_bfloat16 *__restrict__ q, long long nrows, int8_t *__res
 #pragma unroll
     for (int o = NG / 2; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     if (row >= nrows) continue;
-    const float s = amax == 0.f ? 1.f : __fdiv_rn(amax, 127.f);
+    const float s = amax == 0.f ? 1.f : __fdiv_rn(amax, F8 ? 448.f : 127.f);
     const float rcp = __frcp_rn(s);
     uint32_t out[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       uint32_t packed = 0;
+      if (F8) {
+        const uint32_t a0 = w[pi][2 * k], a1 = w[pi][2 * k + 1];
+        packed = f8_pair_div(bf16_lo(a0), bf16_hi(a0), s, rcp) |
+                 (f8_pair_div(bf16_lo(a1), bf16_hi(a1), s, rcp) << 16);
+      } else {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const uint32_t word = w[pi][2 * k + (e >> 1)];
-        const float x = (e & 1) ? bf16_hi(word) : bf16_lo(word);
-        const float c = fminf(fmaxf(rint_div(x, s, rcp), -127.f), 127.f);
-        packed |= ((uint32_t)(int)c & 0xffu) << (8 * e);
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t word = w[pi][2 * k + (e >> 1)];
+          const float x = (e & 1) ? bf16_hi(word) : bf16_lo(word);
+          const float c = fminf(fmaxf(rint_div(x, s, rcp), -127.f), 127.f);
+          packed |= ((uint32_t)(int)c & 0xffu) << (8 * e);
+        }
       }
       out[k] = packed;
     }
@@ -131,7 +151,7 @@ __device__ __forceinline__ int remaining_pos(const int32_t *id, int k_vert, int 
 // (b, kv head): INT8 codes with one symmetric scale per block.  The block's
 // rows are read once, 16 bytes per load, and held in registers for both the
 // maximum and the codes.
-template <int D>
+template <int D, bool F8>
 __global__ void __launch_bounds__(256)
 quant_k_remaining(const __nv_bfloat16 *__restrict__ k, const int32_t *__restrict__ idx, int N,
                   int k_vert, int nblk, int8_t *__restrict__ ki8, float *__restrict__ sk) {
@@ -168,7 +188,7 @@ quant_k_remaining(const __nv_bfloat16 *__restrict__ k, const int32_t *__restrict
   amax = red[0];
 #pragma unroll
   for (int w = 1; w < 8; ++w) amax = fmaxf(amax, red[w]);
-  const float s = amax == 0.f ? 1.f : __fdiv_rn(amax, 127.f);
+  const float s = amax == 0.f ? 1.f : __fdiv_rn(amax, F8 ? 448.f : 127.f);
   const float rcp = __frcp_rn(s);
   uint2 *dst = reinterpret_cast<uint2 *>(ki8 + ((size_t)bh * nr + c0) * D);   // 8 codes per piece
 #pragma unroll
@@ -180,12 +200,18 @@ quant_k_remaining(const __nv_bfloat16 *__restrict__ k, const int32_t *__restrict
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       uint32_t packed = 0;
+      if (F8) {
+        const uint32_t a0 = ww[2 * h], a1 = ww[2 * h + 1];
+        packed = f8_pair_div(bf16_lo(a0), bf16_hi(a0), s, rcp) |
+                 (f8_pair_div(bf16_lo(a1), bf16_hi(a1), s, rcp) << 16);
+      } else {
 #pragma unroll
-      for (int e4 = 0; e4 < 4; ++e4) {
-        const uint32_t word = ww[2 * h + (e4 >> 1)];
-        const float x = (e4 & 1) ? bf16_hi(word) : bf16_lo(word);
-        const float c = fminf(fmaxf(rint_div(x, s, rcp), -127.f), 127.f);
-        packed |= ((uint32_t)(int)c & 0xffu) << (8 * e4);
+        for (int e4 = 0; e4 < 4; ++e4) {
+          const uint32_t word = ww[2 * h + (e4 >> 1)];
+          const float x = (e4 & 1) ? bf16_hi(word) : bf16_lo(word);
+          const float c = fminf(fmaxf(rint_div(x, s, rcp), -127.f), 127.f);
+          packed |= ((uint32_t)(int)c & 0xffu) << (8 * e4);
+        }
       }
       out[h] = packed;
     }
@@ -603,29 +629,33 @@ PrefillWs carve(uint8_t *base, int B, int Hq, int Hkv, int N, int D, int k_vert)
   return w;
 }
 
-template <int D>
+template <int D, bool F8>
 cudaError_t quant_t(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const int32_t *idx, int B,
                     int Hq, int Hkv, int N, int k_vert, int8_t *qi8, float *sq, int8_t *ki8,
                     float *sk, cudaStream_t s) {
   const long long nrows = (long long)B * Hq * N;
   const long long rows_per_block = 8LL * (32 / (D / 32)) * QPASS;        // 8 warps
-  quant_q_rows<D><<<(unsigned)((nrows + rows_per_block - 1) / rows_per_block), 256, 0, s>>>(q, nrows, qi8, sq);
+  quant_q_rows<D, F8><<<(unsigned)((nrows + rows_per_block - 1) / rows_per_block), 256, 0, s>>>(q, nrows, qi8, sq);
   const int nblk_r = (N - k_vert + TILE - 1) / TILE;
   if (nblk_r > 0)
-    quant_k_remaining<D><<<dim3(nblk_r, B * Hkv), 256, 0, s>>>(k, idx, N, k_vert, nblk_r, ki8, sk);
+    quant_k_remaining<D, F8><<<dim3(nblk_r, B * Hkv), 256, 0, s>>>(k, idx, N, k_vert, nblk_r, ki8, sk);
   return cudaGetLastError();
 }
 
 template <int D>
 cudaError_t prefill_t(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
                       const int32_t *idx, int B, int Hq, int Hkv, int N, int window, int k_vert,
-                      float scale, float *out, uint8_t *ws, uint32_t *status, cudaStream_t s) {
+                      float scale, int low_fmt, float *out, uint8_t *ws, uint32_t *status,
+                      cudaStream_t s) {
+  const bool f8 = low_fmt == HQ_KV_FP8;
+  if (f8 && !prefill_tc_supported(D, Hq, Hkv)) return cudaErrorNotSupported;   // FP8: tcgen05 path only
   PrefillWs w = carve(ws, B, Hq, Hkv, N, D, k_vert);
   const int nbh = B * Hkv;
   const int nr = N - k_vert;
   const int nblk_r = (nr + TILE - 1) / TILE;
   const int kpad = (k_vert + 127) / 128 * 128;
-  cudaError_t e = quant_t<D>(q, k, idx, B, Hq, Hkv, N, k_vert, w.qi8, w.sq, w.ki8, w.sk, s);
+  cudaError_t e = f8 ? quant_t<D, true>(q, k, idx, B, Hq, Hkv, N, k_vert, w.qi8, w.sq, w.ki8, w.sk, s)
+                     : quant_t<D, false>(q, k, idx, B, Hq, Hkv, N, k_vert, w.qi8, w.sq, w.ki8, w.sk, s);
   if (e != cudaSuccess) return e;
   {
     const long long blocks = (long long)nbh * ((N + VSPAN - 1) / VSPAN);   // one CTA per span
@@ -658,6 +688,7 @@ cudaError_t prefill_t(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
     p.kpad = kpad;
     p.nblk_r = nblk_r;
     p.scale = scale;
+    p.f8 = f8;
     return launch_prefill_tc(p, s);
   }
   PrefillArgs a;
@@ -691,10 +722,13 @@ cudaError_t prefill_t(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
 
 cudaError_t launch_prefill_quant(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
                                  const int32_t *idx, int B, int Hq, int Hkv, int N, int D,
-                                 int k_vert, int8_t *qi8, float *sq, int8_t *ki8, float *sk,
-                                 cudaStream_t s) {
-  if (D == 128) return quant_t<128>(q, k, idx, B, Hq, Hkv, N, k_vert, qi8, sq, ki8, sk, s);
-  if (D == 64) return quant_t<64>(q, k, idx, B, Hq, Hkv, N, k_vert, qi8, sq, ki8, sk, s);
+                                 int k_vert, int low_fmt, int8_t *qi8, float *sq, int8_t *ki8,
+                                 float *sk, cudaStream_t s) {
+  const bool f8 = low_fmt == HQ_KV_FP8;
+  if (D == 128 && !f8) return quant_t<128, false>(q, k, idx, B, Hq, Hkv, N, k_vert, qi8, sq, ki8, sk, s);
+  if (D == 64 && !f8) return quant_t<64, false>(q, k, idx, B, Hq, Hkv, N, k_vert, qi8, sq, ki8, sk, s);
+  if (D == 128 && f8) return quant_t<128, true>(q, k, idx, B, Hq, Hkv, N, k_vert, qi8, sq, ki8, sk, s);
+  if (D == 64 && f8) return quant_t<64, true>(q, k, idx, B, Hq, Hkv, N, k_vert, qi8, sq, ki8, sk, s);
   return cudaErrorInvalidValue;
 }
 
@@ -704,10 +738,10 @@ size_t prefill_ws_bytes(int B, int Hq, int Hkv, int N, int D, int k_vert) {
 
 cudaError_t launch_prefill(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
                            const __nv_bfloat16 *v, const int32_t *idx, int B, int Hq, int Hkv,
-                           int N, int D, int window, int k_vert, float scale, float *out,
-                           uint8_t *ws, uint32_t *status, cudaStream_t s) {
-  if (D == 128) return prefill_t<128>(q, k, v, idx, B, Hq, Hkv, N, window, k_vert, scale, out, ws, status, s);
-  if (D == 64) return prefill_t<64>(q, k, v, idx, B, Hq, Hkv, N, window, k_vert, scale, out, ws, status, s);
+                           int N, int D, int window, int k_vert, float scale, int low_fmt,
+                           float *out, uint8_t *ws, uint32_t *status, cudaStream_t s) {
+  if (D == 128) return prefill_t<128>(q, k, v, idx, B, Hq, Hkv, N, window, k_vert, scale, low_fmt, out, ws, status, s);
+  if (D == 64) return prefill_t<64>(q, k, v, idx, B, Hq, Hkv, N, window, k_vert, scale, low_fmt, out, ws, status, s);
   return cudaErrorInvalidValue;
 }
 

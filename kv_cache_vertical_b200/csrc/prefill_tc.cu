@@ -14,19 +14,23 @@
 // loaded once feeds both.  Warp roles:
 //   warp 0      TMA producer: the four Q tiles once, then a 2-stage ring of
 //               (K tile, V tile) pairs;
-//   warp 1      allocates 512 TMEM columns; lane 0 issues every MMA:
+//   warp 1      allocates 512 TMEM columns; lane 0 issues head A's MMAs,
+//   warp 2      lane 0 issues head B's MMAs:
 //               S_X = Q_X K^T (kind::i8 into s32, or kind::f16 bf16 into f32)
 //               and O_X += P_X V (kind::f16, P read from tensor memory, in
 //               32-key chunks as the softmax hands them over);
-//   warps 2-3   idle (they keep the softmax warpgroups aligned to TMEM lanes);
+//   warp 3      idle (warps 0-3 keep the softmax warpgroups aligned to TMEM lanes);
 //   warps 4-7   softmax of head A, warps 8-11 softmax of head B: one thread per
 //               query row (TMEM lane), so row max / sum need no shuffles.
 // TMEM: S_A [0,128) (P_A aliases its first 64 columns as packed fp16 pairs),
 // O_A [128,256), S_B [256,384), O_B [384,512).
-// The MMA thread alternates the heads (PV_A(t), QK_A(t+1), PV_B(t), QK_B(t+1)),
-// so one head's softmax overlaps the other head's tensor-core work.
+// Each issuer runs PV_X(t), QK_X(t+1), ...; QK_X(t+1) waits for PV_X(t) to
+// complete, since it overwrites P_X.  While one head waits or runs its
+// softmax the other head's tensor-core work proceeds.
+// Low-bit tiles are INT8 (kind::i8, s32 scores) or FP8 E4M3 (kind::f8f6f4,
+// fp32 scores), one format per launch.
 // Key tiles per query tile, each its own iteration of the online softmax:
-//   INT8 tiles  128 consecutive REMAINING (non-vertical) keys, compacted in
+//   low tiles   128 consecutive REMAINING (non-vertical) keys, compacted in
 //               position order by the pre-pass: keep the keys at positions
 //               <= i - W (a prefix of the compact order, so only the last
 //               tiles need a per-row bound and no tile needs a vertical mask);
@@ -65,6 +69,7 @@ constexpr uint32_t kMagicBits = 0x4B400000u;    // bits of kMagic
 constexpr uint32_t IDESC_I8 = make_idesc(2, 1, 1, 0, 0, 128, 128);   // s32 <- s8 x s8
 constexpr uint32_t IDESC_BF = make_idesc(1, 1, 1, 0, 0, 128, 128);   // f32 <- bf16 x bf16
 constexpr uint32_t IDESC_PV = make_idesc(1, 0, 0, 0, 1, 128, 128);   // f32 <- f16 x f16 (V MN-major)
+constexpr uint32_t IDESC_F8 = make_idesc(1, 0, 0, 0, 0, 128, 128);   // f32 <- e4m3 x e4m3
 
 enum { IT_I8 = 0, IT_WIN = 1, IT_VERT = 2 };
 
@@ -166,6 +171,7 @@ __device__ __forceinline__ Sched make_sched(const TcArgs &a, int i0, size_t bh) 
   return s;
 }
 
+template <bool F8>
 __global__ void __launch_bounds__(NTHR, 1)
 prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ CUtensorMap tm_qbf,
            const __grid_constant__ CUtensorMap tm_ki8, const __grid_constant__ CUtensorMap tm_kbf,
@@ -183,6 +189,7 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
   uint64_t *o_final = bar + 15;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 16);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(bar + 17);
+  uint64_t *pv_done = bar + 18;  // [2 heads]: P.V of the head's current tile has completed
 
   const int ntq = (a.N + BM - 1) / BM;
   const int qt = ntq - 1 - (int)blockIdx.x;      // longest rows first
@@ -199,11 +206,13 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
     mbar_init(q_full, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_free[s], 1);
+      mbar_init(&kv_free[s], F8 ? 2 : 1);   // one arrival per MMA issuer
       mbar_init(&s_full[s], 1);
     }
     for (int s = 0; s < 2 * NCHUNK; ++s) mbar_init(&p_full[s], 4);
-    mbar_init(o_final, 1);
+    mbar_init(o_final, F8 ? 2 : 1);
+    mbar_init(&pv_done[0], 1);
+    mbar_init(&pv_done[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -262,12 +271,91 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
       for (int it = issued > 2 ? issued - 2 : 0; it < issued; ++it)
         if (!mbar_wait(&kv_full[it & 1], (it >> 1) & 1)) raise_status(a.status, HQ_DEV_TIMEOUT);
     }
-  } else if (warp == 1) {
-    // ------------------------------ MMA issuer ------------------------------
+  } else if (F8 && (warp == 1 || warp == 2)) {
+    // ------------------ MMA issuers, FP8 low tiles, one per head ------------------
+    // Warp 1 issues head A's MMAs, warp 2 head B's, each in order per tile t:
+    // P.V(t) chunk by chunk as the softmax hands the chunks over, then QK(t+1).
+    // QK(t+1) writes the TMEM columns that P.V(t) reads P from, and issue order
+    // orders two MMAs only when they share the accumulator (O and S do not), so
+    // QK(t+1) waits until P.V(t) has completed.  With one issuing thread per
+    // head that wait holds up only its own head: the other head's MMAs and
+    // softmax go on meanwhile.  (Measured on B200: kind::f8f6f4 QK issued
+    // right behind the P.V, as the INT8 issuer does, gives wrong scores.)
+    if (lane == 0) {
+      const int x = warp - 1;
+      const uint32_t sQi8 = smem_u32(smem + SM_QI8), sQbf = smem_u32(smem + SM_QBF);
+      const uint32_t sKV = smem_u32(smem + SM_KV);
+      bool ok = mbar_wait(q_full, 0);
+      auto issue_qk = [&](int it) {
+        const uint32_t kslot = sKV + (it & 1) * KV_STAGE;
+        const uint32_t dt = tmem + x * 256;
+        if (sc.type(it) == IT_I8) {
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t ad = make_sdesc_sw128(sQi8 + x * 16384 + ks * 32, 16, 1024);
+            const uint64_t bd = make_sdesc_sw128(kslot + ks * 32, 16, 1024);
+            mma_f8_ss(dt, ad, bd, IDESC_F8, ks > 0);
+          }
+        } else {
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+            const uint64_t ad = make_sdesc_sw128(sQbf + x * 32768 + off, 16, 1024);
+            const uint64_t bd = make_sdesc_sw128(kslot + off, 16, 1024);
+            mma_f16_ss(dt, ad, bd, IDESC_BF, ks > 0);
+          }
+        }
+        tc_commit(&s_full[x]);
+      };
+      if (ok && sc.n > 0) {
+        ok = mbar_wait(&kv_full[0], 0);
+        if (ok) {
+          tc_fence_after();
+          issue_qk(0);
+        }
+      }
+      for (int it = 0; ok && it < sc.n; ++it) {
+        const uint32_t vslot = sKV + (it & 1) * KV_STAGE + 32768;
+        const uint32_t dt = tmem + x * 256 + 128, at = tmem + x * 256;
+#pragma unroll
+        for (int c = 0; c < NCHUNK; ++c) {
+          if (!(ok = mbar_wait(&p_full[x * NCHUNK + c], it & 1))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int ks = 2 * c + j;
+            const uint64_t bd = make_sdesc_sw128(vslot + ks * 2048, 16384, 1024);
+            mma_f16_ts(dt, at + ks * 8, bd, IDESC_PV, (it > 0 || ks > 0) ? 1u : 0u);
+          }
+        }
+        if (!ok) break;
+        tc_commit(&kv_free[it & 1]);                // one of the two arrivals
+        if (it + 1 < sc.n) {
+          tc_commit(&pv_done[x]);
+          if (!(ok = mbar_wait(&kv_full[(it + 1) & 1], ((it + 1) >> 1) & 1))) break;
+          if (!(ok = mbar_wait(&pv_done[x], it & 1))) break;
+          tc_fence_after();
+          issue_qk(it + 1);
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        raise_status(a.status, HQ_DEV_TIMEOUT);
+      }
+      tc_commit(o_final);
+    }
+  } else if (!F8 && warp == 1) {
+    // ---------------------- MMA issuer, INT8 low tiles ----------------------
     // Order per tile t: P.V of head A chunk by chunk as its softmax hands the
     // chunks over, QK of head A for tile t + 1, the same for head B, so one
     // head's softmax overlaps the other head's tensor-core work and most of a
-    // head's own P.V overlaps the end of its exp phase.
+    // head's own P.V overlaps the end of its exp phase.  QK_A(t+1) overwrites
+    // the TMEM columns that P.V_A(t) reads P from and is issued without
+    // waiting for it: this relies on the tensor pipe executing one thread's
+    // MMAs in issue order, which the PTX pipelining rule states only for MMAs
+    // that share an accumulator.  Measured on B200 it holds for these
+    // kind::f16 / kind::i8 sequences (every parity case), and waiting for the
+    // P.V instead costs 20-40% of the kernel.
     if (lane == 0) {
       const uint32_t sQi8 = smem_u32(smem + SM_QI8), sQbf = smem_u32(smem + SM_QBF);
       const uint32_t sKV = smem_u32(smem + SM_KV);
@@ -400,7 +488,20 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
       tmem_ld64x2(tS, xa0, xa1);                    // the whole S row, one wait
       float sc0, sc1, c0, c1, mt;                   // per-half scale and offset (log2 units)
       uint32_t add = 0u;                            // bits added to a raw score before the FMA
-      if (ty == IT_I8) {
+      if (F8 && ty == IT_I8) {                     // fp32 scores of FP8 codes
+        sc0 = sqi * k0;
+        sc1 = sqi * k1;
+        c0 = c1 = 0.f;
+        if (j0 + BN > cnt_lo) {
+          const int nvalid = cnt_i - j0;
+#pragma unroll
+          for (int e = 0; e < 64; ++e) {
+            if (e >= nvalid) xa0[e] = kNegInfBits;
+            if (64 + e >= nvalid) xa1[e] = kNegInfBits;
+          }
+        }
+        mt = fmaxf(max64(xa0) * sc0, max64(xa1) * sc1);
+      } else if (!F8 && ty == IT_I8) {
         sc0 = sqi * k0;
         sc1 = sqi * k1;
         if (j0 + BN > cnt_lo) {                     // same for every row of the tile
@@ -520,14 +621,17 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
 // The kernel redistributes registers with setmaxnreg, which is only valid
 // when the CTA starts with exactly kRegsLaunch registers per thread; that is
 // checked once from the compiled kernel (else the CUDA-core kernel is used).
+template <bool F8>
+static bool kernel_ready() {
+  cudaFuncAttributes fa;
+  return cudaFuncGetAttributes(&fa, prefill_tc<F8>) == cudaSuccess && fa.numRegs == kRegsLaunch &&
+         cudaFuncSetAttribute(prefill_tc<F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              SMEM_BYTES) == cudaSuccess;
+}
+
 static bool prefill_tc_ready() {
   static int ready = -1;
-  if (ready < 0) {
-    cudaFuncAttributes fa;
-    ready = cudaFuncGetAttributes(&fa, prefill_tc) == cudaSuccess && fa.numRegs == kRegsLaunch &&
-            cudaFuncSetAttribute(prefill_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 SMEM_BYTES) == cudaSuccess;
-  }
+  if (ready < 0) ready = kernel_ready<false>() && kernel_ready<true>();
   return ready == 1;
 }
 
@@ -564,7 +668,10 @@ cudaError_t launch_prefill_tc(const TcLaunch &p, cudaStream_t s) {
   a.nblk_r = p.nblk_r;
   a.sl = p.scale * kLog2e;
   dim3 grid((p.N + BM - 1) / BM, p.Hq / 2, p.B);
-  prefill_tc<<<grid, NTHR, SMEM_BYTES, s>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7], a);
+  if (p.f8)
+    prefill_tc<true><<<grid, NTHR, SMEM_BYTES, s>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7], a);
+  else
+    prefill_tc<false><<<grid, NTHR, SMEM_BYTES, s>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7], a);
   return cudaGetLastError();
 }
 

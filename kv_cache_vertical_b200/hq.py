@@ -69,11 +69,15 @@ _pquant = _sig("hq_prefill_quant", _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _
 hq_prefill_workspace_size = _sig("hq_prefill_workspace_size", _SZ, _I, _I, _I, _I, _I, _I)
 _prefill = _sig("hq_prefill_attn", _I, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P,
                 _SZ, _P)
+_pquant_ex = _sig("hq_prefill_quant_ex", _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P)
+_prefill_ex = _sig("hq_prefill_attn_ex", _I, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P,
+                   _P, _SZ, _P)
 
 EXPORTED = ["hq_status_string", "hq_version", "hq_read_device_status", "hq_probe_workspace_size",
             "hq_probe_vertical", "hq_pack_kv", "hq_decode_workspace_size", "hq_decode_attn",
             "hq_prefill_quant", "hq_prefill_workspace_size", "hq_prefill_attn",
-            "hq_decode_attn_static", "hq_kv_append", "hq_decode_merge"]
+            "hq_decode_attn_static", "hq_kv_append", "hq_decode_merge", "hq_prefill_quant_ex",
+            "hq_prefill_attn_ex"]
 
 HQ_ERR_SCRATCH_LIMIT = 7
 STATIC_SCRATCH_BYTES = 8 << 20
@@ -252,6 +256,19 @@ def hq_prefill_quant(q, k, idx, B, Hq, Hkv, N, D, k_vert, qi8, sq, ki8, sk, stre
                    _ptr(ki8), _ptr(sk), _stream(stream)), "hq_prefill_quant")
 
 
+def hq_prefill_quant_ex(q, k, idx, B, Hq, Hkv, N, D, k_vert, low_fmt, qi8, sq, ki8, sk,
+                        stream=None):
+    _check(_pquant_ex(_ptr(q), _ptr(k), _ptr(idx), B, Hq, Hkv, N, D, k_vert, low_fmt, _ptr(qi8),
+                      _ptr(sq), _ptr(ki8), _ptr(sk), _stream(stream)), "hq_prefill_quant_ex")
+
+
+def hq_prefill_attn_ex(q, k, v, idx, B, Hq, Hkv, N, D, window, k_vert, softmax_scale, low_fmt,
+                       out, ws, stream=None):
+    _check(_prefill_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(idx), B, Hq, Hkv, N, D, window, k_vert,
+                       float(softmax_scale), low_fmt, _ptr(out), _ptr(ws),
+                       ws.numel() if ws is not None else 0, _stream(stream)), "hq_prefill_attn_ex")
+
+
 def hq_prefill_attn(q, k, v, idx, B, Hq, Hkv, N, D, window, k_vert, softmax_scale, out, ws,
                     stream=None):
     _check(_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(idx), B, Hq, Hkv, N, D, window, k_vert,
@@ -305,8 +322,9 @@ def decode_attn(q, cache: KVCache, Hkv, scale=0.0, ws=None, want_lse=False):
     return (out, lse) if want_lse else out
 
 
-def prefill_quant(q, k, idx):
-    """INT8 pre-pass: Q per row; K over the remaining (non-vertical) keys."""
+def prefill_quant(q, k, idx, fmt=HQ_KV_INT):
+    """Low-part pre-pass (INT8, or E4M3 code bits with fmt=HQ_KV_FP8): Q per
+    row; K over the remaining (non-vertical) keys."""
     B, Hq, N, D = q.shape
     Hkv = k.shape[1]
     k_vert = idx.shape[2]
@@ -316,11 +334,11 @@ def prefill_quant(q, k, idx):
     sq = torch.empty(B, Hq, N, dtype=torch.float32, device=q.device)
     ki8 = torch.empty(B, Hkv, nr, D, dtype=torch.int8, device=q.device)
     sk = torch.empty(B, Hkv, nblk, dtype=torch.float32, device=q.device)
-    hq_prefill_quant(q, k, idx, B, Hq, Hkv, N, D, k_vert, qi8, sq, ki8, sk)
+    hq_prefill_quant_ex(q, k, idx, B, Hq, Hkv, N, D, k_vert, fmt, qi8, sq, ki8, sk)
     return qi8, sq, ki8, sk
 
 
-def prefill_attn(q, k, v, idx, window, scale=0.0, ws=None, out=None):
+def prefill_attn(q, k, v, idx, window, scale=0.0, ws=None, out=None, fmt=HQ_KV_INT):
     B, Hq, N, D = q.shape
     Hkv = k.shape[1]
     k_vert = idx.shape[2]
@@ -328,7 +346,7 @@ def prefill_attn(q, k, v, idx, window, scale=0.0, ws=None, out=None):
         out = torch.empty(B, Hq, N, D, dtype=torch.float32, device=q.device)
     if ws is None:
         ws = workspace(hq_prefill_workspace_size(B, Hq, Hkv, N, D, k_vert), q.device)
-    hq_prefill_attn(q, k, v, idx, B, Hq, Hkv, N, D, window, k_vert, scale, out, ws)
+    hq_prefill_attn_ex(q, k, v, idx, B, Hq, Hkv, N, D, window, k_vert, scale, fmt, out, ws)
     return out
 
 

@@ -29,7 +29,7 @@ def oracle_idx(x, w: Workload):
     return oracle.topk(sc, w.window, w.k_vert), sc
 
 
-def run_prefill_case(w: Workload, rows=None, check_probe=True):
+def run_prefill_case(w: Workload, rows=None, check_probe=True, fmt=0):
     H = hq()
     x = make_inputs(w)
     d = to_dev(x)
@@ -40,13 +40,13 @@ def run_prefill_case(w: Workload, rows=None, check_probe=True):
         assert_index_sets(gidx.cpu().numpy(), ridx, rsc, w.window)
     # INT8 pre-pass: bit-exact
     idx_d = torch.from_numpy(ridx).cuda()
-    gq = [t.cpu().numpy() for t in H.prefill_quant(d["q"], d["k"], idx_d)]
-    rq = oracle.prefill_quant(x["q"], x["k"], ridx)
+    gq = [t.cpu().numpy() for t in H.prefill_quant(d["q"], d["k"], idx_d, fmt=fmt)]
+    rq = oracle.prefill_quant(x["q"], x["k"], ridx, fmt=fmt)
     for g, r, name in zip(gq, rq, ("qi8", "sq", "ki8", "sk")):
         assert np.array_equal(g, r), f"{name} differs"
-    out = H.prefill_attn(d["q"], d["k"], d["v"], idx_d, w.window)
+    out = H.prefill_attn(d["q"], d["k"], d["v"], idx_d, w.window, fmt=fmt)
     torch.cuda.synchronize()
-    ref = oracle.prefill_attn(x["q"], x["k"], x["v"], ridx, w.window, quant=rq, rows=rows)
+    ref = oracle.prefill_attn(x["q"], x["k"], x["v"], ridx, w.window, quant=rq, rows=rows, fmt=fmt)
     g = out.cpu().numpy()
     if rows is not None:
         g = g[:, :, rows]
@@ -117,3 +117,33 @@ def test_prefill_reports_bad_index_lists():
         H.prefill_attn(d["q"], d["k"], d["v"], torch.from_numpy(bad).cuda(), w.window, ws=ws)
         assert H.hq_read_device_status(ws, clear=True) & H.HQ_DEV_BAD_INDEX
         assert H.hq_read_device_status(ws) == 0
+
+
+# --------------------------------------------------------------------------
+# FP8 (E4M3) low part, tcgen05 kind::f8f6f4
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("G", [2, 4, 8])
+def test_prefill_fp8_small_ragged(G):
+    w = Workload("p_fp8", "prefill", 1, 2 * G, 2, 128, 777, 64, F5, 4, 300 + G)
+    run_prefill_case(w, fmt=1)
+
+
+def test_prefill_fp8_medium_all_rows():
+    w = Workload("p_fp8_med", "prefill", 2, 8, 2, 128, 2100, 128, F5, 4, 71)
+    run_prefill_case(w, fmt=1)
+
+
+def test_prefill_fp8_full_size_sampled_rows():
+    w = WORKLOADS["llama8b_prefill_32k"]
+    rows = np.array([0, 1, 127, 128, 4095, 16385, 32000, w.L - 1], np.int32)
+    run_prefill_case(w, rows=rows, check_probe=False, fmt=1)
+
+
+def test_prefill_fp8_rejected_off_the_tensor_core_path():
+    H = hq()
+    w = Workload("p_fp8_d64", "prefill", 1, 2, 1, 64, 256, 32, F5, 4, 1)
+    d = to_dev(make_inputs(w))
+    idx = torch.zeros(1, 1, 0, dtype=torch.int32, device="cuda")
+    with pytest.raises(H.HQError):
+        H.prefill_attn(d["q"], d["k"], d["v"], idx, w.window, fmt=1)
