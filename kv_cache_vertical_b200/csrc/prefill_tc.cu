@@ -12,25 +12,25 @@
 // One CTA per (128-query tile, pair of query heads that share a KV head): the
 // two heads ("A" and "B") see exactly the same key tiles, so every K / V tile
 // loaded once feeds both.  Warp roles:
-//   warp 0      TMA producer: the four Q tiles once, then a 2-stage ring of
+//   warp 0      TMA producer: the four Q tiles once, then a 4-stage ring of
 //               (K tile, V tile) pairs;
 //   warp 1      allocates 512 TMEM columns; lane 0 issues head A's MMAs,
 //   warp 2      lane 0 issues head B's MMAs:
-//               S_X = Q_X K^T (kind::i8 into s32, or kind::f16 bf16 into f32)
-//               and O_X += P_X V (kind::f16, P read from tensor memory, in
-//               32-key chunks as the softmax hands them over);
+//               S_X = Q_X K^T (kind::i8 into s32, kind::f8f6f4 into f32, or
+//               kind::f16 bf16 into f32) and O_X += P_X V (kind::f16, P read
+//               from tensor memory, in 32-key chunks as the softmax hands
+//               them over);
 //   warp 3      idle (warps 0-3 keep the softmax warpgroups aligned to TMEM lanes);
 //   warps 4-7   softmax of head A, warps 8-11 softmax of head B: one thread per
 //               query row (TMEM lane), so row max / sum need no shuffles.
-// TMEM: S_A [0,128) (P_A aliases its first 64 columns as packed fp16 pairs),
-// O_A [128,256), S_B [256,384), O_B [384,512).
-// Each issuer runs PV_X(t), QK_X(t+1), ...; QK_X(t+1) waits for PV_X(t) to
-// complete, since it overwrites P_X.  While one head waits or runs its
-// softmax the other head's tensor-core work proceeds.
+// Key tiles are 64 keys wide.  TMEM per head X (256 columns): two S buffers
+// of 64 columns, S(t) in buffer t & 1 (P(t), packed fp16 pairs, overwrites the
+// first 32 columns of its buffer), then O_X in the upper 128.  With S double
+// buffered, the QK of the next tile runs while the softmax works on this one.
 // Low-bit tiles are INT8 (kind::i8, s32 scores) or FP8 E4M3 (kind::f8f6f4,
-// fp32 scores), one format per launch.
+// fp32 scores), one format per instantiation.
 // Key tiles per query tile, each its own iteration of the online softmax:
-//   low tiles   128 consecutive REMAINING (non-vertical) keys, compacted in
+//   low tiles   64 consecutive REMAINING (non-vertical) keys, compacted in
 //               position order by the pre-pass: keep the keys at positions
 //               <= i - W (a prefix of the compact order, so only the last
 //               tiles need a per-row bound and no tile needs a vertical mask);
@@ -49,27 +49,29 @@
 namespace hq {
 namespace {
 
-constexpr int BM = 128, BN = 128, D = 128;
+constexpr int BM = 128, BN = 64, D = 128;
 constexpr int NWARPS = 12, NTHR = NWARPS * 32;
 constexpr int SM_WARP0 = 4;                     // warps 4-7: head A, 8-11: head B
 constexpr int kRegsLaunch = 168;                // 65536 / 384, what a 384-thread CTA starts with
 constexpr int kRegsLow = 56, kRegsHigh = 224;   // 128 * 56 + 256 * 224 == 384 * 168
-constexpr int NCHUNK = 4;                       // P handed to the MMA in 32-key chunks
+constexpr int NCHUNK = 2;                       // P handed to the MMA in 32-key chunks
+constexpr int NST = 4;                          // K/V stages
 constexpr uint32_t SM_QI8 = 0;                 // [2 heads][128 rows x 128 B]
 constexpr uint32_t SM_QBF = 32768;             // [2 heads][2 boxes][128 rows x 128 B]
-constexpr uint32_t SM_KV = 98304;              // [2 stages][K 32 KB | V 32 KB]
-constexpr uint32_t KV_STAGE = 65536;
-constexpr uint32_t SM_BAR = SM_KV + 2 * KV_STAGE;
+constexpr uint32_t SM_KV = 98304;              // [NST stages][K 16 KB | V 16 KB]
+constexpr uint32_t KV_STAGE = 32768;
+constexpr uint32_t KV_VOFF = 16384;            // V within a stage; K and V boxes are 8 KB
+constexpr uint32_t SM_BAR = SM_KV + NST * KV_STAGE;
 constexpr uint32_t SMEM_BYTES = SM_BAR + 256 + 1024;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLazy = 8.0f;                   // rescale O only when the max grows by > 2^8
 constexpr float kMagic = 12582912.0f;           // 2^23 + 2^22
 constexpr uint32_t kMagicBits = 0x4B400000u;    // bits of kMagic
 
-constexpr uint32_t IDESC_I8 = make_idesc(2, 1, 1, 0, 0, 128, 128);   // s32 <- s8 x s8
-constexpr uint32_t IDESC_BF = make_idesc(1, 1, 1, 0, 0, 128, 128);   // f32 <- bf16 x bf16
-constexpr uint32_t IDESC_PV = make_idesc(1, 0, 0, 0, 1, 128, 128);   // f32 <- f16 x f16 (V MN-major)
-constexpr uint32_t IDESC_F8 = make_idesc(1, 0, 0, 0, 0, 128, 128);   // f32 <- e4m3 x e4m3
+constexpr uint32_t IDESC_I8 = make_idesc(2, 1, 1, 0, 0, BM, BN);     // s32 <- s8 x s8
+constexpr uint32_t IDESC_BF = make_idesc(1, 1, 1, 0, 0, BM, BN);     // f32 <- bf16 x bf16
+constexpr uint32_t IDESC_F8 = make_idesc(1, 0, 0, 0, 0, BM, BN);     // f32 <- e4m3 x e4m3
+constexpr uint32_t IDESC_PV = make_idesc(1, 0, 0, 0, 1, BM, D);      // f32 <- f16 x f16 (V MN-major)
 
 enum { IT_I8 = 0, IT_WIN = 1, IT_VERT = 2 };
 
@@ -182,14 +184,14 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bar = reinterpret_cast<uint64_t *>(smem + SM_BAR);
   uint64_t *q_full = bar;
-  uint64_t *kv_full = bar + 1;   // [2]
-  uint64_t *kv_free = bar + 3;   // [2]
-  uint64_t *s_full = bar + 5;    // [2 heads]
-  uint64_t *p_full = bar + 7;    // [2 heads][NCHUNK], one arrival per softmax warp
-  uint64_t *o_final = bar + 15;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 16);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(bar + 17);
-  uint64_t *pv_done = bar + 18;  // [2 heads]: P.V of the head's current tile has completed
+  uint64_t *kv_full = bar + 1;   // [NST]
+  uint64_t *kv_free = bar + 5;   // [NST], one arrival per MMA issuer
+  uint64_t *s_full = bar + 9;    // [2 heads][2 S buffers]
+  uint64_t *p_full = bar + 13;   // [2 heads][2 S buffers][NCHUNK], one arrival per softmax warp
+  uint64_t *pv_done = bar + 21;  // [2 heads]: the head's P.V of its latest tile has completed
+  uint64_t *o_final = bar + 23;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 24);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(bar + 25);
 
   const int ntq = (a.N + BM - 1) / BM;
   const int qt = ntq - 1 - (int)blockIdx.x;      // longest rows first
@@ -204,15 +206,15 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < NST; ++s) {
       mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_free[s], F8 ? 2 : 1);   // one arrival per MMA issuer
-      mbar_init(&s_full[s], 1);
+      mbar_init(&kv_free[s], 2);
     }
-    for (int s = 0; s < 2 * NCHUNK; ++s) mbar_init(&p_full[s], 4);
-    mbar_init(o_final, F8 ? 2 : 1);
+    for (int s = 0; s < 4; ++s) mbar_init(&s_full[s], 1);
+    for (int s = 0; s < 4 * NCHUNK; ++s) mbar_init(&p_full[s], 4);
     mbar_init(&pv_done[0], 1);
     mbar_init(&pv_done[1], 1);
+    mbar_init(o_final, 2);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -241,181 +243,105 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
       tma_load_3d(smem + SM_QBF + 49152, &tm_qbf, q_full, 64, i0, bqB);
       int issued = 0;
       for (int it = 0; it < sc.n; ++it) {
-        const int s = it & 1;
-        if (it >= 2 && !mbar_wait(&kv_free[s], ((it >> 1) & 1) ^ 1)) {
+        const int s = it % NST;
+        if (it >= NST && !mbar_wait(&kv_free[s], ((it / NST) & 1) ^ 1)) {
           *abort_flag = 1;
           raise_status(a.status, HQ_DEV_TIMEOUT);
           break;
         }
         if (*abort_flag) break;
         uint8_t *ks = smem + SM_KV + s * KV_STAGE;
-        uint8_t *vs = ks + 32768;
+        uint8_t *vs = ks + KV_VOFF;
         const int ty = sc.type(it), t = sc.tile(it);
         const int row = t * BN;
         if (ty == IT_I8) {
-          mbar_arrive_expect_tx(&kv_full[s], 16384 + 32768);
+          mbar_arrive_expect_tx(&kv_full[s], BN * 128 + BN * 256);
           tma_load_3d(ks, &tm_ki8, &kv_full[s], 0, row, (int)bh);
         } else {
-          mbar_arrive_expect_tx(&kv_full[s], 65536);
+          mbar_arrive_expect_tx(&kv_full[s], 2 * BN * 256);
           const CUtensorMap *km = ty == IT_WIN ? &tm_kbf : &tm_vk;
           tma_load_3d(ks, km, &kv_full[s], 0, row, (int)bh);
-          tma_load_3d(ks + 16384, km, &kv_full[s], 64, row, (int)bh);
+          tma_load_3d(ks + BN * 128, km, &kv_full[s], 64, row, (int)bh);
         }
         const CUtensorMap *vm = ty == IT_VERT ? &tm_vv : (ty == IT_I8 ? &tm_vc : &tm_v16);
         tma_load_3d(vs, vm, &kv_full[s], 0, row, (int)bh);
-        tma_load_3d(vs + 16384, vm, &kv_full[s], 64, row, (int)bh);
+        tma_load_3d(vs + BN * 128, vm, &kv_full[s], 64, row, (int)bh);
         issued = it + 1;
       }
       // do not leave with copies in flight
       if (!mbar_wait(q_full, 0)) raise_status(a.status, HQ_DEV_TIMEOUT);
-      for (int it = issued > 2 ? issued - 2 : 0; it < issued; ++it)
-        if (!mbar_wait(&kv_full[it & 1], (it >> 1) & 1)) raise_status(a.status, HQ_DEV_TIMEOUT);
+      for (int it = issued > NST ? issued - NST : 0; it < issued; ++it)
+        if (!mbar_wait(&kv_full[it % NST], (it / NST) & 1)) raise_status(a.status, HQ_DEV_TIMEOUT);
     }
-  } else if (F8 && (warp == 1 || warp == 2)) {
-    // ------------------ MMA issuers, FP8 low tiles, one per head ------------------
-    // Warp 1 issues head A's MMAs, warp 2 head B's, each in order per tile t:
-    // P.V(t) chunk by chunk as the softmax hands the chunks over, then QK(t+1).
-    // QK(t+1) writes the TMEM columns that P.V(t) reads P from, and issue order
-    // orders two MMAs only when they share the accumulator (O and S do not), so
-    // QK(t+1) waits until P.V(t) has completed.  With one issuing thread per
-    // head that wait holds up only its own head: the other head's MMAs and
-    // softmax go on meanwhile.  (Measured on B200: kind::f8f6f4 QK issued
-    // right behind the P.V, as the INT8 issuer does, gives wrong scores.)
+  } else if (warp == 1 || warp == 2) {
+    // ---------------------- MMA issuers, one per head ----------------------
+    // Warp 1 issues head A's MMAs, warp 2 head B's.  S is double-buffered in
+    // TMEM, so QK(t+1) runs while the softmax works on S(t); per tile t the
+    // issuer hands P(t).V(t) to the tensor core chunk by chunk as the softmax
+    // releases the chunks, then issues QK(t+2) into the buffer of S(t).  P(t)
+    // lives in that buffer and the PTX pipelining rule orders two MMAs only
+    // when they share the accumulator, so QK(t+2) waits for P(t).V(t) to
+    // complete -- by then the softmax of tile t+1 is under way, so the wait
+    // costs the softmax nothing.
     if (lane == 0) {
       const int x = warp - 1;
       const uint32_t sQi8 = smem_u32(smem + SM_QI8), sQbf = smem_u32(smem + SM_QBF);
       const uint32_t sKV = smem_u32(smem + SM_KV);
+      const uint32_t hx = tmem + x * 256;                 // S buffers [0,64), [64,128); O [128,256)
       bool ok = mbar_wait(q_full, 0);
       auto issue_qk = [&](int it) {
-        const uint32_t kslot = sKV + (it & 1) * KV_STAGE;
-        const uint32_t dt = tmem + x * 256;
+        const uint32_t kslot = sKV + (it % NST) * KV_STAGE;
+        const uint32_t dt = hx + (it & 1) * BN;
         if (sc.type(it) == IT_I8) {
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks) {
             const uint64_t ad = make_sdesc_sw128(sQi8 + x * 16384 + ks * 32, 16, 1024);
             const uint64_t bd = make_sdesc_sw128(kslot + ks * 32, 16, 1024);
-            mma_f8_ss(dt, ad, bd, IDESC_F8, ks > 0);
+            if (F8)
+              mma_f8_ss(dt, ad, bd, IDESC_F8, ks > 0);
+            else
+              mma_i8_ss(dt, ad, bd, IDESC_I8, ks > 0);
           }
         } else {
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks) {
-            const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-            const uint64_t ad = make_sdesc_sw128(sQbf + x * 32768 + off, 16, 1024);
-            const uint64_t bd = make_sdesc_sw128(kslot + off, 16, 1024);
+            const uint32_t k16 = (ks & 3) * 32;
+            const uint64_t ad = make_sdesc_sw128(sQbf + x * 32768 + (ks >> 2) * 16384 + k16, 16, 1024);
+            const uint64_t bd = make_sdesc_sw128(kslot + (ks >> 2) * (BN * 128) + k16, 16, 1024);
             mma_f16_ss(dt, ad, bd, IDESC_BF, ks > 0);
           }
         }
-        tc_commit(&s_full[x]);
+        tc_commit(&s_full[x * 2 + (it & 1)]);
       };
-      if (ok && sc.n > 0) {
-        ok = mbar_wait(&kv_full[0], 0);
-        if (ok) {
-          tc_fence_after();
-          issue_qk(0);
-        }
+      for (int it = 0; ok && it < 2 && it < sc.n; ++it) {
+        if (!(ok = mbar_wait(&kv_full[it], 0))) break;
+        tc_fence_after();
+        issue_qk(it);
       }
       for (int it = 0; ok && it < sc.n; ++it) {
-        const uint32_t vslot = sKV + (it & 1) * KV_STAGE + 32768;
-        const uint32_t dt = tmem + x * 256 + 128, at = tmem + x * 256;
+        const int buf = it & 1;
+        const uint32_t vslot = sKV + (it % NST) * KV_STAGE + KV_VOFF;
+        const uint32_t dO = hx + 128, aP = hx + buf * BN;
 #pragma unroll
         for (int c = 0; c < NCHUNK; ++c) {
-          if (!(ok = mbar_wait(&p_full[x * NCHUNK + c], it & 1))) break;
+          if (!(ok = mbar_wait(&p_full[(x * 2 + buf) * NCHUNK + c], (it >> 1) & 1))) break;
           tc_fence_after();
 #pragma unroll
           for (int j = 0; j < 2; ++j) {
-            const int ks = 2 * c + j;
-            const uint64_t bd = make_sdesc_sw128(vslot + ks * 2048, 16384, 1024);
-            mma_f16_ts(dt, at + ks * 8, bd, IDESC_PV, (it > 0 || ks > 0) ? 1u : 0u);
+            const int ks = 2 * c + j;                       // 16 keys per MMA
+            const uint64_t bd = make_sdesc_sw128(vslot + ks * 2048, BN * 128, 1024);
+            mma_f16_ts(dO, aP + ks * 8, bd, IDESC_PV, (it > 0 || ks > 0) ? 1u : 0u);
           }
         }
         if (!ok) break;
-        tc_commit(&kv_free[it & 1]);                // one of the two arrivals
-        if (it + 1 < sc.n) {
-          tc_commit(&pv_done[x]);
-          if (!(ok = mbar_wait(&kv_full[(it + 1) & 1], ((it + 1) >> 1) & 1))) break;
+        tc_commit(&kv_free[it % NST]);              // one of the two arrivals
+        tc_commit(&pv_done[x]);
+        if (it + 2 < sc.n) {
+          if (!(ok = mbar_wait(&kv_full[(it + 2) % NST], ((it + 2) / NST) & 1))) break;
           if (!(ok = mbar_wait(&pv_done[x], it & 1))) break;
           tc_fence_after();
-          issue_qk(it + 1);
+          issue_qk(it + 2);
         }
-      }
-      if (!ok) {
-        *abort_flag = 1;
-        raise_status(a.status, HQ_DEV_TIMEOUT);
-      }
-      tc_commit(o_final);
-    }
-  } else if (!F8 && warp == 1) {
-    // ---------------------- MMA issuer, INT8 low tiles ----------------------
-    // Order per tile t: P.V of head A chunk by chunk as its softmax hands the
-    // chunks over, QK of head A for tile t + 1, the same for head B, so one
-    // head's softmax overlaps the other head's tensor-core work and most of a
-    // head's own P.V overlaps the end of its exp phase.  QK_A(t+1) overwrites
-    // the TMEM columns that P.V_A(t) reads P from and is issued without
-    // waiting for it: this relies on the tensor pipe executing one thread's
-    // MMAs in issue order, which the PTX pipelining rule states only for MMAs
-    // that share an accumulator.  Measured on B200 it holds for these
-    // kind::f16 / kind::i8 sequences (every parity case), and waiting for the
-    // P.V instead costs 20-40% of the kernel.
-    if (lane == 0) {
-      const uint32_t sQi8 = smem_u32(smem + SM_QI8), sQbf = smem_u32(smem + SM_QBF);
-      const uint32_t sKV = smem_u32(smem + SM_KV);
-      bool ok = mbar_wait(q_full, 0);
-      auto issue_qk = [&](int x, int it) {
-        const uint32_t kslot = sKV + (it & 1) * KV_STAGE;
-        const uint32_t dt = tmem + x * 256;
-        if (sc.type(it) == IT_I8) {
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t ad = make_sdesc_sw128(sQi8 + x * 16384 + ks * 32, 16, 1024);
-            const uint64_t bd = make_sdesc_sw128(kslot + ks * 32, 16, 1024);
-            mma_i8_ss(dt, ad, bd, IDESC_I8, ks > 0);
-          }
-        } else {
-#pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
-            const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-            const uint64_t ad = make_sdesc_sw128(sQbf + x * 32768 + off, 16, 1024);
-            const uint64_t bd = make_sdesc_sw128(kslot + off, 16, 1024);
-            mma_f16_ss(dt, ad, bd, IDESC_BF, ks > 0);
-          }
-        }
-        tc_commit(&s_full[x]);
-      };
-      // P.V of head x, tile it, as each 32-key chunk of P arrives
-      auto issue_pv = [&](int x, int it) -> bool {
-        const uint32_t vslot = sKV + (it & 1) * KV_STAGE + 32768;
-        const uint32_t dt = tmem + x * 256 + 128, at = tmem + x * 256;
-#pragma unroll
-        for (int c = 0; c < NCHUNK; ++c) {
-          if (!mbar_wait(&p_full[x * NCHUNK + c], it & 1)) return false;
-          tc_fence_after();
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const int ks = 2 * c + j;
-            const uint64_t bd = make_sdesc_sw128(vslot + ks * 2048, 16384, 1024);
-            mma_f16_ts(dt, at + ks * 8, bd, IDESC_PV, (it > 0 || ks > 0) ? 1u : 0u);
-          }
-        }
-        return true;
-      };
-      if (ok && sc.n > 0) {
-        ok = mbar_wait(&kv_full[0], 0);
-        if (ok) {
-          tc_fence_after();
-          issue_qk(0, 0);
-          issue_qk(1, 0);
-        }
-      }
-      for (int it = 0; ok && it < sc.n; ++it) {
-        if (!(ok = issue_pv(0, it))) break;
-        if (it + 1 < sc.n) {
-          if (!(ok = mbar_wait(&kv_full[(it + 1) & 1], ((it + 1) >> 1) & 1))) break;
-          tc_fence_after();
-          issue_qk(0, it + 1);
-        }
-        if (!(ok = issue_pv(1, it))) break;
-        tc_commit(&kv_free[it & 1]);
-        if (it + 1 < sc.n) issue_qk(1, it + 1);
       }
       if (!ok) {
         *abort_flag = 1;
@@ -449,7 +375,7 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
     const int r = quarter * 32 + lane;
     const int i = i0 + r;
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
-    const uint32_t tS = tl + X * 256, tO = tS + 128;
+    const uint32_t tS = tl + X * 256, tO = tS + 128;   // S buffers at tS, tS + BN
     const size_t bhq = (size_t)b * a.Hq + hq;
     const float sqi = (i < a.N) ? a.sq[bhq * a.N + i] * a.sl : 1.f;
     const int W = a.window;
@@ -459,86 +385,76 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
     const int cnt_lo = remaining_upto(id, a.k_vert, i0 - W);     // ... of the tile's first row
     const int nvert = lim >= 0 ? upper_bound_i32(id, a.k_vert, lim) : 0;
     const float *skp = a.sk + bh * a.nblk_r;
-    // K scales of an INT8 tile (two 64-key blocks), fetched one tile ahead
-    auto fetch_scales = [&](int it, float (&k2)[2]) {
-      k2[0] = k2[1] = 1.f;
+    // K scale of a low tile (one 64-key block), fetched one tile ahead
+    auto fetch_scale = [&](int it) {
+      float k = 1.f;
       if (it < sc.n && sc.type(it) == IT_I8) {
         const int t = sc.tile(it);
-        if (2 * t < a.nblk_r) k2[0] = __ldg(skp + 2 * t);
-        if (2 * t + 1 < a.nblk_r) k2[1] = __ldg(skp + 2 * t + 1);
+        if (t < a.nblk_r) k = __ldg(skp + t);
       }
+      return k;
     };
-    float kn[2];
-    fetch_scales(0, kn);
+    float kn = fetch_scale(0);
     float m = -1e30f;
     float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                      make_float2(0.f, 0.f)};       // independent partial row sums
     bool ok = true;
     for (int it = 0; it < sc.n; ++it) {
-      const float k0 = kn[0], k1 = kn[1];
-      fetch_scales(it + 1, kn);
-      if (!mbar_wait(&s_full[X], it & 1)) {
+      const int buf = it & 1;
+      const float k0 = kn;
+      kn = fetch_scale(it + 1);
+      if (!mbar_wait(&s_full[X * 2 + buf], (it >> 1) & 1)) {
         ok = false;
         break;
       }
       tc_fence_after();
       const int ty = sc.type(it), t = sc.tile(it);
       const int j0 = t * BN;
-      uint32_t xa0[64], xa1[64];
-      tmem_ld64x2(tS, xa0, xa1);                    // the whole S row, one wait
-      float sc0, sc1, c0, c1, mt;                   // per-half scale and offset (log2 units)
+      const uint32_t tSb = tS + buf * BN;
+      uint32_t xa[64];
+      tmem_ld64(tSb, xa);                           // the whole 64-key S row
+      float sc0, c0, mt;                            // scale and offset (log2 units)
       uint32_t add = 0u;                            // bits added to a raw score before the FMA
       if (F8 && ty == IT_I8) {                     // fp32 scores of FP8 codes
         sc0 = sqi * k0;
-        sc1 = sqi * k1;
-        c0 = c1 = 0.f;
+        c0 = 0.f;
         if (j0 + BN > cnt_lo) {
           const int nvalid = cnt_i - j0;
 #pragma unroll
-          for (int e = 0; e < 64; ++e) {
-            if (e >= nvalid) xa0[e] = kNegInfBits;
-            if (64 + e >= nvalid) xa1[e] = kNegInfBits;
-          }
+          for (int e = 0; e < 64; ++e)
+            if (e >= nvalid) xa[e] = kNegInfBits;
         }
-        mt = fmaxf(max64(xa0) * sc0, max64(xa1) * sc1);
+        mt = max64(xa) * sc0;
       } else if (!F8 && ty == IT_I8) {
         sc0 = sqi * k0;
-        sc1 = sqi * k1;
         if (j0 + BN > cnt_lo) {                     // same for every row of the tile
           const int nvalid = cnt_i - j0;
 #pragma unroll
-          for (int e = 0; e < 64; ++e) {
-            if (e >= nvalid) xa0[e] = kMaskRaw;
-            if (64 + e >= nvalid) xa1[e] = kMaskRaw;
-          }
+          for (int e = 0; e < 64; ++e)
+            if (e >= nvalid) xa[e] = kMaskRaw;
         }
         c0 = -kMagic * sc0;
-        c1 = -kMagic * sc1;
         add = kMagicBits;
-        mt = fmaxf(fmaf(__uint_as_float((uint32_t)imax64(xa0) + kMagicBits), sc0, c0),
-                   fmaf(__uint_as_float((uint32_t)imax64(xa1) + kMagicBits), sc1, c1));
+        mt = fmaf(__uint_as_float((uint32_t)imax64(xa) + kMagicBits), sc0, c0);
       } else {
-        sc0 = sc1 = a.sl;
-        c0 = c1 = 0.f;
+        sc0 = a.sl;
+        c0 = 0.f;
         if (ty == IT_WIN) {
 #pragma unroll
           for (int e = 0; e < 64; ++e) {
             const int j = j0 + e;
-            if (j > i || j <= lim) xa0[e] = kNegInfBits;
-            if (j + 64 > i || j + 64 <= lim) xa1[e] = kNegInfBits;
+            if (j > i || j <= lim) xa[e] = kNegInfBits;
           }
         } else {
           const int nvalid = nvert - j0;
 #pragma unroll
-          for (int e = 0; e < 64; ++e) {
-            if (e >= nvalid) xa0[e] = kNegInfBits;
-            if (64 + e >= nvalid) xa1[e] = kNegInfBits;
-          }
+          for (int e = 0; e < 64; ++e)
+            if (e >= nvalid) xa[e] = kNegInfBits;
         }
-        mt = fmaxf(max64(xa0), max64(xa1)) * a.sl;
+        mt = max64(xa) * a.sl;
       }
-      // ---- lazy rescale of the running max (and of O: the commit this
-      // thread waited on covers every MMA issued before it) ----
+      // ---- lazy rescale of the running max, and of O once the P.V of the
+      // previous tile has completed ----
       const bool need = mt > m + kLazy;
       if (__any_sync(0xffffffffu, need)) {
         const float mn = fmaxf(m, mt);
@@ -547,6 +463,11 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
 #pragma unroll
         for (int u = 0; u < 4; ++u) acc[u] = make_float2(acc[u].x * al, acc[u].y * al);
         if (it > 0) {
+          if (!mbar_wait(&pv_done[X], (it - 1) & 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch) {
             uint32_t o[32];
@@ -560,36 +481,32 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
       // ---- P = exp2(x * scale + offset - m) as packed fp16, 32 keys per
       // chunk, each chunk handed to the MMA as soon as it is in TMEM ----
       c0 -= m;
-      c1 -= m;
+      const float2 s2 = make_float2(sc0, sc0), o2 = make_float2(c0, c0);
 #pragma unroll
-      for (int q4 = 0; q4 < NCHUNK; ++q4) {
-        uint32_t(&xh)[64] = (q4 < 2) ? xa0 : xa1;
-        const int base = (q4 & 1) * 32;
-        const float2 s2 = q4 < 2 ? make_float2(sc0, sc0) : make_float2(sc1, sc1);
-        const float2 o2 = q4 < 2 ? make_float2(c0, c0) : make_float2(c1, c1);
+      for (int q = 0; q < NCHUNK; ++q) {
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float2 y = ffma2(make_float2(__uint_as_float(xh[base + 2 * e] + add),
-                                             __uint_as_float(xh[base + 2 * e + 1] + add)), s2, o2);
+          const float2 y = ffma2(make_float2(__uint_as_float(xa[q * 32 + 2 * e] + add),
+                                             __uint_as_float(xa[q * 32 + 2 * e + 1] + add)), s2, o2);
           const float2 p = make_float2(fast_exp2(y.x), fast_exp2(y.y));
           acc[e & 3] = fadd2(acc[e & 3], p);
           pk[e] = pack_f16x2(p.x, p.y);
         }
         // hand over the previous chunk (its store has had this chunk's exps
         // to complete), then store this one
-        if (q4 > 0) {
+        if (q > 0) {
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&p_full[X * NCHUNK + q4 - 1]);
+          if (lane == 0) mbar_arrive(&p_full[(X * 2 + buf) * NCHUNK + q - 1]);
         }
-        tmem_st16(tS + q4 * 16, pk);              // keys 32*q4 .. 32*q4+31
+        tmem_st16(tSb + q * 16, pk);               // keys 32*q .. 32*q+31
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[X * NCHUNK + NCHUNK - 1]);
+      if (lane == 0) mbar_arrive(&p_full[(X * 2 + buf) * NCHUNK + NCHUNK - 1]);
     }
     const float l = (acc[0].x + acc[0].y + acc[1].x + acc[1].y) + (acc[2].x + acc[2].y + acc[3].x + acc[3].y);
     if (ok) ok = mbar_wait(o_final, 0);
