@@ -29,11 +29,18 @@ def oracle_idx(x, w: Workload):
     return oracle.topk(sc, w.window, w.k_vert), sc
 
 
-def run_prefill_case(w: Workload, rows=None, check_probe=True, fmt=0):
+def run_prefill_case(w: Workload, rows=None, check_probe=True, fmt=0, planted_idx=False):
     H = hq()
     x = make_inputs(w)
     d = to_dev(x)
-    ridx, rsc = oracle_idx(x, w)
+    if planted_idx:
+        # the seeded planted positions (sorted, distinct, before the window)
+        # as the vertical set: no probe, so sequences shorter than the 64
+        # probe queries work too
+        ridx, rsc = x["planted"].numpy().astype(np.int32), None
+        check_probe = False
+    else:
+        ridx, rsc = oracle_idx(x, w)
     if check_probe and w.k_vert > 0:
         gidx = H.probe_vertical(d["q"][:, :, w.L - 64:], d["k"], w.window, w.k_vert)
         torch.cuda.synchronize()
@@ -117,6 +124,27 @@ def test_prefill_reports_bad_index_lists():
         H.prefill_attn(d["q"], d["k"], d["v"], torch.from_numpy(bad).cuda(), w.window, ws=ws)
         assert H.hq_read_device_status(ws, clear=True) & H.HQ_DEV_BAD_INDEX
         assert H.hq_read_device_status(ws) == 0
+
+
+# Short sequences on the tensor-core path (D = 128, two query heads per KV
+# head): one, two or three 64-key tiles in all, lengths on and just past a
+# tile edge, windows that are not a multiple of the tile, the diagonal-only
+# window and no window.
+SHORT = [(1, 16, 0), (37, 16, 20), (64, 0, 8), (65, 40, 16), (129, 64, 20), (200, 100, 4),
+         (333, 1, 10)]
+
+
+@pytest.mark.parametrize("N,W,inv_f", SHORT)
+def test_prefill_short_sequences_tile_edges(N, W, inv_f):
+    f = fractions.Fraction(1, inv_f) if inv_f else fractions.Fraction(0)
+    w = Workload("short", "prefill", 1, 4, 2, 128, N, W, f, 4, 400 + N)
+    run_prefill_case(w, planted_idx=True)
+
+
+@pytest.mark.parametrize("N,W,inv_f", [(37, 16, 20), (129, 64, 20), (333, 1, 10)])
+def test_prefill_fp8_short_sequences(N, W, inv_f):
+    w = Workload("short_fp8", "prefill", 1, 4, 2, 128, N, W, fractions.Fraction(1, inv_f), 4, 500 + N)
+    run_prefill_case(w, planted_idx=True, fmt=1)
 
 
 # --------------------------------------------------------------------------
