@@ -243,6 +243,7 @@ def run_hq(args, rank, world, dev):
     d2h = out_p.numel() * 4 + out_d.numel() * 4
 
     loop = decode_loop(H, w, q, k, v, q_dec, dev, stream, world)
+    fp8 = fp8_leg(H, w, q, k, v, idx, q_dec, dev, stream, world)
 
     idx_np = idx.cpu().numpy()
     dbytes = decode_bytes(B, Hq, Hkv, D, cache.n_lo, cache.n_hi, w.bits)
@@ -250,7 +251,43 @@ def run_hq(args, rank, world, dev):
     clocks = clk.summary()
     return dict(per=per, total_ms=max_over_ranks(total_ms / args.steps, world, dev), dbytes=dbytes,
                 i8=i8_ops, bf=bf_flops, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, clocks=clocks,
-                kpad=(kv + 63) // 64 * 64, w=w, loop=loop)
+                kpad=(kv + 63) // 64 * 64, w=w, loop=loop, fp8=fp8)
+
+
+def fp8_leg(H, w, q, k, v, idx, q_dec, dev, stream, world, reps=5):
+    """The FP8 (E4M3) low-bit format on the same layer and vertical set,
+    after the timed steps: the prefill with an FP8 low part, and an FP8 KV
+    cache (pack, then decode).  Median of `reps` calls each (two untimed
+    first), the L2 flushed before every call."""
+    B, Hq, Hkv, D, N, W, kv = w.B, w.Hq, w.Hkv, w.D, w.L, w.window, w.k_vert
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    out_p = torch.empty(B, Hq, N, D, dtype=torch.float32, device=dev)
+    out_d = torch.empty(B, Hq, D, dtype=torch.float32, device=dev)
+    ws_pre = H.workspace(H.hq_prefill_workspace_size(B, Hq, Hkv, N, D, kv), dev)
+    cache = H.KVCache.empty(B, Hkv, N, D, W, kv, 8, dev, with_pos=False, fmt=H.HQ_KV_FP8)
+    ws_pack = H.workspace(256, dev)
+    ws_dec = H.workspace(H.hq_decode_workspace_size(B, Hq, Hkv, D, cache.n_lo, cache.n_hi, 8), dev)
+
+    def timed(fn):
+        ts = []
+        for i in range(reps + 2):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            if i >= 2:
+                ts.append(e0.elapsed_time(e1))
+        return max_over_ranks(float(np.median(ts)), world, dev)
+
+    barrier(world)
+    pre = timed(lambda: H.hq_prefill_attn_ex(q, k, v, idx, B, Hq, Hkv, N, D, W, kv, 0.0,
+                                             H.HQ_KV_FP8, out_p, ws_pre))
+    pack = timed(lambda: H.hq_pack_kv(k, v, idx, B, Hkv, N, D, W, kv, 8, 32, cache, ws_pack))
+    dec = timed(lambda: H.hq_decode_attn(q_dec, cache, B, Hq, Hkv, D, 0.0, out_d, None, ws_dec))
+    return {"prefill_ms": pre, "pack_ms": pack, "decode_ms": dec,
+            "decode_bytes": decode_bytes(B, Hq, Hkv, D, cache.n_lo, cache.n_hi, 8)}
 
 
 def decode_loop(H, w, q, k, v, q_dec, dev, stream, world, T=64):
@@ -445,7 +482,7 @@ def main():
         "dtype": "int4 KV codes -> bf16/fp16 MMA, fp32 accumulate (decode); int8 + bf16/fp16 (prefill)",
         "data": "synthetic (seeded generator: outlier channels, planted vertical lines)",
         "config": config_dict(w, world),
-        # the dominant kernel of the step (84% of its launch time) is the prefill
+        # the dominant kernel of the step (about 90% of its launch time) is the prefill
         "roofline": {"kernel": "prefill_tc (hq_prefill_attn)", "bound": "tensor",
                      "achieved": pre_tflops, "peak": mixed_peak, "unit": "TFLOP/s",
                      "frac": pre_tflops / mixed_peak, "traffic": profiled_traffic("prefill_tc"),
@@ -461,6 +498,16 @@ def main():
         "per_call_ms": {n: per[n] for n in ("probe", "prefill", "pack", "decode")},
         # token-by-token decode after the timed steps: cache maintenance + attention
         "decode_loop": r["loop"],
+        # the FP8 (E4M3) low-bit format on the same layer, after the timed steps
+        "fp8": {"prefill_ms": r["fp8"]["prefill_ms"],
+                "prefill_frac": t_star * 1e3 / r["fp8"]["prefill_ms"],
+                "pack_ms": r["fp8"]["pack_ms"],
+                "decode_us": r["fp8"]["decode_ms"] * 1e3,
+                "decode_gbs": r["fp8"]["decode_bytes"] / (r["fp8"]["decode_ms"] * 1e-3) / 1e9,
+                "decode_frac": r["fp8"]["decode_bytes"] / (r["fp8"]["decode_ms"] * 1e-3) / 1e9
+                / pk["hbm_gbs"],
+                "note": "prefill: FP8 QK at the INT8 rate (nominal FP8 = INT8 on B200), same T*; "
+                        "decode: E4M3 codes + fp16 scales, median of 5, L2 flushed"},
         "e2e": {"value": r["dbytes"] / (r["e2e_ms"] * 1e-3) / 1e12 * world, "unit": "TB/s",
                 "ms_per_step": r["e2e_ms"], "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"],
