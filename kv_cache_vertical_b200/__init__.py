@@ -14,7 +14,9 @@ __all__ = ["hq", "synth"]
 
 
 def __getattr__(name):
-    if name in ("hq", "synth"):
+    # submodules first: `from kv_cache_vertical_b200 import build` must work
+    # before libhq.so exists (it is what builds it)
+    if name in ("hq", "synth", "build"):
         return importlib.import_module(f"{__name__}.{name}")
     mod = importlib.import_module(f"{__name__}.hq")
     try:

@@ -177,3 +177,16 @@ def test_probe_and_prefill_argument_checks(lib):
     assert qq(FAKE, FAKE, FAKE, 1, 4, 2, 256, 64, 12, None, FAKE, FAKE, FAKE, None) == 1
     assert qq(FAKE, FAKE, None, 1, 4, 2, 256, 64, 12, FAKE, FAKE, FAKE, FAKE, None) == 1
     assert qq(FAKE, FAKE, FAKE, 1, 4, 2, 256, 64, 300, FAKE, FAKE, FAKE, FAKE, None) == 1
+
+
+def test_build_module_imports_without_the_library():
+    # `from kv_cache_vertical_b200 import build` is what builds libhq.so, so it
+    # must not load the binding (which raises when the library is missing)
+    import os
+    import subprocess
+    import sys
+    code = ("import sys; from kv_cache_vertical_b200 import build; "
+            "assert 'kv_cache_vertical_b200.hq' not in sys.modules, 'binding loaded'")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
