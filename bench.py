@@ -44,12 +44,14 @@ NOMINAL_INT8_OVER_BF16 = 2.0                     # dense INT8 / dense bf16 (vend
 
 
 def peaks():
-    p = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "src": "fallback"}
+    p = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+         "sm_max_mhz": 1965.0, "src": "fallback"}
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
         with open(path) as f:
             m = json.load(f)
-        p.update({k: m[k] for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained") if k in m})
+        p.update({k: m[k] for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained", "sm_max_mhz")
+                  if k in m})
         p["src"] = "measured"
     return p
 
@@ -243,6 +245,7 @@ def run_hq(args, rank, world, dev):
     d2h = out_p.numel() * 4 + out_d.numel() * 4
 
     loop = decode_loop(H, w, q, k, v, q_dec, dev, stream, world)
+    graph = decode_graph(H, w, q_dec, cache, out_d, ws_dec, dev, world)
     fp8 = fp8_leg(H, w, q, k, v, idx, q_dec, dev, stream, world)
     i8_tops = int8_gemm_peak(dev)
 
@@ -252,7 +255,40 @@ def run_hq(args, rank, world, dev):
     clocks = clk.summary()
     return dict(per=per, total_ms=max_over_ranks(total_ms / args.steps, world, dev), dbytes=dbytes,
                 i8=i8_ops, bf=bf_flops, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, clocks=clocks,
-                kpad=(kv + 63) // 64 * 64, w=w, loop=loop, fp8=fp8, i8_tops=i8_tops)
+                kpad=(kv + 63) // 64 * 64, w=w, loop=loop, fp8=fp8, i8_tops=i8_tops, graph=graph)
+
+
+def decode_graph(H, w, q_dec, cache, out, ws, dev, world, n=50, reps=7):
+    """The packed 32K decode as n back-to-back calls captured in one CUDA
+    graph, replayed `reps` times: per-call median and best.  The 47 MB cache
+    stays in the L2 between calls, so this is the call's latency floor, not
+    an HBM figure."""
+    try:
+        s = torch.cuda.Stream(dev)
+        s.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(s):
+            H.hq_decode_attn(q_dec, cache, w.B, w.Hq, w.Hkv, w.D, 0.0, out, None, ws, s)
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for _ in range(n):
+                H.hq_decode_attn(q_dec, cache, w.B, w.Hq, w.Hkv, w.D, 0.0, out, None, ws, s)
+        ts = []
+        with torch.cuda.stream(s):            # replay() launches on the current stream
+            g.replay()
+            torch.cuda.synchronize(dev)
+            for _ in range(reps):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(s)
+                g.replay()
+                e1.record(s)
+                torch.cuda.synchronize(dev)
+                ts.append(e0.elapsed_time(e1) * 1e3 / n)
+        del g
+        return {"calls_per_graph": n, "us_per_call_median": max_over_ranks(float(np.median(ts)), world, dev),
+                "us_per_call_best": max_over_ranks(min(ts), world, dev), "l2": "warm (cache fits the L2)"}
+    except RuntimeError as e:          # capture unsupported: report, do not fail the bench
+        return {"error": str(e).splitlines()[0][:200]}
 
 
 def int8_gemm_peak(dev, n=8192, reps=10):
@@ -409,11 +445,23 @@ def oracle_decode_sample(w, heads_kv: int):
     return nbytes, dt, oracle.max_threads()
 
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_baseline(w):
     nbytes, dt, cores = oracle_decode_sample(w, w.Hkv)
     return {"value": nbytes / dt / 1e12, "unit": "TB/s", "cores": cores, "kind": "oracle",
             "sample": f"oracle fp64 decode attention over the full {w.L}-token INT4 cache, "
-                      f"{w.Hq} query heads (one call, {dt:.2f} s)"}
+                      f"{w.Hq} query heads (one call, {dt:.2f} s)",
+            "cpu_model": cpu_model(), "nproc": os.cpu_count()}
 
 
 def run_reference(args, rank, world):
@@ -432,7 +480,8 @@ def run_reference(args, rank, world):
     ms = 1e3 * sum(t for _, t in vals) / len(vals)
     cpu = {"value": tb, "unit": "TB/s", "cores": cores, "kind": "oracle",
            "sample": f"oracle fp64 decode of {hk} of {w.Hkv} KV heads ({hk * w.G} query heads) "
-                     f"over the {w.L}-token INT4 cache per step"}
+                     f"over the {w.L}-token INT4 cache per step",
+           "cpu_model": cpu_model(), "nproc": os.cpu_count()}
     return {"impl": "reference", "metric": METRIC, "value": tb, "unit": "TB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
@@ -489,6 +538,9 @@ def main():
     i8_peak = max(pk["bf16_tflops"] * NOMINAL_INT8_OVER_BF16, r["i8_tops"] or 0.0)
     t_star = r["bf"] / (pk["bf16_tflops"] * 1e12) + r["i8"] / (i8_peak * 1e12)
     pre_tflops = (r["bf"] + r["i8"]) / pre_s / 1e12
+    exps = w.Hq * w.B * w.L * (w.L + 1) // 2
+    # nominal ex2 rate: 16 per SM per clock at the maximum SM clock
+    mufu_peak = 16.0 * torch.cuda.get_device_properties(0).multi_processor_count * pk["sm_max_mhz"] * 1e6
     mixed_peak = (r["bf"] + r["i8"]) / t_star / 1e12
     # probe 4 (two QK passes, row stats, top-k); prefill 4 (+1 vertical
     # gather when there are vertical columns); pack 1; decode 1
@@ -514,6 +566,9 @@ def main():
                      "ms": per["prefill"], "roofline_ms": t_star * 1e3,
                      "int8_tops": r["i8"] / 1e12, "bf16_tflop": r["bf"] / 1e12,
                      "int8_gemm_tops_measured": r["i8_tops"],
+                     # the exp is the co-bound: one per (causal pair, query head)
+                     "exps": exps, "exp_rate_tps": exps / pre_s / 1e12,
+                     "exp_frac_of_nominal_mufu": exps / pre_s / mufu_peak,
                      "peak_src": pk["src"] + " bf16 burst GEMM peak; INT8 = the larger of bf16 x "
                                  "nominal ratio 2 and the INT8 GEMM measured in this run "
                                  "(torch._int_mm 8192^3); peak = work-weighted mix of the two"},
@@ -523,8 +578,10 @@ def main():
                    "us": per["decode"] * 1e3, "peak_src": pk["src"] + " (copy bandwidth)",
                    "frac_of_8TBs": dec_tbs / 8.0},
         "per_call_ms": {n: per[n] for n in ("probe", "prefill", "pack", "decode")},
+        "probe_frac_of_prefill": per["probe"] / per["prefill"],
         # token-by-token decode after the timed steps: cache maintenance + attention
         "decode_loop": r["loop"],
+        "decode_graph": r["graph"],
         # the FP8 (E4M3) low-bit format on the same layer, after the timed steps
         "fp8": {"prefill_ms": r["fp8"]["prefill_ms"],
                 "prefill_frac": t_star * 1e3 / r["fp8"]["prefill_ms"],
