@@ -130,17 +130,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&x)[32
       : "memory");
 }
 
-// 32 lanes x 128 columns in one instruction, waited for in the same statement.
-__device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&x)[128]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x128.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95,%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127}, [%128];\n"
-      "tcgen05.wait::ld.sync.aligned;\n"
-      : "=r"(x[0]), "=r"(x[1]), "=r"(x[2]), "=r"(x[3]), "=r"(x[4]), "=r"(x[5]), "=r"(x[6]), "=r"(x[7]), "=r"(x[8]), "=r"(x[9]), "=r"(x[10]), "=r"(x[11]), "=r"(x[12]), "=r"(x[13]), "=r"(x[14]), "=r"(x[15]), "=r"(x[16]), "=r"(x[17]), "=r"(x[18]), "=r"(x[19]), "=r"(x[20]), "=r"(x[21]), "=r"(x[22]), "=r"(x[23]), "=r"(x[24]), "=r"(x[25]), "=r"(x[26]), "=r"(x[27]), "=r"(x[28]), "=r"(x[29]), "=r"(x[30]), "=r"(x[31]), "=r"(x[32]), "=r"(x[33]), "=r"(x[34]), "=r"(x[35]), "=r"(x[36]), "=r"(x[37]), "=r"(x[38]), "=r"(x[39]), "=r"(x[40]), "=r"(x[41]), "=r"(x[42]), "=r"(x[43]), "=r"(x[44]), "=r"(x[45]), "=r"(x[46]), "=r"(x[47]), "=r"(x[48]), "=r"(x[49]), "=r"(x[50]), "=r"(x[51]), "=r"(x[52]), "=r"(x[53]), "=r"(x[54]), "=r"(x[55]), "=r"(x[56]), "=r"(x[57]), "=r"(x[58]), "=r"(x[59]), "=r"(x[60]), "=r"(x[61]), "=r"(x[62]), "=r"(x[63]), "=r"(x[64]), "=r"(x[65]), "=r"(x[66]), "=r"(x[67]), "=r"(x[68]), "=r"(x[69]), "=r"(x[70]), "=r"(x[71]), "=r"(x[72]), "=r"(x[73]), "=r"(x[74]), "=r"(x[75]), "=r"(x[76]), "=r"(x[77]), "=r"(x[78]), "=r"(x[79]), "=r"(x[80]), "=r"(x[81]), "=r"(x[82]), "=r"(x[83]), "=r"(x[84]), "=r"(x[85]), "=r"(x[86]), "=r"(x[87]), "=r"(x[88]), "=r"(x[89]), "=r"(x[90]), "=r"(x[91]), "=r"(x[92]), "=r"(x[93]), "=r"(x[94]), "=r"(x[95]), "=r"(x[96]), "=r"(x[97]), "=r"(x[98]), "=r"(x[99]), "=r"(x[100]), "=r"(x[101]), "=r"(x[102]), "=r"(x[103]), "=r"(x[104]), "=r"(x[105]), "=r"(x[106]), "=r"(x[107]), "=r"(x[108]), "=r"(x[109]), "=r"(x[110]), "=r"(x[111]), "=r"(x[112]), "=r"(x[113]), "=r"(x[114]), "=r"(x[115]), "=r"(x[116]), "=r"(x[117]), "=r"(x[118]), "=r"(x[119]), "=r"(x[120]), "=r"(x[121]), "=r"(x[122]), "=r"(x[123]), "=r"(x[124]), "=r"(x[125]), "=r"(x[126]), "=r"(x[127])
-      : "r"(taddr)
-      : "memory");
-}
-
-
 // 32 lanes x 64 columns in one instruction, waited for in the same statement.
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&x)[64]) {
   asm volatile(
@@ -148,19 +137,6 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&x)[64]) {
       "tcgen05.wait::ld.sync.aligned;\n"
       : "=r"(x[0]), "=r"(x[1]), "=r"(x[2]), "=r"(x[3]), "=r"(x[4]), "=r"(x[5]), "=r"(x[6]), "=r"(x[7]), "=r"(x[8]), "=r"(x[9]), "=r"(x[10]), "=r"(x[11]), "=r"(x[12]), "=r"(x[13]), "=r"(x[14]), "=r"(x[15]), "=r"(x[16]), "=r"(x[17]), "=r"(x[18]), "=r"(x[19]), "=r"(x[20]), "=r"(x[21]), "=r"(x[22]), "=r"(x[23]), "=r"(x[24]), "=r"(x[25]), "=r"(x[26]), "=r"(x[27]), "=r"(x[28]), "=r"(x[29]), "=r"(x[30]), "=r"(x[31]), "=r"(x[32]), "=r"(x[33]), "=r"(x[34]), "=r"(x[35]), "=r"(x[36]), "=r"(x[37]), "=r"(x[38]), "=r"(x[39]), "=r"(x[40]), "=r"(x[41]), "=r"(x[42]), "=r"(x[43]), "=r"(x[44]), "=r"(x[45]), "=r"(x[46]), "=r"(x[47]), "=r"(x[48]), "=r"(x[49]), "=r"(x[50]), "=r"(x[51]), "=r"(x[52]), "=r"(x[53]), "=r"(x[54]), "=r"(x[55]), "=r"(x[56]), "=r"(x[57]), "=r"(x[58]), "=r"(x[59]), "=r"(x[60]), "=r"(x[61]), "=r"(x[62]), "=r"(x[63])
       : "r"(taddr)
-      : "memory");
-}
-
-
-// Two 32-lane x 64-column loads (columns [0,64) and [64,128) of taddr) and one
-// wait, in one statement.
-__device__ __forceinline__ void tmem_ld64x2(uint32_t taddr, uint32_t (&x0)[64], uint32_t (&x1)[64]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%128];\n"
-      "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95,%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127}, [%129];\n"
-      "tcgen05.wait::ld.sync.aligned;\n"
-      : "=r"(x0[0]), "=r"(x0[1]), "=r"(x0[2]), "=r"(x0[3]), "=r"(x0[4]), "=r"(x0[5]), "=r"(x0[6]), "=r"(x0[7]), "=r"(x0[8]), "=r"(x0[9]), "=r"(x0[10]), "=r"(x0[11]), "=r"(x0[12]), "=r"(x0[13]), "=r"(x0[14]), "=r"(x0[15]), "=r"(x0[16]), "=r"(x0[17]), "=r"(x0[18]), "=r"(x0[19]), "=r"(x0[20]), "=r"(x0[21]), "=r"(x0[22]), "=r"(x0[23]), "=r"(x0[24]), "=r"(x0[25]), "=r"(x0[26]), "=r"(x0[27]), "=r"(x0[28]), "=r"(x0[29]), "=r"(x0[30]), "=r"(x0[31]), "=r"(x0[32]), "=r"(x0[33]), "=r"(x0[34]), "=r"(x0[35]), "=r"(x0[36]), "=r"(x0[37]), "=r"(x0[38]), "=r"(x0[39]), "=r"(x0[40]), "=r"(x0[41]), "=r"(x0[42]), "=r"(x0[43]), "=r"(x0[44]), "=r"(x0[45]), "=r"(x0[46]), "=r"(x0[47]), "=r"(x0[48]), "=r"(x0[49]), "=r"(x0[50]), "=r"(x0[51]), "=r"(x0[52]), "=r"(x0[53]), "=r"(x0[54]), "=r"(x0[55]), "=r"(x0[56]), "=r"(x0[57]), "=r"(x0[58]), "=r"(x0[59]), "=r"(x0[60]), "=r"(x0[61]), "=r"(x0[62]), "=r"(x0[63]), "=r"(x1[0]), "=r"(x1[1]), "=r"(x1[2]), "=r"(x1[3]), "=r"(x1[4]), "=r"(x1[5]), "=r"(x1[6]), "=r"(x1[7]), "=r"(x1[8]), "=r"(x1[9]), "=r"(x1[10]), "=r"(x1[11]), "=r"(x1[12]), "=r"(x1[13]), "=r"(x1[14]), "=r"(x1[15]), "=r"(x1[16]), "=r"(x1[17]), "=r"(x1[18]), "=r"(x1[19]), "=r"(x1[20]), "=r"(x1[21]), "=r"(x1[22]), "=r"(x1[23]), "=r"(x1[24]), "=r"(x1[25]), "=r"(x1[26]), "=r"(x1[27]), "=r"(x1[28]), "=r"(x1[29]), "=r"(x1[30]), "=r"(x1[31]), "=r"(x1[32]), "=r"(x1[33]), "=r"(x1[34]), "=r"(x1[35]), "=r"(x1[36]), "=r"(x1[37]), "=r"(x1[38]), "=r"(x1[39]), "=r"(x1[40]), "=r"(x1[41]), "=r"(x1[42]), "=r"(x1[43]), "=r"(x1[44]), "=r"(x1[45]), "=r"(x1[46]), "=r"(x1[47]), "=r"(x1[48]), "=r"(x1[49]), "=r"(x1[50]), "=r"(x1[51]), "=r"(x1[52]), "=r"(x1[53]), "=r"(x1[54]), "=r"(x1[55]), "=r"(x1[56]), "=r"(x1[57]), "=r"(x1[58]), "=r"(x1[59]), "=r"(x1[60]), "=r"(x1[61]), "=r"(x1[62]), "=r"(x1[63])
-      : "r"(taddr), "r"(taddr + 64u)
       : "memory");
 }
 
@@ -173,17 +149,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&x)[16
       : "memory");
 }
 
-// 32 lanes x 64 columns in one instruction (completion: tmem_wait_st).
-__device__ __forceinline__ void tmem_st64(uint32_t taddr, const uint32_t (&x)[64]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,%64};\n" ::"r"(taddr),
-      "r"(x[0]), "r"(x[1]), "r"(x[2]), "r"(x[3]), "r"(x[4]), "r"(x[5]), "r"(x[6]), "r"(x[7]), "r"(x[8]), "r"(x[9]), "r"(x[10]), "r"(x[11]), "r"(x[12]), "r"(x[13]), "r"(x[14]), "r"(x[15]), "r"(x[16]), "r"(x[17]), "r"(x[18]), "r"(x[19]), "r"(x[20]), "r"(x[21]), "r"(x[22]), "r"(x[23]), "r"(x[24]), "r"(x[25]), "r"(x[26]), "r"(x[27]), "r"(x[28]), "r"(x[29]), "r"(x[30]), "r"(x[31]), "r"(x[32]), "r"(x[33]), "r"(x[34]), "r"(x[35]), "r"(x[36]), "r"(x[37]), "r"(x[38]), "r"(x[39]), "r"(x[40]), "r"(x[41]), "r"(x[42]), "r"(x[43]), "r"(x[44]), "r"(x[45]), "r"(x[46]), "r"(x[47]), "r"(x[48]), "r"(x[49]), "r"(x[50]), "r"(x[51]), "r"(x[52]), "r"(x[53]), "r"(x[54]), "r"(x[55]), "r"(x[56]), "r"(x[57]), "r"(x[58]), "r"(x[59]), "r"(x[60]), "r"(x[61]), "r"(x[62]), "r"(x[63])
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_wait_ld() {
-  asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
-}
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
 }
