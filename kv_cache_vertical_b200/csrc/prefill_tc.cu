@@ -364,7 +364,7 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kRegsHigh));
   {
     // ------------------------------ softmax ------------------------------
-    // One thread per query row (TMEM lane), the whole 128-key S row in
+    // One thread per query row (TMEM lane), the whole 64-key S row of a tile in
     // registers.  INT8 scores stay integers until the exp: their row max is an
     // integer max, and adding the bits of 2^23 + 2^22 turns s into the float
     // 2^23 + 2^22 + s (exact for |s| < 2^22), whose offset is folded into the
