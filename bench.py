@@ -255,7 +255,8 @@ def run_hq(args, rank, world, dev):
     clocks = clk.summary()
     return dict(per=per, total_ms=max_over_ranks(total_ms / args.steps, world, dev), dbytes=dbytes,
                 i8=i8_ops, bf=bf_flops, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, clocks=clocks,
-                kpad=(kv + 63) // 64 * 64, w=w, loop=loop, fp8=fp8, i8_tops=i8_tops, graph=graph)
+                kpad=(kv + 63) // 64 * 64, w=w, loop=loop, fp8=fp8, i8_tops=i8_tops, graph=graph,
+                idx=idx_np)
 
 
 def decode_graph(H, w, q_dec, cache, out, ws, dev, world, n=50, reps=7):
@@ -464,6 +465,36 @@ def cpu_baseline(w):
             "cpu_model": cpu_model(), "nproc": os.cpu_count()}
 
 
+def cpu_baseline_prefill(w, idx: np.ndarray, per_stratum: int = 32):
+    """The oracle's hybrid prefill on a stratified sample of query rows (the
+    first rows, rows around the window boundary, the middle and the last),
+    every query head, with the GPU's vertical set; the whole-layer time is
+    extrapolated by causal pairs (a row's cost grows with its key count) and
+    labelled as such."""
+    import oracle
+    N, W = w.L, w.window
+    x = make_inputs(w)
+    t0 = time.perf_counter()
+    quant = oracle.prefill_quant(x["q"], x["k"], idx)
+    t_quant = time.perf_counter() - t0
+    k = per_stratum
+    rows = np.unique(np.concatenate([np.arange(k), max(W - k // 2, 0) + np.arange(k),
+                                     N // 2 - k // 2 + np.arange(k), N - k + np.arange(k)]))
+    rows = rows[(rows >= 0) & (rows < N)].astype(np.int32)
+    t0 = time.perf_counter()
+    oracle.prefill_attn(x["q"], x["k"], x["v"], idx, W, quant=quant, rows=rows)
+    t_rows = time.perf_counter() - t0
+    pairs_sampled = int((rows.astype(np.int64) + 1).sum())
+    pairs_total = N * (N + 1) // 2
+    est_s = t_quant + t_rows * pairs_total / pairs_sampled
+    return {"value": est_s * 1e3, "unit": "ms (whole prefill, extrapolated)", "kind": "oracle",
+            "extrapolated": True, "cores": oracle.max_threads(), "rows_sampled": int(rows.size),
+            "sample_s": t_quant + t_rows,
+            "sample": f"oracle fp64 hybrid prefill of {rows.size} stratified query rows x {w.Hq} "
+                      f"query heads (plus the whole INT8 pre-pass); time per causal pair scaled "
+                      f"to all {pairs_total} pairs"}
+
+
 def run_reference(args, rank, world):
     """--impl reference: the oracle as it stands, timed on the host cores."""
     if rank != 0:
@@ -602,6 +633,7 @@ def main():
     }
     if world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(w)
+        out["cpu_baseline_prefill"] = cpu_baseline_prefill(w, r["idx"])
     print(json.dumps(out), flush=True)
 
 
