@@ -190,3 +190,24 @@ def test_build_module_imports_without_the_library():
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     r = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+def test_prefill_format_argument_checks(lib):
+    # the low-part format is checked on the host, before any launch: an
+    # unknown format, and FP8 where the tensor-core kernel does not apply
+    # (D = 64, or an odd number of query heads per KV head; on a machine
+    # without a GPU the tensor-core kernel is never available)
+    q = lib.hq_prefill_quant_ex
+    q.restype = ctypes.c_int
+    assert q(FAKE, FAKE, FAKE, 1, 2, 1, 256, 64, 8, 7, FAKE, FAKE, FAKE, FAKE, None) == 2
+    assert q(None, FAKE, FAKE, 1, 2, 1, 256, 64, 8, 1, FAKE, FAKE, FAKE, FAKE, None) == 1
+    f = lib.hq_prefill_attn_ex
+    f.restype = ctypes.c_int
+
+    def call(D=128, Hq=2, Hkv=1, fmt=1, q=FAKE):
+        return f(q, FAKE, FAKE, FAKE, 1, Hq, Hkv, 256, D, 32, 8, ctypes.c_float(0.0), fmt, FAKE,
+                 FAKE, ctypes.c_size_t(1 << 30), None)
+    assert call(fmt=7) == 2
+    assert call(D=64, fmt=1) == 2
+    assert call(Hq=3, Hkv=1, fmt=1) == 2
+    assert call(q=None) == 1
