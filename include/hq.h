@@ -156,6 +156,49 @@ hq_status hq_probe_vertical(const void *q_probe, int64_t q_head_stride, const vo
                             float softmax_scale, int32_t *idx_out, float *score_out, void *ws,
                             size_t ws_bytes, void *stream);
 
+/*
+ * The same probe with the context's keys split among ranks (a context too
+ * long for one GPU): rank r holds keys [key_off, key_off + Ls) of the L-key
+ * context, every rank holds the P probe queries (context positions L - P + p).
+ * The probe's two passes need every probe row's softmax max and sum over the
+ * whole context, and the top-k over all candidate columns; so the exchange is
+ * two small gathers (the caller's: e.g. torch.distributed.all_gather):
+ *   1. hq_probe_shard_stats on every rank -> (max, Z) per probe row for its keys;
+ *      gather the R results, hq_probe_merge_stats -> (max, 1/Z) of the context;
+ *   2. hq_probe_shard_topk on every rank -> its best k_vert candidate columns
+ *      (context positions, scores); gather, hq_probe_merge_topk -> the context's
+ *      k_vert columns, ascending, ties to the lower position, as
+ *      hq_probe_vertical would pick them (candidate scores differ from the
+ *      single-GPU probe's only by the order of the row-sum merge).
+ * Layouts: q_probe, softmax_scale and q_head_stride as for hq_probe_vertical;
+ * k_shard bf16 [B, Hkv, Ls, D]; stats f32 pairs [B*Hkv, (Hq/Hkv)*P, 2] in the
+ * log2 domain (row max of s*scale*log2(e), then Z = sum of 2^(x - max), or
+ * 1/Z after the merge); a row that sees none of a rank's keys gets
+ * (-FLT_MAX, 0).  cand_idx i32 / cand_score f32 [B*Hkv, k_vert]: a rank with
+ * fewer than k_vert candidates (keys before L - window) pads with -1 / -FLT_MAX.
+ * Merge inputs are the R ranks' arrays stacked on a leading axis.
+ * Requires 1 <= P <= L, 0 <= key_off, key_off + Ls <= L, Ls >= 1,
+ * 0 <= k_vert <= L - window.  Errors as for hq_probe_vertical; a candidate
+ * position outside [0, L - window) sets HQ_DEV_BAD_INDEX in the merge's status
+ * word and is ignored.
+ */
+size_t hq_probe_shard_workspace_size(int B, int Hq, int Hkv, int P, int Ls, int D, int k_vert);
+hq_status hq_probe_shard_stats(const void *q_probe, int64_t q_head_stride, const void *k_shard,
+                               int B, int Hq, int Hkv, int P, int Ls, int D, int key_off, int L,
+                               float softmax_scale, float *stats_out, void *ws, size_t ws_bytes,
+                               void *stream);
+hq_status hq_probe_merge_stats(const float *parts, int R, int nrows, float *stats_out,
+                               void *stream);
+hq_status hq_probe_shard_topk(const void *q_probe, int64_t q_head_stride, const void *k_shard,
+                              int B, int Hq, int Hkv, int P, int Ls, int D, int key_off, int L,
+                              int window, int k_vert, float softmax_scale, const float *stats,
+                              int32_t *cand_idx, float *cand_score, void *ws, size_t ws_bytes,
+                              void *stream);
+size_t hq_probe_merge_workspace_size(int B, int Hkv, int L, int window);
+hq_status hq_probe_merge_topk(const int32_t *cand_idx, const float *cand_score, int R, int B,
+                              int Hkv, int L, int window, int k_vert, int32_t *idx_out, void *ws,
+                              size_t ws_bytes, void *stream);
+
 /* ------------------------------------------------------------------------ */
 /* KV pack: build the hybrid cache (wiki summary, TL;DR: quantize the rest   */
 /* hard, no smoothing; blog, "What the authors tested": Key-4bit/Value-4bit). */

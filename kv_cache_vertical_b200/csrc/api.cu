@@ -108,6 +108,80 @@ hq_status hq_probe_vertical(const void *q_probe, int64_t q_head_stride, const vo
                                   (uint8_t *)ws, (cudaStream_t)stream));
 }
 
+static bool shard_args_ok(const void *q_probe, int64_t q_head_stride, const void *k, int B, int Hq,
+                          int Hkv, int P, int Ls, int D, int key_off, int L) {
+  return q_probe && k && B > 0 && Hq > 0 && Hkv > 0 && Hq % Hkv == 0 && P > 0 && P <= L &&
+         Ls > 0 && key_off >= 0 && (int64_t)key_off + Ls <= L && q_head_stride >= (int64_t)P * D;
+}
+
+size_t hq_probe_shard_workspace_size(int B, int Hq, int Hkv, int P, int Ls, int D, int k_vert) {
+  if (B <= 0 || !supported_G(Hq, Hkv) || P <= 0 || Ls <= 0 || k_vert < 0 || (D != 64 && D != 128))
+    return 0;
+  return probe_shard_ws_bytes(B, Hq, Hkv, P, Ls, D, k_vert);
+}
+
+hq_status hq_probe_shard_stats(const void *q_probe, int64_t q_head_stride, const void *k_shard,
+                               int B, int Hq, int Hkv, int P, int Ls, int D, int key_off, int L,
+                               float softmax_scale, float *stats_out, void *ws, size_t ws_bytes,
+                               void *stream) {
+  if (!stats_out || !shard_args_ok(q_probe, q_head_stride, k_shard, B, Hq, Hkv, P, Ls, D, key_off, L))
+    return HQ_ERR_INVALID_ARG;
+  if ((D != 64 && D != 128) || !supported_G(Hq, Hkv)) return HQ_ERR_UNSUPPORTED;
+  if (!aligned16(q_probe) || !aligned16(k_shard) || !aligned16(stats_out) || (q_head_stride * 2) % 16)
+    return HQ_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < probe_shard_ws_bytes(B, Hq, Hkv, P, Ls, D, 0)) return HQ_ERR_WORKSPACE;
+  return cuda_status(launch_probe_shard_stats(
+      (const __nv_bfloat16 *)q_probe, q_head_stride, (const __nv_bfloat16 *)k_shard, B, Hq, Hkv, P,
+      Ls, D, key_off, L, resolve_scale(softmax_scale, D), reinterpret_cast<float2 *>(stats_out),
+      (uint8_t *)ws, (cudaStream_t)stream));
+}
+
+hq_status hq_probe_merge_stats(const float *parts, int R, int nrows, float *stats_out,
+                               void *stream) {
+  if (!parts || !stats_out || R <= 0 || nrows <= 0) return HQ_ERR_INVALID_ARG;
+  if (!aligned16(parts) || !aligned16(stats_out)) return HQ_ERR_INVALID_ARG;
+  return cuda_status(launch_probe_merge_stats(reinterpret_cast<const float2 *>(parts), R, nrows,
+                                              reinterpret_cast<float2 *>(stats_out),
+                                              (cudaStream_t)stream));
+}
+
+hq_status hq_probe_shard_topk(const void *q_probe, int64_t q_head_stride, const void *k_shard,
+                              int B, int Hq, int Hkv, int P, int Ls, int D, int key_off, int L,
+                              int window, int k_vert, float softmax_scale, const float *stats,
+                              int32_t *cand_idx, float *cand_score, void *ws, size_t ws_bytes,
+                              void *stream) {
+  if (!shard_args_ok(q_probe, q_head_stride, k_shard, B, Hq, Hkv, P, Ls, D, key_off, L) || !stats ||
+      window < 0 || k_vert < 0 || k_vert > L - window || (k_vert > 0 && (!cand_idx || !cand_score)))
+    return HQ_ERR_INVALID_ARG;
+  if ((D != 64 && D != 128) || !supported_G(Hq, Hkv)) return HQ_ERR_UNSUPPORTED;
+  if (!aligned16(q_probe) || !aligned16(k_shard) || !aligned16(stats) || (q_head_stride * 2) % 16)
+    return HQ_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < probe_shard_ws_bytes(B, Hq, Hkv, P, Ls, D, k_vert)) return HQ_ERR_WORKSPACE;
+  return cuda_status(launch_probe_shard_topk(
+      (const __nv_bfloat16 *)q_probe, q_head_stride, (const __nv_bfloat16 *)k_shard, B, Hq, Hkv, P,
+      Ls, D, key_off, L, window, k_vert, resolve_scale(softmax_scale, D),
+      reinterpret_cast<const float2 *>(stats), cand_idx, cand_score, (uint8_t *)ws,
+      (cudaStream_t)stream));
+}
+
+size_t hq_probe_merge_workspace_size(int B, int Hkv, int L, int window) {
+  if (B <= 0 || Hkv <= 0 || L <= 0 || window < 0) return 0;
+  return probe_merge_ws_bytes(B, Hkv, L, window);
+}
+
+hq_status hq_probe_merge_topk(const int32_t *cand_idx, const float *cand_score, int R, int B,
+                              int Hkv, int L, int window, int k_vert, int32_t *idx_out, void *ws,
+                              size_t ws_bytes, void *stream) {
+  if (R <= 0 || B <= 0 || Hkv <= 0 || L <= 0 || window < 0 || k_vert < 0 || k_vert > L - window)
+    return HQ_ERR_INVALID_ARG;
+  if (k_vert == 0) return HQ_OK;
+  if (!cand_idx || !cand_score || !idx_out) return HQ_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < probe_merge_ws_bytes(B, Hkv, L, window)) return HQ_ERR_WORKSPACE;
+  return cuda_status(launch_probe_merge_topk(cand_idx, cand_score, R, B, Hkv, L, window, k_vert,
+                                             idx_out, (uint8_t *)ws, status_word(ws),
+                                             (cudaStream_t)stream));
+}
+
 hq_status hq_pack_kv(const void *k, const void *v, const int32_t *idx, int B, int Hkv, int L,
                      int D, int window, int k_vert, int bits, int group, const hq_kv_cache *out,
                      void *ws, size_t ws_bytes, void *stream) {

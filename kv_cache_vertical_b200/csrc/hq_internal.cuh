@@ -69,6 +69,23 @@ cudaError_t launch_probe(const __nv_bfloat16 *q_probe, int64_t q_head_stride,
                          const __nv_bfloat16 *k, int B, int Hq, int Hkv, int P, int L, int D,
                          int window, int k_vert, float scale, int32_t *idx_out, float *score_out,
                          uint8_t *ws, cudaStream_t s);
+// context split of the probe (keys [key_off, key_off + Ls) of an L-key context)
+size_t probe_shard_ws_bytes(int B, int Hq, int Hkv, int P, int Ls, int D, int k_vert);
+size_t probe_merge_ws_bytes(int B, int Hkv, int L, int window);
+cudaError_t launch_probe_shard_stats(const __nv_bfloat16 *q_probe, int64_t q_head_stride,
+                                     const __nv_bfloat16 *k, int B, int Hq, int Hkv, int P, int Ls,
+                                     int D, int key_off, int L, float scale, float2 *stats_out,
+                                     uint8_t *ws, cudaStream_t s);
+cudaError_t launch_probe_merge_stats(const float2 *parts, int R, int nrows, float2 *stats,
+                                     cudaStream_t s);
+cudaError_t launch_probe_shard_topk(const __nv_bfloat16 *q_probe, int64_t q_head_stride,
+                                    const __nv_bfloat16 *k, int B, int Hq, int Hkv, int P, int Ls,
+                                    int D, int key_off, int L, int window, int k_vert, float scale,
+                                    const float2 *stats, int32_t *cand_idx, float *cand_score,
+                                    uint8_t *ws, cudaStream_t s);
+cudaError_t launch_probe_merge_topk(const int32_t *cand_idx, const float *cand_score, int R, int B,
+                                    int Hkv, int L, int window, int k_vert, int32_t *idx_out,
+                                    uint8_t *ws, uint32_t *status, cudaStream_t s);
 
 bool decode_tma_supported(int D, int bits, int G);
 size_t decode_tma_ws_bytes(int B, int Hq, int Hkv, int n_lo, int n_hi, int bits);

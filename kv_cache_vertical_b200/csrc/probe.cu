@@ -24,6 +24,8 @@
 //      comes out ascending and ties go to the lower index.
 #include <float.h>
 
+#include <algorithm>
+
 #include "hq_internal.cuh"
 #include "warp_mma.cuh"
 
@@ -41,6 +43,7 @@ struct ProbeArgs {
   int64_t q_head_stride;
   const __nv_bfloat16 *k;
   int Hq, Hkv, P, L, G, R, nchunk;
+  int qpos0;                     // position of probe row 0 counted from key 0 (L - P unsplit)
   float scale_log2;              // softmax scale * log2(e)
   float2 *partial;               // [nbh, R, nchunk] (max, sum) in log2 domain
   const float2 *stats;           // [nbh, R] (max, 1/Z) in log2 domain
@@ -128,14 +131,16 @@ __global__ void __launch_bounds__(PWARPS * 32, 1) probe_qk(ProbeArgs a) {
     for (int rt = warp; rt < ntile_rows; rt += PWARPS) {
       if (!resident) load_q_frag<D>(a, b, kh, rt * 16, qa);
       const uint32_t(&q)[D / 16][4] = qa;
-      // Rows of this thread: rt*16 + r (+8).  Visible keys: j <= L - P + p.
+      // Rows of this thread: rt*16 + r (+8).  Visible keys: j <= qpos0 + p,
+      // and j < L (the zero-filled keys past the end never count, which
+      // matters when the probe rows lie beyond this key range).
       int lastj[2];
       bool valid[2];
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         const int row = rt * 16 + r + hf * 8;
         valid[hf] = row < a.R;
-        lastj[hf] = valid[hf] ? a.L - a.P + (row % a.P) : -1;
+        lastj[hf] = valid[hf] ? min(a.qpos0 + (row % a.P), a.L - 1) : -1;
       }
       float2 sx[2];                              // COLSUM: (max, 1/Z) of the two rows
       if (COLSUM)
@@ -233,10 +238,11 @@ __global__ void __launch_bounds__(PWARPS * 32, 1) probe_qk(ProbeArgs a) {
   }
 }
 
-// Row max / 1/Z from the per-stage partials (log2 domain): one warp per row,
-// lanes over the partials, merged in a fixed order.
+// Row max / 1/Z (or max / Z with invert = false) from the per-stage partials
+// (log2 domain): one warp per row, lanes over the partials, merged in a fixed
+// order.  A row that sees no key keeps max -FLT_MAX and Z = 0.
 __global__ void probe_row_stats(const float2 *__restrict__ partial, float2 *__restrict__ stats,
-                                int nrows, int nchunk) {
+                                int nrows, int nchunk, bool invert = true) {
   const int row = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= nrows) return;
@@ -249,7 +255,64 @@ __global__ void probe_row_stats(const float2 *__restrict__ partial, float2 *__re
   for (int c = lane; c < nchunk; c += 32) z += pr[c].y * exp2f(pr[c].x - m);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-  if (lane == 0) stats[row] = make_float2(m, 1.0f / z);
+  if (lane == 0) stats[row] = make_float2(m, invert ? 1.0f / z : z);
+}
+
+// Context split: merge the ranks' (max, Z) of every probe row into the
+// row's (max, 1/Z) over the whole context, ranks in a fixed order.
+__global__ void probe_merge_stats(const float2 *__restrict__ parts, int R, int nrows,
+                                  float2 *__restrict__ stats) {
+  const int row = blockIdx.x * blockDim.x + threadIdx.x;
+  if (row >= nrows) return;
+  float m = -FLT_MAX;
+  for (int r = 0; r < R; ++r) m = fmaxf(m, parts[(size_t)r * nrows + row].x);
+  float z = 0.f;
+  for (int r = 0; r < R; ++r) {
+    const float2 p = parts[(size_t)r * nrows + row];
+    if (p.y > 0.f) z += p.y * exp2f(p.x - m);
+  }
+  stats[row] = make_float2(m, 1.0f / z);
+}
+
+// Context split: a rank's top-k (local positions, ascending) as candidates in
+// context positions with their scores; slots past the rank's count hold -1.
+__global__ void probe_shard_candidates(const int32_t *__restrict__ local_idx, int kk, int k_vert,
+                                       const float *__restrict__ score, int Ls, int key_off,
+                                       int32_t *__restrict__ cand_idx, float *__restrict__ cand_score) {
+  const int bh = blockIdx.y, t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= k_vert) return;
+  const size_t o = (size_t)bh * k_vert + t;
+  if (t < kk) {
+    const int j = local_idx[(size_t)bh * kk + t];
+    cand_idx[o] = j + key_off;
+    cand_score[o] = score[(size_t)bh * Ls + j];
+  } else {
+    cand_idx[o] = -1;
+    cand_score[o] = -FLT_MAX;
+  }
+}
+
+// Context split: every rank's candidates into one dense score row per
+// (b, kv head) over the context's candidate positions (the rest -inf).
+__global__ void probe_fill(float *__restrict__ x, size_t n, float v) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+    x[i] = v;
+}
+__global__ void probe_scatter_candidates(const int32_t *__restrict__ cand_idx,
+                                         const float *__restrict__ cand_score, int R, int nbh,
+                                         int k_vert, int ncand, float *__restrict__ dense,
+                                         uint32_t *status) {
+  const size_t n = (size_t)R * nbh * k_vert;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+    const int bh = (int)((i / k_vert) % nbh);
+    const int j = cand_idx[i];
+    if (j < 0) continue;
+    if (j >= ncand) {                     // not a candidate position: a caller error
+      if (status) atomicOr(status, HQ_DEV_BAD_INDEX);
+      continue;
+    }
+    dense[(size_t)bh * ncand + j] = cand_score[i];
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -390,23 +453,11 @@ probe_topk(const float *__restrict__ score, int L, int ncand, int k, int32_t *__
   }
 }
 
-template <int D>
-cudaError_t launch_probe_t(ProbeArgs a, int nbh, int k_vert, int window, int32_t *idx,
-                           cudaStream_t s) {
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(probe_qk<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, probe_smem_bytes<D>()) != cudaSuccess ||
-        cudaFuncSetAttribute(probe_qk<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, probe_smem_bytes<D>()) != cudaSuccess)
-      return cudaErrorInvalidValue;
-    attr = true;
-  }
-  dim3 grid((a.L + KC - 1) / KC, nbh);
-  probe_qk<D, false><<<grid, PWARPS * 32, probe_smem_bytes<D>(), s>>>(a);
-  const int nrows = nbh * a.R;
-  probe_row_stats<<<(nrows + 7) / 8, 256, 0, s>>>(a.partial, const_cast<float2 *>(a.stats),   // a warp per row
-                                                      nrows, a.nchunk);
-  probe_qk<D, true><<<grid, PWARPS * 32, probe_smem_bytes<D>(), s>>>(a);
-  const int ncand = a.L - window;
+// Top-k of every (b, kv head) row of `score` (row stride L) over positions
+// [0, ncand): k indices, ascending, ties to the lower index.
+cudaError_t launch_topk(const float *score, int L, int ncand, int k, int nbh, int32_t *idx,
+                        cudaStream_t s) {
+  if (k <= 0 || nbh <= 0) return cudaSuccess;
   const size_t tk_smem = ncand <= TK_STAGE ? (size_t)(ncand + (ncand >> 5) + 1) * 4 : 0;
   static bool tk_attr = false;
   if (!tk_attr) {
@@ -415,8 +466,33 @@ cudaError_t launch_probe_t(ProbeArgs a, int nbh, int k_vert, int window, int32_t
       return cudaErrorInvalidValue;
     tk_attr = true;
   }
-  probe_topk<<<nbh, TK_THREADS, tk_smem, s>>>(a.score, a.L, ncand, k_vert, idx);
+  probe_topk<<<nbh, TK_THREADS, tk_smem, s>>>(score, L, ncand, k, idx);
   return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t probe_attr() {
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(probe_qk<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, probe_smem_bytes<D>()) != cudaSuccess ||
+        cudaFuncSetAttribute(probe_qk<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, probe_smem_bytes<D>()) != cudaSuccess)
+      return cudaErrorInvalidValue;
+    attr = true;
+  }
+  return cudaSuccess;
+}
+
+template <int D>
+cudaError_t launch_probe_t(ProbeArgs a, int nbh, int k_vert, int window, int32_t *idx,
+                           cudaStream_t s) {
+  if (probe_attr<D>() != cudaSuccess) return cudaErrorInvalidValue;
+  dim3 grid((a.L + KC - 1) / KC, nbh);
+  probe_qk<D, false><<<grid, PWARPS * 32, probe_smem_bytes<D>(), s>>>(a);
+  const int nrows = nbh * a.R;
+  probe_row_stats<<<(nrows + 7) / 8, 256, 0, s>>>(a.partial, const_cast<float2 *>(a.stats),   // a warp per row
+                                                      nrows, a.nchunk);
+  probe_qk<D, true><<<grid, PWARPS * 32, probe_smem_bytes<D>(), s>>>(a);
+  return launch_topk(a.score, a.L, a.L - window, k_vert, nbh, idx, s);
 }
 
 }  // namespace
@@ -444,6 +520,7 @@ cudaError_t launch_probe(const __nv_bfloat16 *q_probe, int64_t q_head_stride,
   a.Hkv = Hkv;
   a.P = P;
   a.L = L;
+  a.qpos0 = L - P;
   a.G = Hq / Hkv;
   a.R = a.G * P;
   a.nchunk = (L + KSUB - 1) / KSUB;
@@ -458,6 +535,114 @@ cudaError_t launch_probe(const __nv_bfloat16 *q_probe, int64_t q_head_stride,
   if (D == 128) return launch_probe_t<128>(a, (int)nbh, k_vert, window, idx_out, s);
   if (D == 64) return launch_probe_t<64>(a, (int)nbh, k_vert, window, idx_out, s);
   return cudaErrorInvalidValue;
+}
+
+// ---------------------------------------------------------------------------
+// Context split: the keys [key_off, key_off + Ls) of an L-key context on one
+// rank; the probe rows sit at context positions L - P + p.
+// ---------------------------------------------------------------------------
+size_t probe_shard_ws_bytes(int B, int Hq, int Hkv, int P, int Ls, int D, int k_vert) {
+  return align_up(probe_ws_bytes(B, Hq, Hkv, P, Ls, D) + (size_t)B * Hkv * k_vert * sizeof(int32_t), 256);
+}
+
+namespace {
+ProbeArgs shard_args(const __nv_bfloat16 *q_probe, int64_t q_head_stride, const __nv_bfloat16 *k,
+                     int B, int Hq, int Hkv, int P, int Ls, int key_off, int L, float scale,
+                     uint8_t *ws) {
+  ProbeArgs a;
+  a.qp = q_probe;
+  a.q_head_stride = q_head_stride;
+  a.k = k;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.P = P;
+  a.L = Ls;
+  a.qpos0 = L - P - key_off;
+  a.G = Hq / Hkv;
+  a.R = a.G * P;
+  a.nchunk = (Ls + KSUB - 1) / KSUB;
+  a.scale_log2 = scale * kLog2e;
+  const size_t nbh = (size_t)B * Hkv;
+  size_t off = kWsHeader;
+  a.partial = reinterpret_cast<float2 *>(ws + off);
+  off = align_up(off + nbh * a.R * a.nchunk * sizeof(float2), 256);
+  a.stats = reinterpret_cast<float2 *>(ws + off);
+  off = align_up(off + nbh * a.R * sizeof(float2), 256);
+  a.score = reinterpret_cast<float *>(ws + off);
+  return a;
+}
+}  // namespace
+
+cudaError_t launch_probe_shard_stats(const __nv_bfloat16 *q_probe, int64_t q_head_stride,
+                                     const __nv_bfloat16 *k, int B, int Hq, int Hkv, int P, int Ls,
+                                     int D, int key_off, int L, float scale, float2 *stats_out,
+                                     uint8_t *ws, cudaStream_t s) {
+  ProbeArgs a = shard_args(q_probe, q_head_stride, k, B, Hq, Hkv, P, Ls, key_off, L, scale, ws);
+  const int nbh = B * Hkv, nrows = nbh * a.R;
+  dim3 grid((Ls + KC - 1) / KC, nbh);
+  if (D == 128) {
+    if (probe_attr<128>() != cudaSuccess) return cudaErrorInvalidValue;
+    probe_qk<128, false><<<grid, PWARPS * 32, probe_smem_bytes<128>(), s>>>(a);
+  } else if (D == 64) {
+    if (probe_attr<64>() != cudaSuccess) return cudaErrorInvalidValue;
+    probe_qk<64, false><<<grid, PWARPS * 32, probe_smem_bytes<64>(), s>>>(a);
+  } else {
+    return cudaErrorInvalidValue;
+  }
+  probe_row_stats<<<(nrows + 7) / 8, 256, 0, s>>>(a.partial, stats_out, nrows, a.nchunk, false);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_probe_merge_stats(const float2 *parts, int R, int nrows, float2 *stats,
+                                     cudaStream_t s) {
+  probe_merge_stats<<<(nrows + 255) / 256, 256, 0, s>>>(parts, R, nrows, stats);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_probe_shard_topk(const __nv_bfloat16 *q_probe, int64_t q_head_stride,
+                                    const __nv_bfloat16 *k, int B, int Hq, int Hkv, int P, int Ls,
+                                    int D, int key_off, int L, int window, int k_vert, float scale,
+                                    const float2 *stats, int32_t *cand_idx, float *cand_score,
+                                    uint8_t *ws, cudaStream_t s) {
+  ProbeArgs a = shard_args(q_probe, q_head_stride, k, B, Hq, Hkv, P, Ls, key_off, L, scale, ws);
+  a.stats = stats;                                   // the whole context's (max, 1/Z)
+  const int nbh = B * Hkv;
+  int32_t *local_idx = reinterpret_cast<int32_t *>(ws + probe_ws_bytes(B, Hq, Hkv, P, Ls, D));
+  dim3 grid((Ls + KC - 1) / KC, nbh);
+  if (D == 128) {
+    if (probe_attr<128>() != cudaSuccess) return cudaErrorInvalidValue;
+    probe_qk<128, true><<<grid, PWARPS * 32, probe_smem_bytes<128>(), s>>>(a);
+  } else if (D == 64) {
+    if (probe_attr<64>() != cudaSuccess) return cudaErrorInvalidValue;
+    probe_qk<64, true><<<grid, PWARPS * 32, probe_smem_bytes<64>(), s>>>(a);
+  } else {
+    return cudaErrorInvalidValue;
+  }
+  // candidates of this rank: its keys before the context's window
+  const int ncand = std::max(0, std::min(Ls, L - window - key_off));
+  const int kk = std::min(k_vert, ncand);
+  cudaError_t e = launch_topk(a.score, Ls, ncand, kk, nbh, local_idx, s);
+  if (e != cudaSuccess) return e;
+  if (k_vert > 0)
+    probe_shard_candidates<<<dim3((k_vert + 255) / 256, nbh), 256, 0, s>>>(
+        local_idx, kk, k_vert, a.score, Ls, key_off, cand_idx, cand_score);
+  return cudaGetLastError();
+}
+
+size_t probe_merge_ws_bytes(int B, int Hkv, int L, int window) {
+  return align_up(kWsHeader + (size_t)B * Hkv * (size_t)std::max(0, L - window) * sizeof(float), 256);
+}
+
+cudaError_t launch_probe_merge_topk(const int32_t *cand_idx, const float *cand_score, int R, int B,
+                                    int Hkv, int L, int window, int k_vert, int32_t *idx_out,
+                                    uint8_t *ws, uint32_t *status, cudaStream_t s) {
+  const int nbh = B * Hkv, ncand = L - window;
+  if (k_vert <= 0 || ncand <= 0) return cudaSuccess;
+  float *dense = reinterpret_cast<float *>(ws + kWsHeader);
+  probe_fill<<<592, 256, 0, s>>>(dense, (size_t)nbh * ncand, -FLT_MAX);
+  probe_scatter_candidates<<<148, 256, 0, s>>>(cand_idx, cand_score, R, nbh, k_vert, ncand, dense,
+                                               status);
+  return launch_topk(dense, ncand, ncand, k_vert, nbh, idx_out, s);
 }
 
 }  // namespace hq

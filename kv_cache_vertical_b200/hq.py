@@ -56,6 +56,14 @@ _read_status = _sig("hq_read_device_status", _I, _P, _I, ctypes.POINTER(ctypes.c
 hq_probe_workspace_size = _sig("hq_probe_workspace_size", _SZ, _I, _I, _I, _I, _I, _I)
 _probe = _sig("hq_probe_vertical", _I, _P, ctypes.c_int64, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F,
               _P, _P, _P, _SZ, _P)
+hq_probe_shard_workspace_size = _sig("hq_probe_shard_workspace_size", _SZ, _I, _I, _I, _I, _I, _I, _I)
+_pshard_stats = _sig("hq_probe_shard_stats", _I, _P, ctypes.c_int64, _P, _I, _I, _I, _I, _I, _I, _I,
+                     _I, _F, _P, _P, _SZ, _P)
+_pmerge_stats = _sig("hq_probe_merge_stats", _I, _P, _I, _I, _P, _P)
+_pshard_topk = _sig("hq_probe_shard_topk", _I, _P, ctypes.c_int64, _P, _I, _I, _I, _I, _I, _I, _I,
+                    _I, _I, _I, _F, _P, _P, _P, _P, _SZ, _P)
+hq_probe_merge_workspace_size = _sig("hq_probe_merge_workspace_size", _SZ, _I, _I, _I, _I)
+_pmerge_topk = _sig("hq_probe_merge_topk", _I, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _SZ, _P)
 _pack = _sig("hq_pack_kv", _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I,
              ctypes.POINTER(hq_kv_cache), _P, _SZ, _P)
 hq_decode_workspace_size = _sig("hq_decode_workspace_size", _SZ, _I, _I, _I, _I, _I, _I, _I)
@@ -77,7 +85,9 @@ EXPORTED = ["hq_status_string", "hq_version", "hq_read_device_status", "hq_probe
             "hq_probe_vertical", "hq_pack_kv", "hq_decode_workspace_size", "hq_decode_attn",
             "hq_prefill_quant", "hq_prefill_workspace_size", "hq_prefill_attn",
             "hq_decode_attn_static", "hq_kv_append", "hq_decode_merge", "hq_prefill_quant_ex",
-            "hq_prefill_attn_ex"]
+            "hq_prefill_attn_ex", "hq_probe_shard_workspace_size", "hq_probe_shard_stats",
+            "hq_probe_merge_stats", "hq_probe_shard_topk", "hq_probe_merge_workspace_size",
+            "hq_probe_merge_topk"]
 
 HQ_ERR_SCRATCH_LIMIT = 7
 STATIC_SCRATCH_BYTES = 8 << 20
@@ -213,6 +223,33 @@ def hq_probe_vertical(q_probe, q_head_stride, k, B, Hq, Hkv, P, L, D, window, k_
                   ws.numel() if ws is not None else 0, _stream(stream)), "hq_probe_vertical")
 
 
+def hq_probe_shard_stats(q_probe, q_head_stride, k_shard, B, Hq, Hkv, P, Ls, D, key_off, L,
+                         softmax_scale, stats_out, ws, stream=None):
+    _check(_pshard_stats(_ptr(q_probe), int(q_head_stride), _ptr(k_shard), B, Hq, Hkv, P, Ls, D,
+                         key_off, L, float(softmax_scale), _ptr(stats_out), _ptr(ws),
+                         ws.numel() if ws is not None else 0, _stream(stream)), "hq_probe_shard_stats")
+
+
+def hq_probe_merge_stats(parts, R, nrows, stats_out, stream=None):
+    _check(_pmerge_stats(_ptr(parts), R, nrows, _ptr(stats_out), _stream(stream)),
+           "hq_probe_merge_stats")
+
+
+def hq_probe_shard_topk(q_probe, q_head_stride, k_shard, B, Hq, Hkv, P, Ls, D, key_off, L, window,
+                        k_vert, softmax_scale, stats, cand_idx, cand_score, ws, stream=None):
+    _check(_pshard_topk(_ptr(q_probe), int(q_head_stride), _ptr(k_shard), B, Hq, Hkv, P, Ls, D,
+                        key_off, L, window, k_vert, float(softmax_scale), _ptr(stats), _ptr(cand_idx),
+                        _ptr(cand_score), _ptr(ws), ws.numel() if ws is not None else 0,
+                        _stream(stream)), "hq_probe_shard_topk")
+
+
+def hq_probe_merge_topk(cand_idx, cand_score, R, B, Hkv, L, window, k_vert, idx_out, ws,
+                        stream=None):
+    _check(_pmerge_topk(_ptr(cand_idx), _ptr(cand_score), R, B, Hkv, L, window, k_vert,
+                        _ptr(idx_out), _ptr(ws), ws.numel() if ws is not None else 0,
+                        _stream(stream)), "hq_probe_merge_topk")
+
+
 def hq_pack_kv(k, v, idx, B, Hkv, L, D, window, k_vert, bits, group, cache: KVCache, ws=None,
                stream=None):
     st = cache.struct()
@@ -291,6 +328,78 @@ def probe_vertical(q_probe, k, window, k_vert, scale=0.0, want_scores=False, ws=
     hq_probe_vertical(q_probe, q_probe.stride(1), k, B, Hq, Hkv, P, L, D, window, k_vert, scale,
                       idx, score, ws)
     return (idx, score) if want_scores else idx
+
+
+def probe_context_plan(L: int, R: int):
+    """Contiguous key ranges [key_off, key_off + Ls) of an L-key context for R
+    ranks, as equal as possible (every rank gets at least one key when L >= R)."""
+    return [(L * r // R, L * (r + 1) // R - L * r // R) for r in range(R)]
+
+
+def probe_shard_stats(q_probe, k_shard, key_off, L, scale=0.0, ws=None):
+    """Pass 1 on one rank's keys: (max, Z) per probe row, f32 [B, Hkv, G*P, 2]."""
+    B, Hq, P, D = q_probe.shape
+    Hkv, Ls = k_shard.shape[1], k_shard.shape[2]
+    out = torch.empty(B, Hkv, (Hq // Hkv) * P, 2, dtype=torch.float32, device=k_shard.device)
+    if ws is None:
+        ws = workspace(hq_probe_shard_workspace_size(B, Hq, Hkv, P, Ls, D, 0), k_shard.device)
+    hq_probe_shard_stats(q_probe, q_probe.stride(1), k_shard, B, Hq, Hkv, P, Ls, D, key_off, L,
+                         scale, out, ws)
+    return out
+
+
+def probe_merge_stats(parts):
+    """parts: f32 [R, B, Hkv, rows, 2] (max, Z) -> the context's (max, 1/Z)."""
+    R = parts.shape[0]
+    nrows = parts[0].numel() // 2
+    out = torch.empty(parts.shape[1:], dtype=torch.float32, device=parts.device)
+    hq_probe_merge_stats(parts.contiguous(), R, nrows, out)
+    return out
+
+
+def probe_shard_topk(q_probe, k_shard, key_off, L, window, k_vert, stats, scale=0.0, ws=None):
+    """Pass 2 on one rank's keys with the context's row stats: the rank's best
+    k_vert candidate columns (context positions, -1 padded) and their scores."""
+    B, Hq, P, D = q_probe.shape
+    Hkv, Ls = k_shard.shape[1], k_shard.shape[2]
+    cand_idx = torch.empty(B, Hkv, k_vert, dtype=torch.int32, device=k_shard.device)
+    cand_score = torch.empty(B, Hkv, k_vert, dtype=torch.float32, device=k_shard.device)
+    if ws is None:
+        ws = workspace(hq_probe_shard_workspace_size(B, Hq, Hkv, P, Ls, D, k_vert), k_shard.device)
+    hq_probe_shard_topk(q_probe, q_probe.stride(1), k_shard, B, Hq, Hkv, P, Ls, D, key_off, L,
+                        window, k_vert, scale, stats.contiguous(), cand_idx, cand_score, ws)
+    return cand_idx, cand_score
+
+
+def probe_merge_topk(cand_idx, cand_score, L, window, ws=None):
+    """cand_idx / cand_score: [R, B, Hkv, k_vert] -> the context's index list."""
+    R, B, Hkv, k_vert = cand_idx.shape
+    idx = torch.empty(B, Hkv, k_vert, dtype=torch.int32, device=cand_idx.device)
+    if ws is None:
+        ws = workspace(hq_probe_merge_workspace_size(B, Hkv, L, window), cand_idx.device)
+    hq_probe_merge_topk(cand_idx.contiguous(), cand_score.contiguous(), R, B, Hkv, L, window,
+                        k_vert, idx, ws)
+    return idx
+
+
+def probe_context_parallel(q_probe, k_shard, key_off, L, window, k_vert, group=None, scale=0.0):
+    """The vertical-column probe with the context's keys split over the ranks
+    of `group` (torch.distributed): this rank holds keys [key_off, key_off +
+    k_shard.shape[2]).  Two all-gathers: the probe rows' partial (max, Z), then
+    every rank's top-k candidates.  Returns the context's index list on every
+    rank."""
+    import torch.distributed as dist
+    R = dist.get_world_size(group)
+    st = probe_shard_stats(q_probe, k_shard, key_off, L, scale)
+    parts = [torch.empty_like(st) for _ in range(R)]
+    dist.all_gather(parts, st, group=group)
+    stats = probe_merge_stats(torch.stack(parts))
+    ci, cs = probe_shard_topk(q_probe, k_shard, key_off, L, window, k_vert, stats, scale)
+    cis = [torch.empty_like(ci) for _ in range(R)]
+    css = [torch.empty_like(cs) for _ in range(R)]
+    dist.all_gather(cis, ci, group=group)
+    dist.all_gather(css, cs, group=group)
+    return probe_merge_topk(torch.stack(cis), torch.stack(css), L, window)
 
 
 def pack_kv(k, v, idx, window, bits=4, ws=None, with_pos=True, lo_cap=None,

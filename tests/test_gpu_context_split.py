@@ -90,3 +90,55 @@ def test_merge_kernel_against_numpy():
     ok[2, 3] = False
     ref_lse = m + torch.log(wgt.sum(0))
     assert torch.allclose(lse.cpu().double()[ok], ref_lse[ok], atol=1e-5)
+
+
+# ---------------------------------------------------------------------------
+# Context-split probe: each rank's keys through the shard entry points, the
+# ranks one after another on one GPU, merged by the merge entry points;
+# compared with the oracle's probe of the whole context (index sets equal
+# modulo ties) and with the single-GPU probe.
+# ---------------------------------------------------------------------------
+
+def run_probe_split(w: Workload, R: int):
+    from hq_testutil import assert_index_sets
+    H = hq()
+    x = make_inputs(w)
+    d = to_dev(x)
+    qp, k = d["q_probe"], d["k"]
+    plan = H.probe_context_plan(w.L, R)
+    parts = [H.probe_shard_stats(qp, k[:, :, o:o + n].contiguous(), o, w.L) for o, n in plan]
+    stats = H.probe_merge_stats(torch.stack(parts))
+    cand = [H.probe_shard_topk(qp, k[:, :, o:o + n].contiguous(), o, w.L, w.window, w.k_vert, stats)
+            for o, n in plan]
+    idx = H.probe_merge_topk(torch.stack([c[0] for c in cand]), torch.stack([c[1] for c in cand]),
+                             w.L, w.window)
+    one = H.probe_vertical(qp, k, w.window, w.k_vert)
+    torch.cuda.synchronize()
+    sc = oracle.probe_scores(x["q_probe"], x["k"], w.Hkv)
+    ref = oracle.topk(sc, w.window, w.k_vert)
+    assert_index_sets(idx.cpu().numpy(), ref, sc, w.window)
+    assert_index_sets(one.cpu().numpy(), ref, sc, w.window)
+    # every rank's candidates are context positions before the window, or -1
+    for (o, n), (ci, _) in zip(plan, cand):
+        c = ci.cpu().numpy()
+        v = c[c >= 0]
+        assert ((v >= o) & (v < min(o + n, w.L - w.window))).all()
+
+
+@pytest.mark.parametrize("R", [1, 2, 3])
+@pytest.mark.parametrize("D", [64, 128])
+def test_probe_split_matches_whole_context(R, D):
+    w = Workload("pcp", "decode", 2, 8, 2, D, 5003, 128, F5, 4, 600 + R + D)
+    run_probe_split(w, R)
+
+
+def test_probe_split_rank_without_candidates():
+    # 4 ranks over 300 keys (75 each) with a 100-key window: the last rank's
+    # keys all lie in the window, so it has no candidates, only row stats
+    w = Workload("pcp_w", "decode", 1, 4, 1, 128, 300, 100, F5, 4, 77)
+    run_probe_split(w, 4)
+
+
+def test_probe_split_llama8b_32k():
+    w = WORKLOADS["llama8b_decode_32k"]
+    run_probe_split(w, 4)
