@@ -211,3 +211,34 @@ def test_prefill_format_argument_checks(lib):
     assert call(D=64, fmt=1) == 2
     assert call(Hq=3, Hkv=1, fmt=1) == 2
     assert call(q=None) == 1
+
+
+def test_probe_split_argument_checks(lib):
+    # host checks of the context-split probe, before any launch
+    st = lib.hq_probe_shard_stats
+    st.restype = ctypes.c_int
+
+    def stats(Ls=100, key_off=0, L=300, P=64, q=FAKE, out=FAKE):
+        return st(q, ctypes.c_int64(64 * 128), FAKE, 1, 2, 1, P, Ls, 128, key_off, L,
+                  ctypes.c_float(0.0), out, FAKE, ctypes.c_size_t(1 << 30), None)
+    assert stats(q=None) == 1
+    assert stats(out=None) == 1
+    assert stats(key_off=250) == 1            # key range past the context
+    assert stats(Ls=0) == 1
+    assert stats(P=301) == 1                  # more probe rows than context
+    tk = lib.hq_probe_shard_topk
+    tk.restype = ctypes.c_int
+
+    def topk(k_vert=10, window=64, cand=FAKE):
+        return tk(FAKE, ctypes.c_int64(64 * 128), FAKE, 1, 2, 1, 64, 100, 128, 0, 300, window,
+                  k_vert, ctypes.c_float(0.0), FAKE, cand, FAKE, FAKE, ctypes.c_size_t(1 << 30), None)
+    assert topk(k_vert=237) == 1              # k_vert > L - window
+    assert topk(cand=None) == 1
+    mg = lib.hq_probe_merge_topk
+    mg.restype = ctypes.c_int
+    assert mg(FAKE, FAKE, 0, 1, 1, 300, 64, 10, FAKE, FAKE, ctypes.c_size_t(1 << 30), None) == 1
+    assert mg(FAKE, FAKE, 2, 1, 1, 300, 64, 10, FAKE, None, ctypes.c_size_t(0), None) == 3
+    assert mg(None, None, 2, 1, 1, 300, 64, 0, None, None, ctypes.c_size_t(0), None) == 0
+    ms = lib.hq_probe_merge_stats
+    ms.restype = ctypes.c_int
+    assert ms(FAKE, 0, 10, FAKE, None) == 1
