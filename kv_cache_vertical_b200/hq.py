@@ -390,11 +390,23 @@ def probe_context_parallel(q_probe, k_shard, key_off, L, window, k_vert, group=N
     rank."""
     import torch.distributed as dist
     R = dist.get_world_size(group)
-    st = probe_shard_stats(q_probe, k_shard, key_off, L, scale)
+    B, Hq, P, D = q_probe.shape
+    Hkv = k_shard.shape[1]
+    empty = k_shard.shape[2] == 0          # more ranks than keys: this rank holds none
+    if empty:
+        st = torch.zeros(B, Hkv, (Hq // Hkv) * P, 2, dtype=torch.float32, device=q_probe.device)
+        st[..., 0] = -torch.finfo(torch.float32).max
+    else:
+        st = probe_shard_stats(q_probe, k_shard, key_off, L, scale)
     parts = [torch.empty_like(st) for _ in range(R)]
     dist.all_gather(parts, st, group=group)
     stats = probe_merge_stats(torch.stack(parts))
-    ci, cs = probe_shard_topk(q_probe, k_shard, key_off, L, window, k_vert, stats, scale)
+    if empty:
+        ci = torch.full((B, Hkv, k_vert), -1, dtype=torch.int32, device=q_probe.device)
+        cs = torch.full((B, Hkv, k_vert), -torch.finfo(torch.float32).max, dtype=torch.float32,
+                        device=q_probe.device)
+    else:
+        ci, cs = probe_shard_topk(q_probe, k_shard, key_off, L, window, k_vert, stats, scale)
     cis = [torch.empty_like(ci) for _ in range(R)]
     css = [torch.empty_like(cs) for _ in range(R)]
     dist.all_gather(cis, ci, group=group)

@@ -156,3 +156,13 @@ def test_probe_plan_and_split_equal_the_whole_context(R):
     cand = [shard_candidates_np(score[:, :, o:o + n], o, w.L, w.window, w.k_vert) for o, n in plan]
     idx = merge_candidates_np([c[0] for c in cand], [c[1] for c in cand], w.L, w.window, w.k_vert)
     assert np.array_equal(idx, oracle.topk(full, w.window, w.k_vert))
+
+
+def test_probe_plan_with_more_ranks_than_keys():
+    # ranks beyond the keys get empty ranges; the ranges still tile [0, L)
+    for L, R in [(3, 5), (1, 2), (7, 7), (10, 3)]:
+        plan = hq.probe_context_plan(L, R)
+        assert len(plan) == R and sum(n for _, n in plan) == L
+        pos = [o + i for o, n in plan for i in range(n)]
+        assert pos == list(range(L))
+        assert sum(1 for _, n in plan if n == 0) == max(0, R - L)
