@@ -1,8 +1,10 @@
-"""GPU parity of the context-split decode, its ranks run one after another on
-one GPU: each part of the plan is decoded through a row view of one packed
-cache, the parts are merged by hq_decode_merge, and the result is compared
-with the oracle's decode of the whole cache (the CUDA path's cache is the
-oracle's, bit for bit, as the pack tests show)."""
+"""GPU parity of the context-split paths, their ranks run one after another on
+one GPU.  Decode: each part of the plan is decoded through a row view of one
+packed cache, the parts are merged by hq_decode_merge, and the result is
+compared with the oracle's decode of the whole cache (the CUDA path's cache is
+the oracle's, bit for bit, as the pack tests show).  Probe: each rank's keys
+go through the shard entry points, the merges pick the context's columns, and
+the index lists are compared with the oracle's whole-context probe."""
 import numpy as np
 import pytest
 import torch
