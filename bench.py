@@ -35,7 +35,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from kv_cache_vertical_b200.synth import WORKLOADS, make_inputs  # noqa: E402
+from kv_cache_vertical_b200.synth import WORKLOADS, make_inputs, make_inputs_device  # noqa: E402
 
 METRIC = "hybrid decode attn HBM TB/s (% of peak); hybrid prefill TFLOPS (% of peak)"
 WL = WORKLOADS["llama8b_prefill_32k"]          # prompt; decode uses the same layer
@@ -244,6 +244,7 @@ def run_hq(args, rank, world, dev):
     d2h = out_p.numel() * 4 + out_d.numel() * 4
 
     loop = decode_loop(H, w, q, k, v, q_dec, dev, stream, world)
+    dconf = decode_configs(H, dev, stream, world, rank)
     graph = decode_graph(H, w, q_dec, cache, out_d, ws_dec, dev, world)
     fp8 = fp8_leg(H, w, q, k, v, idx, q_dec, dev, stream, world)
     i8_tops = int8_gemm_peak(dev)
@@ -255,7 +256,58 @@ def run_hq(args, rank, world, dev):
     return dict(per=per, total_ms=max_over_ranks(total_ms / args.steps, world, dev), dbytes=dbytes,
                 i8=i8_ops, bf=bf_flops, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, clocks=clocks,
                 kpad=(kv + 63) // 64 * 64, w=w, loop=loop, fp8=fp8, i8_tops=i8_tops, graph=graph,
-                idx=idx_np)
+                idx=idx_np, dconf=dconf)
+
+
+# The decode workloads timed after the steps, each on its own full-size cache.
+DECODE_CONFIGS = ("llama8b_decode_32k", "batched_decode_128k_int4", "batched_decode_128k_int8",
+                  "70b_decode_64k")
+
+
+def decode_configs(H, dev, stream, world, rank, reps=15):
+    """Decode attention alone on every decode workload of the specification,
+    at full size: inputs drawn on the device (same recipe as the parity
+    inputs), the vertical set from the GPU probe, the cache from the GPU
+    pack; then `reps` timed calls (two untimed first), the L2 flushed before
+    every call, CUDA events on the launching stream; median and best."""
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    pk = peaks()
+    res = {}
+    for name in DECODE_CONFIGS:
+        w = WORKLOADS[name]
+        x = make_inputs_device(w, dev, seed_offset=rank)
+        idx = H.probe_vertical(x["q_probe"], x["k"], w.window, w.k_vert)
+        cache = H.pack_kv(x["k"], x["v"], idx, w.window, w.bits, with_pos=False)
+        q = x["q"]
+        del x
+        ws = H.workspace(H.hq_decode_workspace_size(w.B, w.Hq, w.Hkv, w.D, cache.n_lo, cache.n_hi,
+                                                    w.bits), dev)
+        out = torch.empty(w.B, w.Hq, w.D, dtype=torch.float32, device=dev)
+        barrier(world)
+        ts = []
+        for i in range(reps + 2):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            H.hq_decode_attn(q, cache, w.B, w.Hq, w.Hkv, w.D, 0.0, out, None, ws)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            if i >= 2:
+                ts.append(e0.elapsed_time(e1) * 1e3)
+        med = max_over_ranks(float(np.median(ts)), world, dev)
+        best = max_over_ranks(min(ts), world, dev)
+        nb = decode_bytes(w.B, w.Hq, w.Hkv, w.D, cache.n_lo, cache.n_hi, w.bits)
+        res[name] = {"B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "window": w.window,
+                     "vertical_frac": float(w.frac), "kv_bits": w.bits,
+                     "algorithmic_bytes": nb, "us_median": med, "us_best": best,
+                     "gbs": nb / (med * 1e-6) / 1e9, "frac": nb / (med * 1e-6) / 1e9 / pk["hbm_gbs"],
+                     "frac_of_8TBs": nb / (med * 1e-6) / 8e12}
+        del cache, ws, out, q, idx
+        torch.cuda.empty_cache()
+    res["note"] = (f"decode alone, median of {reps} calls, L2 flushed (256 MB write) before each; "
+                   "frac = algorithmic bytes / median time / measured HBM copy peak; inputs drawn "
+                   "on the device (make_inputs_device)")
+    return res
 
 
 def decode_graph(H, w, q_dec, cache, out, ws, dev, world, n=50, reps=7):
@@ -620,6 +672,8 @@ def main():
         # token-by-token decode after the timed steps: cache maintenance + attention
         "decode_loop": r["loop"],
         "decode_graph": r["graph"],
+        # decode alone on every decode workload of the specification (full size)
+        "decode_configs": r["dconf"],
         # the FP8 (E4M3) low-bit format on the same layer, after the timed steps
         "fp8": {"prefill_ms": r["fp8"]["prefill_ms"],
                 "prefill_frac": t_star * 1e3 / r["fp8"]["prefill_ms"],
@@ -631,10 +685,13 @@ def main():
                 "note": "prefill: FP8 QK at the INT8 rate (nominal FP8 = INT8 on B200), same T*; "
                         "decode: E4M3 codes + fp16 scales, median of 5, L2 flushed"},
         "e2e": {"value": r["dbytes"] / (r["e2e_ms"] * 1e-3) / 1e12 * world, "unit": "TB/s",
-                "ms_per_step": r["e2e_ms"], "h2d_bytes_per_step": r["h2d"],
-                "d2h_bytes_per_step": r["d2h"],
-                "note": "decode bytes / whole-step time with pinned-host inputs copied in and "
-                        "the prefill + decode outputs copied back"},
+                "ms_per_step": r["e2e_ms"],
+                "prompt_tokens_per_s": w.B * w.L / (r["e2e_ms"] * 1e-3) * world,
+                "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
+                "note": "value = decode bytes / whole-step time (the metric's unit); ms_per_step "
+                        "and prompt_tokens_per_s are the same step: pinned-host Q/K/V copied in, "
+                        "probe + prefill + pack + decode, the prefill and decode outputs copied "
+                        "back"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": r["clocks"],
     }

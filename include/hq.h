@@ -37,9 +37,11 @@
  *     launch error (cudaGetLastError).  Checks made on the device (index
  *     lists out of order or out of range; waits that ran out) never trap:
  *     they skip the offending access and set a bit in the device status word.
- *   Supported shapes: D in {64, 128}; Hq % Hkv == 0 with Hq / Hkv <= 8;
- *     KV bits in {4, 8}; quantization group 32.  Others return
- *     HQ_ERR_UNSUPPORTED.  There is no CPU path.
+ *   Supported shapes: D in {64, 128}; Hq % Hkv == 0 with Hq / Hkv in
+ *     {1, 2, 4, 8}; KV bits in {4, 8}; quantization group 32; the prefill
+ *     attention D = 128 with Hq / Hkv in {2, 4, 8} (hq_prefill_supported).
+ *     Others return HQ_ERR_UNSUPPORTED.  There is no CPU path and each
+ *     operation has exactly one kernel per shape.
  */
 #ifndef HQ_H
 #define HQ_H
@@ -267,8 +269,10 @@ hq_status hq_decode_merge(const float *part_out, const float *part_lse, int R, i
  * Its scratch is one file-scope device array of HQ_STATIC_SCRATCH_BYTES that
  * every GPU loading the library holds until the process exits.
  *   - The first call on a device looks up that array's device address (with
- *     that device current) and caches it; make that first call before any
- *     stream capture begins.
+ *     that device current) and caches it with the current CUDA context; make
+ *     that first call before any stream capture begins.  After a device reset
+ *     (cudaDeviceReset) the next call sees a new context and looks the
+ *     address up again, so it too must come before any capture.
  *   - Every call shares the one array and leaves its contents behind; each call
  *     first clears (cudaMemsetAsync on `stream`) the part that must start at
  *     zero.  Calls whose work overlaps on the GPU (different streams, or graph
@@ -281,6 +285,18 @@ hq_status hq_decode_merge(const float *part_out, const float *part_lse, int R, i
 hq_status hq_decode_attn_static(const void *q, const hq_kv_cache *cache, int B, int Hq, int Hkv,
                                 int D, float softmax_scale, float *out, float *lse_out,
                                 void *stream);
+
+/*
+ * The device status word of the fixed scratch array (its first 4 bytes), the
+ * counterpart of hq_read_device_status for hq_decode_attn_static: the OR of
+ * the HQ_DEV_* bits raised by the last hq_decode_attn_static call on the
+ * current device (HQ_DEV_TIMEOUT when a bounded wait ran out and the output
+ * is incomplete).  Each hq_decode_attn_static call clears the word before it
+ * launches, so read it after the call whose result you check and before the
+ * next one.  Synchronizes `stream`; `clear` != 0 resets the word afterwards.
+ * Allocates nothing.
+ */
+hq_status hq_read_static_status(int clear, uint32_t *status_out, void *stream);
 
 /* ------------------------------------------------------------------------ */
 /* Decode cache maintenance (wiki summary, TL;DR: in decode the same rule    */
@@ -352,6 +368,18 @@ hq_status hq_prefill_quant_ex(const void *q, const void *k, const int32_t *idx, 
  *   out: f32 [B, Hq, N, D].  The workspace holds the pre-pass output.
  */
 size_t hq_prefill_workspace_size(int B, int Hq, int Hkv, int N, int D, int k_vert);
+/*
+ * The prefill attention runs on one kernel, written for the 5th-generation
+ * tensor cores: head_dim 128 and an even number of query heads per KV head
+ * (a CTA serves two query heads that share their key and value tiles).
+ * Other shapes (D = 64, Hq == Hkv) return HQ_ERR_UNSUPPORTED from
+ * hq_prefill_attn / hq_prefill_attn_ex, and so does a device on which the
+ * compiled kernel cannot run as built; nothing is launched then.  This query
+ * answers HQ_OK exactly when a prefill call of that shape and low-part format
+ * (HQ_KV_INT or HQ_KV_FP8) will run that kernel on the current device.  (The
+ * pre-pass hq_prefill_quant / _ex also takes D = 64 and any G.)
+ */
+hq_status hq_prefill_supported(int D, int Hq, int Hkv, int low_fmt);
 hq_status hq_prefill_attn(const void *q, const void *k, const void *v, const int32_t *idx, int B,
                           int Hq, int Hkv, int N, int D, int window, int k_vert,
                           float softmax_scale, float *out, void *ws, size_t ws_bytes,
@@ -360,8 +388,7 @@ hq_status hq_prefill_attn(const void *q, const void *k, const void *v, const int
  * The same with a choice of low-part format (HQ_KV_INT: the INT8 low part
  * above; HQ_KV_FP8: the E4M3 codes of hq_prefill_quant_ex, whose low logit is
  * the fp32-accumulated dot product of the E4M3 values times sq[i] and the
- * key block's scale).  HQ_KV_FP8 needs the tcgen05 path (D = 128, an even
- * number of query heads per KV head), else HQ_ERR_UNSUPPORTED.
+ * key block's scale).
  */
 hq_status hq_prefill_attn_ex(const void *q, const void *k, const void *v, const int32_t *idx,
                              int B, int Hq, int Hkv, int N, int D, int window, int k_vert,

@@ -20,6 +20,13 @@ bool supported_G(int Hq, int Hkv) {
 
 float resolve_scale(float s, int D) { return s == 0.0f ? 1.0f / sqrtf((float)D) : s; }
 
+// Shapes and formats the prefill attention takes: the tcgen05 kernel is
+// written for head_dim 128 and a CTA serves two query heads of one KV head.
+bool prefill_shape_ok(int D, int Hq, int Hkv, int low_fmt) {
+  return D == 128 && supported_G(Hq, Hkv) && (Hq / Hkv) % 2 == 0 &&
+         (low_fmt == HQ_KV_INT || low_fmt == HQ_KV_FP8);
+}
+
 hq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? HQ_OK : HQ_ERR_CUDA; }
 
 uint32_t *status_word(void *ws) { return ws ? reinterpret_cast<uint32_t *>(ws) : nullptr; }
@@ -295,6 +302,11 @@ hq_status hq_prefill_quant(const void *q, const void *k, const int32_t *idx, int
                              stream);
 }
 
+hq_status hq_prefill_supported(int D, int Hq, int Hkv, int low_fmt) {
+  if (!prefill_shape_ok(D, Hq, Hkv, low_fmt)) return HQ_ERR_UNSUPPORTED;
+  return prefill_tc_supported(D, Hq, Hkv) ? HQ_OK : HQ_ERR_UNSUPPORTED;
+}
+
 size_t hq_prefill_workspace_size(int B, int Hq, int Hkv, int N, int D, int k_vert) {
   if (B <= 0 || !supported_G(Hq, Hkv) || N <= 0 || (D != 64 && D != 128) || k_vert < 0) return 0;
   return prefill_ws_bytes(B, Hq, Hkv, N, D, k_vert);
@@ -308,13 +320,14 @@ hq_status hq_prefill_attn_ex(const void *q, const void *k, const void *v, const 
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || N <= 0 || window < 0 || k_vert < 0 ||
       k_vert > N - (window < N ? window : N))
     return HQ_ERR_INVALID_ARG;
-  if ((D != 64 && D != 128) || !supported_G(Hq, Hkv)) return HQ_ERR_UNSUPPORTED;
-  if (low_fmt != HQ_KV_INT && (low_fmt != HQ_KV_FP8 || !prefill_tc_supported(D, Hq, Hkv)))
-    return HQ_ERR_UNSUPPORTED;
+  if (!prefill_shape_ok(D, Hq, Hkv, low_fmt)) return HQ_ERR_UNSUPPORTED;
   const void *ptrs[] = {q, k, v, out};
   for (const void *p : ptrs)
     if (!aligned16(p)) return HQ_ERR_INVALID_ARG;
   if (!ws || ws_bytes < prefill_ws_bytes(B, Hq, Hkv, N, D, k_vert)) return HQ_ERR_WORKSPACE;
+  // the compiled tensor-core kernel must be usable on this device (register
+  // count, shared memory): otherwise nothing is launched
+  if (!prefill_tc_supported(D, Hq, Hkv)) return HQ_ERR_UNSUPPORTED;
   return cuda_status(launch_prefill((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k,
                                     (const __nv_bfloat16 *)v, idx, B, Hq, Hkv, N, D, window,
                                     k_vert, resolve_scale(softmax_scale, D), low_fmt, out,

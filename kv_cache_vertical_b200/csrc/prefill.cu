@@ -10,31 +10,24 @@
 // Q scale and per-64-key-block K scale; one online softmax covers both; P.V
 // takes fp16 P and V (V converted exactly from bf16) with fp32 accumulation.
 //
-// Pre-pass (P4): INT8 codes for Q and K, fp16 V, a compact bf16 K / fp16 V copy
-// of the vertical rows (so vertical tiles are dense loads, not gathers), their
-// positions, and a per-64-key bitmap of vertical positions.
-//
-// Main kernel: FA2-style, one CTA per (64-query tile, head, batch), 4 warps of
-// 16 rows, warp-level tensor-core MMAs (s8 m16n8k32 for the low QK tiles, bf16
-// m16n8k16 for the window / vertical QK tiles, f16 m16n8k16 for P.V).  For
-// query tile qt the key tiles are: 64-key tiles kt < qt entirely below the
-// window band (INT8 only, vertical columns masked out), the band tiles that
-// meet the window (INT8 and bf16 both computed, each element takes the one its
-// class asks for), and the compact vertical tiles (bf16, key v counted only for
-// rows with v <= i - W, so every pair is counted exactly once).
+// Pre-pass (P4): INT8 (or E4M3) codes for Q per row and for the remaining
+// (non-vertical) keys per 64 of them, fp16 V in position order and compacted
+// like the remaining keys, and a compact bf16 K / fp16 V copy of the vertical
+// rows with their positions (so vertical tiles are dense TMA loads, not
+// gathers).  The attention kernel that consumes them is prefill_tc.cu's
+// (tcgen05, head_dim 128, an even number of query heads per KV head); other
+// shapes are rejected on the host.
 #include <float.h>
 #include <limits.h>
 
 #include <cuda_fp8.h>
 
 #include "hq_internal.cuh"
-#include "warp_mma.cuh"
 
 namespace hq {
 namespace {
 
 constexpr int TILE = 64;        // queries per CTA, keys per tile, K-scale block
-constexpr int FWARPS = 4;
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ---------------------------------------------------------------------------
@@ -323,278 +316,6 @@ __global__ void gather_vertical(const __nv_bfloat16 *__restrict__ k, const __hal
   if (t == 0) kv_pos[(size_t)bh * kpad + r] = pos;
 }
 
-// ---------------------------------------------------------------------------
-// Main kernel (warp-level MMA version)
-// ---------------------------------------------------------------------------
-struct PrefillArgs {
-  const __nv_bfloat16 *q, *k;
-  const int8_t *qi8, *ki8;       // ki8: remaining keys [nbh, nr, D]
-  const float *sq, *sk;          // sk: per 64 remaining keys [nbh, nblk_r]
-  const __half *vh;              // fp16 V in position order [nbh, N, D]
-  const __half *vc;              // fp16 V of the remaining keys [nbh, nr, D]
-  const __nv_bfloat16 *vk;       // compact vertical K [nbh, kpad, D]
-  const __half *vv;              // compact vertical V
-  const int32_t *idx;            // [nbh, k_vert]
-  float *out;
-  int Hq, Hkv, G, N, window, k_vert, kpad, nr, nblk_r;
-  float scale_log2;
-};
-
-// Remaining (non-vertical) keys at positions <= x.
-__device__ __forceinline__ int remaining_upto(const int32_t *id, int k_vert, int x) {
-  return x < 0 ? 0 : x + 1 - upper_bound_i32(id, k_vert, x);
-}
-
-template <int D>
-struct Smem {
-  uint4 ki8[TILE * D / 16];      // 64 keys x D bytes
-  uint4 kbf[TILE * D / 8];       // 64 keys x D bf16
-  uint4 vh[TILE * D / 8];        // 64 keys x D fp16
-};
-
-// Smem index of 16-byte chunk `ch` of row `row` in a tile with CH chunks per
-// row: the chunk index is XOR-swizzled by the low row bits so that the eight
-// row addresses of one ldmatrix hit distinct bank groups.
-template <int CH>
-__device__ __forceinline__ int swz(int row, int ch) {
-  return row * CH + (ch ^ (row & (CH >= 8 ? 7 : CH - 1)));
-}
-
-// Copy a [rows x RB bytes] tile (rows at stride RB in global) into smem with
-// the 16-byte chunk index XOR-swizzled by (row & 7); rows >= nvalid are zero.
-template <int RB>
-__device__ __forceinline__ void load_tile(uint4 *dst, const uint8_t *src, int nvalid) {
-  constexpr int CH = RB / 16;
-  for (int t = threadIdx.x; t < TILE * CH; t += FWARPS * 32) {
-    const int row = t / CH, ch = t % CH;
-    uint4 val = make_uint4(0, 0, 0, 0);
-    if (row < nvalid) val = *reinterpret_cast<const uint4 *>(src + (size_t)row * RB + ch * 16);
-    dst[swz<CH>(row, ch)] = val;
-  }
-}
-
-template <int D>
-__global__ void __launch_bounds__(FWARPS * 32)
-prefill_mma(PrefillArgs a) {
-  constexpr int CH16 = D / 8;     // 16-byte chunks in a 16-bit row
-  constexpr int CH8 = D / 16;     // 16-byte chunks in an 8-bit row
-  constexpr int NT = TILE / 8;    // 8-key n-tiles per key tile
-  __shared__ Smem<D> sm;
-  const int ntiles = (a.N + TILE - 1) / TILE;
-  const int qt = ntiles - 1 - blockIdx.x;  // heaviest tiles first
-  const int h = blockIdx.y, b = blockIdx.z;
-  const int kh = h / a.G;
-  const size_t bh = (size_t)b * a.Hkv + kh;
-  const size_t bhq = (size_t)b * a.Hq + h;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = lane >> 2, c = lane & 3;
-  const int row0 = qt * TILE + warp * 16;
-  const int rows[2] = {row0 + r, row0 + r + 8};
-  const int W = a.window;
-
-  // Q fragments: bf16 (m16n8k16 A) and INT8 (m16n8k32 A), rows r and r+8.
-  uint32_t qb[D / 16][4], qi[D / 32][4];
-  float sqr[2];
-#pragma unroll
-  for (int hf = 0; hf < 2; ++hf) {
-    const bool ok = rows[hf] < a.N;
-    const uint32_t *pb = reinterpret_cast<const uint32_t *>(a.q + (bhq * a.N + rows[hf]) * D);
-    const uint32_t *pi = reinterpret_cast<const uint32_t *>(a.qi8 + (bhq * a.N + rows[hf]) * D);
-#pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks) {
-      qb[ks][hf] = ok ? pb[ks * 8 + c] : 0u;
-      qb[ks][hf + 2] = ok ? pb[ks * 8 + 4 + c] : 0u;
-    }
-#pragma unroll
-    for (int ks = 0; ks < D / 32; ++ks) {
-      qi[ks][hf] = ok ? pi[ks * 8 + c] : 0u;
-      qi[ks][hf + 2] = ok ? pi[ks * 8 + 4 + c] : 0u;
-    }
-    sqr[hf] = ok ? a.sq[bhq * a.N + rows[hf]] * a.scale_log2 : 0.f;
-  }
-
-  float o[D / 8][4];
-#pragma unroll
-  for (int nt = 0; nt < D / 8; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
-  float m[2] = {-1e30f, -1e30f}, l[2] = {0.f, 0.f};
-
-  // S (16 x 64) -> online softmax -> O += P V for the tile in smem.
-  auto softmax_pv = [&](float (&s)[NT][4]) {
-    float mx[2] = {m[0], m[1]};
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      mx[0] = fmaxf(mx[0], fmaxf(s[nt][0], s[nt][1]));
-      mx[1] = fmaxf(mx[1], fmaxf(s[nt][2], s[nt][3]));
-    }
-#pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
-      mx[hf] = fmaxf(mx[hf], __shfl_xor_sync(0xffffffffu, mx[hf], 1));
-      mx[hf] = fmaxf(mx[hf], __shfl_xor_sync(0xffffffffu, mx[hf], 2));
-    }
-    const float al[2] = {exp2f(m[0] - mx[0]), exp2f(m[1] - mx[1])};
-    m[0] = mx[0];
-    m[1] = mx[1];
-    uint32_t pa[NT / 2][4];
-    float rs[2] = {0.f, 0.f};
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const float p0 = exp2f(s[nt][0] - mx[0]), p1 = exp2f(s[nt][1] - mx[0]);
-      const float p2 = exp2f(s[nt][2] - mx[1]), p3 = exp2f(s[nt][3] - mx[1]);
-      rs[0] += p0 + p1;
-      rs[1] += p2 + p3;
-      pa[nt / 2][(nt & 1) * 2 + 0] = pack_f16x2(p0, p1);
-      pa[nt / 2][(nt & 1) * 2 + 1] = pack_f16x2(p2, p3);
-    }
-    l[0] = l[0] * al[0] + rs[0];
-    l[1] = l[1] * al[1] + rs[1];
-#pragma unroll
-    for (int nt = 0; nt < D / 8; ++nt) {
-      o[nt][0] *= al[0];
-      o[nt][1] *= al[0];
-      o[nt][2] *= al[1];
-      o[nt][3] *= al[1];
-    }
-#pragma unroll
-    for (int kk = 0; kk < NT / 2; ++kk) {
-#pragma unroll
-      for (int dp = 0; dp < D / 16; ++dp) {
-        // V rows kk*16 .. +15, d chunks 2dp, 2dp+1 -> B frags of n-tiles 2dp, 2dp+1
-        const int key = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-        const int ch = dp * 2 + (lane >> 4);
-        uint32_t vb[4];
-        ldsm_x4_t(vb, smem_u32(&sm.vh[swz<CH16>(key, ch)]));
-        mma_f16_16816(o[2 * dp], pa[kk], vb[0], vb[1]);
-        mma_f16_16816(o[2 * dp + 1], pa[kk], vb[2], vb[3]);
-      }
-    }
-  };
-
-  auto qk_int8 = [&](float (&s)[NT][4], float ks_scale) {
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      int acc[4] = {0, 0, 0, 0};
-#pragma unroll
-      for (int kp = 0; kp < D / 64; ++kp) {
-        const int key = nt * 8 + (lane & 7);
-        const int ch = kp * 4 + (lane >> 3);
-        uint32_t kb[4];
-        ldsm_x4(kb, smem_u32(&sm.ki8[swz<CH8>(key, ch)]));
-        mma_s8_16832(acc, qi[2 * kp], kb[0], kb[1]);
-        mma_s8_16832(acc, qi[2 * kp + 1], kb[2], kb[3]);
-      }
-      s[nt][0] = (float)acc[0] * (sqr[0] * ks_scale);
-      s[nt][1] = (float)acc[1] * (sqr[0] * ks_scale);
-      s[nt][2] = (float)acc[2] * (sqr[1] * ks_scale);
-      s[nt][3] = (float)acc[3] * (sqr[1] * ks_scale);
-    }
-  };
-
-  auto qk_bf16 = [&](float (&s)[NT][4]) {
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int kp = 0; kp < D / 32; ++kp) {
-        const int key = nt * 8 + (lane & 7);
-        const int ch = kp * 4 + (lane >> 3);
-        uint32_t kb[4];
-        ldsm_x4(kb, smem_u32(&sm.kbf[swz<CH16>(key, ch)]));
-        mma_bf16_16816(acc, qb[2 * kp], kb[0], kb[1]);
-        mma_bf16_16816(acc, qb[2 * kp + 1], kb[2], kb[3]);
-      }
-#pragma unroll
-      for (int e = 0; e < 4; ++e) s[nt][e] = acc[e] * a.scale_log2;
-    }
-  };
-
-  const int i_min = qt * TILE;
-  const int i_max = min(qt * TILE + TILE - 1, a.N - 1);
-  const int32_t *id = a.idx + bh * a.k_vert;
-  // Per row: remaining keys with position <= i - W (low-bit pairs) and
-  // vertical columns <= i - W (high pairs); both grow with i.
-  int cnt[2], nvt[2];
-#pragma unroll
-  for (int hf = 0; hf < 2; ++hf) {
-    cnt[hf] = remaining_upto(id, a.k_vert, rows[hf] - W);
-    nvt[hf] = rows[hf] - W >= 0 ? upper_bound_i32(id, a.k_vert, rows[hf] - W) : 0;
-  }
-  const int cnt_lo = remaining_upto(id, a.k_vert, i_min - W);
-  const int cnt_hi = remaining_upto(id, a.k_vert, i_max - W);
-  // 1) low-bit tiles over the remaining keys (INT8 QK, compact fp16 V)
-  for (int t = 0; t * TILE < cnt_hi; ++t) {
-    const int c0 = t * TILE;
-    const int nvalid = min(TILE, a.nr - c0);
-    __syncthreads();
-    load_tile<D>(sm.ki8, reinterpret_cast<const uint8_t *>(a.ki8 + (bh * a.nr + c0) * D), nvalid);
-    load_tile<D * 2>(sm.vh, reinterpret_cast<const uint8_t *>(a.vc + (bh * a.nr + c0) * D), nvalid);
-    __syncthreads();
-    float s[NT][4];
-    qk_int8(s, a.sk[bh * a.nblk_r + t]);
-    if (c0 + TILE > cnt_lo) {
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          if (c0 + nt * 8 + 2 * c + (e & 1) >= cnt[e >> 1]) s[nt][e] = -INFINITY;
-    }
-    softmax_pv(s);
-  }
-  // 2) window tiles in position order (bf16 QK): keep i - W < j <= i
-  if (W > 0) {
-    for (int kt = max(0, i_min - W + 1) / TILE; kt * TILE <= i_max; ++kt) {
-      const int j0 = kt * TILE;
-      const int nvalid = min(TILE, a.N - j0);
-      __syncthreads();
-      load_tile<D * 2>(sm.kbf, reinterpret_cast<const uint8_t *>(a.k + (bh * a.N + j0) * D), nvalid);
-      load_tile<D * 2>(sm.vh, reinterpret_cast<const uint8_t *>(a.vh + (bh * a.N + j0) * D), nvalid);
-      __syncthreads();
-      float s[NT][4];
-      qk_bf16(s);
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int i = rows[e >> 1];
-          const int j = j0 + nt * 8 + 2 * c + (e & 1);
-          if (j > i || j <= i - W) s[nt][e] = -INFINITY;
-        }
-      softmax_pv(s);
-    }
-  }
-  // 3) compact vertical tiles (bf16 QK): column v counts for row i when v <= i - W
-  const int nv_max = i_max - W >= 0 ? upper_bound_i32(id, a.k_vert, i_max - W) : 0;
-  for (int vt = 0; vt * TILE < nv_max; ++vt) {
-    __syncthreads();
-    load_tile<D * 2>(sm.kbf, reinterpret_cast<const uint8_t *>(a.vk + (bh * a.kpad + vt * TILE) * D), TILE);
-    load_tile<D * 2>(sm.vh, reinterpret_cast<const uint8_t *>(a.vv + (bh * a.kpad + vt * TILE) * D), TILE);
-    __syncthreads();
-    float s[NT][4];
-    qk_bf16(s);
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if (vt * TILE + nt * 8 + 2 * c + (e & 1) >= nvt[e >> 1]) s[nt][e] = -INFINITY;
-    softmax_pv(s);
-  }
-  // 3) normalize and store fp32 rows
-#pragma unroll
-  for (int hf = 0; hf < 2; ++hf) {
-    l[hf] += __shfl_xor_sync(0xffffffffu, l[hf], 1);
-    l[hf] += __shfl_xor_sync(0xffffffffu, l[hf], 2);
-  }
-#pragma unroll
-  for (int hf = 0; hf < 2; ++hf) {
-    if (rows[hf] >= a.N) continue;
-    const float inv = 1.f / l[hf];
-    float *dst = a.out + (bhq * a.N + rows[hf]) * D;
-#pragma unroll
-    for (int nt = 0; nt < D / 8; ++nt)
-      *reinterpret_cast<float2 *>(dst + nt * 8 + 2 * c) =
-          make_float2(o[nt][2 * hf] * inv, o[nt][2 * hf + 1] * inv);
-  }
-}
-
 struct PrefillWs {
   int8_t *qi8, *ki8;
   float *sq, *sk;
@@ -642,13 +363,16 @@ cudaError_t quant_t(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const int32_
   return cudaGetLastError();
 }
 
+// The pre-pass kernels, then the tcgen05 attention kernel.  Shapes the
+// tensor-core kernel does not take were rejected on the host; if the compiled
+// kernel is not usable (see prefill_tc_supported) nothing is launched.
 template <int D>
 cudaError_t prefill_t(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
                       const int32_t *idx, int B, int Hq, int Hkv, int N, int window, int k_vert,
                       float scale, int low_fmt, float *out, uint8_t *ws, uint32_t *status,
                       cudaStream_t s) {
+  if (!prefill_tc_supported(D, Hq, Hkv)) return cudaErrorNotSupported;
   const bool f8 = low_fmt == HQ_KV_FP8;
-  if (f8 && !prefill_tc_supported(D, Hq, Hkv)) return cudaErrorNotSupported;   // FP8: tcgen05 path only
   PrefillWs w = carve(ws, B, Hq, Hkv, N, D, k_vert);
   const int nbh = B * Hkv;
   const int nr = N - k_vert;
@@ -664,58 +388,31 @@ cudaError_t prefill_t(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
   if (kpad > 0)
     gather_vertical<D><<<dim3(kpad, nbh), D / 8, 0, s>>>(k, w.vh, idx, N, window, k_vert, kpad,
                                                          w.vk, w.vv, w.vpos, status);
-  if (prefill_tc_supported(D, Hq, Hkv)) {
-    TcLaunch p;
-    p.q = q;
-    p.k = k;
-    p.qi8 = w.qi8;
-    p.ki8 = w.ki8;
-    p.sq = w.sq;
-    p.sk = w.sk;
-    p.vh = w.vh;
-    p.vc = w.vc;
-    p.vk = w.vk;
-    p.vv = w.vv;
-    p.idx = idx;
-    p.out = out;
-    p.status = status;
-    p.B = B;
-    p.Hq = Hq;
-    p.Hkv = Hkv;
-    p.N = N;
-    p.window = window;
-    p.k_vert = k_vert;
-    p.kpad = kpad;
-    p.nblk_r = nblk_r;
-    p.scale = scale;
-    p.f8 = f8;
-    return launch_prefill_tc(p, s);
-  }
-  PrefillArgs a;
-  a.q = q;
-  a.k = k;
-  a.qi8 = w.qi8;
-  a.ki8 = w.ki8;
-  a.sq = w.sq;
-  a.sk = w.sk;
-  a.vh = w.vh;
-  a.vc = w.vc;
-  a.vk = w.vk;
-  a.vv = w.vv;
-  a.idx = idx;
-  a.out = out;
-  a.Hq = Hq;
-  a.Hkv = Hkv;
-  a.G = Hq / Hkv;
-  a.N = N;
-  a.window = window;
-  a.k_vert = k_vert;
-  a.kpad = kpad;
-  a.nr = nr;
-  a.nblk_r = nblk_r;
-  a.scale_log2 = scale * kLog2e;
-  prefill_mma<D><<<dim3((N + TILE - 1) / TILE, Hq, B), FWARPS * 32, 0, s>>>(a);
-  return cudaGetLastError();
+  TcLaunch p;
+  p.q = q;
+  p.k = k;
+  p.qi8 = w.qi8;
+  p.ki8 = w.ki8;
+  p.sq = w.sq;
+  p.sk = w.sk;
+  p.vh = w.vh;
+  p.vc = w.vc;
+  p.vk = w.vk;
+  p.vv = w.vv;
+  p.idx = idx;
+  p.out = out;
+  p.status = status;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.window = window;
+  p.k_vert = k_vert;
+  p.kpad = kpad;
+  p.nblk_r = nblk_r;
+  p.scale = scale;
+  p.f8 = f8;
+  return launch_prefill_tc(p, s);
 }
 
 }  // namespace
@@ -741,8 +438,7 @@ cudaError_t launch_prefill(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
                            int N, int D, int window, int k_vert, float scale, int low_fmt,
                            float *out, uint8_t *ws, uint32_t *status, cudaStream_t s) {
   if (D == 128) return prefill_t<128>(q, k, v, idx, B, Hq, Hkv, N, window, k_vert, scale, low_fmt, out, ws, status, s);
-  if (D == 64) return prefill_t<64>(q, k, v, idx, B, Hq, Hkv, N, window, k_vert, scale, low_fmt, out, ws, status, s);
-  return cudaErrorInvalidValue;
+  return cudaErrorNotSupported;
 }
 
 }  // namespace hq

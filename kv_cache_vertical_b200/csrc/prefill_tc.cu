@@ -537,7 +537,8 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
 
 // The kernel redistributes registers with setmaxnreg, which is only valid
 // when the CTA starts with exactly kRegsLaunch registers per thread; that is
-// checked once from the compiled kernel (else the CUDA-core kernel is used).
+// checked once from the compiled kernel.  If the check fails the prefill is
+// reported unsupported and nothing is launched (there is no other kernel).
 template <bool F8>
 static bool kernel_ready() {
   cudaFuncAttributes fa;

@@ -9,11 +9,15 @@
 //
 // The array lives in every GPU that loads the library, until the process
 // exits.  In host code its name only stands for it (a host-side shadow): the
-// device address is looked up once per device with cudaGetSymbolAddress, with
-// that device current, on the first call made on it, and cached.  Every call
-// shares the array: it first clears the part that must start at zero (status
-// word and split tickets); calls that overlap on the GPU race on it.
-#include <atomic>
+// device address is looked up with cudaGetSymbolAddress, with the device
+// current, on the first call made in a CUDA context, and cached for that
+// context.  Every call shares the array: it first clears the part that must
+// start at zero (status word and split tickets); calls that overlap on the
+// GPU race on it.  The first 4 bytes are the device status word of the last
+// call (hq_read_static_status).
+#include <cuda.h>
+
+#include <mutex>
 
 #include "hq_internal.cuh"
 
@@ -22,16 +26,46 @@ namespace {
 __device__ __align__(256) uint8_t g_static_scratch[HQ_STATIC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
-std::atomic<void *> g_scratch_addr[kMaxDevices];
+struct ScratchAddr {
+  CUcontext ctx;   // the context the address belongs to
+  void *addr;
+};
+ScratchAddr g_scratch[kMaxDevices];
+std::mutex g_scratch_mu;
 
-// Device address of g_static_scratch on the current device (nullptr on error).
+// The current CUDA context (driver entry point, looked up once), or nullptr.
+CUcontext current_context() {
+  using Fn = CUresult (*)(CUcontext *);
+  static Fn fn = [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return (Fn) nullptr;
+    return reinterpret_cast<Fn>(p);
+  }();
+  CUcontext c = nullptr;
+  if (!fn || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
+
+// Device address of g_static_scratch in the current device's context
+// (nullptr on error).  Looked up again whenever the context differs from the
+// one the cached address came from (a reset device gets a new context, and
+// the module, with the array, is loaded again at a possibly new address).
 void *scratch_address() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  void *p = g_scratch_addr[dev].load(std::memory_order_acquire);
-  if (p) return p;
+  CUcontext ctx = current_context();
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  ScratchAddr &e = g_scratch[dev];
+  if (ctx && e.addr && e.ctx == ctx) return e.addr;
+  void *p = nullptr;
   if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return nullptr;
-  g_scratch_addr[dev].store(p, std::memory_order_release);
+  ctx = current_context();             // the lookup makes the device's context current if none was
+  if (!ctx) return nullptr;
+  e.ctx = ctx;
+  e.addr = p;
   return p;
 }
 
@@ -54,4 +88,17 @@ extern "C" hq_status hq_decode_attn_static(const void *q, const hq_kv_cache *cac
                         hq::resolve_softmax_scale(softmax_scale, D), out, lse_out, ws,
                         reinterpret_cast<uint32_t *>(ws), s);
   return e == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+}
+
+extern "C" hq_status hq_read_static_status(int clear, uint32_t *status_out, void *stream) {
+  if (!status_out) return HQ_ERR_INVALID_ARG;
+  uint8_t *ws = static_cast<uint8_t *>(scratch_address());
+  if (!ws) return HQ_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t v = 0;
+  if (cudaMemcpyAsync(&v, ws, sizeof v, cudaMemcpyDeviceToHost, s) != cudaSuccess) return HQ_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return HQ_ERR_CUDA;
+  if (clear && cudaMemsetAsync(ws, 0, sizeof v, s) != cudaSuccess) return HQ_ERR_CUDA;
+  *status_out = v;
+  return HQ_OK;
 }

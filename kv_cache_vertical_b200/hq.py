@@ -73,10 +73,12 @@ _append = _sig("hq_kv_append", _I, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.POINTE
 _merge = _sig("hq_decode_merge", _I, _P, _P, _I, _I, _I, _I, _P, _P, _P)
 _decode_static = _sig("hq_decode_attn_static", _I, _P, ctypes.POINTER(hq_kv_cache), _I, _I, _I,
                       _I, _F, _P, _P, _P)
+_read_static_status = _sig("hq_read_static_status", _I, _I, ctypes.POINTER(ctypes.c_uint32), _P)
 _pquant = _sig("hq_prefill_quant", _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P)
 hq_prefill_workspace_size = _sig("hq_prefill_workspace_size", _SZ, _I, _I, _I, _I, _I, _I)
 _prefill = _sig("hq_prefill_attn", _I, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P,
                 _SZ, _P)
+_prefill_supported = _sig("hq_prefill_supported", _I, _I, _I, _I, _I)
 _pquant_ex = _sig("hq_prefill_quant_ex", _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P)
 _prefill_ex = _sig("hq_prefill_attn_ex", _I, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P,
                    _P, _SZ, _P)
@@ -84,10 +86,10 @@ _prefill_ex = _sig("hq_prefill_attn_ex", _I, _P, _P, _P, _P, _I, _I, _I, _I, _I,
 EXPORTED = ["hq_status_string", "hq_version", "hq_read_device_status", "hq_probe_workspace_size",
             "hq_probe_vertical", "hq_pack_kv", "hq_decode_workspace_size", "hq_decode_attn",
             "hq_prefill_quant", "hq_prefill_workspace_size", "hq_prefill_attn",
-            "hq_decode_attn_static", "hq_kv_append", "hq_decode_merge", "hq_prefill_quant_ex",
+            "hq_decode_attn_static", "hq_read_static_status", "hq_kv_append", "hq_decode_merge", "hq_prefill_quant_ex",
             "hq_prefill_attn_ex", "hq_probe_shard_workspace_size", "hq_probe_shard_stats",
             "hq_probe_merge_stats", "hq_probe_shard_topk", "hq_probe_merge_workspace_size",
-            "hq_probe_merge_topk"]
+            "hq_probe_merge_topk", "hq_prefill_supported"]
 
 HQ_ERR_SCRATCH_LIMIT = 7
 STATIC_SCRATCH_BYTES = 8 << 20
@@ -288,6 +290,15 @@ def hq_decode_attn_static(q, cache: KVCache, B, Hq, Hkv, D, softmax_scale, out, 
                           _ptr(out), _ptr(lse_out), _stream(stream)), "hq_decode_attn_static")
 
 
+def hq_read_static_status(clear: bool = False, stream=None) -> int:
+    """Device status word of the last hq_decode_attn_static call on the
+    current device (HQ_DEV_* bits; synchronizes the stream)."""
+    v = ctypes.c_uint32(0)
+    _check(_read_static_status(int(clear), ctypes.byref(v), _stream(stream)),
+           "hq_read_static_status")
+    return v.value
+
+
 def hq_prefill_quant(q, k, idx, B, Hq, Hkv, N, D, k_vert, qi8, sq, ki8, sk, stream=None):
     _check(_pquant(_ptr(q), _ptr(k), _ptr(idx), B, Hq, Hkv, N, D, k_vert, _ptr(qi8), _ptr(sq),
                    _ptr(ki8), _ptr(sk), _stream(stream)), "hq_prefill_quant")
@@ -297,6 +308,12 @@ def hq_prefill_quant_ex(q, k, idx, B, Hq, Hkv, N, D, k_vert, low_fmt, qi8, sq, k
                         stream=None):
     _check(_pquant_ex(_ptr(q), _ptr(k), _ptr(idx), B, Hq, Hkv, N, D, k_vert, low_fmt, _ptr(qi8),
                       _ptr(sq), _ptr(ki8), _ptr(sk), _stream(stream)), "hq_prefill_quant_ex")
+
+
+def hq_prefill_supported(D, Hq, Hkv, low_fmt=HQ_KV_INT) -> int:
+    """HQ_OK (0) when a prefill of this shape and low-part format runs the
+    tensor-core kernel on the current device, else HQ_ERR_UNSUPPORTED."""
+    return _prefill_supported(D, Hq, Hkv, low_fmt)
 
 
 def hq_prefill_attn_ex(q, k, v, idx, B, Hq, Hkv, N, D, window, k_vert, softmax_scale, low_fmt,

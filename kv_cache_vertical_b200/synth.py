@@ -151,3 +151,38 @@ def make_inputs(w: Workload, threads: int | None = None, pin: bool = False) -> d
     else:
         out.update(q=q)
     return out
+
+
+def make_inputs_device(w: Workload, device, seed_offset: int = 0) -> dict:
+    """The recipe of make_inputs drawn directly on the GPU with torch's seeded
+    generator (a different stream of numbers than the host generator's, the
+    same distributions and structure).  For timing runs at full size, where
+    drawing gigabytes on the host would take minutes; parity tests use
+    make_inputs.  Decode workloads only (q [B,Hq,D], q_probe [B,Hq,64,D])."""
+    assert w.mode == "decode"
+    B, Hq, Hkv, D, L, G, W = w.B, w.Hq, w.Hkv, w.D, w.L, w.G, w.window
+    kv = w.k_vert
+    g = torch.Generator(device=device)
+    g.manual_seed(w.seed + seed_offset)
+    f32 = dict(dtype=torch.float32, device=device, generator=g)
+    u = torch.randn(B, Hkv, D, **f32)
+    u /= u.norm(dim=-1, keepdim=True)
+    k = torch.empty(B, Hkv, L, D, dtype=torch.bfloat16, device=device)
+    v = torch.empty_like(k)
+    planted = torch.empty(B, Hkv, kv, dtype=torch.int32, device=device)
+    for b in range(B):                       # one batch element at a time bounds the fp32 temporaries
+        kk = torch.randn(Hkv, L, D, **f32)
+        outl = torch.rand(Hkv, D, **f32).argsort(dim=-1)[:, :4]
+        mult = torch.ones(Hkv, D, device=device).scatter_(1, outl, 10.0)
+        kk *= mult[:, None, :]
+        if kv:
+            pos = torch.rand(Hkv, L - W, **f32).argsort(dim=-1)[:, :kv].sort(dim=-1).values
+            rows = 3.0 * u[b][:, None, :] + 0.3 * torch.randn(Hkv, kv, D, **f32)
+            kk.scatter_(1, pos[..., None].expand(-1, -1, D), rows)
+            planted[b] = pos.to(torch.int32)
+        k[b] = kk.to(torch.bfloat16)
+        del kk
+        v[b] = torch.randn(Hkv, L, D, **f32).to(torch.bfloat16)
+    q = (torch.randn(B, Hkv, G, D, **f32) + 2.0 * u[:, :, None, :]).to(torch.bfloat16)
+    qp = (torch.randn(B, Hkv, G, PROBE_ROWS, D, **f32) + 2.0 * u[:, :, None, None, :]).to(torch.bfloat16)
+    return dict(k=k, v=v, planted=planted, q=q.view(B, Hq, D), q_probe=qp.view(B, Hq, PROBE_ROWS, D))

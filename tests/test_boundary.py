@@ -162,16 +162,22 @@ def test_probe_and_prefill_argument_checks(lib):
     q = lib.hq_prefill_attn
     q.restype = ctypes.c_int
     lib.hq_prefill_workspace_size.restype = ctypes.c_size_t
-    need = lib.hq_prefill_workspace_size(1, 4, 2, 256, 64, 12)
+    need = lib.hq_prefill_workspace_size(1, 4, 2, 256, 128, 12)
 
-    def pre(N=256, D=64, W=32, kv=12, idx=FAKE, ws=FAKE, wsb=need):
-        return q(FAKE, FAKE, FAKE, idx, 1, 4, 2, N, D, W, kv, ctypes.c_float(0), FAKE, ws,
+    def pre(N=256, D=128, Hq=4, Hkv=2, W=32, kv=12, idx=FAKE, ws=FAKE, wsb=need):
+        return q(FAKE, FAKE, FAKE, idx, 1, Hq, Hkv, N, D, W, kv, ctypes.c_float(0), FAKE, ws,
                  ctypes.c_size_t(wsb), None)
     assert pre(idx=None) == 1
     assert pre(kv=300) == 1
     assert pre(D=256) == 2
+    # the prefill attention has one kernel: head_dim 128, two query heads per CTA
+    assert pre(D=64) == 2
+    assert pre(Hq=2, Hkv=2) == 2
     assert pre(ws=None) == 3
     assert pre(wsb=need - 1) == 3
+    sup = lib.hq_prefill_supported
+    sup.restype = ctypes.c_int
+    assert sup(64, 4, 2, 0) == 2 and sup(128, 2, 2, 0) == 2 and sup(128, 4, 2, 7) == 2
     qq = lib.hq_prefill_quant
     qq.restype = ctypes.c_int
     assert qq(FAKE, FAKE, FAKE, 1, 4, 2, 256, 64, 12, None, FAKE, FAKE, FAKE, None) == 1

@@ -60,15 +60,29 @@ def run_prefill_case(w: Workload, rows=None, check_probe=True, fmt=0, planted_id
     return assert_close(g, ref, f"prefill {w.name}")
 
 
-@pytest.mark.parametrize("G", [1, 4])
+@pytest.mark.parametrize("G", [2, 4])
 def test_prefill_small_ragged(G):
     w = Workload("p", "prefill", 1, 2 * G, 2, 128, 1000, 128, F5, 4, 11 + G)
     run_prefill_case(w)
 
 
-def test_prefill_head_dim_64_batch_2():
-    w = Workload("p64", "prefill", 2, 4, 1, 64, 700, 64, F5, 4, 21)
-    run_prefill_case(w)
+def test_prefill_tensor_core_kernel_is_the_path():
+    """The accepted shapes run the tcgen05 kernel (the query checks that the
+    compiled kernel is usable on this device); the others are refused before
+    any launch, never run on another kernel."""
+    H = hq()
+    for fmt in (0, 1):
+        for G in (2, 4, 8):
+            assert H.hq_prefill_supported(128, 8 * G, 8, fmt) == 0
+        assert H.hq_prefill_supported(128, 8, 8, fmt) == 2          # one query head per KV head
+        assert H.hq_prefill_supported(64, 4, 1, fmt) == 2           # head_dim 64
+    for w in (Workload("g1", "prefill", 1, 2, 2, 128, 300, 32, F5, 4, 12),
+              Workload("p64", "prefill", 2, 4, 1, 64, 700, 64, F5, 4, 21)):
+        d = to_dev(make_inputs(w))
+        idx = torch.from_numpy(make_inputs(w)["planted"].numpy()).cuda()
+        with pytest.raises(H.HQError) as e:
+            H.prefill_attn(d["q"], d["k"], d["v"], idx, w.window)
+        assert e.value.status == 2
 
 
 def test_prefill_window_larger_than_sequence():

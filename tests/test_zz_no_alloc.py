@@ -42,6 +42,8 @@ def test_static_scratch_decode_matches_workspace_decode(name):
         assert err.max().item() <= MAX_ABS and err.mean().item() <= MEAN_ABS, \
             f"max {err.max().item():.3e} mean {err.mean().item():.3e}"
         assert np.allclose(lse.cpu().numpy(), ref_lse.cpu().numpy(), atol=1e-5)
+        # the fixed array's status word: no bounded wait ran out, no bad input
+        assert H.hq_read_static_status() == 0
 
 
 def test_static_scratch_rejects_problems_beyond_its_size():
