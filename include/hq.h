@@ -150,7 +150,9 @@ hq_status hq_read_device_status(const void *ws, int clear, uint32_t *status_out,
  *   idx_out   : i32 [B, Hkv, k_vert], ascending.
  *   score_out : f32 [B, Hkv, L] or NULL (the column sums; keys never seen 0).
  *   softmax_scale: 0 selects 1 / sqrt(D).
- * Requires 1 <= P <= L, 0 <= window, 0 <= k_vert <= L - window.
+ * Requires 1 <= P <= L, 0 <= window, 0 <= k_vert <= L - window; P <= 64
+ * (the method probes with the 64 most recent queries; larger P returns
+ * HQ_ERR_UNSUPPORTED).
  */
 size_t hq_probe_workspace_size(int B, int Hq, int Hkv, int P, int L, int D);
 hq_status hq_probe_vertical(const void *q_probe, int64_t q_head_stride, const void *k, int B,
@@ -179,7 +181,7 @@ hq_status hq_probe_vertical(const void *q_probe, int64_t q_head_stride, const vo
  * (-FLT_MAX, 0).  cand_idx i32 / cand_score f32 [B*Hkv, k_vert]: a rank with
  * fewer than k_vert candidates (keys before L - window) pads with -1 / -FLT_MAX.
  * Merge inputs are the R ranks' arrays stacked on a leading axis.
- * Requires 1 <= P <= L, 0 <= key_off, key_off + Ls <= L, Ls >= 1,
+ * Requires 1 <= P <= min(L, 64), 0 <= key_off, key_off + Ls <= L, Ls >= 1,
  * 0 <= k_vert <= L - window.  Errors as for hq_probe_vertical; a candidate
  * position outside [0, L - window) sets HQ_DEV_BAD_INDEX in the merge's status
  * word and is ignored.
@@ -224,6 +226,26 @@ hq_status hq_probe_merge_topk(const int32_t *cand_idx, const float *cand_score, 
 hq_status hq_pack_kv(const void *k, const void *v, const int32_t *idx, int B, int Hkv, int L,
                      int D, int window, int k_vert, int bits, int group, const hq_kv_cache *out,
                      void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * One part of the hybrid cache, for a context split across GPUs: the rows
+ * [lo0, lo0 + out->n_lo) of the low segment and [hi0, hi0 + out->n_hi) of the
+ * bf16 segment of the cache hq_pack_kv would build from the same arguments,
+ * written to `out` (row lo0 of the cache becomes row 0 of the part, and so
+ * on), bit-identical to those rows of the whole cache.  A rank that decodes
+ * only its part (hq_decode_attn with lse_out, then hq_decode_merge over the
+ * ranks) holds only these rows: attention does not depend on the order of
+ * the cached rows (wiki summary, "Key results": one softmax over all cached
+ * positions).  Equal shares of both segments give every rank the same bytes
+ * to read.  k and v are the whole context's [B, Hkv, L, D] (the rows of a
+ * part come from positions spread over the context); idx is the whole list.
+ * Requires 0 <= lo0, lo0 + out->n_lo <= L - window - k_vert, 0 <= hi0,
+ * hi0 + out->n_hi <= k_vert + window; an empty part (both counts 0) is a
+ * no-op.  Other arguments, layouts and errors as for hq_pack_kv.
+ */
+hq_status hq_pack_kv_part(const void *k, const void *v, const int32_t *idx, int B, int Hkv, int L,
+                          int D, int window, int k_vert, int bits, int group, int lo0, int hi0,
+                          const hq_kv_cache *out, void *ws, size_t ws_bytes, void *stream);
 
 /* ------------------------------------------------------------------------ */
 /* Decode attention with fused dequantization (wiki summary, "Key results":  */
@@ -326,6 +348,22 @@ hq_status hq_read_static_status(int clear, uint32_t *status_out, void *stream);
  */
 hq_status hq_kv_append(const void *k_new, const void *v_new, int B, int Hkv, int D, int L,
                        int window, int k_vert, const hq_kv_cache *cache, void *stream);
+
+/*
+ * hq_kv_append on the part of a context-split cache that ends where the whole
+ * cache ends (see hq_pack_kv_part): it holds low rows [lo0, L - window -
+ * k_vert) and bf16 rows [hi0, k_vert + window) with hi0 <= k_vert, i.e. the
+ * last low rows and the whole window.  The appended low row is row lo0 +
+ * cache->n_lo of the whole cache, the window ring row k_vert + L mod window
+ * is row k_vert - hi0 + L mod window of the part; the result is
+ * bit-identical to those rows of hq_kv_append on the whole cache.  The other
+ * ranks' parts do not change.  Requires cache->n_lo == L - window - k_vert -
+ * lo0, cache->n_hi == k_vert + window - hi0 and a spare low row; otherwise as
+ * hq_kv_append (which is this call with lo0 = hi0 = 0).
+ */
+hq_status hq_kv_append_part(const void *k_new, const void *v_new, int B, int Hkv, int D, int L,
+                            int window, int k_vert, int lo0, int hi0, const hq_kv_cache *cache,
+                            void *stream);
 
 /* ------------------------------------------------------------------------ */
 /* Hybrid-precision prefill (abstract: Prefill stage keeps vertical-line     */

@@ -12,6 +12,10 @@ namespace {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// The probe keeps the probe rows of a KV head in shared memory (the method
+// probes with the 64 most recent queries).
+constexpr int kMaxProbeRows = 64;
+
 bool supported_G(int Hq, int Hkv) {
   if (Hq <= 0 || Hkv <= 0 || Hq % Hkv) return false;
   const int G = Hq / Hkv;
@@ -94,7 +98,8 @@ hq_status hq_read_device_status(const void *ws, int clear, uint32_t *status_out,
 }
 
 size_t hq_probe_workspace_size(int B, int Hq, int Hkv, int P, int L, int D) {
-  if (B <= 0 || !supported_G(Hq, Hkv) || P <= 0 || L <= 0 || (D != 64 && D != 128)) return 0;
+  if (B <= 0 || !supported_G(Hq, Hkv) || P <= 0 || P > kMaxProbeRows || L <= 0 || (D != 64 && D != 128))
+    return 0;
   return probe_ws_bytes(B, Hq, Hkv, P, L, D);
 }
 
@@ -106,7 +111,7 @@ hq_status hq_probe_vertical(const void *q_probe, int64_t q_head_stride, const vo
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || P <= 0 || P > L || window < 0 ||
       k_vert < 0 || k_vert > L - window || q_head_stride < (int64_t)P * D)
     return HQ_ERR_INVALID_ARG;
-  if ((D != 64 && D != 128) || !supported_G(Hq, Hkv)) return HQ_ERR_UNSUPPORTED;
+  if ((D != 64 && D != 128) || !supported_G(Hq, Hkv) || P > kMaxProbeRows) return HQ_ERR_UNSUPPORTED;
   if (!aligned16(q_probe) || !aligned16(k) || (q_head_stride * 2) % 16) return HQ_ERR_INVALID_ARG;
   if (!ws || ws_bytes < probe_ws_bytes(B, Hq, Hkv, P, L, D)) return HQ_ERR_WORKSPACE;
   return cuda_status(launch_probe((const __nv_bfloat16 *)q_probe, q_head_stride,
@@ -122,7 +127,8 @@ static bool shard_args_ok(const void *q_probe, int64_t q_head_stride, const void
 }
 
 size_t hq_probe_shard_workspace_size(int B, int Hq, int Hkv, int P, int Ls, int D, int k_vert) {
-  if (B <= 0 || !supported_G(Hq, Hkv) || P <= 0 || Ls <= 0 || k_vert < 0 || (D != 64 && D != 128))
+  if (B <= 0 || !supported_G(Hq, Hkv) || P <= 0 || P > kMaxProbeRows || Ls <= 0 || k_vert < 0 ||
+      (D != 64 && D != 128))
     return 0;
   return probe_shard_ws_bytes(B, Hq, Hkv, P, Ls, D, k_vert);
 }
@@ -133,7 +139,7 @@ hq_status hq_probe_shard_stats(const void *q_probe, int64_t q_head_stride, const
                                void *stream) {
   if (!stats_out || !shard_args_ok(q_probe, q_head_stride, k_shard, B, Hq, Hkv, P, Ls, D, key_off, L))
     return HQ_ERR_INVALID_ARG;
-  if ((D != 64 && D != 128) || !supported_G(Hq, Hkv)) return HQ_ERR_UNSUPPORTED;
+  if ((D != 64 && D != 128) || !supported_G(Hq, Hkv) || P > kMaxProbeRows) return HQ_ERR_UNSUPPORTED;
   if (!aligned16(q_probe) || !aligned16(k_shard) || !aligned16(stats_out) || (q_head_stride * 2) % 16)
     return HQ_ERR_INVALID_ARG;
   if (!ws || ws_bytes < probe_shard_ws_bytes(B, Hq, Hkv, P, Ls, D, 0)) return HQ_ERR_WORKSPACE;
@@ -160,7 +166,7 @@ hq_status hq_probe_shard_topk(const void *q_probe, int64_t q_head_stride, const 
   if (!shard_args_ok(q_probe, q_head_stride, k_shard, B, Hq, Hkv, P, Ls, D, key_off, L) || !stats ||
       window < 0 || k_vert < 0 || k_vert > L - window || (k_vert > 0 && (!cand_idx || !cand_score)))
     return HQ_ERR_INVALID_ARG;
-  if ((D != 64 && D != 128) || !supported_G(Hq, Hkv)) return HQ_ERR_UNSUPPORTED;
+  if ((D != 64 && D != 128) || !supported_G(Hq, Hkv) || P > kMaxProbeRows) return HQ_ERR_UNSUPPORTED;
   if (!aligned16(q_probe) || !aligned16(k_shard) || !aligned16(stats) || (q_head_stride * 2) % 16)
     return HQ_ERR_INVALID_ARG;
   if (!ws || ws_bytes < probe_shard_ws_bytes(B, Hq, Hkv, P, Ls, D, k_vert)) return HQ_ERR_WORKSPACE;
@@ -189,39 +195,53 @@ hq_status hq_probe_merge_topk(const int32_t *cand_idx, const float *cand_score, 
                                              (cudaStream_t)stream));
 }
 
-hq_status hq_pack_kv(const void *k, const void *v, const int32_t *idx, int B, int Hkv, int L,
-                     int D, int window, int k_vert, int bits, int group, const hq_kv_cache *out,
-                     void *ws, size_t ws_bytes, void *stream) {
+hq_status hq_pack_kv_part(const void *k, const void *v, const int32_t *idx, int B, int Hkv, int L,
+                          int D, int window, int k_vert, int bits, int group, int lo0, int hi0,
+                          const hq_kv_cache *out, void *ws, size_t ws_bytes, void *stream) {
   if (!k || !v || !out || (k_vert > 0 && !idx)) return HQ_ERR_INVALID_ARG;
   if (B <= 0 || Hkv <= 0 || L <= 0 || window < 0 || k_vert < 0 || k_vert > L - window)
     return HQ_ERR_INVALID_ARG;
   if ((D != 64 && D != 128) || (bits != 4 && bits != 8) || group != 32) return HQ_ERR_UNSUPPORTED;
   if (out->bits == bits && !fmt_ok(*out)) return HQ_ERR_UNSUPPORTED;
   const int n_lo = L - window - k_vert, n_hi = k_vert + window;
-  if (out->n_lo != n_lo || out->n_hi != n_hi || out->bits != bits || out->group != group ||
-      !lo_cap_ok(*out))
+  if (lo0 < 0 || hi0 < 0 || out->n_lo < 0 || out->n_hi < 0 || lo0 + out->n_lo > n_lo ||
+      hi0 + out->n_hi > n_hi || out->bits != bits || out->group != group || !lo_cap_ok(*out))
     return HQ_ERR_INVALID_ARG;
-  if ((n_lo > 0 && (!out->k_codes || !out->v_codes || !out->k_sz || !out->v_sz)) ||
-      (n_hi > 0 && (!out->k_hi || !out->v_hi)))
+  if ((out->n_lo > 0 && (!out->k_codes || !out->v_codes || !out->k_sz || !out->v_sz)) ||
+      (out->n_hi > 0 && (!out->k_hi || !out->v_hi)))
     return HQ_ERR_INVALID_ARG;
   const void *ptrs[] = {k, v, out->k_codes, out->v_codes, out->k_sz, out->v_sz, out->k_hi, out->v_hi};
   for (const void *p : ptrs)
     if (p && !aligned16(p)) return HQ_ERR_INVALID_ARG;
   if (ws && ws_bytes < kWsHeader) return HQ_ERR_WORKSPACE;
+  if (out->n_lo + out->n_hi == 0) return HQ_OK;            // an empty part: nothing to write
   return cuda_status(launch_pack((const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, idx, B, Hkv,
                                  L, D, window, k_vert, bits, *out, status_word(ws),
-                                 (cudaStream_t)stream));
+                                 (cudaStream_t)stream, lo0, hi0));
 }
 
-hq_status hq_kv_append(const void *k_new, const void *v_new, int B, int Hkv, int D, int L,
-                       int window, int k_vert, const hq_kv_cache *cache, void *stream) {
+hq_status hq_pack_kv(const void *k, const void *v, const int32_t *idx, int B, int Hkv, int L,
+                     int D, int window, int k_vert, int bits, int group, const hq_kv_cache *out,
+                     void *ws, size_t ws_bytes, void *stream) {
+  if (out && L - window - k_vert >= 0 &&
+      (out->n_lo != L - window - k_vert || out->n_hi != k_vert + window))
+    return HQ_ERR_INVALID_ARG;
+  return hq_pack_kv_part(k, v, idx, B, Hkv, L, D, window, k_vert, bits, group, 0, 0, out, ws,
+                         ws_bytes, stream);
+}
+
+hq_status hq_kv_append_part(const void *k_new, const void *v_new, int B, int Hkv, int D, int L,
+                            int window, int k_vert, int lo0, int hi0, const hq_kv_cache *cache,
+                            void *stream) {
   if (!k_new || !v_new || !cache) return HQ_ERR_INVALID_ARG;
   if (B <= 0 || Hkv <= 0 || window < 0 || k_vert < 0 || L < window + k_vert) return HQ_ERR_INVALID_ARG;
   if ((D != 64 && D != 128) || (cache->bits != 4 && cache->bits != 8) || cache->group != 32 ||
       !fmt_ok(*cache))
     return HQ_ERR_UNSUPPORTED;
-  if (cache->n_lo != L - window - k_vert || cache->n_hi != k_vert + window ||
-      cache->lo_cap <= cache->n_lo)
+  // the part must end where the cache ends: the last low rows and the window
+  if (lo0 < 0 || hi0 < 0 || hi0 > k_vert || cache->n_lo < 0 ||
+      lo0 + cache->n_lo != L - window - k_vert || cache->n_hi != k_vert + window - hi0 ||
+      lo_rows(*cache) <= cache->n_lo)
     return HQ_ERR_INVALID_ARG;
   if (!cache->k_codes || !cache->v_codes || !cache->k_sz || !cache->v_sz ||
       (window > 0 && (!cache->k_hi || !cache->v_hi)))
@@ -231,7 +251,13 @@ hq_status hq_kv_append(const void *k_new, const void *v_new, int B, int Hkv, int
   for (const void *p : ptrs)
     if (p && !aligned16(p)) return HQ_ERR_INVALID_ARG;
   return cuda_status(launch_kv_append((const __nv_bfloat16 *)k_new, (const __nv_bfloat16 *)v_new,
-                                      B, Hkv, D, L, window, k_vert, *cache, (cudaStream_t)stream));
+                                      B, Hkv, D, L, window, k_vert - hi0, *cache,
+                                      (cudaStream_t)stream));
+}
+
+hq_status hq_kv_append(const void *k_new, const void *v_new, int B, int Hkv, int D, int L,
+                       int window, int k_vert, const hq_kv_cache *cache, void *stream) {
+  return hq_kv_append_part(k_new, v_new, B, Hkv, D, L, window, k_vert, 0, 0, cache, stream);
 }
 
 hq_status hq_decode_merge(const float *part_out, const float *part_lse, int R, int B, int Hq,

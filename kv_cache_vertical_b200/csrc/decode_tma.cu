@@ -10,7 +10,7 @@
 // (b, kv head) pairs form two lines, shared out over one wave of CTAs in
 // proportion to their cost; a CTA serves one or a few consecutive pairs and
 // claims their tiles dynamically (see Line below).  Tiles stream global ->
-// shared memory by TMA (one producer warp, mbarrier ring of NSTAGE stages,
+// shared memory by TMA (one producer warp, an mbarrier ring of stages,
 // 64B/128B swizzle so that ldmatrix reads are bank-conflict free).  Each of
 // the four consumer warps takes one 16-token sub-tile of every stage:
 //
@@ -49,19 +49,24 @@ constexpr float kLazy = 8.0f;               // rescale only when the max grows b
 // Every consumer warp takes one 16-token sub-tile of EVERY stage, so each warp
 // waits on every phase of every barrier in order (a warp that skipped stages
 // could wait on a phase two ahead, which the parity scheme cannot tell apart).
-// A low-bit CTA runs NSTAGE stages of STAGE bytes; a bf16 CTA runs NSTAGE/2
-// stages of 2*STAGE bytes (its 64-token tiles are larger).
+// Every CTA owns a ring of RING bytes: a low-bit CTA cuts it into NLO stages
+// of one low tile each, a bf16 CTA into NHI stages of one bf16 tile, so the
+// bytes in flight per CTA are about the same whatever the code width (an
+// INT4 tile is 10 KB, an INT8 tile 18 KB, a bf16 tile 32 KB).
 template <int BITS>
 struct Cfg {
   static constexpr int ROWB = D * BITS / 8;               // packed bytes per low row
   static constexpr int KC = T_LO * ROWB;                  // codes per stage (K or V)
   static constexpr int SZ = T_LO * 16;                    // (scale, zero) x 4 groups per token
-  static constexpr int LO_BYTES = 2 * KC + 2 * SZ;
+  static constexpr int LO_BYTES = 2 * KC + 2 * SZ;        // a multiple of 1024 (swizzle alignment)
   static constexpr int HI_BOX = T_HI * 128;               // 64 channels x 64 tokens, bf16
   static constexpr int HI_BYTES = 4 * HI_BOX;
-  static constexpr int STAGE = LO_BYTES > HI_BYTES / 2 ? LO_BYTES : HI_BYTES / 2;
-  static constexpr int NSTAGE = 4;
-  static constexpr int SMEM = NSTAGE * STAGE + 1024 + 512;  // + alignment slack + barriers
+  static constexpr int RING = 72 * 1024;
+  static constexpr int NLO = RING / LO_BYTES;             // 7 (INT4) / 4 (INT8)
+  static constexpr int NHI = RING / HI_BYTES;             // 2
+  static constexpr int NMAX = NLO > NHI ? NLO : NHI;
+  static constexpr int SMEM = RING + 1024 + 512;          // + alignment slack + barriers
+  static_assert(LO_BYTES % 1024 == 0 && NMAX <= 8, "stage layout");
 };
 
 struct DecArgs {
@@ -135,8 +140,11 @@ __device__ __forceinline__ uint32_t f8pair(uint32_t w, uint32_t sel) {
   const uint32_t t = x >> 1;
   return t + (t & 0x40004000u);
 }
+// The fp16 in the low half of w, widened (one conversion, no masking).
 __device__ __forceinline__ float half_lo_f(uint32_t w) {
-  return __half2float(__ushort_as_half((unsigned short)(w & 0xffffu)));
+  float f;
+  asm("{\n .reg .b16 lo, hi;\n mov.b32 {lo, hi}, %1;\n cvt.f32.f16 %0, lo;\n}\n" : "=f"(f) : "r"(w));
+  return f;
 }
 
 // Codes enter the MMAs as fp16 subnormals: the bit pattern c (0 <= c < 2^10)
@@ -164,14 +172,14 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
   using C = Cfg<BITS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::NSTAGE * C::STAGE);
-  uint64_t *empty = full + C::NSTAGE;
-  uint64_t *merged = empty + C::NSTAGE;                         // one phase per finished piece
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::RING);
+  uint64_t *empty = full + 8;
+  uint64_t *merged = empty + 8;                                 // one phase per finished piece
   uint64_t *cbar = merged + 1;                                  // [2] partial chunks of a pair merge
   float *qsum = reinterpret_cast<float *>(cbar + 2);            // [8 heads][4 groups]
   volatile int *abort_flag = reinterpret_cast<volatile int *>(qsum + 32);
   int *last_flag = reinterpret_cast<int *>(qsum + 33);
-  int *meta = last_flag + 1;                                     // [NSTAGE] tile of each stage, -1: end of piece
+  int *meta = last_flag + 1;                                     // [nst] tile of each stage, -1: end of piece
 
   const bool hi = (int)blockIdx.x >= a.nc_lo;
   const int cta = hi ? (int)blockIdx.x - a.nc_lo : (int)blockIdx.x;
@@ -179,10 +187,8 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
   const long long g0 = range_start(L, cta), g1 = range_start(L, cta + 1);
   const int bh_a = (int)(g0 / L.t), bh_b = (int)((g1 - 1) / L.t);   // pairs of this CTA's pieces
   const int T = hi ? T_HI : T_LO;
-  const int nst = hi ? C::NSTAGE / 2 : C::NSTAGE;              // stages of this CTA (power of 2)
-  const int lnst = hi ? 1 : 2;                                  // log2(nst)
-  static_assert(C::NSTAGE == 4, "stage arithmetic assumes 4 / 2 stages");
-  const int stage_bytes = hi ? 2 * C::STAGE : C::STAGE;
+  const int nst = hi ? C::NHI : C::NLO;                        // stages of this CTA's ring
+  const int stage_bytes = hi ? C::HI_BYTES : C::LO_BYTES;
   const int n_tok = hi ? a.n_hi : a.n_lo;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = lane >> 2, c = lane & 3;
@@ -191,7 +197,7 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
   auto consumer_sync = [] { asm volatile("bar.sync 1, %0;\n" ::"n"(NCW * 32) : "memory"); };
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::NSTAGE; ++s) {
+    for (int s = 0; s < C::NMAX; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], NCW);
     }
@@ -225,12 +231,17 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
         tma_prefetch_desc(&tm_vsz);
       }
       // A CTA whose range spans pairs streams exactly its own tiles of each.
-      // The CTAs whose ranges lie inside one pair share the middle of that
-      // pair (everything but its boundary CTAs' tiles): each claims the next
-      // tile from the pair's counter, one claim ahead of use so that the
-      // atomic's latency hides behind the stage wait.  A stage with tile -1
-      // and no copy ends the piece.
+      // The CTAs whose ranges lie inside one pair (the pool) share the middle
+      // of that pair (everything but its boundary CTAs' tiles): the first
+      // three quarters of the pool's tiles are dealt out round-robin (pool CTA
+      // c takes tiles c, c + npool, ...), so the ring fills at once and the
+      // pool's CTAs read neighbouring tiles at the same time; the rest are
+      // claimed one at a time from the pair's counter (issued one claim ahead
+      // of use, so the atomic's latency hides behind the stage wait), which
+      // evens out uneven CTA speeds.  A stage with tile -1 and no copy ends
+      // the piece.
       int n = 0;                                   // stages issued
+      int ps = 0, pu = 0;                          // stage of issue n, parity of n / nst
       bool stop = false;
       for (int bh = bh_a; bh <= bh_b && !stop; ++bh) {
         if (bh > bh_a && !mbar_wait(merged, (bh - bh_a - 1) & 1)) {
@@ -240,22 +251,32 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
         }
         const long long base = (long long)bh * L.t;
         const bool dyn = bh_a == bh_b;
-        int t0, t1;
+        int t0, t1, q = 0, pc = 0, npool = 1;
         if (dyn) {
           const int i0 = cta_of(L, base), i1 = cta_of(L, base + L.t - 1);
-          const long long s0 = range_start(L, i0) < base ? range_start(L, i0 + 1) : base;
-          const long long s1 = range_start(L, i1 + 1) > base + L.t ? range_start(L, i1) : base + L.t;
-          t0 = (int)(s0 - base);
-          t1 = (int)(s1 - base);
+          const int first = range_start(L, i0) < base ? i0 + 1 : i0;
+          const int last = range_start(L, i1 + 1) > base + L.t ? i1 - 1 : i1;
+          t0 = (int)(range_start(L, first) - base);
+          t1 = (int)(range_start(L, last + 1) - base);
+          npool = last - first + 1;
+          pc = cta - first;
+          q = (t1 - t0) * 3 / (4 * npool);         // dealt tiles per pool CTA
         } else {
           t0 = (int)((g0 > base ? g0 : base) - base);
           t1 = (int)((g1 < base + L.t ? g1 : base + L.t) - base);
         }
         unsigned *ctr = a.tilectr + (hi ? a.nbh : 0) + bh;
-        int t = dyn ? t0 + (int)atomicAdd(ctr, 1u) : t0;
+        int nclaim = 0;
+        auto claim = [&]() -> int {
+          const int kk = nclaim++;
+          if (!dyn) return t0 + kk;
+          if (kk < q) return t0 + pc + npool * kk;
+          return t0 + npool * q + (int)atomicAdd(ctr, 1u);
+        };
+        int t = claim();
         for (;;) {
-          const int s = n & (nst - 1);
-          if (n >= nst && !mbar_wait(&empty[s], ((n >> lnst) & 1) ^ 1)) {
+          const int s = ps;
+          if (n >= nst && !mbar_wait(&empty[s], pu ^ 1)) {
             *abort_flag = 1;
             raise_status(a.status, HQ_DEV_TIMEOUT);
             stop = true;
@@ -266,12 +287,16 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
             break;
           }
           ++n;
+          if (++ps == nst) {
+            ps = 0;
+            pu ^= 1;
+          }
           if (t >= t1) {                           // the piece is done: end marker
             meta[s] = -1;
             mbar_arrive(&full[s]);
             break;
           }
-          const int t_next = dyn ? t0 + (int)atomicAdd(ctr, 1u) : t + 1;
+          const int t_next = claim();
           meta[s] = t;
           uint8_t *st = smem + s * stage_bytes;
           const int tok = t * T;
@@ -293,7 +318,7 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
       }
       // Never leave the CTA with copies in flight.
       for (int i = n > nst ? n - nst : 0; i < n; ++i)
-        if (!mbar_wait(&full[i & (nst - 1)], (i >> lnst) & 1)) raise_status(a.status, HQ_DEV_TIMEOUT);
+        if (!mbar_wait(&full[i % nst], (i / nst) & 1)) raise_status(a.status, HQ_DEV_TIMEOUT);
     }
     __syncwarp();
   }
@@ -304,7 +329,8 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
   // for the last arrival, the merge of all the pair's pieces.
   if (warp < NCW) {
     const int j = warp;  // this warp's 16-token sub-tile of every stage
-    int n = 0;           // tiles consumed
+    int n = 0;           // stages consumed
+    int cs = 0, cu = 0;  // stage of consumption n, parity of n / nst
     int cq = 0;          // partial chunks loaded so far (phases of cbar)
     for (int bh = bh_a; bh <= bh_b; ++bh) {
       const int b = bh / a.Hkv, kh = bh % a.Hkv;
@@ -376,22 +402,27 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
         const __half ql16 = __float2half_rn(Q - __half2float(qh16));
         zb0 = (uint32_t)__half_as_ushort(qh16) | ((uint32_t)__half_as_ushort(ql16) << 16);
       }
+      // (A producer that gave up issues no more stages: the bounded wait below
+      // then runs out here too, so the tiles need no abort check of their own.)
       for (;;) {
-        if (*abort_flag) break;
-        const int s = n & (nst - 1);
-        if (!mbar_wait(&full[s], (n >> lnst) & 1)) {
+        const int s = cs;
+        if (!mbar_wait(&full[s], cu)) {
           *abort_flag = 1;
           raise_status(a.status, HQ_DEV_TIMEOUT);
           break;
         }
         ++n;
+        if (++cs == nst) {
+          cs = 0;
+          cu ^= 1;
+        }
         const int t = meta[s];
         if (t < 0) {                               // end of this piece
           __syncwarp();
           if (lane == 0) mbar_arrive(&empty[s]);
           break;
         }
-        if (!*abort_flag) {
+        {
         uint8_t *const stp = smem + s * stage_bytes;
         const uint32_t st = smem_u32(stp);
         const int tok0 = t * T + j * 16;
@@ -401,10 +432,6 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
         // ---------------- scores S^T (16 tokens x 8 heads) ----------------
         if (!hi) {
           float acc[4][4];
-  #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            acc[g][0] = acc[g][1] = acc[g][2] = acc[g][3] = 0.f;
-          }
           const int mi = lane >> 3;
           const int lrow = row0 + (mi & 1) * 8 + (lane & 7);
           if (BITS == 4) {
@@ -426,7 +453,7 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
                 fb[1] = A18 & 0x000F000Fu;
                 fb[2] = A08 & 0x00F000F0u;
                 fb[3] = A18 & 0x00F000F0u;
-                mma_f16_16816(acc[g], fa, qb[2 * g][0], qb[2 * g][1]);
+                mma_f16_16816_z(acc[g], fa, qb[2 * g][0], qb[2 * g][1]);
                 mma_f16_16816(acc[g], fb, qb[2 * g + 1][0], qb[2 * g + 1][1]);
               }
             }
@@ -446,7 +473,8 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
                 fa[1] = f8pair(A1, 0x1404);
                 fa[2] = f8pair(A0, 0x3424);       // bytes 2, 3
                 fa[3] = f8pair(A1, 0x3424);
-                mma_f16_16816(acc[kc >> 1], fa, qb[kc][0], qb[kc][1]);
+                if (kc & 1) mma_f16_16816(acc[kc >> 1], fa, qb[kc][0], qb[kc][1]);
+                else mma_f16_16816_z(acc[kc >> 1], fa, qb[kc][0], qb[kc][1]);
               }
             }
           } else {
@@ -464,7 +492,8 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
                 fa[1] = prmt(A1, 0u, 0x4140);
                 fa[2] = prmt(A0, 0u, 0x4342);
                 fa[3] = prmt(A1, 0u, 0x4342);
-                mma_f16_16816(acc[kc >> 1], fa, qb[kc][0], qb[kc][1]);
+                if (kc & 1) mma_f16_16816(acc[kc >> 1], fa, qb[kc][0], qb[kc][1]);
+                else mma_f16_16816_z(acc[kc >> 1], fa, qb[kc][0], qb[kc][1]);
               }
             }
           }
@@ -474,16 +503,16 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
           const uint32_t wr[4] = {s_r.x, s_r.y, s_r.z, s_r.w};
           const uint32_t wr8[4] = {s_r8.x, s_r8.y, s_r8.z, s_r8.w};
           uint32_t za[4];
-          // (z of group c) in both halves; c is lane-dependent, so select
-          // instead of indexing (an indexed array would live in local memory)
-          const uint32_t wc_ = c == 0 ? wr[0] : c == 1 ? wr[1] : c == 2 ? wr[2] : wr[3];
-          const uint32_t wc8 = c == 0 ? wr8[0] : c == 1 ? wr8[1] : c == 2 ? wr8[2] : wr8[3];
+          // (z of group c) in both halves: the (s, z) word of group c of the
+          // two tokens, loaded on its own (c is lane-dependent)
+          const uint32_t wc_ = *reinterpret_cast<const uint32_t *>(stp + 2 * C::KC + (row0 + r) * 16 + c * 4);
+          const uint32_t wc8 = *reinterpret_cast<const uint32_t *>(stp + 2 * C::KC + (row0 + r + 8) * 16 + c * 4);
           za[0] = prmt(wc_, wc_, 0x3232);
           za[1] = prmt(wc8, wc8, 0x3232);
           za[2] = 0u;
           za[3] = 0u;
           float zacc[4] = {0.f, 0.f, 0.f, 0.f};
-          if (!F8) mma_f16_16816(zacc, za, zb0, 0u);   // FP8 has no zero point
+          if (!F8) mma_f16_16816_z(zacc, za, zb0, 0u);   // FP8 has no zero point
           float y[4] = {0.f, 0.f, 0.f, 0.f};
   #pragma unroll
           for (int g = 0; g < 4; ++g) {
@@ -766,7 +795,7 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
         float *cstar = cl + G * np;                           // [G] 1 / total sum
         uint8_t *cbuf0 = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(cstar + 8) + 127) & ~uintptr_t(127));
         constexpr uint32_t PB = G * D * 4;                    // bytes of one piece's partial output
-        const uint32_t avail = (uint32_t)(smem + C::NSTAGE * C::STAGE - cbuf0);
+        const uint32_t avail = (uint32_t)(smem + C::RING - cbuf0);
         int chk = (int)(avail / 2 / PB);
         chk = chk < 1 ? 1 : (chk > 32 ? 32 : chk);
         uint8_t *const cbuf1 = cbuf0 + chk * PB;

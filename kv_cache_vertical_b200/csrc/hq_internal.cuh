@@ -57,9 +57,12 @@ cudaError_t pdl_launch(void (*kernel)(Params...), dim3 grid, dim3 block, size_t 
 // Low rows allocated per (b, kv head) of a cache (lo_cap, 0 meaning n_lo).
 inline int lo_rows(const hq_kv_cache &c) { return c.lo_cap > 0 ? c.lo_cap : c.n_lo; }
 
+// The pack writes the rows [lo0, lo0 + out.n_lo) of the low segment and
+// [hi0, hi0 + out.n_hi) of the bf16 segment (the whole cache: lo0 = hi0 = 0).
 cudaError_t launch_pack(const __nv_bfloat16 *k, const __nv_bfloat16 *v, const int32_t *idx,
                         int B, int Hkv, int L, int D, int window, int k_vert, int bits,
-                        const hq_kv_cache &out, uint32_t *status, cudaStream_t s);
+                        const hq_kv_cache &out, uint32_t *status, cudaStream_t s, int lo0 = 0,
+                        int hi0 = 0);
 cudaError_t launch_kv_append(const __nv_bfloat16 *k_new, const __nv_bfloat16 *v_new, int B,
                              int Hkv, int D, int L, int window, int k_vert,
                              const hq_kv_cache &c, cudaStream_t s);
@@ -86,6 +89,15 @@ cudaError_t launch_probe_shard_topk(const __nv_bfloat16 *q_probe, int64_t q_head
 cudaError_t launch_probe_merge_topk(const int32_t *cand_idx, const float *cand_score, int R, int B,
                                     int Hkv, int L, int window, int k_vert, int32_t *idx_out,
                                     uint8_t *ws, uint32_t *status, cudaStream_t s);
+
+// tcgen05 probe passes (probe_tc.cu) over keys [0, Ls) whose probe rows sit
+// at key positions qpos0 + p; D in {64, 128}, G <= 8, P <= 64.
+bool probe_tc_supported(int D, int G, int P);
+int probe_tc_chunks(int nbh, int Ls);
+cudaError_t launch_probe_pass(bool colsum, const __nv_bfloat16 *q_probe, int64_t q_head_stride,
+                              const __nv_bfloat16 *k, int B, int Hq, int Hkv, int P, int Ls, int D,
+                              int qpos0, float scale, float2 *partial, int nchunk,
+                              const float2 *stats, float *score, uint32_t *status, cudaStream_t s);
 
 bool decode_tma_supported(int D, int bits, int G);
 size_t decode_tma_ws_bytes(int B, int Hq, int Hkv, int n_lo, int n_hi, int bits);

@@ -262,11 +262,14 @@ constexpr int kSpan = kWarps * kChunks * 8;   // 256
 // those inside it in a shared bit mask, while every warp issues the row loads
 // of its first chunk; then each warp classifies and writes its four chunks of
 // eight positions (copy the bf16 rows, or quantize them into the next low
-// rows), each lane one 32-channel group of one row.
+// rows), each lane one 32-channel group of one row.  With a part [lo0, lo1) x
+// [hi0, hi1) of the cache's rows (a context split across GPUs), only the rows
+// inside it are written, at their offsets from lo0 / hi0.
 template <int D, int BITS, bool F8>
 __global__ void __launch_bounds__(kWarps * 32)
 pack_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ v,
-            const int32_t *__restrict__ idx, int nbh, int L, int window, int k_vert, int lo_cap,
+            const int32_t *__restrict__ idx, int nbh, int L, int window, int k_vert,
+            int lo0, int lo1, int hi0, int hi1, int lo_cap,
             uint8_t *__restrict__ k_codes, uint8_t *__restrict__ v_codes,
             __half2 *__restrict__ k_sz, __half2 *__restrict__ v_sz,
             __nv_bfloat16 *__restrict__ k_hi, __nv_bfloat16 *__restrict__ v_hi,
@@ -278,6 +281,7 @@ pack_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict
   __shared__ int s_lo;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int n_lo = L - window - k_vert, n_hi = k_vert + window;
+  const int part_hi = hi1 - hi0;               // bf16 rows of the part (its row stride)
   const int nspan = (L + kSpan - 1) / kSpan;
   const int bh = (int)(blockIdx.x / nspan);
   const int p0 = (int)(blockIdx.x % nspan) * kSpan;
@@ -359,7 +363,9 @@ pack_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict
           raise_status(status, HQ_DEV_BAD_INDEX);
           continue;
         }
-        uint4 *dst = reinterpret_cast<uint4 *>((is_v ? v_hi : k_hi) + ((size_t)bh * n_hi + hi_row) * D + g * 32);
+        if (hi_row < hi0 || hi_row >= hi1) continue;   // another part's row
+        uint4 *dst = reinterpret_cast<uint4 *>((is_v ? v_hi : k_hi) +
+                                               ((size_t)bh * part_hi + hi_row - hi0) * D + g * 32);
 #pragma unroll
         for (int u = 0; u < 4; ++u)
           dst[u] = make_uint4(w[pi][4 * u], w[pi][4 * u + 1], w[pi][4 * u + 2], w[pi][4 * u + 3]);
@@ -368,7 +374,8 @@ pack_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict
           raise_status(status, HQ_DEV_BAD_INDEX);
           continue;
         }
-        const size_t r = (size_t)bh * lo_cap + lo_row;
+        if (lo_row < lo0 || lo_row >= lo1) continue;   // another part's row
+        const size_t r = (size_t)bh * lo_cap + lo_row - lo0;
         quant_group_lane<BITS, F8>(w[pi], (is_v ? v_codes : k_codes) + r * ROWB + g * (32 * BITS / 8),
                                    (is_v ? v_sz : k_sz) + r * NG + g);
         if (lo_pos && !is_v && g == 0) lo_pos[r] = j;
@@ -379,12 +386,13 @@ pack_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict
 
 template <int D, int BITS, bool F8>
 cudaError_t launch_pack_t(const __nv_bfloat16 *k, const __nv_bfloat16 *v, const int32_t *idx,
-                          int nbh, int L, int window, int k_vert, const hq_kv_cache &o,
-                          uint32_t *status, cudaStream_t s) {
+                          int nbh, int L, int window, int k_vert, int lo0, int hi0,
+                          const hq_kv_cache &o, uint32_t *status, cudaStream_t s) {
   const long long blocks = (long long)nbh * ((L + kSpan - 1) / kSpan);
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
   pack_kernel<D, BITS, F8><<<(unsigned)blocks, kWarps * 32, 0, s>>>(
-      k, v, idx, nbh, L, window, k_vert, lo_rows(o), (uint8_t *)o.k_codes, (uint8_t *)o.v_codes,
+      k, v, idx, nbh, L, window, k_vert, lo0, lo0 + o.n_lo, hi0, hi0 + o.n_hi, lo_rows(o),
+      (uint8_t *)o.k_codes, (uint8_t *)o.v_codes,
       (__half2 *)o.k_sz, (__half2 *)o.v_sz, (__nv_bfloat16 *)o.k_hi, (__nv_bfloat16 *)o.v_hi,
       o.lo_pos, status);
   return cudaGetLastError();
@@ -461,11 +469,11 @@ cudaError_t launch_kv_append_t(const __nv_bfloat16 *k_new, const __nv_bfloat16 *
 
 cudaError_t launch_pack(const __nv_bfloat16 *k, const __nv_bfloat16 *v, const int32_t *idx,
                         int B, int Hkv, int L, int D, int window, int k_vert, int bits,
-                        const hq_kv_cache &out, uint32_t *status, cudaStream_t s) {
+                        const hq_kv_cache &out, uint32_t *status, cudaStream_t s, int lo0, int hi0) {
   const int nbh = B * Hkv;
   const bool f8 = out.fmt == HQ_KV_FP8;
 #define HQ_P(DD, BB, FF) \
-  if (D == DD && bits == BB && f8 == FF) return launch_pack_t<DD, BB, FF>(k, v, idx, nbh, L, window, k_vert, out, status, s);
+  if (D == DD && bits == BB && f8 == FF) return launch_pack_t<DD, BB, FF>(k, v, idx, nbh, L, window, k_vert, lo0, hi0, out, status, s);
   HQ_P(128, 4, false) HQ_P(128, 8, false) HQ_P(64, 4, false) HQ_P(64, 8, false)
   HQ_P(128, 8, true) HQ_P(64, 8, true)
 #undef HQ_P

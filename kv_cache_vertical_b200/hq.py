@@ -70,6 +70,10 @@ hq_decode_workspace_size = _sig("hq_decode_workspace_size", _SZ, _I, _I, _I, _I,
 _decode = _sig("hq_decode_attn", _I, _P, ctypes.POINTER(hq_kv_cache), _I, _I, _I, _I, _F, _P, _P,
                _P, _SZ, _P)
 _append = _sig("hq_kv_append", _I, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.POINTER(hq_kv_cache), _P)
+_pack_part = _sig("hq_pack_kv_part", _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _I,
+                  ctypes.POINTER(hq_kv_cache), _P, _SZ, _P)
+_append_part = _sig("hq_kv_append_part", _I, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I,
+                    ctypes.POINTER(hq_kv_cache), _P)
 _merge = _sig("hq_decode_merge", _I, _P, _P, _I, _I, _I, _I, _P, _P, _P)
 _decode_static = _sig("hq_decode_attn_static", _I, _P, ctypes.POINTER(hq_kv_cache), _I, _I, _I,
                       _I, _F, _P, _P, _P)
@@ -89,7 +93,8 @@ EXPORTED = ["hq_status_string", "hq_version", "hq_read_device_status", "hq_probe
             "hq_decode_attn_static", "hq_read_static_status", "hq_kv_append", "hq_decode_merge", "hq_prefill_quant_ex",
             "hq_prefill_attn_ex", "hq_probe_shard_workspace_size", "hq_probe_shard_stats",
             "hq_probe_merge_stats", "hq_probe_shard_topk", "hq_probe_merge_workspace_size",
-            "hq_probe_merge_topk", "hq_prefill_supported"]
+            "hq_probe_merge_topk", "hq_prefill_supported", "hq_pack_kv_part",
+            "hq_kv_append_part"]
 
 HQ_ERR_SCRATCH_LIMIT = 7
 STATIC_SCRATCH_BYTES = 8 << 20
@@ -158,7 +163,13 @@ class KVCache:
               lo_cap=None, fmt=HQ_KV_INT):
         """Buffers for a cache of L tokens.  lo_cap (default: exactly the
         n_lo low rows) reserves low rows per (b, kv head) for decode appends."""
-        n_lo, n_hi = L - window - k_vert, k_vert + window
+        return cls.alloc(B, Hkv, D, L - window - k_vert, k_vert + window, bits, device, with_pos,
+                         lo_cap, fmt)
+
+    @classmethod
+    def alloc(cls, B, Hkv, D, n_lo, n_hi, bits, device="cuda", with_pos=True, lo_cap=None,
+              fmt=HQ_KV_INT):
+        """Buffers for n_lo low rows (lo_cap allocated) and n_hi bf16 rows."""
         C = n_lo if lo_cap is None else int(lo_cap)
         assert C >= n_lo, "lo_cap below the number of low rows"
         u8 = dict(dtype=torch.uint8, device=device)
@@ -258,6 +269,21 @@ def hq_pack_kv(k, v, idx, B, Hkv, L, D, window, k_vert, bits, group, cache: KVCa
     _check(_pack(_ptr(k), _ptr(v), _ptr(idx), B, Hkv, L, D, window, k_vert, bits, group,
                  ctypes.byref(st), _ptr(ws), ws.numel() if ws is not None else 0,
                  _stream(stream)), "hq_pack_kv")
+
+
+def hq_pack_kv_part(k, v, idx, B, Hkv, L, D, window, k_vert, bits, group, lo0, hi0,
+                    cache: KVCache, ws=None, stream=None):
+    st = cache.struct()
+    _check(_pack_part(_ptr(k), _ptr(v), _ptr(idx), B, Hkv, L, D, window, k_vert, bits, group, lo0,
+                      hi0, ctypes.byref(st), _ptr(ws), ws.numel() if ws is not None else 0,
+                      _stream(stream)), "hq_pack_kv_part")
+
+
+def hq_kv_append_part(k_new, v_new, B, Hkv, D, L, window, k_vert, lo0, hi0, cache: KVCache,
+                      stream=None):
+    st = cache.struct()
+    _check(_append_part(_ptr(k_new), _ptr(v_new), B, Hkv, D, L, window, k_vert, lo0, hi0,
+                        ctypes.byref(st), _stream(stream)), "hq_kv_append_part")
 
 
 def hq_kv_append(k_new, v_new, B, Hkv, D, L, window, k_vert, cache: KVCache, stream=None):
@@ -402,11 +428,9 @@ def probe_merge_topk(cand_idx, cand_score, L, window, ws=None):
 def probe_context_parallel(q_probe, k_shard, key_off, L, window, k_vert, group=None, scale=0.0):
     """The vertical-column probe with the context's keys split over the ranks
     of `group` (torch.distributed): this rank holds keys [key_off, key_off +
-    k_shard.shape[2]).  Two all-gathers: the probe rows' partial (max, Z), then
-    every rank's top-k candidates.  Returns the context's index list on every
-    rank."""
-    import torch.distributed as dist
-    R = dist.get_world_size(group)
+    k_shard.shape[2]).  Two all-gathers (NCCL on device memory, gloo through
+    the host): the probe rows' partial (max, Z), then every rank's top-k
+    candidates.  Returns the context's index list on every rank."""
     B, Hq, P, D = q_probe.shape
     Hkv = k_shard.shape[1]
     empty = k_shard.shape[2] == 0          # more ranks than keys: this rank holds none
@@ -415,20 +439,15 @@ def probe_context_parallel(q_probe, k_shard, key_off, L, window, k_vert, group=N
         st[..., 0] = -torch.finfo(torch.float32).max
     else:
         st = probe_shard_stats(q_probe, k_shard, key_off, L, scale)
-    parts = [torch.empty_like(st) for _ in range(R)]
-    dist.all_gather(parts, st, group=group)
-    stats = probe_merge_stats(torch.stack(parts))
+    stats = probe_merge_stats(torch.stack(_all_gather(st, group)))
     if empty:
         ci = torch.full((B, Hkv, k_vert), -1, dtype=torch.int32, device=q_probe.device)
         cs = torch.full((B, Hkv, k_vert), -torch.finfo(torch.float32).max, dtype=torch.float32,
                         device=q_probe.device)
     else:
         ci, cs = probe_shard_topk(q_probe, k_shard, key_off, L, window, k_vert, stats, scale)
-    cis = [torch.empty_like(ci) for _ in range(R)]
-    css = [torch.empty_like(cs) for _ in range(R)]
-    dist.all_gather(cis, ci, group=group)
-    dist.all_gather(css, cs, group=group)
-    return probe_merge_topk(torch.stack(cis), torch.stack(css), L, window)
+    return probe_merge_topk(torch.stack(_all_gather(ci, group)), torch.stack(_all_gather(cs, group)),
+                            L, window)
 
 
 def pack_kv(k, v, idx, window, bits=4, ws=None, with_pos=True, lo_cap=None,
@@ -438,6 +457,30 @@ def pack_kv(k, v, idx, window, bits=4, ws=None, with_pos=True, lo_cap=None,
     cache = KVCache.empty(B, Hkv, L, D, window, k_vert, bits, k.device, with_pos, lo_cap, fmt)
     hq_pack_kv(k, v, idx, B, Hkv, L, D, window, k_vert, bits, 32, cache, ws)
     return cache
+
+
+def pack_kv_part(k, v, idx, window, part, bits=4, ws=None, with_pos=True, lo_cap=None,
+                 fmt=HQ_KV_INT) -> KVCache:
+    """One rank's part (lo0, lo1, hi0, hi1) of the cache pack_kv would build
+    (a context split; see context_split_plan): only those rows are allocated
+    and written, bit-identical to the whole cache's rows."""
+    B, Hkv, L, D = k.shape
+    k_vert = idx.shape[2]
+    lo0, lo1, hi0, hi1 = part
+    cache = KVCache.alloc(B, Hkv, D, lo1 - lo0, hi1 - hi0, bits, k.device, with_pos, lo_cap, fmt)
+    hq_pack_kv_part(k, v, idx, B, Hkv, L, D, window, k_vert, bits, 32, lo0, hi0, cache, ws)
+    return cache
+
+
+def kv_append_part(part_cache: KVCache, part, k_new, v_new, L, window, k_vert, stream=None):
+    """Token L enters a context-split cache on the rank whose part ends where
+    the cache ends (the last rank of context_split_plan(..., window=W)); the
+    other ranks' parts do not change.  The part's n_lo grows by one."""
+    B, Hkv, D = k_new.shape
+    lo0, _, hi0, _ = part
+    hq_kv_append_part(k_new, v_new, B, Hkv, D, L, window, k_vert, lo0, hi0, part_cache, stream)
+    part_cache.n_lo += 1
+    return part_cache
 
 
 def kv_append(cache: KVCache, k_new, v_new, L, window, stream=None):
@@ -495,18 +538,38 @@ def default_scale(D: int) -> float:
 # ---------------------------------------------------------------------------
 # Context split of the decode across ranks
 # ---------------------------------------------------------------------------
-def context_split_plan(n_lo: int, n_hi: int, R: int, align: int = 64):
+def context_split_plan(n_lo: int, n_hi: int, R: int, align: int = 64, window: int = 0):
     """Share the rows of one cache among R ranks for a context-split decode:
     rank r gets low rows [lo0, lo1) and bf16 rows [hi0, hi1).  Attention does
     not depend on the order of the rows, so any disjoint cover works; equal
     shares of both kinds give every rank the same bytes to read.  Low
     boundaries fall on multiples of `align` rows (whole decode tiles, 16-byte
-    aligned views).  Returns [(lo0, lo1, hi0, hi1)] * R."""
+    aligned views).  With window > 0 the last rank's bf16 rows include the
+    whole window (the last `window` bf16 rows), so that decode appends
+    (kv_append_part) touch that rank only.  Returns [(lo0, lo1, hi0, hi1)] * R."""
     if R < 1:
         raise ValueError("R must be at least 1")
     lo = [min(n_lo, (n_lo * r // R) // align * align) for r in range(R)] + [n_lo]
     hi = [n_hi * r // R for r in range(R + 1)]
+    if window > 0:
+        cap = max(0, n_hi - window)
+        hi = [min(h, cap) for h in hi[:-1]] + [n_hi]
     return [(lo[r], lo[r + 1], hi[r], hi[r + 1]) for r in range(R)]
+
+
+def _all_gather(t: torch.Tensor, group=None):
+    """All-gather of a device tensor: NCCL gathers device memory directly;
+    a process group without device collectives (gloo) gathers host copies."""
+    import torch.distributed as dist
+    R = dist.get_world_size(group)
+    if dist.get_backend(group) == "nccl":
+        parts = [torch.empty_like(t) for _ in range(R)]
+        dist.all_gather(parts, t, group=group)
+        return parts
+    th = t.cpu()
+    parts = [torch.empty_like(th) for _ in range(R)]
+    dist.all_gather(parts, th, group=group)
+    return [x.to(t.device) for x in parts]
 
 
 def decode_merge(part_out, part_lse):
@@ -518,24 +581,19 @@ def decode_merge(part_out, part_lse):
     return out, lse
 
 
-def decode_context_parallel(q, cache: KVCache, Hkv, group=None, scale=0.0):
-    """Decode one step with the cache's rows split over the ranks of `group`
-    (torch.distributed, NCCL): each rank decodes its part of context_split_plan
-    (taken from its copy of the packed cache), the
-    (out, lse) pairs are all-gathered, and every rank merges them.  Returns
-    (out, lse) of the whole cache."""
-    import torch.distributed as dist
-    R = dist.get_world_size(group)
-    r = dist.get_rank(group)
+def decode_context_parallel(q, part: KVCache, Hkv, group=None, scale=0.0):
+    """Decode one step of a cache whose rows are split over the ranks of
+    `group` (torch.distributed): `part` is this rank's rows (pack_kv_part with
+    this rank's entry of context_split_plan, or rows_part of a replica).  Each
+    rank decodes its part with its log-sum-exp, the (out, lse) pairs are
+    all-gathered (NCCL on device memory, gloo through the host), and every
+    rank merges them exactly.  Returns (out, lse) of the whole cache."""
     B, Hq, D = q.shape
-    part = cache.rows_part(*context_split_plan(cache.n_lo, cache.n_hi, R)[r])
     if part.n_lo + part.n_hi > 0:
         out_r, lse_r = decode_attn(q, part, Hkv, scale=scale, want_lse=True)
     else:
         out_r = torch.zeros(B, Hq, D, dtype=torch.float32, device=q.device)
         lse_r = torch.full((B, Hq), float("-inf"), dtype=torch.float32, device=q.device)
-    outs = [torch.empty_like(out_r) for _ in range(R)]
-    lses = [torch.empty_like(lse_r) for _ in range(R)]
-    dist.all_gather(outs, out_r, group=group)
-    dist.all_gather(lses, lse_r, group=group)
+    outs = _all_gather(out_r, group)
+    lses = _all_gather(lse_r, group)
     return decode_merge(torch.stack(outs), torch.stack(lses))
