@@ -310,6 +310,18 @@ def decode_configs(H, dev, stream, world, rank, reps=15):
     return res
 
 
+def decode_roofline(dconf, name, pk):
+    """Roofline fields of the decode kernel on one decode workload of the
+    decode_configs leg (DRAM traffic from the committed ncu record of that
+    workload, or null once the kernel's sources have changed)."""
+    c = dconf[name]
+    return {"kernel": "decode_tma (hq_decode_attn)", "workload": name, "bound": "hbm",
+            "achieved": c["gbs"], "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": c["frac"],
+            "traffic": profiled_traffic("decode_tma"), "algorithmic_bytes": c["algorithmic_bytes"],
+            "us": c["us_median"], "peak_src": pk["src"] + " (copy bandwidth)",
+            "frac_of_8TBs": c["frac_of_8TBs"]}
+
+
 def decode_graph(H, w, q_dec, cache, out, ws, dev, world, n=50, reps=7):
     """The packed 32K decode as n back-to-back calls captured in one CUDA
     graph, replayed `reps` times: per-call median and best.  The 47 MB cache
@@ -662,11 +674,16 @@ def main():
                      "peak_src": pk["src"] + " bf16 burst GEMM peak; INT8 = the larger of bf16 x "
                                  "nominal ratio 2 and the INT8 GEMM measured in this run "
                                  "(torch._int_mm 8192^3); peak = work-weighted mix of the two"},
-        "decode": {"kernel": "decode_tma (hq_decode_attn)", "bound": "hbm", "achieved": dec_tbs * 1e3,
-                   "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": dec_tbs * 1e3 / pk["hbm_gbs"],
-                   "traffic": profiled_traffic("decode_tma"), "algorithmic_bytes": r["dbytes"],
-                   "us": per["decode"] * 1e3, "peak_src": pk["src"] + " (copy bandwidth)",
-                   "frac_of_8TBs": dec_tbs / 8.0},
+        # the decode kernel's roofline on the largest decode workload of the
+        # specification (70B-shaped, 2.9 GB cache: HBM-bound); the step's 32K
+        # decode, whose throughput is `value`, follows as decode_step
+        "decode": decode_roofline(r["dconf"], "70b_decode_64k", pk),
+        "decode_step": {"kernel": "decode_tma (hq_decode_attn)", "bound": "hbm",
+                        "achieved": dec_tbs * 1e3, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                        "frac": dec_tbs * 1e3 / pk["hbm_gbs"], "algorithmic_bytes": r["dbytes"],
+                        "us": per["decode"] * 1e3, "peak_src": pk["src"] + " (copy bandwidth)",
+                        "frac_of_8TBs": dec_tbs / 8.0,
+                        "note": "the 32K layer's decode inside the step (latency-bound at 47 MB)"},
         "per_call_ms": {n: per[n] for n in ("probe", "prefill", "pack", "decode")},
         "probe_frac_of_prefill": per["probe"] / per["prefill"],
         # token-by-token decode after the timed steps: cache maintenance + attention

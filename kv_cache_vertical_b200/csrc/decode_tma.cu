@@ -232,14 +232,13 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
       }
       // A CTA whose range spans pairs streams exactly its own tiles of each.
       // The CTAs whose ranges lie inside one pair (the pool) share the middle
-      // of that pair (everything but its boundary CTAs' tiles): the first
-      // three quarters of the pool's tiles are dealt out round-robin (pool CTA
-      // c takes tiles c, c + npool, ...), so the ring fills at once and the
-      // pool's CTAs read neighbouring tiles at the same time; the rest are
-      // claimed one at a time from the pair's counter (issued one claim ahead
-      // of use, so the atomic's latency hides behind the stage wait), which
-      // evens out uneven CTA speeds.  A stage with tile -1 and no copy ends
-      // the piece.
+      // of that pair (everything but its boundary CTAs' tiles): each claims
+      // the next tile from the pair's counter, one claim ahead of use so that
+      // the atomic's latency hides behind the stage wait; the pool's CTAs read
+      // neighbouring tiles at the same time and uneven CTA speeds even out.
+      // (Dealing most of the pool out round-robin or in static blocks before
+      // claiming the rest was measured slower on every decode workload.)  A
+      // stage with tile -1 and no copy ends the piece.
       int n = 0;                                   // stages issued
       int ps = 0, pu = 0;                          // stage of issue n, parity of n / nst
       bool stop = false;
@@ -251,16 +250,13 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
         }
         const long long base = (long long)bh * L.t;
         const bool dyn = bh_a == bh_b;
-        int t0, t1, q = 0, pc = 0, npool = 1;
+        int t0, t1;
         if (dyn) {
           const int i0 = cta_of(L, base), i1 = cta_of(L, base + L.t - 1);
           const int first = range_start(L, i0) < base ? i0 + 1 : i0;
           const int last = range_start(L, i1 + 1) > base + L.t ? i1 - 1 : i1;
           t0 = (int)(range_start(L, first) - base);
           t1 = (int)(range_start(L, last + 1) - base);
-          npool = last - first + 1;
-          pc = cta - first;
-          q = (t1 - t0) * 3 / (4 * npool);         // dealt tiles per pool CTA
         } else {
           t0 = (int)((g0 > base ? g0 : base) - base);
           t1 = (int)((g1 < base + L.t ? g1 : base + L.t) - base);
@@ -268,10 +264,7 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
         unsigned *ctr = a.tilectr + (hi ? a.nbh : 0) + bh;
         int nclaim = 0;
         auto claim = [&]() -> int {
-          const int kk = nclaim++;
-          if (!dyn) return t0 + kk;
-          if (kk < q) return t0 + pc + npool * kk;
-          return t0 + npool * q + (int)atomicAdd(ctr, 1u);
+          return dyn ? t0 + (int)atomicAdd(ctr, 1u) : t0 + nclaim++;
         };
         int t = claim();
         for (;;) {
