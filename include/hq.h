@@ -25,10 +25,11 @@
  *     and keeps no state between calls.  `stream` is a cudaStream_t (NULL is
  *     the legacy default stream); all work is stream-ordered.
  *   Workspace: calls that need scratch take (ws, ws_bytes).  Size it with the
- *     matching hq_*_workspace_size query, allocate it on the device,
- *     zero it ONCE before its first use (cudaMemset), and keep using it; the
- *     library leaves it in a reusable state (the decode's arrival tickets and
- *     tile counters return to zero at the end of every call).  After a call
+ *     matching hq_*_workspace_size query, allocate it on the device
+ *     (16-byte aligned, as cudaMalloc returns it), zero it ONCE before its
+ *     first use (cudaMemset), and keep using it; the library leaves it in a
+ *     reusable state (the decode's tile counters return to zero at the end
+ *     of every call).  After a call
  *     that reported HQ_DEV_TIMEOUT, zero it again.  The first 16 bytes hold a
  *     device status word (see hq_read_device_status).  Calls that share one
  *     workspace must not run concurrently.

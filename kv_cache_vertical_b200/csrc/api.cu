@@ -298,6 +298,7 @@ hq_status hq_decode_attn(const void *q, const hq_kv_cache *cache, int B, int Hq,
     if (p && !aligned16(p)) return HQ_ERR_INVALID_ARG;
   if (!ws || ws_bytes < decode_ws_bytes(B, Hq, Hkv, D, cache->n_lo, cache->n_hi, cache->bits))
     return HQ_ERR_WORKSPACE;
+  if (!aligned16(ws)) return HQ_ERR_INVALID_ARG;
   return cuda_status(launch_decode((const __nv_bfloat16 *)q, *cache, B, Hq, Hkv, D,
                                    resolve_scale(softmax_scale, D), out, lse_out, (uint8_t *)ws,
                                    status_word(ws), (cudaStream_t)stream));

@@ -26,9 +26,11 @@
 //       unit 2^24 is undone when the warps are merged.
 //
 // Online softmax per head with lazy rescaling (the running max only moves when
-// a tile exceeds it by more than 2^8), a merge of the warps per piece, then the
-// last piece of each (b, kv head) to finish merges all pieces (an atomic
-// ticket, no spin waits) and writes the fp32 output and log-sum-exp.
+// a tile exceeds it by more than 2^8) and a merge of the warps per piece into
+// the piece's partial (max, sum, unnormalized output).  A second kernel,
+// launched as a programmatic dependent of the first, merges every pair's
+// pieces in parallel once they are all written and writes the fp32 output and
+// log-sum-exp.
 #include <cuda.h>
 #include <float.h>
 
@@ -73,8 +75,8 @@ struct DecArgs {
   const __nv_bfloat16 *q;
   float *part_o;          // [nslot][G][D]  unnormalized partial outputs
   float2 *part_ml;        // [nslot][G]     (max in log2 units, sum)
-  unsigned *counters;     // [B*Hkv] arrival tickets, left at zero
-  unsigned *tilectr;      // [2][B*Hkv] next unclaimed tile of each pair (low, bf16 line), left at zero
+  unsigned *tilectr;      // [2][B*Hkv] next unclaimed tile of each pair (low, bf16 line),
+                          // returned to zero by the combine kernel
   float *out, *lse;
   uint32_t *status;
   int Hq, Hkv, n_lo, n_hi;
@@ -175,11 +177,9 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::RING);
   uint64_t *empty = full + 8;
   uint64_t *merged = empty + 8;                                 // one phase per finished piece
-  uint64_t *cbar = merged + 1;                                  // [2] partial chunks of a pair merge
-  float *qsum = reinterpret_cast<float *>(cbar + 2);            // [8 heads][4 groups]
+  float *qsum = reinterpret_cast<float *>(merged + 1);          // [8 heads][4 groups]
   volatile int *abort_flag = reinterpret_cast<volatile int *>(qsum + 32);
-  int *last_flag = reinterpret_cast<int *>(qsum + 33);
-  int *meta = last_flag + 1;                                     // [nst] tile of each stage, -1: end of piece
+  int *meta = const_cast<int *>(abort_flag) + 1;                 // [nst] tile of each stage, -1: end of piece
 
   const bool hi = (int)blockIdx.x >= a.nc_lo;
   const int cta = hi ? (int)blockIdx.x - a.nc_lo : (int)blockIdx.x;
@@ -202,11 +202,8 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
       mbar_init(&empty[s], NCW);
     }
     mbar_init(merged, NCW);
-    mbar_init(&cbar[0], 1);
-    mbar_init(&cbar[1], 1);
     fence_mbar_init();
     *abort_flag = 0;
-    *last_flag = 0;
   }
   __syncthreads();
   // Everything above touched only shared memory and kernel parameters; the
@@ -324,7 +321,6 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
     const int j = warp;  // this warp's 16-token sub-tile of every stage
     int n = 0;           // stages consumed
     int cs = 0, cu = 0;  // stage of consumption n, parity of n / nst
-    int cq = 0;          // partial chunks loaded so far (phases of cbar)
     for (int bh = bh_a; bh <= bh_b; ++bh) {
       const int b = bh / a.Hkv, kh = bh % a.Hkv;
       // B fragments of q: 8 k16-chunks x 2 registers.
@@ -751,147 +747,110 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
         a.part_o[(slot * G + h) * D + d] = oo;
         if (d == 0) a.part_ml[slot * G + h] = make_float2(wm[h], wm[8 + h]);
       }
-      __threadfence();
-      consumer_sync();
-      // ---------------- arrival ticket of the pair ----------------
-      // Pieces of pair bh: CTAs i0l..i1l of the low line, i0h..i1h of the
-      // bf16 line; their partial slots are consecutive on each line.
-      int i0l = 0, i1l = -1, i0h = 0, i1h = -1;
-      if (a.tl > 0) {
-        const Line Ll = line_of(a, false);
-        i0l = cta_of(Ll, (long long)bh * a.tl);
-        i1l = cta_of(Ll, (long long)bh * a.tl + a.tl - 1);
-      }
-      if (a.th > 0) {
-        const Line Lh = line_of(a, true);
-        i0h = cta_of(Lh, (long long)bh * a.th);
-        i1h = cta_of(Lh, (long long)bh * a.th + a.th - 1);
-      }
-      const int np_lo = i1l - i0l + 1, np = np_lo + (i1h - i0h + 1);
-      if (threadIdx.x == 0) {
-        const unsigned ticket = atomicAdd(&a.counters[bh], 1u);
-        *last_flag = (ticket == (unsigned)(np - 1));
-      }
-      consumer_sync();
-      if (*last_flag) {
-        // ------------- last arrival: merge all pieces of the pair -------------
-        // (max, sum) of every piece into shared memory and one warp per head
-        // turns them into weights; the pieces' partial outputs (consecutive
-        // slots on each line) stream into two shared buffers by bulk copies,
-        // chunk k+1 in flight while chunk k is accumulated.
-        __threadfence();
-        auto slot_of = [&](int sp) -> size_t {
-          return sp < np_lo ? (size_t)(i0l + bh + sp) : (size_t)(a.nc_lo + a.nbh + i0h + bh + (sp - np_lo));
-        };
-        float *cm = reinterpret_cast<float *>(smem);          // [G][np] piece maxima -> weights
-        float *cl = cm + G * np;                              // [G][np] piece sums
-        float *cstar = cl + G * np;                           // [G] 1 / total sum
-        uint8_t *cbuf0 = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(cstar + 8) + 127) & ~uintptr_t(127));
-        constexpr uint32_t PB = G * D * 4;                    // bytes of one piece's partial output
-        const uint32_t avail = (uint32_t)(smem + C::RING - cbuf0);
-        int chk = (int)(avail / 2 / PB);
-        chk = chk < 1 ? 1 : (chk > 32 ? 32 : chk);
-        uint8_t *const cbuf1 = cbuf0 + chk * PB;
-        const size_t hq0 = (size_t)b * a.Hq + kh * G;
-        for (int e = threadIdx.x; e < G * np; e += NCW * 32) {
-          const int h = e / np, sp = e % np;
-          const float2 ml = __ldcg(&a.part_ml[slot_of(sp) * G + h]);
-          cm[e] = ml.x;
-          cl[e] = ml.y;
-        }
-        consumer_sync();
-        for (int h = warp; h < G; h += NCW) {
-          float mm = -1e30f;
-          for (int sp = lane; sp < np; sp += 32) mm = fmaxf(mm, cm[h * np + sp]);
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) mm = fmaxf(mm, __shfl_xor_sync(0xffffffffu, mm, off));
-          float ll = 0.f;
-          for (int sp = lane; sp < np; sp += 32) {
-            const float f = exp2f(cm[h * np + sp] - mm);
-            cm[h * np + sp] = f;
-            ll += f * cl[h * np + sp];
-          }
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) ll += __shfl_xor_sync(0xffffffffu, ll, off);
-          if (lane == 0) {
-            cstar[h] = 1.f / ll;
-            if (a.lse) a.lse[hq0 + h] = (mm + log2f(ll)) * 0.6931471805599453f;
-          }
-        }
-        // chunks of at most chk consecutive pieces, never across the two lines
-        const int ncl = (np_lo + chk - 1) / chk, nchunks = ncl + (np - np_lo + chk - 1) / chk;
-        auto chunk = [&](int k, int &sp0, int &cnt) {
-          if (k < ncl) {
-            sp0 = k * chk;
-            cnt = min(chk, np_lo - sp0);
-          } else {
-            sp0 = np_lo + (k - ncl) * chk;
-            cnt = min(chk, np - sp0);
-          }
-        };
-        auto issue = [&](int k) {
-          int sp0, cnt;
-          chunk(k, sp0, cnt);
-          const int gk = cq + k;
-          mbar_arrive_expect_tx(&cbar[gk & 1], cnt * PB);
-          bulk_load((gk & 1) ? cbuf1 : cbuf0, a.part_o + slot_of(sp0) * G * D, cnt * PB, &cbar[gk & 1]);
-        };
-        consumer_sync();                                      // weights ready; buffers free
-        if (threadIdx.x == 0) issue(0);
-        constexpr int NCOL = D / 4;
-        float4 acc[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
-        for (int k = 0; k < nchunks; ++k) {
-          if (threadIdx.x == 0 && k + 1 < nchunks) issue(k + 1);   // its buffer was released below
-          const int gk = cq + k;
-          const bool ready = !*abort_flag && mbar_wait(&cbar[gk & 1], (gk >> 1) & 1);
-          if (!ready && !*abort_flag) {
-            *abort_flag = 1;
-            raise_status(a.status, HQ_DEV_TIMEOUT);
-          }
-          if (ready) {
-            int sp0, cnt;
-            chunk(k, sp0, cnt);
-            const float4 *buf = reinterpret_cast<const float4 *>((gk & 1) ? cbuf1 : cbuf0);
-#pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {
-              const int item = threadIdx.x + jj * NCW * 32;
-              if (item < G * NCOL) {
-                const int h = item / NCOL, d4 = item % NCOL;
-                const float *f = cm + h * np + sp0;
-                for (int u = 0; u < cnt; ++u) {
-                  const float4 x = buf[(u * G + h) * NCOL + d4];
-                  acc[jj].x = fmaf(f[u], x.x, acc[jj].x);
-                  acc[jj].y = fmaf(f[u], x.y, acc[jj].y);
-                  acc[jj].z = fmaf(f[u], x.z, acc[jj].z);
-                  acc[jj].w = fmaf(f[u], x.w, acc[jj].w);
-                }
-              }
-            }
-          }
-          consumer_sync();                                    // buffer gk & 1 may be refilled
-        }
-        cq += nchunks;
-#pragma unroll
-        for (int jj = 0; jj < 2; ++jj) {
-          const int item = threadIdx.x + jj * NCW * 32;
-          if (item < G * NCOL) {
-            const int h = item / NCOL, d4 = item % NCOL;
-            const float inv = cstar[h];
-            reinterpret_cast<float4 *>(a.out + (hq0 + h) * D)[d4] =
-                make_float4(acc[jj].x * inv, acc[jj].y * inv, acc[jj].z * inv, acc[jj].w * inv);
-          }
-        }
-        if (threadIdx.x == 0) {
-          // every piece of the pair has stopped claiming tiles: rearm
-          a.tilectr[bh] = 0u;
-          a.tilectr[a.nbh + bh] = 0u;
-          a.counters[bh] = 0u;
-        }
-      }
       // the stage memory goes back to the producer
       asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
       consumer_sync();
       if (lane == 0) mbar_arrive(merged);
+    }
+  }
+}
+
+// Merge of every piece of one (b, kv head) pair: m* = max m_s, out = sum
+// 2^(m_s - m*) O_s / sum 2^(m_s - m*) l_s.  One CTA per (query head, pair),
+// launched as a programmatic dependent of decode_tma: its CTAs may be resident
+// early and start once every piece is written, and all heads of all pairs
+// merge in parallel.  Each of the CMW warps folds every CMW-th piece into its
+// own running (max, sum, output) -- lane l holds channels 4l..4l+3 -- taking
+// four pieces per round so that eight loads of each lane are in flight at
+// once; the warps' results are then folded the same way through shared
+// memory.  Pieces of a pair: CTAs i0l..i1l of the low line and i0h..i1h of
+// the bf16 line, their partial slots consecutive on each line.  The CTA of
+// the pair's first head also returns the pair's tile counters to zero for the
+// next call.
+constexpr int CMW = 8;                           // warps per combine CTA
+template <int G>
+__global__ void __launch_bounds__(CMW * 32)
+decode_tma_combine(DecArgs a) {
+  __shared__ float4 so[CMW][32];
+  __shared__ float sm_[CMW], sl_[CMW];
+  pdl_wait();                                    // decode_tma has completed: every partial is written
+  pdl_trigger();
+  const int h = blockIdx.x, bh = blockIdx.y;
+  const int b = bh / a.Hkv, kh = bh % a.Hkv;
+  int i0l = 0, i1l = -1, i0h = 0, i1h = -1;
+  if (a.tl > 0) {
+    const Line Ll = line_of(a, false);
+    i0l = cta_of(Ll, (long long)bh * a.tl);
+    i1l = cta_of(Ll, (long long)bh * a.tl + a.tl - 1);
+  }
+  if (a.th > 0) {
+    const Line Lh = line_of(a, true);
+    i0h = cta_of(Lh, (long long)bh * a.th);
+    i1h = cta_of(Lh, (long long)bh * a.th + a.th - 1);
+  }
+  const int np_lo = i1l - i0l + 1, np = np_lo + (i1h - i0h + 1);
+  auto slot_of = [&](int sp) -> size_t {
+    return sp < np_lo ? (size_t)(i0l + bh + sp) : (size_t)(a.nc_lo + a.nbh + i0h + bh + (sp - np_lo));
+  };
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float m = -1e30f, l = 0.f;
+  float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s0 = warp; s0 < np; s0 += 4 * CMW) {
+    float2 ml[4];
+    float4 x[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int sp = s0 + j * CMW;
+      ml[j] = make_float2(-1e30f, 0.f);
+      x[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (sp < np) {
+        const size_t slot = slot_of(sp);
+        ml[j] = __ldcg(&a.part_ml[slot * G + h]);
+        x[j] = __ldcg(reinterpret_cast<const float4 *>(a.part_o + (slot * G + h) * D) + lane);
+      }
+    }
+    const float mn = fmaxf(fmaxf(m, fmaxf(ml[0].x, ml[1].x)), fmaxf(ml[2].x, ml[3].x));
+    const float r = exp2f(m - mn);
+    l *= r;
+    o.x *= r; o.y *= r; o.z *= r; o.w *= r;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float f = exp2f(ml[j].x - mn);
+      l = fmaf(f, ml[j].y, l);
+      o.x = fmaf(f, x[j].x, o.x); o.y = fmaf(f, x[j].y, o.y);
+      o.z = fmaf(f, x[j].z, o.z); o.w = fmaf(f, x[j].w, o.w);
+    }
+    m = mn;
+  }
+  so[warp][lane] = o;
+  if (lane == 0) {
+    sm_[warp] = m;
+    sl_[warp] = l;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    float mm = sm_[0];
+#pragma unroll
+    for (int w = 1; w < CMW; ++w) mm = fmaxf(mm, sm_[w]);
+    float ll = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int w = 0; w < CMW; ++w) {
+      const float f = exp2f(sm_[w] - mm);
+      const float4 y = so[w][lane];
+      ll = fmaf(f, sl_[w], ll);
+      acc.x = fmaf(f, y.x, acc.x); acc.y = fmaf(f, y.y, acc.y);
+      acc.z = fmaf(f, y.z, acc.z); acc.w = fmaf(f, y.w, acc.w);
+    }
+    const float c = 1.f / ll;
+    const size_t hq = (size_t)b * a.Hq + kh * G + h;
+    reinterpret_cast<float4 *>(a.out + hq * D)[lane] = make_float4(acc.x * c, acc.y * c, acc.z * c, acc.w * c);
+    if (lane == 0) {
+      if (a.lse) a.lse[hq] = (mm + log2f(ll)) * 0.6931471805599453f;
+      if (h == 0) {
+        a.tilectr[bh] = 0u;                      // every piece has stopped claiming tiles
+        a.tilectr[a.nbh + bh] = 0u;
+      }
     }
   }
 }
@@ -1003,14 +962,14 @@ int occupancy_for(int bits, int G) {
 }
 
 struct WsLayout {
-  size_t counters, part_ml, part_o, total;
+  size_t tilectr, part_ml, part_o, total;
 };
 
 WsLayout ws_layout(int B, int Hkv, int G, int nslot) {
   WsLayout w;
   size_t off = kWsHeader;
-  w.counters = off;
-  off = align_up(off + (size_t)3 * B * Hkv * sizeof(unsigned), 256);   // tickets + two tile counters
+  w.tilectr = off;
+  off = align_up(off + (size_t)2 * B * Hkv * sizeof(unsigned), 256);   // two tile counters per pair
   w.part_ml = off;
   off = align_up(off + (size_t)nslot * G * sizeof(float2), 256);
   w.part_o = off;
@@ -1060,8 +1019,10 @@ cudaError_t launch_tg(const DecArgs &a0, const hq_kv_cache &c, int nbh, cudaStre
   }
   const CUtensorMap *m = mc.m;
   occupancy<BITS, G, F8>();  // sets the dynamic shared memory attribute once
-  return pdl_launch(decode_tma<BITS, G, F8>, dim3(a.nc_lo + a.nc_hi), dim3(NTHREADS), Cfg<BITS>::SMEM, s,
-                    m[0], m[1], m[2], m[3], m[4], m[5], a);
+  const cudaError_t e = pdl_launch(decode_tma<BITS, G, F8>, dim3(a.nc_lo + a.nc_hi), dim3(NTHREADS),
+                                   Cfg<BITS>::SMEM, s, m[0], m[1], m[2], m[3], m[4], m[5], a);
+  if (e != cudaSuccess) return e;
+  return pdl_launch(decode_tma_combine<G>, dim3(G, nbh), dim3(CMW * 32), 0, s, a);
 }
 
 }  // namespace
@@ -1092,8 +1053,7 @@ cudaError_t launch_decode_tma(const __nv_bfloat16 *q, const hq_kv_cache &c, int 
   a.q = q;
   a.part_o = reinterpret_cast<float *>(ws + w.part_o);
   a.part_ml = reinterpret_cast<float2 *>(ws + w.part_ml);
-  a.counters = reinterpret_cast<unsigned *>(ws + w.counters);
-  a.tilectr = a.counters + nbh;
+  a.tilectr = reinterpret_cast<unsigned *>(ws + w.tilectr);
   a.out = out;
   a.lse = lse;
   a.status = status;

@@ -160,6 +160,12 @@ __device__ __forceinline__ T warp_sum(T x) {
   return x;
 }
 
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+
 // Index of the first element of sorted a[0..n) that is > x.
 __device__ __forceinline__ int upper_bound_i32(const int32_t *a, int n, int x) {
   int lo = 0, hi = n;
