@@ -304,7 +304,7 @@ hq_status hq_decode_merge(const float *part_out, const float *part_lse, int R, i
  *     hq_decode_workspace_size) return HQ_ERR_SCRATCH_LIMIT and launch nothing.
  *   - No cudaMalloc / cudaFree or allocating library routine is called.
  */
-#define HQ_STATIC_SCRATCH_BYTES (8u << 20)
+#define HQ_STATIC_SCRATCH_BYTES (16u << 20)
 hq_status hq_decode_attn_static(const void *q, const hq_kv_cache *cache, int B, int Hq, int Hkv,
                                 int D, float softmax_scale, float *out, float *lse_out,
                                 void *stream);

@@ -8,8 +8,9 @@
 //
 // Layout of the work: the low-bit tiles (64 tokens) and the bf16 tiles of all
 // (b, kv head) pairs form two lines, shared out over one wave of CTAs in
-// proportion to their cost; a CTA serves one or a few consecutive pairs and
-// claims their tiles dynamically (see Line below).  Tiles stream global ->
+// proportion to their cost; every tile is claimed from its pair's counter, a
+// CTA first serving the pairs of its own share of the line, then joining the
+// pair with the most unclaimed tiles (see Line below).  Tiles stream global ->
 // shared memory by TMA (one producer warp, an mbarrier ring of stages,
 // 64B/128B swizzle so that ldmatrix reads are bank-conflict free).  Each of
 // the four consumer warps takes one 16-token sub-tile of every stage:
@@ -71,34 +72,47 @@ struct Cfg {
   static_assert(LO_BYTES % 1024 == 0 && NMAX <= 8, "stage layout");
 };
 
+constexpr int JMAX = 3;     // pairs a CTA may join after its own
+constexpr int JCAP = 16;    // joined pieces a pair accepts per line
+
 struct DecArgs {
   const __nv_bfloat16 *q;
   float *part_o;          // [nslot][G][D]  unnormalized partial outputs
   float2 *part_ml;        // [nslot][G]     (max in log2 units, sum)
-  unsigned *tilectr;      // [2][B*Hkv] next unclaimed tile of each pair (low, bf16 line),
-                          // returned to zero by the combine kernel
+  unsigned *tilectr;      // [2][B*Hkv] tiles claimed of each pair (low, bf16 line)
+  unsigned *njoin;        // [2][B*Hkv] pieces that joined each pair
+  int *joins;             // [2][B*Hkv][JCAP] partial slots of those pieces
+  unsigned *cdone;        // [B*Hkv] combine CTAs that have read the pair's join counts
+                          // (the counters return to zero in the combine kernel)
   float *out, *lse;
   uint32_t *status;
   int Hq, Hkv, n_lo, n_hi;
   int nbh;                // B * Hkv
   int tl, th;             // 64-token tiles of the low / bf16 segment per (b, kv head)
   int nc_lo, nc_hi;       // CTAs streaming low tiles (blockIdx.x < nc_lo) and bf16 tiles
+  int kmax_lo, kmax_hi;   // partial slots per CTA of each line (see Line)
   float sl;               // softmax scale * log2(e)
 };
 
 // Each kind of tile (low-bit, bf16) of all (b, kv head) pairs is laid end to
 // end, pair-major, and cut into equal contiguous ranges, one per CTA of that
-// kind.  A CTA's tiles of one pair form a "piece" with its own partial
-// result.  The CTAs whose ranges lie inside one pair pool their tiles and
-// claim them one at a time from a shared counter, so uneven CTA speeds even
-// out; a CTA spanning pairs keeps exactly its own tiles.
-// Partial slots: low CTA i on pair bh -> i + bh; bf16 CTA j on pair bh ->
-// (nc_lo + nbh) + j + bh (consecutive pieces of one pair get consecutive
-// slots, and no two pieces share one).
+// kind: a CTA's "home" pairs are those its range meets, and its share of
+// each is the part of its range inside it.  Every tile is claimed one at a
+// time from its pair's counter, in order.  A CTA works through its home
+// pairs in turn, claiming at most its share of each but the last and as
+// many tiles as are left of the last; then, up to JMAX times, it joins the
+// pair of its line with the most unclaimed tiles.  CTA speeds differ by
+// +-10% on B200 (the pair being read and the SM's other CTAs both matter),
+// and the joins move the work where it is left.  A CTA's tiles of one pair
+// form a "piece" with its own partial result, in slot slot0 + i * kmax + j
+// for the j-th piece of the line's CTA i; the combine finds a pair's home
+// pieces from the plan and its joined pieces in the pair's list.
 struct Line {
   int n;          // CTAs on this line
   int t;          // tiles per pair
   long long T;    // tiles in all
+  int x0;         // blockIdx.x of the line's first CTA
+  int kmax;       // partial slots per CTA: most home pairs of one CTA + JMAX
   int slot0;      // first partial slot of the line
 };
 __device__ __forceinline__ Line line_of(const DecArgs &a, bool hi) {
@@ -106,7 +120,9 @@ __device__ __forceinline__ Line line_of(const DecArgs &a, bool hi) {
   L.n = hi ? a.nc_hi : a.nc_lo;
   L.t = hi ? a.th : a.tl;
   L.T = (long long)L.t * a.nbh;
-  L.slot0 = hi ? a.nc_lo + a.nbh : 0;
+  L.x0 = hi ? a.nc_lo : 0;
+  L.kmax = hi ? a.kmax_hi : a.kmax_lo;
+  L.slot0 = hi ? a.nc_lo * a.kmax_lo : 0;
   return L;
 }
 __device__ __forceinline__ long long range_start(const Line &L, int i) { return L.T * i / L.n; }
@@ -180,12 +196,13 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
   float *qsum = reinterpret_cast<float *>(merged + 1);          // [8 heads][4 groups]
   volatile int *abort_flag = reinterpret_cast<volatile int *>(qsum + 32);
   int *meta = const_cast<int *>(abort_flag) + 1;                 // [nst] tile of each stage, -1: end of piece
+  int *meta_pair = meta + 8;                                    // [nst] pair of each stage, -2: no more pieces
 
   const bool hi = (int)blockIdx.x >= a.nc_lo;
-  const int cta = hi ? (int)blockIdx.x - a.nc_lo : (int)blockIdx.x;
   const Line L = line_of(a, hi);
+  const int cta = (int)blockIdx.x - L.x0;
   const long long g0 = range_start(L, cta), g1 = range_start(L, cta + 1);
-  const int bh_a = (int)(g0 / L.t), bh_b = (int)((g1 - 1) / L.t);   // pairs of this CTA's pieces
+  const int bh_a = (int)(g0 / L.t), bh_b = (int)((g1 - 1) / L.t);   // home pairs
   const int T = hi ? T_HI : T_LO;
   const int nst = hi ? C::NHI : C::NLO;                        // stages of this CTA's ring
   const int stage_bytes = hi ? C::HI_BYTES : C::LO_BYTES;
@@ -216,7 +233,8 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
     // Streams the tiles of every piece back to back; before the first tile of
     // a new piece it waits until the consumers have merged the previous one
     // (the merge borrows the stage memory).  Starts at once: the consumers'
-    // per-pair prologue overlaps the first copies.
+    // per-pair prologue overlaps the first copies.  Lane 0 issues; the whole
+    // warp looks for a pair to join.
     if (lane == 0) {
       if (hi) {
         tma_prefetch_desc(&tm_khi);
@@ -227,67 +245,52 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
         tma_prefetch_desc(&tm_ksz);
         tma_prefetch_desc(&tm_vsz);
       }
-      // A CTA whose range spans pairs streams exactly its own tiles of each.
-      // The CTAs whose ranges lie inside one pair (the pool) share the middle
-      // of that pair (everything but its boundary CTAs' tiles): each claims
-      // the next tile from the pair's counter, one claim ahead of use so that
-      // the atomic's latency hides behind the stage wait; the pool's CTAs read
-      // neighbouring tiles at the same time and uneven CTA speeds even out.
-      // (Dealing most of the pool out round-robin or in static blocks before
-      // claiming the rest was measured slower on every decode workload.)  A
-      // stage with tile -1 and no copy ends the piece.
-      int n = 0;                                   // stages issued
-      int ps = 0, pu = 0;                          // stage of issue n, parity of n / nst
-      bool stop = false;
-      for (int bh = bh_a; bh <= bh_b && !stop; ++bh) {
-        if (bh > bh_a && !mbar_wait(merged, (bh - bh_a - 1) & 1)) {
-          *abort_flag = 1;
-          raise_status(a.status, HQ_DEV_TIMEOUT);
-          break;
+    }
+    unsigned *const ctr_line = a.tilectr + (hi ? a.nbh : 0);
+    int n = 0;                                     // stages issued (lane 0)
+    int ps = 0, pu = 0;                            // stage of issue n, parity of n / nst
+    bool stop = false;
+    // Next stage of the ring (lane 0): false if the wait for it ran out or
+    // another role gave up.
+    auto next_stage = [&](int &s) -> bool {
+      s = ps;
+      if (n >= nst && !mbar_wait(&empty[s], pu ^ 1)) {
+        *abort_flag = 1;
+        raise_status(a.status, HQ_DEV_TIMEOUT);
+        return false;
+      }
+      if (*abort_flag) return false;
+      ++n;
+      if (++ps == nst) {
+        ps = 0;
+        pu ^= 1;
+      }
+      return true;
+    };
+    // One piece (lane 0): claims tiles of pair bh from its counter, at most
+    // `quota`, one claim ahead of use so that the atomic's latency hides
+    // behind the stage wait; the CTAs on one pair read neighbouring tiles at
+    // the same time.  Every stage names its pair; one with tile -1 and no
+    // copy ends the piece.  (Dealing tiles out round-robin or in static
+    // blocks was measured slower on every decode workload.)
+    auto piece = [&](int bh, int quota) {
+      unsigned *const ctr = ctr_line + bh;
+      auto claim = [&]() -> int { return quota-- > 0 ? (int)atomicAdd(ctr, 1u) : L.t; };
+      int t = claim();
+      for (;;) {
+        int s;
+        if (!next_stage(s)) {
+          stop = true;
+          return;
         }
-        const long long base = (long long)bh * L.t;
-        const bool dyn = bh_a == bh_b;
-        int t0, t1;
-        if (dyn) {
-          const int i0 = cta_of(L, base), i1 = cta_of(L, base + L.t - 1);
-          const int first = range_start(L, i0) < base ? i0 + 1 : i0;
-          const int last = range_start(L, i1 + 1) > base + L.t ? i1 - 1 : i1;
-          t0 = (int)(range_start(L, first) - base);
-          t1 = (int)(range_start(L, last + 1) - base);
-        } else {
-          t0 = (int)((g0 > base ? g0 : base) - base);
-          t1 = (int)((g1 < base + L.t ? g1 : base + L.t) - base);
+        meta_pair[s] = bh;
+        if (t >= L.t) {                            // the piece is done: end marker
+          meta[s] = -1;
+          mbar_arrive(&full[s]);
+          return;
         }
-        unsigned *ctr = a.tilectr + (hi ? a.nbh : 0) + bh;
-        int nclaim = 0;
-        auto claim = [&]() -> int {
-          return dyn ? t0 + (int)atomicAdd(ctr, 1u) : t0 + nclaim++;
-        };
-        int t = claim();
-        for (;;) {
-          const int s = ps;
-          if (n >= nst && !mbar_wait(&empty[s], pu ^ 1)) {
-            *abort_flag = 1;
-            raise_status(a.status, HQ_DEV_TIMEOUT);
-            stop = true;
-            break;
-          }
-          if (*abort_flag) {
-            stop = true;
-            break;
-          }
-          ++n;
-          if (++ps == nst) {
-            ps = 0;
-            pu ^= 1;
-          }
-          if (t >= t1) {                           // the piece is done: end marker
-            meta[s] = -1;
-            mbar_arrive(&full[s]);
-            break;
-          }
-          const int t_next = claim();
-          meta[s] = t;
+        const int t_next = claim();
+        meta[s] = t;
           uint8_t *st = smem + s * stage_bytes;
           const int tok = t * T;
           if (!hi) {
@@ -304,7 +307,81 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
             tma_load_3d(st + 3 * C::HI_BOX, &tm_vhi, &full[s], 64, tok, bh);
           }
           t = t_next;
+      }
+    };
+    int j = 0;                                     // pieces started
+    auto merged_wait = [&]() {                     // lane 0, before piece j >= 1
+      if (!mbar_wait(merged, (j - 1) & 1)) {
+        *abort_flag = 1;
+        raise_status(a.status, HQ_DEV_TIMEOUT);
+        stop = true;
+      }
+    };
+    if (lane == 0) {
+      for (int bh = bh_a; bh <= bh_b && !stop; ++bh, ++j) {
+        if (j > 0) merged_wait();
+        if (stop) break;
+        const long long base = (long long)bh * L.t;
+        const long long e0 = g0 > base ? g0 : base, e1 = g1 < base + L.t ? g1 : base + L.t;
+        piece(bh, bh < bh_b ? (int)(e1 - e0) : L.t);
+      }
+    }
+    stop = __shfl_sync(0xffffffffu, (int)stop, 0) != 0;
+    j = __shfl_sync(0xffffffffu, j, 0);
+    // Joins: the pair of this line whose unclaimed tiles are the most per
+    // CTA already on it (its home CTAs and those that joined it), while one
+    // has enough left to be worth a new piece.  (Taking simply the most
+    // unclaimed tiles sends every CTA that finishes at about the same time
+    // to the same pair.)
+    const int jmin = hi ? 4 : 16;
+    unsigned *const njoin_line = a.njoin + (hi ? a.nbh : 0);
+    for (int tries = 0; !stop && j < L.kmax && tries < 2 * JMAX; ++tries) {
+      int best = -1, rem = 0, on = 1;              // maximize rem / on
+#pragma unroll 2
+      for (int p = lane; p < a.nbh; p += 32) {
+        const int left = L.t - (int)__ldcg(ctr_line + p);
+        const int nj = (int)__ldcg(njoin_line + p);
+        if (left >= jmin && nj < JCAP) {
+          const long long base = (long long)p * L.t;
+          const int o = cta_of(L, base + L.t - 1) - cta_of(L, base) + 1 + nj;
+          if (best < 0 || (long long)left * on > (long long)rem * o) {
+            rem = left;
+            on = o;
+            best = p;
+          }
         }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const int r2 = __shfl_xor_sync(0xffffffffu, rem, off);
+        const int o2 = __shfl_xor_sync(0xffffffffu, on, off);
+        const int b2 = __shfl_xor_sync(0xffffffffu, best, off);
+        if (b2 >= 0 && (best < 0 || (long long)r2 * on > (long long)rem * o2 ||
+                        ((long long)r2 * on == (long long)rem * o2 && b2 < best))) {
+          rem = r2;
+          on = o2;
+          best = b2;
+        }
+      }
+      if (best < 0) break;
+      int k = 0;
+      if (lane == 0) k = (int)atomicAdd(njoin_line + best, 1u);
+      k = __shfl_sync(0xffffffffu, k, 0);
+      if (k >= JCAP) continue;                     // full since the search: look again
+      if (lane == 0) {
+        a.joins[((hi ? a.nbh : 0) + best) * JCAP + k] = L.slot0 + cta * L.kmax + j;
+        merged_wait();
+        if (!stop) piece(best, L.t);
+      }
+      ++j;
+      stop = __shfl_sync(0xffffffffu, (int)stop, 0) != 0;
+    }
+    if (lane == 0) {
+      int s;
+      if (!stop && next_stage(s)) {                // no more pieces
+        meta[s] = -1;
+        meta_pair[s] = -2;
+        mbar_arrive(&full[s]);
       }
       // Never leave the CTA with copies in flight.
       for (int i = n > nst ? n - nst : 0; i < n; ++i)
@@ -315,13 +392,27 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
 
   // ------------------------------ consumers -------------------------------
   // One pass per piece: per-pair q set-up, the piece's tiles, then the warps'
-  // merge into the piece's partial result, the arrival ticket of the pair and,
-  // for the last arrival, the merge of all the pair's pieces.
+  // merge into the piece's partial result (decode_tma_combine merges the
+  // pieces of each pair).
   if (warp < NCW) {
     const int j = warp;  // this warp's 16-token sub-tile of every stage
     int n = 0;           // stages consumed
     int cs = 0, cu = 0;  // stage of consumption n, parity of n / nst
-    for (int bh = bh_a; bh <= bh_b; ++bh) {
+    for (int pc = 0;; ++pc) {
+      // The home pieces come first, in pair order, so their pair is known
+      // before any stage lands and the q set-up overlaps the first copies.  A
+      // joined piece names its pair in its first stage (-2: no more pieces),
+      // which stays unconsumed here; the tile loop waits on it again.
+      int bh = bh_a + pc;
+      if (bh > bh_b) {
+        if (!mbar_wait(&full[cs], cu)) {
+          *abort_flag = 1;
+          raise_status(a.status, HQ_DEV_TIMEOUT);
+          break;
+        }
+        bh = meta_pair[cs];
+        if (bh < 0) break;
+      }
       const int b = bh / a.Hkv, kh = bh % a.Hkv;
       // B fragments of q: 8 k16-chunks x 2 registers.
       uint32_t qb[8][2];
@@ -737,7 +828,7 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
         wm[8 + h] = ll;
       }
       consumer_sync();
-      const size_t slot = (size_t)L.slot0 + cta + bh;
+      const size_t slot = (size_t)L.slot0 + (size_t)cta * L.kmax + pc;
       for (int e = threadIdx.x; e < G * D; e += NCW * 32) {
         const int h = e / D, d = e % D;
         float oo = 0.f;
@@ -751,6 +842,7 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
       asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
       consumer_sync();
       if (lane == 0) mbar_arrive(merged);
+      if (*abort_flag) break;
     }
   }
 }
@@ -759,39 +851,68 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
 // 2^(m_s - m*) O_s / sum 2^(m_s - m*) l_s.  One CTA per (query head, pair),
 // launched as a programmatic dependent of decode_tma: its CTAs may be resident
 // early and start once every piece is written, and all heads of all pairs
-// merge in parallel.  Each of the CMW warps folds every CMW-th piece into its
-// own running (max, sum, output) -- lane l holds channels 4l..4l+3 -- taking
-// four pieces per round so that eight loads of each lane are in flight at
-// once; the warps' results are then folded the same way through shared
-// memory.  Pieces of a pair: CTAs i0l..i1l of the low line and i0h..i1h of
-// the bf16 line, their partial slots consecutive on each line.  The CTA of
-// the pair's first head also returns the pair's tile counters to zero for the
-// next call.
+// merge in parallel.  The pair's pieces: on each line the home pieces of the
+// CTAs whose ranges meet the pair (a CTA's piece for its k-th home pair is
+// its k-th), then the pieces that joined it.  Each of the CMW warps folds
+// every CMW-th piece into its own running (max, sum, output) -- lane l holds
+// channels 4l..4l+3 -- four pieces per round so that eight loads of each lane
+// are in flight at once; the warps' results are then folded the same way
+// through shared memory.  The last of the pair's G CTAs to read its join
+// counts returns the pair's counters to zero for the next call.
 constexpr int CMW = 8;                           // warps per combine CTA
 template <int G>
 __global__ void __launch_bounds__(CMW * 32)
 decode_tma_combine(DecArgs a) {
+  extern __shared__ int pslot[];                 // [np] partial slot of each piece
   __shared__ float4 so[CMW][32];
   __shared__ float sm_[CMW], sl_[CMW];
+  __shared__ int s_nj[2];
   pdl_wait();                                    // decode_tma has completed: every partial is written
   pdl_trigger();
   const int h = blockIdx.x, bh = blockIdx.y;
   const int b = bh / a.Hkv, kh = bh % a.Hkv;
-  int i0l = 0, i1l = -1, i0h = 0, i1h = -1;
-  if (a.tl > 0) {
-    const Line Ll = line_of(a, false);
-    i0l = cta_of(Ll, (long long)bh * a.tl);
-    i1l = cta_of(Ll, (long long)bh * a.tl + a.tl - 1);
+  if (threadIdx.x == 0) {
+    s_nj[0] = min((int)__ldcg(a.njoin + bh), JCAP);
+    s_nj[1] = min((int)__ldcg(a.njoin + a.nbh + bh), JCAP);
+    __threadfence();                             // the reads above come before the ticket
+    if (atomicAdd(a.cdone + bh, 1u) == (unsigned)(G - 1)) {
+      a.tilectr[bh] = 0u;                        // every piece has stopped claiming and joining,
+      a.tilectr[a.nbh + bh] = 0u;                // and every CTA of the pair has its counts
+      a.njoin[bh] = 0u;
+      a.njoin[a.nbh + bh] = 0u;
+      a.cdone[bh] = 0u;
+    }
   }
-  if (a.th > 0) {
-    const Line Lh = line_of(a, true);
-    i0h = cta_of(Lh, (long long)bh * a.th);
-    i1h = cta_of(Lh, (long long)bh * a.th + a.th - 1);
+  const Line Ll = line_of(a, false), Lh = line_of(a, true);
+  int i0l = 0, nhl = 0, i0h = 0, nhh = 0;
+  if (Ll.t > 0 && Ll.n > 0) {
+    i0l = cta_of(Ll, (long long)bh * Ll.t);
+    nhl = cta_of(Ll, (long long)bh * Ll.t + Ll.t - 1) - i0l + 1;
   }
-  const int np_lo = i1l - i0l + 1, np = np_lo + (i1h - i0h + 1);
-  auto slot_of = [&](int sp) -> size_t {
-    return sp < np_lo ? (size_t)(i0l + bh + sp) : (size_t)(a.nc_lo + a.nbh + i0h + bh + (sp - np_lo));
-  };
+  if (Lh.t > 0 && Lh.n > 0) {
+    i0h = cta_of(Lh, (long long)bh * Lh.t);
+    nhh = cta_of(Lh, (long long)bh * Lh.t + Lh.t - 1) - i0h + 1;
+  }
+  __syncthreads();
+  const int njl = s_nj[0], njh = s_nj[1];
+  const int np = nhl + nhh + njl + njh;
+  // pieces in the order: low home, bf16 home, low joined, bf16 joined
+  for (int e = threadIdx.x; e < np; e += blockDim.x) {
+    int sl;
+    if (e < nhl) {
+      const int i = i0l + e;
+      sl = Ll.slot0 + i * Ll.kmax + (bh - (int)(range_start(Ll, i) / Ll.t));
+    } else if (e < nhl + nhh) {
+      const int i = i0h + (e - nhl);
+      sl = Lh.slot0 + i * Lh.kmax + (bh - (int)(range_start(Lh, i) / Lh.t));
+    } else if (e < nhl + nhh + njl) {
+      sl = __ldcg(a.joins + bh * JCAP + (e - nhl - nhh));
+    } else {
+      sl = __ldcg(a.joins + (a.nbh + bh) * JCAP + (e - nhl - nhh - njl));
+    }
+    pslot[e] = sl;
+  }
+  __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   float m = -1e30f, l = 0.f;
   float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -799,14 +920,14 @@ decode_tma_combine(DecArgs a) {
     float2 ml[4];
     float4 x[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int sp = s0 + j * CMW;
-      ml[j] = make_float2(-1e30f, 0.f);
-      x[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int k = 0; k < 4; ++k) {
+      const int sp = s0 + k * CMW;
+      ml[k] = make_float2(-1e30f, 0.f);
+      x[k] = make_float4(0.f, 0.f, 0.f, 0.f);
       if (sp < np) {
-        const size_t slot = slot_of(sp);
-        ml[j] = __ldcg(&a.part_ml[slot * G + h]);
-        x[j] = __ldcg(reinterpret_cast<const float4 *>(a.part_o + (slot * G + h) * D) + lane);
+        const size_t slot = (size_t)pslot[sp];
+        ml[k] = __ldcg(&a.part_ml[slot * G + h]);
+        x[k] = __ldcg(reinterpret_cast<const float4 *>(a.part_o + (slot * G + h) * D) + lane);
       }
     }
     const float mn = fmaxf(fmaxf(m, fmaxf(ml[0].x, ml[1].x)), fmaxf(ml[2].x, ml[3].x));
@@ -814,11 +935,11 @@ decode_tma_combine(DecArgs a) {
     l *= r;
     o.x *= r; o.y *= r; o.z *= r; o.w *= r;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float f = exp2f(ml[j].x - mn);
-      l = fmaf(f, ml[j].y, l);
-      o.x = fmaf(f, x[j].x, o.x); o.y = fmaf(f, x[j].y, o.y);
-      o.z = fmaf(f, x[j].z, o.z); o.w = fmaf(f, x[j].w, o.w);
+    for (int k = 0; k < 4; ++k) {
+      const float f = exp2f(ml[k].x - mn);
+      l = fmaf(f, ml[k].y, l);
+      o.x = fmaf(f, x[k].x, o.x); o.y = fmaf(f, x[k].y, o.y);
+      o.z = fmaf(f, x[k].z, o.z); o.w = fmaf(f, x[k].w, o.w);
     }
     m = mn;
   }
@@ -845,13 +966,7 @@ decode_tma_combine(DecArgs a) {
     const float c = 1.f / ll;
     const size_t hq = (size_t)b * a.Hq + kh * G + h;
     reinterpret_cast<float4 *>(a.out + hq * D)[lane] = make_float4(acc.x * c, acc.y * c, acc.z * c, acc.w * c);
-    if (lane == 0) {
-      if (a.lse) a.lse[hq] = (mm + log2f(ll)) * 0.6931471805599453f;
-      if (h == 0) {
-        a.tilectr[bh] = 0u;                      // every piece has stopped claiming tiles
-        a.tilectr[a.nbh + bh] = 0u;
-      }
-    }
+    if (lane == 0 && a.lse) a.lse[hq] = (mm + log2f(ll)) * 0.6931471805599453f;
   }
 }
 
@@ -872,9 +987,24 @@ int sm_count() {
 }
 
 struct Plan {
-  int nbh, tl, th, nc_lo, nc_hi;
-  int nslot() const { return nc_lo + nc_hi + 2 * nbh; }
+  int nbh, tl, th, nc_lo, nc_hi, kmax_lo, kmax_hi;
+  int nslot() const { return nc_lo * kmax_lo + nc_hi * kmax_hi; }
 };
+
+// Most pairs one CTA's range meets on a line of n CTAs (t tiles per pair).
+int max_home(int n, int t, int nbh) {
+  if (n <= 0 || t <= 0) return 0;
+  const long long T = (long long)t * nbh;
+  int m = 0;
+  for (int i = 0; i < n; ++i) {
+    const long long g0 = T * i / n, g1 = T * (i + 1) / n;
+    if (g1 > g0) {
+      const int k = (int)((g1 - 1) / t - g0 / t + 1);
+      if (k > m) m = k;
+    }
+  }
+  return m;
+}
 
 // Resident CTAs per SM of one kernel variant (sets its shared memory limit
 // once).  Plans (and so workspace sizes) use the integer variant's figure for
@@ -950,6 +1080,8 @@ Plan make_plan(int nbh, int n_lo, int n_hi, int bits, int occ) {
   };
   p.nc_lo = fit(p.nc_lo, p.tl, 8);
   p.nc_hi = fit(p.nc_hi, p.th, 4);   // bf16 tiles: a 2-deep ring, so keep their CTAs short
+  p.kmax_lo = max_home(p.nc_lo, p.tl, nbh) + JMAX;
+  p.kmax_hi = max_home(p.nc_hi, p.th, nbh) + JMAX;
   return p;
 }
 
@@ -962,14 +1094,18 @@ int occupancy_for(int bits, int G) {
 }
 
 struct WsLayout {
-  size_t tilectr, part_ml, part_o, total;
+  size_t tilectr, njoin, cdone, joins, part_ml, part_o, total;
 };
 
 WsLayout ws_layout(int B, int Hkv, int G, int nslot) {
   WsLayout w;
   size_t off = kWsHeader;
-  w.tilectr = off;
-  off = align_up(off + (size_t)2 * B * Hkv * sizeof(unsigned), 256);   // two tile counters per pair
+  w.tilectr = off;                                   // claim and join counters: zero at rest
+  w.njoin = off + (size_t)2 * B * Hkv * sizeof(unsigned);
+  w.cdone = off + (size_t)4 * B * Hkv * sizeof(unsigned);
+  off = align_up(off + (size_t)5 * B * Hkv * sizeof(unsigned), 256);
+  w.joins = off;
+  off = align_up(off + (size_t)2 * B * Hkv * JCAP * sizeof(int), 256);
   w.part_ml = off;
   off = align_up(off + (size_t)nslot * G * sizeof(float2), 256);
   w.part_o = off;
@@ -1022,7 +1158,9 @@ cudaError_t launch_tg(const DecArgs &a0, const hq_kv_cache &c, int nbh, cudaStre
   const cudaError_t e = pdl_launch(decode_tma<BITS, G, F8>, dim3(a.nc_lo + a.nc_hi), dim3(NTHREADS),
                                    Cfg<BITS>::SMEM, s, m[0], m[1], m[2], m[3], m[4], m[5], a);
   if (e != cudaSuccess) return e;
-  return pdl_launch(decode_tma_combine<G>, dim3(G, nbh), dim3(CMW * 32), 0, s, a);
+  // a pair has at most every CTA's home piece and JCAP joined pieces per line
+  const size_t cmb_smem = (size_t)(a.nc_lo + a.nc_hi + 2 * JCAP) * sizeof(int);
+  return pdl_launch(decode_tma_combine<G>, dim3(G, nbh), dim3(CMW * 32), cmb_smem, s, a);
 }
 
 }  // namespace
@@ -1040,7 +1178,7 @@ size_t decode_tma_ws_bytes(int B, int Hq, int Hkv, int n_lo, int n_hi, int bits)
 size_t decode_tma_ws_zero_bytes(int B, int Hq, int Hkv, int n_lo, int n_hi, int bits) {
   const int G = Hq / Hkv;
   const Plan p = make_plan(B * Hkv, n_lo, n_hi, bits, occupancy_for(bits, G));
-  return ws_layout(B, Hkv, G, p.nslot()).part_ml;
+  return ws_layout(B, Hkv, G, p.nslot()).joins;      // the counters
 }
 
 cudaError_t launch_decode_tma(const __nv_bfloat16 *q, const hq_kv_cache &c, int B, int Hq,
@@ -1054,6 +1192,9 @@ cudaError_t launch_decode_tma(const __nv_bfloat16 *q, const hq_kv_cache &c, int 
   a.part_o = reinterpret_cast<float *>(ws + w.part_o);
   a.part_ml = reinterpret_cast<float2 *>(ws + w.part_ml);
   a.tilectr = reinterpret_cast<unsigned *>(ws + w.tilectr);
+  a.njoin = reinterpret_cast<unsigned *>(ws + w.njoin);
+  a.joins = reinterpret_cast<int *>(ws + w.joins);
+  a.cdone = reinterpret_cast<unsigned *>(ws + w.cdone);
   a.out = out;
   a.lse = lse;
   a.status = status;
@@ -1066,6 +1207,8 @@ cudaError_t launch_decode_tma(const __nv_bfloat16 *q, const hq_kv_cache &c, int 
   a.th = p.th;
   a.nc_lo = p.nc_lo;
   a.nc_hi = p.nc_hi;
+  a.kmax_lo = p.kmax_lo;
+  a.kmax_hi = p.kmax_hi;
   a.sl = scale * kLog2e;
   const bool f8 = c.fmt == HQ_KV_FP8;
 #define HQ_L(BITS, GG, FF) \

@@ -97,7 +97,7 @@ EXPORTED = ["hq_status_string", "hq_version", "hq_read_device_status", "hq_probe
             "hq_kv_append_part"]
 
 HQ_ERR_SCRATCH_LIMIT = 7
-STATIC_SCRATCH_BYTES = 8 << 20
+STATIC_SCRATCH_BYTES = 16 << 20
 
 
 class HQError(RuntimeError):
