@@ -871,6 +871,11 @@ decode_tma_combine(DecArgs a) {
   pdl_trigger();
   const int h = blockIdx.x, bh = blockIdx.y;
   const int b = bh / a.Hkv, kh = bh % a.Hkv;
+  // the pair's join lists, read before their lengths are known (one round
+  // trip to the L2 for both)
+  __shared__ int s_js[2 * JCAP];
+  if (threadIdx.x < 2 * JCAP)
+    s_js[threadIdx.x] = __ldcg(a.joins + ((threadIdx.x / JCAP) * a.nbh + bh) * JCAP + threadIdx.x % JCAP);
   if (threadIdx.x == 0) {
     s_nj[0] = min((int)__ldcg(a.njoin + bh), JCAP);
     s_nj[1] = min((int)__ldcg(a.njoin + a.nbh + bh), JCAP);
@@ -906,9 +911,9 @@ decode_tma_combine(DecArgs a) {
       const int i = i0h + (e - nhl);
       sl = Lh.slot0 + i * Lh.kmax + (bh - (int)(range_start(Lh, i) / Lh.t));
     } else if (e < nhl + nhh + njl) {
-      sl = __ldcg(a.joins + bh * JCAP + (e - nhl - nhh));
+      sl = s_js[e - nhl - nhh];
     } else {
-      sl = __ldcg(a.joins + (a.nbh + bh) * JCAP + (e - nhl - nhh - njl));
+      sl = s_js[JCAP + (e - nhl - nhh - njl)];
     }
     pslot[e] = sl;
   }
