@@ -482,7 +482,7 @@ def decode_loop(H, w, q, k, v, q_dec, dev, stream, world, T=64):
             "decode_us": max_over_ranks(dec, world, dev),
             "us_per_token_with_events": max_over_ranks(tot_ev, world, dev),
             "us_per_token": max_over_ranks(tot_b2b, world, dev),
-            "launches_per_token": 2, "l2": "not flushed",
+            "launches_per_token": 3, "l2": "not flushed",
             "queued_ahead": bool(ahead1 and ahead2)}
 
 
@@ -645,8 +645,9 @@ def main():
     mufu_peak = 16.0 * torch.cuda.get_device_properties(0).multi_processor_count * pk["sm_max_mhz"] * 1e6
     mixed_peak = (r["bf"] + r["i8"]) / t_star / 1e12
     # probe 4 (two QK passes, row stats, top-k); prefill 4 (+1 vertical
-    # gather when there are vertical columns); pack 1; decode 1
-    launches_per_step = 4 + (4 + (1 if r["kpad"] > 0 else 0)) + 1 + 1
+    # gather when there are vertical columns); pack 1; decode 2 (split-KV
+    # kernel and the combine)
+    launches_per_step = 4 + (4 + (1 if r["kpad"] > 0 else 0)) + 1 + 2
     out = {
         "metric": METRIC,
         "value": dec_tbs * world,
