@@ -593,17 +593,28 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
           za[3] = 0u;
           float zacc[4] = {0.f, 0.f, 0.f, 0.f};
           if (!F8) mma_f16_16816_z(zacc, za, zb0, 0u);   // FP8 has no zero point
-          float y[4] = {0.f, 0.f, 0.f, 0.f};
+          // (paired fp32 FMAs: each lane of ffma2 rounds once, as fmaf does)
+          float2 y01 = make_float2(0.f, 0.f), y23 = make_float2(0.f, 0.f);
   #pragma unroll
           for (int g = 0; g < 4; ++g) {
             const float sa = half_lo_f(wr[g]), sb = half_lo_f(wr8[g]);
-            y[0] = fmaf(sa, acc[g][0], y[0]);
-            y[1] = fmaf(sa, acc[g][1], y[1]);
-            y[2] = fmaf(sb, acc[g][2], y[2]);
-            y[3] = fmaf(sb, acc[g][3], y[3]);
+            y01 = ffma2(make_float2(sa, sa), make_float2(acc[g][0], acc[g][1]), y01);
+            y23 = ffma2(make_float2(sb, sb), make_float2(acc[g][2], acc[g][3]), y23);
           }
-  #pragma unroll
-          for (int e = 0; e < 4; ++e) x[e] = F8 ? y[e] * kF8Unit : fmaf(y[e], kCodeUnit, zacc[e]);
+          if (F8) {
+            x[0] = y01.x * kF8Unit;
+            x[1] = y01.y * kF8Unit;
+            x[2] = y23.x * kF8Unit;
+            x[3] = y23.y * kF8Unit;
+          } else {
+            const float2 u2 = make_float2(kCodeUnit, kCodeUnit);
+            const float2 x01 = ffma2(y01, u2, make_float2(zacc[0], zacc[1]));
+            const float2 x23 = ffma2(y23, u2, make_float2(zacc[2], zacc[3]));
+            x[0] = x01.x;
+            x[1] = x01.y;
+            x[2] = x23.x;
+            x[3] = x23.y;
+          }
         } else {
           float acc[4] = {0.f, 0.f, 0.f, 0.f};
           const int mi = lane >> 3;
@@ -652,10 +663,13 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
           oz[2] *= al0;
           oz[3] *= al1;
         }
-        const float p0 = fast_exp2(fmaf(x[0], a.sl, -m0)), p1 = fast_exp2(fmaf(x[1], a.sl, -m1));
-        const float p2 = fast_exp2(fmaf(x[2], a.sl, -m0)), p3 = fast_exp2(fmaf(x[3], a.sl, -m1));
-        l0 += p0 + p2;
-        l1 += p1 + p3;
+        const float2 sl2 = make_float2(a.sl, a.sl), nm = make_float2(-m0, -m1);
+        const float2 y01 = ffma2(make_float2(x[0], x[1]), sl2, nm), y23 = ffma2(make_float2(x[2], x[3]), sl2, nm);
+        const float p0 = fast_exp2(y01.x), p1 = fast_exp2(y01.y);
+        const float p2 = fast_exp2(y23.x), p3 = fast_exp2(y23.y);
+        const float2 l01 = fadd2(make_float2(l0, l1), fadd2(make_float2(p0, p1), make_float2(p2, p3)));
+        l0 = l01.x;
+        l1 = l01.y;
         const uint32_t pb0 = movmatrix_t(pack_f16x2(p0, p1));   // (head r; tokens 2c, 2c+1)
         const uint32_t pb1 = movmatrix_t(pack_f16x2(p2, p3));   // (head r; tokens 2c+8, 2c+9)
 
