@@ -94,10 +94,12 @@ cudaError_t launch_probe_merge_topk(const int32_t *cand_idx, const float *cand_s
 // at key positions qpos0 + p; D in {64, 128}, G <= 8, P <= 64.
 bool probe_tc_supported(int D, int G, int P);
 int probe_tc_chunks(int nbh, int Ls);
+// `pdl`: launch as a programmatic dependent of the kernel before it.
 cudaError_t launch_probe_pass(bool colsum, const __nv_bfloat16 *q_probe, int64_t q_head_stride,
                               const __nv_bfloat16 *k, int B, int Hq, int Hkv, int P, int Ls, int D,
                               int qpos0, float scale, float2 *partial, int nchunk,
-                              const float2 *stats, float *score, uint32_t *status, cudaStream_t s);
+                              const float2 *stats, float *score, uint32_t *status, cudaStream_t s,
+                              bool pdl = false);
 
 bool decode_tma_supported(int D, int bits, int G);
 size_t decode_tma_ws_bytes(int B, int Hq, int Hkv, int n_lo, int n_hi, int bits);

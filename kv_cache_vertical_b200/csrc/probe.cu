@@ -35,6 +35,8 @@ constexpr int KTILE = 128;       // keys per probe tile (probe_tc.cu)
 // order.  A row that sees no key keeps max -FLT_MAX and Z = 0.
 __global__ void probe_row_stats(const float2 *__restrict__ partial, float2 *__restrict__ stats,
                                 int nrows, int nchunk, bool invert = true) {
+  pdl_wait();                            // the partials come from the kernel before this one
+  pdl_trigger();
   const int row = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= nrows) return;
@@ -166,6 +168,7 @@ probe_topk(const float *__restrict__ score, int L, int ncand, int k, int32_t *__
   __shared__ int tmp[32];
   __shared__ uint32_t sel_prefix, sel_mask;
   __shared__ int remain;
+  pdl_wait();                            // the scores come from the kernel before this one
   const int bh = blockIdx.x;
   const float *s = score + (size_t)bh * L;
   int32_t *out = idx + (size_t)bh * k;
@@ -274,12 +277,13 @@ probe_topk(const float *__restrict__ score, int L, int ncand, int k, int32_t *__
     pos += __popc(tm);
     e += __popc(eqm);
   }
+  pdl_trigger();
 }
 
 // Top-k of every (b, kv head) row of `score` (row stride L) over positions
 // [0, ncand): k indices, ascending, ties to the lower index.
 cudaError_t launch_topk(const float *score, int L, int ncand, int k, int nbh, int32_t *idx,
-                        cudaStream_t s) {
+                        cudaStream_t s, bool pdl = false) {
   if (k <= 0 || nbh <= 0) return cudaSuccess;
   const size_t tk_smem = ncand <= TK_STAGE ? (size_t)(ncand + (ncand >> 5) + 1) * 4 : 0;
   static bool tk_attr = false;
@@ -289,8 +293,21 @@ cudaError_t launch_topk(const float *score, int L, int ncand, int k, int nbh, in
       return cudaErrorInvalidValue;
     tk_attr = true;
   }
+  if (pdl) return pdl_launch(probe_topk, dim3(nbh), dim3(TK_THREADS), tk_smem, s, score, L, ncand, k, idx);
   probe_topk<<<nbh, TK_THREADS, tk_smem, s>>>(score, L, ncand, k, idx);
   return cudaGetLastError();
+}
+
+// The probe's four kernels are chained by programmatic dependent launch when
+// the tensor-core passes are short (at most 64 key tiles per CTA): each
+// launch then overlaps the previous kernel's last CTAs, which saves ~6 us of
+// a ~120 us probe of the 32K layer (15 tiles per CTA).  With long passes
+// there is no launch gap worth hiding, and the chained launches were
+// measured slower (batched 128K cache, 512 tiles per CTA: 1975 -> 2023 us;
+// 70B-shaped: 7782 -> 7870 us), so those probes launch plainly.
+bool probe_chain_pdl(int nbh, int Ls) {
+  const int tiles = (Ls + KTILE - 1) / KTILE, nchunk = probe_tc_chunks(nbh, Ls);
+  return (tiles + nchunk - 1) / nchunk <= 64;
 }
 
 // The probe of keys [key_off, key_off + Ls) of an L-key context whose probe
@@ -303,14 +320,22 @@ cudaError_t probe_passes(const __nv_bfloat16 *q_probe, int64_t q_head_stride,
   const int nbh = B * Hkv, R = (Hq / Hkv) * P;
   const int nchunk = probe_tc_chunks(nbh, Ls);
   const int qpos0 = L - P - key_off;
+  const bool pdl = probe_chain_pdl(nbh, Ls);
   cudaError_t e = launch_probe_pass(false, q_probe, q_head_stride, k, B, Hq, Hkv, P, Ls, D, qpos0,
-                                    scale, partial, nchunk, nullptr, nullptr, status, s);
+                                    scale, partial, nchunk, nullptr, nullptr, status, s, pdl);
   if (e != cudaSuccess) return e;
   const int nrows = nbh * R;
-  probe_row_stats<<<(nrows + 7) / 8, 256, 0, s>>>(partial, stats, nrows, nchunk, invert);   // a warp per row
-  if ((e = cudaGetLastError()) != cudaSuccess || !score) return e;
+  const dim3 rs_grid((nrows + 7) / 8), rs_block(256);                 // a warp per row
+  if (pdl) {
+    e = pdl_launch(probe_row_stats, rs_grid, rs_block, 0, s, (const float2 *)partial, stats, nrows, nchunk,
+                   invert);
+  } else {
+    probe_row_stats<<<rs_grid, rs_block, 0, s>>>(partial, stats, nrows, nchunk, invert);
+    e = cudaGetLastError();
+  }
+  if (e != cudaSuccess || !score) return e;
   return launch_probe_pass(true, q_probe, q_head_stride, k, B, Hq, Hkv, P, Ls, D, qpos0, scale,
-                           nullptr, nchunk, stats, score, status, s);
+                           nullptr, nchunk, stats, score, status, s, pdl);
 }
 
 }  // namespace
@@ -354,7 +379,7 @@ cudaError_t launch_probe(const __nv_bfloat16 *q_probe, int64_t q_head_stride,
   cudaError_t e = probe_passes(q_probe, q_head_stride, k, B, Hq, Hkv, P, L, D, 0, L, scale,
                                w.partial, w.stats, true, score, reinterpret_cast<uint32_t *>(ws), s);
   if (e != cudaSuccess) return e;
-  return launch_topk(score, L, L - window, k_vert, B * Hkv, idx_out, s);
+  return launch_topk(score, L, L - window, k_vert, B * Hkv, idx_out, s, probe_chain_pdl(B * Hkv, L));
 }
 
 // ---------------------------------------------------------------------------

@@ -138,6 +138,9 @@ probe_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       reinterpret_cast<uint4 *>(smem)[i] = make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();
   }
+  // Everything above touched only shared and tensor memory; q, k and the row
+  // statistics may be written by the kernel before this one.
+  pdl_wait();
   if (COLSUM) {
     for (int r = threadIdx.x; r < a.Rpad; r += NTHR) {
       const int g = r / a.Ppad, p = r % a.Ppad;
@@ -454,6 +457,9 @@ probe_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
       raise_status(a.status, HQ_DEV_TIMEOUT);
     }
   }
+  // The next kernel may be scheduled once every CTA is here: not earlier, or
+  // its CTAs would take SMs from this grid's later waves.
+  pdl_trigger();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -481,7 +487,7 @@ bool make_map_bf16(CUtensorMap *m, const void *base, uint64_t inner, uint64_t ro
 
 template <int D, bool COLSUM>
 cudaError_t launch_t(const CUtensorMap &mq, const CUtensorMap &mk, const PtArgs &a, int nbh,
-                     int nchunk, uint32_t smem, cudaStream_t s) {
+                     int nchunk, uint32_t smem, cudaStream_t s, bool pdl) {
   static bool attr = false;
   if (!attr) {
     if (cudaFuncSetAttribute(probe_tc<D, COLSUM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -489,6 +495,7 @@ cudaError_t launch_t(const CUtensorMap &mq, const CUtensorMap &mk, const PtArgs 
       return cudaErrorInvalidValue;
     attr = true;
   }
+  if (pdl) return pdl_launch(probe_tc<D, COLSUM>, dim3(nchunk, nbh), dim3(NTHR), smem, s, mq, mk, a);
   probe_tc<D, COLSUM><<<dim3(nchunk, nbh), NTHR, smem, s>>>(mq, mk, a);
   return cudaGetLastError();
 }
@@ -513,7 +520,8 @@ bool probe_tc_supported(int D, int G, int P) { return (D == 64 || D == 128) && G
 cudaError_t launch_probe_pass(bool colsum, const __nv_bfloat16 *q_probe, int64_t q_head_stride,
                               const __nv_bfloat16 *k, int B, int Hq, int Hkv, int P, int Ls, int D,
                               int qpos0, float scale, float2 *partial, int nchunk,
-                              const float2 *stats, float *score, uint32_t *status, cudaStream_t s) {
+                              const float2 *stats, float *score, uint32_t *status, cudaStream_t s,
+                              bool pdl) {
   if (!probe_tc_supported(D, Hq / Hkv, P)) return cudaErrorNotSupported;
   PtArgs a;
   a.stats = stats;
@@ -552,10 +560,10 @@ cudaError_t launch_probe_pass(bool colsum, const __nv_bfloat16 *q_probe, int64_t
   const int nch = nchunk;
   if ((nch - 1) * a.tpc >= a.tiles) return cudaErrorInvalidValue;
   if (D == 128)
-    return colsum ? launch_t<128, true>(mq, mk, a, nbh, nch, smem, s)
-                  : launch_t<128, false>(mq, mk, a, nbh, nch, smem, s);
-  return colsum ? launch_t<64, true>(mq, mk, a, nbh, nch, smem, s)
-                : launch_t<64, false>(mq, mk, a, nbh, nch, smem, s);
+    return colsum ? launch_t<128, true>(mq, mk, a, nbh, nch, smem, s, pdl)
+                  : launch_t<128, false>(mq, mk, a, nbh, nch, smem, s, pdl);
+  return colsum ? launch_t<64, true>(mq, mk, a, nbh, nch, smem, s, pdl)
+                : launch_t<64, false>(mq, mk, a, nbh, nch, smem, s, pdl);
 }
 
 }  // namespace hq
