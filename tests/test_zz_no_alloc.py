@@ -66,3 +66,15 @@ def test_static_scratch_rejects_problems_beyond_its_size():
     with pytest.raises(H.HQError) as e:
         H.hq_decode_attn_static(q, cache, B, Hq, Hkv, D, 0.0, out, None)
     assert e.value.status == H.HQ_ERR_SCRATCH_LIMIT
+
+
+def test_static_scratch_covers_every_decode_workload():
+    # The decode's scratch holds one partial slot per piece a CTA may write,
+    # the pieces it may join included; its size depends on the device's SM
+    # count and residency, so it is checked here, on the device.
+    H = hq()
+    for name, w in WORKLOADS.items():
+        if w.mode != "decode":
+            continue
+        need = H.hq_decode_workspace_size(w.B, w.Hq, w.Hkv, w.D, w.n_lo, w.n_hi, w.bits)
+        assert need <= H.STATIC_SCRATCH_BYTES, (name, need)
