@@ -264,9 +264,11 @@ constexpr int kSpan = kWarps * kChunks * 8;   // 256
 // eight positions (copy the bf16 rows, or quantize them into the next low
 // rows), each lane one 32-channel group of one row.  With a part [lo0, lo1) x
 // [hi0, hi1) of the cache's rows (a context split across GPUs), only the rows
-// inside it are written, at their offsets from lo0 / hi0.
+// inside it are written, at their offsets from lo0 / hi0.  The kernel is
+// bound by the latency of each warp's chunk loads, so it is held to three
+// CTAs per SM (a few registers spill; 32K layer 115 -> 103 us).
 template <int D, int BITS, bool F8>
-__global__ void __launch_bounds__(kWarps * 32)
+__global__ void __launch_bounds__(kWarps * 32, 3)
 pack_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ v,
             const int32_t *__restrict__ idx, int nbh, int L, int window, int k_vert,
             int lo0, int lo1, int hi0, int hi1, int lo_cap,
