@@ -10,7 +10,7 @@
 // (b, kv head) pairs form two lines, shared out over one wave of CTAs in
 // proportion to their cost; every tile is claimed from its pair's counter, a
 // CTA first serving the pairs of its own share of the line, then joining the
-// pair with the most unclaimed tiles (see Line below).  Tiles stream global ->
+// pair with the most unclaimed tiles per CTA on it (see Line below).  Tiles stream global ->
 // shared memory by TMA (one producer warp, an mbarrier ring of stages,
 // 64B/128B swizzle so that ldmatrix reads are bank-conflict free).  Each of
 // the four consumer warps takes one 16-token sub-tile of every stage:
@@ -101,7 +101,8 @@ struct DecArgs {
 // time from its pair's counter, in order.  A CTA works through its home
 // pairs in turn, claiming at most its share of each but the last and as
 // many tiles as are left of the last; then, up to JMAX times, it joins the
-// pair of its line with the most unclaimed tiles.  CTA speeds differ by
+// pair of its line (among the 256 after its own) with the most unclaimed
+// tiles per CTA already on it.  CTA speeds differ by
 // +-10% on B200 (the pair being read and the SM's other CTAs both matter),
 // and the joins move the work where it is left.  A CTA's tiles of one pair
 // form a "piece" with its own partial result, in slot slot0 + i * kmax + j
@@ -337,8 +338,13 @@ decode_tma(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CU
     unsigned *const njoin_line = a.njoin + (hi ? a.nbh : 0);
     for (int tries = 0; !stop && j < L.kmax && tries < 2 * JMAX; ++tries) {
       int best = -1, rem = 0, on = 1;              // maximize rem / on
+      // the (up to) 256 pairs after this CTA's last home pair, so that a
+      // search stays short however many pairs there are
+      const int nscan = a.nbh < 256 ? a.nbh : 256;
 #pragma unroll 2
-      for (int p = lane; p < a.nbh; p += 32) {
+      for (int q = lane; q < nscan; q += 32) {
+        int p = bh_b + 1 + q;
+        if (p >= a.nbh) p -= a.nbh;
         const int left = L.t - (int)__ldcg(ctr_line + p);
         const int nj = (int)__ldcg(njoin_line + p);
         if (left >= jmin && nj < JCAP) {

@@ -108,7 +108,7 @@ cudaError_t launch_decode_tma(const __nv_bfloat16 *q, const hq_kv_cache &c, int 
                               uint32_t *status, cudaStream_t s);
 size_t decode_ws_bytes(int B, int Hq, int Hkv, int D, int n_lo, int n_hi, int bits);
 // Leading bytes of the decode workspace that must be zero before a call
-// (status word and split tickets).
+// (status word and the split counters).
 size_t decode_ws_zero_bytes(int B, int Hq, int Hkv, int D, int n_lo, int n_hi, int bits);
 size_t decode_tma_ws_zero_bytes(int B, int Hq, int Hkv, int n_lo, int n_hi, int bits);
 hq_status check_decode_args(const void *q, const hq_kv_cache *cache, int B, int Hq, int Hkv,

@@ -12,7 +12,7 @@
 // device address is looked up with cudaGetSymbolAddress, with the device
 // current, on the first call made in a CUDA context, and cached for that
 // context.  Every call shares the array: it first clears the part that must
-// start at zero (status word and split tickets); calls that overlap on the
+// start at zero (status word and the split counters); calls that overlap on the
 // GPU race on it.  The first 4 bytes are the device status word of the last
 // call (hq_read_static_status).
 #include <cuda.h>
