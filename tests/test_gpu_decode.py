@@ -118,6 +118,15 @@ def test_decode_many_tiles_per_cta(bits):
     run_decode_case(w, planted_idx=True)
 
 
+def test_decode_more_pairs_than_a_join_search_covers():
+    # 384 (b, kv head) pairs, more than the 256 a CTA looks through when it
+    # joins another pair (the search wraps around the pair index), with a
+    # ragged context so that the last tile of every pair is partial
+    w = Workload("manypairs", "decode", 48, 16, 8, 128, 2011, 64, F5, 4, 41)
+    assert w.B * w.Hkv > 256
+    run_decode_case(w, planted_idx=True)
+
+
 def test_llama8b_decode_full_size():
     run_decode_case(WORKLOADS["llama8b_decode_32k"])
 
