@@ -253,6 +253,16 @@ __device__ __forceinline__ void quant_group_lane(const uint32_t (&w)[16], uint8_
   *sz = __halves2half2(hs, hz);
 }
 
+// Asynchronous 16-byte copy global -> shared (completion: cp_async_wait).
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+// Wait until at most N of this thread's committed copy groups are pending.
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
+
 // Positions per CTA: kWarps warps x kChunks chunks x 8 positions.
 constexpr int kChunks = 4;
 constexpr int kSpan = kWarps * kChunks * 8;   // 256
@@ -262,11 +272,12 @@ constexpr int kSpan = kWarps * kChunks * 8;   // 256
 // those inside it in a shared bit mask, while every warp issues the row loads
 // of its first chunk; then each warp classifies and writes its four chunks of
 // eight positions (copy the bf16 rows, or quantize them into the next low
-// rows), each lane one 32-channel group of one row.  With a part [lo0, lo1) x
+// rows), each lane one 32-channel group of one row.  A chunk's 16 rows (K and
+// V of its eight positions) are copied into the warp's shared-memory stage by
+// cp.async while the warp works on the chunk before, so each warp has the
+// next chunk's loads in flight during its quantization.  With a part [lo0, lo1) x
 // [hi0, hi1) of the cache's rows (a context split across GPUs), only the rows
-// inside it are written, at their offsets from lo0 / hi0.  The kernel is
-// bound by the latency of each warp's chunk loads, so it is held to three
-// CTAs per SM (a few registers spill; 32K layer 115 -> 103 us).
+// inside it are written, at their offsets from lo0 / hi0.  Three CTAs per SM.
 template <int D, int BITS, bool F8>
 __global__ void __launch_bounds__(kWarps * 32, 3)
 pack_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ v,
@@ -304,25 +315,24 @@ pack_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict
   constexpr int RP = 32 / NG;                 // rows per pass: 8 (D = 128) or 16 (D = 64)
   constexpr int NPASS = 16 / RP;
   const int g = lane % NG, rsub = lane / NG;
-  uint32_t w[NPASS][16];
-  auto load_chunk = [&](int j0) {
+  // The warp's stage: 2 buffers x 16 rows (0-7: K of the chunk's positions,
+  // 8-15: V), each row D bf16 plus 16 bytes of padding against bank conflicts.
+  constexpr int ROWQ = D / 8 + 1;              // 16-byte units per staged row
+  extern __shared__ uint4 pack_stage[];
+  uint4 *const stg = pack_stage + warp * 2 * 16 * ROWQ;
+  auto issue_chunk = [&](int j0, int b) {
 #pragma unroll
-    for (int pi = 0; pi < NPASS; ++pi) {
-      const int rho = pi * RP + rsub;          // 0-7: K of position rho, 8-15: V of rho - 8
+    for (int u = 0; u < 16 * (D / 8) / 32; ++u) {
+      const int qd = lane + 32 * u;
+      const int rho = qd / (D / 8), c16 = qd % (D / 8);
       const int j = min(j0 + (rho & 7), L - 1);
-      const __nv_bfloat16 *src = (rho < 8 ? k : v) + ((size_t)bh * L + j) * D + g * 32;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const uint4 t = __ldg(reinterpret_cast<const uint4 *>(src) + u);
-        w[pi][4 * u] = t.x;
-        w[pi][4 * u + 1] = t.y;
-        w[pi][4 * u + 2] = t.z;
-        w[pi][4 * u + 3] = t.w;
-      }
+      const __nv_bfloat16 *src = (rho < 8 ? k : v) + ((size_t)bh * L + j) * D + c16 * 8;
+      cp_async16(stg + (b * 16 + rho) * ROWQ + c16, src);
     }
+    cp_async_commit();
   };
   const int jw = p0 + warp * kChunks * PCH;    // this warp's first position
-  if (jw < p1) load_chunk(jw);
+  if (jw < p1) issue_chunk(jw, 0);
   __syncthreads();                             // mask cleared
   if (warp == 0) {
     const int lo = warp_count_below(id, k_vert, p0, lane);
@@ -340,7 +350,15 @@ pack_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict
   for (int ci = 0; ci < kChunks; ++ci) {
     const int j0 = jw + ci * PCH;
     if (j0 >= p1) break;
-    if (ci > 0) load_chunk(j0);
+    const bool more = ci + 1 < kChunks && j0 + PCH < p1;
+    if (more) {
+      issue_chunk(j0 + PCH, (ci + 1) & 1);     // the next chunk streams in meanwhile
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncwarp();                              // every lane's copies of this chunk have landed
+    const uint4 *cst = stg + (ci & 1) * 16 * ROWQ;
     const int o = j0 - p0;                     // offset in the span, a multiple of 8
     uint32_t before = 0;                       // verticals in the span before j0
     for (int wdx = 0; wdx < (o >> 5); ++wdx) before += __popc(vmask[wdx]);
@@ -355,6 +373,15 @@ pack_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict
       const int p = rho & 7;
       const int j = j0 + p;
       if (j >= L) continue;
+      uint32_t w[16];                          // this lane's 32 channels of row rho
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint4 t = cst[rho * ROWQ + g * 4 + u];
+        w[4 * u] = t.x;
+        w[4 * u + 1] = t.y;
+        w[4 * u + 2] = t.z;
+        w[4 * u + 3] = t.w;
+      }
       const int cnt = cnt0 + __popc(vbits & ((1u << p) - 1u));            // verticals before j
       int hi_row = -1, lo_row = -1;
       if (j >= L - window) hi_row = k_vert + j % window;          // the window ring
@@ -370,7 +397,7 @@ pack_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict
                                                ((size_t)bh * part_hi + hi_row - hi0) * D + g * 32);
 #pragma unroll
         for (int u = 0; u < 4; ++u)
-          dst[u] = make_uint4(w[pi][4 * u], w[pi][4 * u + 1], w[pi][4 * u + 2], w[pi][4 * u + 3]);
+          dst[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
       } else {
         if (lo_row < 0 || lo_row >= n_lo) {
           raise_status(status, HQ_DEV_BAD_INDEX);
@@ -378,11 +405,12 @@ pack_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict
         }
         if (lo_row < lo0 || lo_row >= lo1) continue;   // another part's row
         const size_t r = (size_t)bh * lo_cap + lo_row - lo0;
-        quant_group_lane<BITS, F8>(w[pi], (is_v ? v_codes : k_codes) + r * ROWB + g * (32 * BITS / 8),
+        quant_group_lane<BITS, F8>(w, (is_v ? v_codes : k_codes) + r * ROWB + g * (32 * BITS / 8),
                                    (is_v ? v_sz : k_sz) + r * NG + g);
         if (lo_pos && !is_v && g == 0) lo_pos[r] = j;
       }
     }
+    __syncwarp();                              // this buffer is refilled two chunks on
   }
 }
 
@@ -392,7 +420,16 @@ cudaError_t launch_pack_t(const __nv_bfloat16 *k, const __nv_bfloat16 *v, const 
                           const hq_kv_cache &o, uint32_t *status, cudaStream_t s) {
   const long long blocks = (long long)nbh * ((L + kSpan - 1) / kSpan);
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
-  pack_kernel<D, BITS, F8><<<(unsigned)blocks, kWarps * 32, 0, s>>>(
+  // the warps' chunk stages: 2 buffers x 16 rows of D bf16 + 16 bytes each
+  const size_t smem = (size_t)kWarps * 2 * 16 * (D / 8 + 1) * 16;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(pack_kernel<D, BITS, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+      return cudaErrorInvalidValue;
+    attr = true;
+  }
+  pack_kernel<D, BITS, F8><<<(unsigned)blocks, kWarps * 32, smem, s>>>(
       k, v, idx, nbh, L, window, k_vert, lo0, lo0 + o.n_lo, hi0, hi0 + o.n_hi, lo_rows(o),
       (uint8_t *)o.k_codes, (uint8_t *)o.v_codes,
       (__half2 *)o.k_sz, (__half2 *)o.v_sz, (__nv_bfloat16 *)o.k_hi, (__nv_bfloat16 *)o.v_hi,
