@@ -172,13 +172,8 @@ prefill_tc(const __grid_constant__ CUtensorMap tm_qi8, const __grid_constant__ C
   volatile int *abort_flag = reinterpret_cast<volatile int *>(bar + 25);
 
   const int ntq = (a.N + BM - 1) / BM;
-  // CTAs start in launch order (x fastest): the launch index walks the query
-  // tiles from the longest down, all head pairs and batch rows of one tile
-  // before the next, so the last CTAs to start are the shortest everywhere.
-  const int nrow = gridDim.y * gridDim.z;        // (head pair, batch) rows
-  const int lin = (int)(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z));
-  const int qt = ntq - 1 - lin / nrow;
-  const int hp = (lin % nrow) % (int)gridDim.y, b = (lin % nrow) / (int)gridDim.y;
+  const int qt = ntq - 1 - (int)blockIdx.x;      // longest rows first
+  const int hp = blockIdx.y, b = blockIdx.z;
   const int G = a.Hq / a.Hkv;
   const int hA = 2 * hp;
   const int kh = hA / G;
